@@ -1,0 +1,368 @@
+"""Seeded synthetic workloads and offline predictor calibration.
+
+This module produces *inputs*: K/V traces shaped like the video backbones the
+codec targets, queries, and the predictor weights fitted offline on a separate
+calibration trace (least squares for the linear predictors, k-means for the
+centres).  It contains none of the codec's own arithmetic (prediction at run
+time, residual quantization, packing, attention); both the CUDA path and the
+fp64 oracle receive what it returns.
+
+Shapes follow the pages' backbones: Wan-1.3B at 832x480 gives 1560 latent
+tokens per frame, 12 heads of 128 channels, 30 layers ("TempoKV: Predictive KV
+Cache Quantization for Autoregressive Video Generation", Tables 1-3: 832x480,
+717 frames); a 13B/14B-class backbone has 40 heads and 40 layers.  Calibration
+follows "TempoKV ...", Fig. 2(a) (linear regression on a clean trace) and
+"CORAL-KV ...", Fig. 4 (block-diagonal plus low-rank predictors fitted offline).
+
+All randomness comes from ``torch.Generator`` objects seeded from the integer
+seed; the same seed on the same device type gives the same tensors.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+SEED_BASE = 20261202
+FRAME_TOKENS_480P = 1560
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _randn(g, *shape, device, dtype=torch.float32):
+    return torch.randn(*shape, generator=g, device=device, dtype=dtype)
+
+
+def _orthogonal(g, n: int, count: int, device) -> torch.Tensor:
+    """`count` independent n x n orthogonal matrices (QR of Gaussians)."""
+    a = _randn(g, count, n, n, device=device, dtype=torch.float64)
+    q, r = torch.linalg.qr(a)
+    d = torch.sign(torch.diagonal(r, dim1=-2, dim2=-1))
+    return (q * d[:, None, :]).float()
+
+
+# ---------------------------------------------------------------------------
+# Cross-layer (block-DPLR) workloads
+# ---------------------------------------------------------------------------
+
+
+@dataclass
+class XLayerWorkload:
+    """K/V of every layer plus fitted (or true) block-DPLR predictors.
+
+    K[l], V[l]: [T,H,D] in the state dtype.  weights[l] (l >= 1) holds
+    k_block [H,D,D], k_w [r,C], k_u [C,r], v_block [H,D,2D], v_w [r,2C],
+    v_u [C,r] in the state dtype ([out][in] convention, y = x @ W^T).
+    """
+
+    K: list
+    V: list
+    weights: list
+    n_heads: int
+    head_dim: int
+    rank: int
+    dtype: torch.dtype
+    extra: dict = field(default_factory=dict)
+
+
+def tiny_xlayer(seed: int = SEED_BASE + 0, device="cpu", T: int = 512, H: int = 2,
+                D: int = 64, rank: int = 8, n_outliers: int = 4) -> XLayerWorkload:
+    """The tiny fp32 cross-layer case: 2 layers.  Layer-0 K, V ~ N(0,1) with
+    `n_outliers` channels per head scaled 8x; K_1 = A K_0 + 0.1 N, V_1 = B
+    [K_1, V_0] + 0.1 N with A, B block-DPLR (entries N(0, 1/64)); the true A, B
+    serve as the predictors."""
+    g = _gen(seed, device)
+    C = H * D
+    sd = 1.0 / 8.0
+
+    def with_outliers(x):
+        for h in range(H):
+            idx = torch.randperm(D, generator=g, device=device)[:n_outliers]
+            x[:, h, idx] *= 8.0
+        return x
+
+    K0 = with_outliers(_randn(g, T, H, D, device=device))
+    V0 = with_outliers(_randn(g, T, H, D, device=device))
+    w = {
+        "k_block": _randn(g, H, D, D, device=device) * sd,
+        "k_w": _randn(g, rank, C, device=device) * sd,
+        "k_u": _randn(g, C, rank, device=device) * sd,
+        "v_block": _randn(g, H, D, 2 * D, device=device) * sd,
+        "v_w": _randn(g, rank, 2 * C, device=device) * sd,
+        "v_u": _randn(g, C, rank, device=device) * sd,
+    }
+
+    def dplr(x_head, x_flat, blk, wm, um):
+        y = torch.einsum("thi,hoi->tho", x_head, blk)
+        return y + ((x_flat @ wm.T) @ um.T).reshape(T, H, D)
+
+    K1 = dplr(K0, K0.reshape(T, C), w["k_block"], w["k_w"], w["k_u"]) + 0.1 * _randn(g, T, H, D, device=device)
+    kv = torch.cat([K1, V0], dim=-1)
+    kvf = torch.cat([K1.reshape(T, C), V0.reshape(T, C)], dim=-1)
+    V1 = dplr(kv, kvf, w["v_block"], w["v_w"], w["v_u"]) + 0.1 * _randn(g, T, H, D, device=device)
+    return XLayerWorkload([K0, K1], [V0, V1], [None, w], H, D, rank, torch.float32)
+
+
+@dataclass
+class _BackboneModel:
+    """Per-layer linear transition of a synthetic backbone's KV trace."""
+
+    Mk: list  # per layer: (blocks [H,D,D], P [C,q], Qm [C,q]) for K
+    Nv: list  # per layer: (blocks, P, Qm) for the V self term
+    Gv: list  # per layer: blocks [H,D,D] for the K -> V coupling
+
+
+def _backbone(seed: int, L: int, H: int, D: int, device, cross_rank: int = 8) -> _BackboneModel:
+    g = _gen(seed, device)
+    C = H * D
+    Mk, Nv, Gv = [], [], []
+    for _ in range(L):
+        Mk.append((_orthogonal(g, D, H, device), _randn(g, C, cross_rank, device=device) / math.sqrt(C),
+                   _randn(g, C, cross_rank, device=device) / math.sqrt(C)))
+        Nv.append((_orthogonal(g, D, H, device), _randn(g, C, cross_rank, device=device) / math.sqrt(C),
+                   _randn(g, C, cross_rank, device=device) / math.sqrt(C)))
+        Gv.append(_orthogonal(g, D, H, device))
+    return _BackboneModel(Mk, Nv, Gv)
+
+
+def _apply_mix(x, blocks, P, Qm, cross: float):
+    T, H, D = x.shape
+    y = torch.einsum("thi,hoi->tho", x, blocks)
+    return y + cross * ((x.reshape(T, H * D) @ Qm) @ P.T).reshape(T, H, D)
+
+
+def _trace(model: _BackboneModel, seed: int, T: int, L: int, H: int, D: int, device, rho: float = 0.9,
+           chunk: int = 8192):
+    """x_l = rho * M_l x_{l-1} + sqrt(1 - rho^2) eps for K; V couples to K."""
+    g = _gen(seed, device)
+    K = [_randn(g, T, H, D, device=device)]
+    V = [_randn(g, T, H, D, device=device)]
+    a_v, c_v = 0.6, 0.6
+    s_k = math.sqrt(1.0 - rho * rho)
+    s_v = math.sqrt(max(0.0, 1.0 - a_v * a_v - c_v * c_v))
+    for l in range(1, L):
+        bk, pk, qk = model.Mk[l]
+        bn, pn, qn = model.Nv[l]
+        kl = torch.empty(T, H, D, device=device)
+        vl = torch.empty(T, H, D, device=device)
+        for a in range(0, T, chunk):
+            b = min(T, a + chunk)
+            kl[a:b] = rho * _apply_mix(K[-1][a:b], bk, pk, qk, 0.3) + s_k * _randn(g, b - a, H, D, device=device)
+            vl[a:b] = (a_v * _apply_mix(V[-1][a:b], bn, pn, qn, 0.3)
+                       + c_v * torch.einsum("thi,hoi->tho", kl[a:b], model.Gv[l])
+                       + s_v * _randn(g, b - a, H, D, device=device))
+        K.append(kl)
+        V.append(vl)
+    return K, V
+
+
+def _ridge_lstsq(X: torch.Tensor, Y: torch.Tensor, lam: float = 1e-3) -> torch.Tensor:
+    """argmin_W |X W - Y|^2 + lam*n |W|^2 in float64 (X [n,p], Y [n,q])."""
+    X = X.double()
+    Y = Y.double()
+    n, p = X.shape
+    A = X.T @ X + lam * n * torch.eye(p, dtype=torch.float64, device=X.device)
+    return torch.linalg.solve(A, X.T @ Y)
+
+
+def fit_block_dplr(X_head: torch.Tensor, X_flat: torch.Tensor, Y: torch.Tensor, rank: int):
+    """Least-squares block-DPLR fit ("CORAL-KV ...", Fig. 4): per-head blocks by
+    least squares, then a rank-`rank` reduced-rank regression of the remainder
+    on the whole-token input.  Returns (block [H,D,Din_h], w [r,Cin], u [C,r])."""
+    T, H, Din = X_head.shape
+    D = Y.shape[-1]
+    blocks = torch.empty(H, D, Din, dtype=torch.float64, device=X_head.device)
+    R = torch.empty(T, H, D, dtype=torch.float64, device=X_head.device)
+    for h in range(H):
+        Bh = _ridge_lstsq(X_head[:, h], Y[:, h])  # [Din, D]
+        blocks[h] = Bh.T
+        R[:, h] = Y[:, h].double() - X_head[:, h].double() @ Bh
+    if rank == 0:
+        return blocks, None, None
+    Rf = R.reshape(T, H * D)
+    M = _ridge_lstsq(X_flat, Rf)  # [Cin, C]
+    F = X_flat.double() @ M
+    _, _, Vh = torch.linalg.svd(F, full_matrices=False)
+    Vr = Vh[:rank].T  # [C, r]
+    w = (M @ Vr).T  # [r, Cin]
+    return blocks, w, Vr
+
+
+def wan_xlayer(seed: int = SEED_BASE + 1, device="cpu", L: int = 30, T: int = 21 * FRAME_TOKENS_480P,
+               H: int = 12, D: int = 128, rank: int = 64, calib_tokens: int = 4096,
+               dtype=torch.bfloat16, layers_needed=None) -> XLayerWorkload:
+    """Wan-1.3B-shaped cross-layer trace (inter-layer correlation 0.9) with
+    block-DPLR predictors fitted on a separate 4096-token calibration trace.
+
+    `layers_needed` (an iterable of layer indices) limits which predictors are
+    fitted; the trace itself always has L layers.
+    """
+    model = _backbone(seed * 7 + 1, L, H, D, device)
+    K, V = _trace(model, seed * 7 + 2, T, L, H, D, device)
+    Kc, Vc = _trace(model, seed * 7 + 3, calib_tokens, L, H, D, device)
+    C = H * D
+    need = set(range(1, L)) if layers_needed is None else set(layers_needed)
+    weights = [None]
+    for l in range(1, L):
+        if l not in need:
+            weights.append(None)
+            continue
+        kb, kw, ku = fit_block_dplr(Kc[l - 1], Kc[l - 1].reshape(-1, C), Kc[l], rank)
+        xin = torch.cat([Kc[l], Vc[l - 1]], dim=-1)
+        xf = torch.cat([Kc[l].reshape(-1, C), Vc[l - 1].reshape(-1, C)], dim=-1)
+        vb, vw, vu = fit_block_dplr(xin, xf, Vc[l], rank)
+        weights.append({k: t.to(dtype).contiguous() for k, t in
+                        dict(k_block=kb, k_w=kw, k_u=ku, v_block=vb, v_w=vw, v_u=vu).items()})
+    K = [k.to(dtype).contiguous() for k in K]
+    V = [v.to(dtype).contiguous() for v in V]
+    return XLayerWorkload(K, V, weights, H, D, rank, dtype)
+
+
+def queries(seed: int, n: int, H: int, D: int, device="cpu", dtype=torch.bfloat16) -> torch.Tensor:
+    """Q ~ N(0,1) [n,H,D]."""
+    g = _gen(seed, device)
+    return _randn(g, n, H, D, device=device).to(dtype).contiguous()
+
+
+# ---------------------------------------------------------------------------
+# Temporal workloads
+# ---------------------------------------------------------------------------
+
+
+@dataclass
+class TemporalWorkload:
+    K: torch.Tensor  # [T,H,D]
+    V: torch.Tensor
+    ak: torch.Tensor  # [H,D,2D] over [K_{f-1} | K_{f-2}]
+    av: torch.Tensor  # [H,D,2D] over [K_f | V_{f-1}]
+    frame_tokens: int
+
+
+def _ar2_trace(g, n_frames: int, F: int, H: int, D: int, Gk, device, T: int | None = None):
+    """K_f = 0.7 K_{f-1} + 0.2 K_{f-2} + 0.3 eps per (position, head);
+    V_f = 0.5 G_h K_f + 0.5 V_{f-1} + 0.3 eps."""
+    T = n_frames * F if T is None else T
+    K = torch.empty(T, H, D, device=device)
+    V = torch.empty(T, H, D, device=device)
+    k1 = torch.zeros(F, H, D, device=device)
+    k2 = torch.zeros(F, H, D, device=device)
+    v1 = torch.zeros(F, H, D, device=device)
+    for f in range(n_frames):
+        a, b = f * F, min(T, (f + 1) * F)
+        if a >= T:
+            break
+        if f == 0:
+            kf = 0.63 * _randn(g, F, H, D, device=device)
+            vf = 0.63 * _randn(g, F, H, D, device=device)
+        else:
+            kf = 0.7 * k1 + 0.2 * k2 + 0.3 * _randn(g, F, H, D, device=device)
+            vf = 0.5 * torch.einsum("thi,hoi->tho", kf, Gk) + 0.5 * v1 + 0.3 * _randn(g, F, H, D, device=device)
+        K[a:b] = kf[: b - a]
+        V[a:b] = vf[: b - a]
+        k2, k1, v1 = k1, kf, vf
+    return K, V
+
+
+def temporal_layer(seed: int = SEED_BASE + 3, device="cpu", T: int = 65536, H: int = 40, D: int = 128,
+                   F: int = FRAME_TOKENS_480P, calib_frames: int = 8, dtype=torch.bfloat16) -> TemporalWorkload:
+    """One layer of the large-backbone temporal case: AR(2) keys (0.7/0.2,
+    sigma 0.3), values coupled to the aligned key; per-head 128x256 maps fitted
+    by least squares on a separate calibration trace."""
+    g_model = _gen(seed * 11 + 1, device)
+    Gk = _orthogonal(g_model, D, H, device)
+    g_cal = _gen(seed * 11 + 2, device)
+    cal_F = min(F, 1560)
+    Kc, Vc = _ar2_trace(g_cal, calib_frames, cal_F, H, D, Gk, device)
+    ak = torch.empty(H, D, 2 * D, dtype=torch.float64, device=device)
+    av = torch.empty(H, D, 2 * D, dtype=torch.float64, device=device)
+    # regress frame f on frames f-1, f-2 (f >= 2)
+    for h in range(H):
+        kc = Kc[:, h].reshape(calib_frames, cal_F, D)
+        vc = Vc[:, h].reshape(calib_frames, cal_F, D)
+        Xk = torch.cat([kc[1:-1], kc[:-2]], dim=-1).reshape(-1, 2 * D)
+        Yk = kc[2:].reshape(-1, D)
+        ak[h] = _ridge_lstsq(Xk, Yk, 1e-4).T
+        Xv = torch.cat([kc[1:], vc[:-1]], dim=-1).reshape(-1, 2 * D)
+        Yv = vc[1:].reshape(-1, D)
+        av[h] = _ridge_lstsq(Xv, Yv, 1e-4).T
+    g_data = _gen(seed * 11 + 3, device)
+    n_frames = (T + F - 1) // F
+    K, V = _ar2_trace(g_data, n_frames, F, H, D, Gk, device, T=T)
+    return TemporalWorkload(K.to(dtype).contiguous(), V.to(dtype).contiguous(),
+                            ak.to(dtype).contiguous(), av.to(dtype).contiguous(), F)
+
+
+# ---------------------------------------------------------------------------
+# Clustered workloads
+# ---------------------------------------------------------------------------
+
+
+@dataclass
+class ClusterWorkload:
+    K: torch.Tensor  # [T,H,D]
+    V: torch.Tensor
+    k_centroids: torch.Tensor  # [n_c, C]
+    v_centroids: torch.Tensor
+    k_enc: torch.Tensor  # [m, C]
+    k_dec: torch.Tensor  # [C, m]
+    v_enc: torch.Tensor
+    v_dec: torch.Tensor
+
+
+def _gmm(g, T: int, C: int, n_comp: int, sigma: float, device, chunk: int = 8192):
+    means = _randn(g, n_comp, C, device=device)
+    comp = torch.randint(0, n_comp, (T,), generator=g, device=device)
+    X = torch.empty(T, C, device=device)
+    for a in range(0, T, chunk):
+        b = min(T, a + chunk)
+        X[a:b] = means[comp[a:b]] + sigma * _randn(g, b - a, C, device=device)
+    return X, comp
+
+
+def _kmeans(X: torch.Tensor, comp: torch.Tensor, n_c: int, iters: int, chunk: int = 8192):
+    """Lloyd's k-means (offline calibration), initialised from one sample of
+    each mixture component so that no two centres start in one component."""
+    T, C = X.shape
+    first = torch.full((n_c,), -1, dtype=torch.long, device=X.device)
+    order = torch.arange(T, device=X.device)
+    first.scatter_reduce_(0, comp, order, reduce="amin", include_self=False)
+    first = torch.where(first < 0, torch.arange(n_c, device=X.device) % T, first)
+    cent = X[first].clone()
+    for _ in range(iters):
+        lab = torch.empty(T, dtype=torch.long, device=X.device)
+        c2 = (cent * cent).sum(1)
+        for a in range(0, T, chunk):
+            b = min(T, a + chunk)
+            lab[a:b] = torch.argmin(c2[None, :] - 2.0 * X[a:b] @ cent.T, dim=1)
+        sums = torch.zeros_like(cent).index_add_(0, lab, X)
+        cnt = torch.bincount(lab, minlength=n_c).to(X.dtype)
+        keep = cnt > 0
+        cent[keep] = sums[keep] / cnt[keep, None]
+    return cent
+
+
+def cluster_layer(seed: int = SEED_BASE + 4, device="cpu", T: int = 32768, H: int = 16, D: int = 128,
+                  n_c: int = 256, m: int = 128, sigma: float = 0.2, iters: int = 20,
+                  dtype=torch.bfloat16) -> ClusterWorkload:
+    """One layer of the clustered case: K and V drawn from two Gaussian mixtures
+    (n_c components, means N(0,1) in H*D dims, sigma 0.2); centres by k-means;
+    a fixed orthonormal C x m encoder (QR of a Gaussian) used as both encoder
+    (its transpose) and decoder."""
+    C = H * D
+    g = _gen(seed * 13 + 1, device)
+    out = {}
+    for name in ("k", "v"):
+        X, comp = _gmm(g, T, C, n_c, sigma, device)
+        out[name] = X.to(dtype).reshape(T, H, D).contiguous()
+        out[name + "_cent"] = _kmeans(X.to(dtype).float(), comp, n_c, iters).to(dtype).contiguous()
+        E, _ = torch.linalg.qr(_randn(g, C, m, device=device, dtype=torch.float64))
+        out[name + "_dec"] = E.to(dtype).contiguous()
+        out[name + "_enc"] = E.T.to(dtype).contiguous()
+    return ClusterWorkload(out["k"], out["v"], out["k_cent"], out["v_cent"], out["k_enc"], out["k_dec"],
+                           out["v_enc"], out["v_dec"])

@@ -1,0 +1,403 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a library
+routine, a value printed on the pages (tests/golden), a hand-worked example, a
+closed form, an invariant, or brute force on tiny inputs.  None needs a GPU.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import kvc_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(20261202)
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- rounding
+
+
+def test_round_to_f16_f32_match_numpy_casts():
+    x = RNG.standard_normal(200_000) * np.exp2(RNG.integers(-30, 20, 200_000))
+    # exact ties of both formats
+    ties = np.array([1 + 2.0**-11, 1 + 3 * 2.0**-11, 2049.0, 2051.0, 1 + 2.0**-24, 1 + 3 * 2.0**-24,
+                     65519.99, 65520.0, 2.0**-25, 3 * 2.0**-25, 6e-8])
+    x = np.concatenate([x, ties, -ties])
+    with np.errstate(over="ignore"):
+        ref16 = x.astype(np.float16).astype(np.float64)
+    np.testing.assert_array_equal(O.round_to(x, "f16"), ref16)
+    np.testing.assert_array_equal(O.round_to(x, "f32"), x.astype(np.float32).astype(np.float64))
+
+
+def test_round_to_bf16_matches_torch_on_float32_inputs():
+    x32 = (RNG.standard_normal(200_000) * np.exp2(RNG.integers(-40, 40, 200_000))).astype(np.float32)
+    ties = np.array([1 + 2.0**-8, 1 + 3 * 2.0**-8, 257.0, 259.0, -(1 + 2.0**-8)], np.float32)
+    x32 = np.concatenate([x32, ties])
+    ref = torch.from_numpy(x32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(O.round_to(x32.astype(np.float64), "bf16"), ref)
+
+
+# ---------------------------------------------------------------- quantizer
+
+
+@pytest.mark.parametrize("bits,group,param", [(2, 32, "f16"), (4, 32, "f16"), (4, 64, "f16"),
+                                              (4, 32, "f32"), (8, 16, "f16")])
+def test_quantizer_matches_brute_force_nearest_level(bits, group, param):
+    r = RNG.standard_normal((64, 4 * group)) * np.exp2(RNG.integers(-3, 4, (64, 1)))
+    q, s, z = O.quantize_groups(r, bits, group, param)
+    L = (1 << bits) - 1
+    rg = r.reshape(64, 4, group)
+    levels = z[..., None, None] + s[..., None, None] * np.arange(L + 1)  # [64,4,1,L+1]
+    dist = np.abs(rg[..., None] - levels)
+    best = dist.argmin(-1)
+    qg = q.reshape(64, 4, group)
+    srt = np.sort(dist, axis=-1)
+    tie = (srt[..., 1] - srt[..., 0]) < 1e-12 * (1 + np.abs(rg))
+    assert np.all((best == qg) | tie)
+    # error bound: half a step, plus what fp rounding of s and z moved the grid
+    mn, mx = rg.min(-1), rg.max(-1)
+    s_exact = (mx - mn) / L
+    bound = s / 2 + np.abs(z - mn) + L * np.abs(s - s_exact) + 1e-12
+    err = np.abs(rg - O.dequantize_groups(q, s, z, group).reshape(64, 4, group))
+    assert np.all(err <= bound[..., None])
+    assert np.all(q <= L)
+
+
+def test_quantizer_degenerate_group_and_exact_grid():
+    r = np.full((3, 32), 0.3)
+    q, s, z = O.quantize_groups(r, 2, 32, "f16")
+    assert np.all(q == 0) and np.all(s == 0)
+    np.testing.assert_array_equal(z, np.float16(0.3).astype(np.float64))
+    # values exactly on a representable grid with both ends present: lossless
+    grid = -1.5 + 1.0 * RNG.integers(0, 4, (5, 32))
+    grid[:, 0], grid[:, 1] = -1.5, 1.5
+    q, s, z = O.quantize_groups(grid, 2, 32, "f16")
+    np.testing.assert_array_equal(O.dequantize_groups(q, s, z, 32), grid)
+
+
+# ---------------------------------------------------------------- packing
+
+
+def test_pack_hand_worked_examples():
+    for case in _golden("pack_worked_example.json")["cases"]:
+        codes = np.array(case["codes"], np.uint8)
+        got = O.pack_codes(codes, case["bits"])
+        assert got.tolist() == case["bytes"], case
+        np.testing.assert_array_equal(O.unpack_codes(got, case["bits"], len(codes)), codes)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_pack_matches_numpy_unpackbits(bits):
+    codes = RNG.integers(0, 1 << bits, (17, 128)).astype(np.uint8)
+    packed = O.pack_codes(codes, bits)
+    assert packed.shape == (17, 128 * bits // 8)
+    bitstr = np.unpackbits(packed, axis=-1, bitorder="little").reshape(17, 128, bits)
+    rebuilt = (bitstr * (1 << np.arange(bits))).sum(-1)
+    np.testing.assert_array_equal(rebuilt, codes)
+
+
+# ---------------------------------------------------------------- storage accounting
+
+
+def test_group_quantizer_ratios_printed_on_pages():
+    g = _golden("page_compression_ratios.json")
+    for key in ("int2_group_quantizer", "int4_group_quantizer"):
+        e = g[key]
+        ratio = 16.0 / O.bits_per_element(e["bits"], 32, "f16")
+        assert round(ratio, e["printed_decimals"]) == pytest.approx(e["ratio"]), key
+    d = O.Desc(n_tokens=1000, n_heads=12, head_dim=128, bits=2, group=32)
+    elems = 2 * 1000 * 12 * 128
+    assert O.codes_bytes(d) * 8 / elems == pytest.approx(O.bits_per_element(2, 32, "f16"))
+
+
+def test_tempokv_anchor_sweep_slope():
+    """One anchor latent frame among ~180 (717 video frames): each extra anchor
+    bit costs 1/180 bit per element; the printed ratios give the same slope."""
+    e = _golden("page_compression_ratios.json")["tempokv_anchor_sweep"]
+    printed_bits = 16.0 / np.array(e["ratio"])
+    n_lat = (e["video_frames"] - 1) // 4 + 1
+    F, H, D = 16, 2, 64
+    model = []
+    for ab in e["anchor_bits"]:
+        d = O.Desc(n_tokens=n_lat * F, n_heads=H, head_dim=D, bits=2, group=32, frame_tokens=F, anchor_bits=ab)
+        model.append(O.codes_bytes(d, "temporal") * 8 / (2 * n_lat * F * H * D))
+    model = np.array(model)
+    tol = 2 * 16.0 * 0.5 * 10.0 ** -e["printed_decimals"] / np.array(e["ratio"]) ** 2
+    np.testing.assert_array_less(np.abs(np.diff(printed_bits) - np.diff(model)), tol[1:] + tol[:-1])
+
+
+# ---------------------------------------------------------------- cross-layer predictor
+
+
+def _dense_dplr(block, w, u, H, D, Din_head, Cin_order):
+    """Dense Cin x C matrix of a block-DPLR map, built entry by entry."""
+    Cin = w.shape[1]
+    C = H * D
+    M = np.zeros((Cin, C))
+    for h in range(H):
+        for o in range(D):
+            for i in range(Din_head):
+                M[Cin_order(h, i), h * D + o] += block[h, o, i]
+    M += w.T @ u.T
+    return M
+
+
+def test_dplr_prediction_equals_dense_map():
+    H, D, r, T = 3, 8, 2, 11
+    rng = np.random.default_rng(1)
+    Ks, Vs = rng.standard_normal((T, H, D)), rng.standard_normal((T, H, D))
+    kb, vb = rng.standard_normal((H, D, D)), rng.standard_normal((H, D, 2 * D))
+    kw, ku = rng.standard_normal((r, H * D)), rng.standard_normal((H * D, r))
+    vw, vu = rng.standard_normal((r, 2 * H * D)), rng.standard_normal((H * D, r))
+    Mk = _dense_dplr(kb, kw, ku, H, D, D, lambda h, i: h * D + i)
+    got = O.xlayer_predict_k(Ks, kb, kw, ku, "f64").reshape(T, -1)
+    np.testing.assert_allclose(got, Ks.reshape(T, -1) @ Mk, rtol=1e-12, atol=1e-12)
+    # V's per-head input is [K_h | V_h]; its global input is [K (all heads) | V (all heads)]
+    Mv = _dense_dplr(vb, vw, vu, H, D, 2 * D,
+                     lambda h, i: h * D + i if i < D else H * D + h * D + (i - D))
+    flat = np.concatenate([Ks.reshape(T, -1), Vs.reshape(T, -1)], axis=1)
+    got = O.xlayer_predict_v(Ks, Vs, vb, vw, vu, "f64").reshape(T, -1)
+    np.testing.assert_allclose(got, flat @ Mv, rtol=1e-12, atol=1e-12)
+    # rank 0 is the pure block-diagonal map
+    got0 = O.xlayer_predict_k(Ks, kb, kw[:0], ku[:, :0], "f64").reshape(T, -1)
+    np.testing.assert_allclose(got0, Ks.reshape(T, -1) @ _dense_dplr(kb, kw[:0], ku[:, :0], H, D, D,
+                                                                      lambda h, i: h * D + i), rtol=1e-12)
+
+
+def test_low_rank_latent_is_rounded_to_state_dtype():
+    H, D, r, T = 2, 4, 3, 5
+    rng = np.random.default_rng(2)
+    Ks = rng.standard_normal((T, H, D))
+    kb = np.zeros((H, D, D))
+    kw, ku = rng.standard_normal((r, H * D)), np.eye(H * D, r)
+    got = O.xlayer_predict_k(Ks, kb, kw, ku, "bf16").reshape(T, -1)[:, :r]
+    lat = Ks.reshape(T, -1) @ kw.T
+    ref = torch.from_numpy(lat.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    # the f32 pre-rounding of the reference can only matter at bf16 ties, which random data avoids
+    np.testing.assert_array_equal(got, ref)
+
+
+def _grid_values(rng, shape):
+    """Values in {-1.5,-0.5,0.5,1.5} with both ends in every 32-group: INT2 lossless."""
+    v = -1.5 + rng.integers(0, 4, shape).astype(np.float64)
+    v[..., 0::32] = -1.5
+    v[..., 1::32] = 1.5
+    return v
+
+
+def test_exact_predictor_gives_zero_residual():
+    H, D, r, T = 2, 64, 4, 40
+    rng = np.random.default_rng(3)
+    K0, V0 = _grid_values(rng, (T, H, D)), _grid_values(rng, (T, H, D))
+    d0 = O.Desc(T, H, D, state="bf16", bits=2, group=32)
+    ck0, cv0, K0h, V0h = O.encode_layer_none(d0, K0, V0)
+    np.testing.assert_array_equal(K0h, K0)  # anchor lossless on its grid
+
+    def sparse(shape, nnz_per_row):
+        m = np.zeros(shape)
+        for idx in np.ndindex(*shape[:-1]):
+            cols = rng.choice(shape[-1], nnz_per_row, replace=False)
+            m[idx + (cols,)] = rng.choice([-1.0, 1.0], nnz_per_row)
+        return m
+
+    w = dict(k_block=sparse((H, D, D), 3), k_w=sparse((r, H * D), 3), k_u=sparse((H * D, r), 2),
+             v_block=sparse((H, D, 2 * D), 3), v_w=sparse((r, 2 * H * D), 3), v_u=sparse((H * D, r), 2))
+    Mk = _dense_dplr(w["k_block"], w["k_w"], w["k_u"], H, D, D, lambda h, i: h * D + i)
+    K1 = (K0.reshape(T, -1) @ Mk).reshape(T, H, D)
+    Mv = _dense_dplr(w["v_block"], w["v_w"], w["v_u"], H, D, 2 * D,
+                     lambda h, i: h * D + i if i < D else H * D + h * D + (i - D))
+    V1 = (np.concatenate([K1.reshape(T, -1), V0.reshape(T, -1)], 1) @ Mv).reshape(T, H, D)
+    assert np.array_equal(O.round_to(K1, "bf16"), K1) and np.array_equal(O.round_to(V1, "bf16"), V1)
+    ck, cv, K1h, V1h = O.encode_layer_xlayer(d0, w, K1, V1, K0h, V0h)
+    for c in (ck, cv):
+        assert np.all(c.q == 0) and np.all(c.s == 0)
+    np.testing.assert_array_equal(K1h, K1)
+    np.testing.assert_array_equal(V1h, V1)
+
+
+def _chain_workload(L=6, T=300, H=2, D=64, r=4, seed=5):
+    rng = np.random.default_rng(seed)
+    C = H * D
+    K = [rng.standard_normal((T, H, D))]
+    V = [rng.standard_normal((T, H, D))]
+    W = [None]
+    for _ in range(1, L):
+        w = dict(k_block=0.9 * np.stack([np.linalg.qr(rng.standard_normal((D, D)))[0] for _ in range(H)]),
+                 k_w=rng.standard_normal((r, C)) / np.sqrt(C), k_u=0.1 * rng.standard_normal((C, r)),
+                 v_block=0.5 * rng.standard_normal((H, D, 2 * D)) / np.sqrt(2 * D),
+                 v_w=rng.standard_normal((r, 2 * C)) / np.sqrt(2 * C), v_u=0.1 * rng.standard_normal((C, r)))
+        w = {k: O.round_to(v, "bf16") for k, v in w.items()}
+        W.append(w)
+        K.append(O.round_to(O.xlayer_predict_k(K[-1], w["k_block"], w["k_w"], w["k_u"], "f64")
+                            + 0.3 * rng.standard_normal((T, H, D)), "bf16"))
+        V.append(O.round_to(O.xlayer_predict_v(K[-1], V[-1], w["v_block"], w["v_w"], w["v_u"], "f64")
+                            + 0.3 * rng.standard_normal((T, H, D)), "bf16"))
+    K[0], V[0] = O.round_to(K[0], "bf16"), O.round_to(V[0], "bf16")
+    return K, V, W
+
+
+def test_closed_loop_error_does_not_accumulate_and_decode_replays_encode():
+    K, V, W = _chain_workload()
+    T, H, D = K[0].shape
+    d_anchor = O.Desc(T, H, D, bits=4, group=32)
+    d = O.Desc(T, H, D, bits=2, group=32)
+    ck, cv, Kh, Vh = O.encode_layer_none(d_anchor, K[0], V[0])
+    Kd, Vd = O.decode_layer_none(d_anchor, ck, cv)
+    np.testing.assert_array_equal(Kd, Kh)
+    open_K = Kh  # decoder-side state of an open-loop encoder
+    open_err = []
+    for l in range(1, len(K)):
+        Ks, Vs = Kh, Vh
+        ck, cv, Kh, Vh = O.encode_layer_xlayer(d, W[l], K[l], V[l], Ks, Vs)
+        Kd, Vd = O.decode_layer_xlayer(d, W[l], ck, cv, Ks, Vs)
+        np.testing.assert_array_equal(Kd, Kh)
+        np.testing.assert_array_equal(Vd, Vh)
+        # closed loop: the error of every layer is its own quantization error only
+        for x, xh, c in ((K[l], Kh, ck), (V[l], Vh, cv)):
+            s = np.repeat(c.s, 32, axis=-1)
+            assert np.all(np.abs(x - xh) <= 0.5 * s + 2.0 ** -7 * np.abs(x) + 1e-3 * s + 1e-30)
+        # open loop: predict from clean K_{l-1}; the decoder only has its own state
+        pk_clean = O.xlayer_predict_k(K[l - 1], W[l]["k_block"], W[l]["k_w"], W[l]["k_u"], "bf16")
+        qo, so, zo = O.quantize_groups(K[l] - pk_clean, 2, 32, "f16")
+        pk_dec = O.xlayer_predict_k(open_K, W[l]["k_block"], W[l]["k_w"], W[l]["k_u"], "bf16")
+        open_K = O.round_to(pk_dec + O.dequantize_groups(qo, so, zo, 32), "bf16")
+        open_err.append(np.abs(open_K - K[l]).max() / np.repeat(so, 32, -1).max())
+    assert open_err[-1] > 0.75  # drift beyond the half-step bound the closed loop keeps
+
+
+# ---------------------------------------------------------------- temporal predictor
+
+
+def test_temporal_exact_predictor_and_ragged_frame():
+    H, D, F = 2, 64, 10
+    T = 4 * F + 3  # ragged last frame
+    rng = np.random.default_rng(7)
+    ak = np.zeros((H, D, 2 * D))
+    av = np.zeros((H, D, 2 * D))
+    for h in range(H):
+        ak[h, :, :D] = 0.5 * np.eye(D)  # K_f = 0.5 K_{f-1} + 0.5 K_{f-2}
+        ak[h, :, D:] = 0.5 * np.eye(D)
+        av[h, :, :D] = np.eye(D)[rng.permutation(D)]  # V_f = P K_f + 0.5 V_{f-1}
+        av[h, :, D:] = 0.5 * np.eye(D)
+    K = np.zeros((T, H, D))
+    V = np.zeros((T, H, D))
+    K[:F] = _grid_values(rng, (F, H, D))
+    V[:F] = _grid_values(rng, (F, H, D))
+    for f in range(1, 5):
+        a, b = f * F, min(T, (f + 1) * F)
+        n = b - a
+        k1 = K[a - F:a - F + n]
+        k2 = K[a - 2 * F:a - 2 * F + n] if f >= 2 else 0.0
+        K[a:b] = 0.5 * k1 + 0.5 * k2
+        V[a:b] = np.einsum("thi,hoi->tho", K[a:b], av[:, :, :D]) + 0.5 * V[a - F:a - F + n]
+    assert np.array_equal(O.round_to(K, "bf16"), K) and np.array_equal(O.round_to(V, "bf16"), V)
+    d = O.Desc(T, H, D, bits=2, group=32, frame_tokens=F, anchor_bits=2)
+    ck, cv, Kh, Vh = O.encode_layer_temporal(d, dict(ak=ak, av=av), K, V)
+    np.testing.assert_array_equal(Kh, K)
+    np.testing.assert_array_equal(Vh, V)
+    assert np.all(ck.s[F:] == 0) and np.all(cv.s[F:] == 0)
+    Kd, Vd = O.decode_layer_temporal(d, dict(ak=ak, av=av), ck, cv)
+    np.testing.assert_array_equal(Kd, K)
+    np.testing.assert_array_equal(Vd, V)
+
+
+def test_temporal_frame_zero_is_plain_group_rtn_at_anchor_bits():
+    H, D, F, T = 2, 64, 8, 20
+    rng = np.random.default_rng(8)
+    K = O.round_to(rng.standard_normal((T, H, D)), "bf16")
+    V = O.round_to(rng.standard_normal((T, H, D)), "bf16")
+    w = dict(ak=rng.standard_normal((H, D, 2 * D)) * 0.05, av=rng.standard_normal((H, D, 2 * D)) * 0.05)
+    d = O.Desc(T, H, D, bits=2, group=32, frame_tokens=F, anchor_bits=4)
+    ck, _, Kh, _ = O.encode_layer_temporal(d, w, K, V)
+    assert ck.q[:F].max() > 3  # anchor rows use 4-bit codes
+    assert ck.q[F:].max() <= 3
+    # frame 0 against brute-force nearest level at 4 bits
+    q, s, z = ck.q[:F], ck.s[:F], ck.z[:F]
+    lv = z[..., None] + s[..., None] * np.arange(16)
+    dist = np.abs(K[:F].reshape(F, H, 2, 32)[..., None] - lv[:, :, :, None, :])
+    assert np.mean(dist.argmin(-1) == q.reshape(F, H, 2, 32)) > 0.999
+
+
+# ---------------------------------------------------------------- clustered predictor
+
+
+def test_cluster_assignment_is_nearest_centre_by_euclidean_distance():
+    rng = np.random.default_rng(9)
+    cent = rng.standard_normal((16, 64))
+    X = cent[rng.integers(0, 16, 200)] + 0.3 * rng.standard_normal((200, 64))
+    a = O.cluster_assign(X, cent)
+    brute = np.array([min(range(16), key=lambda j: float(np.sum((x - cent[j]) ** 2))) for x in X])
+    np.testing.assert_array_equal(a, brute)
+    # ties go to the lowest index
+    cent2 = np.stack([cent[0], cent[0], cent[1]])
+    assert O.cluster_assign(cent[:1], cent2)[0] == 0
+
+
+def test_cluster_codec_is_exact_when_residual_is_on_grid_in_decoder_span():
+    H, D, m, T, nc = 2, 32, 32, 24, 4
+    C = H * D
+    rng = np.random.default_rng(10)
+    E, _ = np.linalg.qr(rng.standard_normal((C, m)))
+    # an orthonormal basis made of signed unit vectors keeps every product exact
+    E = np.zeros((C, m))
+    E[rng.permutation(C)[:m], np.arange(m)] = rng.choice([-1.0, 1.0], m)
+    cent = np.round(rng.standard_normal((nc, C)) * 4) * 4.0  # far apart, integers
+    coef = _grid_values(rng, (T, m))  # on the INT2 grid of each 32-group
+    a = rng.integers(0, nc, T)
+    X = (cent[a] + coef @ E.T).reshape(T, H, D)
+    d = O.Desc(T, H, D, bits=2, group=32)
+    c, xh = O.encode_tensor_cluster(d, X, cent, E.T, E)
+    np.testing.assert_array_equal(c.assign, a)
+    np.testing.assert_array_equal(xh, X)
+    np.testing.assert_array_equal(O.decode_tensor_cluster(d, c, cent, E), X)
+
+
+# ---------------------------------------------------------------- attention
+
+
+def test_attention_matches_torch_sdpa_in_float64():
+    rng = np.random.default_rng(11)
+    Q, K, V = rng.standard_normal((7, 3, 16)), rng.standard_normal((29, 3, 16)), rng.standard_normal((29, 3, 16))
+    got = O.attention(Q, K, V, 0.37)
+    t = lambda x: torch.from_numpy(x).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(Q), t(K), t(V), scale=0.37)[0].permute(1, 0, 2)
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(12)
+    Q = rng.standard_normal((4, 2, 8))
+    K1 = np.repeat(rng.standard_normal((1, 2, 8)), 9, axis=0)
+    V = rng.standard_normal((9, 2, 8))
+    np.testing.assert_allclose(O.attention(Q, K1, V, 1.0), np.broadcast_to(V.mean(0), (4, 2, 8)), atol=1e-13)
+    np.testing.assert_allclose(O.attention(Q, K1[:1], V[:1], 1.0), np.broadcast_to(V[0], (4, 2, 8)), atol=1e-14)
+    K = rng.standard_normal((9, 2, 8))
+    shift = np.zeros_like(K) + rng.standard_normal((1, 2, 8))  # q.shift is constant over keys
+    np.testing.assert_allclose(O.attention(Q, K + shift, V, 0.5), O.attention(Q, K, V, 0.5), atol=1e-12)
+
+
+def test_mixed_attention_equals_attention_on_reconstructed_keys():
+    H, D, m, T, nc = 2, 32, 16, 50, 8
+    C = H * D
+    rng = np.random.default_rng(13)
+    E, _ = np.linalg.qr(rng.standard_normal((C, m)))
+    cent_k, cent_v = rng.standard_normal((nc, C)), rng.standard_normal((nc, C))
+    K = (cent_k[rng.integers(0, nc, T)] + 0.2 * rng.standard_normal((T, C))).reshape(T, H, D)
+    V = (cent_v[rng.integers(0, nc, T)] + 0.2 * rng.standard_normal((T, C))).reshape(T, H, D)
+    d = O.Desc(T, H, D, bits=4, group=16)
+    ck, _ = O.encode_tensor_cluster(d, K, cent_k, E.T, E)
+    cv, _ = O.encode_tensor_cluster(d, V, cent_v, E.T, E)
+    Q = rng.standard_normal((6, H, D))
+    fast = O.mixed_attention(Q, ck, cent_k, E, cv, cent_v, E, d, 0.25)
+    Kx = O.decode_tensor_cluster(d, ck, cent_k, E, exact=True)
+    Vx = O.decode_tensor_cluster(d, cv, cent_v, E, exact=True)
+    np.testing.assert_allclose(fast, O.attention(Q, Kx, Vx, 0.25), rtol=1e-11, atol=1e-12)
