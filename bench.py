@@ -1,0 +1,524 @@
+#!/usr/bin/env python
+"""Benchmark of the predict-then-quantize-residual KV codec on one B200.
+
+One step = closed-loop encode of every layer of a Wan-1.3B-shaped history
+(30 layers x 32760 tokens x 12 heads x 128 channels, bf16; layer 0 INT4 anchor,
+layers 1-29 block-DPLR prediction with rank-64 low-rank term and INT2 g32
+residual with fp16 scale/zero) followed by the decode of every layer from the
+codes.  Inputs (6 GB) are resident in HBM and larger than L2, so every step
+streams from DRAM.  Metric: KV tokens encoded + decoded per second.
+
+Also measured, in the same run (N = 1): the attention of a 4680-query chunk over
+the compressed history of layer 15, one layer of the temporal codec (40 heads,
+65536 tokens, INT4 g64), and one layer of the clustered codec with
+mixed-dimensional attention (16 heads, 32768 tokens, 1560 queries).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 run under torch.distributed.run; every rank codes its own 32760-token
+shard (weak scaling, no collective on the data path).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from clustered_kv_cache_b200 import kvc, synth  # noqa: E402
+
+L_LAYERS, T_TOK, H, D, RANK = 30, 21 * 1560, 12, 128, 64
+METRIC = "KV tokens/s encoded+decoded (GB/s vs HBM peak); compressed-attn TFLOP/s vs roofline"
+UNIT = "KV tokens/s"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.dev)], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the cross-layer workload
+
+
+class XLayerBench:
+    """Buffers and calls of the 30-layer encode + decode step."""
+
+    def __init__(self, device, seed):
+        self.wl = synth.wan_xlayer(seed=seed, device=device, L=L_LAYERS, T=T_TOK, H=H, D=D, rank=RANK)
+        bf, hf = torch.bfloat16, torch.float16
+        self.desc0 = kvc.make_desc(T_TOK, H, D, bf, 4, 32, hf)  # INT4 anchor
+        self.desc = kvc.make_desc(T_TOK, H, D, bf, 2, 32, hf)
+        self.pred0 = kvc.make_predictor(kvc.PRED_NONE)
+        self.preds = [None] + [kvc.make_predictor(kvc.PRED_XLAYER_DPLR, self.wl.weights[l], rank=RANK)
+                               for l in range(1, L_LAYERS)]
+        self.codes = [kvc.alloc_codes(self.desc0, self.pred0, device)] + \
+                     [kvc.alloc_codes(self.desc, self.preds[l], device) for l in range(1, L_LAYERS)]
+        self.ws_enc = kvc.alloc_workspace(kvc.OP_ENCODE, self.desc, self.preds[1], device=device)
+        self.ws_dec = kvc.alloc_workspace(kvc.OP_DECODE, self.desc, self.preds[1], device=device)
+        mk = lambda: torch.empty(T_TOK, H, D, dtype=bf, device=device)
+        self.er = [(mk(), mk()), (mk(), mk())]  # encode-chain reconstructions (ping-pong)
+        self.dr = [(mk(), mk()), (mk(), mk())]  # decode-chain reconstructions
+        self.keep = None  # (K^_14, V^_14) for the attention row
+
+    def encode_chain(self, ev=None, keep_layer=None):
+        K, V = self.wl.K, self.wl.V
+        Kr, Vr = self.er[0]
+        kvc.kvc_encode_layer(self.desc0, self.pred0, K[0], V[0], None, None, self.codes[0], Kr, Vr)
+        for l in range(1, L_LAYERS):
+            Ks, Vs = self.er[(l - 1) % 2]
+            Kr, Vr = self.er[l % 2]
+            if ev is not None:
+                ev[l][0].record()
+            kvc.kvc_encode_layer(self.desc, self.preds[l], K[l], V[l], Ks, Vs, self.codes[l], Kr, Vr, self.ws_enc)
+            if ev is not None:
+                ev[l][1].record()
+            if keep_layer is not None and l == keep_layer - 1:
+                self.keep = (Kr.clone(), Vr.clone())
+
+    def decode_chain(self, ev=None):
+        Kr, Vr = self.dr[0]
+        kvc.kvc_decode_layer(self.desc0, self.pred0, self.codes[0], None, None, Kr, Vr)
+        for l in range(1, L_LAYERS):
+            Ks, Vs = self.dr[(l - 1) % 2]
+            Kr, Vr = self.dr[l % 2]
+            if ev is not None:
+                ev[l][0].record()
+            kvc.kvc_decode_layer(self.desc, self.preds[l], self.codes[l], Ks, Vs, Kr, Vr, self.ws_dec)
+            if ev is not None:
+                ev[l][1].record()
+
+    def step(self, ev_enc=None, ev_dec=None):
+        self.encode_chain(ev_enc)
+        self.decode_chain(ev_dec)
+
+    # algorithmic traffic / work of one predicted layer
+    def layer_bytes(self, encode: bool) -> int:
+        C = H * D
+        codes = kvc.kvc_codes_bytes(self.desc, self.preds[1])
+        w = sum(t.numel() * t.element_size() for t in self.wl.weights[1].values())
+        io = 2 * T_TOK * C * 2 * (3 if encode else 2)  # K,V in (encode) + sources in + recon out
+        return io + codes + w
+
+    @staticmethod
+    def layer_flops() -> int:
+        C = H * D
+        return 2 * T_TOK * (H * D * D + C * RANK + RANK * C + H * 2 * D * D + 2 * C * RANK + RANK * C)
+
+
+def time_events(pairs):
+    return [s.elapsed_time(e) for s, e in pairs]
+
+
+# ---------------------------------------------------------------- oracle timing (CPU)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_xlayer_rate(wl, n_tok: int, layers: int, budget_s: float) -> dict:
+    """Times the fp64 oracle's closed-loop encode + decode of `n_tok` tokens
+    through `layers` layers (tokens are independent, so this is an exact sample
+    of the workload).  Returns tokens/s (encoded + decoded)."""
+    from oracle import kvc_oracle as O
+
+    idx = torch.linspace(0, wl.K[0].shape[0] - 1, n_tok).long()
+    t64 = lambda t: t[idx.to(t.device)].detach().cpu().double().numpy()
+    K = [t64(k) for k in wl.K[:layers]]
+    V = [t64(v) for v in wl.V[:layers]]
+    W = [None] + [{k: v.detach().cpu().double().numpy() for k, v in wl.weights[l].items()} for l in range(1, layers)]
+    d0 = O.Desc(n_tok, H, D, "bf16", 4, 32, "f16")
+    d = O.Desc(n_tok, H, D, "bf16", 2, 32, "f16")
+    t0 = time.perf_counter()
+    done = 0
+    ck, cv, Kh, Vh = O.encode_layer_none(d0, K[0], V[0])
+    Kd, Vd = O.decode_layer_none(d0, ck, cv)
+    done += 2
+    for l in range(1, layers):
+        ck, cv, Kh2, Vh2 = O.encode_layer_xlayer(d, W[l], K[l], V[l], Kh, Vh)
+        Kd, Vd = O.decode_layer_xlayer(d, W[l], ck, cv, Kd, Vd)
+        Kh, Vh = Kh2, Vh2
+        done += 2
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done * n_tok / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n_tok} of {T_TOK} tokens (evenly spaced) through {done // 2} of {L_LAYERS} layers, "
+                      f"encode + decode, fp64 numpy; {dt:.1f} s"}
+
+
+def run_reference(args, rank: int):
+    """Reference arm: the fp64 oracle on the host cores, same metric and config."""
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 1, device=dev, L=L_LAYERS, T=T_TOK if dev == "cuda" else 512,
+                          H=H, D=D, rank=RANK)
+    for _ in range(args.warmup):
+        oracle_xlayer_rate(wl, 64, 2, 5.0)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        r = oracle_xlayer_rate(wl, 256, L_LAYERS, 8.0)
+        secs.append(time.perf_counter() - t0)
+        vals.append(r["value"])
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.median(secs),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded Wan-1.3B-shaped trace, least-squares block-DPLR predictors)",
+            "config": {"workload": "cross-layer codec, 30 layers x 32760 tokens x 12 heads x 128, INT2 g32 + INT4 "
+                                   "anchor, rank 64; each step a bounded token sample", "global_batch": T_TOK,
+                       "seq_len": T_TOK, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- extra rows (N = 1)
+
+
+def row_attention(xb: XLayerBench, hbm, tf_burst, tf_sust, reps=3) -> dict:
+    """4680 queries (3 latent frames) over layer 15's compressed history plus the
+    chunk itself; the history is decoded inside the attention kernel."""
+    dev = xb.wl.K[0].device
+    n_q = 3 * 1560
+    Q = synth.queries(synth.SEED_BASE + 2, n_q, H, D, device=dev)
+    Ks = synth.queries(synth.SEED_BASE + 12, n_q, H, D, device=dev)
+    Vs = synth.queries(synth.SEED_BASE + 22, n_q, H, D, device=dev)
+    O_ = torch.empty(n_q, H, D, dtype=torch.bfloat16, device=dev)
+    l = 15
+    ws = kvc.alloc_workspace(kvc.OP_ATTEND, xb.desc, xb.preds[l], n_q, device=dev)
+    Kh, Vh = xb.keep
+    call = lambda: kvc.kvc_attend_compressed(xb.desc, xb.preds[l], Q, xb.codes[l], Kh, Vh, Ks, Vs, D ** -0.5,
+                                             O_, ws)
+    call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for s, e in ev:
+        s.record()
+        call()
+        e.record()
+    torch.cuda.synchronize()
+    ms = statistics.median(time_events(ev))
+    attn_flops = 4 * n_q * (T_TOK + n_q) * H * D
+    total = attn_flops + XLayerBench.layer_flops()
+    tflops = total / (ms * 1e-3) / 1e12
+    return {"workload": "4680 queries x (32760 compressed + 4680 chunk) keys, 12 heads x 128, layer 15",
+            "ms": ms, "value": tflops, "unit": "TFLOP/s (attention + one in-kernel decode of the history)",
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_burst, "unit": "TFLOP/s",
+                         "frac": tflops / tf_burst, "traffic": None, "peak_kind": "burst bf16"}}
+
+
+def row_temporal(dev, hbm, reps=3) -> dict:
+    tw = synth.temporal_layer(seed=synth.SEED_BASE + 3, device=dev)
+    T, Hh, Dd = tw.K.shape
+    desc = kvc.make_desc(T, Hh, Dd, torch.bfloat16, 4, 64, torch.float16, tw.frame_tokens, 4)
+    pred = kvc.make_predictor(kvc.PRED_TEMPORAL, {"k_block": tw.ak, "v_block": tw.av})
+    buf = kvc.alloc_codes(desc, pred, dev)
+    Kr, Vr = torch.empty_like(tw.K), torch.empty_like(tw.V)
+    enc = lambda: kvc.kvc_encode_layer(desc, pred, tw.K, tw.V, None, None, buf, None, None)
+    dec = lambda: kvc.kvc_decode_layer(desc, pred, buf, None, None, Kr, Vr)
+    out = {}
+    for name, fn in (("encode", enc), ("decode", dec)):
+        fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for s, e in ev:
+            s.record()
+            fn()
+            e.record()
+        torch.cuda.synchronize()
+        ms = statistics.median(time_events(ev))
+        codes = kvc.kvc_codes_bytes(desc, pred)
+        byts = 2 * T * Hh * Dd * 2 + codes + 2 * tw.ak.numel() * 2
+        gbs = byts / (ms * 1e-3) / 1e9
+        out[name] = {"ms": ms, "tokens_per_s": T / (ms * 1e-3),
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                                  "traffic": None}}
+    out["workload"] = "temporal codec, one layer: 65536 tokens x 40 heads x 128, 1560-token frames, INT4 g64"
+    return out
+
+
+def row_cluster(dev, hbm, tf_burst, reps=3) -> dict:
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 4, device=dev)
+    T, Hh, Dd = cw.K.shape
+    desc = kvc.make_desc(T, Hh, Dd, torch.bfloat16, 4, 32, torch.float16)
+    w = dict(k_centroids=cw.k_centroids, k_enc=cw.k_enc, k_dec=cw.k_dec, v_centroids=cw.v_centroids,
+             v_enc=cw.v_enc, v_dec=cw.v_dec)
+    pred = kvc.make_predictor(kvc.PRED_CLUSTER, w, n_clusters=256, code_dim=128)
+    buf = kvc.alloc_codes(desc, pred, dev)
+    Kr, Vr = torch.empty_like(cw.K), torch.empty_like(cw.V)
+    wse = kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred, device=dev)
+    wsd = kvc.alloc_workspace(kvc.OP_DECODE, desc, pred, device=dev)
+    n_q = 1560
+    Q = synth.queries(synth.SEED_BASE + 5, n_q, Hh, Dd, device=dev)
+    O_ = torch.empty(n_q, Hh, Dd, dtype=torch.bfloat16, device=dev)
+    wsa = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q, device=dev)
+    calls = {"encode": lambda: kvc.kvc_encode_layer(desc, pred, cw.K, cw.V, None, None, buf, None, None, wse),
+             "decode": lambda: kvc.kvc_decode_layer(desc, pred, buf, None, None, Kr, Vr, wsd),
+             "attention": lambda: kvc.kvc_attend_compressed(desc, pred, Q, buf, None, None, None, None, Dd ** -0.5,
+                                                            O_, wsa)}
+    out = {"workload": "clustered codec, one layer: 32768 tokens x 16 heads x 128, 256 centres, 128 INT4 g32 "
+                       "coefficients; mixed-dimensional attention of 1560 queries"}
+    for name, fn in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for s, e in ev:
+            s.record()
+            fn()
+            e.record()
+        torch.cuda.synchronize()
+        ms = statistics.median(time_events(ev))
+        C = Hh * Dd
+        if name == "attention":
+            fl = 4 * n_q * T * Hh * 128
+            tf = fl / (ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": tf, "peak": tf_burst, "unit": "TFLOP/s", "frac": tf / tf_burst}
+        elif name == "encode":
+            fl = 2 * 2 * T * C * (256 + 128 + 128)
+            tf = fl / (ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": tf, "peak": tf_burst, "unit": "TFLOP/s", "frac": tf / tf_burst}
+        else:
+            byts = 2 * T * C * 2 + kvc.kvc_codes_bytes(desc, pred)
+            gbs = byts / (ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
+        roof["traffic"] = None
+        out[name] = {"ms": ms, "roofline": roof}
+    return out
+
+
+# ---------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-rows", action="store_true", help="skip the extra per-row measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the codec has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from clustered_kv_cache_b200 import build
+
+    build.build()
+    hbm, tf_burst, tf_sust, peak_kind = peaks()
+
+    xb = XLayerBench(dev, synth.SEED_BASE + 1 + 1000 * rank)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        xb.step()
+    torch.cuda.synchronize()
+    assert kvc.kvc_get_device_error() == 0
+
+    mk = lambda: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(L_LAYERS)]
+    ev_enc = [mk() for _ in range(args.steps)]
+    ev_dec = [mk() for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    clocks = Clocks(vis.split(",")[local] if vis else local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = kvc.kvc_launch_counter()
+    t_start.record()
+    for k in range(args.steps):
+        xb.step(ev_enc[k], ev_dec[k])
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    launches = kvc.kvc_launch_counter() - launches0
+    clk = clocks.stop()
+    assert kvc.kvc_get_device_error() == 0
+    ms_total = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    units_per_step = 2 * T_TOK * L_LAYERS * world
+    value = units_per_step / (ms_step * 1e-3)
+
+    enc_ms = statistics.mean(x for k in range(args.steps) for x in time_events(ev_enc[k][1:]))
+    dec_ms = statistics.mean(x for k in range(args.steps) for x in time_events(ev_dec[k][1:]))
+    enc_b, dec_b = xb.layer_bytes(True), xb.layer_bytes(False)
+    enc_gbs, dec_gbs = enc_b / (enc_ms * 1e-3) / 1e9, dec_b / (dec_ms * 1e-3) / 1e9
+    dom_enc = enc_ms >= dec_ms
+    roof = {"bound": "hbm", "achieved": enc_gbs if dom_enc else dec_gbs, "peak": hbm, "unit": "GB/s",
+            "frac": (enc_gbs if dom_enc else dec_gbs) / hbm, "traffic": None,
+            "kernel": "kvc_encode_layer (cross-layer, one layer)" if dom_enc else
+                      "kvc_decode_layer (cross-layer, one layer)",
+            "bytes_per_launch": enc_b if dom_enc else dec_b, "ms_per_launch": enc_ms if dom_enc else dec_ms,
+            "peak_kind": peak_kind}
+    flops = XLayerBench.layer_flops()
+    detail = {"encode_layer": {"ms": enc_ms, "GB/s": enc_gbs, "frac_hbm": enc_gbs / hbm, "bytes": enc_b,
+                               "TFLOP/s": flops / (enc_ms * 1e-3) / 1e12},
+              "decode_layer": {"ms": dec_ms, "GB/s": dec_gbs, "frac_hbm": dec_gbs / hbm, "bytes": dec_b,
+                               "TFLOP/s": flops / (dec_ms * 1e-3) / 1e12}}
+
+    # end to end: inputs from pinned host memory, codes back to the host
+    e2e = None
+    if args.e2e_steps > 0:
+        hK = [k.cpu().pin_memory() for k in xb.wl.K]
+        hV = [v.cpu().pin_memory() for v in xb.wl.V]
+        hcodes = [[torch.empty_like(t, device="cpu").pin_memory() for t in (c.k_codes, c.k_params, c.v_codes,
+                                                                            c.v_params)] for c in xb.codes]
+        bi = sum(t.numel() * t.element_size() for t in hK + hV)
+        bo = sum(t.numel() * t.element_size() for c in hcodes for t in c)
+
+        def e2e_step():
+            for l in range(L_LAYERS):
+                xb.wl.K[l].copy_(hK[l], non_blocking=True)
+                xb.wl.V[l].copy_(hV[l], non_blocking=True)
+            xb.step()
+            for c, hc in zip(xb.codes, hcodes):
+                for src, dst in zip((c.k_codes, c.k_params, c.v_codes, c.v_params), hc):
+                    dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e.record()
+        torch.cuda.synchronize()
+        ms_e2e = s.elapsed_time(e) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": units_per_step / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": bo, "ms_per_step": ms_e2e}
+        del hK, hV, hcodes
+
+    rows = None
+    cpu = None
+    if world == 1:
+        if not args.no_rows:
+            xb.encode_chain(keep_layer=15)
+            torch.cuda.synchronize()
+            rows = {"c2_attention": row_attention(xb, hbm, tf_burst, tf_sust)}
+            xb.keep = None
+            torch.cuda.empty_cache()
+            rows["c3_temporal"] = row_temporal(dev, hbm)
+            torch.cuda.empty_cache()
+            rows["c4_cluster"] = row_cluster(dev, hbm, tf_burst)
+        if not args.no_cpu:
+            cpu = oracle_xlayer_rate(xb.wl, 192, L_LAYERS, 20.0)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded Wan-1.3B-shaped trace, inter-layer correlation 0.9; block-DPLR "
+                        "predictors fitted by least squares on a separate 4096-token trace)",
+                "config": {"workload": "cross-layer codec: encode + decode of 30 layers x 32760 tokens x 12 heads "
+                                       "x 128, bf16, INT2 g32 residual (INT4 anchor), block-DPLR rank 64",
+                           "global_batch": T_TOK * world, "seq_len": T_TOK, "parallelism": f"dp{world}",
+                           "l2": "inputs larger than L2 (6 GB per step streamed)"},
+                "roofline": roof, "layers": detail, "clocks": clk, "gpu_launches": launches,
+                "e2e": e2e, "cpu_baseline": cpu, "rows": rows}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

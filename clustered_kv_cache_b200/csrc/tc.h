@@ -1,0 +1,20 @@
+// Tensor-core (tcgen05 / TMEM / TMA) kernels for bf16, head_dim 128 (internal).
+#pragma once
+
+#include "common.cuh"
+
+namespace kvc {
+
+bool tc_codec_supported(const kvc_layer_desc* d, const kvc_predictor* p);
+size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int64_t n_q);
+cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
+                           const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, void* ws,
+                           size_t ws_bytes, cudaStream_t st);
+bool tc_attend_supported(const kvc_layer_desc* d, const kvc_predictor* p, int64_t n_self);
+cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
+                      const kvc_codes* c, const void* Ks, const void* Vs, const void* K_self, const void* V_self,
+                      int64_t n_self, float scale, void* O, void* ws, size_t ws_bytes, cudaStream_t st);
+// reads the device error word of the current device and resets it to 0
+cudaError_t tc_read_and_clear_error(unsigned int* value);
+
+}  // namespace kvc

@@ -188,8 +188,9 @@ def fit_block_dplr(X_head: torch.Tensor, X_flat: torch.Tensor, Y: torch.Tensor, 
     Rf = R.reshape(T, H * D)
     M = _ridge_lstsq(X_flat, Rf)  # [Cin, C]
     F = X_flat.double() @ M
-    _, _, Vh = torch.linalg.svd(F, full_matrices=False)
-    Vr = Vh[:rank].T  # [C, r]
+    # top right singular vectors of F = top eigenvectors of F^T F
+    _, vecs = torch.linalg.eigh(F.T @ F)
+    Vr = vecs[:, -rank:].flip(-1).contiguous()  # [C, r]
     w = (M @ Vr).T  # [r, Cin]
     return blocks, w, Vr
 

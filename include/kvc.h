@@ -1,0 +1,222 @@
+/*
+ * kvc.h - C ABI of libkvc.so, a predict-then-quantize-residual KV-cache codec
+ * for autoregressive video diffusion, and attention over the compressed
+ * history, written for NVIDIA B200 (sm_100a).
+ *
+ * What the codec computes (sources by page title and figure / table):
+ *  - Every K/V row gets a prediction; only the residual (row - prediction) is
+ *    stored, as b-bit codes with one (scale, zero) pair per group of `group`
+ *    consecutive channels.  Scale s = (max - min) / (2^b - 1), zero z = min,
+ *    code q = clamp(rint((r - z) / s), 0, 2^b - 1); the reconstruction is
+ *    round_state(prediction + z + s*q).  ("CORAL-KV: Compact Cross-Layer
+ *    Prediction and Residual Coding for Autoregressive Video KV Caches",
+ *    Fig. 3 and Fig. 5; "TempoKV: Predictive KV Cache Quantization for
+ *    Autoregressive Video Generation", Fig. 2(b), Tables 1-3.)
+ *  - Predictions always use reconstructed, never clean, states (closed loop).
+ *  - KVC_PRED_NONE: prediction 0 (the anchor: CORAL-KV layer 0, Fig. 8;
+ *    TempoKV frame 0, appendix Table 7).
+ *  - KVC_PRED_XLAYER_DPLR: K_l from the reconstructed K_{l-1}, V_l from the
+ *    reconstructed [K_l, V_{l-1}], each by a per-head block-diagonal map plus
+ *    a global rank-r map ("CORAL-KV ...", abstract and Fig. 3).
+ *  - KVC_PRED_TEMPORAL: inside one layer, K of frame f from the reconstructed K
+ *    of frames f-1 and f-2 at the same spatial position, V of frame f from the
+ *    reconstructed K of frame f plus V of frame f-1 ("TempoKV ...", Fig. 2(b)).
+ *    Frame 0 is coded with prediction 0 at anchor_bits; at frame 1 the missing
+ *    lag-2 frame is zero.
+ *  - KVC_PRED_CLUSTER: each token's whole (all heads) K row is predicted by its
+ *    nearest centre c_a (ties to the lowest index); the residual is mapped to
+ *    code_dim coefficients by an encoder, those are coded, and decoding is
+ *    c_a + W_dec * coefficients ("NanoKV: High-Ratio KV Cache Compression for
+ *    Autoregressive Video Generation", abstract).
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors are row-major.  K, V, Q, O and reconstructions are [T][H][D].
+ *    Weights use the [out][in] convention, y = x * W^T.
+ *  - Every pointer is caller-owned device memory unless stated otherwise;
+ *    the library keeps no allocation between calls.  All device pointers must
+ *    be 16-byte aligned (KVC_ERR_MISALIGNED otherwise).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls validate their arguments synchronously, enqueue work on `stream`
+ *    and return; nothing is launched when validation fails.
+ *  - Kernel launch failures return KVC_ERR_CUDA.  Kernels that wait on
+ *    hardware barriers give up after a bounded time and record
+ *    KVC_ERR_DEVICE_TIMEOUT in a device word read by kvc_get_device_error().
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVC_API __attribute__((visibility("default")))
+#else
+#define KVC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVC_OK = 0,
+  KVC_ERR_INVALID_ARGUMENT = 1, /* NULL where a buffer is required, bad sizes */
+  KVC_ERR_UNSUPPORTED = 2,      /* a combination this build does not implement */
+  KVC_ERR_MISALIGNED = 3,       /* a device pointer not 16-byte aligned */
+  KVC_ERR_WORKSPACE_TOO_SMALL = 4,
+  KVC_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed */
+  KVC_ERR_DEVICE_TIMEOUT = 6    /* a bounded device-side wait gave up */
+} kvc_status;
+
+typedef enum { KVC_F32 = 0, KVC_BF16 = 1, KVC_F16 = 2 } kvc_dtype;
+
+typedef enum {
+  KVC_PRED_NONE = 0,
+  KVC_PRED_XLAYER_DPLR = 1,
+  KVC_PRED_TEMPORAL = 2,
+  KVC_PRED_CLUSTER = 3
+} kvc_pred_kind;
+
+/* One layer's history.
+ *  n_tokens T >= 0; n_heads H >= 1; head_dim D in {64, 128}.
+ *  dtype: KVC_F32 or KVC_BF16; the type of K, V, Q, O, reconstructions and
+ *         predictor weights.  Arithmetic accumulates in fp32.
+ *  bits in {2, 4, 8}; group divides D (clustered: divides code_dim) and is a
+ *         multiple of D/32.
+ *  param_dtype: KVC_F16 or KVC_F32; the (scale, zero) storage type.
+ *  frame_tokens: tokens per frame (temporal only; token t = f*frame_tokens+s).
+ *  anchor_bits: bits of frame 0 (temporal only). */
+typedef struct {
+  int64_t n_tokens;
+  int32_t n_heads;
+  int32_t head_dim;
+  int32_t dtype;
+  int32_t bits;
+  int32_t group;
+  int32_t param_dtype;
+  int32_t frame_tokens;
+  int32_t anchor_bits;
+} kvc_layer_desc;
+
+/* Predictor weights (device pointers, dtype of the layer, read only).
+ *  XLAYER_DPLR: k_block [H][D][D], k_w [rank][C], k_u [C][rank],
+ *               v_block [H][D][2D] over the per-head input [K_l,h | V_{l-1},h],
+ *               v_w [rank][2C] over [K_l | V_{l-1}], v_u [C][rank];
+ *               C = H*D; rank may be 0 (then k_w, k_u, v_w, v_u may be NULL).
+ *  TEMPORAL:    k_block [H][D][2D] over [K_{f-1},h | K_{f-2},h],
+ *               v_block [H][D][2D] over [K_f,h | V_{f-1},h].
+ *  CLUSTER:     k_centroids [n_clusters][C], k_enc [code_dim][C],
+ *               k_dec [C][code_dim], and the same for v; n_clusters <= 256. */
+typedef struct {
+  int32_t kind;
+  int32_t rank;
+  int32_t n_clusters;
+  int32_t code_dim;
+  const void *k_block, *k_w, *k_u;
+  const void *v_block, *v_w, *v_u;
+  const void *k_centroids, *k_enc, *k_dec;
+  const void *v_centroids, *v_enc, *v_dec;
+} kvc_predictor;
+
+/* Compressed storage of one layer (device pointers, caller-owned).
+ *  NONE / XLAYER: k_codes [T][H][D*bits/8] bytes, k_params [T][H][D/group][2]
+ *    of (scale, zero) in param_dtype; element j of a row sits at bits
+ *    [j*bits, (j+1)*bits) of the row, least significant bit first.
+ *  TEMPORAL: as above, except that the rows of frame 0 come first at
+ *    anchor_bits, followed by the rows of all later frames at bits.
+ *  CLUSTER: k_codes [T][code_dim*bits/8], k_params [T][code_dim/group][2],
+ *    k_assign [T] uint8 centre index.
+ *  The v_* members hold V the same way.  Sizes: kvc_codes_sizes(). */
+typedef struct {
+  void *k_codes, *k_params, *v_codes, *v_params;
+  void *k_assign, *v_assign;
+} kvc_codes;
+
+/* Bytes of each buffer of kvc_codes for one tensor (K; V is the same). */
+typedef struct {
+  size_t codes;
+  size_t params;
+  size_t assign;
+} kvc_codes_size;
+
+/* Closed-form storage of one tensor's codes, parameters and assignments.
+ * Returns KVC_ERR_INVALID_ARGUMENT / KVC_ERR_UNSUPPORTED for bad descriptors.
+ * The ratio 16 / (bits + 32/group) of bf16 data to INT-b codes with fp16
+ * (scale, zero) pairs is the 5.33x (INT2) / 3.20x (INT4) of "TempoKV ...",
+ * Tables 1-3 and appendix Table 8. */
+KVC_API kvc_status kvc_codes_sizes(const kvc_layer_desc* desc, const kvc_predictor* pred, kvc_codes_size* out);
+
+/* Total bytes (K and V) of codes + parameters + assignments of one layer;
+ * 0 for an invalid descriptor. */
+KVC_API size_t kvc_codes_bytes(const kvc_layer_desc* desc, const kvc_predictor* pred);
+
+/* Operation codes of kvc_workspace_bytes. */
+enum { KVC_OP_ENCODE = 0, KVC_OP_DECODE = 1, KVC_OP_ATTEND = 2 };
+
+/* Device workspace (bytes) that `op` needs for this layer; n_q = number of
+ * query rows (attend only).  The caller passes a buffer of at least this size
+ * as `ws`; its contents are scratch and need no initialisation. */
+KVC_API size_t kvc_workspace_bytes(int op, const kvc_layer_desc* desc, const kvc_predictor* pred, int64_t n_q);
+
+/* Encode one layer: prediction, residual, group quantization, packing, and the
+ * closed-loop reconstruction.
+ *  K, V:         [T][H][D] clean values of this layer (read).
+ *  K_src, V_src: XLAYER: reconstructions of layer l-1 [T][H][D] (read);
+ *                ignored (may be NULL) for the other kinds.
+ *  out:          codes / params / assignments (written).
+ *  K_rec, V_rec: reconstructions of this layer (written); may be NULL unless
+ *                the caller chains them into the next layer, except that
+ *                XLAYER needs K_rec (V's prediction reads the reconstructed K).
+ *  ws, ws_bytes: workspace of kvc_workspace_bytes(KVC_OP_ENCODE, ...).
+ * Temporal layers need T >= 1 and frame_tokens >= 1; the whole layer's frame
+ * chain runs inside this call. */
+KVC_API kvc_status kvc_encode_layer(const kvc_layer_desc* desc, const kvc_predictor* pred, const void* K,
+                            const void* V, const void* K_src, const void* V_src, const kvc_codes* out,
+                            void* K_rec, void* V_rec, void* ws, size_t ws_bytes, void* stream);
+
+/* Decode one layer: unpack, dequantize, replay the same prediction chain and
+ * add; K_rec and V_rec [T][H][D] are required.  K_src / V_src as for encode. */
+KVC_API kvc_status kvc_decode_layer(const kvc_layer_desc* desc, const kvc_predictor* pred, const kvc_codes* codes,
+                            const void* K_src, const void* V_src, void* K_rec, void* V_rec, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* Softmax attention of Q [n_q][H][D] over this layer's compressed history,
+ * followed by n_self uncompressed tokens K_self / V_self [n_self][H][D]
+ * (non-causal; n_self may be 0 and the pointers NULL):
+ *   O = softmax(scale * Q [K_hist; K_self]^T) [V_hist; V_self].
+ * NONE / XLAYER: the history is decoded tile by tile on chip (bf16, D = 128:
+ * never written to device memory).  CLUSTER: scores and values are computed on
+ * the stored coefficients, q.c_a + (W_dec^T q).coef, without rebuilding full
+ * keys ("NanoKV ...", abstract: the Fast variant); n_self must be 0.
+ * TEMPORAL: KVC_ERR_UNSUPPORTED.  O [n_q][H][D] is written. */
+KVC_API kvc_status kvc_attend_compressed(const kvc_layer_desc* desc, const kvc_predictor* pred, const void* Q,
+                                 int64_t n_q, const kvc_codes* codes, const void* K_src, const void* V_src,
+                                 const void* K_self, const void* V_self, int64_t n_self, float scale,
+                                 void* O, void* ws, size_t ws_bytes, void* stream);
+
+/* Pack n codes (uint8, each < 2^bits) into n*bits/8 bytes, LSB first;
+ * n*bits must be a multiple of 128 (whole 16-byte words). */
+KVC_API kvc_status kvc_pack_codes(const uint8_t* codes, int64_t n, int bits, void* packed, void* stream);
+
+/* Inverse of kvc_pack_codes. */
+KVC_API kvc_status kvc_unpack_codes(const void* packed, int64_t n, int bits, uint8_t* codes, void* stream);
+
+/* Synchronizes `stream`, returns the first device-side error recorded since
+ * the last call (KVC_OK if none) and clears it. */
+KVC_API kvc_status kvc_get_device_error(void* stream);
+
+/* Static description of a status code. */
+KVC_API const char* kvc_status_string(kvc_status status);
+
+/* Text of the last CUDA error seen by this thread's calls (or ""). */
+KVC_API const char* kvc_last_cuda_error(void);
+
+/* Number of kernels this process has launched through the library so far
+ * (all threads, all devices); for counting launches in a timed region. */
+KVC_API uint64_t kvc_launch_counter(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVC_H */

@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI: the library loads on a machine without a GPU,
+exports every entry point include/kvc.h declares, reports the closed-form
+storage the oracle computes, and rejects bad arguments before any launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from clustered_kv_cache_b200 import build as kbuild
+from clustered_kv_cache_b200 import kvc
+from oracle import kvc_oracle as O
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "kvc.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    kbuild.build()
+    return kvc.lib()
+
+
+def test_exports_every_declared_entry_point(L):
+    with open(HEADER) as f:
+        declared = re.findall(r"KVC_API\s+[\w\s\*]+?\b(kvc_\w+)\s*\(", f.read())
+    assert len(declared) >= 11
+    assert sorted(declared) == sorted(set(declared))
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) <= set(kvc.EXPORTED) | set(declared)
+
+
+@pytest.mark.parametrize("kind,bits,group,param,T,H,D,F,ab", [
+    ("none", 2, 32, "f16", 32760, 12, 128, 0, 4),
+    ("none", 4, 32, "f32", 512, 2, 64, 0, 4),
+    ("temporal", 4, 64, "f16", 65536, 40, 128, 1560, 4),
+    ("temporal", 2, 32, "f16", 1000, 2, 64, 64, 8),
+    ("cluster", 4, 32, "f16", 32768, 16, 128, 0, 4),
+])
+def test_codes_bytes_match_oracle_accounting(L, kind, bits, group, param, T, H, D, F, ab):
+    kinds = {"none": kvc.PRED_NONE, "temporal": kvc.PRED_TEMPORAL, "cluster": kvc.PRED_CLUSTER}
+    dt = torch.float16 if param == "f16" else torch.float32
+    desc = kvc.make_desc(T, H, D, torch.bfloat16, bits, group, dt, F, ab)
+    pred = kvc.make_predictor(kinds[kind], n_clusters=256 if kind == "cluster" else 0,
+                              code_dim=128 if kind == "cluster" else 0)
+    od = O.Desc(T, H, D, bits=bits, group=group, param=param, frame_tokens=F, anchor_bits=ab)
+    assert kvc.kvc_codes_bytes(desc, pred) == O.codes_bytes(od, kind, code_dim=128)
+
+
+def _call_encode(L, desc, pred, K=0x1000, V=0x1000, Ks=0x1000, Vs=0x1000, codes=None, Kr=0x1000, Vr=0x1000,
+                 ws=None, wsn=0):
+    c = codes or kvc.Codes(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    return L.kvc_encode_layer(ctypes.byref(desc), ctypes.byref(pred), K, V, Ks, Vs, ctypes.byref(c), Kr, Vr, ws, wsn,
+                              None)
+
+
+def test_validation_errors_without_launch(L):
+    good = kvc.make_desc(100, 2, 128, torch.bfloat16, 2, 32)
+    none = kvc.make_predictor(kvc.PRED_NONE)
+    assert _call_encode(L, good, none, K=None) == 1  # NULL input
+    assert _call_encode(L, good, none, K=0x1008) == 3  # misaligned
+    for bad in (kvc.make_desc(100, 2, 96, torch.bfloat16, 2, 32),    # head_dim
+                kvc.make_desc(100, 2, 128, torch.bfloat16, 3, 32),   # bits
+                kvc.make_desc(100, 2, 128, torch.bfloat16, 2, 48),   # group does not divide D
+                kvc.make_desc(100, 2, 128, torch.bfloat16, 2, 2)):   # group narrower than a lane's share
+        assert _call_encode(L, bad, none) == 2
+    assert _call_encode(L, kvc.make_desc(-1, 2, 128), none) == 1
+    xl = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, rank=8)
+    assert _call_encode(L, good, xl) == 1  # missing weights
+    xl = kvc.Predictor(kvc.PRED_XLAYER_DPLR, 8, 0, 0, *([0x1000] * 12))
+    need = kvc.kvc_workspace_bytes(kvc.OP_ENCODE, good, xl)
+    assert need >= 2 * 100 * 8 * 4
+    assert _call_encode(L, good, xl, ws=0x1000, wsn=need - 1) == 4
+    assert _call_encode(L, good, xl, Kr=None) == 1  # V's prediction needs K_rec
+    tmp = kvc.make_predictor(kvc.PRED_TEMPORAL)
+    assert _call_encode(L, kvc.make_desc(100, 2, 128, frame_tokens=0), tmp) == 2 or \
+        _call_encode(L, kvc.make_desc(100, 2, 128, frame_tokens=0), tmp) == 1
+    c = kvc.Codes(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    q = ctypes.c_void_p(0x1000)
+    # attention over a temporal history is not offered; clustered attention takes no self tokens
+    tp = kvc.Predictor(kvc.PRED_TEMPORAL, 0, 0, 0, *([0x1000] * 12))
+    st = L.kvc_attend_compressed(ctypes.byref(kvc.make_desc(100, 2, 128, frame_tokens=10)), ctypes.byref(tp), q, 4,
+                                 ctypes.byref(c), None, None, None, None, 0, 1.0, q, None, 0, None)
+    assert st == 2
+    cp = kvc.Predictor(kvc.PRED_CLUSTER, 0, 16, 128, *([0x1000] * 12))
+    st = L.kvc_attend_compressed(ctypes.byref(good), ctypes.byref(cp), q, 4, ctypes.byref(c), None, None, q, q, 8,
+                                 1.0, q, None, 0, None)
+    assert st == 2
+    assert L.kvc_pack_codes(q, 100, 2, q, None) == 1  # not whole 16-byte words
+    assert L.kvc_pack_codes(q, 64, 3, q, None) == 2
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert kvc.kvc_status_string(s)
+    assert kvc.kvc_status_string(99) == "unknown status"

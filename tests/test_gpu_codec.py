@@ -1,0 +1,435 @@
+"""Parity of the CUDA codec (through the C ABI) with the fp64 oracle.
+
+Each test feeds the GPU and the oracle the same seeded inputs; where a layer's
+prediction source is a reconstruction, both receive the oracle's (teacher
+forcing), so each call is checked on its own.  Tolerances: tests/kvc_testutil.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from clustered_kv_cache_b200 import kvc, synth
+from oracle import kvc_oracle as O
+
+import kvc_testutil as U
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from clustered_kv_cache_b200 import build
+
+    build.build()
+    kvc.lib()
+
+
+def _sync_ok():
+    torch.cuda.synchronize()
+    assert kvc.kvc_get_device_error() == 0
+
+
+def _desc(T, H, D, dtype, bits, group, param, F=0, ab=4):
+    return kvc.make_desc(T, H, D, dtype, bits, group, param, F, ab)
+
+
+def _odesc(T, H, D, dtype, bits, group, param, F=0, ab=4):
+    return O.Desc(T, H, D, U.np_state(dtype), bits, group, U.np_param(param), F, ab)
+
+
+def _gpu_coded(buf: kvc.CodeBuffers, T, H, D, bits, group, param, which="k"):
+    codes = getattr(buf, which + "_codes")
+    params = getattr(buf, which + "_params")
+    q = U.codes_from_gpu(codes, (T, H, D), bits)
+    s, z = U.params_from_gpu(params, (T, H, D // group), param)
+    return O.Coded(q, s, z)
+
+
+def _compare(gc: O.Coded, oc: O.Coded, rec_gpu, rec_ref, exact, x, state, group, what):
+    U.assert_codes_close(gc.q, oc.q, what + " codes")
+    flip = gc.q != oc.q
+    U.assert_recon_close(rec_gpu, rec_ref, exact, x, flip, state, what + " recon")
+    # parameters: the same fp16 / fp32 values except where fp rounding of min/max moved them
+    same = (gc.s == oc.s).mean()
+    assert same > 0.999, f"{what} scales agree on {same:.5f}"
+
+
+# ---------------------------------------------------------------- packing
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_pack_unpack_bit_exact(bits):
+    rng = np.random.default_rng(bits)
+    n = (128 // bits) * 16 * 37
+    q = rng.integers(0, 1 << bits, n, dtype=np.uint8)
+    ref = O.pack_codes(q, bits)
+    out = torch.empty(n * bits // 8, dtype=torch.uint8, device="cuda")
+    kvc.kvc_pack_codes(torch.from_numpy(q).cuda(), bits, out)
+    back = torch.empty(n, dtype=torch.uint8, device="cuda")
+    kvc.kvc_unpack_codes(torch.from_numpy(ref).cuda(), n, bits, back)
+    _sync_ok()
+    np.testing.assert_array_equal(out.cpu().numpy(), ref)
+    np.testing.assert_array_equal(back.cpu().numpy(), q)
+
+
+# ---------------------------------------------------------------- anchor / plain group RTN
+
+
+@pytest.mark.parametrize("dtype,param,bits,group,T,H,D", [
+    (torch.bfloat16, torch.float16, 4, 32, 300, 12, 128),
+    (torch.bfloat16, torch.float16, 2, 32, 97, 3, 128),
+    (torch.bfloat16, torch.float16, 2, 64, 65, 2, 64),
+    (torch.float32, torch.float32, 4, 32, 130, 2, 64),
+    (torch.bfloat16, torch.float16, 8, 16, 40, 2, 128),
+])
+def test_anchor_codec_parity(dtype, param, bits, group, T, H, D):
+    g = torch.Generator().manual_seed(T * 7 + bits)
+    K = (torch.randn(T, H, D, generator=g) * torch.exp2(torch.randint(-2, 3, (1, 1, D), generator=g))).to(dtype)
+    V = torch.randn(T, H, D, generator=g).to(dtype)
+    desc = _desc(T, H, D, dtype, bits, group, param)
+    pred = kvc.make_predictor(kvc.PRED_NONE)
+    buf = kvc.alloc_codes(desc, pred)
+    Kr, Vr = torch.empty_like(K, device="cuda"), torch.empty_like(V, device="cuda")
+    kvc.kvc_encode_layer(desc, pred, K.cuda(), V.cuda(), None, None, buf, Kr, Vr)
+    Kd, Vd = torch.empty_like(Kr), torch.empty_like(Vr)
+    kvc.kvc_decode_layer(desc, pred, buf, None, None, Kd, Vd)
+    _sync_ok()
+    assert torch.equal(Kd, Kr) and torch.equal(Vd, Vr)
+    od = _odesc(T, H, D, dtype, bits, group, param)
+    ck, cv, Kh, Vh = O.encode_layer_none(od, U.to64(K), U.to64(V))
+    for which, oc, rec, ref, x in (("k", ck, Kr, Kh, K), ("v", cv, Vr, Vh, V)):
+        gc = _gpu_coded(buf, T, H, D, bits, group, U.np_param(param), which)
+        _compare(gc, oc, U.to64(rec), ref, U.exact_none(oc, group), U.to64(x), od.state, group, which)
+
+
+def test_empty_layer_is_a_no_op():
+    desc = _desc(0, 2, 128, torch.bfloat16, 2, 32, torch.float16)
+    pred = kvc.make_predictor(kvc.PRED_NONE)
+    buf = kvc.alloc_codes(desc, pred)
+    e = torch.empty(0, 2, 128, dtype=torch.bfloat16, device="cuda")
+    kvc.kvc_encode_layer(desc, pred, e, e, None, None, buf, e, e)
+    _sync_ok()
+
+
+# ---------------------------------------------------------------- cross-layer block-DPLR
+
+
+def _xlayer_gpu(desc, pred, K, V, Ks, Vs):
+    buf = kvc.alloc_codes(desc, pred)
+    Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+    ws = kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred)
+    kvc.kvc_encode_layer(desc, pred, K, V, Ks, Vs, buf, Kr, Vr, ws)
+    Kd, Vd = torch.empty_like(K), torch.empty_like(V)
+    wsd = kvc.alloc_workspace(kvc.OP_DECODE, desc, pred)
+    kvc.kvc_decode_layer(desc, pred, buf, Ks, Vs, Kd, Vd, wsd)
+    _sync_ok()
+    assert torch.equal(Kd, Kr) and torch.equal(Vd, Vr), "decode must replay encode exactly"
+    return buf, Kr, Vr
+
+
+def _check_xlayer_layer(w, K, V, Ks, Vs, dtype, param, bits, group, rank):
+    """GPU vs oracle on one predicted layer, both fed the same K_src / V_src."""
+    T, H, D = K.shape
+    wg = {k: v.cuda() for k, v in w.items()}
+    desc = _desc(T, H, D, dtype, bits, group, param)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wg, rank=rank)
+    buf, Kr, Vr = _xlayer_gpu(desc, pred, K.cuda(), V.cuda(), Ks.cuda(), Vs.cuda())
+    od = _odesc(T, H, D, dtype, bits, group, param)
+    w64 = {k: U.to64(v) for k, v in w.items()}
+    Ks64, Vs64 = U.to64(Ks), U.to64(Vs)
+    ck, cv, Kh, Vh = O.encode_layer_xlayer(od, w64, U.to64(K), U.to64(V), Ks64, Vs64)
+    ek, ev = U.exact_xlayer(od, w64, ck, cv, Ks64, Vs64, Kh)
+    p = U.np_param(param)
+    # V is predicted from the GPU's own K_rec; where K codes agree the inputs are the same values
+    _compare(_gpu_coded(buf, T, H, D, bits, group, p, "k"), ck, U.to64(Kr), Kh, ek, U.to64(K), od.state, group, "K")
+    _compare(_gpu_coded(buf, T, H, D, bits, group, p, "v"), cv, U.to64(Vr), Vh, ev, U.to64(V), od.state, group, "V")
+    return Kh, Vh
+
+
+def test_tiny_fp32_cross_layer_chain():
+    """The tiny fp32 case: INT4 g32 anchor, then the true block-DPLR maps."""
+    wl = synth.tiny_xlayer()
+    T, H, D = wl.K[0].shape
+    f32 = torch.float32
+    # layer 0 (anchor)
+    desc0 = _desc(T, H, D, f32, 4, 32, f32)
+    p0 = kvc.make_predictor(kvc.PRED_NONE)
+    buf0 = kvc.alloc_codes(desc0, p0)
+    K0r, V0r = torch.empty(T, H, D, device="cuda"), torch.empty(T, H, D, device="cuda")
+    kvc.kvc_encode_layer(desc0, p0, wl.K[0].cuda(), wl.V[0].cuda(), None, None, buf0, K0r, V0r)
+    _sync_ok()
+    od0 = _odesc(T, H, D, f32, 4, 32, f32)
+    ck0, cv0, K0h, V0h = O.encode_layer_none(od0, U.to64(wl.K[0]), U.to64(wl.V[0]))
+    U.assert_codes_close(_gpu_coded(buf0, T, H, D, 4, 32, "f32", "k").q, ck0.q, "K0")
+    # layer 1 from the oracle's layer-0 reconstruction
+    _check_xlayer_layer(wl.weights[1], wl.K[1], wl.V[1], torch.from_numpy(K0h).float(),
+                        torch.from_numpy(V0h).float(), f32, f32, 4, 32, wl.rank)
+    # the GPU chain end to end against the oracle chain
+    w = {k: v.cuda() for k, v in wl.weights[1].items()}
+    desc1 = _desc(T, H, D, f32, 4, 32, f32)
+    p1 = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, w, rank=wl.rank)
+    buf1, K1r, V1r = _xlayer_gpu(desc1, p1, wl.K[1].cuda(), wl.V[1].cuda(), K0r, V0r)
+    ck1, cv1, K1h, V1h = O.encode_layer_xlayer(od0, {k: U.to64(v) for k, v in wl.weights[1].items()},
+                                               U.to64(wl.K[1]), U.to64(wl.V[1]), K0h, V0h)
+    U.assert_codes_close(_gpu_coded(buf1, T, H, D, 4, 32, "f32", "k").q, ck1.q, "chain K1")
+    U.assert_codes_close(_gpu_coded(buf1, T, H, D, 4, 32, "f32", "v").q, cv1.q, "chain V1")
+    np.testing.assert_allclose(U.to64(V1r), V1h, rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("T,rank", [(3 * 128 + 57, 64), (200, 0), (131, 16)])
+def test_bf16_cross_layer_parity(T, rank):
+    """Wan-shaped heads (12 x 128), INT2 g32 with fp16 (scale, zero); T spans
+    several 128-token tiles plus a ragged tail."""
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 101, L=3, T=T, rank=rank, calib_tokens=1024)
+    bf, hf = torch.bfloat16, torch.float16
+    for l in (1, 2):
+        # teacher forcing: layer l-1 sources are the clean values (bf16), shared by both sides
+        _check_xlayer_layer(wl.weights[l], wl.K[l], wl.V[l], wl.K[l - 1], wl.V[l - 1], bf, hf, 2, 32, rank)
+
+
+def test_bf16_cross_layer_full_size_sampled():
+    """Full Wan-shaped layer (32760 tokens); the oracle checks sampled tokens,
+    which are independent of one another through the whole layer."""
+    dev = "cuda"
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 1, device=dev, L=3, layers_needed=[2])
+    T, H, D = wl.K[2].shape
+    bf, hf = torch.bfloat16, torch.float16
+    w = wl.weights[2]
+    desc = _desc(T, H, D, bf, 2, 32, hf)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, w, rank=wl.rank)
+    buf, Kr, Vr = _xlayer_gpu(desc, pred, wl.K[2], wl.V[2], wl.K[1], wl.V[1])
+    idx = torch.cat([torch.arange(0, 64), torch.randint(64, T - 64, (320,), generator=torch.Generator().manual_seed(3)),
+                     torch.arange(T - 64, T)]).sort().values
+    sub = lambda t: U.to64(t[idx.to(t.device)])
+    od = _odesc(len(idx), H, D, bf, 2, 32, hf)
+    w64 = {k: U.to64(v) for k, v in w.items()}
+    ck, cv, Kh, Vh = O.encode_layer_xlayer(od, w64, sub(wl.K[2]), sub(wl.V[2]), sub(wl.K[1]), sub(wl.V[1]))
+    ek, ev = U.exact_xlayer(od, w64, ck, cv, sub(wl.K[1]), sub(wl.V[1]), Kh)
+    qk = U.codes_from_gpu(buf.k_codes, (T, H, D), 2)[idx.numpy()]
+    qv = U.codes_from_gpu(buf.v_codes, (T, H, D), 2)[idx.numpy()]
+    U.assert_codes_close(qk, ck.q, "K codes (sampled)")
+    U.assert_codes_close(qv, cv.q, "V codes (sampled)")
+    U.assert_recon_close(sub(Kr), Kh, ek, sub(wl.K[2]), qk != ck.q, "bf16", "K recon (sampled)")
+    U.assert_recon_close(sub(Vr), Vh, ev, sub(wl.V[2]), qv != cv.q, "bf16", "V recon (sampled)")
+
+
+# ---------------------------------------------------------------- temporal
+
+
+def _temporal_gpu(tw: synth.TemporalWorkload, bits, group, param, ab):
+    T, H, D = tw.K.shape
+    dtype = tw.K.dtype
+    desc = _desc(T, H, D, dtype, bits, group, param, tw.frame_tokens, ab)
+    pred = kvc.make_predictor(kvc.PRED_TEMPORAL, {"k_block": tw.ak.cuda(), "v_block": tw.av.cuda()})
+    buf = kvc.alloc_codes(desc, pred)
+    K, V = tw.K.cuda(), tw.V.cuda()
+    Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_encode_layer(desc, pred, K, V, None, None, buf, Kr, Vr)
+    Kd, Vd = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_decode_layer(desc, pred, buf, None, None, Kd, Vd)
+    _sync_ok()
+    assert torch.equal(Kd, Kr) and torch.equal(Vd, Vr)
+    return buf, Kr, Vr
+
+
+def _temporal_gpu_coded(buf, T, H, D, F, bits, ab, group, param, which):
+    F0 = min(F, T)
+    raw = getattr(buf, which + "_codes")
+    n0 = F0 * H * D * ab // 8
+    q0 = U.codes_from_gpu(raw[:n0], (F0, H, D), ab)
+    q1 = U.codes_from_gpu(raw[n0:], (T - F0, H, D), bits) if T > F0 else np.zeros((0, H, D), np.uint8)
+    s, z = U.params_from_gpu(getattr(buf, which + "_params"), (T, H, D // group), param)
+    return O.Coded(np.concatenate([q0, q1]), s, z)
+
+
+@pytest.mark.parametrize("T,H,D,F,bits,group,ab,dtype", [
+    (4 * 100 + 16, 4, 128, 100, 4, 64, 4, torch.bfloat16),
+    (3 * 50 + 7, 2, 64, 50, 2, 32, 8, torch.float32),
+    (37, 2, 128, 64, 4, 64, 4, torch.bfloat16),  # a single partial frame
+])
+def test_temporal_parity(T, H, D, F, bits, group, ab, dtype):
+    tw = synth.temporal_layer(seed=synth.SEED_BASE + 103, T=T, H=H, D=D, F=F, dtype=dtype)
+    param = torch.float16 if dtype == torch.bfloat16 else torch.float32
+    buf, Kr, Vr = _temporal_gpu(tw, bits, group, param, ab)
+    od = _odesc(T, H, D, dtype, bits, group, param, F, ab)
+    w64 = dict(ak=U.to64(tw.ak), av=U.to64(tw.av))
+    ck, cv, Kh, Vh = O.encode_layer_temporal(od, w64, U.to64(tw.K), U.to64(tw.V))
+    ek, ev = U.exact_temporal(od, w64, ck, cv, Kh, Vh)
+    p = U.np_param(param)
+    gk = _temporal_gpu_coded(buf, T, H, D, F, bits, ab, group, p, "k")
+    gv = _temporal_gpu_coded(buf, T, H, D, F, bits, ab, group, p, "v")
+    # the frame chain runs on both sides independently; flips can propagate one frame
+    _compare(gk, ck, U.to64(Kr), Kh, ek, U.to64(tw.K), od.state, group, "K")
+    _compare(gv, cv, U.to64(Vr), Vh, ev, U.to64(tw.V), od.state, group, "V")
+
+
+def test_temporal_full_size_sampled_positions():
+    """One full layer of the large-backbone case (65536 tokens, 40 heads, 1560
+    tokens per frame, INT4 g64): spatial positions are independent chains, so
+    the oracle replays a sample of positions through all 43 frames."""
+    tw = synth.temporal_layer(seed=synth.SEED_BASE + 3, device="cuda")
+    T, H, D = tw.K.shape
+    F = tw.frame_tokens
+    buf, Kr, Vr = _temporal_gpu(tw, 4, 64, torch.float16, 4)
+    n_last = T - (T // F) * F
+    pos = np.sort(np.concatenate([np.arange(0, 4), np.arange(n_last - 2, n_last + 2), [F - 1],
+                                  np.random.default_rng(5).choice(np.arange(n_last + 2, F - 1), 15, replace=False)]))
+    n_frames = (T + F - 1) // F
+    rows = []
+    for f in range(n_frames):
+        for s in pos:
+            if f * F + s < T:
+                rows.append(f * F + s)
+    rows = np.array(rows)
+    sub = lambda t: U.to64(t[torch.from_numpy(rows).to(t.device)])
+    od = _odesc(len(rows), H, D, torch.bfloat16, 4, 64, torch.float16, len(pos), 4)
+    w64 = dict(ak=U.to64(tw.ak), av=U.to64(tw.av))
+    ck, cv, Kh, Vh = O.encode_layer_temporal(od, w64, sub(tw.K), sub(tw.V))
+    qk = U.codes_from_gpu(buf.k_codes, (T, H, D), 4)[rows]
+    qv = U.codes_from_gpu(buf.v_codes, (T, H, D), 4)[rows]
+    U.assert_codes_close(qk, ck.q, "K codes (sampled positions)")
+    U.assert_codes_close(qv, cv.q, "V codes (sampled positions)")
+    ek, ev = U.exact_temporal(od, w64, ck, cv, Kh, Vh)
+    U.assert_recon_close(sub(Kr), Kh, ek, sub(tw.K), qk != ck.q, "bf16", "K recon")
+    U.assert_recon_close(sub(Vr), Vh, ev, sub(tw.V), qv != cv.q, "bf16", "V recon")
+
+
+# ---------------------------------------------------------------- clustered
+
+
+def _cluster_pred(cw: synth.ClusterWorkload, n_c):
+    w = dict(k_centroids=cw.k_centroids.cuda(), k_enc=cw.k_enc.cuda(), k_dec=cw.k_dec.cuda(),
+             v_centroids=cw.v_centroids.cuda(), v_enc=cw.v_enc.cuda(), v_dec=cw.v_dec.cuda())
+    return kvc.make_predictor(kvc.PRED_CLUSTER, w, n_clusters=n_c, code_dim=cw.k_enc.shape[0])
+
+
+@pytest.mark.parametrize("T,H,n_c", [(1000, 4, 32), (77, 16, 256)])
+def test_cluster_codec_parity(T, H, n_c):
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 104, T=T, H=H, n_c=n_c, iters=5)
+    D = 128
+    bf, hf = torch.bfloat16, torch.float16
+    desc = _desc(T, H, D, bf, 4, 32, hf)
+    pred = _cluster_pred(cw, n_c)
+    buf = kvc.alloc_codes(desc, pred)
+    K, V = cw.K.cuda(), cw.V.cuda()
+    Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+    ws = kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred)
+    kvc.kvc_encode_layer(desc, pred, K, V, None, None, buf, Kr, Vr, ws)
+    Kd, Vd = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_decode_layer(desc, pred, buf, None, None, Kd, Vd, kvc.alloc_workspace(kvc.OP_DECODE, desc, pred))
+    _sync_ok()
+    assert torch.equal(Kd, Kr) and torch.equal(Vd, Vr)
+    od = _odesc(T, H, D, bf, 4, 32, hf)
+    for which, X, cent, enc, dec, rec in (("k", cw.K, cw.k_centroids, cw.k_enc, cw.k_dec, Kr),
+                                          ("v", cw.V, cw.v_centroids, cw.v_enc, cw.v_dec, Vr)):
+        X64, c64 = U.to64(X), U.to64(cent)
+        oc, xh = O.encode_tensor_cluster(od, X64, c64, U.to64(enc), U.to64(dec))
+        a_gpu = getattr(buf, which + "_assign")[:T].cpu().numpy().astype(np.int64)
+        # the assignment is unique where the best and second-best scores are apart
+        sc = O.cluster_scores(X64.reshape(T, -1), c64)
+        srt = np.sort(sc, axis=1)
+        margin = srt[:, 1] - srt[:, 0]
+        clear = margin > 1e-4 * np.abs(srt[:, 0]) + 1e-3
+        np.testing.assert_array_equal(a_gpu[clear], oc.assign[clear])
+        assert np.all(sc[np.arange(T), a_gpu] <= srt[:, 0] + 1e-4 * np.abs(srt[:, 0]) + 1e-3)
+        assert clear.mean() > 0.99
+        q = U.codes_from_gpu(getattr(buf, which + "_codes"), (T, 128), 4)
+        s, z = U.params_from_gpu(getattr(buf, which + "_params"), (T, 4), "f16")
+        U.assert_codes_close(q, oc.q, which + " coefficient codes")
+        exact = (c64[oc.assign] + O.dequantize_groups(oc.q, oc.s, oc.z, 32) @ U.to64(dec).T).reshape(T, H, D)
+        flip = np.repeat((q != oc.q).any(axis=1), H * D).reshape(T, H, D)
+        U.assert_recon_close(U.to64(rec), xh, exact, X64, flip, "bf16", which + " recon")
+
+
+# ---------------------------------------------------------------- attention
+
+
+def _oracle_codes_to_gpu(ck, cv, bits, param, assign=False):
+    t = lambda q: U.pad16(U.codes_to_gpu(q, bits))
+    p = lambda c: U.pad16(U.params_to_gpu(c.s, c.z, param))
+    buf = kvc.CodeBuffers(t(ck.q), p(ck), t(cv.q), p(cv))
+    if assign:
+        buf.k_assign = U.pad16(torch.from_numpy(ck.assign.astype(np.uint8)).cuda())
+        buf.v_assign = U.pad16(torch.from_numpy(cv.assign.astype(np.uint8)).cuda())
+    return buf
+
+
+@pytest.mark.parametrize("n_q,n_self,T,rank", [(300, 130, 3 * 128 + 5, 64), (129, 0, 256, 16), (64, 128, 100, 0)])
+def test_compressed_attention_cross_layer(n_q, n_self, T, rank):
+    """Attention over a decoded cross-layer history plus uncompressed chunk
+    tokens, history codes written by the oracle."""
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 102, L=2, T=T, rank=rank, calib_tokens=1024)
+    H, D = 12, 128
+    bf, hf = torch.bfloat16, torch.float16
+    od = _odesc(T, H, D, bf, 2, 32, hf)
+    w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
+    Ks, Vs = U.to64(wl.K[0]), U.to64(wl.V[0])
+    ck, cv, _, _ = O.encode_layer_xlayer(od, w64, U.to64(wl.K[1]), U.to64(wl.V[1]), Ks, Vs)
+    buf = _oracle_codes_to_gpu(ck, cv, 2, "f16")
+    Q = synth.queries(11, n_q, H, D)
+    Kself = synth.queries(12, n_self, H, D)
+    Vself = synth.queries(13, n_self, H, D)
+    desc = _desc(T, H, D, bf, 2, 32, hf)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=rank)
+    Og = torch.empty(n_q, H, D, dtype=bf, device="cuda")
+    ws = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q)
+    kvc.kvc_attend_compressed(desc, pred, Q.cuda(), buf, wl.K[0].cuda(), wl.V[0].cuda(),
+                              Kself.cuda() if n_self else None, Vself.cuda() if n_self else None,
+                              D ** -0.5, Og, ws)
+    _sync_ok()
+    ref = O.attend_compressed_xlayer(od, w64, U.to64(Q), ck, cv, Ks, Vs, U.to64(Kself) if n_self else None,
+                                     U.to64(Vself) if n_self else None, D ** -0.5)
+    err = U.rel_l2(U.to64(Og), ref)
+    assert err <= U.ATT_TOL[bf], err
+
+
+def test_tiny_fp32_attention():
+    """64 fp32 queries over the decoded 512-token tiny history (both layers)."""
+    wl = synth.tiny_xlayer()
+    T, H, D = wl.K[0].shape
+    f32 = torch.float32
+    od = _odesc(T, H, D, f32, 4, 32, f32)
+    ck0, cv0, K0h, V0h = O.encode_layer_none(od, U.to64(wl.K[0]), U.to64(wl.V[0]))
+    w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
+    ck1, cv1, _, _ = O.encode_layer_xlayer(od, w64, U.to64(wl.K[1]), U.to64(wl.V[1]), K0h, V0h)
+    Q = synth.queries(7, 64, H, D, dtype=f32)
+    desc = _desc(T, H, D, f32, 4, 32, f32)
+    for layer, (ck, cv) in enumerate(((ck0, cv0), (ck1, cv1))):
+        buf = _oracle_codes_to_gpu(ck, cv, 4, "f32")
+        if layer == 0:
+            pred = kvc.make_predictor(kvc.PRED_NONE)
+            src = (None, None)
+            ref = O.attention(U.to64(Q), *O.decode_layer_none(od, ck, cv), 0.125)
+        else:
+            pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()},
+                                      rank=wl.rank)
+            src = (torch.from_numpy(K0h).float().cuda(), torch.from_numpy(V0h).float().cuda())
+            ref = O.attend_compressed_xlayer(od, w64, U.to64(Q), ck, cv, K0h, V0h, None, None, 0.125)
+        Og = torch.empty(64, H, D, device="cuda")
+        ws = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, 64)
+        kvc.kvc_attend_compressed(desc, pred, Q.cuda(), buf, *src, None, None, 0.125, Og, ws)
+        _sync_ok()
+        assert U.rel_l2(U.to64(Og), ref) <= U.ATT_TOL[f32]
+
+
+@pytest.mark.parametrize("n_q,T,H,n_c", [(100, 1000, 4, 32), (33, 300, 16, 256)])
+def test_mixed_dimensional_attention(n_q, T, H, n_c):
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 105, T=T, H=H, n_c=n_c, iters=3)
+    D = 128
+    od = _odesc(T, H, D, torch.bfloat16, 4, 32, torch.float16)
+    ck, _ = O.encode_tensor_cluster(od, U.to64(cw.K), U.to64(cw.k_centroids), U.to64(cw.k_enc), U.to64(cw.k_dec))
+    cv, _ = O.encode_tensor_cluster(od, U.to64(cw.V), U.to64(cw.v_centroids), U.to64(cw.v_enc), U.to64(cw.v_dec))
+    buf = _oracle_codes_to_gpu(ck, cv, 4, "f16", assign=True)
+    Q = synth.queries(17, n_q, H, D)
+    desc = _desc(T, H, D, torch.bfloat16, 4, 32, torch.float16)
+    pred = _cluster_pred(cw, n_c)
+    Og = torch.empty(n_q, H, D, dtype=torch.bfloat16, device="cuda")
+    kvc.kvc_attend_compressed(desc, pred, Q.cuda(), buf, None, None, None, None, D ** -0.5, Og,
+                              kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q))
+    _sync_ok()
+    ref = O.mixed_attention(U.to64(Q), ck, U.to64(cw.k_centroids), U.to64(cw.k_dec), cv, U.to64(cw.v_centroids),
+                            U.to64(cw.v_dec), od, D ** -0.5)
+    assert U.rel_l2(U.to64(Og), ref) <= U.ATT_TOL[torch.bfloat16]
