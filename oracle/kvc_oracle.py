@@ -41,12 +41,15 @@ R4  groups are runs of `group` consecutive channels inside one (token, head) row
     (for the clustered codec: inside the 128 coefficients of a token).
 R5  the reconstruction x_hat = round_state(pred + (z + s*q)) is what later
     predictions consume (closed loop); state dtype is bf16 or fp32.
-R6  the low-rank latent z = x_hat @ W^T is rounded to the state dtype before
-    the second factor is applied.
+R6  the low-rank latent z = x_hat @ W^T is kept at full precision (the pages
+    give no rounding for it) before the second factor is applied.
 R7  weights use the [out][in] convention: y = x @ W^T.
 R8  temporal: frame 0 of a layer is coded with the null predictor at
     `anchor_bits`; at frame 1 the missing lag-2 frame is taken as zero; a
     partial last frame uses the first n spatial positions of earlier frames.
+    A sequence may also be continued from a supplied reconstructed history
+    (the two previous K frames, the previous V frame); no frame is then an
+    anchor.
 R9  the temporal K map takes [K_{f-1} | K_{f-2}] (2D inputs per head); the V map
     takes [K_f | V_{f-1}] (2D inputs per head).
 R10 clustered codec: a(t) = argmin_j (|c_j|^2 - 2 x_t.c_j), ties to the lowest
@@ -208,7 +211,7 @@ def codes_bytes(desc: Desc, kind: str = "none", code_dim: int = 0) -> int:
         return 2 * T * per_tok
     row_params = (D // desc.group) * pb
     if kind == "temporal":
-        n0 = min(desc.frame_tokens, T)
+        n0 = min(desc.frame_tokens, T) if desc.anchor_bits else 0
         rows_anchor = n0 * H
         rows_rest = (T - n0) * H
         one = rows_anchor * (D * desc.anchor_bits // 8) + rows_rest * (D * desc.bits // 8)
@@ -246,32 +249,32 @@ def _blockdiag(x, block) -> np.ndarray:
     return out.transpose(1, 0, 2)
 
 
-def _lowrank(flat_in, w, u, state: str, T: int, H: int, D: int) -> np.ndarray:
-    """Global low-rank term: round_state(flat_in @ w^T) @ u^T (reading R6)."""
+def _lowrank(flat_in, w, u, T: int, H: int, D: int) -> np.ndarray:
+    """Global low-rank term: (flat_in @ w^T) @ u^T (reading R6)."""
     if w is None or w.shape[0] == 0:
         return np.zeros((T, H, D))
-    z = round_to(flat_in @ w.T, state)
+    z = flat_in @ w.T
     return (z @ u.T).reshape(T, H, D)
 
 
-def xlayer_predict_k(K_src, k_block, k_w, k_u, state: str) -> np.ndarray:
-    """K~_l = blockdiag_h(K^_{l-1,h} B_h^T) + round(K^_{l-1} W^T) U^T.
+def xlayer_predict_k(K_src, k_block, k_w, k_u) -> np.ndarray:
+    """K~_l = blockdiag_h(K^_{l-1,h} B_h^T) + (K^_{l-1} W^T) U^T.
 
     K_src [T,H,D] reconstructed layer l-1; k_block [H,D,D]; k_w [r,C]; k_u [C,r].
     """
     T, H, D = K_src.shape
     pred = _blockdiag(K_src, k_block)
-    return pred + _lowrank(K_src.reshape(T, H * D), k_w, k_u, state, T, H, D)
+    return pred + _lowrank(K_src.reshape(T, H * D), k_w, k_u, T, H, D)
 
 
-def xlayer_predict_v(K_rec, V_src, v_block, v_w, v_u, state: str) -> np.ndarray:
+def xlayer_predict_v(K_rec, V_src, v_block, v_w, v_u) -> np.ndarray:
     """V~_l from the reconstructed pair [K^_l, V^_{l-1}]: per head the 2D-wide
     input [K^_{l,h} | V^_{l-1,h}] through v_block [H,D,2D]; globally the 2C-wide
     input [K^_l | V^_{l-1}] through v_w [r,2C] and v_u [C,r]."""
     T, H, D = K_rec.shape
     pred = _blockdiag(np.concatenate([K_rec, V_src], axis=-1), v_block)
     flat = np.concatenate([K_rec.reshape(T, H * D), V_src.reshape(T, H * D)], axis=-1)
-    return pred + _lowrank(flat, v_w, v_u, state, T, H, D)
+    return pred + _lowrank(flat, v_w, v_u, T, H, D)
 
 
 @dataclass
@@ -309,18 +312,18 @@ def encode_layer_xlayer(desc: Desc, w: dict, K, V, K_src, V_src):
     w holds k_block, k_w, k_u, v_block, v_w, v_u (float64 copies of the weights).
     Returns (coded K, coded V, K^_l, V^_l).
     """
-    pk = xlayer_predict_k(K_src, w["k_block"], w["k_w"], w["k_u"], desc.state)
+    pk = xlayer_predict_k(K_src, w["k_block"], w["k_w"], w["k_u"])
     qk, sk, zk, K_hat = code_residual(K, pk, desc.bits, desc.group, desc.param, desc.state)
-    pv = xlayer_predict_v(K_hat, V_src, w["v_block"], w["v_w"], w["v_u"], desc.state)
+    pv = xlayer_predict_v(K_hat, V_src, w["v_block"], w["v_w"], w["v_u"])
     qv, sv, zv, V_hat = code_residual(V, pv, desc.bits, desc.group, desc.param, desc.state)
     return Coded(qk, sk, zk), Coded(qv, sv, zv), K_hat, V_hat
 
 
 def decode_layer_xlayer(desc: Desc, w: dict, ck: Coded, cv: Coded, K_src, V_src):
     """Replays the encoder's prediction chain from the codes."""
-    pk = xlayer_predict_k(K_src, w["k_block"], w["k_w"], w["k_u"], desc.state)
+    pk = xlayer_predict_k(K_src, w["k_block"], w["k_w"], w["k_u"])
     K_hat = decode_residual(ck.q, ck.s, ck.z, pk, desc.group, desc.state)
-    pv = xlayer_predict_v(K_hat, V_src, w["v_block"], w["v_w"], w["v_u"], desc.state)
+    pv = xlayer_predict_v(K_hat, V_src, w["v_block"], w["v_w"], w["v_u"])
     V_hat = decode_residual(cv.q, cv.s, cv.z, pv, desc.group, desc.state)
     return K_hat, V_hat
 
@@ -337,65 +340,80 @@ def _frame_rows(desc: Desc):
     return [(f * F, min(T, (f + 1) * F)) for f in range(n_frames)]
 
 
-def encode_layer_temporal(desc: Desc, w: dict, K, V):
+def _history(hist, F, H, D, n_back):
+    """Reconstructed frames before the first one of this call, oldest first,
+    as a [n_back*F, H, D] block (zeros where absent)."""
+    if hist is None:
+        return np.zeros((n_back * F, H, D))
+    return np.asarray(hist, dtype=np.float64).reshape(n_back * F, H, D)
+
+
+def encode_layer_temporal(desc: Desc, w: dict, K, V, k_hist=None, v_hist=None):
     """Frame by frame in time order (readings R8, R9).
 
     w: ak [H,D,2D] over [K^_{f-1} | K^_{f-2}], av [H,D,2D] over [K^_f | V^_{f-1}].
-    Returns (coded K, coded V, K^, V^) over all T tokens; the codes of frame 0
-    are at desc.anchor_bits, the rest at desc.bits.
+    k_hist [2,F,H,D] (frames f0-2, f0-1) and v_hist [F,H,D] (frame f0-1), when
+    given, continue an earlier sequence: frame 0 of this call is then predicted
+    and coded at desc.bits.  Without them the codes of frame 0 are the anchor at
+    desc.anchor_bits.  Returns (coded K, coded V, K^, V^) over all T tokens.
     """
     T, H, D = K.shape
     F = desc.frame_tokens
-    K_hat = np.zeros((T, H, D))
-    V_hat = np.zeros((T, H, D))
+    cont = k_hist is not None
+    K_hat = np.concatenate([_history(k_hist, F, H, D, 2), np.zeros((T, H, D))])
+    V_hat = np.concatenate([_history(v_hist, F, H, D, 1), np.zeros((T, H, D))])
+    ko, vo = 2 * F, F  # offsets of this call's frame 0 in K_hat / V_hat
     qk = np.zeros((T, H, D), np.uint8)
     qv = np.zeros((T, H, D), np.uint8)
     ng = D // desc.group
     sk, zk, sv, zv = (np.zeros((T, H, ng)) for _ in range(4))
     for f, (a, b) in enumerate(_frame_rows(desc)):
         n = b - a
-        if f == 0:
-            bits = desc.anchor_bits
+        anchor = f == 0 and not cont
+        bits = desc.anchor_bits if anchor else desc.bits
+        if anchor:
             pk = np.zeros((n, H, D))
         else:
-            bits = desc.bits
-            k1 = K_hat[a - F : a - F + n]
-            k2 = K_hat[a - 2 * F : a - 2 * F + n] if f >= 2 else np.zeros((n, H, D))
+            k1 = K_hat[ko + a - F : ko + a - F + n]
+            k2 = K_hat[ko + a - 2 * F : ko + a - 2 * F + n]  # zeros before frame 0 of a sequence
             pk = _blockdiag(np.concatenate([k1, k2], axis=-1), w["ak"])
-        qk[a:b], sk[a:b], zk[a:b], K_hat[a:b] = code_residual(
+        qk[a:b], sk[a:b], zk[a:b], K_hat[ko + a:ko + b] = code_residual(
             K[a:b], pk, bits, desc.group, desc.param, desc.state)
-        if f == 0:
+        if anchor:
             pv = np.zeros((n, H, D))
         else:
-            v1 = V_hat[a - F : a - F + n]
-            pv = _blockdiag(np.concatenate([K_hat[a:b], v1], axis=-1), w["av"])
-        qv[a:b], sv[a:b], zv[a:b], V_hat[a:b] = code_residual(
+            v1 = V_hat[vo + a - F : vo + a - F + n]
+            pv = _blockdiag(np.concatenate([K_hat[ko + a:ko + b], v1], axis=-1), w["av"])
+        qv[a:b], sv[a:b], zv[a:b], V_hat[vo + a:vo + b] = code_residual(
             V[a:b], pv, bits, desc.group, desc.param, desc.state)
-    return Coded(qk, sk, zk), Coded(qv, sv, zv), K_hat, V_hat
+    return Coded(qk, sk, zk), Coded(qv, sv, zv), K_hat[ko:], V_hat[vo:]
 
 
-def decode_layer_temporal(desc: Desc, w: dict, ck: Coded, cv: Coded):
+def decode_layer_temporal(desc: Desc, w: dict, ck: Coded, cv: Coded, k_hist=None, v_hist=None):
+    """Replays the frame chain of encode_layer_temporal from the codes."""
     T, H, D = ck.q.shape
     F = desc.frame_tokens
-    K_hat = np.zeros((T, H, D))
-    V_hat = np.zeros((T, H, D))
+    cont = k_hist is not None
+    K_hat = np.concatenate([_history(k_hist, F, H, D, 2), np.zeros((T, H, D))])
+    V_hat = np.concatenate([_history(v_hist, F, H, D, 1), np.zeros((T, H, D))])
+    ko, vo = 2 * F, F
     for f, (a, b) in enumerate(_frame_rows(desc)):
         n = b - a
-        if f == 0:
+        anchor = f == 0 and not cont
+        if anchor:
             pk = np.zeros((n, H, D))
-            pv_needs = None
         else:
-            k1 = K_hat[a - F : a - F + n]
-            k2 = K_hat[a - 2 * F : a - 2 * F + n] if f >= 2 else np.zeros((n, H, D))
+            k1 = K_hat[ko + a - F : ko + a - F + n]
+            k2 = K_hat[ko + a - 2 * F : ko + a - 2 * F + n]
             pk = _blockdiag(np.concatenate([k1, k2], axis=-1), w["ak"])
-            pv_needs = V_hat[a - F : a - F + n]
-        K_hat[a:b] = decode_residual(ck.q[a:b], ck.s[a:b], ck.z[a:b], pk, desc.group, desc.state)
-        if pv_needs is None:
+        K_hat[ko + a:ko + b] = decode_residual(ck.q[a:b], ck.s[a:b], ck.z[a:b], pk, desc.group, desc.state)
+        if anchor:
             pv = np.zeros((n, H, D))
         else:
-            pv = _blockdiag(np.concatenate([K_hat[a:b], pv_needs], axis=-1), w["av"])
-        V_hat[a:b] = decode_residual(cv.q[a:b], cv.s[a:b], cv.z[a:b], pv, desc.group, desc.state)
-    return K_hat, V_hat
+            v1 = V_hat[vo + a - F : vo + a - F + n]
+            pv = _blockdiag(np.concatenate([K_hat[ko + a:ko + b], v1], axis=-1), w["av"])
+        V_hat[vo + a:vo + b] = decode_residual(cv.q[a:b], cv.s[a:b], cv.z[a:b], pv, desc.group, desc.state)
+    return K_hat[ko:], V_hat[vo:]
 
 
 # --------------------------------------------------------------------------

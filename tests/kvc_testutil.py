@@ -105,8 +105,8 @@ def exact_none(c: "O.Coded", group: int):
 
 
 def exact_xlayer(d: "O.Desc", w: dict, ck, cv, K_src, V_src, K_hat):
-    pk = O.xlayer_predict_k(K_src, w["k_block"], w["k_w"], w["k_u"], d.state)
-    pv = O.xlayer_predict_v(K_hat, V_src, w["v_block"], w["v_w"], w["v_u"], d.state)
+    pk = O.xlayer_predict_k(K_src, w["k_block"], w["k_w"], w["k_u"])
+    pv = O.xlayer_predict_v(K_hat, V_src, w["v_block"], w["v_w"], w["v_u"])
     return pk + O.dequantize_groups(ck.q, ck.s, ck.z, d.group), pv + O.dequantize_groups(cv.q, cv.s, cv.z, d.group)
 
 

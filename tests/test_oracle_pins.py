@@ -159,31 +159,32 @@ def test_dplr_prediction_equals_dense_map():
     kw, ku = rng.standard_normal((r, H * D)), rng.standard_normal((H * D, r))
     vw, vu = rng.standard_normal((r, 2 * H * D)), rng.standard_normal((H * D, r))
     Mk = _dense_dplr(kb, kw, ku, H, D, D, lambda h, i: h * D + i)
-    got = O.xlayer_predict_k(Ks, kb, kw, ku, "f64").reshape(T, -1)
+    got = O.xlayer_predict_k(Ks, kb, kw, ku).reshape(T, -1)
     np.testing.assert_allclose(got, Ks.reshape(T, -1) @ Mk, rtol=1e-12, atol=1e-12)
     # V's per-head input is [K_h | V_h]; its global input is [K (all heads) | V (all heads)]
     Mv = _dense_dplr(vb, vw, vu, H, D, 2 * D,
                      lambda h, i: h * D + i if i < D else H * D + h * D + (i - D))
     flat = np.concatenate([Ks.reshape(T, -1), Vs.reshape(T, -1)], axis=1)
-    got = O.xlayer_predict_v(Ks, Vs, vb, vw, vu, "f64").reshape(T, -1)
+    got = O.xlayer_predict_v(Ks, Vs, vb, vw, vu).reshape(T, -1)
     np.testing.assert_allclose(got, flat @ Mv, rtol=1e-12, atol=1e-12)
     # rank 0 is the pure block-diagonal map
-    got0 = O.xlayer_predict_k(Ks, kb, kw[:0], ku[:, :0], "f64").reshape(T, -1)
+    got0 = O.xlayer_predict_k(Ks, kb, kw[:0], ku[:, :0]).reshape(T, -1)
     np.testing.assert_allclose(got0, Ks.reshape(T, -1) @ _dense_dplr(kb, kw[:0], ku[:, :0], H, D, D,
                                                                       lambda h, i: h * D + i), rtol=1e-12)
 
 
-def test_low_rank_latent_is_rounded_to_state_dtype():
+def test_low_rank_latent_is_not_rounded():
+    """The latent passes to the second factor at full precision: with U = I
+    the first r outputs of a zero-block map are x W^T exactly."""
     H, D, r, T = 2, 4, 3, 5
     rng = np.random.default_rng(2)
     Ks = rng.standard_normal((T, H, D))
     kb = np.zeros((H, D, D))
     kw, ku = rng.standard_normal((r, H * D)), np.eye(H * D, r)
-    got = O.xlayer_predict_k(Ks, kb, kw, ku, "bf16").reshape(T, -1)[:, :r]
-    lat = Ks.reshape(T, -1) @ kw.T
-    ref = torch.from_numpy(lat.astype(np.float32)).to(torch.bfloat16).double().numpy()
-    # the f32 pre-rounding of the reference can only matter at bf16 ties, which random data avoids
-    np.testing.assert_array_equal(got, ref)
+    got = O.xlayer_predict_k(Ks, kb, kw, ku).reshape(T, -1)[:, :r]
+    ref = np.einsum("tc,jc->tj", Ks.reshape(T, -1), kw)
+    np.testing.assert_allclose(got, ref, rtol=1e-14, atol=1e-14)
+    assert not np.array_equal(got, O.round_to(got, "bf16"))
 
 
 def _grid_values(rng, shape):
@@ -237,9 +238,9 @@ def _chain_workload(L=6, T=300, H=2, D=64, r=4, seed=5):
                  v_w=rng.standard_normal((r, 2 * C)) / np.sqrt(2 * C), v_u=0.1 * rng.standard_normal((C, r)))
         w = {k: O.round_to(v, "bf16") for k, v in w.items()}
         W.append(w)
-        K.append(O.round_to(O.xlayer_predict_k(K[-1], w["k_block"], w["k_w"], w["k_u"], "f64")
+        K.append(O.round_to(O.xlayer_predict_k(K[-1], w["k_block"], w["k_w"], w["k_u"])
                             + 0.3 * rng.standard_normal((T, H, D)), "bf16"))
-        V.append(O.round_to(O.xlayer_predict_v(K[-1], V[-1], w["v_block"], w["v_w"], w["v_u"], "f64")
+        V.append(O.round_to(O.xlayer_predict_v(K[-1], V[-1], w["v_block"], w["v_w"], w["v_u"])
                             + 0.3 * rng.standard_normal((T, H, D)), "bf16"))
     K[0], V[0] = O.round_to(K[0], "bf16"), O.round_to(V[0], "bf16")
     return K, V, W
@@ -266,9 +267,9 @@ def test_closed_loop_error_does_not_accumulate_and_decode_replays_encode():
             s = np.repeat(c.s, 32, axis=-1)
             assert np.all(np.abs(x - xh) <= 0.5 * s + 2.0 ** -7 * np.abs(x) + 1e-3 * s + 1e-30)
         # open loop: predict from clean K_{l-1}; the decoder only has its own state
-        pk_clean = O.xlayer_predict_k(K[l - 1], W[l]["k_block"], W[l]["k_w"], W[l]["k_u"], "bf16")
+        pk_clean = O.xlayer_predict_k(K[l - 1], W[l]["k_block"], W[l]["k_w"], W[l]["k_u"])
         qo, so, zo = O.quantize_groups(K[l] - pk_clean, 2, 32, "f16")
-        pk_dec = O.xlayer_predict_k(open_K, W[l]["k_block"], W[l]["k_w"], W[l]["k_u"], "bf16")
+        pk_dec = O.xlayer_predict_k(open_K, W[l]["k_block"], W[l]["k_w"], W[l]["k_u"])
         open_K = O.round_to(pk_dec + O.dequantize_groups(qo, so, zo, 32), "bf16")
         open_err.append(np.abs(open_K - K[l]).max() / np.repeat(so, 32, -1).max())
     assert open_err[-1] > 0.75  # drift beyond the half-step bound the closed loop keeps
@@ -308,6 +309,31 @@ def test_temporal_exact_predictor_and_ragged_frame():
     Kd, Vd = O.decode_layer_temporal(d, dict(ak=ak, av=av), ck, cv)
     np.testing.assert_array_equal(Kd, K)
     np.testing.assert_array_equal(Vd, V)
+
+
+def test_temporal_continuation_equals_one_sequence():
+    """Coding frames [0, 3) and then [3, 5) from the reconstructed history
+    (K of frames 1 and 2, V of frame 2) gives the codes of one 5-frame call."""
+    H, D, F = 2, 64, 12
+    rng = np.random.default_rng(14)
+    T = 5 * F
+    K = O.round_to(rng.standard_normal((T, H, D)), "bf16")
+    V = O.round_to(rng.standard_normal((T, H, D)), "bf16")
+    w = dict(ak=rng.standard_normal((H, D, 2 * D)) * 0.05, av=rng.standard_normal((H, D, 2 * D)) * 0.05)
+    d = O.Desc(T, H, D, bits=2, group=32, frame_tokens=F, anchor_bits=4)
+    ck, cv, Kh, Vh = O.encode_layer_temporal(d, w, K, V)
+    d1 = O.Desc(3 * F, H, D, bits=2, group=32, frame_tokens=F, anchor_bits=4)
+    ck1, cv1, Kh1, Vh1 = O.encode_layer_temporal(d1, w, K[:3 * F], V[:3 * F])
+    d2 = O.Desc(2 * F, H, D, bits=2, group=32, frame_tokens=F, anchor_bits=0)
+    kh = Kh1[F:3 * F].reshape(2, F, H, D)
+    ck2, cv2, Kh2, Vh2 = O.encode_layer_temporal(d2, w, K[3 * F:], V[3 * F:], kh, Vh1[2 * F:])
+    np.testing.assert_array_equal(np.concatenate([ck1.q, ck2.q]), ck.q)
+    np.testing.assert_array_equal(np.concatenate([cv1.q, cv2.q]), cv.q)
+    np.testing.assert_array_equal(np.concatenate([Vh1, Vh2]), Vh)
+    Kd, Vd = O.decode_layer_temporal(d2, w, ck2, cv2, kh, Vh1[2 * F:])
+    np.testing.assert_array_equal(Kd, Kh2)
+    # a continued call stores every frame at `bits`
+    assert O.codes_bytes(d2, "temporal") == 2 * 2 * F * H * (D * 2 // 8 + 2 * 2 * 2)
 
 
 def test_temporal_frame_zero_is_plain_group_rtn_at_anchor_bits():
