@@ -56,7 +56,8 @@ kvc_status check_desc(const kvc_layer_desc* d, const kvc_predictor* p) {
     case KVC_PRED_TEMPORAL:
       if (!row_layout_ok(d->head_dim, d->group)) return KVC_ERR_UNSUPPORTED;
       if (d->frame_tokens < 1) return KVC_ERR_INVALID_ARGUMENT;
-      if (d->anchor_bits != 2 && d->anchor_bits != 4 && d->anchor_bits != 8) return KVC_ERR_UNSUPPORTED;
+      if (d->anchor_bits != 0 && d->anchor_bits != 2 && d->anchor_bits != 4 && d->anchor_bits != 8)
+        return KVC_ERR_UNSUPPORTED;
       return KVC_OK;
     case KVC_PRED_CLUSTER:
       if (p->code_dim != 128 || !row_layout_ok(128, d->group)) return KVC_ERR_UNSUPPORTED;
@@ -81,7 +82,7 @@ Sizes sizes_of(const kvc_layer_desc* d, const kvc_predictor* p) {
     s.params = T * (m / d->group) * pair;
     s.assign = T;
   } else if (p->kind == KVC_PRED_TEMPORAL) {
-    const size_t F0 = (size_t)d->frame_tokens < T ? (size_t)d->frame_tokens : T;
+    const size_t F0 = d->anchor_bits == 0 ? 0 : ((size_t)d->frame_tokens < T ? (size_t)d->frame_tokens : T);
     s.codes = F0 * H * D * d->anchor_bits / 8 + (T - F0) * H * D * d->bits / 8;
     s.params = T * H * (D / d->group) * pair;
   } else {
@@ -167,9 +168,10 @@ cudaError_t codec_xlayer(const kvc_layer_desc* d, const kvc_predictor* p, bool e
 
 template <typename TS, typename TP>
 cudaError_t codec_temporal(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
-                           const kvc_codes* c, void* Kr, void* Vr, cudaStream_t st) {
+                           const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, cudaStream_t st) {
   TemporalArgs<TS, TP> a{d->n_tokens, d->frame_tokens, d->n_heads, d->bits, d->anchor_bits, d->group,
-                         (const TS*)K, (const TS*)V, (const TS*)p->k_block, (const TS*)p->v_block,
+                         (const TS*)K, (const TS*)V, (const TS*)Ks, (const TS*)Vs,
+                         (const TS*)p->k_block, (const TS*)p->v_block,
                          (uint8_t*)c->k_codes, (Pair<TP>*)c->k_params, (uint8_t*)c->v_codes,
                          (Pair<TP>*)c->v_params, (TS*)Kr, (TS*)Vr};
   return launch_temporal(a, d->head_dim, enc, st);
@@ -244,9 +246,11 @@ kvc_status codec_common(const kvc_layer_desc* d, const kvc_predictor* p, bool en
                         size_t ws_bytes, void* stream) {
   kvc_status s = check_desc(d, p);
   if (s != KVC_OK) return s;
+  if (d->n_tokens == 0) return KVC_OK;  // nothing to code
   if ((s = check_weights(p)) != KVC_OK) return s;
   if (!codes_ok(p, c)) return KVC_ERR_INVALID_ARGUMENT;
   if (enc && (!K || !V)) return KVC_ERR_INVALID_ARGUMENT;
+  if (p->kind == KVC_PRED_TEMPORAL && d->anchor_bits == 0 && (!Ks || !Vs)) return KVC_ERR_INVALID_ARGUMENT;
   if (!enc && (!Kr || !Vr)) return KVC_ERR_INVALID_ARGUMENT;
   if (p->kind == KVC_PRED_XLAYER_DPLR && (!Ks || !Vs || !Kr)) return KVC_ERR_INVALID_ARGUMENT;
   const void* ptrs[] = {K, V, Ks, Vs, Kr, Vr, ws};
@@ -257,7 +261,6 @@ kvc_status codec_common(const kvc_layer_desc* d, const kvc_predictor* p, bool en
   const size_t need = kvc_workspace_bytes(op, d, p, 0);
   if (ws_bytes < need || (need && !ws)) return KVC_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = (cudaStream_t)stream;
-  if (d->n_tokens == 0) return KVC_OK;
   // tensor-core path for the bf16, D = 128 cross-layer / anchor codec
   if (tc_codec_supported(d, p)) {
     cudaError_t e = tc_codec_layer(d, p, enc, K, V, Ks, Vs, c, Kr, Vr, ws, ws_bytes, st);
@@ -269,7 +272,7 @@ kvc_status codec_common(const kvc_layer_desc* d, const kvc_predictor* p, bool en
     using TP = std::remove_pointer_t<decltype(tp)>;
     switch (p->kind) {
       case KVC_PRED_TEMPORAL:
-        return codec_temporal<TS, TP>(d, p, enc, K, V, c, Kr, Vr, st);
+        return codec_temporal<TS, TP>(d, p, enc, K, V, Ks, Vs, c, Kr, Vr, st);
       case KVC_PRED_CLUSTER:
         return codec_cluster<TS, TP>(d, p, enc, K, V, c, Kr, Vr, cv, st);
       default:

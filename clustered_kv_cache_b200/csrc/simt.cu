@@ -54,7 +54,7 @@ __device__ __forceinline__ void zero_acc(float (&acc)[4][NJ]) {
     for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
 }
 
-// ============================================================== latent z = round(x W^T)
+// ============================================================== latent z = x W^T (fp32, not rounded)
 
 template <typename TS, int NJ>
 __global__ void __launch_bounds__(kThreads) latent_kernel(LatentArgs<TS> a) {
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) latent_kernel(LatentArgs<TS> a) {
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       const int jj = tx + 32 * j;
-      if (t < a.T && jj < a.r) a.Z[t * a.r + jj] = round_as<TS>(acc[i][j]);
+      if (t < a.T && jj < a.r) a.Z[t * a.r + jj] = acc[i][j];
     }
   }
 }
@@ -179,21 +179,36 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(TemporalArgs<TS, TP>
   const int H = a.H;
   const int64_t F = a.F;
   const int64_t n_frames = (a.T + F - 1) / F;
-  const int64_t F0 = F < a.T ? F : a.T;
+  const bool cont = a.anchor_bits == 0;  // continues a sequence from K_src / V_src
+  const int64_t F0 = cont ? 0 : (F < a.T ? F : a.T);
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5, lane = tx, warp = ty;
   const int row_groups = D / a.group;
   for (int e = threadIdx.x; e < 5 * 32 * D; e += kThreads) buf[0][e] = 0.f;
   __syncthreads();
+  if (cont) {
+    // history: K_src = [K^ of frame f0-2 ; K^ of frame f0-1], V_src = V^ of frame f0-1
+    for (int e = threadIdx.x; e < 32 * D; e += kThreads) {
+      const int i = e / D, d = e % D;
+      const int64_t s = s0 + i;
+      if (s >= F) continue;
+      Kp2[e] = to_f(a.ksrc[(s * H + h) * D + d]);
+      Kp1[e] = to_f(a.ksrc[((F + s) * H + h) * D + d]);
+      Vp1[e] = to_f(a.vsrc[(s * H + h) * D + d]);
+    }
+    __syncthreads();
+  }
 
   for (int64_t f = 0; f < n_frames; ++f) {
     const int64_t n_f = (a.T - f * F) < F ? (a.T - f * F) : F;
-    const int bits = f == 0 ? a.anchor_bits : a.bits;
+    const bool anchor = f == 0 && !cont;
+    const int bits = anchor ? a.anchor_bits : a.bits;
     const int row_bytes = D * bits / 8;
+    const int anchor_row_bytes = D * a.anchor_bits / 8;
     RowCodec<E> rc{bits, a.group};
     for (int pass = 0; pass < 2; ++pass) {  // 0: K, 1: V
       float acc[4][NJ];
       zero_acc(acc);
-      if (f > 0) {
+      if (!anchor) {
         const float* in0 = pass == 0 ? Kp1 : Kc;
         const float* in1 = pass == 0 ? Kp2 : Vp1;
         const TS* W = (pass == 0 ? a.ak : a.av) + (int64_t)h * D * 2 * D;
@@ -216,8 +231,8 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(TemporalArgs<TS, TP>
         if (s >= n_f) break;
         const int64_t t = f * F + s;
         const int64_t row = t * H + h;
-        const int64_t cofs = f == 0 ? row * row_bytes
-                                    : F0 * H * (D * a.anchor_bits / 8) + (row - F0 * H) * row_bytes;
+        const int64_t cofs = row < F0 * H ? row * anchor_row_bytes
+                                          : F0 * H * anchor_row_bytes + (row - F0 * H) * row_bytes;
         float p[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) p[e] = sP[i * D + lane * E + e];

@@ -5,7 +5,7 @@
 
 namespace kvc {
 
-// Z[t][j] = round_TS(sum_c X[t][c] W[j][c]),  X[t] = [in0[t] | in1[t]] (in1 may be NULL)
+// Z[t][j] = sum_c X[t][c] W[j][c] (fp32),  X[t] = [in0[t] | in1[t]] (in1 may be NULL)
 template <typename TS>
 struct LatentArgs {
   int64_t T;
@@ -24,7 +24,7 @@ struct HeadsArgs {
   const TS* in0;    // [T][H][D] (NULL with block == NULL)
   const TS* in1;    // [T][H][D] or NULL
   const TS* block;  // [H][D][Din] or NULL (no block term)
-  const float* Z;   // [T][r] latent (r > 0)
+  const float* Z;   // [T][r] latent, fp32 (r > 0)
   const TS* U;      // [C][r]
   const TS* x;      // clean rows (encode)
   uint8_t* codes;   // [T][H][D*bits/8]
@@ -35,9 +35,11 @@ struct HeadsArgs {
 template <typename TS, typename TP>
 struct TemporalArgs {
   int64_t T, F;
-  int H, bits, anchor_bits, group;
+  int H, bits, anchor_bits, group;  // anchor_bits == 0: continue from ksrc / vsrc
   const TS* K;
   const TS* V;
+  const TS* ksrc;  // [2][F][H][D] reconstructed K of the two frames before this call
+  const TS* vsrc;  // [F][H][D] reconstructed V of the frame before this call
   const TS* ak;  // [H][D][2D]
   const TS* av;
   uint8_t* kcodes;

@@ -106,7 +106,9 @@ def tiny_xlayer(seed: int = SEED_BASE + 0, device="cpu", T: int = 512, H: int = 
     kv = torch.cat([K1, V0], dim=-1)
     kvf = torch.cat([K1.reshape(T, C), V0.reshape(T, C)], dim=-1)
     V1 = dplr(kv, kvf, w["v_block"], w["v_w"], w["v_u"]) + 0.1 * _randn(g, T, H, D, device=device)
-    return XLayerWorkload([K0, K1], [V0, V1], [None, w], H, D, rank, torch.float32)
+    K = [K0.contiguous(), K1.contiguous()]
+    V = [V0.contiguous(), V1.contiguous()]
+    return XLayerWorkload(K, V, [None, {k: t.contiguous() for k, t in w.items()}], H, D, rank, torch.float32)
 
 
 @dataclass
@@ -184,7 +186,9 @@ def fit_block_dplr(X_head: torch.Tensor, X_flat: torch.Tensor, Y: torch.Tensor, 
         blocks[h] = Bh.T
         R[:, h] = Y[:, h].double() - X_head[:, h].double() @ Bh
     if rank == 0:
-        return blocks, None, None
+        Cin = X_flat.shape[1]
+        zero = X_head.new_zeros
+        return blocks, zero((0, Cin), dtype=torch.float64), zero((H * D, 0), dtype=torch.float64)
     Rf = R.reshape(T, H * D)
     M = _ridge_lstsq(X_flat, Rf)  # [Cin, C]
     F = X_flat.double() @ M

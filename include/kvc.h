@@ -85,7 +85,9 @@ typedef enum {
  *         multiple of D/32.
  *  param_dtype: KVC_F16 or KVC_F32; the (scale, zero) storage type.
  *  frame_tokens: tokens per frame (temporal only; token t = f*frame_tokens+s).
- *  anchor_bits: bits of frame 0 (temporal only). */
+ *  anchor_bits: temporal only: bits of frame 0, coded with prediction 0
+ *         (2, 4 or 8); or 0 when the call continues a sequence, whose
+ *         reconstructed history then arrives in K_src / V_src. */
 typedef struct {
   int64_t n_tokens;
   int32_t n_heads;
@@ -122,8 +124,9 @@ typedef struct {
  *  NONE / XLAYER: k_codes [T][H][D*bits/8] bytes, k_params [T][H][D/group][2]
  *    of (scale, zero) in param_dtype; element j of a row sits at bits
  *    [j*bits, (j+1)*bits) of the row, least significant bit first.
- *  TEMPORAL: as above, except that the rows of frame 0 come first at
- *    anchor_bits, followed by the rows of all later frames at bits.
+ *  TEMPORAL: as above, except that (unless anchor_bits is 0) the rows of
+ *    frame 0 come first at anchor_bits, followed by the rows of all later
+ *    frames at bits.
  *  CLUSTER: k_codes [T][code_dim*bits/8], k_params [T][code_dim/group][2],
  *    k_assign [T] uint8 centre index.
  *  The v_* members hold V the same way.  Sizes: kvc_codes_sizes(). */
@@ -161,15 +164,18 @@ KVC_API size_t kvc_workspace_bytes(int op, const kvc_layer_desc* desc, const kvc
 /* Encode one layer: prediction, residual, group quantization, packing, and the
  * closed-loop reconstruction.
  *  K, V:         [T][H][D] clean values of this layer (read).
- *  K_src, V_src: XLAYER: reconstructions of layer l-1 [T][H][D] (read);
- *                ignored (may be NULL) for the other kinds.
+ *  K_src, V_src: XLAYER: reconstructions of layer l-1 [T][H][D] (read).
+ *                TEMPORAL with anchor_bits == 0: the reconstructed K of the
+ *                two frames before this call, [2][frame_tokens][H][D] (older
+ *                first), and the reconstructed V of the frame before,
+ *                [frame_tokens][H][D].  Otherwise ignored (may be NULL).
  *  out:          codes / params / assignments (written).
  *  K_rec, V_rec: reconstructions of this layer (written); may be NULL unless
  *                the caller chains them into the next layer, except that
  *                XLAYER needs K_rec (V's prediction reads the reconstructed K).
  *  ws, ws_bytes: workspace of kvc_workspace_bytes(KVC_OP_ENCODE, ...).
- * Temporal layers need T >= 1 and frame_tokens >= 1; the whole layer's frame
- * chain runs inside this call. */
+ * T = 0 is a no-op.  For temporal layers the whole frame chain of the call
+ * runs inside it, in time order. */
 KVC_API kvc_status kvc_encode_layer(const kvc_layer_desc* desc, const kvc_predictor* pred, const void* K,
                             const void* V, const void* K_src, const void* V_src, const kvc_codes* out,
                             void* K_rec, void* V_rec, void* ws, size_t ws_bytes, void* stream);

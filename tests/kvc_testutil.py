@@ -76,6 +76,25 @@ def assert_codes_close(q_gpu, q_ref, what="codes", min_agree=CODE_AGREE):
     return agree
 
 
+def param_ulp(v, param: str) -> np.ndarray:
+    """Spacing of the parameter dtype at v."""
+    return np.spacing(np.abs(v).astype(np.float16 if param == "f16" else np.float32)).astype(np.float64)
+
+
+def assert_params_close(s_gpu, z_gpu, s_ref, z_ref, param: str, what="params"):
+    """Stored (scale, zero) pairs: equal, or one rounding step of the parameter
+    dtype apart (the min / max they round came from fp32 vs fp64 residuals).
+    Returns the mask of groups whose pair differs."""
+    ds = np.abs(s_gpu - s_ref)
+    dz = np.abs(z_gpu - z_ref)
+    assert np.all(ds <= param_ulp(s_ref, param) * 1.0001 + 1e-30), f"{what}: a scale differs by more than 1 ulp"
+    assert np.all(dz <= param_ulp(z_ref, param) * 1.0001 + 1e-30), f"{what}: a zero differs by more than 1 ulp"
+    diff = (ds > 0) | (dz > 0)
+    if param == "f16":
+        assert diff.mean() <= 1e-3, f"{what}: {diff.mean():.2e} of the groups differ"
+    return diff
+
+
 def assert_recon_close(rec_gpu, rec_ref, exact_ref, x, code_flip, state: str, what="recon"):
     """rec_gpu, rec_ref: values in the state dtype; exact_ref: the oracle's
     value before rounding to the state dtype; code_flip: elements whose code
