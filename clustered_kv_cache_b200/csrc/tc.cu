@@ -1,4 +1,30 @@
 // Tensor-core kernels (tcgen05 + TMEM + TMA) of the bf16 / head_dim 128 hot path.
+//
+// Cross-layer block-DPLR codec, one CTA per 128-token tile, all heads fused
+// ("CORAL-KV: Compact Cross-Layer Prediction and Residual Coding for
+// Autoregressive Video KV Caches", Fig. 3: K_l from the reconstructed K_{l-1};
+// V_l from the reconstructed [K_l, V_{l-1}]; block-diagonal per-head maps plus
+// a global rank-r term).  Per tile:
+//
+//   Z_K  = K^_{l-1} W_K^T                         (TMEM, 24 chunks of 64 channels)
+//   for each head h (K):  acc = K^_{l-1,h} B_h^T + [Z_K hi | lo] U_h^T
+//        epilogue: residual, group min/max, fp16 (scale, zero), codes, packing,
+//        reconstruction K^_{l,h} -> shared memory -> TMA store, and
+//        Z_V += K^_{l,h} W_V[:, h]^T (the V latent grows head by head)
+//   Z_V += V^_{l-1} W_V[:, C:]^T
+//   for each head h (V):  acc = [K^_{l,h} | V^_{l-1,h}] BV_h^T + [Z_V hi | lo] UV_h^T
+//        epilogue as above, writing V^_{l,h}
+//
+// The latent is carried to the second factor as a pair of bf16 values whose
+// sum is within 2^-16 of the fp32 accumulator, so no rounding decision is taken
+// on it.  Warp roles: warp 0 issues TMA loads, warp 1 allocates TMEM and one
+// thread issues every tcgen05.mma, warps 2..9 run the epilogue (two warps per
+// TMEM lane quarter, 64 columns each).  Every wait is bounded: a wait that runs
+// out records an error word, raises an abort flag seen by all roles, and the
+// CTA drains what it issued and returns.
+#include <cuda.h>
+#include <string.h>
+
 #include "tc.h"
 
 namespace kvc {
@@ -13,12 +39,697 @@ cudaError_t tc_read_and_clear_error(unsigned int* value) {
   return *value ? cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) : cudaSuccess;
 }
 
-bool tc_codec_supported(const kvc_layer_desc*, const kvc_predictor*) { return false; }
-size_t tc_workspace(int, const kvc_layer_desc*, const kvc_predictor*, int64_t) { return 0; }
-cudaError_t tc_codec_layer(const kvc_layer_desc*, const kvc_predictor*, bool, const void*, const void*, const void*,
-                           const void*, const kvc_codes*, void*, void*, void*, size_t, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace tc {
+
+constexpr int kThreads = 320;  // 10 warps
+constexpr int kEpiThreads = 256;
+constexpr long long kWaitBudget = 1ll << 32;  // cycles (about 2 s) before a wait gives up
+
+// ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return r != 0;
+}
+
+// Waits for the phase of parity `parity` of barrier b; false if the CTA aborted
+// or the budget ran out (which records `where` and raises the abort flag).
+__device__ __forceinline__ bool wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, unsigned where) {
+  if (mbar_test(b, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_test(b, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitBudget) {
+      *abort_flag = 1;
+      atomicCAS(&g_device_error, 0u, where);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* m, int x, int y, uint64_t* bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store(const CUtensorMap* m, int x, int y, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row core groups 1024 bytes apart (the layout TMA writes with
+// CU_TENSOR_MAP_SWIZZLE_128B and a 64-element inner box).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor: kind::f16, bf16 A and B (K-major), fp32 D, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Byte offset of the 16-byte chunk `c` (0..7) of row `row` inside a [rows][64]
+// bf16 sub-tile written with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw128_off(int row, int c) { return row * 128 + ((c ^ (row & 7)) << 4); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+template <int N>
+__device__ __forceinline__ void unpack_bf16x8(uint4 u, float (&v)[N], int base) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(p[i]);
+    v[base + 2 * i] = f.x;
+    v[base + 2 * i + 1] = f.y;
+  }
+}
+
+// ---------------------------------------------------------------- kernel arguments
+
+struct Maps {
+  CUtensorMap ks, vs;  // reconstructions of layer l-1, [T][C]
+  CUtensorMap ko, vo;  // reconstructions of layer l (written; K also read back), [T][C]
+  CUtensorMap wk, wv;  // [r][C], [r][2C]
+  CUtensorMap bk, bv;  // [H*128][128], [H*128][256]
+  CUtensorMap uk, uv;  // [C][r]
+};
+
+struct Args {
+  int64_t T;
+  int H, bits;
+  const __nv_bfloat16* xk;  // clean K (encode)
+  const __nv_bfloat16* xv;  // clean V (encode)
+  uint8_t* kcodes;
+  __half2* kparams;
+  uint8_t* vcodes;
+  __half2* vparams;
+  int store_v;  // V^_l is written (always for decode)
+};
+
+template <int RC>
+struct Layout {
+  static constexpr int S = RC == 2 ? 3 : 4;  // pipeline stages
+  static constexpr int kStage = 32768;        // A 16 KB + B 16 KB
+  static constexpr int kRecon = 32768;        // [128][128] bf16 as two 64-column sub-tiles
+  static constexpr int kStageOff = 0;
+  static constexpr int kReconOff = S * kStage;
+  static constexpr int kZOff = kReconOff + 2 * kRecon;  // latent hi / lo sub-tiles
+  static constexpr int kBarOff = kZOff + RC * 2 * 16384;
+  static constexpr int kBytes = kBarOff + 1024;
+};
+
+// ---------------------------------------------------------------- the kernel
+
+template <bool ENC, int G, int RC>
+__global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_constant__ Maps maps, const Args a) {
+  using L = Layout<RC>;
+  constexpr int S = L::S;
+  constexpr int R = RC * 64;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* full = bars;                 // [S]
+  uint64_t* empty = bars + S;            // [S]
+  uint64_t* acc_full = bars + 2 * S;     // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint64_t* rec_full = acc_empty + 2;    // [2]
+  uint64_t* rec_free = rec_full + 2;     // [2]
+  uint64_t* zk_full = rec_free + 2;
+  uint64_t* zv_full = zk_full + 1;
+  uint64_t* z_ready = zv_full + 1;
+  uint64_t* khat_stored = z_ready + 1;
+  uint64_t* mma_done = khat_stored + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = a.H;
+  const int C = H * 128;
+  const int NCH = C / 64;
+  const int t0 = blockIdx.x * 128;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kEpiThreads);
+      mbar_init(&rec_full[i], 1);
+      mbar_init(&rec_free[i], 1);
+    }
+    mbar_init(zk_full, 1);
+    mbar_init(zv_full, 1);
+    mbar_init(z_ready, kEpiThreads);
+    mbar_init(khat_stored, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto stageA = [&](int s) { return smem + L::kStageOff + s * L::kStage; };
+  auto stageB = [&](int s) { return smem + L::kStageOff + s * L::kStage + 16384; };
+  auto recon = [&](int b) { return smem + L::kReconOff + b * L::kRecon; };
+  auto zhi = [&](int j) { return smem + L::kZOff + j * 16384; };
+  auto zlo = [&](int j) { return smem + L::kZOff + (RC + j) * 16384; };
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+      int s = 0;
+      uint32_t ph = 0;
+      int issued[S];          // a load was issued into stage i ...
+      uint32_t issued_ph[S];  // ... in this phase of full[i]
+      for (int i = 0; i < S; ++i) issued[i] = 0, issued_ph[i] = 0;
+      bool ok = true;
+      auto load = [&](const CUtensorMap* ma, int ax, uint64_t pa, const CUtensorMap* mb, int bx, int by,
+                      uint32_t bbytes) {
+        if (!ok) return;
+        if (!wait(&empty[s], ph ^ 1, abort_flag, 0x100u + s)) {
+          ok = false;
+          return;
+        }
+        mbar_arrive_expect_tx(&full[s], (ma ? 16384u : 0u) + bbytes);
+        if (ma) tma_load(stageA(s), ma, ax, t0, &full[s], pa);
+        tma_load(stageB(s), mb, bx, by, &full[s], pol_keep);
+        issued[s] = 1;
+        issued_ph[s] = ph;
+        if (++s == S) {
+          s = 0;
+          ph ^= 1;
+        }
+      };
+      const uint32_t wbytes = R * 128;
+      if (RC) {
+        for (int c = 0; c < NCH; ++c) load(&maps.ks, c * 64, pol_keep, &maps.wk, c * 64, 0, wbytes);
+      }
+      for (int h = 0; h < H && ok; ++h) {
+        for (int j = 0; j < 2; ++j) load(&maps.ks, h * 128 + j * 64, pol_stream, &maps.bk, j * 64, h * 128, 16384);
+        for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, &maps.uk, j * 64, h * 128, 16384);
+        if (RC && h >= 1)
+          for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, &maps.wv, (h - 1) * 128 + j * 64, 0, wbytes);
+      }
+      if (RC) {
+        for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, &maps.wv, (H - 1) * 128 + j * 64, 0, wbytes);
+        for (int c = 0; c < NCH; ++c) load(&maps.vs, c * 64, pol_keep, &maps.wv, C + c * 64, 0, wbytes);
+      }
+      if (ok && !wait(khat_stored, 0, abort_flag, 0x200u)) ok = false;
+      if (ok) fence_async_global();
+      for (int h = 0; h < H && ok; ++h) {
+        for (int j = 0; j < 2; ++j) load(&maps.ko, h * 128 + j * 64, pol_stream, &maps.bv, j * 64, h * 128, 16384);
+        for (int j = 0; j < 2; ++j)
+          load(&maps.vs, h * 128 + j * 64, pol_stream, &maps.bv, 128 + j * 64, h * 128, 16384);
+        for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, &maps.uv, j * 64, h * 128, 16384);
+      }
+      if (!ok) {
+        // drain: the loads already issued must land before the CTA exits
+        for (int i = 0; i < S; ++i) {
+          if (!issued[i]) continue;
+          const long long w0 = clock64();
+          while (!mbar_test(&full[i], issued_ph[i]) && clock64() - w0 < kWaitBudget) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t acc_col[2] = {tmem, tmem + 128};
+      const uint32_t zk_col = tmem + 256, zv_col = tmem + 256 + R;
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int use[2] = {0, 0};
+      // one 64-wide K chunk: A from the stage (resA == 0) or resident smem
+      auto chunk = [&](uint32_t d, int N, bool first, const uint8_t* resA, const uint8_t* resA2) {
+        if (!ok) return;
+        if (!wait(&full[s], ph, abort_flag, 0x300u + s)) {
+          ok = false;
+          return;
+        }
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16(128, N);
+        const uint64_t bd = desc_sw128(smem_u32(stageB(s)));
+        const uint64_t ad = desc_sw128(smem_u32(resA ? resA : stageA(s)));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) umma(d, ad + 2 * k, bd + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
+        if (resA2) {
+          const uint64_t ad2 = desc_sw128(smem_u32(resA2));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) umma(d, ad2 + 2 * k, bd + 2 * k, idesc, 1u);
+        }
+        umma_commit(&empty[s]);
+        if (++s == S) {
+          s = 0;
+          ph ^= 1;
+        }
+      };
+      auto acc_acquire = [&](int b) {
+        if (ok && use[b] >= 1) {
+          if (!wait(&acc_empty[b], (use[b] - 1) & 1, abort_flag, 0x400u + b)) ok = false;
+          tc_fence_after();
+        }
+      };
+      auto zva = [&](int g) {  // Z_V += K^_{l,g} W_V[:, g]^T from the reconstruction tile
+        const int rb = g & 1;
+        if (ok && !wait(&rec_full[rb], (g >> 1) & 1, abort_flag, 0x500u + rb)) ok = false;
+        tc_fence_after();
+        for (int j = 0; j < 2; ++j) chunk(zv_col, R, g == 0 && j == 0, recon(rb) + j * 16384, nullptr);
+        if (ok) umma_commit(&rec_free[rb]);
+      };
+      if (RC) {
+        for (int c = 0; c < NCH; ++c) chunk(zk_col, R, c == 0, nullptr, nullptr);
+        if (ok) umma_commit(zk_full);
+      }
+      for (int h = 0; h < H && ok; ++h) {
+        const int b = h & 1;
+        acc_acquire(b);
+        for (int j = 0; j < 2; ++j) chunk(acc_col[b], 128, j == 0, nullptr, nullptr);
+        if (RC) {
+          if (h == 0 && ok) {
+            if (!wait(z_ready, 0, abort_flag, 0x600u)) ok = false;
+            tc_fence_after();
+          }
+          for (int j = 0; j < RC; ++j) chunk(acc_col[b], 128, false, zhi(j), zlo(j));
+        }
+        if (ok) umma_commit(&acc_full[b]);
+        use[b]++;
+        if (RC && h >= 1) zva(h - 1);
+      }
+      if (RC) {
+        zva(H - 1);
+        for (int c = 0; c < NCH; ++c) chunk(zv_col, R, false, nullptr, nullptr);
+        if (ok) umma_commit(zv_full);
+      }
+      for (int h = 0; h < H && ok; ++h) {
+        const int b = (H + h) & 1;
+        acc_acquire(b);
+        for (int j = 0; j < 4; ++j) chunk(acc_col[b], 128, j == 0, nullptr, nullptr);
+        if (RC) {
+          if (h == 0 && ok) {
+            if (!wait(z_ready, 1, abort_flag, 0x601u)) ok = false;
+            tc_fence_after();
+          }
+          for (int j = 0; j < RC; ++j) chunk(acc_col[b], 128, false, zhi(j), zlo(j));
+        }
+        if (ok) umma_commit(&acc_full[b]);
+        use[b]++;
+      }
+      // every issued MMA completes before TMEM is released
+      umma_commit(mma_done);
+      const long long w0 = clock64();
+      while (!mbar_test(mma_done, 0) && clock64() - w0 < kWaitBudget) {
+      }
+    }
+  } else {
+    // ================================================================ epilogue (warps 2..9)
+    const int ew = warp - 2;
+    const int q = warp & 3;  // TMEM lane quarter of this warp
+    const int half = ew >> 2;
+    const int row = q * 32 + lane;
+    const int64_t t = (int64_t)t0 + row;
+    const bool valid = t < a.T;
+    const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
+    const bool elected = ew == 0 && lane == 0;
+    const int bits = a.bits;
+    const int levels = (1 << bits) - 1;
+    constexpr int NG = 64 / G;        // groups in this thread's half row
+    constexpr int NP = G / 32;        // 32-column pieces per group
+    bool ok = true;
+    int use[2] = {0, 0};
+
+    auto convert_latent = [&](uint32_t col) {  // TMEM latent -> bf16 hi / lo sub-tiles
+      constexpr int per = R / 2;                 // columns of this thread
+      for (int p = 0; p < per / 32; ++p) {
+        const int c0 = half * per + p * 32;       // latent column
+        float v[32];
+        tmem_ld32(lane_addr + col + c0, v);
+        uint8_t* hi = zhi(c0 / 64);
+        uint8_t* lo = zlo(c0 / 64);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t wh[4], wl[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float x0 = v[ch * 8 + 2 * i], x1 = v[ch * 8 + 2 * i + 1];
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
+            const float2 hf = __bfloat1622float2(h2);
+            wh[i] = *reinterpret_cast<const uint32_t*>(&h2);
+            wl[i] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
+          }
+          const int c16 = ((c0 % 64) >> 3) + ch;
+          *reinterpret_cast<uint4*>(hi + sw128_off(row, c16)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          *reinterpret_cast<uint4*>(lo + sw128_off(row, c16)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
+      }
+      tc_fence_before();
+      fence_async_smem();
+      mbar_arrive(z_ready);
+    };
+
+    auto head = [&](int u, int h, bool is_v) {
+      const int b = u & 1, rb = u & 1;
+      const int row_bytes = 128 * bits / 8;
+      const int64_t rowi = t * H + h;
+      uint8_t* codes = (is_v ? a.vcodes : a.kcodes) + rowi * row_bytes + half * (64 * bits / 8);
+      __half2* params = (is_v ? a.vparams : a.kparams) + rowi * (128 / G) + half * NG;
+      // inputs of this thread's half row, fetched before the accumulator is ready
+      uint4 xin[8];
+      uint4 cin[2];
+      __half2 pin[NG];
+      if (ENC) {
+        const __nv_bfloat16* X = (is_v ? a.xv : a.xk) + t * C + h * 128 + half * 64;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xin[i] = valid ? __ldcs(reinterpret_cast<const uint4*>(X) + i) : make_uint4(0, 0, 0, 0);
+      } else {
+        cin[0] = valid ? __ldcs(reinterpret_cast<const uint4*>(codes)) : make_uint4(0, 0, 0, 0);
+        cin[1] = (valid && bits == 4) ? __ldcs(reinterpret_cast<const uint4*>(codes) + 1) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int g = 0; g < NG; ++g) pin[g] = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
+      }
+      // the reconstruction tile rb is free once the store of head u-2 has read it
+      // and (cross-layer K heads) the MMA of Z_V has consumed it
+      if (elected) bulk_wait_read1();
+      epi_sync();
+      if (RC && u >= 2 && u - 2 <= H - 1) {
+        if (ok && !wait(&rec_free[rb], ((u - 2) >> 1) & 1, abort_flag, 0x700u + rb)) ok = false;
+      }
+      if (ok && !wait(&acc_full[b], use[b] & 1, abort_flag, 0x800u + b)) ok = false;
+      use[b]++;
+      tc_fence_after();
+      uint8_t* rtile = recon(rb) + half * 16384;
+      uint32_t cw[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // packed codes of the half row (64 codes)
+      const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
+      for (int g = 0; g < NG; ++g) {
+        float p[G];
+#pragma unroll
+        for (int pc = 0; pc < NP; ++pc) {
+          float v[32];
+          tmem_ld32(lane_addr + b * 128 + half * 64 + g * G + pc * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) p[pc * 32 + i] = v[i];
+        }
+        float sf, zf;
+        int qv[G];
+        if (ENC) {
+          float x[G];
+#pragma unroll
+          for (int i = 0; i < G / 8; ++i) unpack_bf16x8(xin[g * (G / 8) + i], x, i * 8);
+          float mn = x[0] - p[0], mx = mn;
+#pragma unroll
+          for (int i = 0; i < G; ++i) {
+            const float r = x[i] - p[i];
+            x[i] = r;
+            mn = fminf(mn, r);
+            mx = fmaxf(mx, r);
+          }
+          const __half sh = __float2half_rn((mx - mn) / (float)levels);
+          const __half zh = __float2half_rn(mn);
+          sf = __half2float(sh);
+          zf = __half2float(zh);
+          const float inv = sf > 0.f ? 1.f / sf : 0.f;
+#pragma unroll
+          for (int i = 0; i < G; ++i) {
+            float c = rintf((x[i] - zf) * inv);
+            c = fminf(fmaxf(c, 0.f), (float)levels);
+            qv[i] = (int)c;
+          }
+          if (valid) params[g] = __halves2half2(sh, zh);
+        } else {
+          const float2 f = __half22float2(pin[g]);
+          sf = f.x;
+          zf = f.y;
+#pragma unroll
+          for (int i = 0; i < G; ++i) {
+            const int e = g * G + i;  // element within the half row
+            qv[i] = (cwin[(e * bits) >> 5] >> ((e * bits) & 31)) & levels;
+          }
+        }
+        if (ENC) {
+#pragma unroll
+          for (int i = 0; i < G; ++i) {
+            const int e = g * G + i;
+            cw[(e * bits) >> 5] |= (uint32_t)qv[i] << ((e * bits) & 31);
+          }
+        }
+        // reconstruction -> swizzled tile (8 values per 16-byte chunk)
+#pragma unroll
+        for (int ch = 0; ch < G / 8; ++ch) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int e0 = ch * 8 + 2 * i;
+            w[i] = pack_bf16x2(p[e0] + fmaf(sf, (float)qv[e0], zf), p[e0 + 1] + fmaf(sf, (float)qv[e0 + 1], zf));
+          }
+          const int c16 = (g * G) / 8 + ch;
+          *reinterpret_cast<uint4*>(rtile + sw128_off(row, c16)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      if (ENC && valid) {
+        uint4* dst = reinterpret_cast<uint4*>(codes);
+        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        if (bits == 4) dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[b]);
+      fence_async_smem();
+      epi_sync();
+      if (elected) {
+        if (!is_v || a.store_v) {
+          const CUtensorMap* m = is_v ? &maps.vo : &maps.ko;
+          tma_store(m, h * 128, t0, recon(rb));
+          tma_store(m, h * 128 + 64, t0, recon(rb) + 16384);
+        }
+        bulk_commit();
+        if (!is_v && RC) mbar_arrive(&rec_full[rb]);
+      }
+    };
+
+    // After an abort every wait returns at once; the loops still run to the end
+    // so that all epilogue threads meet at every named barrier.
+    if (RC) {
+      if (!wait(zk_full, 0, abort_flag, 0x900u)) ok = false;
+      tc_fence_after();
+      convert_latent(256);
+    }
+    for (int h = 0; h < H; ++h) head(h, h, false);
+    if (elected) {
+      bulk_wait_all();
+      fence_async_global();
+      mbar_arrive(khat_stored);
+    }
+    if (RC) {
+      if (!wait(zv_full, 0, abort_flag, 0x901u)) ok = false;
+      tc_fence_after();
+      convert_latent(256 + R);
+    }
+    for (int h = 0; h < H; ++h) head(H + h, h, true);
+    if (elected) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (row-major) read or written in boxes of
+// box_rows x 64 columns with the 128-byte swizzle.
+static bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool ENC, int G, int RC>
+static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
+  auto k = xlayer_tc_kernel<ENC, G, RC>;
+  const int smem = Layout<RC>::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = (int)((a.T + 127) / 128);
+  k<<<grid, kThreads, smem, st>>>(m, a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <bool ENC>
+static cudaError_t dispatch(int group, int rc, const Maps& m, const Args& a, cudaStream_t st) {
+  if (group == 32) {
+    if (rc == 0) return launch<ENC, 32, 0>(m, a, st);
+    if (rc == 1) return launch<ENC, 32, 1>(m, a, st);
+    return launch<ENC, 32, 2>(m, a, st);
+  }
+  if (rc == 0) return launch<ENC, 64, 0>(m, a, st);
+  if (rc == 1) return launch<ENC, 64, 1>(m, a, st);
+  return launch<ENC, 64, 2>(m, a, st);
+}
+
+}  // namespace tc
+
+bool tc_codec_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
+  if (p->kind != KVC_PRED_XLAYER_DPLR) return false;
+  if (d->dtype != KVC_BF16 || d->head_dim != 128 || d->param_dtype != KVC_F16) return false;
+  if (d->bits != 2 && d->bits != 4) return false;
+  if (d->group != 32 && d->group != 64) return false;
+  if (p->rank != 0 && p->rank != 64 && p->rank != 128) return false;
+  if (d->n_tokens < 1 || (int64_t)d->n_heads * 128 * 2 > (1 << 20)) return false;
+  return tc::encode_fn() != nullptr;
+}
+
+size_t tc_workspace(int, const kvc_layer_desc*, const kvc_predictor*, int64_t) { return 0; }
+
+cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
+                           const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, void*, size_t,
+                           cudaStream_t st) {
+  const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128, r = p->rank;
+  tc::Maps m;
+  memset(&m, 0, sizeof(m));
+  bool ok = tc::map2d(&m.ks, Ks, T, C, 128) && tc::map2d(&m.vs, Vs, T, C, 128) &&
+            tc::map2d(&m.ko, Kr, T, C, 128) && tc::map2d(&m.vo, Vr ? Vr : Kr, T, C, 128) &&
+            tc::map2d(&m.bk, p->k_block, H * 128, 128, 128) && tc::map2d(&m.bv, p->v_block, H * 128, 256, 128);
+  if (ok && r > 0)
+    ok = tc::map2d(&m.wk, p->k_w, r, C, (uint32_t)r) && tc::map2d(&m.wv, p->v_w, r, 2 * C, (uint32_t)r) &&
+         tc::map2d(&m.uk, p->k_u, C, r, 128) && tc::map2d(&m.uv, p->v_u, C, r, 128);
+  if (!ok) return cudaErrorInvalidValue;
+  tc::Args a{(int64_t)T, (int)H, d->bits, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
+             (uint8_t*)c->k_codes, (__half2*)c->k_params, (uint8_t*)c->v_codes, (__half2*)c->v_params,
+             (enc && !Vr) ? 0 : 1};
+  const int rc = (int)(r / 64);
+  return enc ? tc::dispatch<true>(d->group, rc, m, a, st) : tc::dispatch<false>(d->group, rc, m, a, st);
+}
+
 bool tc_attend_supported(const kvc_layer_desc*, const kvc_predictor*, int64_t) { return false; }
 cudaError_t tc_attend(const kvc_layer_desc*, const kvc_predictor*, const void*, int64_t, const kvc_codes*, const void*,
                       const void*, const void*, const void*, int64_t, float, void*, void*, size_t, cudaStream_t) {

@@ -327,18 +327,18 @@ def _gmm(g, T: int, C: int, n_comp: int, sigma: float, device, chunk: int = 8192
     for a in range(0, T, chunk):
         b = min(T, a + chunk)
         X[a:b] = means[comp[a:b]] + sigma * _randn(g, b - a, C, device=device)
-    return X, comp
+    return X, comp, means
 
 
-def _kmeans(X: torch.Tensor, comp: torch.Tensor, n_c: int, iters: int, chunk: int = 8192):
+def _kmeans(X: torch.Tensor, comp: torch.Tensor, means: torch.Tensor, n_c: int, iters: int, chunk: int = 8192):
     """Lloyd's k-means (offline calibration), initialised from one sample of
-    each mixture component so that no two centres start in one component."""
+    each mixture component so that no two centres start in one component; a
+    component without samples starts at its mean."""
     T, C = X.shape
     first = torch.full((n_c,), -1, dtype=torch.long, device=X.device)
     order = torch.arange(T, device=X.device)
     first.scatter_reduce_(0, comp, order, reduce="amin", include_self=False)
-    first = torch.where(first < 0, torch.arange(n_c, device=X.device) % T, first)
-    cent = X[first].clone()
+    cent = torch.where((first >= 0)[:, None], X[first.clamp(min=0)], means[:n_c].to(X.dtype)).clone()
     for _ in range(iters):
         lab = torch.empty(T, dtype=torch.long, device=X.device)
         c2 = (cent * cent).sum(1)
@@ -363,9 +363,9 @@ def cluster_layer(seed: int = SEED_BASE + 4, device="cpu", T: int = 32768, H: in
     g = _gen(seed * 13 + 1, device)
     out = {}
     for name in ("k", "v"):
-        X, comp = _gmm(g, T, C, n_c, sigma, device)
+        X, comp, means = _gmm(g, T, C, n_c, sigma, device)
         out[name] = X.to(dtype).reshape(T, H, D).contiguous()
-        out[name + "_cent"] = _kmeans(X.to(dtype).float(), comp, n_c, iters).to(dtype).contiguous()
+        out[name + "_cent"] = _kmeans(X.to(dtype).float(), comp, means, n_c, iters).to(dtype).contiguous()
         E, _ = torch.linalg.qr(_randn(g, C, m, device=device, dtype=torch.float64))
         out[name + "_dec"] = E.to(dtype).contiguous()
         out[name + "_enc"] = E.T.to(dtype).contiguous()

@@ -81,18 +81,30 @@ def param_ulp(v, param: str) -> np.ndarray:
     return np.spacing(np.abs(v).astype(np.float16 if param == "f16" else np.float32)).astype(np.float64)
 
 
-def assert_params_close(s_gpu, z_gpu, s_ref, z_ref, param: str, what="params"):
-    """Stored (scale, zero) pairs: equal, or one rounding step of the parameter
-    dtype apart (the min / max they round came from fp32 vs fp64 residuals).
+PARAM_FLIP_BUDGET = 1e-2
+
+
+def assert_params_close(s_gpu, z_gpu, s_ref, z_ref, param: str, what="params", levels: int = 3):
+    """Stored (scale, zero) pairs.  They round the group's min and max of the
+    residual, which the GPU forms in fp32 (about 1e-6 relative away from the
+    oracle's fp64).  fp16 pairs: equal, or one fp16 rounding step apart, on at
+    most 1 % of the groups (a shift of 1e-6 crosses an fp16 rounding boundary
+    with probability about 2e-6 / 2^-11).  fp32 pairs: equal to 1e-5 relative.
     Returns the mask of groups whose pair differs."""
     ds = np.abs(s_gpu - s_ref)
     dz = np.abs(z_gpu - z_ref)
-    assert np.all(ds <= param_ulp(s_ref, param) * 1.0001 + 1e-30), f"{what}: a scale differs by more than 1 ulp"
-    assert np.all(dz <= param_ulp(z_ref, param) * 1.0001 + 1e-30), f"{what}: a zero differs by more than 1 ulp"
-    diff = (ds > 0) | (dz > 0)
     if param == "f16":
-        assert diff.mean() <= 1e-3, f"{what}: {diff.mean():.2e} of the groups differ"
-    return diff
+        us = np.maximum(param_ulp(s_ref, param), param_ulp(s_gpu, param))
+        uz = np.maximum(param_ulp(z_ref, param), param_ulp(z_gpu, param))
+        assert np.all(ds <= us * 1.0001), f"{what}: a scale differs by more than one fp16 step"
+        assert np.all(dz <= uz * 1.0001), f"{what}: a zero differs by more than one fp16 step"
+        diff = (ds > 0) | (dz > 0)
+        assert diff.mean() <= PARAM_FLIP_BUDGET, f"{what}: {diff.mean():.2e} of the groups differ"
+        return diff
+    span = np.abs(z_ref) + levels * np.abs(s_ref) + 1e-6
+    assert np.all(ds <= 1e-5 * span), f"{what}: a scale differs by more than 1e-5 of the group's span"
+    assert np.all(dz <= 1e-5 * span), f"{what}: a zero differs by more than 1e-5 of the group's span"
+    return np.zeros(s_ref.shape, bool)
 
 
 def assert_recon_close(rec_gpu, rec_ref, exact_ref, x, code_flip, state: str, what="recon"):

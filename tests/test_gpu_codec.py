@@ -51,7 +51,7 @@ def _gpu_coded(buf: kvc.CodeBuffers, T, H, D, bits, group, param, which="k"):
 def _compare(gc: O.Coded, oc: O.Coded, rec_gpu, rec_ref, exact, x, state, group, what, param="f16"):
     """Codes, parameters and reconstructions of one coded tensor [T,H,D]."""
     U.assert_codes_close(gc.q, oc.q, what + " codes")
-    pdiff = U.assert_params_close(gc.s, gc.z, oc.s, oc.z, param, what + " params")
+    pdiff = U.assert_params_close(gc.s, gc.z, oc.s, oc.z, param, what + " params", levels=int(max(3, oc.q.max())))
     flip = gc.q != oc.q
     if param == "f16":  # a different fp16 (scale, zero) moves the whole group
         flip = flip | np.repeat(pdiff, group, axis=-1)
@@ -192,6 +192,64 @@ def test_bf16_cross_layer_parity(T, rank):
     for l in (1, 2):
         # teacher forcing: layer l-1 sources are the clean values (bf16), shared by both sides
         _check_xlayer_layer(wl.weights[l], wl.K[l], wl.V[l], wl.K[l - 1], wl.V[l - 1], bf, hf, 2, 32, rank)
+
+
+def _exact_xlayer_chain(L, T, H, D, r, seed):
+    """Layers whose K / V are exact bf16 images of sparse +-1 block-DPLR maps of
+    the previous (reconstructed) layer, with an INT2-grid anchor: every residual
+    of layers >= 1 is exactly 0 and no rounding decision is near a tie."""
+    rng = np.random.default_rng(seed)
+    C = H * D
+
+    def sparse(shape, nnz):
+        m = np.zeros(shape)
+        for idx in np.ndindex(*shape[:-1]):
+            m[idx + (rng.choice(shape[-1], nnz, replace=False),)] = rng.choice([-1.0, 1.0], nnz)
+        return m
+
+    grid = -1.5 + rng.integers(0, 4, (T, H, D)).astype(np.float64)
+    grid[..., 0::32], grid[..., 1::32] = -1.5, 1.5
+    K = [grid]
+    g2 = -1.5 + rng.integers(0, 4, (T, H, D)).astype(np.float64)
+    g2[..., 0::32], g2[..., 1::32] = -1.5, 1.5
+    V = [g2]
+    W = [None]
+    for _ in range(1, L):
+        w = dict(k_block=sparse((H, D, D), 1), k_w=sparse((r, C), 1) if r else np.zeros((0, C)),
+                 k_u=sparse((C, r), 1) * 0.5 if r else np.zeros((C, 0)),
+                 v_block=sparse((H, D, 2 * D), 1), v_w=sparse((r, 2 * C), 1) if r else np.zeros((0, 2 * C)),
+                 v_u=sparse((C, r), 1) * 0.5 if r else np.zeros((C, 0)))
+        Kl = O.xlayer_predict_k(K[-1], w["k_block"], w["k_w"], w["k_u"])
+        Vl = O.xlayer_predict_v(Kl, V[-1], w["v_block"], w["v_w"], w["v_u"])
+        assert np.array_equal(O.round_to(Kl, "bf16"), Kl) and np.array_equal(O.round_to(Vl, "bf16"), Vl)
+        K.append(Kl)
+        V.append(Vl)
+        W.append(w)
+    t = lambda x: torch.from_numpy(x).float().to(torch.bfloat16).contiguous()
+    return [t(k) for k in K], [t(v) for v in V], [None] + [{k: t(v) for k, v in w.items()} for w in W[1:]]
+
+
+@pytest.mark.parametrize("rank", [64, 0])
+def test_cross_layer_chain_exact_predictor(rank):
+    """The GPU's own closed-loop chain over several layers (each layer
+    predicted from the GPU's reconstruction of the previous one) stays
+    bit-identical to the exact values when every prediction is exact."""
+    L, T, H, D = 3, 2 * 128 + 40, 12, 128
+    K, V, W = _exact_xlayer_chain(L, T, H, D, rank, 31 + rank)
+    bf, hf = torch.bfloat16, torch.float16
+    desc0 = _desc(T, H, D, bf, 2, 32, hf)
+    p0 = kvc.make_predictor(kvc.PRED_NONE)
+    buf = kvc.alloc_codes(desc0, p0)
+    Kr, Vr = torch.empty(T, H, D, dtype=bf, device="cuda"), torch.empty(T, H, D, dtype=bf, device="cuda")
+    kvc.kvc_encode_layer(desc0, p0, K[0].cuda(), V[0].cuda(), None, None, buf, Kr, Vr)
+    for l in range(1, L):
+        pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in W[l].items()}, rank=rank)
+        b2, Kn, Vn = _xlayer_gpu(desc0, pred, K[l].cuda(), V[l].cuda(), Kr, Vr)
+        assert torch.equal(Kn.cpu(), K[l]) and torch.equal(Vn.cpu(), V[l]), f"layer {l}"
+        assert int(b2.k_codes.count_nonzero()) == 0 and int(b2.v_codes.count_nonzero()) == 0
+        s_, z_ = U.params_from_gpu(b2.k_params, (T, H, D // 32), "f16")
+        assert np.all(s_ == 0) and np.all(z_ == 0)
+        Kr, Vr = Kn, Vn
 
 
 def test_bf16_cross_layer_full_size_sampled():
@@ -396,7 +454,7 @@ def _cluster_pred(cw: synth.ClusterWorkload, n_c):
     return kvc.make_predictor(kvc.PRED_CLUSTER, w, n_clusters=n_c, code_dim=cw.k_enc.shape[0])
 
 
-@pytest.mark.parametrize("T,H,n_c", [(1000, 4, 32), (77, 16, 256)])
+@pytest.mark.parametrize("T,H,n_c", [(1000, 4, 32), (300, 16, 256)])
 def test_cluster_codec_parity(T, H, n_c):
     cw = synth.cluster_layer(seed=synth.SEED_BASE + 104, T=T, H=H, n_c=n_c, iters=5)
     D = 128
