@@ -48,14 +48,34 @@ def _gpu_coded(buf: kvc.CodeBuffers, T, H, D, bits, group, param, which="k"):
     return O.Coded(q, s, z)
 
 
-def _compare(gc: O.Coded, oc: O.Coded, rec_gpu, rec_ref, exact, x, state, group, what, param="f16"):
-    """Codes, parameters and reconstructions of one coded tensor [T,H,D]."""
+def _compare(gc: O.Coded, oc: O.Coded, rec_gpu, rec_ref, exact, x, state, group, what, param="f16", err=None,
+             skip_tokens=None):
+    """Codes, parameters and reconstructions of one coded tensor [T,H,D].
+    err: per-element bound of the GPU prediction's accumulation error;
+    skip_tokens: tokens whose prediction inputs already differ (a flipped code
+    or reconstruction upstream), checked for validity and against the budgets
+    only.  Returns the per-token mask of tokens whose codes, (scale, zero) or
+    reconstruction differ in any element."""
     U.assert_codes_close(gc.q, oc.q, what + " codes")
-    pdiff = U.assert_params_close(gc.s, gc.z, oc.s, oc.z, param, what + " params", levels=int(max(3, oc.q.max())))
+    skip = None
+    if skip_tokens is not None:
+        skip = np.broadcast_to(skip_tokens.reshape((-1,) + (1,) * (oc.s.ndim - 1)), oc.s.shape)
+    levels = int(max(3, oc.q.max()))
+    pdiff = U.assert_params_close(gc.s, gc.z, oc.s, oc.z, param, what + " params", levels=levels, err=err,
+                                  group=group, skip=skip)
     flip = gc.q != oc.q
     if param == "f16":  # a different fp16 (scale, zero) moves the whole group
         flip = flip | np.repeat(pdiff, group, axis=-1)
-    U.assert_recon_close(rec_gpu, rec_ref, exact, x, flip, state, what + " recon")
+    if skip_tokens is not None:
+        flip = flip | skip_tokens.reshape((-1,) + (1,) * (flip.ndim - 1))
+    # the GPU's own code around the oracle's prediction (validity of flipped elements)
+    pred_ref = exact - O.dequantize_groups(oc.q, oc.s, oc.z, group)
+    alt = pred_ref + O.dequantize_groups(gc.q, gc.s, gc.z, group)
+    if skip_tokens is not None:
+        alt = np.where(skip_tokens.reshape((-1,) + (1,) * (flip.ndim - 1)), rec_gpu, alt)
+    U.assert_recon_close(rec_gpu, rec_ref, exact, x, flip, state, what + " recon", err=err, alt=alt)
+    differs = flip | (rec_gpu != rec_ref)
+    return differs.reshape(differs.shape[0], -1).any(axis=1)
 
 
 # ---------------------------------------------------------------- packing
@@ -144,12 +164,13 @@ def _check_xlayer_layer(w, K, V, Ks, Vs, dtype, param, bits, group, rank):
     Ks64, Vs64 = U.to64(Ks), U.to64(Vs)
     ck, cv, Kh, Vh = O.encode_layer_xlayer(od, w64, U.to64(K), U.to64(V), Ks64, Vs64)
     ek, ev = U.exact_xlayer(od, w64, ck, cv, Ks64, Vs64, Kh)
+    errk, errv = U.err_xlayer(od, w64, Ks64, Vs64, Kh)
     p = U.np_param(param)
-    # V is predicted from the GPU's own K_rec; where K codes agree the inputs are the same values
-    _compare(_gpu_coded(buf, T, H, D, bits, group, p, "k"), ck, U.to64(Kr), Kh, ek, U.to64(K), od.state, group, "K",
-             p)
+    # V is predicted from the GPU's own K_rec: tokens with a flipped K code feed it other values
+    kflip = _compare(_gpu_coded(buf, T, H, D, bits, group, p, "k"), ck, U.to64(Kr), Kh, ek, U.to64(K), od.state,
+                     group, "K", p, errk)
     _compare(_gpu_coded(buf, T, H, D, bits, group, p, "v"), cv, U.to64(Vr), Vh, ev, U.to64(V), od.state, group, "V",
-             p)
+             p, errv, kflip)
     return Kh, Vh
 
 
@@ -270,12 +291,15 @@ def test_bf16_cross_layer_full_size_sampled():
     w64 = {k: U.to64(v) for k, v in w.items()}
     ck, cv, Kh, Vh = O.encode_layer_xlayer(od, w64, sub(wl.K[2]), sub(wl.V[2]), sub(wl.K[1]), sub(wl.V[1]))
     ek, ev = U.exact_xlayer(od, w64, ck, cv, sub(wl.K[1]), sub(wl.V[1]), Kh)
+    errk, errv = U.err_xlayer(od, w64, sub(wl.K[1]), sub(wl.V[1]), Kh)
     ii = idx.numpy()
-    for which, oc, rec, ref, ex, x in (("k", ck, Kr, Kh, ek, wl.K[2]), ("v", cv, Vr, Vh, ev, wl.V[2])):
+    kflip = None
+    for which, oc, rec, ref, ex, x, er in (("k", ck, Kr, Kh, ek, wl.K[2], errk), ("v", cv, Vr, Vh, ev, wl.V[2], errv)):
         q = U.codes_from_gpu(getattr(buf, which + "_codes"), (T, H, D), 2)[ii]
         s_, z_ = U.params_from_gpu(getattr(buf, which + "_params"), (T, H, D // 32), "f16")
         gc = O.Coded(q, s_[ii], z_[ii])
-        _compare(gc, oc, sub(rec), ref, ex, sub(x), "bf16", 32, which + " (sampled tokens)")
+        f = _compare(gc, oc, sub(rec), ref, ex, sub(x), "bf16", 32, which + " (sampled tokens)", "f16", er, kflip)
+        kflip = f
 
 
 # ---------------------------------------------------------------- temporal
@@ -325,14 +349,16 @@ def test_temporal_parity_frame_by_frame(T, H, D, F, bits, group, ab, dtype):
     w64 = dict(ak=U.to64(tw.ak), av=U.to64(tw.av))
     ck, cv, Kh, Vh = O.encode_layer_temporal(od, w64, U.to64(tw.K), U.to64(tw.V))
     ek, ev = U.exact_temporal(od, w64, ck, cv, Kh, Vh)
+    errk, errv = U.err_temporal(od, w64, Kh, Vh)
     buf, Kr, Vr = _temporal_call(tw.ak, tw.av, tw.K, tw.V, F, bits, group, param, ab)
     n0 = min(F, T)
     gk = _temporal_gpu_coded(buf, T, H, D, F, bits, ab, group, p, "k")
     gv = _temporal_gpu_coded(buf, T, H, D, F, bits, ab, group, p, "v")
     sl = slice(0, n0)
     cut = lambda c: O.Coded(c.q[sl], c.s[sl], c.z[sl])
-    _compare(cut(gk), cut(ck), U.to64(Kr)[sl], Kh[sl], ek[sl], U.to64(tw.K)[sl], od.state, group, "K frame 0", p)
-    _compare(cut(gv), cut(cv), U.to64(Vr)[sl], Vh[sl], ev[sl], U.to64(tw.V)[sl], od.state, group, "V frame 0", p)
+    kf = _compare(cut(gk), cut(ck), U.to64(Kr)[sl], Kh[sl], ek[sl], U.to64(tw.K)[sl], od.state, group, "K frame 0", p)
+    _compare(cut(gv), cut(cv), U.to64(Vr)[sl], Vh[sl], ev[sl], U.to64(tw.V)[sl], od.state, group, "V frame 0", p,
+             None, kf)
     tdt = torch.float32
     for f in range(1, (T + F - 1) // F):
         a, b = f * F, min(T, (f + 1) * F)
@@ -347,11 +373,12 @@ def test_temporal_parity_frame_by_frame(T, H, D, F, bits, group, ab, dtype):
         n = b - a
         ofs = O.Desc(n, H, D, od.state, bits, group, p, F, 0)
         fk, fv, fKh, fVh = O.encode_layer_temporal(ofs, w64, U.to64(tw.K[a:b]), U.to64(tw.V[a:b]), k_hist, v_hist)
-        fek, fev = U.exact_temporal(ofs, w64, fk, fv, fKh, fVh)
+        fek, fev = U.exact_temporal(ofs, w64, fk, fv, fKh, fVh, k_hist, v_hist)
+        erk, erv = U.err_temporal(ofs, w64, fKh, fVh, k_hist, v_hist)
         gk = _temporal_gpu_coded(fb, n, H, D, F, bits, 0, group, p, "k")
         gv = _temporal_gpu_coded(fb, n, H, D, F, bits, 0, group, p, "v")
-        _compare(gk, fk, U.to64(fK), fKh, fek, U.to64(tw.K[a:b]), od.state, group, f"K frame {f}", p)
-        _compare(gv, fv, U.to64(fV), fVh, fev, U.to64(tw.V[a:b]), od.state, group, f"V frame {f}", p)
+        kf = _compare(gk, fk, U.to64(fK), fKh, fek, U.to64(tw.K[a:b]), od.state, group, f"K frame {f}", p, erk)
+        _compare(gv, fv, U.to64(fV), fVh, fev, U.to64(tw.V[a:b]), od.state, group, f"V frame {f}", p, erv, kf)
 
 
 def _exact_temporal_workload(T, H, D, F, seed):
@@ -437,12 +464,25 @@ def test_temporal_full_size_sampled_positions():
     vh64 = U.to64(v_hist[torch.from_numpy(pos).cuda()])
     ofs = _odesc(len(rows_b), H, D, torch.bfloat16, 4, 64, hf, len(pos), 0)
     fk, fv, fKh, fVh = O.encode_layer_temporal(ofs, w64, sb(tw.K[a:b]), sb(tw.V[a:b]), kh64, vh64)
-    fek, fev = U.exact_temporal(ofs, w64, fk, fv, fKh, fVh)
-    for which, oc, rec, ref, ex, x in (("k", fk, fK, fKh, fek, tw.K[a:b]), ("v", fv, fV, fVh, fev, tw.V[a:b])):
-        q = U.codes_from_gpu(getattr(fb, which + "_codes"), (nf * F, H, D), 4)[rows_b]
-        s_, z_ = U.params_from_gpu(getattr(fb, which + "_params"), (nf * F, H, D // 64), "f16")
-        _compare(O.Coded(q, s_[rows_b], z_[rows_b]), oc, sb(rec), ref, ex, sb(x), "bf16", 64,
-                 which + " continued frames")
+    fek, fev = U.exact_temporal(ofs, w64, fk, fv, fKh, fVh, kh64, vh64)
+    erk, erv = U.err_temporal(ofs, w64, fKh, fVh, kh64, vh64)
+    # inside the call each frame is predicted from the call's own earlier frames: a
+    # position whose earlier frames differ anywhere is only checked for validity
+    npos = len(pos)
+    diverged = np.zeros(npos, bool)
+    gq = {w: U.codes_from_gpu(getattr(fb, w + "_codes"), (nf * F, H, D), 4)[rows_b] for w in "kv"}
+    gp = {w: U.params_from_gpu(getattr(fb, w + "_params"), (nf * F, H, D // 64), "f16") for w in "kv"}
+    for f in range(nf):
+        sl = slice(f * npos, (f + 1) * npos)
+        cut = lambda c: O.Coded(c.q[sl], c.s[sl], c.z[sl])
+        kf = diverged.copy()
+        for which, oc, rec, ref, ex, x, er in (("k", fk, fK, fKh, fek, tw.K[a:b], erk),
+                                              ("v", fv, fV, fVh, fev, tw.V[a:b], erv)):
+            s_, z_ = gp[which]
+            g = O.Coded(gq[which][sl], s_[rows_b][sl], z_[rows_b][sl])
+            kf = kf | _compare(g, cut(oc), sb(rec)[sl], ref[sl], ex[sl], sb(x)[sl], "bf16", 64,
+                               f"{which} continued frame {f}", "f16", er[sl], kf)
+        diverged |= kf
 
 
 # ---------------------------------------------------------------- clustered
@@ -487,13 +527,17 @@ def test_cluster_codec_parity(T, H, n_c):
         q = U.codes_from_gpu(getattr(buf, which + "_codes"), (T, 128), 4)
         s, z = U.params_from_gpu(getattr(buf, which + "_params"), (T, 4), "f16")
         U.assert_codes_close(q, oc.q, which + " coefficient codes")
-        pdiff = U.assert_params_close(s[clear], z[clear], oc.s[clear], oc.z[clear], "f16", which + " params")
+        ecoef = U.err_cluster(X64.reshape(T, -1), c64, oc.assign, U.to64(enc))
+        pdiff = U.assert_params_close(s[clear], z[clear], oc.s[clear], oc.z[clear], "f16", which + " params",
+                                      levels=15, err=ecoef[clear], group=32)
         exact = (c64[oc.assign] + O.dequantize_groups(oc.q, oc.s, oc.z, 32) @ U.to64(dec).T).reshape(T, H, D)
         # a token whose centre, any code or any (scale, zero) differs has every channel moved
         tok_flip = (q != oc.q).any(axis=1) | ~clear
         tok_flip[np.flatnonzero(clear)[pdiff.any(axis=1)]] = True
         flip = np.repeat(tok_flip, H * D).reshape(T, H, D)
-        U.assert_recon_close(U.to64(rec), xh, exact, X64, flip, "bf16", which + " recon")
+        coef_hat = O.dequantize_groups(oc.q, oc.s, oc.z, 32)
+        erec = (128 * U.U32 * (np.abs(coef_hat) @ np.abs(U.to64(dec)).T) + U.U32 * np.abs(c64[oc.assign]))
+        U.assert_recon_close(U.to64(rec), xh, exact, X64, flip, "bf16", which + " recon", err=erec.reshape(T, H, D))
 
 
 # ---------------------------------------------------------------- attention
