@@ -239,3 +239,16 @@ def kvc_launch_counter() -> int:
 
 def kvc_status_string(status: int) -> str:
     return lib().kvc_status_string(status).decode()
+
+
+def kvc_encode_layer_cluster_static(desc, pred, K, V, codes: CodeBuffers, K_rec=None, V_rec=None, stream=None):
+    """Clustered-codec encode that allocates nothing (its centre tables live in
+    a static device array inside the library); for callers that cannot
+    allocate device memory at encode time.  Same results as kvc_encode_layer."""
+    fn = lib().kvc_encode_layer_cluster_static
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(LayerDesc), ctypes.POINTER(Predictor), ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.POINTER(Codes), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    c = codes.struct()
+    _check(fn(ctypes.byref(desc), ctypes.byref(pred), _ptr(K), _ptr(V), ctypes.byref(c), _ptr(K_rec), _ptr(V_rec),
+              _stream(stream)), "kvc_encode_layer_cluster_static")

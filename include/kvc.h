@@ -221,6 +221,28 @@ KVC_API const char* kvc_last_cuda_error(void);
  * (all threads, all devices); for counting launches in a timed region. */
 KVC_API uint64_t kvc_launch_counter(void);
 
+/* kvc_encode_layer for the clustered predictor, for callers that cannot
+ * allocate device memory when they encode (code inside an allocator or memory
+ * pool callback, a runtime that hands out pre-carved device memory, a plugin
+ * host that forbids cudaMalloc on its threads).  The pages have no counterpart:
+ * this is an interface choice of this library.
+ *  Same meaning, layouts and results as kvc_encode_layer with
+ *  pred->kind == KVC_PRED_CLUSTER (no K_src / V_src, no workspace); K_rec and
+ *  V_rec may be NULL.
+ *  The centre tables it needs live in a file-scope __device__ array sized for
+ *  at most 256 centres of 128 coefficients (about 264 KB, held by every GPU that
+ *  loads the library until the process exits); larger n_clusters or another
+ *  code_dim return KVC_ERR_UNSUPPORTED before anything runs.
+ *  It calls no cudaMalloc / cudaFree.  The first call on a device looks up the
+ *  array's device address (cudaGetSymbolAddress), so make that first call
+ *  before any stream capture.  Every call writes the whole table before
+ *  reading it, so nothing carries over between calls, but all calls share the
+ *  one array: calls that can overlap on the GPU (other streams, other threads)
+ *  race and must be serialized by the caller. */
+KVC_API kvc_status kvc_encode_layer_cluster_static(const kvc_layer_desc* desc, const kvc_predictor* pred,
+                                                   const void* K, const void* V, const kvc_codes* out,
+                                                   void* K_rec, void* V_rec, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
