@@ -105,16 +105,17 @@ class Clocks:
 class XLayerBench:
     """Buffers and calls of the 30-layer encode + decode step."""
 
-    def __init__(self, device, seed):
-        self.wl = synth.wan_xlayer(seed=seed, device=device, L=L_LAYERS, T=T_TOK, H=H, D=D, rank=RANK)
+    def __init__(self, device, seed, layers=L_LAYERS):
+        self.L = layers
+        self.wl = synth.wan_xlayer(seed=seed, device=device, L=layers, T=T_TOK, H=H, D=D, rank=RANK)
         bf, hf = torch.bfloat16, torch.float16
         self.desc0 = kvc.make_desc(T_TOK, H, D, bf, 4, 32, hf)  # INT4 anchor
         self.desc = kvc.make_desc(T_TOK, H, D, bf, 2, 32, hf)
         self.pred0 = kvc.make_predictor(kvc.PRED_NONE)
         self.preds = [None] + [kvc.make_predictor(kvc.PRED_XLAYER_DPLR, self.wl.weights[l], rank=RANK)
-                               for l in range(1, L_LAYERS)]
+                               for l in range(1, layers)]
         self.codes = [kvc.alloc_codes(self.desc0, self.pred0, device)] + \
-                     [kvc.alloc_codes(self.desc, self.preds[l], device) for l in range(1, L_LAYERS)]
+                     [kvc.alloc_codes(self.desc, self.preds[l], device) for l in range(1, layers)]
         self.ws_enc = kvc.alloc_workspace(kvc.OP_ENCODE, self.desc, self.preds[1], device=device)
         self.ws_dec = kvc.alloc_workspace(kvc.OP_DECODE, self.desc, self.preds[1], device=device)
         mk = lambda: torch.empty(T_TOK, H, D, dtype=bf, device=device)
@@ -126,7 +127,7 @@ class XLayerBench:
         K, V = self.wl.K, self.wl.V
         Kr, Vr = self.er[0]
         kvc.kvc_encode_layer(self.desc0, self.pred0, K[0], V[0], None, None, self.codes[0], Kr, Vr)
-        for l in range(1, L_LAYERS):
+        for l in range(1, self.L):
             Ks, Vs = self.er[(l - 1) % 2]
             Kr, Vr = self.er[l % 2]
             if ev is not None:
@@ -140,7 +141,7 @@ class XLayerBench:
     def decode_chain(self, ev=None):
         Kr, Vr = self.dr[0]
         kvc.kvc_decode_layer(self.desc0, self.pred0, self.codes[0], None, None, Kr, Vr)
-        for l in range(1, L_LAYERS):
+        for l in range(1, self.L):
             Ks, Vs = self.dr[(l - 1) % 2]
             Kr, Vr = self.dr[l % 2]
             if ev is not None:
@@ -370,6 +371,8 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the extra per-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--layers", type=int, default=L_LAYERS,
+                    help="layers of the cross-layer workload (the headline number uses all 30)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -393,7 +396,8 @@ def main():
     build.build()
     hbm, tf_burst, tf_sust, peak_kind = peaks()
 
-    xb = XLayerBench(dev, synth.SEED_BASE + 1 + 1000 * rank)
+    xb = XLayerBench(dev, synth.SEED_BASE + 1 + 1000 * rank, args.layers)
+    L_RUN = args.layers
     torch.cuda.synchronize()
 
     def barrier():
@@ -406,7 +410,7 @@ def main():
     assert kvc.kvc_get_device_error() == 0
 
     mk = lambda: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(L_LAYERS)]
+                  for _ in range(L_RUN)]
     ev_enc = [mk() for _ in range(args.steps)]
     ev_dec = [mk() for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -431,7 +435,7 @@ def main():
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms_total = float(t.item())
     ms_step = ms_total / args.steps
-    units_per_step = 2 * T_TOK * L_LAYERS * world
+    units_per_step = 2 * T_TOK * L_RUN * world
     value = units_per_step / (ms_step * 1e-3)
 
     enc_ms = statistics.mean(x for k in range(args.steps) for x in time_events(ev_enc[k][1:]))
@@ -462,7 +466,7 @@ def main():
         bo = sum(t.numel() * t.element_size() for c in hcodes for t in c)
 
         def e2e_step():
-            for l in range(L_LAYERS):
+            for l in range(L_RUN):
                 xb.wl.K[l].copy_(hK[l], non_blocking=True)
                 xb.wl.V[l].copy_(hV[l], non_blocking=True)
             xb.step()
@@ -491,7 +495,7 @@ def main():
     rows = None
     cpu = None
     if world == 1:
-        if not args.no_rows:
+        if not args.no_rows and L_RUN > 15:
             xb.encode_chain(keep_layer=15)
             torch.cuda.synchronize()
             rows = {"c2_attention": row_attention(xb, hbm, tf_burst, tf_sust)}
@@ -501,7 +505,7 @@ def main():
             torch.cuda.empty_cache()
             rows["c4_cluster"] = row_cluster(dev, hbm, tf_burst)
         if not args.no_cpu:
-            cpu = oracle_xlayer_rate(xb.wl, 192, L_LAYERS, 20.0)
+            cpu = oracle_xlayer_rate(xb.wl, 192, L_RUN, 20.0)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -509,8 +513,8 @@ def main():
                 "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded Wan-1.3B-shaped trace, inter-layer correlation 0.9; block-DPLR "
                         "predictors fitted by least squares on a separate 4096-token trace)",
-                "config": {"workload": "cross-layer codec: encode + decode of 30 layers x 32760 tokens x 12 heads "
-                                       "x 128, bf16, INT2 g32 residual (INT4 anchor), block-DPLR rank 64",
+                "config": {"workload": f"cross-layer codec: encode + decode of {L_RUN} layers x 32760 tokens x 12 "
+                                       "heads x 128, bf16, INT2 g32 residual (INT4 anchor), block-DPLR rank 64",
                            "global_batch": T_TOK * world, "seq_len": T_TOK, "parallelism": f"dp{world}",
                            "l2": "inputs larger than L2 (6 GB per step streamed)"},
                 "roofline": roof, "layers": detail, "clocks": clk, "gpu_launches": launches,
