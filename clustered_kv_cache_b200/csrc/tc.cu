@@ -26,11 +26,24 @@
 #include <string.h>
 
 #include "tc.h"
+#include "tc_ptx.cuh"
 
 namespace kvc {
 
 // First error recorded by a bounded device-side wait (0 = none).
 __device__ unsigned int g_device_error = 0;
+
+unsigned int* tc_error_word() {
+  static unsigned int* ptr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<unsigned int*>(p);
+  }
+  return ptr[dev];
+}
 
 cudaError_t tc_read_and_clear_error(unsigned int* value) {
   cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(unsigned int));
@@ -41,159 +54,10 @@ cudaError_t tc_read_and_clear_error(unsigned int* value) {
 
 namespace tc {
 
-constexpr int kThreads = 320;  // 10 warps
-constexpr int kEpiThreads = 256;
-constexpr long long kWaitBudget = 1ll << 32;  // cycles (about 2 s) before a wait gives up
+constexpr int kThreads = 576;     // 18 warps: producer, MMA, two epilogue groups of 8
+constexpr int kGroupThreads = 256;
 
-// ---------------------------------------------------------------- PTX wrappers
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t n) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(n) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return r != 0;
-}
-
-// Waits for the phase of parity `parity` of barrier b; false if the CTA aborted
-// or the budget ran out (which records `where` and raises the abort flag).
-__device__ __forceinline__ bool wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, unsigned where) {
-  if (mbar_test(b, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_test(b, parity)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitBudget) {
-      *abort_flag = 1;
-      atomicCAS(&g_device_error, 0u, where);
-      return false;
-    }
-  }
-  return true;
-}
-
-__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* m, int x, int y, uint64_t* bar,
-                                         uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ void tma_store(const CUtensorMap* m, int x, int y, const void* src) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y), "r"(smem_u32(src))
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                     uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
-// 128 bytes, 8-row core groups 1024 bytes apart (the layout TMA writes with
-// CU_TENSOR_MAP_SWIZZLE_128B and a 64-element inner box).
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// Instruction descriptor: kind::f16, bf16 A and B (K-major), fp32 D, M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// Byte offset of the 16-byte chunk `c` (0..7) of row `row` inside a [rows][64]
-// bf16 sub-tile written with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t sw128_off(int row, int c) { return row * 128 + ((c ^ (row & 7)) << 4); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-template <int N>
-__device__ __forceinline__ void unpack_bf16x8(uint4 u, float (&v)[N], int base) {
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __bfloat1622float2(p[i]);
-    v[base + 2 * i] = f.x;
-    v[base + 2 * i + 1] = f.y;
-  }
-}
+enum Mode { kEncode = 0, kDecode = 1, kLatent = 2 };
 
 // ---------------------------------------------------------------- kernel arguments
 
@@ -206,6 +70,7 @@ struct Maps {
 };
 
 struct Args {
+  unsigned* err;  // device error word
   int64_t T;
   int H, bits;
   const __nv_bfloat16* xk;  // clean K (encode)
@@ -215,6 +80,8 @@ struct Args {
   uint8_t* vcodes;
   __half2* vparams;
   int store_v;  // V^_l is written (always for decode)
+  // latent mode: the layer's latents as bf16 hi / lo pairs, [T][r] each
+  __nv_bfloat16 *zk_hi, *zk_lo, *zv_hi, *zv_lo;
 };
 
 template <int RC>
@@ -231,8 +98,10 @@ struct Layout {
 
 // ---------------------------------------------------------------- the kernel
 
-template <bool ENC, int G, int RC>
-__global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_constant__ Maps maps, const Args a) {
+template <int MODE, int G, int RC>
+__global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps maps, const Args a) {
+  constexpr bool ENC = MODE == kEncode;
+  constexpr bool LAT = MODE == kLatent;
   using L = Layout<RC>;
   constexpr int S = L::S;
   constexpr int R = RC * 64;
@@ -266,14 +135,14 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kEpiThreads);
+      mbar_init(&acc_empty[i], kGroupThreads);
       mbar_init(&rec_full[i], 1);
       mbar_init(&rec_free[i], 1);
     }
     mbar_init(zk_full, 1);
     mbar_init(zv_full, 1);
-    mbar_init(z_ready, kEpiThreads);
-    mbar_init(khat_stored, 1);
+    mbar_init(z_ready, kGroupThreads);
+    mbar_init(khat_stored, 2);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -308,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       auto load = [&](const CUtensorMap* ma, int ax, uint64_t pa, const CUtensorMap* mb, int bx, int by,
                       uint32_t bbytes) {
         if (!ok) return;
-        if (!wait(&empty[s], ph ^ 1, abort_flag, 0x100u + s)) {
+        if (!wait(&empty[s], ph ^ 1, abort_flag, a.err, 0x100u + s)) {
           ok = false;
           return;
         }
@@ -334,15 +203,19 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       }
       if (RC) {
         for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, &maps.wv, (H - 1) * 128 + j * 64, 0, wbytes);
-        for (int c = 0; c < NCH; ++c) load(&maps.vs, c * 64, pol_keep, &maps.wv, C + c * 64, 0, wbytes);
+        for (int c = 0; c < NCH; ++c) load(&maps.vs, c * 64, LAT ? pol_stream : pol_keep, &maps.wv, C + c * 64, 0,
+                                           wbytes);
       }
-      if (ok && !wait(khat_stored, 0, abort_flag, 0x200u)) ok = false;
-      if (ok) fence_async_global();
-      for (int h = 0; h < H && ok; ++h) {
-        for (int j = 0; j < 2; ++j) load(&maps.ko, h * 128 + j * 64, pol_stream, &maps.bv, j * 64, h * 128, 16384);
-        for (int j = 0; j < 2; ++j)
-          load(&maps.vs, h * 128 + j * 64, pol_stream, &maps.bv, 128 + j * 64, h * 128, 16384);
-        for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, &maps.uv, j * 64, h * 128, 16384);
+      if (!LAT) {
+        if (ok && !wait(khat_stored, 0, abort_flag, a.err, 0x200u)) ok = false;
+        if (ok) fence_async_global();
+        for (int h = 0; h < H && ok; ++h) {
+          for (int j = 0; j < 2; ++j)
+            load(&maps.ko, h * 128 + j * 64, pol_stream, &maps.bv, j * 64, h * 128, 16384);
+          for (int j = 0; j < 2; ++j)
+            load(&maps.vs, h * 128 + j * 64, pol_stream, &maps.bv, 128 + j * 64, h * 128, 16384);
+          for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, &maps.uv, j * 64, h * 128, 16384);
+        }
       }
       if (!ok) {
         // drain: the loads already issued must land before the CTA exits
@@ -366,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       // one 64-wide K chunk: A from the stage (resA == 0) or resident smem
       auto chunk = [&](uint32_t d, int N, bool first, const uint8_t* resA, const uint8_t* resA2) {
         if (!ok) return;
-        if (!wait(&full[s], ph, abort_flag, 0x300u + s)) {
+        if (!wait(&full[s], ph, abort_flag, a.err, 0x300u + s)) {
           ok = false;
           return;
         }
@@ -389,13 +262,13 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       };
       auto acc_acquire = [&](int b) {
         if (ok && use[b] >= 1) {
-          if (!wait(&acc_empty[b], (use[b] - 1) & 1, abort_flag, 0x400u + b)) ok = false;
+          if (!wait(&acc_empty[b], (use[b] - 1) & 1, abort_flag, a.err, 0x400u + b)) ok = false;
           tc_fence_after();
         }
       };
       auto zva = [&](int g) {  // Z_V += K^_{l,g} W_V[:, g]^T from the reconstruction tile
         const int rb = g & 1;
-        if (ok && !wait(&rec_full[rb], (g >> 1) & 1, abort_flag, 0x500u + rb)) ok = false;
+        if (ok && !wait(&rec_full[rb], (g >> 1) & 1, abort_flag, a.err, 0x500u + rb)) ok = false;
         tc_fence_after();
         for (int j = 0; j < 2; ++j) chunk(zv_col, R, g == 0 && j == 0, recon(rb) + j * 16384, nullptr);
         if (ok) umma_commit(&rec_free[rb]);
@@ -410,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         for (int j = 0; j < 2; ++j) chunk(acc_col[b], 128, j == 0, nullptr, nullptr);
         if (RC) {
           if (h == 0 && ok) {
-            if (!wait(z_ready, 0, abort_flag, 0x600u)) ok = false;
+            if (!wait(z_ready, 0, abort_flag, a.err, 0x600u)) ok = false;
             tc_fence_after();
           }
           for (int j = 0; j < RC; ++j) chunk(acc_col[b], 128, false, zhi(j), zlo(j));
@@ -424,19 +297,21 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         for (int c = 0; c < NCH; ++c) chunk(zv_col, R, false, nullptr, nullptr);
         if (ok) umma_commit(zv_full);
       }
-      for (int h = 0; h < H && ok; ++h) {
-        const int b = (H + h) & 1;
-        acc_acquire(b);
-        for (int j = 0; j < 4; ++j) chunk(acc_col[b], 128, j == 0, nullptr, nullptr);
-        if (RC) {
-          if (h == 0 && ok) {
-            if (!wait(z_ready, 1, abort_flag, 0x601u)) ok = false;
-            tc_fence_after();
+      if (!LAT) {
+        for (int h = 0; h < H && ok; ++h) {
+          const int b = (H + h) & 1;
+          acc_acquire(b);
+          for (int j = 0; j < 4; ++j) chunk(acc_col[b], 128, j == 0, nullptr, nullptr);
+          if (RC) {
+            if (h == 0 && ok) {
+              if (!wait(z_ready, 1, abort_flag, a.err, 0x601u)) ok = false;
+              tc_fence_after();
+            }
+            for (int j = 0; j < RC; ++j) chunk(acc_col[b], 128, false, zhi(j), zlo(j));
           }
-          for (int j = 0; j < RC; ++j) chunk(acc_col[b], 128, false, zhi(j), zlo(j));
+          if (ok) umma_commit(&acc_full[b]);
+          use[b]++;
         }
-        if (ok) umma_commit(&acc_full[b]);
-        use[b]++;
       }
       // every issued MMA completes before TMEM is released
       umma_commit(mma_done);
@@ -445,8 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       }
     }
   } else {
-    // ================================================================ epilogue (warps 2..9)
-    const int ew = warp - 2;
+    // ================================================================ epilogue: two groups of 8 warps
+    // Group g owns TMEM accumulator g and reconstruction tile g, i.e. the heads
+    // u (K heads u = h, V heads u = H + h) with u % 2 == g; within a group two
+    // warps share each TMEM lane quarter and take 64 columns each.
+    const int grp = (warp - 2) >> 3;
+    const int ew = (warp - 2) & 7;
     const int q = warp & 3;  // TMEM lane quarter of this warp
     const int half = ew >> 2;
     const int row = q * 32 + lane;
@@ -456,15 +335,20 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     const bool elected = ew == 0 && lane == 0;
     const int bits = a.bits;
     const int levels = (1 << bits) - 1;
-    constexpr int NG = 64 / G;        // groups in this thread's half row
-    constexpr int NP = G / 32;        // 32-column pieces per group
-    bool ok = true;
-    int use[2] = {0, 0};
+    constexpr int NG = 64 / G;  // groups in this thread's half row
+    constexpr int NP = G / 32;  // 32-column passes per group
+    int use = 0;
+    auto gsync = [&]() {
+      if (grp == 0)
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+      else
+        asm volatile("bar.sync 2, 256;" ::: "memory");
+    };
 
-    auto convert_latent = [&](uint32_t col) {  // TMEM latent -> bf16 hi / lo sub-tiles
-      constexpr int per = R / 2;                 // columns of this thread
+    auto convert_latent = [&](uint32_t col, __nv_bfloat16* ghi, __nv_bfloat16* glo) {  // TMEM -> bf16 hi / lo
+      constexpr int per = R / 2;                                                         // columns of this thread
       for (int p = 0; p < per / 32; ++p) {
-        const int c0 = half * per + p * 32;       // latent column
+        const int c0 = half * per + p * 32;  // latent column
         float v[32];
         tmem_ld32(lane_addr + col + c0, v);
         uint8_t* hi = zhi(c0 / 64);
@@ -483,6 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           const int c16 = ((c0 % 64) >> 3) + ch;
           *reinterpret_cast<uint4*>(hi + sw128_off(row, c16)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
           *reinterpret_cast<uint4*>(lo + sw128_off(row, c16)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          if (LAT && valid) {
+            reinterpret_cast<uint4*>(ghi + t * R + c0)[ch] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            reinterpret_cast<uint4*>(glo + t * R + c0)[ch] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          }
         }
       }
       tc_fence_before();
@@ -490,8 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       mbar_arrive(z_ready);
     };
 
+    // one head of this group: u = global head index (K: h, V: H + h)
     auto head = [&](int u, int h, bool is_v) {
-      const int b = u & 1, rb = u & 1;
+      const int b = grp;  // == u & 1
       const int row_bytes = 128 * bits / 8;
       const int64_t rowi = t * H + h;
       uint8_t* codes = (is_v ? a.vcodes : a.kcodes) + rowi * row_bytes + half * (64 * bits / 8);
@@ -503,89 +392,95 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       if (ENC) {
         const __nv_bfloat16* X = (is_v ? a.xv : a.xk) + t * C + h * 128 + half * 64;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xin[i] = valid ? __ldcs(reinterpret_cast<const uint4*>(X) + i) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 8; ++i)
+          xin[i] = valid ? __ldcs(reinterpret_cast<const uint4*>(X) + i) : make_uint4(0, 0, 0, 0);
       } else {
         cin[0] = valid ? __ldcs(reinterpret_cast<const uint4*>(codes)) : make_uint4(0, 0, 0, 0);
         cin[1] = (valid && bits == 4) ? __ldcs(reinterpret_cast<const uint4*>(codes) + 1) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int g = 0; g < NG; ++g) pin[g] = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
       }
-      // the reconstruction tile rb is free once the store of head u-2 has read it
+      // the reconstruction tile is free once its previous TMA store has read it
       // and (cross-layer K heads) the MMA of Z_V has consumed it
-      if (elected) bulk_wait_read1();
-      epi_sync();
-      if (RC && u >= 2 && u - 2 <= H - 1) {
-        if (ok && !wait(&rec_free[rb], ((u - 2) >> 1) & 1, abort_flag, 0x700u + rb)) ok = false;
-      }
-      if (ok && !wait(&acc_full[b], use[b] & 1, abort_flag, 0x800u + b)) ok = false;
-      use[b]++;
+      if (elected) bulk_wait_read0();
+      gsync();
+      if (RC && u >= 2 && u - 2 <= H - 1) wait(&rec_free[b], ((u - 2) >> 1) & 1, abort_flag, a.err, 0x700u + b);
+      wait(&acc_full[b], use & 1, abort_flag, a.err, 0x800u + b);
+      use++;
       tc_fence_after();
-      uint8_t* rtile = recon(rb) + half * 16384;
+      uint8_t* rtile = recon(b) + half * 16384;
       uint32_t cw[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // packed codes of the half row (64 codes)
       const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
+#pragma unroll
       for (int g = 0; g < NG; ++g) {
-        float p[G];
-#pragma unroll
-        for (int pc = 0; pc < NP; ++pc) {
-          float v[32];
-          tmem_ld32(lane_addr + b * 128 + half * 64 + g * G + pc * 32, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) p[pc * 32 + i] = v[i];
-        }
         float sf, zf;
-        int qv[G];
         if (ENC) {
-          float x[G];
+          // group min / max of the residual over its NP passes of 32 columns
+          float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < G / 8; ++i) unpack_bf16x8(xin[g * (G / 8) + i], x, i * 8);
-          float mn = x[0] - p[0], mx = mn;
+          for (int pc = 0; pc < NP; ++pc) {
+            float p[32];
+            tmem_ld32(lane_addr + b * 128 + half * 64 + g * G + pc * 32, p);
 #pragma unroll
-          for (int i = 0; i < G; ++i) {
-            const float r = x[i] - p[i];
-            x[i] = r;
-            mn = fminf(mn, r);
-            mx = fmaxf(mx, r);
+            for (int ch = 0; ch < 4; ++ch) {
+              float x[8];
+              unpack_bf16x8(xin[(g * G + pc * 32) / 8 + ch], x, 0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float r = x[i] - p[ch * 8 + i];
+                mn = fminf(mn, r);
+                mx = fmaxf(mx, r);
+              }
+            }
           }
           const __half sh = __float2half_rn((mx - mn) / (float)levels);
           const __half zh = __float2half_rn(mn);
           sf = __half2float(sh);
           zf = __half2float(zh);
-          const float inv = sf > 0.f ? 1.f / sf : 0.f;
-#pragma unroll
-          for (int i = 0; i < G; ++i) {
-            float c = rintf((x[i] - zf) * inv);
-            c = fminf(fmaxf(c, 0.f), (float)levels);
-            qv[i] = (int)c;
-          }
           if (valid) params[g] = __halves2half2(sh, zh);
         } else {
           const float2 f = __half22float2(pin[g]);
           sf = f.x;
           zf = f.y;
-#pragma unroll
-          for (int i = 0; i < G; ++i) {
-            const int e = g * G + i;  // element within the half row
-            qv[i] = (cwin[(e * bits) >> 5] >> ((e * bits) & 31)) & levels;
-          }
         }
-        if (ENC) {
+        const float inv = sf > 0.f ? 1.f / sf : 0.f;
 #pragma unroll
-          for (int i = 0; i < G; ++i) {
-            const int e = g * G + i;
-            cw[(e * bits) >> 5] |= (uint32_t)qv[i] << ((e * bits) & 31);
+        for (int pc = 0; pc < NP; ++pc) {
+          const int e0 = g * G + pc * 32;  // first element (of the half row) of this pass
+          float p[32];
+          tmem_ld32(lane_addr + b * 128 + half * 64 + e0, p);
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {  // 8 elements: codes, packing, reconstruction
+            const int e = e0 + ch * 8;
+            int qv[8];
+            if (ENC) {
+              float x[8];
+              unpack_bf16x8(xin[e / 8], x, 0);
+              uint32_t v = 0;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                float c = rintf((x[i] - p[ch * 8 + i] - zf) * inv);
+                c = fminf(fmaxf(c, 0.f), (float)levels);
+                qv[i] = (int)c;
+                v |= (uint32_t)qv[i] << (i * bits);
+              }
+              if (bits == 2)
+                cw[e / 16] |= v << ((e % 16) * 2);
+              else
+                cw[e / 8] = v;
+            } else {
+              const uint32_t v = bits == 2 ? (cwin[e / 16] >> ((e % 16) * 2)) : cwin[e / 8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) qv[i] = (v >> (i * bits)) & levels;
+            }
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int k = ch * 8 + 2 * i;
+              w[i] = pack_bf16x2(p[k] + fmaf(sf, (float)qv[2 * i], zf), p[k + 1] + fmaf(sf, (float)qv[2 * i + 1], zf));
+            }
+            *reinterpret_cast<uint4*>(rtile + sw128_off(row, e / 8)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-        }
-        // reconstruction -> swizzled tile (8 values per 16-byte chunk)
-#pragma unroll
-        for (int ch = 0; ch < G / 8; ++ch) {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int e0 = ch * 8 + 2 * i;
-            w[i] = pack_bf16x2(p[e0] + fmaf(sf, (float)qv[e0], zf), p[e0 + 1] + fmaf(sf, (float)qv[e0 + 1], zf));
-          }
-          const int c16 = (g * G) / 8 + ch;
-          *reinterpret_cast<uint4*>(rtile + sw128_off(row, c16)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       if (ENC && valid) {
@@ -596,37 +491,40 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);
       fence_async_smem();
-      epi_sync();
+      gsync();
       if (elected) {
-        if (!is_v || a.store_v) {
+        if (!LAT && (!is_v || a.store_v)) {
           const CUtensorMap* m = is_v ? &maps.vo : &maps.ko;
-          tma_store(m, h * 128, t0, recon(rb));
-          tma_store(m, h * 128 + 64, t0, recon(rb) + 16384);
+          tma_store(m, h * 128, t0, recon(b));
+          tma_store(m, h * 128 + 64, t0, recon(b) + 16384);
         }
         bulk_commit();
-        if (!is_v && RC) mbar_arrive(&rec_full[rb]);
+        if (!is_v && RC) mbar_arrive(&rec_full[b]);
       }
     };
 
     // After an abort every wait returns at once; the loops still run to the end
-    // so that all epilogue threads meet at every named barrier.
-    if (RC) {
-      if (!wait(zk_full, 0, abort_flag, 0x900u)) ok = false;
+    // so that all threads of a group meet at every named barrier.
+    if (RC && grp == 0) {
+      wait(zk_full, 0, abort_flag, a.err, 0x900u);
       tc_fence_after();
-      convert_latent(256);
+      convert_latent(256, a.zk_hi, a.zk_lo);
     }
-    for (int h = 0; h < H; ++h) head(h, h, false);
+    for (int h = grp; h < H; h += 2) head(h, h, false);
     if (elected) {
       bulk_wait_all();
       fence_async_global();
       mbar_arrive(khat_stored);
     }
-    if (RC) {
-      if (!wait(zv_full, 0, abort_flag, 0x901u)) ok = false;
+    if (RC && grp == 0) {
+      wait(zv_full, 0, abort_flag, a.err, 0x901u);
       tc_fence_after();
-      convert_latent(256 + R);
+      convert_latent(256 + R, a.zv_hi, a.zv_lo);
     }
-    for (int h = 0; h < H; ++h) head(H + h, h, true);
+    if (!LAT) {
+      for (int u = H; u < 2 * H; ++u)
+        if ((u & 1) == grp) head(u, u - H, true);
+    }
     if (elected) bulk_wait_all();
   }
 
@@ -644,7 +542,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-static EncodeTiledFn encode_fn() {
+EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static bool tried = false;
   if (!tried) {
@@ -660,7 +558,7 @@ static EncodeTiledFn encode_fn() {
 
 // 2-D bf16 tensor [rows][cols] (row-major) read or written in boxes of
 // box_rows x 64 columns with the 128-byte swizzle.
-static bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -672,9 +570,9 @@ static bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool ENC, int G, int RC>
+template <int MODE, int G, int RC>
 static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
-  auto k = xlayer_tc_kernel<ENC, G, RC>;
+  auto k = xlayer_tc_kernel<MODE, G, RC>;
   const int smem = Layout<RC>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -684,16 +582,16 @@ static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <bool ENC>
+template <int MODE>
 static cudaError_t dispatch(int group, int rc, const Maps& m, const Args& a, cudaStream_t st) {
   if (group == 32) {
-    if (rc == 0) return launch<ENC, 32, 0>(m, a, st);
-    if (rc == 1) return launch<ENC, 32, 1>(m, a, st);
-    return launch<ENC, 32, 2>(m, a, st);
+    if (rc == 0) return launch<MODE, 32, 0>(m, a, st);
+    if (rc == 1) return launch<MODE, 32, 1>(m, a, st);
+    return launch<MODE, 32, 2>(m, a, st);
   }
-  if (rc == 0) return launch<ENC, 64, 0>(m, a, st);
-  if (rc == 1) return launch<ENC, 64, 1>(m, a, st);
-  return launch<ENC, 64, 2>(m, a, st);
+  if (rc == 0) return launch<MODE, 64, 0>(m, a, st);
+  if (rc == 1) return launch<MODE, 64, 1>(m, a, st);
+  return launch<MODE, 64, 2>(m, a, st);
 }
 
 }  // namespace tc
@@ -723,11 +621,13 @@ cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool
     ok = tc::map2d(&m.wk, p->k_w, r, C, (uint32_t)r) && tc::map2d(&m.wv, p->v_w, r, 2 * C, (uint32_t)r) &&
          tc::map2d(&m.uk, p->k_u, C, r, 128) && tc::map2d(&m.uv, p->v_u, C, r, 128);
   if (!ok) return cudaErrorInvalidValue;
-  tc::Args a{(int64_t)T, (int)H, d->bits, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
+  unsigned* err = tc_error_word();
+  if (!err) return cudaErrorInvalidDevice;
+  tc::Args a{err, (int64_t)T, (int)H, d->bits, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
              (uint8_t*)c->k_codes, (__half2*)c->k_params, (uint8_t*)c->v_codes, (__half2*)c->v_params,
-             (enc && !Vr) ? 0 : 1};
+             (enc && !Vr) ? 0 : 1, nullptr, nullptr, nullptr, nullptr};
   const int rc = (int)(r / 64);
-  return enc ? tc::dispatch<true>(d->group, rc, m, a, st) : tc::dispatch<false>(d->group, rc, m, a, st);
+  return enc ? tc::dispatch<tc::kEncode>(d->group, rc, m, a, st) : tc::dispatch<tc::kDecode>(d->group, rc, m, a, st);
 }
 
 bool tc_attend_supported(const kvc_layer_desc*, const kvc_predictor*, int64_t) { return false; }

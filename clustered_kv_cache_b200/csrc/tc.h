@@ -16,5 +16,7 @@ cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const voi
                       int64_t n_self, float scale, void* O, void* ws, size_t ws_bytes, cudaStream_t st);
 // reads the device error word of the current device and resets it to 0
 cudaError_t tc_read_and_clear_error(unsigned int* value);
+// device address of the error word on the current device (nullptr on failure)
+unsigned int* tc_error_word();
 
 }  // namespace kvc
