@@ -54,8 +54,8 @@ cudaError_t tc_read_and_clear_error(unsigned int* value) {
 
 namespace tc {
 
-constexpr int kThreads = 576;     // 18 warps: producer, MMA, two epilogue groups of 8
-constexpr int kGroupThreads = 256;
+constexpr int kThreads = 320;     // 10 warps: producer, MMA, two epilogue groups of 4
+constexpr int kGroupThreads = 128;
 
 enum Mode { kEncode = 0, kDecode = 1, kLatent = 2 };
 
@@ -99,7 +99,7 @@ struct Layout {
 // ---------------------------------------------------------------- the kernel
 
 template <int MODE, int G, int RC>
-__global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps maps, const Args a) {
+__global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_constant__ Maps maps, const Args a) {
   constexpr bool ENC = MODE == kEncode;
   constexpr bool LAT = MODE == kLatent;
   using L = Layout<RC>;
@@ -320,14 +320,13 @@ __global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps m
       }
     }
   } else {
-    // ================================================================ epilogue: two groups of 8 warps
+    // ================================================================ epilogue: two groups of 4 warps
     // Group g owns TMEM accumulator g and reconstruction tile g, i.e. the heads
-    // u (K heads u = h, V heads u = H + h) with u % 2 == g; within a group two
-    // warps share each TMEM lane quarter and take 64 columns each.
-    const int grp = (warp - 2) >> 3;
-    const int ew = (warp - 2) & 7;
+    // u (K heads u = h, V heads u = H + h) with u % 2 == g; each warp of a group
+    // covers one TMEM lane quarter (32 tokens) and all 128 channels.
+    const int grp = (warp - 2) >> 2;
+    const int ew = (warp - 2) & 3;
     const int q = warp & 3;  // TMEM lane quarter of this warp
-    const int half = ew >> 2;
     const int row = q * 32 + lane;
     const int64_t t = (int64_t)t0 + row;
     const bool valid = t < a.T;
@@ -335,20 +334,19 @@ __global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps m
     const bool elected = ew == 0 && lane == 0;
     const int bits = a.bits;
     const int levels = (1 << bits) - 1;
-    constexpr int NG = 64 / G;  // groups in this thread's half row
-    constexpr int NP = G / 32;  // 32-column passes per group
+    constexpr int NG = 128 / G;  // groups in a row
+    constexpr int NP = G / 32;   // 32-column passes per group
     int use = 0;
     auto gsync = [&]() {
       if (grp == 0)
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, 128;" ::: "memory");
       else
-        asm volatile("bar.sync 2, 256;" ::: "memory");
+        asm volatile("bar.sync 2, 128;" ::: "memory");
     };
 
     auto convert_latent = [&](uint32_t col, __nv_bfloat16* ghi, __nv_bfloat16* glo) {  // TMEM -> bf16 hi / lo
-      constexpr int per = R / 2;                                                         // columns of this thread
-      for (int p = 0; p < per / 32; ++p) {
-        const int c0 = half * per + p * 32;  // latent column
+      for (int p = 0; p < R / 32; ++p) {
+        const int c0 = p * 32;  // latent column
         float v[32];
         tmem_ld32(lane_addr + col + c0, v);
         uint8_t* hi = zhi(c0 / 64);
@@ -383,20 +381,21 @@ __global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps m
       const int b = grp;  // == u & 1
       const int row_bytes = 128 * bits / 8;
       const int64_t rowi = t * H + h;
-      uint8_t* codes = (is_v ? a.vcodes : a.kcodes) + rowi * row_bytes + half * (64 * bits / 8);
-      __half2* params = (is_v ? a.vparams : a.kparams) + rowi * (128 / G) + half * NG;
-      // inputs of this thread's half row, fetched before the accumulator is ready
-      uint4 xin[8];
-      uint4 cin[2];
+      uint8_t* codes = (is_v ? a.vcodes : a.kcodes) + rowi * row_bytes;
+      __half2* params = (is_v ? a.vparams : a.kparams) + rowi * (128 / G);
+      // inputs of this thread's row, fetched before the accumulator is ready
+      uint4 xin[16];
+      uint4 cin[4];
       __half2 pin[NG];
       if (ENC) {
-        const __nv_bfloat16* X = (is_v ? a.xv : a.xk) + t * C + h * 128 + half * 64;
+        const __nv_bfloat16* X = (is_v ? a.xv : a.xk) + t * C + h * 128;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 16; ++i)
           xin[i] = valid ? __ldcs(reinterpret_cast<const uint4*>(X) + i) : make_uint4(0, 0, 0, 0);
       } else {
-        cin[0] = valid ? __ldcs(reinterpret_cast<const uint4*>(codes)) : make_uint4(0, 0, 0, 0);
-        cin[1] = (valid && bits == 4) ? __ldcs(reinterpret_cast<const uint4*>(codes) + 1) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          cin[i] = (valid && i < bits) ? __ldcs(reinterpret_cast<const uint4*>(codes) + i) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int g = 0; g < NG; ++g) pin[g] = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
       }
@@ -408,8 +407,7 @@ __global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps m
       wait(&acc_full[b], use & 1, abort_flag, a.err, 0x800u + b);
       use++;
       tc_fence_after();
-      uint8_t* rtile = recon(b) + half * 16384;
-      uint32_t cw[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // packed codes of the half row (64 codes)
+      uint32_t cw[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};  // packed codes of the row
       const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
@@ -420,7 +418,7 @@ __global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps m
 #pragma unroll
           for (int pc = 0; pc < NP; ++pc) {
             float p[32];
-            tmem_ld32(lane_addr + b * 128 + half * 64 + g * G + pc * 32, p);
+            tmem_ld32(lane_addr + b * 128 + g * G + pc * 32, p);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
               float x[8];
@@ -446,9 +444,9 @@ __global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps m
         const float inv = sf > 0.f ? 1.f / sf : 0.f;
 #pragma unroll
         for (int pc = 0; pc < NP; ++pc) {
-          const int e0 = g * G + pc * 32;  // first element (of the half row) of this pass
+          const int e0 = g * G + pc * 32;  // first element of this pass
           float p[32];
-          tmem_ld32(lane_addr + b * 128 + half * 64 + e0, p);
+          tmem_ld32(lane_addr + b * 128 + e0, p);
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {  // 8 elements: codes, packing, reconstruction
             const int e = e0 + ch * 8;
@@ -479,14 +477,16 @@ __global__ void __maxnreg__(112) xlayer_tc_kernel(const __grid_constant__ Maps m
               const int k = ch * 8 + 2 * i;
               w[i] = pack_bf16x2(p[k] + fmaf(sf, (float)qv[2 * i], zf), p[k + 1] + fmaf(sf, (float)qv[2 * i + 1], zf));
             }
-            *reinterpret_cast<uint4*>(rtile + sw128_off(row, e / 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(recon(b) + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
       if (ENC && valid) {
         uint4* dst = reinterpret_cast<uint4*>(codes);
-        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        if (bits == 4) dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i < bits) dst[i] = make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]);
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);
@@ -606,7 +606,9 @@ bool tc_codec_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
   return tc::encode_fn() != nullptr;
 }
 
-size_t tc_workspace(int, const kvc_layer_desc*, const kvc_predictor*, int64_t) { return 0; }
+size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int64_t) {
+  return op == KVC_OP_ATTEND && tc_attend_supported(d, p, 0) ? tc_attend_workspace(d, p) : 0;
+}
 
 cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
                            const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, void*, size_t,
@@ -630,10 +632,27 @@ cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool
   return enc ? tc::dispatch<tc::kEncode>(d->group, rc, m, a, st) : tc::dispatch<tc::kDecode>(d->group, rc, m, a, st);
 }
 
-bool tc_attend_supported(const kvc_layer_desc*, const kvc_predictor*, int64_t) { return false; }
-cudaError_t tc_attend(const kvc_layer_desc*, const kvc_predictor*, const void*, int64_t, const kvc_codes*, const void*,
-                      const void*, const void*, const void*, int64_t, float, void*, void*, size_t, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace tc {
+// The layer's low-rank latents (bf16 hi / lo, [T][r] each) for attention: the
+// K half of a decode plus the V latent, without writing the reconstruction.
+cudaError_t latent_layer(const kvc_layer_desc* d, const kvc_predictor* p, const kvc_codes* c, const void* Ks,
+                         const void* Vs, void* zk_hi, void* zk_lo, void* zv_hi, void* zv_lo, cudaStream_t st) {
+  const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128, r = p->rank;
+  Maps m;
+  memset(&m, 0, sizeof(m));
+  bool ok = map2d(&m.ks, Ks, T, C, 128) && map2d(&m.vs, Vs, T, C, 128) && map2d(&m.ko, Ks, T, C, 128) &&
+            map2d(&m.vo, Ks, T, C, 128) && map2d(&m.bk, p->k_block, H * 128, 128, 128) &&
+            map2d(&m.bv, p->v_block, H * 128, 256, 128) && map2d(&m.wk, p->k_w, r, C, (uint32_t)r) &&
+            map2d(&m.wv, p->v_w, r, 2 * C, (uint32_t)r) && map2d(&m.uk, p->k_u, C, r, 128) &&
+            map2d(&m.uv, p->v_u, C, r, 128);
+  if (!ok) return cudaErrorInvalidValue;
+  unsigned* err = tc_error_word();
+  if (!err) return cudaErrorInvalidDevice;
+  Args a{err, (int64_t)T, (int)H, d->bits, nullptr, nullptr, (uint8_t*)c->k_codes, (__half2*)c->k_params,
+         (uint8_t*)c->v_codes, (__half2*)c->v_params, 0, (__nv_bfloat16*)zk_hi, (__nv_bfloat16*)zk_lo,
+         (__nv_bfloat16*)zv_hi, (__nv_bfloat16*)zv_lo};
+  return dispatch<kLatent>(d->group, (int)(r / 64), m, a, st);
 }
+}  // namespace tc
 
 }  // namespace kvc

@@ -11,6 +11,7 @@ cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool
                            const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, void* ws,
                            size_t ws_bytes, cudaStream_t st);
 bool tc_attend_supported(const kvc_layer_desc* d, const kvc_predictor* p, int64_t n_self);
+size_t tc_attend_workspace(const kvc_layer_desc* d, const kvc_predictor* p);
 cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
                       const kvc_codes* c, const void* Ks, const void* Vs, const void* K_self, const void* V_self,
                       int64_t n_self, float scale, void* O, void* ws, size_t ws_bytes, cudaStream_t st);
