@@ -369,6 +369,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the extra per-row measurements")
+    ap.add_argument("--rows", default="c2,c3,c4", help="which extra rows to measure (comma-separated)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--layers", type=int, default=L_LAYERS,
@@ -495,15 +496,20 @@ def main():
     rows = None
     cpu = None
     if world == 1:
-        if not args.no_rows and L_RUN > 15:
+        want = set(args.rows.split(",")) if not args.no_rows else set()
+        rows = {}
+        if "c2" in want and L_RUN > 15:
             xb.encode_chain(keep_layer=15)
             torch.cuda.synchronize()
-            rows = {"c2_attention": row_attention(xb, hbm, tf_burst, tf_sust)}
+            rows["c2_attention"] = row_attention(xb, hbm, tf_burst, tf_sust)
             xb.keep = None
             torch.cuda.empty_cache()
+        if "c3" in want:
             rows["c3_temporal"] = row_temporal(dev, hbm)
             torch.cuda.empty_cache()
+        if "c4" in want:
             rows["c4_cluster"] = row_cluster(dev, hbm, tf_burst)
+        rows = rows or None
         if not args.no_cpu:
             cpu = oracle_xlayer_rate(xb.wl, 192, L_RUN, 20.0)
 
