@@ -261,9 +261,13 @@ kvc_status codec_common(const kvc_layer_desc* d, const kvc_predictor* p, bool en
   const size_t need = kvc_workspace_bytes(op, d, p, 0);
   if (ws_bytes < need || (need && !ws)) return KVC_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = (cudaStream_t)stream;
-  // tensor-core path for the bf16, D = 128 cross-layer / anchor codec
+  // tensor-core paths for bf16, D = 128
   if (tc_codec_supported(d, p)) {
     cudaError_t e = tc_codec_layer(d, p, enc, K, V, Ks, Vs, c, Kr, Vr, ws, ws_bytes, st);
+    return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+  }
+  if (tc_temporal_supported(d, p)) {
+    cudaError_t e = tc_temporal_layer(d, p, enc, K, V, Ks, Vs, c, Kr, Vr, st);
     return e == cudaSuccess ? KVC_OK : cuda_fail(e);
   }
   Carve cv{(char*)ws, ws_bytes};

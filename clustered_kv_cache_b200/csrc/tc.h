@@ -10,6 +10,9 @@ size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int
 cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
                            const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, void* ws,
                            size_t ws_bytes, cudaStream_t st);
+bool tc_temporal_supported(const kvc_layer_desc* d, const kvc_predictor* p);
+cudaError_t tc_temporal_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
+                              const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, cudaStream_t st);
 bool tc_attend_supported(const kvc_layer_desc* d, const kvc_predictor* p, int64_t n_self);
 size_t tc_attend_workspace(const kvc_layer_desc* d, const kvc_predictor* p);
 cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
