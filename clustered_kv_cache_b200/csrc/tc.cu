@@ -67,6 +67,9 @@ struct Maps {
   CUtensorMap wk, wv;  // [r][C], [r][2C]
   CUtensorMap bk, bv;  // [H*128][128], [H*128][256]
   CUtensorMap uk, uv;  // [C][r]
+  // L2 prefetch only: clean inputs [T][C] (encode), codes [T][H*row_bytes] and
+  // params [T][H*16] as bytes (decode)
+  CUtensorMap xk, xv, ck, cv, pk, pv;
 };
 
 struct Args {
@@ -195,7 +198,21 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       if (RC) {
         for (int c = 0; c < NCH; ++c) load(&maps.ks, c * 64, pol_keep, &maps.wk, c * 64, 0, wbytes);
       }
+      // the epilogue of head h reads its clean inputs (encode) or codes (decode) from
+      // global memory: bring them into L2 while the head's operands stream in
+      const int rbytes = 128 * a.bits / 8;
+      auto prefetch_head = [&](bool is_v, int h) {
+        if (ENC) {
+          const CUtensorMap* m = is_v ? &maps.xv : &maps.xk;
+          tma_prefetch(m, h * 128, t0);
+          tma_prefetch(m, h * 128 + 64, t0);
+        } else if (!LAT || !is_v) {
+          tma_prefetch(is_v ? &maps.cv : &maps.ck, h * rbytes, t0);
+          if (G == 32) tma_prefetch(is_v ? &maps.pv : &maps.pk, h * 16, t0);
+        }
+      };
       for (int h = 0; h < H && ok; ++h) {
+        prefetch_head(false, h);
         for (int j = 0; j < 2; ++j) load(&maps.ks, h * 128 + j * 64, pol_stream, &maps.bk, j * 64, h * 128, 16384);
         for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, &maps.uk, j * 64, h * 128, 16384);
         if (RC && h >= 1)
@@ -210,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         if (ok && !wait(khat_stored, 0, abort_flag, a.err, 0x200u)) ok = false;
         if (ok) fence_async_global();
         for (int h = 0; h < H && ok; ++h) {
+          prefetch_head(true, h);
           for (int j = 0; j < 2; ++j)
             load(&maps.ko, h * 128 + j * 64, pol_stream, &maps.bv, j * 64, h * 128, 16384);
           for (int j = 0; j < 2; ++j)
@@ -556,6 +574,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// 2-D byte tensor [rows][cols] for L2 prefetches of box_rows x box_cols bytes.
+bool map2d_bytes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                 uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 tensor [rows][cols] (row-major) read or written in boxes of
 // box_rows x 64 columns with the 128-byte swizzle.
 bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -622,6 +654,13 @@ cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool
   if (ok && r > 0)
     ok = tc::map2d(&m.wk, p->k_w, r, C, (uint32_t)r) && tc::map2d(&m.wv, p->v_w, r, 2 * C, (uint32_t)r) &&
          tc::map2d(&m.uk, p->k_u, C, r, 128) && tc::map2d(&m.uv, p->v_u, C, r, 128);
+  const uint64_t rb = 128 * (uint64_t)d->bits / 8;
+  if (ok && enc) ok = tc::map2d(&m.xk, K, T, C, 128) && tc::map2d(&m.xv, V, T, C, 128);
+  if (ok && !enc)
+    ok = tc::map2d_bytes(&m.ck, c->k_codes, T, H * rb, (uint32_t)rb, 128) &&
+         tc::map2d_bytes(&m.cv, c->v_codes, T, H * rb, (uint32_t)rb, 128) &&
+         (d->group != 32 || (tc::map2d_bytes(&m.pk, c->k_params, T, H * 16, 16, 128) &&
+                             tc::map2d_bytes(&m.pv, c->v_params, T, H * 16, 16, 128)));
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
@@ -640,11 +679,13 @@ cudaError_t latent_layer(const kvc_layer_desc* d, const kvc_predictor* p, const 
   const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128, r = p->rank;
   Maps m;
   memset(&m, 0, sizeof(m));
+  const uint64_t rb = 128 * (uint64_t)d->bits / 8;
   bool ok = map2d(&m.ks, Ks, T, C, 128) && map2d(&m.vs, Vs, T, C, 128) && map2d(&m.ko, Ks, T, C, 128) &&
             map2d(&m.vo, Ks, T, C, 128) && map2d(&m.bk, p->k_block, H * 128, 128, 128) &&
             map2d(&m.bv, p->v_block, H * 128, 256, 128) && map2d(&m.wk, p->k_w, r, C, (uint32_t)r) &&
             map2d(&m.wv, p->v_w, r, 2 * C, (uint32_t)r) && map2d(&m.uk, p->k_u, C, r, 128) &&
-            map2d(&m.uv, p->v_u, C, r, 128);
+            map2d(&m.uv, p->v_u, C, r, 128) && map2d_bytes(&m.ck, c->k_codes, T, H * rb, (uint32_t)rb, 128) &&
+            (d->group != 32 || map2d_bytes(&m.pk, c->k_params, T, H * 16, 16, 128));
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;

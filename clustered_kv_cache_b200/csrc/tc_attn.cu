@@ -27,6 +27,8 @@ namespace kvc {
 namespace tc {
 
 bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool map2d_bytes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                 uint32_t box_rows);
 
 namespace attn {
 
@@ -49,6 +51,7 @@ struct Maps {
   CUtensorMap bk, bv;        // [H*128][128], [H*128][256]
   CUtensorMap uk, uv;        // [C][r]
   CUtensorMap zkh, zkl, zvh, zvl;  // latents [T][r]
+  CUtensorMap ck, cv, pk, pv;      // codes / params as bytes, for L2 prefetches
 };
 
 struct Args {
@@ -186,6 +189,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
         const int b = j & 1;
         if (j < NH) {
           const int t0 = j * 128;
+          const int rbytes = 128 * a.bits / 8;
+          tma_prefetch(&maps.ck, h * rbytes, t0);
+          tma_prefetch(&maps.cv, h * rbytes, t0);
+          if (a.group == 32) {
+            tma_prefetch(&maps.pk, h * 16, t0);
+            tma_prefetch(&maps.pv, h * 16, t0);
+          }
           // decode K: K^_{l-1,h} B_h^T + [Z_K hi | lo] U_h^T
           for (int c = 0; c < 2; ++c) load(&maps.ks, h * 128 + c * 64, t0, &maps.bk, c * 64, h * 128);
           for (int c = 0; c < RC; ++c) {
@@ -543,6 +553,12 @@ cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const voi
     ok = tc::map2d(&m.uk, p->k_u, C, r, 128) && tc::map2d(&m.uv, p->v_u, C, r, 128) &&
          tc::map2d(&m.zkh, zkh, T, r, 128) && tc::map2d(&m.zkl, zkl, T, r, 128) &&
          tc::map2d(&m.zvh, zvh, T, r, 128) && tc::map2d(&m.zvl, zvl, T, r, 128);
+  const uint64_t rb = 128 * (uint64_t)d->bits / 8;
+  if (ok && T > 0)
+    ok = tc::map2d_bytes(&m.ck, c->k_codes, T, H * rb, (uint32_t)rb, 128) &&
+         tc::map2d_bytes(&m.cv, c->v_codes, T, H * rb, (uint32_t)rb, 128) &&
+         (d->group != 32 || (tc::map2d_bytes(&m.pk, c->k_params, T, H * 16, 16, 128) &&
+                             tc::map2d_bytes(&m.pv, c->v_params, T, H * 16, 16, 128)));
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
