@@ -1,27 +1,30 @@
 // Tensor-core kernels (tcgen05 + TMEM + TMA) of the bf16 / head_dim 128 hot path.
 //
-// Cross-layer block-DPLR codec, one CTA per 128-token tile, all heads fused
-// ("CORAL-KV: Compact Cross-Layer Prediction and Residual Coding for
-// Autoregressive Video KV Caches", Fig. 3: K_l from the reconstructed K_{l-1};
-// V_l from the reconstructed [K_l, V_{l-1}]; block-diagonal per-head maps plus
-// a global rank-r term).  Per tile:
+// Cross-layer block-DPLR codec, persistent CTAs (one per SM) looping over
+// 128-token tiles, all heads fused ("CORAL-KV: Compact Cross-Layer Prediction
+// and Residual Coding for Autoregressive Video KV Caches", Fig. 3: K_l from the
+// reconstructed K_{l-1}; V_l from the reconstructed [K_l, V_{l-1}];
+// block-diagonal per-head maps plus a global rank-r term).  Per tile:
 //
-//   Z_K  = K^_{l-1} W_K^T                         (TMEM, 24 chunks of 64 channels)
+//   Z_K  = K^_{l-1} W_K^T                         (TMEM, 64-channel chunks)
 //   for each head h (K):  acc = K^_{l-1,h} B_h^T + [Z_K hi | lo] U_h^T
 //        epilogue: residual, group min/max, fp16 (scale, zero), codes, packing,
 //        reconstruction K^_{l,h} -> shared memory -> TMA store, and
 //        Z_V += K^_{l,h} W_V[:, h]^T (the V latent grows head by head)
-//   Z_V += V^_{l-1} W_V[:, C:]^T
+//        Z_V += V^_{l-1,h} W_V[:, C + h]^T (the other half, interleaved)
 //   for each head h (V):  acc = [K^_{l,h} | V^_{l-1,h}] BV_h^T + [Z_V hi | lo] UV_h^T
 //        epilogue as above, writing V^_{l,h}
 //
+// The latent GEMMs are spread over the head loops so the tensor pipe and the
+// epilogue warps stay busy while the latent's operands stream in; at rank 64
+// the next tile's Z_K is accumulated in a second TMEM slot during the V heads.
 // The latent is carried to the second factor as a pair of bf16 values whose
 // sum is within 2^-16 of the fp32 accumulator, so no rounding decision is taken
 // on it.  Warp roles: warp 0 issues TMA loads, warp 1 allocates TMEM and one
-// thread issues every tcgen05.mma, warps 2..9 run the epilogue (two warps per
-// TMEM lane quarter, 64 columns each).  Every wait is bounded: a wait that runs
-// out records an error word, raises an abort flag seen by all roles, and the
-// CTA drains what it issued and returns.
+// thread issues every tcgen05.mma, warps 2..9 run the epilogue as two groups of
+// four warps (one TMEM lane quarter each) taking alternate heads.  Every wait is
+// bounded: a wait that runs out records an error word, raises an abort flag
+// seen by all roles, and the CTA drains what it issued and returns.
 #include <cuda.h>
 #include <string.h>
 
@@ -54,7 +57,8 @@ cudaError_t tc_read_and_clear_error(unsigned int* value) {
 
 namespace tc {
 
-constexpr int kThreads = 320;     // 10 warps: producer, MMA, two epilogue groups of 4
+constexpr int kThreads = 352;     // 11 warps: producer, MMA, two epilogue groups of 4, MMA sync
+constexpr int kSyncWarp = 10;
 constexpr int kGroupThreads = 128;
 
 enum Mode { kEncode = 0, kDecode = 1, kLatent = 2 };
@@ -101,7 +105,7 @@ struct Layout {
 
 // ---------------------------------------------------------------- the kernel
 
-template <int MODE, int G, int RC>
+template <int MODE, int G, int RC, int BITS>
 __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_constant__ Maps maps, const Args a) {
   constexpr bool ENC = MODE == kEncode;
   constexpr bool LAT = MODE == kLatent;
@@ -129,7 +133,14 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   const int H = a.H;
   const int C = H * 128;
   const int NCH = C / 64;
-  const int t0 = blockIdx.x * 128;
+  // persistent CTAs: this CTA codes tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int ntiles = (int)((a.T + 127) / 128);
+  const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto tile_t0 = [&](int it) { return ((int)blockIdx.x + it * (int)gridDim.x) * 128; };
+  // With rank 64 the TMEM has room for two latent slots, so the next tile's K
+  // latent streams in during this tile's V heads.
+  constexpr bool OVL = RC == 1 && !LAT;
+  const int HH = 2 * H;  // heads per tile (K then V)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -159,6 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // TMEM columns: accumulators [0,128) and [128,256); latent slot k of Z_K / Z_V
+  auto zk_col = [&](int it) { return tmem + 256 + (OVL ? (it & 1) * 128 : 0); };
+  auto zv_col = [&](int it) { return tmem + 256 + (OVL ? (it & 1) * 128 + 64 : R); };
 
   auto stageA = [&](int s) { return smem + L::kStageOff + s * L::kStage; };
   auto stageB = [&](int s) { return smem + L::kStageOff + s * L::kStage + 16384; };
@@ -177,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       uint32_t issued_ph[S];  // ... in this phase of full[i]
       for (int i = 0; i < S; ++i) issued[i] = 0, issued_ph[i] = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap* ma, int ax, uint64_t pa, const CUtensorMap* mb, int bx, int by,
+      auto load = [&](const CUtensorMap* ma, int ax, int ay, uint64_t pa, const CUtensorMap* mb, int bx, int by,
                       uint32_t bbytes) {
         if (!ok) return;
         if (!wait(&empty[s], ph ^ 1, abort_flag, a.err, 0x100u + s)) {
@@ -185,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           return;
         }
         mbar_arrive_expect_tx(&full[s], (ma ? 16384u : 0u) + bbytes);
-        if (ma) tma_load(stageA(s), ma, ax, t0, &full[s], pa);
+        if (ma) tma_load(stageA(s), ma, ax, ay, &full[s], pa);
         tma_load(stageB(s), mb, bx, by, &full[s], pol_keep);
         issued[s] = 1;
         issued_ph[s] = ph;
@@ -195,44 +209,54 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         }
       };
       const uint32_t wbytes = R * 128;
-      if (RC) {
-        for (int c = 0; c < NCH; ++c) load(&maps.ks, c * 64, pol_keep, &maps.wk, c * 64, 0, wbytes);
-      }
-      // the epilogue of head h reads its clean inputs (encode) or codes (decode) from
-      // global memory: bring them into L2 while the head's operands stream in
-      const int rbytes = 128 * a.bits / 8;
-      auto prefetch_head = [&](bool is_v, int h) {
-        if (ENC) {
-          const CUtensorMap* m = is_v ? &maps.xv : &maps.xk;
-          tma_prefetch(m, h * 128, t0);
-          tma_prefetch(m, h * 128 + 64, t0);
-        } else if (!LAT || !is_v) {
-          tma_prefetch(is_v ? &maps.cv : &maps.ck, h * rbytes, t0);
-          if (G == 32) tma_prefetch(is_v ? &maps.pv : &maps.pk, h * 16, t0);
-        }
-      };
-      for (int h = 0; h < H && ok; ++h) {
-        prefetch_head(false, h);
-        for (int j = 0; j < 2; ++j) load(&maps.ks, h * 128 + j * 64, pol_stream, &maps.bk, j * 64, h * 128, 16384);
-        for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, &maps.uk, j * 64, h * 128, 16384);
-        if (RC && h >= 1)
-          for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, &maps.wv, (h - 1) * 128 + j * 64, 0, wbytes);
-      }
-      if (RC) {
-        for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, &maps.wv, (H - 1) * 128 + j * 64, 0, wbytes);
-        for (int c = 0; c < NCH; ++c) load(&maps.vs, c * 64, LAT ? pol_stream : pol_keep, &maps.wv, C + c * 64, 0,
-                                           wbytes);
-      }
-      if (!LAT) {
-        if (ok && !wait(khat_stored, 0, abort_flag, a.err, 0x200u)) ok = false;
-        if (ok) fence_async_global();
+      constexpr int rbytes = 128 * BITS / 8;
+      for (int it = 0; it < my_tiles && ok; ++it) {
+        const int t0 = tile_t0(it);
+        const int nt0 = it + 1 < my_tiles ? tile_t0(it + 1) : -1;
+        // the epilogue of head h reads its clean inputs (encode) or codes (decode)
+        // from global memory: bring them into L2 as the head's operands stream in
+        auto prefetch_head = [&](bool is_v, int h) {
+          if (ENC) {
+            const CUtensorMap* m = is_v ? &maps.xv : &maps.xk;
+            tma_prefetch(m, h * 128, t0);
+            tma_prefetch(m, h * 128 + 64, t0);
+          } else if (!LAT || !is_v) {
+            tma_prefetch(is_v ? &maps.cv : &maps.ck, h * rbytes, t0);
+            if (G == 32) tma_prefetch(is_v ? &maps.pv : &maps.pk, h * 16, t0);
+          }
+        };
+        if (RC && (!OVL || it == 0))
+          for (int c = 0; c < NCH; ++c) load(&maps.ks, c * 64, t0, pol_keep, &maps.wk, c * 64, 0, wbytes);
         for (int h = 0; h < H && ok; ++h) {
-          prefetch_head(true, h);
+          prefetch_head(false, h);
           for (int j = 0; j < 2; ++j)
-            load(&maps.ko, h * 128 + j * 64, pol_stream, &maps.bv, j * 64, h * 128, 16384);
-          for (int j = 0; j < 2; ++j)
-            load(&maps.vs, h * 128 + j * 64, pol_stream, &maps.bv, 128 + j * 64, h * 128, 16384);
-          for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, &maps.uv, j * 64, h * 128, 16384);
+            load(&maps.ks, h * 128 + j * 64, t0, pol_stream, &maps.bk, j * 64, h * 128, 16384);
+          for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, 0, &maps.uk, j * 64, h * 128, 16384);
+          if (RC && h >= 2)
+            for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, 0, &maps.wv, (h - 2) * 128 + j * 64, 0, wbytes);
+          if (RC)  // the V latent's V^_{l-1} half, interleaved with the K heads
+            for (int c = 2 * h; c < 2 * h + 2; ++c)
+              load(&maps.vs, c * 64, t0, LAT ? pol_stream : pol_keep, &maps.wv, C + c * 64, 0, wbytes);
+        }
+        if (RC)
+          for (int g = H >= 2 ? H - 2 : 0; g < H; ++g)
+            for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, 0, &maps.wv, g * 128 + j * 64, 0, wbytes);
+        if (!LAT) {
+          for (int h = 0; h < H && ok; ++h) {
+            prefetch_head(true, h);
+            for (int j = 0; j < 2; ++j)
+              load(&maps.vs, h * 128 + j * 64, t0, pol_stream, &maps.bv, 128 + j * 64, h * 128, 16384);
+            if (h == 0) {  // K^_l is read back once both epilogue groups have stored it
+              if (ok && !wait(khat_stored, it & 1, abort_flag, a.err, 0x200u)) ok = false;
+              if (ok) fence_async_global();
+            }
+            for (int j = 0; j < 2; ++j)
+              load(&maps.ko, h * 128 + j * 64, t0, pol_stream, &maps.bv, j * 64, h * 128, 16384);
+            for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, 0, &maps.uv, j * 64, h * 128, 16384);
+            if (OVL && nt0 >= 0)  // the next tile's K latent, interleaved with the V heads
+              for (int c = 2 * h; c < 2 * h + 2; ++c)
+                load(&maps.ks, c * 64, nt0, pol_keep, &maps.wk, c * 64, 0, wbytes);
+          }
         }
       }
       if (!ok) {
@@ -245,116 +269,167 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         }
       }
     }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
+  } else if (warp == 1 || warp == kSyncWarp) {
+    // ================================================================ MMA issue and its waits
+    // The MMA schedule is walked by two warps in lock step.  The sync warp waits
+    // on every mbarrier a group of chunks needs (operands landed, accumulator
+    // drained, latent converted ...) and hands the group to the MMA warp through
+    // named barrier 3; the MMA warp, converged, issues the group's MMAs and
+    // commits from one lane.  The MMA warp never polls shared memory: a poll
+    // from the issuing warp waits for that warp's in-flight MMA operand reads,
+    // which leaves the tensor pipe idle between chunks.
+    auto walk = [&](auto issue_tag) {
+      constexpr bool ISSUE = decltype(issue_tag)::value;
+      const uint32_t lead = lane == 0;
       const uint32_t acc_col[2] = {tmem, tmem + 128};
-      const uint32_t zk_col = tmem + 256, zv_col = tmem + 256 + R;
       int s = 0;
       uint32_t ph = 0;
-      bool ok = true;
-      int use[2] = {0, 0};
-      // one 64-wide K chunk: A from the stage (resA == 0) or resident smem
-      auto chunk = [&](uint32_t d, int N, bool first, const uint8_t* resA, const uint8_t* resA2) {
-        if (!ok) return;
-        if (!wait(&full[s], ph, abort_flag, a.err, 0x300u + s)) {
-          ok = false;
-          return;
-        }
-        tc_fence_after();
+      int use[2] = {0, 0};   // uses of each accumulator
+      int recf[2] = {0, 0};  // rec_full completions consumed per reconstruction tile
+      int zr = 0;            // z_ready completions consumed
+      auto wt = [&](uint64_t* bar, uint32_t parity, unsigned where) {
+        if (!ISSUE && lane == 0) wait(bar, parity, abort_flag, a.err, where);
+      };
+      auto commit = [&](uint64_t* bar) {
+        if (ISSUE) umma_commit_if(lead, bar);
+      };
+      // one 64-wide K chunk from stage st: A from the stage (resA == 0) or resident smem
+      auto issue = [&](int st, uint32_t d, int N, bool first, const uint8_t* resA, const uint8_t* resA2) {
+        if (!ISSUE) return;
         const uint32_t idesc = idesc_bf16(128, N);
-        const uint64_t bd = desc_sw128(smem_u32(stageB(s)));
-        const uint64_t ad = desc_sw128(smem_u32(resA ? resA : stageA(s)));
+        const uint64_t bd = desc_sw128(smem_u32(stageB(st)));
+        const uint64_t ad = desc_sw128(smem_u32(resA ? resA : stageA(st)));
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma(d, ad + 2 * k, bd + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
+        for (int k = 0; k < 4; ++k) umma_if(lead, d, ad + 2 * k, bd + 2 * k, idesc, (first && k == 0) ? 0u : 1u);
         if (resA2) {
           const uint64_t ad2 = desc_sw128(smem_u32(resA2));
 #pragma unroll
-          for (int k = 0; k < 4; ++k) umma(d, ad2 + 2 * k, bd + 2 * k, idesc, 1u);
-        }
-        umma_commit(&empty[s]);
-        if (++s == S) {
-          s = 0;
-          ph ^= 1;
+          for (int k = 0; k < 4; ++k) umma_if(lead, d, ad2 + 2 * k, bd + 2 * k, idesc, 1u);
         }
       };
-      auto acc_acquire = [&](int b) {
-        if (ok && use[b] >= 1) {
-          if (!wait(&acc_empty[b], (use[b] - 1) & 1, abort_flag, a.err, 0x400u + b)) ok = false;
-          tc_fence_after();
-        }
-      };
-      auto zva = [&](int g) {  // Z_V += K^_{l,g} W_V[:, g]^T from the reconstruction tile
-        const int rb = g & 1;
-        if (ok && !wait(&rec_full[rb], (g >> 1) & 1, abort_flag, a.err, 0x500u + rb)) ok = false;
-        tc_fence_after();
-        for (int j = 0; j < 2; ++j) chunk(zv_col, R, g == 0 && j == 0, recon(rb) + j * 16384, nullptr);
-        if (ok) umma_commit(&rec_free[rb]);
-      };
-      if (RC) {
-        for (int c = 0; c < NCH; ++c) chunk(zk_col, R, c == 0, nullptr, nullptr);
-        if (ok) umma_commit(zk_full);
-      }
-      for (int h = 0; h < H && ok; ++h) {
-        const int b = h & 1;
-        acc_acquire(b);
-        for (int j = 0; j < 2; ++j) chunk(acc_col[b], 128, j == 0, nullptr, nullptr);
-        if (RC) {
-          if (h == 0 && ok) {
-            if (!wait(z_ready, 0, abort_flag, a.err, 0x600u)) ok = false;
-            tc_fence_after();
-          }
-          for (int j = 0; j < RC; ++j) chunk(acc_col[b], 128, false, zhi(j), zlo(j));
-        }
-        if (ok) umma_commit(&acc_full[b]);
-        use[b]++;
-        if (RC && h >= 1) zva(h - 1);
-      }
-      if (RC) {
-        zva(H - 1);
-        for (int c = 0; c < NCH; ++c) chunk(zv_col, R, false, nullptr, nullptr);
-        if (ok) umma_commit(zv_full);
-      }
-      if (!LAT) {
-        for (int h = 0; h < H && ok; ++h) {
-          const int b = (H + h) & 1;
-          acc_acquire(b);
-          for (int j = 0; j < 4; ++j) chunk(acc_col[b], 128, j == 0, nullptr, nullptr);
-          if (RC) {
-            if (h == 0 && ok) {
-              if (!wait(z_ready, 1, abort_flag, a.err, 0x601u)) ok = false;
-              tc_fence_after();
+      // n chunks from the next n stages, after the waits in pre(): one hand-off
+      auto group = [&](int n, auto&& pre, auto&& body) {
+        if (!ISSUE) {
+          pre();
+          int ss = s;
+          uint32_t pp = ph;
+          for (int i = 0; i < n; ++i) {
+            wt(&full[ss], pp, 0x300u + ss);
+            if (++ss == S) {
+              ss = 0;
+              pp ^= 1;
             }
-            for (int j = 0; j < RC; ++j) chunk(acc_col[b], 128, false, zhi(j), zlo(j));
           }
-          if (ok) umma_commit(&acc_full[b]);
+          __syncwarp();
+        }
+        asm volatile("bar.sync 3, 64;" ::: "memory");
+        if (ISSUE) tc_fence_after();
+        for (int i = 0; i < n; ++i) {
+          body(i, s);
+          commit(&empty[s]);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      };
+      auto nop = [] {};
+      auto acq = [&](int b) {
+        if (use[b] >= 1) wt(&acc_empty[b], (use[b] - 1) & 1, 0x400u + b);
+      };
+      for (int it = 0; it < my_tiles; ++it) {
+        const uint32_t zk = zk_col(it), zv = zv_col(it);
+        const bool has_next = it + 1 < my_tiles;
+        if (RC && (!OVL || it == 0)) {
+          for (int c = 0; c < NCH; c += 2)
+            group(2, nop, [&](int i, int st) { issue(st, zk, R, c + i == 0, nullptr, nullptr); });
+          commit(zk_full);
+        }
+        // Z_V += K^_{l,g} W_V[:, g]^T from the reconstruction tile of K head g
+        auto zva = [&](int g) {
+          const int rb = (it * HH + g) & 1;
+          group(
+              2, [&] { wt(&rec_full[rb], recf[rb] & 1, 0x500u + rb); },
+              [&](int i, int st) { issue(st, zv, R, false, recon(rb) + i * 16384, nullptr); });
+          recf[rb]++;
+          commit(&rec_free[rb]);
+        };
+        // the latent factor of a head: acc += [Z hi | Z lo] U^T
+        auto lowrank = [&](int b, bool first_head, unsigned where) {
+          group(
+              RC, [&] { if (first_head) wt(z_ready, zr & 1, where); },
+              [&](int i, int st) { issue(st, acc_col[b], 128, false, zhi(i), zlo(i)); });
+          if (first_head) zr++;
+        };
+        for (int h = 0; h < H; ++h) {
+          const int b = (it * HH + h) & 1;
+          group(2, [&] { acq(b); }, [&](int i, int st) { issue(st, acc_col[b], 128, i == 0, nullptr, nullptr); });
+          if (RC) lowrank(b, h == 0, 0x600u);
+          commit(&acc_full[b]);
           use[b]++;
+          // two heads behind, so that the epilogue of head h-2 is long done
+          if (RC && h >= 2) zva(h - 2);
+          if (RC)  // V^_{l-1} half of the V latent; its first chunk initialises Z_V
+            group(2, nop, [&](int i, int st) { issue(st, zv, R, 2 * h + i == 0, nullptr, nullptr); });
+        }
+        if (RC) {
+          for (int g = H >= 2 ? H - 2 : 0; g < H; ++g) zva(g);
+          commit(zv_full);
+        }
+        if (!LAT) {
+          for (int h = 0; h < H; ++h) {
+            const int b = (it * HH + H + h) & 1;
+            // V^_{l-1,h} part first (chunks 2, 3 of BV_h), then K^_{l,h} (chunks 0, 1)
+            group(2, [&] { acq(b); }, [&](int i, int st) { issue(st, acc_col[b], 128, i == 0, nullptr, nullptr); });
+            group(2, nop, [&](int i, int st) { issue(st, acc_col[b], 128, false, nullptr, nullptr); });
+            if (RC) lowrank(b, h == 0, 0x601u);
+            commit(&acc_full[b]);
+            use[b]++;
+            if (OVL && has_next)
+              group(2, nop, [&](int i, int st) { issue(st, zk_col(it + 1), R, 2 * h + i == 0, nullptr, nullptr); });
+          }
+          if (OVL && has_next) commit(zk_full);
         }
       }
-      // every issued MMA completes before TMEM is released
-      umma_commit(mma_done);
-      const long long w0 = clock64();
-      while (!mbar_test(mma_done, 0) && clock64() - w0 < kWaitBudget) {
+      if (ISSUE) {
+        // every issued MMA completes before TMEM is released
+        commit(mma_done);
+        if (lane == 0) {
+          const long long w0 = clock64();
+          while (!mbar_test(mma_done, 0) && clock64() - w0 < kWaitBudget) {
+          }
+        }
+        __syncwarp();
       }
-    }
+    };
+    if (warp == 1)
+      walk(Tag<true>{});
+    else
+      walk(Tag<false>{});
   } else {
     // ================================================================ epilogue: two groups of 4 warps
     // Group g owns TMEM accumulator g and reconstruction tile g, i.e. the heads
-    // u (K heads u = h, V heads u = H + h) with u % 2 == g; each warp of a group
-    // covers one TMEM lane quarter (32 tokens) and all 128 channels.
+    // whose running index (over tiles, K heads then V heads) is congruent to g
+    // mod 2; each warp of a group covers one TMEM lane quarter (32 tokens) and
+    // all 128 channels.
     const int grp = (warp - 2) >> 2;
     const int ew = (warp - 2) & 3;
     const int q = warp & 3;  // TMEM lane quarter of this warp
     const int row = q * 32 + lane;
-    const int64_t t = (int64_t)t0 + row;
-    const bool valid = t < a.T;
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
     const bool elected = ew == 0 && lane == 0;
-    const int bits = a.bits;
-    const int levels = (1 << bits) - 1;
-    constexpr int NG = 128 / G;  // groups in a row
-    constexpr int NP = G / 32;   // 32-column passes per group
-    int use = 0;
+    constexpr int LEVELS = (1 << BITS) - 1;
+    constexpr int NG = 128 / G;          // groups in a row
+    constexpr int NP = G / 32;           // 32-column passes per group
+    constexpr int RB = 128 * BITS / 8;   // code bytes of a row
+    constexpr int GW = G * BITS / 32;    // code words of a group
+    constexpr int XQ = G / 8;            // 16-byte words of x in a group
+    constexpr bool KEEP = ENC && NP == 1;  // encode of a one-pass group keeps its prediction
+    constexpr uint32_t kBias8 = grid_pack_bias(BITS, 8);
+    int use = 0;                 // uses of this group's accumulator
+    int recfree = 0;             // rec_free completions consumed
+    bool prev_k = false;         // the previous use of this group's tile fed Z_V
+    int zk_use = 0, zv_use = 0;
     auto gsync = [&]() {
       if (grp == 0)
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -362,11 +437,13 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         asm volatile("bar.sync 2, 128;" ::: "memory");
     };
 
-    auto convert_latent = [&](uint32_t col, __nv_bfloat16* ghi, __nv_bfloat16* glo) {  // TMEM -> bf16 hi / lo
+    auto convert_latent = [&](uint32_t col, int t0, __nv_bfloat16* ghi, __nv_bfloat16* glo) {  // TMEM -> bf16 hi / lo
+      const int64_t t = (int64_t)t0 + row;
+      const bool valid = t < a.T;
       for (int p = 0; p < R / 32; ++p) {
         const int c0 = p * 32;  // latent column
         float v[32];
-        tmem_ld32(lane_addr + col + c0, v);
+        tmem_ld32(lane_addr + (col - tmem) + c0, v);
         uint8_t* hi = zhi(c0 / 64);
         uint8_t* lo = zlo(c0 / 64);
 #pragma unroll
@@ -394,117 +471,151 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       mbar_arrive(z_ready);
     };
 
-    // one head of this group: u = global head index (K: h, V: H + h)
-    auto head = [&](int u, int h, bool is_v) {
-      const int b = grp;  // == u & 1
-      const int row_bytes = 128 * bits / 8;
+    // one head of this group: h its index, is_v K or V, t0 the tile.  The
+    // groups of the row are processed by a rolled loop (the kernel's code must
+    // stay small enough for the instruction caches); the global inputs of group
+    // g+1 are fetched while group g is worked on.
+    auto head = [&](int h, bool is_v, int t0) {
+      const int b = grp;
+      const int64_t t = (int64_t)t0 + row;
+      const bool valid = t < a.T;
       const int64_t rowi = t * H + h;
-      uint8_t* codes = (is_v ? a.vcodes : a.kcodes) + rowi * row_bytes;
-      __half2* params = (is_v ? a.vparams : a.kparams) + rowi * (128 / G);
-      // inputs of this thread's row, fetched before the accumulator is ready
-      uint4 xin[16];
-      uint4 cin[4];
-      __half2 pin[NG];
-      if (ENC) {
-        const __nv_bfloat16* X = (is_v ? a.xv : a.xk) + t * C + h * 128;
+      uint32_t* codes = reinterpret_cast<uint32_t*>((is_v ? a.vcodes : a.kcodes) + rowi * RB);
+      __half2* params = (is_v ? a.vparams : a.kparams) + rowi * NG;
+      const uint4* X = reinterpret_cast<const uint4*>((is_v ? a.xv : a.xk) + t * C + h * 128);
+      // inputs of the current group: x (encode) or code words and (scale, zero)
+      uint4 xc[ENC ? XQ : 1];
+      uint32_t cc[ENC ? 1 : GW];
+      __half2 pc = __floats2half2_rn(0.f, 0.f);
+      auto fetch = [&](int g, uint4 (&xo)[ENC ? XQ : 1], uint32_t (&co)[ENC ? 1 : GW], __half2& po) {
+        if (ENC) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          xin[i] = valid ? __ldcs(reinterpret_cast<const uint4*>(X) + i) : make_uint4(0, 0, 0, 0);
-      } else {
+          for (int i = 0; i < XQ; ++i) xo[i] = valid ? __ldcs(X + g * XQ + i) : make_uint4(0, 0, 0, 0);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          cin[i] = (valid && i < bits) ? __ldcs(reinterpret_cast<const uint4*>(codes) + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int g = 0; g < NG; ++g) pin[g] = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
-      }
+          for (int i = 0; i < GW; i += 2) {
+            const uint2 w = valid ? __ldcs(reinterpret_cast<const uint2*>(codes + g * GW + i)) : make_uint2(0, 0);
+            co[i] = w.x;
+            co[i + 1] = w.y;
+          }
+          po = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
+        }
+      };
+      fetch(0, xc, cc, pc);
       // the reconstruction tile is free once its previous TMA store has read it
-      // and (cross-layer K heads) the MMA of Z_V has consumed it
+      // and, if it held a K head, the MMA of Z_V has consumed it
       if (elected) bulk_wait_read0();
       gsync();
-      if (RC && u >= 2 && u - 2 <= H - 1) wait(&rec_free[b], ((u - 2) >> 1) & 1, abort_flag, a.err, 0x700u + b);
       wait(&acc_full[b], use & 1, abort_flag, a.err, 0x800u + b);
       use++;
+      if (RC && prev_k) wait(&rec_free[b], recfree++ & 1, abort_flag, a.err, 0x700u + b);
+      prev_k = !is_v && RC;
       tc_fence_after();
-      uint32_t cw[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};  // packed codes of the row
-      const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
-#pragma unroll
+      const uint32_t acc = lane_addr + b * 128;
+#pragma unroll 1
       for (int g = 0; g < NG; ++g) {
+        uint4 xn[ENC ? XQ : 1];
+        uint32_t cn[ENC ? 1 : GW];
+        __half2 pn = pc;
+        if (g + 1 < NG) fetch(g + 1, xn, cn, pn);
+        float pk[KEEP ? 32 : 1];  // prediction of a one-pass group, kept for the second pass
         float sf, zf;
         if (ENC) {
           // group min / max of the residual over its NP passes of 32 columns
-          float mn = INFINITY, mx = -INFINITY;
+          float mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY;
 #pragma unroll
-          for (int pc = 0; pc < NP; ++pc) {
+          for (int q = 0; q < NP; ++q) {
             float p[32];
-            tmem_ld32(lane_addr + b * 128 + g * G + pc * 32, p);
+            tmem_ld32(acc + g * G + q * 32, p);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
               float x[8];
-              unpack_bf16x8(xin[(g * G + pc * 32) / 8 + ch], x, 0);
+              unpack_bf16x8(xc[q * 4 + ch], x, 0);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float r = x[i] - p[ch * 8 + i];
-                mn = fminf(mn, r);
-                mx = fmaxf(mx, r);
+              for (int i = 0; i < 8; i += 2) {
+                const float r0 = x[i] - p[ch * 8 + i], r1 = x[i + 1] - p[ch * 8 + i + 1];
+                mn0 = fminf(mn0, r0);
+                mx0 = fmaxf(mx0, r0);
+                mn1 = fminf(mn1, r1);
+                mx1 = fmaxf(mx1, r1);
               }
             }
+            if (KEEP) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) pk[i] = p[i];
+            }
           }
-          const __half sh = __float2half_rn((mx - mn) / (float)levels);
+          const float mn = fminf(mn0, mn1), mx = fmaxf(mx0, mx1);
+          const __half sh = __float2half_rn((mx - mn) / (float)LEVELS);
           const __half zh = __float2half_rn(mn);
           sf = __half2float(sh);
           zf = __half2float(zh);
           if (valid) params[g] = __halves2half2(sh, zh);
         } else {
-          const float2 f = __half22float2(pin[g]);
+          const float2 f = __half22float2(pc);
           sf = f.x;
           zf = f.y;
         }
         const float inv = sf > 0.f ? 1.f / sf : 0.f;
+        uint32_t gw[GW];  // packed codes of the group (encode)
 #pragma unroll
-        for (int pc = 0; pc < NP; ++pc) {
-          const int e0 = g * G + pc * 32;  // first element of this pass
+        for (int q = 0; q < NP; ++q) {
           float p[32];
-          tmem_ld32(lane_addr + b * 128 + e0, p);
+          if (KEEP) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) p[i] = pk[i];
+          } else {
+            tmem_ld32(acc + g * G + q * 32, p);
+          }
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {  // 8 elements: codes, packing, reconstruction
-            const int e = e0 + ch * 8;
-            int qv[8];
+            const int eg = q * 32 + ch * 8;  // element within the group
+            float c[8];                      // grid points
             if (ENC) {
               float x[8];
-              unpack_bf16x8(xin[e / 8], x, 0);
+              unpack_bf16x8(xc[eg / 8], x, 0);
               uint32_t v = 0;
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                float c = rintf((x[i] - p[ch * 8 + i] - zf) * inv);
-                c = fminf(fmaxf(c, 0.f), (float)levels);
-                qv[i] = (int)c;
-                v |= (uint32_t)qv[i] << (i * bits);
+                c[i] = grid_point(x[i] - p[ch * 8 + i] - zf, inv, kGridMagic + (float)LEVELS);
+                v += __float_as_uint(c[i]) << (i * BITS);
               }
-              if (bits == 2)
-                cw[e / 16] |= v << ((e % 16) * 2);
-              else
-                cw[e / 8] = v;
+              v -= kBias8;
+              if (BITS == 2) {
+                if ((eg % 16) == 0)
+                  gw[eg / 16] = v;
+                else
+                  gw[eg / 16] |= v << 16;
+              } else {
+                gw[eg / 8] = v;
+              }
             } else {
-              const uint32_t v = bits == 2 ? (cwin[e / 16] >> ((e % 16) * 2)) : cwin[e / 8];
+              const uint32_t v = BITS == 2 ? (cc[eg / 16] >> ((eg % 16) * 2)) : cc[eg / 8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) qv[i] = (v >> (i * bits)) & levels;
+              for (int i = 0; i < 8; ++i) c[i] = grid_from_code((v >> (i * BITS)) & LEVELS);
             }
             uint32_t w[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int k = ch * 8 + 2 * i;
-              w[i] = pack_bf16x2(p[k] + fmaf(sf, (float)qv[2 * i], zf), p[k + 1] + fmaf(sf, (float)qv[2 * i + 1], zf));
+              w[i] = pack_bf16x2(p[k] + fmaf(sf, grid_code(c[2 * i]), zf), p[k + 1] + fmaf(sf, grid_code(c[2 * i + 1]), zf));
             }
-            *reinterpret_cast<uint4*>(recon(b) + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =
+            const int e = g * G + eg;  // element of the row
+            *reinterpret_cast<uint4*>(recon(b) + (e >> 6) * 16384 + sw128_off(row, (e & 63) >> 3)) =
                 make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
-      }
-      if (ENC && valid) {
-        uint4* dst = reinterpret_cast<uint4*>(codes);
+        if (ENC && valid) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (i < bits) dst[i] = make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]);
+          for (int i = 0; i < GW; i += 2) *reinterpret_cast<uint2*>(codes + g * GW + i) = make_uint2(gw[i], gw[i + 1]);
+        }
+        if (g + 1 < NG) {
+#pragma unroll
+          for (int i = 0; i < (ENC ? XQ : 1); ++i) xc[i] = xn[i];
+#pragma unroll
+          for (int i = 0; i < (ENC ? 1 : GW); ++i) cc[i] = cn[i];
+          pc = pn;
+        }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);
@@ -523,25 +634,39 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
 
     // After an abort every wait returns at once; the loops still run to the end
     // so that all threads of a group meet at every named barrier.
-    if (RC && grp == 0) {
-      wait(zk_full, 0, abort_flag, a.err, 0x900u);
-      tc_fence_after();
-      convert_latent(256, a.zk_hi, a.zk_lo);
-    }
-    for (int h = grp; h < H; h += 2) head(h, h, false);
-    if (elected) {
-      bulk_wait_all();
-      fence_async_global();
-      mbar_arrive(khat_stored);
-    }
-    if (RC && grp == 0) {
-      wait(zv_full, 0, abort_flag, a.err, 0x901u);
-      tc_fence_after();
-      convert_latent(256 + R, a.zv_hi, a.zv_lo);
-    }
-    if (!LAT) {
-      for (int u = H; u < 2 * H; ++u)
-        if ((u & 1) == grp) head(u, u - H, true);
+    for (int it = 0; it < my_tiles; ++it) {
+      const int t0 = tile_t0(it);
+      if (RC && grp == 0 && (!OVL || it == 0)) {
+        wait(zk_full, zk_use++ & 1, abort_flag, a.err, 0x900u);
+        tc_fence_after();
+        convert_latent(zk_col(it), t0, a.zk_hi, a.zk_lo);
+      }
+      // K heads u < H, then V heads; head u of the tile goes to group (it*2H + u) mod 2
+      const int nu = LAT ? H + 1 : 2 * H;
+#pragma unroll 1
+      for (int u = 0; u < nu; ++u) {
+        if (u == H) {  // between the K and the V heads
+          if (elected) {
+            bulk_wait_all();
+            fence_async_global();
+            mbar_arrive(khat_stored);
+          }
+          if (RC && grp == 0) {
+            wait(zv_full, zv_use++ & 1, abort_flag, a.err, 0x901u);
+            tc_fence_after();
+            convert_latent(zv_col(it), t0, a.zv_hi, a.zv_lo);
+          }
+          if (LAT) break;
+        }
+        if (((it * HH + u) & 1) == grp) head(u < H ? u : u - H, u >= H, t0);
+      }
+      if (OVL && RC && grp == 0 && it + 1 < my_tiles) {
+        // the next tile's K latent: its last chunk follows this tile's last V MMA,
+        // so the latent tile in shared memory is free
+        wait(zk_full, zk_use++ & 1, abort_flag, a.err, 0x902u);
+        tc_fence_after();
+        convert_latent(zk_col(it + 1), tile_t0(it + 1), a.zk_hi, a.zk_lo);
+      }
     }
     if (elected) bulk_wait_all();
   }
@@ -602,28 +727,50 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint3
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int G, int RC>
+// Streaming multiprocessors of the current device (0 on error).
+static int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int MODE, int G, int RC, int BITS>
 static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
-  auto k = xlayer_tc_kernel<MODE, G, RC>;
+  auto k = xlayer_tc_kernel<MODE, G, RC, BITS>;
   const int smem = Layout<RC>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int grid = (int)((a.T + 127) / 128);
+  // persistent: at most one CTA per SM, each looping over token tiles
+  const int64_t ntiles = (a.T + 127) / 128;
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int grid = (int)(ntiles < sms ? ntiles : sms);
   k<<<grid, kThreads, smem, st>>>(m, a);
   count_launches(1);
   return cudaGetLastError();
 }
 
+template <int MODE, int BITS>
+static cudaError_t dispatch_bits(int group, int rc, const Maps& m, const Args& a, cudaStream_t st) {
+  if (group == 32) {
+    if (rc == 0) return launch<MODE, 32, 0, BITS>(m, a, st);
+    if (rc == 1) return launch<MODE, 32, 1, BITS>(m, a, st);
+    return launch<MODE, 32, 2, BITS>(m, a, st);
+  }
+  if (rc == 0) return launch<MODE, 64, 0, BITS>(m, a, st);
+  if (rc == 1) return launch<MODE, 64, 1, BITS>(m, a, st);
+  return launch<MODE, 64, 2, BITS>(m, a, st);
+}
+
 template <int MODE>
 static cudaError_t dispatch(int group, int rc, const Maps& m, const Args& a, cudaStream_t st) {
-  if (group == 32) {
-    if (rc == 0) return launch<MODE, 32, 0>(m, a, st);
-    if (rc == 1) return launch<MODE, 32, 1>(m, a, st);
-    return launch<MODE, 32, 2>(m, a, st);
-  }
-  if (rc == 0) return launch<MODE, 64, 0>(m, a, st);
-  if (rc == 1) return launch<MODE, 64, 1>(m, a, st);
-  return launch<MODE, 64, 2>(m, a, st);
+  return a.bits == 2 ? dispatch_bits<MODE, 2>(group, rc, m, a, st) : dispatch_bits<MODE, 4>(group, rc, m, a, st);
 }
 
 }  // namespace tc

@@ -366,8 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
           uint32_t w[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float c0 = (float)((v >> ((2 * i) * bits)) & levels);
-            const float c1 = (float)((v >> ((2 * i + 1) * bits)) & levels);
+            const float c0 = grid_code(grid_from_code((v >> ((2 * i) * bits)) & levels));
+            const float c1 = grid_code(grid_from_code((v >> ((2 * i + 1) * bits)) & levels));
             w[i] = pack_bf16x2(p[ch * 8 + 2 * i] + fmaf(sf, c0, zf), p[ch * 8 + 2 * i + 1] + fmaf(sf, c1, zf));
           }
           *reinterpret_cast<uint4*>(tile + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =

@@ -115,6 +115,29 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t b
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same, issued only where `lead` is non-zero (the MMA warp runs converged;
+// one lane issues every tcgen05 instruction).
+__device__ __forceinline__ void umma_if(uint32_t lead, uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 e, %5, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(lead)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_if(uint32_t lead, uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\tsetp.ne.b32 e, %1, 0;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar)),
+      "r"(lead)
+      : "memory");
+}
+template <bool B>
+struct Tag {
+  static constexpr bool value = B;
+};
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
@@ -152,6 +175,33 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 // Byte offset of the 16-byte chunk `c` (0..7) of row `row` inside a [rows][64]
 // bf16 sub-tile written with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw128_off(int row, int c) { return row * 128 + ((c ^ (row & 7)) << 4); }
+
+// Quantization onto the integer grid [0, levels] without float <-> int
+// conversions (they run on the narrow conversion pipe).  Adding 1.5 * 2^23 to a
+// float of magnitude below 2^22 rounds it to the nearest integer (ties to even,
+// the mode of the addition) and leaves that integer in the low mantissa bits;
+// the grid point is then clamped while still a float.  A code's float value is
+// recovered exactly by subtracting the constant again.
+constexpr float kGridMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr uint32_t kGridMagicBits = 0x4B400000u;
+// grid point of t * inv, as a float in [kGridMagic, top] with top = kGridMagic + levels.
+// The product is rounded to fp32 before the integer rounding (no fused
+// multiply-add), so a quotient that is exactly k + 1/2 stays a tie and goes to
+// the even code, as rintf(t * inv) would.
+__device__ __forceinline__ float grid_point(float t, float inv, float top) {
+  return fminf(fmaxf(__fadd_rn(__fmul_rn(t, inv), kGridMagic), kGridMagic), top);
+}
+// the code of a grid point as a float
+__device__ __forceinline__ float grid_code(float c) { return c - kGridMagic; }
+// the grid point of a code (0 <= k < 2^22)
+__device__ __forceinline__ float grid_from_code(uint32_t k) { return __uint_as_float(kGridMagicBits | k); }
+// sum over i < n of kGridMagicBits << (i * bits), modulo 2^32: subtracting it from
+// sum_i bits(grid point i) << (i * bits) leaves the packed codes
+__host__ __device__ constexpr uint32_t grid_pack_bias(int bits, int n) {
+  uint32_t s = 0;
+  for (int i = 0; i < n; ++i) s += kGridMagicBits << (i * bits);
+  return s;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);

@@ -212,6 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
       __nv_bfloat16* rec = isv ? a.vrec : a.krec;
 #pragma unroll
+      const float top = kGridMagic + (float)levels;
+      const uint32_t bias8 = grid_pack_bias(bits, 8);
       for (int g = 0; g < NG; ++g) {
         float sf, zf;
         if (ENC) {
@@ -262,18 +264,17 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             const int e = e0 + ch * 8;
-            int qv[8];
+            float c[8];  // grid points
             if (ENC) {
               float x[8];
               unpack_bf16x8(xin[e / 8], x, 0);
               uint32_t v = 0;
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                float c = rintf((x[i] - p[ch * 8 + i] - zf) * inv);
-                c = fminf(fmaxf(c, 0.f), (float)levels);
-                qv[i] = (int)c;
-                v |= (uint32_t)qv[i] << (i * bits);
+                c[i] = grid_point(x[i] - p[ch * 8 + i] - zf, inv, top);
+                v += __float_as_uint(c[i]) << (i * bits);
               }
+              v -= bias8;
               if (bits == 2)
                 cw[e / 16] |= v << ((e % 16) * 2);
               else
@@ -281,13 +282,13 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
             } else {
               const uint32_t v = bits == 2 ? (cwin[e / 16] >> ((e % 16) * 2)) : cwin[e / 8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) qv[i] = (v >> (i * bits)) & levels;
+              for (int i = 0; i < 8; ++i) c[i] = grid_from_code((v >> (i * bits)) & levels);
             }
             uint32_t w[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int k = ch * 8 + 2 * i;
-              w[i] = pack_bf16x2(p[k] + fmaf(sf, (float)qv[2 * i], zf), p[k + 1] + fmaf(sf, (float)qv[2 * i + 1], zf));
+              w[i] = pack_bf16x2(p[k] + fmaf(sf, grid_code(c[2 * i]), zf), p[k + 1] + fmaf(sf, grid_code(c[2 * i + 1]), zf));
             }
             recw[ch] = make_uint4(w[0], w[1], w[2], w[3]);
           }
