@@ -1,22 +1,25 @@
-// Attention over a compressed cross-layer history (tcgen05 + TMEM + TMA).
+// Attention over a compressed cross-layer history (tcgen05 + TMEM + TMA,
+// thread-block clusters).
 //
 //   O = softmax(scale Q [K^_hist ; K_self]^T) [V^_hist ; V_self]
 //
 // ("NanoKV: High-Ratio KV Cache Compression for Autoregressive Video
 // Generation", abstract: attention over the compressed history is the
 // bottleneck; "CORAL-KV ...", Fig. 3: the history of layer l is decoded from
-// its codes and the reconstruction of layer l-1.)  One CTA per (head, 128-query
-// tile).  The history is decoded tile by tile on chip and never written to
-// device memory: for each 128-key tile the CTA runs the block-DPLR prediction on
-// the tensor cores (the layer's low-rank latents come precomputed, as bf16
-// hi / lo pairs, from the latent-only codec kernel), adds the dequantized codes
-// and keeps the bf16 K^ / V^ tile in shared memory.  Then S = Q K^T and
-// O += P V^ run on tcgen05 with the softmax on four warps.
+// its codes and the reconstruction of layer l-1.)  The history is decoded tile
+// by tile on chip and never written to device memory: for a 128-key tile the
+// block-DPLR prediction runs on the tensor cores (the layer's low-rank latents
+// come precomputed, as bf16 hi / lo pairs, from the latent-only codec kernel),
+// the dequantized codes are added and the bf16 K^ / V^ tile is kept in shared
+// memory.  A cluster of CTAs (consecutive query tiles of one head) shares that
+// work: each CTA decodes every CQ-th key tile and pushes it into the others'
+// shared memory, so a key tile is decoded once per cluster instead of once per
+// query tile.  S = Q K^T and O += P V^ run on tcgen05; P stays in tensor memory.
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2-5 decode
-// epilogue (TMEM -> K^ / V^ tiles), 6-9 softmax (S -> P, running max / sum,
-// lazy rescaling of O, final normalisation).  TMEM: decode-K accumulator, decode-V
-// accumulator, S, O (128 columns each).
+// epilogue (TMEM -> K^ / V^ tiles, pushed to the cluster), 6-9 softmax (S -> P,
+// running max / sum, lazy rescaling of O, final normalisation).  TMEM: decode
+// accumulator, S / P slots [2], O (128 columns each).
 #include <cuda.h>
 #include <string.h>
 
@@ -33,14 +36,19 @@ bool map2d_bytes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
 namespace attn {
 
 constexpr int kThreads = 320;
+#ifndef KVC_ATTN_CLUSTER
+#define KVC_ATTN_CLUSTER 4
+#endif
+// CTAs per cluster (even, at most 8): consecutive query tiles of one head share the decoded history
+constexpr int CQ = KVC_ATTN_CLUSTER;
+static_assert(CQ % 2 == 0 && CQ <= 8, "cluster of an even size up to 8");
 constexpr int kStages = 2;
 constexpr int kStage = 32768;
 // shared memory (offsets from a 1024-aligned base)
 constexpr int kQ = 0;                        // Q tile, 2 sub-tiles
-constexpr int kK = kQ + 32768;               // K^ tiles [2]
-constexpr int kV = kK + 2 * 32768;           // V^ tile
-constexpr int kP = kV + 32768;               // P tile
-constexpr int kSt = kP + 32768;              // operand stages
+constexpr int kK = kQ + 32768;               // K^ slots [2]
+constexpr int kV = kK + 2 * 32768;           // V^ slots [2]
+constexpr int kSt = kV + 2 * 32768;          // decode operand stages
 constexpr int kBar = kSt + kStages * kStage;
 constexpr int kSmem = kBar + 1024 + 1024;    // + barriers + alignment slack
 
@@ -87,36 +95,151 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-template <int RC>
-__global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid_constant__ Maps maps, const Args a) {
+// ---------------------------------------------------------------- cluster primitives
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory location in cluster CTA `rank`
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// arrive on a peer's mbarrier announcing `bytes` of transfer
+__device__ __forceinline__ void peer_arrive_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// bulk copy of `bytes` from this CTA's shared memory into a peer's, completing on the peer's mbarrier
+__device__ __forceinline__ void push_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// commit whose arrival lands on the mbarrier at the same offset in the CTAs of `mask`
+__device__ __forceinline__ void umma_commit_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]: A (bf16 pairs per 32-bit column) from tensor memory
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 columns of this thread's TMEM lane, without waiting: the values are valid
+// only after tmem_ld_wait on the same arrays
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, float (&v)[32]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+// keeps the compiler from touching v before this point
+__device__ __forceinline__ void tie32(float (&v)[32]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]),
+                 "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait(float (&a)[32], float (&b)[32], float (&c)[32], float (&d)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  tie32(a);
+  tie32(b);
+  tie32(c);
+  tie32(d);
+}
+__device__ __forceinline__ void tmem_ld_wait2(float (&a)[32], float (&b)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  tie32(a);
+  tie32(b);
+}
+// 2^x by the hardware approximation (flush-to-zero; softmax weights only)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]), "r"(w[9]),
+      "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
+
+// ---------------------------------------------------------------- the kernel
+//
+// Cluster of CQ CTAs = CQ consecutive 128-query tiles of one head.  History key
+// tile j is decoded by cluster rank j mod CQ and pushed, as bf16 K^ / V^ tiles,
+// into the same double-buffered tile slots of every CTA of the cluster; the
+// chunk's own keys (K_self, V_self) are loaded by each CTA.  Per key tile j
+// (slot b = j mod 2) every CTA runs S(j) = Q K^(j)^T into TMEM S[b], the softmax
+// writes P(j) over S[b] as bf16 pairs, and O += P(j) V^(j) takes P from TMEM.
+//
+// Slot reuse across the cluster: the decoder of tile j writes slot b only after
+// every CTA has finished with tile j-2 in that slot (kfree / vfree gather CQ
+// arrivals, sent by tcgen05.commit multicast after S(j-2) / PV(j-2)); the
+// decoder announces the bytes on each peer's kfull / vfull and pushes the tile
+// with a bulk copy that completes there.
+
+template <int RC, int G, int BITS>
+__global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __grid_constant__ Maps maps, const Args a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBar);
-  uint64_t* full = bars;                  // [kStages]
-  uint64_t* empty = bars + kStages;       // [kStages]
-  uint64_t* q_full = bars + 2 * kStages;
-  uint64_t* d0_full = q_full + 1;         // decode-K accumulator ready
-  uint64_t* d1_full = d0_full + 1;        // decode-V accumulator ready
-  uint64_t* kt_ready = d1_full + 1;       // [2] K tile in smem (decode warps)
-  uint64_t* vt_ready = kt_ready + 2;      // V tile in smem (decode warps)
-  uint64_t* s_full = vt_ready + 1;
-  uint64_t* p_full = s_full + 1;          // P written (softmax warps)
-  uint64_t* pv_done = p_full + 1;         // a PV product finished (O stable, P / V tiles free)
-  uint64_t* kt_free = pv_done + 1;        // [2] S and DEC_V of a K tile finished
-  uint64_t* self_kfull = kt_free + 2;     // [2] a K_self tile landed
-  uint64_t* self_vfull = self_kfull + 2;  // a V_self tile landed
-  uint64_t* o_done = self_vfull + 1;
+  uint64_t* full = bars;               // [kStages] decode operands landed
+  uint64_t* empty = full + kStages;    // [kStages]
+  uint64_t* q_full = empty + kStages;
+  uint64_t* d_full = q_full + 1;       // decode accumulator ready
+  uint64_t* kfull = d_full + 1;        // [2] K^ slot holds tile j
+  uint64_t* vfull = kfull + 2;         // [2] V^ slot holds tile j
+  uint64_t* kfree = vfull + 2;         // cluster gather: K^ slot free for this CTA's next decoded tile
+  uint64_t* vfree = kfree + 1;         // cluster gather: V^ slot free
+  uint64_t* kt_free = vfree + 1;       // [2] local: K^ slot free for a chunk tile
+  uint64_t* vt_free = kt_free + 2;     // [2] local: V^ slot free for a chunk tile
+  uint64_t* s_full = vt_free + 2;      // [2]
+  uint64_t* p_full = s_full + 2;       // [2]
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* o_done = pv_done + 1;
   uint64_t* mma_done = o_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  constexpr int R = RC * 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
   const int q0 = blockIdx.x * 128;
+  const bool has_q = q0 < a.n_q;  // the last cluster of a head may hold CTAs past the queries
+  const int rank = (int)cluster_rank();
   const int NH = (int)((a.T + 127) / 128);       // history key tiles
   const int NS = (int)((a.n_self + 127) / 128);  // chunk key tiles
   const int NT = NH + NS;
+  auto own = [&](int j) { return j < NH && j % CQ == rank; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -124,19 +247,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
       mbar_init(&empty[i], 1);
     }
     mbar_init(q_full, 1);
-    mbar_init(d0_full, 1);
-    mbar_init(d1_full, 1);
-    mbar_init(&kt_ready[0], 128);
-    mbar_init(&kt_ready[1], 128);
-    mbar_init(vt_ready, 128);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(d_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kfull[i], 1);
+      mbar_init(&vfull[i], 1);
+      mbar_init(&kt_free[i], 1);
+      mbar_init(&vt_free[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(kfree, CQ);
+    mbar_init(vfree, CQ);
     mbar_init(pv_done, 1);
-    mbar_init(&kt_free[0], 1);
-    mbar_init(&kt_free[1], 1);
-    mbar_init(&self_kfull[0], 1);
-    mbar_init(&self_kfull[1], 1);
-    mbar_init(self_vfull, 1);
     mbar_init(o_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -149,16 +271,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // every CTA's barriers exist before any remote arrival or push
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t D0 = tmem, D1 = tmem + 128, SC = tmem + 256, OC = tmem + 384;
+  const uint32_t DC = tmem, OC = tmem + 384;
+  auto SC = [&](int b) { return tmem + 128 + 128 * b; };
 
   auto stA = [&](int s) { return smem + kSt + s * kStage; };
   auto stB = [&](int s) { return smem + kSt + s * kStage + 16384; };
   uint8_t* Qs = smem + kQ;
   auto Kt = [&](int b) { return smem + kK + b * 32768; };
-  uint8_t* Vt = smem + kV;
-  uint8_t* Ps = smem + kP;
+  auto Vt = [&](int b) { return smem + kV + b * 32768; };
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -168,6 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      // the last phase armed on each barrier this thread loads into (drained after an abort)
+      int st_issued[kStages] = {}, self_issued[2][2] = {};
+      uint32_t st_ph[kStages] = {}, self_ph[2][2] = {};
       auto load = [&](const CUtensorMap* ma, int ax, int ay, const CUtensorMap* mb, int bx, int by) {
         if (!ok) return;
         if (!wait(&empty[s], ph ^ 1, abort_flag, a.err, 0x1100u + s)) {
@@ -177,52 +303,75 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
         mbar_arrive_expect_tx(&full[s], (ma ? 16384u : 0u) + 16384u);
         if (ma) tma_load(stA(s), ma, ax, ay, &full[s], pol_stream);
         tma_load(stB(s), mb, bx, by, &full[s], pol_keep);
+        st_issued[s] = 1;
+        st_ph[s] = ph;
         if (++s == kStages) {
           s = 0;
           ph ^= 1;
         }
       };
-      mbar_arrive_expect_tx(q_full, 32768u);
-      tma_load(Qs, &maps.q, h * 128, q0, q_full, pol_stream);
-      tma_load(Qs + 16384, &maps.q, h * 128 + 64, q0, q_full, pol_stream);
-      for (int j = 0; j < NT && ok; ++j) {
+      if (has_q) {
+        mbar_arrive_expect_tx(q_full, 32768u);
+        tma_load(Qs, &maps.q, h * 128, q0, q_full, pol_stream);
+        tma_load(Qs + 16384, &maps.q, h * 128 + 64, q0, q_full, pol_stream);
+      }
+      // decode operands of this CTA's history tiles, in the order the MMA warp takes them
+      for (int j = rank; j < NH && ok; j += CQ) {
+        const int t0 = j * 128;
+        constexpr int rbytes = 128 * BITS / 8;
+        tma_prefetch(&maps.ck, h * rbytes, t0);
+        tma_prefetch(&maps.cv, h * rbytes, t0);
+        if (G == 32) {
+          tma_prefetch(&maps.pk, h * 16, t0);
+          tma_prefetch(&maps.pv, h * 16, t0);
+        }
+        // K: K^_{l-1,h} B_h^T + [Z_K hi | lo] U_h^T
+        for (int c = 0; c < 2; ++c) load(&maps.ks, h * 128 + c * 64, t0, &maps.bk, c * 64, h * 128);
+        for (int c = 0; c < RC; ++c) {
+          load(&maps.zkh, c * 64, t0, &maps.uk, c * 64, h * 128);
+          load(&maps.zkl, c * 64, t0, &maps.uk, c * 64, h * 128);
+        }
+        // V: [K^_{l,h} (resident) | V^_{l-1,h}] BV_h^T + [Z_V hi | lo] UV_h^T
+        for (int c = 0; c < 2; ++c) load(nullptr, 0, 0, &maps.bv, c * 64, h * 128);
+        for (int c = 0; c < 2; ++c) load(&maps.vs, h * 128 + c * 64, t0, &maps.bv, 128 + c * 64, h * 128);
+        for (int c = 0; c < RC; ++c) {
+          load(&maps.zvh, c * 64, t0, &maps.uv, c * 64, h * 128);
+          load(&maps.zvl, c * 64, t0, &maps.uv, c * 64, h * 128);
+        }
+      }
+      // the chunk's own key tiles, into the slots once this CTA is done with them
+      int ktf[2] = {0, 0}, vtf[2] = {0, 0};
+      for (int j = NH; j < NT && ok && has_q; ++j) {
         const int b = j & 1;
-        if (j < NH) {
-          const int t0 = j * 128;
-          const int rbytes = 128 * a.bits / 8;
-          tma_prefetch(&maps.ck, h * rbytes, t0);
-          tma_prefetch(&maps.cv, h * rbytes, t0);
-          if (a.group == 32) {
-            tma_prefetch(&maps.pk, h * 16, t0);
-            tma_prefetch(&maps.pv, h * 16, t0);
+        const int s0 = (j - NH) * 128;
+        if (j >= 2 && !wait(&kt_free[b], ktf[b]++ & 1, abort_flag, a.err, 0x1200u + b)) ok = false;
+        if (!ok) break;
+        mbar_arrive_expect_tx(&kfull[b], 32768u);
+        tma_load(Kt(b), &maps.kself, h * 128, s0, &kfull[b], pol_stream);
+        tma_load(Kt(b) + 16384, &maps.kself, h * 128 + 64, s0, &kfull[b], pol_stream);
+        self_issued[0][b] = 1;
+        self_ph[0][b] = (j >> 1) & 1;
+        if (j >= 2 && !wait(&vt_free[b], vtf[b]++ & 1, abort_flag, a.err, 0x1210u + b)) ok = false;
+        if (!ok) break;
+        mbar_arrive_expect_tx(&vfull[b], 32768u);
+        tma_load(Vt(b), &maps.vself, h * 128, s0, &vfull[b], pol_stream);
+        tma_load(Vt(b) + 16384, &maps.vself, h * 128 + 64, s0, &vfull[b], pol_stream);
+        self_issued[1][b] = 1;
+        self_ph[1][b] = (j >> 1) & 1;
+      }
+      if (*abort_flag) {
+        // every load this thread issued lands before the CTA can leave
+        auto drain = [&](uint64_t* bar, uint32_t parity) {
+          const long long w0 = clock64();
+          while (!mbar_test(bar, parity) && clock64() - w0 < kWaitBudget) {
           }
-          // decode K: K^_{l-1,h} B_h^T + [Z_K hi | lo] U_h^T
-          for (int c = 0; c < 2; ++c) load(&maps.ks, h * 128 + c * 64, t0, &maps.bk, c * 64, h * 128);
-          for (int c = 0; c < RC; ++c) {
-            load(&maps.zkh, c * 64, t0, &maps.uk, c * 64, h * 128);
-            load(&maps.zkl, c * 64, t0, &maps.uk, c * 64, h * 128);
-          }
-          // decode V: [K^_{l,h} (resident) | V^_{l-1,h}] BV_h^T + [Z_V hi | lo] UV_h^T
-          for (int c = 0; c < 2; ++c) load(nullptr, 0, 0, &maps.bv, c * 64, h * 128);
-          for (int c = 0; c < 2; ++c) load(&maps.vs, h * 128 + c * 64, t0, &maps.bv, 128 + c * 64, h * 128);
-          for (int c = 0; c < RC; ++c) {
-            load(&maps.zvh, c * 64, t0, &maps.uv, c * 64, h * 128);
-            load(&maps.zvl, c * 64, t0, &maps.uv, c * 64, h * 128);
-          }
-        } else {
-          // chunk tile: K_self into the K tile once S and DEC_V of tile j-2 are done,
-          // V_self into the V tile once PV(j-1) is done (PV(j-1) follows S(j))
-          const int s0 = (j - NH) * 128;
-          if (j >= 2 && !wait(&kt_free[b], ((j - 2) >> 1) & 1, abort_flag, a.err, 0x1200u + b)) ok = false;
-          if (!ok) break;
-          mbar_arrive_expect_tx(&self_kfull[b], 32768u);
-          tma_load(Kt(b), &maps.kself, h * 128, s0, &self_kfull[b], pol_stream);
-          tma_load(Kt(b) + 16384, &maps.kself, h * 128 + 64, s0, &self_kfull[b], pol_stream);
-          if (j >= 1 && !wait(pv_done, (j - 1) & 1, abort_flag, a.err, 0x1210u)) ok = false;
-          if (!ok) break;
-          mbar_arrive_expect_tx(self_vfull, 32768u);
-          tma_load(Vt, &maps.vself, h * 128, s0, self_vfull, pol_stream);
-          tma_load(Vt + 16384, &maps.vself, h * 128 + 64, s0, self_vfull, pol_stream);
+        };
+        if (has_q) drain(q_full, 0);
+        for (int i = 0; i < kStages; ++i)
+          if (st_issued[i]) drain(&full[i], st_ph[i]);
+        for (int b = 0; b < 2; ++b) {
+          if (self_issued[0][b]) drain(&kfull[b], self_ph[0][b]);
+          if (self_issued[1][b]) drain(&vfull[b], self_ph[1][b]);
         }
       }
     }
@@ -251,79 +400,79 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
         }
       };
       auto dec_k = [&]() {
-        for (int c = 0; c < 2; ++c) chunk(D0, c == 0, nullptr);
-        for (int c = 0; c < 2 * RC; ++c) chunk(D0, false, nullptr);
-        if (ok) umma_commit(d0_full);
+        for (int c = 0; c < 2; ++c) chunk(DC, c == 0, nullptr);
+        for (int c = 0; c < 2 * RC; ++c) chunk(DC, false, nullptr);
+        umma_commit(d_full);
       };
-      int kt_use[2] = {0, 0};
-      if (!wait(q_full, 0, abort_flag, a.err, 0x1310u)) ok = false;
-      tc_fence_after();
-      if (NH > 0) dec_k();
-      for (int j = 0; j < NT && ok; ++j) {
-        const int b = j & 1;
-        if (!wait(&kt_ready[b], kt_use[b] & 1, abort_flag, a.err, 0x1320u + b)) ok = false;
-        kt_use[b]++;
-        // S(j) = Q K^(j)^T; the S columns are free once the softmax of tile j-1 wrote P
-        if (ok && j >= 1 && !wait(p_full, (j - 1) & 1, abort_flag, a.err, 0x1330u)) ok = false;
-        if (!ok) break;
+      auto dec_v = [&](int b) {
+        for (int c = 0; c < 2; ++c) chunk(DC, c == 0, Kt(b) + c * 16384);
+        for (int c = 0; c < 2 + 2 * RC; ++c) chunk(DC, false, nullptr);
+        umma_commit(d_full);
+      };
+      // slot of tile t released (S(t) / PV(t) issued): to the decoder of tile t+2, or locally
+      auto release = [&](int t, uint64_t* gather, uint64_t* local) {
+        const int j2 = t + 2;
+        if (j2 < NH)
+          umma_commit_mc(gather, (uint16_t)(1u << (j2 % CQ)));
+        else if (j2 < NT && has_q)
+          umma_commit(&local[t & 1]);
+      };
+      if (has_q && !wait(q_full, 0, abort_flag, a.err, 0x1310u)) ok = false;
+      if (own(rank)) dec_k();
+      if (own(0)) {  // tile 0 has no earlier iteration to take its V decode
+        wait(&kfull[0], 0, abort_flag, a.err, 0x1324u);
         tc_fence_after();
-        {
-          const uint64_t qd = desc_sw128(smem_u32(Qs));
-          const uint64_t kd = desc_sw128(smem_u32(Kt(b)));
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
-            umma(SC, qd + off, kd + off, id128, k == 0 ? 0u : 1u);
-          }
-          umma_commit(s_full);
-        }
-        // PV(j-1): O += P V^(j-1)
-        if (j >= 1) {
-          if (!wait(vt_ready, (j - 1) & 1, abort_flag, a.err, 0x1340u)) ok = false;
+        dec_v(0);
+      }
+      const int NE = has_q ? NT : NH;  // key tiles this CTA takes part in
+      for (int j = 0; j <= NE; ++j) {
+        if (j < NE) {
+          const int b = j & 1;
+          wait(&kfull[b], (j >> 1) & 1, abort_flag, a.err, 0x1320u + b);
           tc_fence_after();
-          if (ok) {
-            const uint64_t pd = desc_sw128(smem_u32(Ps));
-            const uint64_t vd = desc_mn_sw128(smem_u32(Vt), 16384);
-            const uint32_t idv = idesc_bf16_bmn(128, 128);
+          if (has_q) {
+            // S(j) = Q K^(j)^T into S[b]; S[b] last held P(j-2), read by PV(j-2) issued before
+            const uint64_t qd = desc_sw128(smem_u32(Qs));
+            const uint64_t kd = desc_sw128(smem_u32(Kt(b)));
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-              const uint64_t poff = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
-              const uint64_t voff = (uint64_t)k * (2048 >> 4);
-              umma(OC, pd + poff, vd + voff, idv, j == 1 && k == 0 ? 0u : 1u);
+              const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
+              umma(SC(b), qd + off, kd + off, id128, k == 0 ? 0u : 1u);
             }
-            umma_commit(pv_done);
+            umma_commit(&s_full[b]);
           }
+          release(j, kfree, kt_free);
         }
-        // decode V(j) (needs K^(j) as an operand) and K(j+1)
-        if (j < NH) {
-          for (int c = 0; c < 2; ++c) chunk(D1, c == 0, Kt(b) + c * 16384);
-          for (int c = 0; c < 2; ++c) chunk(D1, false, nullptr);
-          for (int c = 0; c < 2 * RC; ++c) chunk(D1, false, nullptr);
-          if (ok) umma_commit(d1_full);
-        }
-        if (ok) umma_commit(&kt_free[b]);
-        if (j + 1 < NH) dec_k();
-      }
-      // last PV
-      if (ok && NT >= 1) {
-        const int j = NT;
-        if (!wait(p_full, (j - 1) & 1, abort_flag, a.err, 0x1350u)) ok = false;
-        if (ok && !wait(vt_ready, (j - 1) & 1, abort_flag, a.err, 0x1351u)) ok = false;
-        tc_fence_after();
-        if (ok) {
-          const uint64_t pd = desc_sw128(smem_u32(Ps));
-          const uint64_t vd = desc_mn_sw128(smem_u32(Vt), 16384);
-          const uint32_t idv = idesc_bf16_bmn(128, 128);
+        if (j >= 1) {
+          const int t = j - 1, b = t & 1;
+          if (has_q) {
+            // O += P(t) V^(t), P from TMEM
+            wait(&p_full[b], (t >> 1) & 1, abort_flag, a.err, 0x1330u + b);
+            wait(&vfull[b], (t >> 1) & 1, abort_flag, a.err, 0x1340u + b);
+            tc_fence_after();
+            const uint64_t vd = desc_mn_sw128(smem_u32(Vt(b)), 16384);
+            const uint32_t idv = idesc_bf16_bmn(128, 128);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint64_t poff = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
-            const uint64_t voff = (uint64_t)k * (2048 >> 4);
-            umma(OC, pd + poff, vd + voff, idv, j == 1 && k == 0 ? 0u : 1u);
+            for (int k = 0; k < 8; ++k)
+              umma_ts(OC, SC(b) + k * 8, vd + (uint64_t)k * (2048 >> 4), idv, (t == 0 && k == 0) ? 0u : 1u);
+            umma_commit(pv_done);
+          } else {
+            wait(&vfull[b], (t >> 1) & 1, abort_flag, a.err, 0x1341u + b);
           }
-          umma_commit(pv_done);
+          release(t, vfree, vt_free);
+          // the decode accumulator is free once V^(t) is out: start this CTA's next tile
+          if (own(t) && t + CQ < NH) dec_k();
+        }
+        // V decode of this CTA's tile j+1 one iteration early, as soon as its K^ is
+        // published here (that also means the decode accumulator was drained)
+        if (j + 1 < NH && own(j + 1)) {
+          const int b1 = (j + 1) & 1;
+          wait(&kfull[b1], ((j + 1) >> 1) & 1, abort_flag, a.err, 0x1325u);
+          tc_fence_after();
+          dec_v(b1);
         }
       }
-      umma_commit(o_done);
+      if (has_q) umma_commit(o_done);
       umma_commit(mma_done);
       const long long w0 = clock64();
       while (!mbar_test(mma_done, 0) && clock64() - w0 < kWaitBudget) {
@@ -334,71 +483,88 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
     const int qd = warp & 3;
     const int row = qd * 32 + lane;  // key row of the tile (TMEM lane)
     const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16);
-    const int bits = a.bits, levels = (1 << bits) - 1, G = a.group;
-    const int row_bytes = 128 * bits / 8;
-    int d0_use = 0, d1_use = 0, kself_use[2] = {0, 0}, vself_use = 0;
-    // TMEM accumulator + dequantized codes -> bf16 row of a K^ / V^ tile
-    auto emit = [&](uint32_t acc, const uint8_t* codes, const __half2* params, bool valid, uint8_t* tile) {
-      uint32_t cw[16];
-      __half2 pr[4];
+    constexpr int LEVELS = (1 << BITS) - 1;
+    constexpr int RB = 128 * BITS / 8;  // code bytes of a row
+    constexpr int NW = RB / 4;          // code words of a row
+    constexpr int NG = 128 / G;
+    const bool elected = warp == 2 && lane == 0;
+    int dfu = 0, kfu = 0, vfu = 0;
+    // the codes and (scale, zero) pairs of one row of one tile
+    struct RowIn {
+      uint32_t cw[NW];
+      __half2 pr[NG];
+    };
+    auto fetch = [&](const uint8_t* codes, const __half2* params, bool valid, RowIn& in) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) cw[i] = 0;
-      if (valid) {
-        const uint4* cp = reinterpret_cast<const uint4*>(codes);
-        const int nw = row_bytes / 16;
-        for (int i = 0; i < nw; ++i) reinterpret_cast<uint4*>(cw)[i] = __ldcs(cp + i);
-        for (int g = 0; g < 128 / G; ++g) pr[g] = params[g];
+      for (int i = 0; i < NW / 4; ++i) {
+        const uint4 w = valid ? __ldcs(reinterpret_cast<const uint4*>(codes) + i) : make_uint4(0, 0, 0, 0);
+        in.cw[4 * i] = w.x;
+        in.cw[4 * i + 1] = w.y;
+        in.cw[4 * i + 2] = w.z;
+        in.cw[4 * i + 3] = w.w;
       }
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        float p[32];
-        tmem_ld32(lane_addr + acc + pc * 32, p);
+      for (int g = 0; g < NG; ++g) in.pr[g] = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
+    };
+    // TMEM accumulator + dequantized codes -> bf16 row of a K^ / V^ tile
+    auto emit = [&](const RowIn& in, uint8_t* tile) {
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int e = pc * 32 + ch * 8;  // element of the row
-          float sf = 0.f, zf = 0.f;
-          if (valid) {
-            const float2 f = __half22float2(pr[e / G]);
-            sf = f.x;
-            zf = f.y;
-          }
-          const uint32_t v = bits == 2 ? (cw[e / 16] >> ((e % 16) * 2)) : cw[e / 8];
-          uint32_t w[4];
+      for (int half = 0; half < 2; ++half) {
+        float p[2][32];
+        tmem_ld32_async(lane_addr + (DC - tmem) + half * 64, p[0]);
+        tmem_ld32_async(lane_addr + (DC - tmem) + half * 64 + 32, p[1]);
+        tmem_ld_wait2(p[0], p[1]);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float c0 = grid_code(grid_from_code((v >> ((2 * i) * bits)) & levels));
-            const float c1 = grid_code(grid_from_code((v >> ((2 * i + 1) * bits)) & levels));
-            w[i] = pack_bf16x2(p[ch * 8 + 2 * i] + fmaf(sf, c0, zf), p[ch * 8 + 2 * i + 1] + fmaf(sf, c1, zf));
+        for (int q = 0; q < 2; ++q) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int e = (half * 2 + q) * 32 + ch * 8;  // element of the row
+            const float2 f = __half22float2(in.pr[e / G]);
+            float r[8];
+            dequant8<BITS>(in.cw[BITS == 2 ? e / 16 : e / 8], e, f.x, f.y, &p[q][ch * 8], r);
+            *reinterpret_cast<uint4*>(tile + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =
+                make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
+                           pack_bf16x2(r[6], r[7]));
           }
-          *reinterpret_cast<uint4*>(tile + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       tc_fence_before();
       fence_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
     };
-    for (int j = 0; j < NT; ++j) {
-      const int b = j & 1;
-      if (j < NH) {
-        const int64_t t = (int64_t)j * 128 + row;
-        const bool valid = t < a.T;
-        const int64_t rowi = t * a.H + h;
-        wait(d0_full, d0_use++ & 1, abort_flag, a.err, 0x1400u);
-        tc_fence_after();
-        emit(0, a.kcodes + rowi * row_bytes, a.kparams + rowi * (128 / G), valid, Kt(b));
-        mbar_arrive(&kt_ready[b]);
-        wait(d1_full, d1_use++ & 1, abort_flag, a.err, 0x1401u);
-        tc_fence_after();
-        emit(128, a.vcodes + rowi * row_bytes, a.vparams + rowi * (128 / G), valid, Vt);
-        mbar_arrive(vt_ready);
-      } else {
-        wait(&self_kfull[b], kself_use[b]++ & 1, abort_flag, a.err, 0x1402u + b);
-        mbar_arrive(&kt_ready[b]);
-        wait(self_vfull, vself_use++ & 1, abort_flag, a.err, 0x1404u);
-        mbar_arrive(vt_ready);
+    // the tile is complete here: announce it to every peer, push it, and mark it locally
+    auto publish = [&](uint8_t* tile, uint64_t* bar) {
+      if (!elected) return;
+      for (int p = 1; p < CQ; ++p) {
+        const uint32_t peer = (uint32_t)((rank + p) % CQ);
+        const uint32_t pb = peer_addr(bar, peer);
+        peer_arrive_expect(pb, 32768u);
+        push_to_peer(peer_addr(tile, peer), tile, 32768u, pb);
       }
+      bulk_commit();
+      mbar_arrive(bar);
+    };
+    for (int j = rank; j < NH; j += CQ) {
+      const int b = j & 1;
+      const int64_t t = (int64_t)j * 128 + row;
+      const bool valid = t < a.T;
+      const int64_t rowi = t * a.H + h;
+      RowIn kin, vin;
+      fetch(a.kcodes + rowi * RB, a.kparams + rowi * NG, valid, kin);
+      wait(d_full, dfu++ & 1, abort_flag, a.err, 0x1400u);
+      if (j >= 2) wait(kfree, kfu++ & 1, abort_flag, a.err, 0x1401u);
+      tc_fence_after();
+      emit(kin, Kt(b));
+      publish(Kt(b), &kfull[b]);
+      fetch(a.vcodes + rowi * RB, a.vparams + rowi * NG, valid, vin);
+      wait(d_full, dfu++ & 1, abort_flag, a.err, 0x1402u);
+      if (j >= 2) wait(vfree, vfu++ & 1, abort_flag, a.err, 0x1403u);
+      tc_fence_after();
+      emit(vin, Vt(b));
+      publish(Vt(b), &vfull[b]);
     }
-  } else {
+    if (elected) bulk_wait_all();
+  } else if (has_q) {
     // ================================================================ softmax (warps 6-9)
     const int qd = warp & 3;
     const int row = qd * 32 + lane;  // query row
@@ -406,26 +572,60 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
     const float c = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < NT; ++j) {
-      wait(s_full, j & 1, abort_flag, a.err, 0x1500u);
+      const int b = j & 1;
+      const uint32_t sc = lane_addr + (SC(b) - tmem);
+      wait(&s_full[b], (j >> 1) & 1, abort_flag, a.err, 0x1500u + b);
       tc_fence_after();
       const int64_t kbase = j < NH ? (int64_t)j * 128 : (int64_t)(j - NH) * 128;
       const int64_t klim = j < NH ? a.T : a.n_self;
       const int nvalid = klim - kbase < 128 ? (int)(klim - kbase) : 128;
-      float mt = -INFINITY;
+      // the whole S row in registers: four loads, one wait
+      float sv[4][32];
+      tmem_ld32_async(sc, sv[0]);
+      tmem_ld32_async(sc + 32, sv[1]);
+      tmem_ld32_async(sc + 64, sv[2]);
+      tmem_ld32_async(sc + 96, sv[3]);
+      tmem_ld_wait(sv[0], sv[1], sv[2], sv[3]);
+      if (nvalid < 128) {
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        float sv[32];
-        tmem_ld32(lane_addr + (SC - tmem) + pc * 32, sv);
+        for (int pc = 0; pc < 4; ++pc)
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (pc * 32 + i < nvalid) mt = fmaxf(mt, sv[i] * c);
+          for (int i = 0; i < 32; ++i)
+            if (pc * 32 + i >= nvalid) sv[pc][i] = -INFINITY;
       }
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], sv[pc][i]);
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
       // lazy rescale: only when the tile's max exceeds the one in use by 2^8
       const bool need = mt > m_used + 8.f;
+      float alpha = 1.f;
+      if (need) {
+        alpha = m_used == -INFINITY ? 0.f : ex2_approx(m_used - mt);
+        l *= alpha;
+        m_used = mt;
+      }
+      // P over S: the 16 packed columns of pass pc land on S columns already read
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(sv[pc][2 * i], c, -m_used));
+          const float p1 = ex2_approx(fmaf(sv[pc][2 * i + 1], c, -m_used));
+          ls[i & 3] += p0 + p1;
+          w[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(sc + pc * 16, w);
+      }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      // O is rescaled before P(j) is handed over (PV(j) follows p_full)
       if (__any_sync(0xffffffffu, need && j > 0)) {
-        wait(pv_done, (j - 1) & 1, abort_flag, a.err, 0x1501u);  // O holds PV(j-1)
+        wait(pv_done, (j - 1) & 1, abort_flag, a.err, 0x1502u);  // O holds PV(j-1)
         tc_fence_after();
-        const float alpha = need ? exp2f(m_used - mt) : 1.f;
 #pragma unroll
         for (int pc = 0; pc < 4; ++pc) {
           float ov[32];
@@ -435,35 +635,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
           tmem_st32(lane_addr + (OC - tmem) + pc * 32, ov);
         }
       }
-      if (need) {
-        l = (m_used == -INFINITY) ? 0.f : l * exp2f(m_used - mt);
-        m_used = mt;
-      }
-#pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        float sv[32];
-        tmem_ld32(lane_addr + (SC - tmem) + pc * 32, sv);
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int k0 = pc * 32 + ch * 8 + 2 * i;
-            const float p0 = k0 < nvalid ? exp2f(sv[ch * 8 + 2 * i] * c - m_used) : 0.f;
-            const float p1 = k0 + 1 < nvalid ? exp2f(sv[ch * 8 + 2 * i + 1] * c - m_used) : 0.f;
-            l += p0 + p1;
-            w[i] = pack_bf16x2(p0, p1);
-          }
-          const int e = pc * 32 + ch * 8;
-          *reinterpret_cast<uint4*>(Ps + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      fence_async_smem();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[b]);
     }
-    wait(o_done, 0, abort_flag, a.err, 0x1502u);
+    wait(o_done, 0, abort_flag, a.err, 0x1503u);
     tc_fence_after();
     const int64_t qrow = (int64_t)q0 + row;
     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -486,21 +662,47 @@ __global__ void __launch_bounds__(kThreads, 1) attend_xlayer_kernel(const __grid
 
   tc_fence_before();
   __syncthreads();
+  // no CTA leaves while a peer may still push into it or arrive on its barriers
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-template <int RC>
+template <int RC, int G, int BITS>
 static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
-  auto k = attend_xlayer_kernel<RC>;
+  auto k = attend_cluster_kernel<RC, G, BITS>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((a.n_q + 127) / 128), (unsigned)a.H);
-  k<<<grid, kThreads, kSmem, st>>>(m, a);
+  const unsigned nqt = (unsigned)((a.n_q + 127) / 128);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((nqt + CQ - 1) / CQ * CQ, (unsigned)a.H);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CQ;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, m, a);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int RC>
+static cudaError_t dispatch_gb(int group, int bits, const Maps& m, const Args& a, cudaStream_t st) {
+  if (group == 32) return bits == 2 ? launch<RC, 32, 2>(m, a, st) : launch<RC, 32, 4>(m, a, st);
+  return bits == 2 ? launch<RC, 64, 2>(m, a, st) : launch<RC, 64, 4>(m, a, st);
+}
+static cudaError_t dispatch(int rc, int group, int bits, const Maps& m, const Args& a, cudaStream_t st) {
+  if (rc == 0) return dispatch_gb<0>(group, bits, m, a, st);
+  if (rc == 1) return dispatch_gb<1>(group, bits, m, a, st);
+  return dispatch_gb<2>(group, bits, m, a, st);
 }
 
 }  // namespace attn
@@ -565,9 +767,7 @@ cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const voi
   tc::attn::Args a{err, n_q, (int64_t)T, n_self, (int)H, d->bits, d->group, scale * 1.4426950408889634f,
                    (const uint8_t*)c->k_codes, (const __half2*)c->k_params, (const uint8_t*)c->v_codes,
                    (const __half2*)c->v_params, (__nv_bfloat16*)O};
-  if (r == 0) return tc::attn::launch<0>(m, a, st);
-  if (r == 64) return tc::attn::launch<1>(m, a, st);
-  return tc::attn::launch<2>(m, a, st);
+  return tc::attn::dispatch(r == 0 ? 0 : r == 64 ? 1 : 2, d->group, d->bits, m, a, st);
 }
 
 }  // namespace kvc

@@ -203,6 +203,61 @@ __host__ __device__ constexpr uint32_t grid_pack_bias(int bits, int n) {
   return s;
 }
 
+// Packed fp32 pairs (one instruction for two lanes of work; same rounding as
+// the scalar forms).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// Dequantization of 8 codes (elements e..e+7 of a row) without shifting each
+// code down: OR-ing code field i of a 16-bit half in place into kGridMagic gives
+// kGridMagic + k * 2^(BITS * i) exactly; subtracting kGridMagic and multiplying
+// by s * 2^-(BITS * i) (exact power-of-two scalings) gives k * s, the same
+// product as k times s.  out[i] = pred[i] + (s * k_i + z).
+template <int BITS>
+__device__ __forceinline__ void dequant8(uint32_t word, int e, float s, float z, const float* pred, float* out) {
+  constexpr int PER = 16 / BITS;  // codes per 16-bit half
+  constexpr uint32_t MASK = (1u << BITS) - 1;
+  float sc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) sc[i] = s * __uint_as_float((uint32_t)(127 - BITS * i) << 23);
+  // the 16-bit halves holding codes e..e+7
+  uint32_t h[2];
+  if (BITS == 2) {
+    h[0] = h[1] = (e % 16) ? (word >> 16) : word;
+  } else {
+    h[0] = word;
+    h[1] = word >> 16;
+  }
+  const float2 zz = make_float2(z, z), mm = make_float2(-kGridMagic, -kGridMagic);
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const int i0 = i % PER, i1 = (i + 1) % PER;
+    const uint32_t s0 = h[i / PER], s1 = h[(i + 1) / PER];
+    const float2 x = make_float2(__uint_as_float(kGridMagicBits | (s0 & (MASK << (BITS * i0)))),
+                                 __uint_as_float(kGridMagicBits | (s1 & (MASK << (BITS * i1)))));
+    const float2 k = add2(x, mm);
+    const float2 d = fma2(k, make_float2(sc[i0], sc[i1]), zz);
+    const float2 r = add2(make_float2(pred[i], pred[i + 1]), d);
+    out[i] = r.x;
+    out[i + 1] = r.y;
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);

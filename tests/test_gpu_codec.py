@@ -554,7 +554,8 @@ def _oracle_codes_to_gpu(ck, cv, bits, param, assign=False):
     return buf
 
 
-@pytest.mark.parametrize("n_q,n_self,T,rank", [(300, 130, 3 * 128 + 5, 64), (129, 0, 256, 16), (64, 128, 100, 0)])
+@pytest.mark.parametrize("n_q,n_self,T,rank", [(300, 130, 3 * 128 + 5, 64), (129, 0, 256, 16), (64, 128, 100, 0),
+                                               (700, 300, 16 * 128 - 7, 64), (1100, 0, 9 * 128, 128)])
 def test_compressed_attention_cross_layer(n_q, n_self, T, rank):
     """Attention over a decoded cross-layer history plus uncompressed chunk
     tokens, history codes written by the oracle."""
