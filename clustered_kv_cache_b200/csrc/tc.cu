@@ -425,7 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     constexpr int GW = G * BITS / 32;    // code words of a group
     constexpr int XQ = G / 8;            // 16-byte words of x in a group
     constexpr bool KEEP = ENC && NP == 1;  // encode of a one-pass group keeps its prediction
-    constexpr uint32_t kBias8 = grid_pack_bias(BITS, 8);
     int use = 0;                 // uses of this group's accumulator
     int recfree = 0;             // rec_free completions consumed
     bool prev_k = false;         // the previous use of this group's tile fed Z_V
@@ -533,11 +532,11 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
               unpack_bf16x8(xc[q * 4 + ch], x, 0);
 #pragma unroll
               for (int i = 0; i < 8; i += 2) {
-                const float r0 = x[i] - p[ch * 8 + i], r1 = x[i + 1] - p[ch * 8 + i + 1];
-                mn0 = fminf(mn0, r0);
-                mx0 = fmaxf(mx0, r0);
-                mn1 = fminf(mn1, r1);
-                mx1 = fmaxf(mx1, r1);
+                const float2 r = sub2(make_float2(x[i], x[i + 1]), make_float2(p[ch * 8 + i], p[ch * 8 + i + 1]));
+                mn0 = fminf(mn0, r.x);
+                mx0 = fmaxf(mx0, r.x);
+                mn1 = fminf(mn1, r.y);
+                mx1 = fmaxf(mx1, r.y);
               }
             }
             if (KEEP) {
@@ -570,17 +569,11 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {  // 8 elements: codes, packing, reconstruction
             const int eg = q * 32 + ch * 8;  // element within the group
-            float c[8];                      // grid points
+            float r[8];  // reconstruction
             if (ENC) {
               float x[8];
               unpack_bf16x8(xc[eg / 8], x, 0);
-              uint32_t v = 0;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                c[i] = grid_point(x[i] - p[ch * 8 + i] - zf, inv, kGridMagic + (float)LEVELS);
-                v += __float_as_uint(c[i]) << (i * BITS);
-              }
-              v -= kBias8;
+              const uint32_t v = quant8<BITS>(x, &p[ch * 8], sf, zf, inv, r);
               if (BITS == 2) {
                 if ((eg % 16) == 0)
                   gw[eg / 16] = v;
@@ -590,16 +583,11 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
                 gw[eg / 8] = v;
               }
             } else {
-              const uint32_t v = BITS == 2 ? (cc[eg / 16] >> ((eg % 16) * 2)) : cc[eg / 8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) c[i] = grid_from_code((v >> (i * BITS)) & LEVELS);
+              dequant8<BITS>(BITS == 2 ? cc[eg / 16] : cc[eg / 8], eg, sf, zf, &p[ch * 8], r);
             }
             uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int k = ch * 8 + 2 * i;
-              w[i] = pack_bf16x2(p[k] + fmaf(sf, grid_code(c[2 * i]), zf), p[k + 1] + fmaf(sf, grid_code(c[2 * i + 1]), zf));
-            }
+            for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(r[2 * i], r[2 * i + 1]);
             const int e = g * G + eg;  // element of the row
             *reinterpret_cast<uint4*>(recon(b) + (e >> 6) * 16384 + sw128_off(row, (e & 63) >> 3)) =
                 make_uint4(w[0], w[1], w[2], w[3]);

@@ -111,11 +111,6 @@ __device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// arrive on a peer's mbarrier announcing `bytes` of transfer
-__device__ __forceinline__ void peer_arrive_expect(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
 // bulk copy of `bytes` from this CTA's shared memory into a peer's, completing on the peer's mbarrier
 __device__ __forceinline__ void push_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -262,6 +257,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
     mbar_init(o_done, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
+    // slots of history tiles 0 and 1 decoded elsewhere expect their pushed bytes
+    for (int j = 0; j < 2 && j < NH; ++j)
+      if (j % CQ != rank) {
+        mbar_arrive_expect_tx(&kfull[j], 32768u);
+        mbar_arrive_expect_tx(&vfull[j], 32768u);
+      }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
   }
@@ -429,6 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
         if (j < NE) {
           const int b = j & 1;
           wait(&kfull[b], (j >> 1) & 1, abort_flag, a.err, 0x1320u + b);
+          // the slot's next history tile, if a peer decodes it, will be pushed here
+          if (j + 2 < NH && (j + 2) % CQ != rank) mbar_arrive_expect_tx(&kfull[b], 32768u);
           tc_fence_after();
           if (has_q) {
             // S(j) = Q K^(j)^T into S[b]; S[b] last held P(j-2), read by PV(j-2) issued before
@@ -449,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
             // O += P(t) V^(t), P from TMEM
             wait(&p_full[b], (t >> 1) & 1, abort_flag, a.err, 0x1330u + b);
             wait(&vfull[b], (t >> 1) & 1, abort_flag, a.err, 0x1340u + b);
+            if (t + 2 < NH && (t + 2) % CQ != rank) mbar_arrive_expect_tx(&vfull[b], 32768u);
             tc_fence_after();
             const uint64_t vd = desc_mn_sw128(smem_u32(Vt(b)), 16384);
             const uint32_t idv = idesc_bf16_bmn(128, 128);
@@ -458,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
             umma_commit(pv_done);
           } else {
             wait(&vfull[b], (t >> 1) & 1, abort_flag, a.err, 0x1341u + b);
+            if (t + 2 < NH && (t + 2) % CQ != rank) mbar_arrive_expect_tx(&vfull[b], 32768u);
           }
           release(t, vfree, vt_free);
           // the decode accumulator is free once V^(t) is out: start this CTA's next tile
@@ -535,11 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
     // the tile is complete here: announce it to every peer, push it, and mark it locally
     auto publish = [&](uint8_t* tile, uint64_t* bar) {
       if (!elected) return;
+      // each peer armed its slot barrier for these bytes (see the MMA warp)
       for (int p = 1; p < CQ; ++p) {
         const uint32_t peer = (uint32_t)((rank + p) % CQ);
-        const uint32_t pb = peer_addr(bar, peer);
-        peer_arrive_expect(pb, 32768u);
-        push_to_peer(peer_addr(tile, peer), tile, 32768u, pb);
+        push_to_peer(peer_addr(tile, peer), tile, 32768u, peer_addr(bar, peer));
       }
       bulk_commit();
       mbar_arrive(bar);

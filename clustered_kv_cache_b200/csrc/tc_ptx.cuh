@@ -223,6 +223,49 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// Quantization of 8 residuals (x - pred) onto the code grid and their
+// reconstruction: rounding as grid_point (product rounded, then the integer
+// rounding by kGridMagic), clamp to [0, LEVELS]; returns the 8 packed codes
+// (code i at bits BITS * i) and writes pred + (s * k + z) to out.
+template <int BITS>
+__device__ __forceinline__ uint32_t quant8(const float* x, const float* pred, float s, float z, float inv, float* out) {
+  constexpr float top = kGridMagic + (float)((1 << BITS) - 1);
+  const float2 zz = make_float2(z, z), ss = make_float2(s, s);
+  const float2 mg = make_float2(kGridMagic, kGridMagic);
+  uint32_t v = 0;
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const float2 p = make_float2(pred[i], pred[i + 1]);
+    const float2 t = sub2(sub2(make_float2(x[i], x[i + 1]), p), zz);
+    // scalar: the packed multiply followed by the packed add did not keep the
+    // product's own rounding (exact k + 1/2 quotients then miss round-to-even)
+    const float c0 = grid_point(t.x, inv, top), c1 = grid_point(t.y, inv, top);
+    v += __float_as_uint(c0) << (i * BITS);
+    v += __float_as_uint(c1) << ((i + 1) * BITS);
+    const float2 r = add2(p, fma2(sub2(make_float2(c0, c1), mg), ss, zz));
+    out[i] = r.x;
+    out[i + 1] = r.y;
+  }
+  return v - grid_pack_bias(BITS, 8);
+}
 // Dequantization of 8 codes (elements e..e+7 of a row) without shifting each
 // code down: OR-ing code field i of a 16-bit half in place into kGridMagic gives
 // kGridMagic + k * 2^(BITS * i) exactly; subtracting kGridMagic and multiplying

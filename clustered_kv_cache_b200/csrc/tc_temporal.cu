@@ -212,8 +212,6 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
       __nv_bfloat16* rec = isv ? a.vrec : a.krec;
 #pragma unroll
-      const float top = kGridMagic + (float)levels;
-      const uint32_t bias8 = grid_pack_bias(bits, 8);
       for (int g = 0; g < NG; ++g) {
         float sf, zf;
         if (ENC) {
@@ -264,32 +262,23 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             const int e = e0 + ch * 8;
-            float c[8];  // grid points
+            float r[8];  // reconstruction
             if (ENC) {
               float x[8];
               unpack_bf16x8(xin[e / 8], x, 0);
-              uint32_t v = 0;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                c[i] = grid_point(x[i] - p[ch * 8 + i] - zf, inv, top);
-                v += __float_as_uint(c[i]) << (i * bits);
-              }
-              v -= bias8;
               if (bits == 2)
-                cw[e / 16] |= v << ((e % 16) * 2);
+                cw[e / 16] |= quant8<2>(x, &p[ch * 8], sf, zf, inv, r) << ((e % 16) * 2);
               else
-                cw[e / 8] = v;
+                cw[e / 8] = quant8<4>(x, &p[ch * 8], sf, zf, inv, r);
             } else {
-              const uint32_t v = bits == 2 ? (cwin[e / 16] >> ((e % 16) * 2)) : cwin[e / 8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) c[i] = grid_from_code((v >> (i * bits)) & levels);
+              if (bits == 2)
+                dequant8<2>(cwin[e / 16], e, sf, zf, &p[ch * 8], r);
+              else
+                dequant8<4>(cwin[e / 8], e, sf, zf, &p[ch * 8], r);
             }
             uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int k = ch * 8 + 2 * i;
-              w[i] = pack_bf16x2(p[k] + fmaf(sf, grid_code(c[2 * i]), zf), p[k + 1] + fmaf(sf, grid_code(c[2 * i + 1]), zf));
-            }
+            for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(r[2 * i], r[2 * i + 1]);
             recw[ch] = make_uint4(w[0], w[1], w[2], w[3]);
           }
           // the tile of K^_f is being read by K(f)'s MMA (lag 2) until acc_full: safe now
