@@ -351,6 +351,10 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
     cudaError_t e = tc_attend(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, ws, ws_bytes, st);
     return e == cudaSuccess ? KVC_OK : cuda_fail(e);
   }
+  if (tc_mixed_supported(d, p)) {
+    cudaError_t e = tc_mixed_attend(d, p, Q, n_q, codes, scale, O, ws, ws_bytes, st);
+    return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+  }
   Carve cv{(char*)ws, ws_bytes};
   return dispatch(d, [&](auto* ts, auto* tp) -> cudaError_t {
     using TS = std::remove_pointer_t<decltype(ts)>;

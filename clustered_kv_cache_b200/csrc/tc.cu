@@ -774,7 +774,10 @@ bool tc_codec_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
 }
 
 size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int64_t) {
-  return op == KVC_OP_ATTEND && tc_attend_supported(d, p, 0) ? tc_attend_workspace(d, p) : 0;
+  if (op != KVC_OP_ATTEND) return 0;
+  if (tc_attend_supported(d, p, 0)) return tc_attend_workspace(d, p);
+  if (tc_mixed_supported(d, p)) return tc_mixed_workspace(d);
+  return 0;
 }
 
 cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,

@@ -1,0 +1,567 @@
+// Mixed-dimensional attention over the clustered codec (tcgen05 + TMEM + TMA).
+//
+// ("NanoKV: High-Ratio KV Cache Compression for Autoregressive Video
+// Generation", abstract and the Fast variant: the score of a key is computed
+// from its cluster centre and its stored coefficients, without reconstructing
+// the full-dimension key.)  With a(t) the key's cluster, coef^ its dequantized
+// coefficients and W_dec,h the head's rows of the decoder:
+//
+//   s(q, t) = scale * (q_h . c_{a(t),h} + (q_h W_dec,h) . coef^_t)
+//           = scale * [q_h | q_h W_dec,h] . [c_{a(t),h} | coef^_t]
+//   o_h     = sum_t p_t c^V_{a_v(t),h} + W^V_dec,h (sum_t p_t coef^V_t)
+//
+// so per (128-query tile, head) the kernel is a flash attention with 256-wide
+// rows on both sides: A = [q_h | q_h W_dec,h] (its second half computed on the
+// tensor cores at the start), key tiles [centre rows | coefficients] and value
+// tiles [centre rows | coefficients]; the value product accumulates
+// [O_c | cbar] (256 TMEM columns) and the end adds cbar W^V_dec,h^T.  The sum
+// over p_t c_{a(t)} equals the oracle's sum over clusters of the per-cluster
+// mass times the centre (the same terms, grouped differently).
+//
+// The coefficients of all tokens are dequantized once per call into the
+// workspace as bf16 [T][128] (the compressed-domain representation, 1/16 of
+// the history's size), because every head and every query tile reads them.
+//
+// Warp roles: 0 TMA producer, 1 MMA issuer (TMEM owner), 2-5 prep (centre rows
+// gathered into the key / value tiles; q W_dec and cbar converted to bf16),
+// 6-9 softmax (P written over S in TMEM, lazy rescaling, final output).
+#include <cuda.h>
+#include <string.h>
+
+#include "tc.h"
+#include "tc_ptx.cuh"
+
+namespace kvc {
+namespace tc {
+
+bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
+namespace mixed {
+
+constexpr int kThreads = 320;
+// shared memory (offsets from a 1024-aligned base); each region is four [128][64] bf16 sub-tiles
+constexpr int kA = 0;              // [q_h | q_h W_dec,h]
+constexpr int kKt = kA + 65536;    // key tile [centre rows | coef]; at the start W_dec,h; at the end cbar
+constexpr int kVt = kKt + 65536;   // value tile [centre rows | coef] (MN-major B); at the end W^V_dec,h
+constexpr int kBar = kVt + 65536;
+constexpr int kSmem = kBar + 1024 + 1024;
+
+struct Maps {
+  CUtensorMap q;           // [n_q][C]
+  CUtensorMap deck, decv;  // [C][128]
+  CUtensorMap ckh, cvh;    // dequantized coefficients [T][128]
+};
+
+struct Args {
+  unsigned* err;
+  int64_t n_q, T;
+  int H, n_c;
+  float scale_log2;  // softmax scale * log2(e)
+  const __nv_bfloat16* cent_k;  // [n_c][C]
+  const __nv_bfloat16* cent_v;
+  const uint8_t* assign_k;  // [T]
+  const uint8_t* assign_v;
+  __nv_bfloat16* O;  // [n_q][H][128]
+};
+
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
+
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, float (&v)[32]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+// keeps the compiler from touching v before this point
+__device__ __forceinline__ void tie32(float (&v)[32]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]),
+                 "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait4(float (&a)[32], float (&b)[32], float (&c)[32], float (&d)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  tie32(a);
+  tie32(b);
+  tie32(c);
+  tie32(d);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]), "r"(w[9]),
+      "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+      "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
+      "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
+      "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------- coefficient dequantization
+
+// coef^ = s q + z of every token (128 coefficients, groups of G), as bf16 rows.
+template <int BITS, int G>
+__global__ void coef_dequant_kernel(const uint8_t* codes, const __half2* params, int64_t T, __nv_bfloat16* out) {
+  constexpr int RB = 128 * BITS / 8;
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  uint32_t cw[RB / 4];
+#pragma unroll
+  for (int i = 0; i < RB / 16; ++i) {
+    const uint4 w = __ldcs(reinterpret_cast<const uint4*>(codes + t * RB) + i);
+    cw[4 * i] = w.x;
+    cw[4 * i + 1] = w.y;
+    cw[4 * i + 2] = w.z;
+    cw[4 * i + 3] = w.w;
+  }
+  const float zero[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  uint4* dst = reinterpret_cast<uint4*>(out + t * 128);
+#pragma unroll
+  for (int e = 0; e < 128; e += 8) {
+    const float2 f = __half22float2(params[t * (128 / G) + e / G]);
+    float r[8];
+    dequant8<BITS>(cw[BITS == 2 ? e / 16 : e / 8], e, f.x, f.y, zero, r);
+    dst[e / 8] = make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
+                            pack_bf16x2(r[6], r[7]));
+  }
+}
+
+// ---------------------------------------------------------------- the attention kernel
+
+__global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constant__ Maps maps, const Args a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBar);
+  uint64_t* setup_full = bars;         // q_h and W_dec,h landed
+  uint64_t* qw_acc = setup_full + 1;   // q_h W_dec,h in TMEM
+  uint64_t* qw_ready = qw_acc + 1;     // ... and in the A tile as bf16 (prep)
+  uint64_t* kfull = qw_ready + 1;      // key tile complete (producer tx + 128 prep arrivals)
+  uint64_t* vfull = kfull + 1;         // value tile complete
+  uint64_t* kfree = vfull + 1;         // S(j) done: the key tile may be refilled
+  uint64_t* vfree = kfree + 1;         // PV(j) done: the value tile may be refilled
+  uint64_t* s_full = vfree + 1;        // [2]
+  uint64_t* p_full = s_full + 2;       // [2]
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* acc_done = pv_done + 1;    // the last PV finished: O_c and cbar final
+  uint64_t* cbar_ready = acc_done + 1; // cbar as bf16 in the key-tile area (prep)
+  uint64_t* dv_full = cbar_ready + 1;  // W^V_dec,h landed in the value-tile area
+  uint64_t* o_done = dv_full + 1;
+  uint64_t* mma_done = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int q0 = blockIdx.x * 128;
+  const int C = a.H * 128;
+  const int NT = (int)((a.T + 127) / 128);
+
+  if (threadIdx.x == 0) {
+    mbar_init(setup_full, 1);
+    mbar_init(qw_acc, 1);
+    mbar_init(qw_ready, 128);
+    mbar_init(kfull, 129);
+    mbar_init(vfull, 129);
+    mbar_init(kfree, 1);
+    mbar_init(vfree, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(pv_done, 1);
+    mbar_init(acc_done, 1);
+    mbar_init(cbar_ready, 128);
+    mbar_init(dv_full, 1);
+    mbar_init(o_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto SC = [&](int b) { return tmem + 128 * b; };  // S / P slots; slot 0 holds q W_dec at the start
+  const uint32_t OC = tmem + 256;                   // [O_c | cbar], 256 columns
+  uint8_t* At = smem + kA;
+  uint8_t* Kt = smem + kKt;
+  uint8_t* Vt = smem + kVt;
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+      bool ok = true;
+      mbar_arrive_expect_tx(setup_full, 65536u);
+      tma_load(At, &maps.q, h * 128, q0, setup_full, pol_stream);
+      tma_load(At + 16384, &maps.q, h * 128 + 64, q0, setup_full, pol_stream);
+      tma_load(Kt, &maps.deck, 0, h * 128, setup_full, pol_keep);  // [K = d][N = i], MN-major B
+      tma_load(Kt + 16384, &maps.deck, 64, h * 128, setup_full, pol_keep);
+      int pk = 0, pv = 0;
+      int k_armed = -1, v_armed = -1;  // last tile whose loads were issued (drained after an abort)
+      bool dv_armed = false;
+      for (int j = 0; j < NT && ok; ++j) {
+        // coefficients of the key tile, once S(j-1) (or the q W_dec product) is done with the tile
+        if (j == 0) {
+          if (!wait(qw_acc, 0, abort_flag, a.err, 0x2100u)) ok = false;
+        } else if (!wait(kfree, pk++ & 1, abort_flag, a.err, 0x2101u)) {
+          ok = false;
+        }
+        if (!ok) break;
+        mbar_arrive_expect_tx(kfull, 32768u);
+        tma_load(Kt + 32768, &maps.ckh, 0, j * 128, kfull, pol_keep);
+        tma_load(Kt + 49152, &maps.ckh, 64, j * 128, kfull, pol_keep);
+        k_armed = j;
+        if (j >= 1 && !wait(vfree, pv++ & 1, abort_flag, a.err, 0x2102u)) ok = false;
+        if (!ok) break;
+        mbar_arrive_expect_tx(vfull, 32768u);
+        tma_load(Vt + 32768, &maps.cvh, 0, j * 128, vfull, pol_keep);
+        tma_load(Vt + 49152, &maps.cvh, 64, j * 128, vfull, pol_keep);
+        v_armed = j;
+      }
+      // W^V_dec,h for the final product, once the last PV is done with the value tile
+      if (ok && wait(vfree, pv++ & 1, abort_flag, a.err, 0x2103u)) {
+        mbar_arrive_expect_tx(dv_full, 32768u);
+        tma_load(Vt, &maps.decv, 0, h * 128, dv_full, pol_keep);  // [N = d][K = i], K-major B
+        tma_load(Vt + 16384, &maps.decv, 64, h * 128, dv_full, pol_keep);
+        dv_armed = true;
+      }
+      if (*abort_flag) {
+        // the loads this thread issued land before the CTA can leave (the prep
+        // arrivals of an aborted tile may be missing, so only the bytes are awaited)
+        auto drain = [&](uint64_t* bar, uint32_t parity) {
+          const long long w0 = clock64();
+          while (!mbar_test(bar, parity) && clock64() - w0 < kWaitBudget) {
+          }
+        };
+        drain(setup_full, 0);
+        if (k_armed >= 0) drain(kfull, k_armed & 1);
+        if (v_armed >= 0) drain(vfull, v_armed & 1);
+        if (dv_armed) drain(dv_full, 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t id128 = idesc_bf16(128, 128);
+      const uint64_t ad = desc_sw128(smem_u32(At));
+      const uint64_t kd = desc_sw128(smem_u32(Kt));
+      // q W_dec,h: A = q_h (K = d), B = W_dec,h (MN-major)
+      wait(setup_full, 0, abort_flag, a.err, 0x2200u);
+      tc_fence_after();
+      {
+        const uint64_t bd = desc_mn_sw128(smem_u32(Kt), 16384);
+        const uint32_t idm = idesc_bf16_bmn(128, 128);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
+          umma(SC(0), ad + off, bd + (uint64_t)k * (2048 >> 4), idm, k == 0 ? 0u : 1u);
+        }
+        umma_commit(qw_acc);
+      }
+      wait(qw_ready, 0, abort_flag, a.err, 0x2201u);
+      tc_fence_after();
+      for (int j = 0; j <= NT; ++j) {
+        if (j < NT) {
+          const int b = j & 1;
+          // S(j) = [q | q W_dec] [centres | coef]^T, K = 256
+          wait(kfull, j & 1, abort_flag, a.err, 0x2210u);
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
+            umma(SC(b), ad + off, kd + off, id128, k == 0 ? 0u : 1u);
+          }
+          umma_commit(&s_full[b]);
+          umma_commit(kfree);
+        }
+        if (j >= 1) {
+          const int t = j - 1, b = t & 1;
+          // [O_c | cbar] += P(t) [centres | coef], N = 256, P from TMEM
+          wait(&p_full[b], (t >> 1) & 1, abort_flag, a.err, 0x2220u + b);
+          wait(vfull, t & 1, abort_flag, a.err, 0x2230u);
+          tc_fence_after();
+          const uint64_t vd = desc_mn_sw128(smem_u32(Vt), 16384);
+          const uint32_t idv = idesc_bf16_bmn(128, 256);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_ts(OC, SC(b) + k * 8, vd + (uint64_t)k * (2048 >> 4), idv, (t == 0 && k == 0) ? 0u : 1u);
+          umma_commit(pv_done);
+          umma_commit(vfree);
+        }
+      }
+      umma_commit(acc_done);
+      // O_c += cbar W^V_dec,h^T
+      wait(cbar_ready, 0, abort_flag, a.err, 0x2240u);
+      wait(dv_full, 0, abort_flag, a.err, 0x2241u);
+      tc_fence_after();
+      {
+        const uint64_t cd = desc_sw128(smem_u32(Kt));
+        const uint64_t dd = desc_sw128(smem_u32(Vt));
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
+          umma(OC, cd + off, dd + off, id128, 1u);
+        }
+      }
+      umma_commit(o_done);
+      umma_commit(mma_done);
+      const long long w0 = clock64();
+      while (!mbar_test(mma_done, 0) && clock64() - w0 < kWaitBudget) {
+      }
+    }
+  } else if (warp < 6) {
+    // ================================================================ prep (warps 2-5)
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;  // key row of a tile, or query row (TMEM lane) for conversions
+    const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16);
+    // 128 fp32 TMEM columns of this lane -> bf16 row of a K-major pair of sub-tiles
+    auto to_bf16 = [&](uint32_t col, uint8_t* tile) {
+      float v[4][32];
+      tmem_ld32_async(lane_addr + (col - tmem), v[0]);
+      tmem_ld32_async(lane_addr + (col - tmem) + 32, v[1]);
+      tmem_ld32_async(lane_addr + (col - tmem) + 64, v[2]);
+      tmem_ld32_async(lane_addr + (col - tmem) + 96, v[3]);
+      tmem_ld_wait4(v[0], v[1], v[2], v[3]);
+#pragma unroll
+      for (int c16 = 0; c16 < 16; ++c16) {
+        const float* x = &v[c16 / 4][(c16 % 4) * 8];
+        *reinterpret_cast<uint4*>(tile + (c16 / 8) * 16384 + sw128_off(row, c16 % 8)) =
+            make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                       pack_bf16x2(x[6], x[7]));
+      }
+      tc_fence_before();
+      fence_async_smem();
+    };
+    // the head's 128 channels of the centre of this row's key into sub-tiles 0, 1 of `tile`
+    auto gather = [&](const __nv_bfloat16* cent, const uint8_t* assign, int j, uint8_t* tile) {
+      const int64_t t = (int64_t)j * 128 + row;
+      int c = t < a.T ? (int)assign[t] : 0;
+      c = c < a.n_c ? c : a.n_c - 1;
+      const uint4* src = reinterpret_cast<const uint4*>(cent + (int64_t)c * C + h * 128);
+      uint4 w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) w[i] = __ldg(src + i);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) *reinterpret_cast<uint4*>(tile + (i / 8) * 16384 + sw128_off(row, i % 8)) = w[i];
+      fence_async_smem();
+    };
+    wait(qw_acc, 0, abort_flag, a.err, 0x2300u);
+    tc_fence_after();
+    to_bf16(SC(0), At + 32768);
+    mbar_arrive(qw_ready);
+    int pk = 0, pv = 0;
+    for (int j = 0; j < NT; ++j) {
+      if (j >= 1) wait(kfree, pk++ & 1, abort_flag, a.err, 0x2301u);
+      gather(a.cent_k, a.assign_k, j, Kt);
+      mbar_arrive(kfull);
+      if (j >= 1) wait(vfree, pv++ & 1, abort_flag, a.err, 0x2302u);
+      gather(a.cent_v, a.assign_v, j, Vt);
+      mbar_arrive(vfull);
+    }
+    // cbar (TMEM) -> bf16 A operand in the key-tile area, once every S and PV is done
+    wait(acc_done, 0, abort_flag, a.err, 0x2303u);
+    tc_fence_after();
+    to_bf16(OC + 128, Kt);
+    mbar_arrive(cbar_ready);
+  } else {
+    // ================================================================ softmax (warps 6-9)
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;  // query row
+    const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16);
+    const float c = a.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    for (int j = 0; j < NT; ++j) {
+      const int b = j & 1;
+      const uint32_t sc = lane_addr + (SC(b) - tmem);
+      wait(&s_full[b], (j >> 1) & 1, abort_flag, a.err, 0x2400u + b);
+      tc_fence_after();
+      const int64_t kbase = (int64_t)j * 128;
+      const int nvalid = a.T - kbase < 128 ? (int)(a.T - kbase) : 128;
+      float sv[4][32];
+      tmem_ld32_async(sc, sv[0]);
+      tmem_ld32_async(sc + 32, sv[1]);
+      tmem_ld32_async(sc + 64, sv[2]);
+      tmem_ld32_async(sc + 96, sv[3]);
+      tmem_ld_wait4(sv[0], sv[1], sv[2], sv[3]);
+      if (nvalid < 128) {
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (pc * 32 + i >= nvalid) sv[pc][i] = -INFINITY;
+      }
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], sv[pc][i]);
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+      // lazy rescale: only when the tile's max exceeds the one in use by 2^8
+      const bool need = mt > m_used + 8.f;
+      float alpha = 1.f;
+      if (need) {
+        alpha = m_used == -INFINITY ? 0.f : ex2_approx(m_used - mt);
+        l *= alpha;
+        m_used = mt;
+      }
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(sv[pc][2 * i], c, -m_used));
+          const float p1 = ex2_approx(fmaf(sv[pc][2 * i + 1], c, -m_used));
+          ls[i & 3] += p0 + p1;
+          w[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(sc + pc * 16, w);
+      }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      // O (both halves) is rescaled before P(j) is handed over
+      if (__any_sync(0xffffffffu, need && j > 0)) {
+        wait(pv_done, (j - 1) & 1, abort_flag, a.err, 0x2401u);
+        tc_fence_after();
+#pragma unroll
+        for (int pc = 0; pc < 8; ++pc) {
+          float ov[32];
+          tmem_ld32(lane_addr + (OC - tmem) + pc * 32, ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          tmem_st32(lane_addr + (OC - tmem) + pc * 32, ov);
+        }
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    wait(o_done, 0, abort_flag, a.err, 0x2402u);
+    tc_fence_after();
+    const int64_t qrow = (int64_t)q0 + row;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int pc = 0; pc < 4; ++pc) {
+      float ov[32];
+      tmem_ld32(lane_addr + (OC - tmem) + pc * 32, ov);
+      if (qrow < a.n_q) {
+        uint4* dst = reinterpret_cast<uint4*>(a.O + (qrow * a.H + h) * 128 + pc * 32);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(ov[ch * 8 + 2 * i] * inv, ov[ch * 8 + 2 * i + 1] * inv);
+          dst[ch] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace mixed
+}  // namespace tc
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool tc_mixed_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
+  if (p->kind != KVC_PRED_CLUSTER) return false;
+  if (d->dtype != KVC_BF16 || d->head_dim != 128 || d->param_dtype != KVC_F16) return false;
+  if (d->bits != 2 && d->bits != 4) return false;
+  if (d->group != 32 && d->group != 64) return false;
+  if (p->code_dim != 128 || p->n_clusters < 1 || p->n_clusters > 256) return false;
+  if (d->n_tokens < 1 || (int64_t)d->n_heads * 128 * 2 > (1 << 20)) return false;
+  return true;
+}
+
+size_t tc_mixed_workspace(const kvc_layer_desc* d) { return 2 * align256((size_t)d->n_tokens * 128 * 2); }
+
+cudaError_t tc_mixed_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
+                            const kvc_codes* c, float scale, void* O, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128;
+  if (ws_bytes < tc_mixed_workspace(d)) return cudaErrorInvalidValue;
+  __nv_bfloat16* ckh = static_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* cvh = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + align256(T * 128 * 2));
+  // dequantized coefficients of every token
+  {
+    const unsigned blocks = (unsigned)((T + 127) / 128);
+    auto k = d->bits == 2 ? (d->group == 32 ? tc::mixed::coef_dequant_kernel<2, 32> : tc::mixed::coef_dequant_kernel<2, 64>)
+                          : (d->group == 32 ? tc::mixed::coef_dequant_kernel<4, 32> : tc::mixed::coef_dequant_kernel<4, 64>);
+    k<<<blocks, 128, 0, st>>>((const uint8_t*)c->k_codes, (const __half2*)c->k_params, (int64_t)T, ckh);
+    k<<<blocks, 128, 0, st>>>((const uint8_t*)c->v_codes, (const __half2*)c->v_params, (int64_t)T, cvh);
+    count_launches(2);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  tc::mixed::Maps m;
+  memset(&m, 0, sizeof(m));
+  bool ok = tc::map2d(&m.q, Q, (uint64_t)n_q, C, 128) && tc::map2d(&m.deck, p->k_dec, C, 128, 128) &&
+            tc::map2d(&m.decv, p->v_dec, C, 128, 128) && tc::map2d(&m.ckh, ckh, T, 128, 128) &&
+            tc::map2d(&m.cvh, cvh, T, 128, 128);
+  if (!ok) return cudaErrorInvalidValue;
+  unsigned* err = tc_error_word();
+  if (!err) return cudaErrorInvalidDevice;
+  tc::mixed::Args a{err, n_q, (int64_t)T, (int)H, p->n_clusters, scale * 1.4426950408889634f,
+                    (const __nv_bfloat16*)p->k_centroids, (const __nv_bfloat16*)p->v_centroids,
+                    (const uint8_t*)c->k_assign, (const uint8_t*)c->v_assign, (__nv_bfloat16*)O};
+  auto k = tc::mixed::mixed_kernel;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::mixed::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((n_q + 127) / 128), (unsigned)H);
+  k<<<grid, tc::mixed::kThreads, tc::mixed::kSmem, st>>>(m, a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc
