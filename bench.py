@@ -42,6 +42,13 @@ METRIC = "KV tokens/s encoded+decoded (GB/s vs HBM peak); compressed-attn TFLOP/
 UNIT = "KV tokens/s"
 
 
+# DRAM bytes (read + write) per launch, from the ncu captures summarised under
+# profiles/ (codec_xlayer_wan_layer.md, attention_cluster_wan.md,
+# mixed_attention_cluster.md); set to None when a kernel changes after its capture.
+TRAFFIC = {"encode_xlayer": 697936128 + 187771136, "decode_xlayer": 490159360 + 148607744,
+           "attention_c2": 769948672 + 8668416, "attention_c4": 26633216 + 512}
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -277,7 +284,7 @@ def row_attention(xb: XLayerBench, hbm, tf_burst, tf_sust, reps=3) -> dict:
     return {"workload": "4680 queries x (32760 compressed + 4680 chunk) keys, 12 heads x 128, layer 15",
             "ms": ms, "value": tflops, "unit": "TFLOP/s (attention + one in-kernel decode of the history)",
             "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_burst, "unit": "TFLOP/s",
-                         "frac": tflops / tf_burst, "traffic": None, "peak_kind": "burst bf16"}}
+                         "frac": tflops / tf_burst, "traffic": TRAFFIC["attention_c2"], "peak_kind": "burst bf16"}}
 
 
 def row_temporal(dev, hbm, reps=3) -> dict:
@@ -354,7 +361,7 @@ def row_cluster(dev, hbm, tf_burst, reps=3) -> dict:
             byts = 2 * T * C * 2 + kvc.kvc_codes_bytes(desc, pred)
             gbs = byts / (ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
-        roof["traffic"] = None
+        roof["traffic"] = TRAFFIC["attention_c4"] if name == "attention" else None
         out[name] = {"ms": ms, "roofline": roof}
     return out
 
@@ -445,7 +452,8 @@ def main():
     enc_gbs, dec_gbs = enc_b / (enc_ms * 1e-3) / 1e9, dec_b / (dec_ms * 1e-3) / 1e9
     dom_enc = enc_ms >= dec_ms
     roof = {"bound": "hbm", "achieved": enc_gbs if dom_enc else dec_gbs, "peak": hbm, "unit": "GB/s",
-            "frac": (enc_gbs if dom_enc else dec_gbs) / hbm, "traffic": None,
+            "frac": (enc_gbs if dom_enc else dec_gbs) / hbm,
+            "traffic": TRAFFIC["encode_xlayer"] if dom_enc else TRAFFIC["decode_xlayer"],
             "kernel": "kvc_encode_layer (cross-layer, one layer)" if dom_enc else
                       "kvc_decode_layer (cross-layer, one layer)",
             "bytes_per_launch": enc_b if dom_enc else dec_b, "ms_per_launch": enc_ms if dom_enc else dec_ms,

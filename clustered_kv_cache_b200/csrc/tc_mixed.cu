@@ -378,19 +378,23 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
       tc_fence_before();
       fence_async_smem();
     };
-    // the head's 128 channels of the centre of this row's key into sub-tiles 0, 1 of `tile`
-    auto gather = [&](const __nv_bfloat16* cent, const uint8_t* assign, int j, uint8_t* tile) {
+    // the head's 128 channels of the centre of this row's key, fetched ahead of
+    // the wait for the tile, then stored into sub-tiles 0, 1 of it
+    auto fetch_rows = [&](const __nv_bfloat16* cent, const uint8_t* assign, int j, uint4 (&w)[16]) {
       const int64_t t = (int64_t)j * 128 + row;
       int c = t < a.T ? (int)assign[t] : 0;
       c = c < a.n_c ? c : a.n_c - 1;
       const uint4* src = reinterpret_cast<const uint4*>(cent + (int64_t)c * C + h * 128);
-      uint4 w[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) w[i] = __ldg(src + i);
+    };
+    auto store_rows = [&](const uint4 (&w)[16], uint8_t* tile) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) *reinterpret_cast<uint4*>(tile + (i / 8) * 16384 + sw128_off(row, i % 8)) = w[i];
       fence_async_smem();
     };
+    uint4 wk[16], wv[16];
+    fetch_rows(a.cent_k, a.assign_k, 0, wk);
     wait(qw_acc, 0, abort_flag, a.err, 0x2300u);
     tc_fence_after();
     to_bf16(SC(0), At + 32768);
@@ -398,11 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
     int pk = 0, pv = 0;
     for (int j = 0; j < NT; ++j) {
       if (j >= 1) wait(kfree, pk++ & 1, abort_flag, a.err, 0x2301u);
-      gather(a.cent_k, a.assign_k, j, Kt);
+      store_rows(wk, Kt);
       mbar_arrive(kfull);
+      fetch_rows(a.cent_v, a.assign_v, j, wv);
       if (j >= 1) wait(vfree, pv++ & 1, abort_flag, a.err, 0x2302u);
-      gather(a.cent_v, a.assign_v, j, Vt);
+      store_rows(wv, Vt);
       mbar_arrive(vfull);
+      if (j + 1 < NT) fetch_rows(a.cent_k, a.assign_k, j + 1, wk);
     }
     // cbar (TMEM) -> bf16 A operand in the key-tile area, once every S and PV is done
     wait(acc_done, 0, abort_flag, a.err, 0x2303u);
