@@ -194,6 +194,20 @@ cudaError_t codec_cluster(const kvc_layer_desc* d, const kvc_predictor* p, bool 
       ClusterPrepArgs<TS> pa{nc, C, m, cent, encw, cn, P};
       if ((e = launch_cluster_prep(pa, st)) != cudaSuccess) return e;
     }
+    if constexpr (std::is_same<TS, __nv_bfloat16>::value && std::is_same<TP, __half>::value) {
+      if (tc_cluster_supported(d, p)) {
+        void* codes = which ? c->v_codes : c->k_codes;
+        void* params = which ? c->v_params : c->k_params;
+        void* assign = which ? c->v_assign : c->k_assign;
+        void* rec = which ? Vr : Kr;
+        if (enc && (e = tc_cluster_encode(d, p, which ? V : K, cent, encw, cn, P, codes, params, assign, st)) !=
+                       cudaSuccess)
+          return e;
+        // the encode's reconstruction is the decode of what it wrote, so the two agree bit for bit
+        if (rec && (e = tc_cluster_decode(d, p, codes, params, assign, cent, dec, rec, st)) != cudaSuccess) return e;
+        continue;
+      }
+    }
     ClusterArgs<TS, TP> a{d->n_tokens, C, m, nc, d->bits, d->group, (const TS*)(which ? V : K), cent, encw, dec,
                           cn, P, (uint8_t*)(which ? c->v_codes : c->k_codes),
                           (Pair<TP>*)(which ? c->v_params : c->k_params),

@@ -22,6 +22,12 @@ bool tc_mixed_supported(const kvc_layer_desc* d, const kvc_predictor* p);
 size_t tc_mixed_workspace(const kvc_layer_desc* d);
 cudaError_t tc_mixed_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
                             const kvc_codes* c, float scale, void* O, void* ws, size_t ws_bytes, cudaStream_t st);
+bool tc_cluster_supported(const kvc_layer_desc* d, const kvc_predictor* p);
+cudaError_t tc_cluster_encode(const kvc_layer_desc* d, const kvc_predictor* p, const void* X, const void* cent,
+                              const void* enc, const float* cnorm, float* P, void* codes, void* params,
+                              void* assign, cudaStream_t st);
+cudaError_t tc_cluster_decode(const kvc_layer_desc* d, const kvc_predictor* p, const void* codes, const void* params,
+                              const void* assign, const void* cent, const void* dec, void* out, cudaStream_t st);
 // reads the device error word of the current device and resets it to 0
 cudaError_t tc_read_and_clear_error(unsigned int* value);
 // device address of the error word on the current device (nullptr on failure)

@@ -495,7 +495,7 @@ def _cluster_pred(cw: synth.ClusterWorkload, n_c):
     return kvc.make_predictor(kvc.PRED_CLUSTER, w, n_clusters=n_c, code_dim=cw.k_enc.shape[0])
 
 
-@pytest.mark.parametrize("T,H,n_c", [(1000, 4, 32), (300, 16, 256)])
+@pytest.mark.parametrize("T,H,n_c", [(1000, 4, 32), (300, 16, 256), (2000 - 5, 16, 256)])
 def test_cluster_codec_parity(T, H, n_c):
     cw = synth.cluster_layer(seed=synth.SEED_BASE + 104, T=T, H=H, n_c=n_c, iters=5)
     D = 128

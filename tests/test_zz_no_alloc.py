@@ -5,7 +5,9 @@ callbacks, runtimes that hand out pre-carved memory, plugin hosts that forbid
 cudaMalloc).  kvc_encode_layer_cluster_static serves them from a static device
 array inside the library.  Its results must match kvc_encode_layer's within the
 tolerances of the other parity tests, on consecutive calls (the array is shared
-and keeps the previous call's contents).  This file is collected last.
+and keeps the previous call's contents); the reconstructions may differ by one
+bf16 step where the two kernels' fp32 sums round across a boundary.  This file
+is collected last.
 """
 
 import ctypes
@@ -67,4 +69,13 @@ def test_static_scratch_encode_matches_workspace_encode_twice():
             r_s, r_r = U.to64(rec_s), U.to64(rec_r)
             tol = 1e-3 * (np.abs(U.to64(X)) + 1.0)
             flip = np.repeat((q_s != q_r).any(axis=1), H * D).reshape(T, H, D)
-            assert np.all((np.abs(r_s - r_r) <= tol) | flip), f"call {call} {which} recon"
+            # The static entry point runs the CUDA-core kernels and kvc_encode_layer the
+            # tensor-core ones: the same products summed in another fp32 order, so where
+            # the exact value sits next to a bf16 rounding boundary the two round to
+            # adjacent bf16 values.  One such step is accepted, rarely.
+            mag = np.maximum(np.abs(r_s), np.abs(r_r))
+            ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - 7)
+            diff = np.abs(r_s - r_r)
+            one_step = (diff > tol) & (diff <= ulp * 1.0001)
+            assert np.all((diff <= tol) | one_step | flip), f"call {call} {which} recon"
+            assert one_step.mean() < 1e-2, f"call {call} {which} recon: {one_step.mean()} one-step differences"
