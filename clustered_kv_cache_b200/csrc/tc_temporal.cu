@@ -141,9 +141,11 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       };
       if (cont && ok) issue_k(0);
       for (int f = 0; f < nf && ok; ++f) {
-        // K^_f is needed by V(f) and K(f+1)
+        // K^_f is needed by K(f+1) and V(f); K(f+1) goes first, it is the next link
+        // of the K chain, while V(f) may still wait for V^_{f-1}
         if (!wait(kready, kr++ & 1, abort_flag, a.err, 0x2110u)) ok = false;
         tc_fence_after();
+        if (ok && f + 1 < nf) issue_k(f + 1);
         if (ok && (f > 0 || cont)) {  // the anchor frame has no prediction
           // V(f) reads V^_{f-1}: wait for its epilogue unless it is the supplied history
           if (f > 0 && !wait(vready, vr++ & 1, abort_flag, a.err, 0x2111u)) ok = false;
@@ -153,7 +155,6 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
             umma_commit(vacc_full);
           }
         }
-        if (ok && f + 1 < nf) issue_k(f + 1);
       }
       umma_commit(mma_done);
       const long long w0 = clock64();
