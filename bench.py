@@ -45,7 +45,7 @@ UNIT = "KV tokens/s"
 # DRAM bytes (read + write) per launch, from the ncu captures summarised under
 # profiles/ (codec_xlayer_wan_layer.md, attention_cluster_wan.md,
 # mixed_attention_cluster.md); set to None when a kernel changes after its capture.
-TRAFFIC = {"encode_xlayer": 697936128 + 187771136, "decode_xlayer": 490159360 + 148607744,
+TRAFFIC = {"encode_xlayer": None, "decode_xlayer": None,
            "attention_c2": 769948672 + 8668416, "attention_c4": 26633216 + 512}
 
 
@@ -255,6 +255,15 @@ def run_reference(args, rank: int):
 # ---------------------------------------------------------------- extra rows (N = 1)
 
 
+def synced_ok():
+    """Waits for the device and fails on a kernel-reported error (an expired
+    wait, a bad launch): a timing of such a run is no measurement."""
+    torch.cuda.synchronize()
+    err = kvc.kvc_get_device_error()
+    if err:
+        raise RuntimeError(f"device error word 0x{err:x} after a timed row")
+
+
 def row_attention(xb: XLayerBench, hbm, tf_burst, tf_sust, reps=3) -> dict:
     """4680 queries (3 latent frames) over layer 15's compressed history plus the
     chunk itself; the history is decoded inside the attention kernel."""
@@ -276,7 +285,7 @@ def row_attention(xb: XLayerBench, hbm, tf_burst, tf_sust, reps=3) -> dict:
         s.record()
         call()
         e.record()
-    torch.cuda.synchronize()
+    synced_ok()
     ms = statistics.median(time_events(ev))
     attn_flops = 4 * n_q * (T_TOK + n_q) * H * D
     total = attn_flops + XLayerBench.layer_flops()
@@ -305,7 +314,7 @@ def row_temporal(dev, hbm, reps=3) -> dict:
             s.record()
             fn()
             e.record()
-        torch.cuda.synchronize()
+        synced_ok()
         ms = statistics.median(time_events(ev))
         codes = kvc.kvc_codes_bytes(desc, pred)
         byts = 2 * T * Hh * Dd * 2 + codes + 2 * tw.ak.numel() * 2
@@ -346,7 +355,7 @@ def row_cluster(dev, hbm, tf_burst, reps=3) -> dict:
             s.record()
             fn()
             e.record()
-        torch.cuda.synchronize()
+        synced_ok()
         ms = statistics.median(time_events(ev))
         C = Hh * Dd
         if name == "attention":

@@ -93,13 +93,14 @@ struct Args {
 
 template <int RC>
 struct Layout {
-  static constexpr int S = RC == 2 ? 3 : 4;  // pipeline stages
-  static constexpr int kStage = 32768;        // A 16 KB + B 16 KB
-  static constexpr int kRecon = 32768;        // [128][128] bf16 as two 64-column sub-tiles
+  static constexpr int S = 4;           // pipeline stages (the latent lives in TMEM, not here)
+  static constexpr int kStage = 32768;  // A 16 KB + B 16 KB
+  static constexpr int kRecon = 32768;  // [128][128] bf16 as two 64-column sub-tiles
+  static constexpr int kIn = 128;       // staged epilogue inputs: bytes per epilogue thread
   static constexpr int kStageOff = 0;
   static constexpr int kReconOff = S * kStage;
-  static constexpr int kZOff = kReconOff + 2 * kRecon;  // latent hi / lo sub-tiles
-  static constexpr int kBarOff = kZOff + RC * 2 * 16384;
+  static constexpr int kInOff = kReconOff + 2 * kRecon;
+  static constexpr int kBarOff = kInOff + 256 * kIn;
   static constexpr int kBytes = kBarOff + 1024;
 };
 
@@ -177,8 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   auto stageA = [&](int s) { return smem + L::kStageOff + s * L::kStage; };
   auto stageB = [&](int s) { return smem + L::kStageOff + s * L::kStage + 16384; };
   auto recon = [&](int b) { return smem + L::kReconOff + b * L::kRecon; };
-  auto zhi = [&](int j) { return smem + L::kZOff + j * 16384; };
-  auto zlo = [&](int j) { return smem + L::kZOff + (RC + j) * 16384; };
+  const uint32_t in_base = smem_u32(smem + L::kInOff);
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -354,17 +354,28 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           recf[rb]++;
           commit(&rec_free[rb]);
         };
-        // the latent factor of a head: acc += [Z hi | Z lo] U^T
-        auto lowrank = [&](int b, bool first_head, unsigned where) {
+        // the latent factor of a head: acc += [Z hi | Z lo] U^T, Z as bf16 pairs in TMEM
+        // (64 rank columns per chunk i: hi pairs at +0, lo pairs at +32)
+        auto lowrank = [&](int b, uint32_t zcol, bool first_head, unsigned where) {
           group(
               RC, [&] { if (first_head) wt(z_ready, zr & 1, where); },
-              [&](int i, int st) { issue(st, acc_col[b], 128, false, zhi(i), zlo(i)); });
+              [&](int i, int st) {
+                if (!ISSUE) return;
+                const uint32_t idesc = idesc_bf16(128, 128);
+                const uint64_t bd = desc_sw128(smem_u32(stageB(st)));
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  umma_ts_if(lead, acc_col[b], zcol + i * 64 + k * 8, bd + 2 * k, idesc, 1u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  umma_ts_if(lead, acc_col[b], zcol + i * 64 + 32 + k * 8, bd + 2 * k, idesc, 1u);
+              });
           if (first_head) zr++;
         };
         for (int h = 0; h < H; ++h) {
           const int b = (it * HH + h) & 1;
           group(2, [&] { acq(b); }, [&](int i, int st) { issue(st, acc_col[b], 128, i == 0, nullptr, nullptr); });
-          if (RC) lowrank(b, h == 0, 0x600u);
+          if (RC) lowrank(b, zk, h == 0, 0x600u);
           commit(&acc_full[b]);
           use[b]++;
           // two heads behind, so that the epilogue of head h-2 is long done
@@ -376,13 +387,20 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           for (int g = H >= 2 ? H - 2 : 0; g < H; ++g) zva(g);
           commit(zv_full);
         }
+        if (LAT && RC && has_next) {
+          // No V head reads the V latent here, so its conversion is waited for
+          // before the next tile's latent MMAs overwrite it; this also keeps
+          // one z_ready phase consumed per conversion.
+          group(0, [&] { wt(z_ready, zr & 1, 0x602u); }, [](int, int) {});
+          zr++;
+        }
         if (!LAT) {
           for (int h = 0; h < H; ++h) {
             const int b = (it * HH + H + h) & 1;
             // V^_{l-1,h} part first (chunks 2, 3 of BV_h), then K^_{l,h} (chunks 0, 1)
             group(2, [&] { acq(b); }, [&](int i, int st) { issue(st, acc_col[b], 128, i == 0, nullptr, nullptr); });
             group(2, nop, [&](int i, int st) { issue(st, acc_col[b], 128, false, nullptr, nullptr); });
-            if (RC) lowrank(b, h == 0, 0x601u);
+            if (RC) lowrank(b, zv, h == 0, 0x601u);
             commit(&acc_full[b]);
             use[b]++;
             if (OVL && has_next)
@@ -436,44 +454,56 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         asm volatile("bar.sync 2, 128;" ::: "memory");
     };
 
-    auto convert_latent = [&](uint32_t col, int t0, __nv_bfloat16* ghi, __nv_bfloat16* glo) {  // TMEM -> bf16 hi / lo
+    // fp32 latent in TMEM -> bf16 hi / lo pairs written back over it (per 64 rank
+    // columns: 32 columns of hi pairs, then 32 of lo pairs), the A operand of the
+    // low-rank MMAs
+    auto convert_latent = [&](uint32_t col, int t0, __nv_bfloat16* ghi, __nv_bfloat16* glo) {
       const int64_t t = (int64_t)t0 + row;
       const bool valid = t < a.T;
-      for (int p = 0; p < R / 32; ++p) {
-        const int c0 = p * 32;  // latent column
-        float v[32];
-        tmem_ld32(lane_addr + (col - tmem) + c0, v);
-        uint8_t* hi = zhi(c0 / 64);
-        uint8_t* lo = zlo(c0 / 64);
+      for (int j = 0; j < RC; ++j) {
+        const uint32_t base = lane_addr + (col - tmem) + j * 64;
+        float v[2][32];
+        tmem_ld32(base, v[0]);
+        tmem_ld32(base + 32, v[1]);
+        uint32_t wh[32], wl[32];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t wh[4], wl[4];
+        for (int i = 0; i < 32; ++i) {
+          const float x0 = v[i / 16][(2 * i) % 32], x1 = v[i / 16][(2 * i + 1) % 32];
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
+          const float2 hf = __bfloat1622float2(h2);
+          wh[i] = *reinterpret_cast<const uint32_t*>(&h2);
+          wl[i] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
+        }
+        tmem_st32u(base, wh);
+        tmem_st32u(base + 32, wl);
+        if (LAT && valid) {
+          uint4* gh = reinterpret_cast<uint4*>(ghi + t * R + j * 64);
+          uint4* gl = reinterpret_cast<uint4*>(glo + t * R + j * 64);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float x0 = v[ch * 8 + 2 * i], x1 = v[ch * 8 + 2 * i + 1];
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
-            const float2 hf = __bfloat1622float2(h2);
-            wh[i] = *reinterpret_cast<const uint32_t*>(&h2);
-            wl[i] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
-          }
-          const int c16 = ((c0 % 64) >> 3) + ch;
-          *reinterpret_cast<uint4*>(hi + sw128_off(row, c16)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          *reinterpret_cast<uint4*>(lo + sw128_off(row, c16)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-          if (LAT && valid) {
-            reinterpret_cast<uint4*>(ghi + t * R + c0)[ch] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-            reinterpret_cast<uint4*>(glo + t * R + c0)[ch] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+          for (int i = 0; i < 8; ++i) {
+            gh[i] = make_uint4(wh[4 * i], wh[4 * i + 1], wh[4 * i + 2], wh[4 * i + 3]);
+            gl[i] = make_uint4(wl[4 * i], wl[4 * i + 1], wl[4 * i + 2], wl[4 * i + 3]);
           }
         }
       }
       tc_fence_before();
-      fence_async_smem();
       mbar_arrive(z_ready);
     };
 
+    // Global inputs of a head reach a per-thread slot of shared memory by the
+    // thread's own asynchronous copies, issued before the accumulator wait, so
+    // their latency overlaps the MMAs.  A slot is 8 chunks of 16 bytes, swizzled
+    // by row so that a warp's 16-byte reads are free of bank conflicts.  Decode:
+    // the row's code words (chunks 0 ..) and its (scale, zero) pairs (chunk 4).
+    // Encode with 32-element groups: x of two groups in flight (chunks 0-3 and
+    // 4-7, group g in half g & 1); wider groups fetch x into registers.
+    constexpr bool STX = ENC && G == 32;
+    const uint32_t slot = in_base + (uint32_t)(grp * 128 + row) * L::kIn;
+    auto chunk = [&](int c) { return slot + (((uint32_t)c ^ (uint32_t)(row & 7)) << 4); };
+
     // one head of this group: h its index, is_v K or V, t0 the tile.  The
     // groups of the row are processed by a rolled loop (the kernel's code must
-    // stay small enough for the instruction caches); the global inputs of group
-    // g+1 are fetched while group g is worked on.
+    // stay small enough for the instruction caches).
     auto head = [&](int h, bool is_v, int t0) {
       const int b = grp;
       const int64_t t = (int64_t)t0 + row;
@@ -486,21 +516,52 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       uint4 xc[ENC ? XQ : 1];
       uint32_t cc[ENC ? 1 : GW];
       __half2 pc = __floats2half2_rn(0.f, 0.f);
+      auto stage_x = [&](int g) {
+#pragma unroll
+        for (int i = 0; i < XQ; ++i)
+          cp_async16(chunk((g & 1) * XQ + i), valid ? (const void*)(X + g * XQ + i) : (const void*)a.xk,
+                     valid ? 16u : 0u);
+        cp_async_commit();
+      };
+      if (STX) {
+        stage_x(0);
+        if (NG > 1) stage_x(1);
+      }
+      if (!ENC) {  // rows past T copy nothing and read zeros (source: the buffers' first bytes)
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(codes);
+        const void* c0 = is_v ? a.vcodes : a.kcodes;
+        const __half2* p0 = is_v ? a.vparams : a.kparams;
+#pragma unroll
+        for (int i = 0; i < RB / 16; ++i) cp_async16(chunk(i), valid ? (const void*)(src + 16 * i) : c0, valid ? 16u : 0u);
+        if (G == 32) {
+          cp_async16(chunk(4), valid ? params : p0, valid ? 16u : 0u);
+        } else {
+#pragma unroll
+          for (int i = 0; i < NG; ++i) cp_async4(chunk(4) + 4 * i, valid ? params + i : p0, valid ? 4u : 0u);
+        }
+        cp_async_commit();
+      }
+      // group g's inputs into registers (from the slot, or from global memory)
       auto fetch = [&](int g, uint4 (&xo)[ENC ? XQ : 1], uint32_t (&co)[ENC ? 1 : GW], __half2& po) {
-        if (ENC) {
+        if (STX) {
+#pragma unroll
+          for (int i = 0; i < XQ; ++i) xo[i] = lds128(chunk((g & 1) * XQ + i));
+        } else if (ENC) {
 #pragma unroll
           for (int i = 0; i < XQ; ++i) xo[i] = valid ? __ldcs(X + g * XQ + i) : make_uint4(0, 0, 0, 0);
         } else {
 #pragma unroll
           for (int i = 0; i < GW; i += 2) {
-            const uint2 w = valid ? __ldcs(reinterpret_cast<const uint2*>(codes + g * GW + i)) : make_uint2(0, 0);
+            const int wi = g * GW + i;  // code word of the row
+            const uint2 w = lds64(chunk(wi / 4) + (wi % 4) * 4);
             co[i] = w.x;
             co[i + 1] = w.y;
           }
-          po = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
+          const uint32_t pw = lds32(chunk(4) + 4 * g);
+          po = *reinterpret_cast<const __half2*>(&pw);
         }
       };
-      fetch(0, xc, cc, pc);
+      if (ENC && !STX) fetch(0, xc, cc, pc);
       // the reconstruction tile is free once its previous TMA store has read it
       // and, if it held a K head, the MMA of Z_V has consumed it
       if (elected) bulk_wait_read0();
@@ -510,13 +571,25 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       if (RC && prev_k) wait(&rec_free[b], recfree++ & 1, abort_flag, a.err, 0x700u + b);
       prev_k = !is_v && RC;
       tc_fence_after();
+      if (!ENC) {
+        cp_async_wait<0>();
+        fetch(0, xc, cc, pc);
+      }
       const uint32_t acc = lane_addr + b * 128;
 #pragma unroll 1
       for (int g = 0; g < NG; ++g) {
         uint4 xn[ENC ? XQ : 1];
         uint32_t cn[ENC ? 1 : GW];
         __half2 pn = pc;
-        if (g + 1 < NG) fetch(g + 1, xn, cn, pn);
+        if (STX) {
+          if (g + 1 < NG)
+            cp_async_wait<1>();
+          else
+            cp_async_wait<0>();
+          fetch(g, xc, cc, pc);
+        } else if (g + 1 < NG) {
+          fetch(g + 1, xn, cn, pn);
+        }
         float pk[KEEP ? 32 : 1];  // prediction of a one-pass group, kept for the second pass
         float sf, zf;
         if (ENC) {
@@ -550,6 +623,9 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           sf = __half2float(sh);
           zf = __half2float(zh);
           if (valid) params[g] = __halves2half2(sh, zh);
+          // x of group g is in registers (the pass above consumed it): its half
+          // of the slot takes group g + 2
+          if (STX && g + 2 < NG) stage_x(g + 2);
         } else {
           const float2 f = __half22float2(pc);
           sf = f.x;
@@ -597,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
 #pragma unroll
           for (int i = 0; i < GW; i += 2) *reinterpret_cast<uint2*>(codes + g * GW + i) = make_uint2(gw[i], gw[i + 1]);
         }
-        if (g + 1 < NG) {
+        if (!STX && g + 1 < NG) {
 #pragma unroll
           for (int i = 0; i < (ENC ? XQ : 1); ++i) xc[i] = xn[i];
 #pragma unroll

@@ -274,11 +274,13 @@ def test_cross_layer_chain_exact_predictor(rank):
         Kr, Vr = Kn, Vn
 
 
-def test_bf16_cross_layer_full_size_sampled():
-    """Full Wan-shaped layer (32760 tokens); the oracle checks sampled tokens,
-    which are independent of one another through the whole layer."""
+@pytest.mark.parametrize("rank", [64, 128])
+def test_bf16_cross_layer_full_size_sampled(rank):
+    """Full Wan-shaped layer (32760 tokens, so every CTA of the persistent
+    kernel codes two tiles); the oracle checks sampled tokens, which are
+    independent of one another through the whole layer."""
     dev = "cuda"
-    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 1, device=dev, L=3, layers_needed=[2])
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 1, device=dev, L=3, rank=rank, layers_needed=[2])
     T, H, D = wl.K[2].shape
     bf, hf = torch.bfloat16, torch.float16
     w = wl.weights[2]
@@ -580,6 +582,34 @@ def test_compressed_attention_cross_layer(n_q, n_self, T, rank):
     _sync_ok()
     ref = O.attend_compressed_xlayer(od, w64, U.to64(Q), ck, cv, Ks, Vs, U.to64(Kself) if n_self else None,
                                      U.to64(Vself) if n_self else None, D ** -0.5)
+    err = U.rel_l2(U.to64(Og), ref)
+    assert err <= U.ATT_TOL[bf], err
+
+
+@pytest.mark.parametrize("rank", [64, 128])
+def test_compressed_attention_full_size(rank):
+    """256 queries over a full Wan-shaped history (32760 tokens, 21 latent
+    frames) plus 130 chunk tokens: the latent pass codes two tiles per CTA."""
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 106, L=2, rank=rank, calib_tokens=1024)
+    T, H, D = wl.K[1].shape
+    n_q, n_self = 256, 130
+    bf, hf = torch.bfloat16, torch.float16
+    od = _odesc(T, H, D, bf, 2, 32, hf)
+    w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
+    Ks, Vs = U.to64(wl.K[0]), U.to64(wl.V[0])
+    ck, cv, _, _ = O.encode_layer_xlayer(od, w64, U.to64(wl.K[1]), U.to64(wl.V[1]), Ks, Vs)
+    buf = _oracle_codes_to_gpu(ck, cv, 2, "f16")
+    Q = synth.queries(21, n_q, H, D)
+    Kself = synth.queries(22, n_self, H, D)
+    Vself = synth.queries(23, n_self, H, D)
+    desc = _desc(T, H, D, bf, 2, 32, hf)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=rank)
+    Og = torch.empty(n_q, H, D, dtype=bf, device="cuda")
+    ws = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q)
+    kvc.kvc_attend_compressed(desc, pred, Q.cuda(), buf, wl.K[0].cuda(), wl.V[0].cuda(), Kself.cuda(),
+                              Vself.cuda(), D ** -0.5, Og, ws)
+    _sync_ok()
+    ref = O.attend_compressed_xlayer(od, w64, U.to64(Q), ck, cv, Ks, Vs, U.to64(Kself), U.to64(Vself), D ** -0.5)
     err = U.rel_l2(U.to64(Og), ref)
     assert err <= U.ATT_TOL[bf], err
 
