@@ -208,6 +208,23 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           ph ^= 1;
         }
       };
+      // two B boxes of the same map in one stage (first in the A half, second in the B half)
+      auto load2 = [&](const CUtensorMap* mb, int bx0, int bx1, int by, uint32_t bbytes) {
+        if (!ok) return;
+        if (!wait(&empty[s], ph ^ 1, abort_flag, a.err, 0x100u + s)) {
+          ok = false;
+          return;
+        }
+        mbar_arrive_expect_tx(&full[s], 2 * bbytes);
+        tma_load(stageA(s), mb, bx0, by, &full[s], pol_keep);
+        tma_load(stageB(s), mb, bx1, by, &full[s], pol_keep);
+        issued[s] = 1;
+        issued_ph[s] = ph;
+        if (++s == S) {
+          s = 0;
+          ph ^= 1;
+        }
+      };
       const uint32_t wbytes = R * 128;
       constexpr int rbytes = 128 * BITS / 8;
       for (int it = 0; it < my_tiles && ok; ++it) {
@@ -232,15 +249,13 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           for (int j = 0; j < 2; ++j)
             load(&maps.ks, h * 128 + j * 64, t0, pol_stream, &maps.bk, j * 64, h * 128, 16384);
           for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, 0, &maps.uk, j * 64, h * 128, 16384);
-          if (RC && h >= 2)
-            for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, 0, &maps.wv, (h - 2) * 128 + j * 64, 0, wbytes);
+          if (RC && h >= 2) load2(&maps.wv, (h - 2) * 128, (h - 2) * 128 + 64, 0, wbytes);
           if (RC)  // the V latent's V^_{l-1} half, interleaved with the K heads
             for (int c = 2 * h; c < 2 * h + 2; ++c)
               load(&maps.vs, c * 64, t0, LAT ? pol_stream : pol_keep, &maps.wv, C + c * 64, 0, wbytes);
         }
         if (RC)
-          for (int g = H >= 2 ? H - 2 : 0; g < H; ++g)
-            for (int j = 0; j < 2; ++j) load(nullptr, 0, 0, 0, &maps.wv, g * 128 + j * 64, 0, wbytes);
+          for (int g = H >= 2 ? H - 2 : 0; g < H; ++g) load2(&maps.wv, g * 128, g * 128 + 64, 0, wbytes);
         if (!LAT) {
           for (int h = 0; h < H && ok; ++h) {
             prefetch_head(true, h);
@@ -348,9 +363,20 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         // Z_V += K^_{l,g} W_V[:, g]^T from the reconstruction tile of K head g
         auto zva = [&](int g) {
           const int rb = (it * HH + g) & 1;
+          // both 64-channel halves of the head from one stage (W_V boxes in its A and B halves)
           group(
-              2, [&] { wt(&rec_full[rb], recf[rb] & 1, 0x500u + rb); },
-              [&](int i, int st) { issue(st, zv, R, false, recon(rb) + i * 16384, nullptr); });
+              1, [&] { wt(&rec_full[rb], recf[rb] & 1, 0x500u + rb); },
+              [&](int, int st) {
+                if (!ISSUE) return;
+                const uint32_t idesc = idesc_bf16(128, R);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  const uint64_t bd = desc_sw128(smem_u32(j ? stageB(st) : stageA(st)));
+                  const uint64_t ad = desc_sw128(smem_u32(recon(rb) + j * 16384));
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) umma_if(lead, zv, ad + 2 * k, bd + 2 * k, idesc, 1u);
+                }
+              });
           recf[rb]++;
           commit(&rec_free[rb]);
         };
