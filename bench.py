@@ -45,7 +45,7 @@ UNIT = "KV tokens/s"
 # DRAM bytes (read + write) per launch, from the ncu captures summarised under
 # profiles/ (codec_xlayer_wan_layer.md, attention_cluster_wan.md,
 # mixed_attention_cluster.md); set to None when a kernel changes after its capture.
-TRAFFIC = {"encode_xlayer": None, "decode_xlayer": None,
+TRAFFIC = {"encode_xlayer": 674717696 + 202756608, "decode_xlayer": 437384192 + 152241920,
            "attention_c2": 769948672 + 8668416, "attention_c4": 26633216 + 512}
 
 
