@@ -191,11 +191,12 @@ cudaError_t codec_cluster(const kvc_layer_desc* d, const kvc_predictor* p, bool 
     if (enc) {
       cn = (float*)ws.take(nc * sizeof(float));
       P = (float*)ws.take((size_t)nc * m * sizeof(float));
-      ClusterPrepArgs<TS> pa{nc, C, m, cent, encw, cn, P};
-      if ((e = launch_cluster_prep(pa, st)) != cudaSuccess) return e;
     }
     if constexpr (std::is_same<TS, __nv_bfloat16>::value && std::is_same<TP, __half>::value) {
       if (tc_cluster_supported(d, p)) {
+        // the tensor-core encode forms P itself (the same accumulation as the tokens' coefficients)
+        ClusterPrepArgs<TS> pa{nc, C, m, cent, encw, cn, P};
+        if (enc && (e = launch_cluster_norms(pa, st)) != cudaSuccess) return e;
         void* codes = which ? c->v_codes : c->k_codes;
         void* params = which ? c->v_params : c->k_params;
         void* assign = which ? c->v_assign : c->k_assign;
@@ -207,6 +208,10 @@ cudaError_t codec_cluster(const kvc_layer_desc* d, const kvc_predictor* p, bool 
         if (rec && (e = tc_cluster_decode(d, p, codes, params, assign, cent, dec, rec, st)) != cudaSuccess) return e;
         continue;
       }
+    }
+    if (enc) {
+      ClusterPrepArgs<TS> pa{nc, C, m, cent, encw, cn, P};
+      if ((e = launch_cluster_prep(pa, st)) != cudaSuccess) return e;
     }
     ClusterArgs<TS, TP> a{d->n_tokens, C, m, nc, d->bits, d->group, (const TS*)(which ? V : K), cent, encw, dec,
                           cn, P, (uint8_t*)(which ? c->v_codes : c->k_codes),

@@ -271,6 +271,22 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(TemporalArgs<TS, TP>
 
 // ============================================================== clustered codec
 
+// cnorm[j] = |c_j|^2 (fp32), one warp per centre: the norms alone, for the
+// tensor-core encode, which forms P on the tensor cores
+template <typename TS>
+__global__ void __launch_bounds__(kThreads) cluster_norms_kernel(ClusterPrepArgs<TS> a) {
+  const int tx = threadIdx.x & 31;
+  const int jc = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+  if (jc >= a.n_c) return;
+  float s = 0.f;
+  for (int k = tx; k < a.C; k += 32) {
+    const float v = to_f(a.cent[(int64_t)jc * a.C + k]);
+    s = fmaf(v, v, s);
+  }
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (tx == 0) a.cnorm[jc] = s;
+}
+
 // cnorm[j] = |c_j|^2, P[j][i] = enc_i . c_j (fp32)
 template <typename TS>
 __global__ void __launch_bounds__(kThreads) cluster_prep_kernel(ClusterPrepArgs<TS> a) {
@@ -752,6 +768,13 @@ cudaError_t launch_temporal(const TemporalArgs<TS, TP>& a, int D, bool encode, c
 }
 
 template <typename TS>
+cudaError_t launch_cluster_norms(const ClusterPrepArgs<TS>& a, cudaStream_t st) {
+  cluster_norms_kernel<TS><<<div_up(a.n_c, kThreads / 32), kThreads, 0, st>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <typename TS>
 cudaError_t launch_cluster_prep(const ClusterPrepArgs<TS>& a, cudaStream_t st) {
   const size_t smem = (32 * 33 + 128 * 33) * sizeof(float);
   auto k = cluster_prep_kernel<TS>;
@@ -845,6 +868,7 @@ KVC_INST(__nv_bfloat16, __half)
 template cudaError_t launch_latent<float>(const LatentArgs<float>&, cudaStream_t);
 template cudaError_t launch_latent<__nv_bfloat16>(const LatentArgs<__nv_bfloat16>&, cudaStream_t);
 template cudaError_t launch_cluster_prep<float>(const ClusterPrepArgs<float>&, cudaStream_t);
+template cudaError_t launch_cluster_norms<__nv_bfloat16>(const ClusterPrepArgs<__nv_bfloat16>&, cudaStream_t);
 template cudaError_t launch_cluster_prep<__nv_bfloat16>(const ClusterPrepArgs<__nv_bfloat16>&, cudaStream_t);
 template cudaError_t launch_attention<float>(const AttnArgs<float>&, int, cudaStream_t);
 template cudaError_t launch_attention<__nv_bfloat16>(const AttnArgs<__nv_bfloat16>&, int, cudaStream_t);

@@ -115,6 +115,8 @@ template <typename TS, typename TP>
 cudaError_t launch_temporal(const TemporalArgs<TS, TP>& a, int D, bool encode, cudaStream_t st);
 template <typename TS>
 cudaError_t launch_cluster_prep(const ClusterPrepArgs<TS>& a, cudaStream_t st);
+template <typename TS>
+cudaError_t launch_cluster_norms(const ClusterPrepArgs<TS>& a, cudaStream_t st);  // cnorm only
 template <typename TS, typename TP>
 cudaError_t launch_cluster(const ClusterArgs<TS, TP>& a, bool encode, cudaStream_t st);
 template <typename TS>

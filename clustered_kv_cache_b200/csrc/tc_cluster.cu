@@ -442,19 +442,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_kernel(const __grid_consta
     const __nv_bfloat16* crow = a.cent + (int64_t)c * a.C;
     for (int n = 0; n < NN; ++n) {
       const int b = n & 1;
+      // this half chunk's centre values, fetched while the MMAs run
+      uint4 cv[16];
+      {
+        const uint4* cr = reinterpret_cast<const uint4*>(crow + n * 256 + grp * 128);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cv[i] = __ldg(cr + i);
+      }
       wait(&acc_full[b], (n >> 1) & 1, abort_flag, a.err, 0x3600u + b);
       tc_fence_after();
-#pragma unroll 1
+#pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
         const int col = n * 256 + grp * 128 + cb * 32;  // output channel
         float v[32];
         tmem_ld32(lane_addr + b * 256 + grp * 128 + cb * 32, v);
-        const uint4* cr = reinterpret_cast<const uint4*>(crow + col);
         uint4 w[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float cc[8];
-          unpack_bf16x8(__ldg(cr + i), cc, 0);
+          unpack_bf16x8(cv[cb * 4 + i], cc, 0);
           w[i] = make_uint4(pack_bf16x2(cc[0] + v[8 * i], cc[1] + v[8 * i + 1]),
                             pack_bf16x2(cc[2] + v[8 * i + 2], cc[3] + v[8 * i + 3]),
                             pack_bf16x2(cc[4] + v[8 * i + 4], cc[5] + v[8 * i + 5]),
