@@ -27,6 +27,8 @@ namespace kvc {
 namespace tc {
 
 bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool map2d_bytes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                 uint32_t box_rows);
 
 namespace cluster {
 
@@ -267,11 +269,13 @@ constexpr int kDecThreads = 320;
 constexpr int kDecStages = 2;
 constexpr int kDecStage = 65536;  // W_dec rows of one 256-wide output chunk, two [256][64] sub-tiles
 constexpr int kDecA = kDecStages * kDecStage;  // [coef^ hi | coef^ lo], four [128][64] sub-tiles
-constexpr int kDecBar = kDecA + 65536;
+constexpr int kDecOut = kDecA + 65536;          // output boxes [32 rows][64 bytes], two per epilogue warp
+constexpr int kDecBar = kDecOut + 8 * 2 * 2048;
 constexpr int kDecSmem = kDecBar + 1024 + 1024;
 
 struct DecMaps {
   CUtensorMap dec;  // [C][128], box 256 rows
+  CUtensorMap out;  // x^ [T][C] as bytes, box 32 rows x 64 bytes
 };
 struct DecArgs {
   unsigned* err;
@@ -440,6 +444,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_kernel(const __grid_consta
     int c = t < a.T ? (int)a.assign[t] : 0;
     c = c < a.n_c ? c : a.n_c - 1;
     const __nv_bfloat16* crow = a.cent + (int64_t)c * a.C;
+    // x^ leaves through shared memory and TMA stores (row-per-thread global
+    // stores cost a request per 16 bytes): per 32 columns the warp fills one of
+    // its two [32 rows][64 bytes] boxes, a lane writing its row's 16-byte pieces
+    // in an order rotated by lane / 2 so that a store instruction touches eight
+    // different bank groups
+    uint8_t* obox = smem + kDecOut + (warp - 2) * 4096;
+    int ob = 0;
     for (int n = 0; n < NN; ++n) {
       const int b = n & 1;
       // this half chunk's centre values, fetched while the MMAs run
@@ -466,15 +477,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_kernel(const __grid_consta
                             pack_bf16x2(cc[4] + v[8 * i + 4], cc[5] + v[8 * i + 5]),
                             pack_bf16x2(cc[6] + v[8 * i + 6], cc[7] + v[8 * i + 7]));
         }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(a.out + t * a.C + col);
+        uint8_t* box = obox + ob * 2048;
+        if (lane == 0) bulk_wait_read1();  // the store that last read this box is done with it
+        __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = w[i];
+        for (int i = 0; i < 4; ++i) {
+          const int j = (i + (lane >> 1)) & 3;
+          const uint4 val = j == 0 ? w[0] : (j == 1 ? w[1] : (j == 2 ? w[2] : w[3]));
+          *reinterpret_cast<uint4*>(box + lane * 64 + j * 16) = val;
         }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && t0 + qd * 32 < a.T) {  // the tensor map clips rows past T
+          tma_store(&maps.out, col * 2, t0 + qd * 32, box);
+          bulk_commit();
+        }
+        ob ^= 1;
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -549,7 +572,8 @@ cudaError_t tc_cluster_decode(const kvc_layer_desc* d, const kvc_predictor* p, c
   const uint64_t T = (uint64_t)d->n_tokens, C = (uint64_t)d->n_heads * d->head_dim;
   tc::cluster::DecMaps m;
   memset(&m, 0, sizeof(m));
-  if (!tc::map2d(&m.dec, dec, C, 128, 256)) return cudaErrorInvalidValue;
+  if (!tc::map2d(&m.dec, dec, C, 128, 256) || !tc::map2d_bytes(&m.out, out, T, C * 2, 64, 32))
+    return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
   tc::cluster::DecArgs a{err, (int64_t)T, (int)C, p->n_clusters, (const uint8_t*)codes, (const __half2*)params,
