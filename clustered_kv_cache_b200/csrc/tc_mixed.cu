@@ -12,8 +12,9 @@
 //
 // so per (128-query tile, head) the kernel is a flash attention with 256-wide
 // rows on both sides: A = [q_h | q_h W_dec,h] (its second half computed on the
-// tensor cores at the start), key tiles [centre rows | coefficients] and value
-// tiles [centre rows | coefficients]; the value product accumulates
+// tensor cores at the start), 64-key tiles [centre rows | coefficients] for the
+// keys and for the values, double-buffered so that a tile's gather and load
+// overlap the MMAs of the one before; the value product accumulates
 // [O_c | cbar] (256 TMEM columns) and the end adds cbar W^V_dec,h^T.  The sum
 // over p_t c_{a(t)} equals the oracle's sum over clusters of the per-cluster
 // mass times the centre (the same terms, grouped differently).
@@ -39,10 +40,15 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint3
 namespace mixed {
 
 constexpr int kThreads = 320;
-// shared memory (offsets from a 1024-aligned base); each region is four [128][64] bf16 sub-tiles
-constexpr int kA = 0;              // [q_h | q_h W_dec,h]
-constexpr int kKt = kA + 65536;    // key tile [centre rows | coef]; at the start W_dec,h; at the end cbar
-constexpr int kVt = kKt + 65536;   // value tile [centre rows | coef] (MN-major B); at the end W^V_dec,h
+constexpr int kKeys = 64;  // keys per tile
+// shared memory (offsets from a 1024-aligned base)
+constexpr int kA = 0;              // [q_h | q_h W_dec,h], four [128][64] bf16 sub-tiles
+constexpr int kKt = kA + 65536;    // key tiles [2], each [centre rows | coef] as four [64][64] sub-tiles;
+                                   // at the start W_dec,h, at the end cbar (both [128][64] x 2)
+constexpr int kVt = kKt + 65536;   // value tiles [2] (MN-major B: four 64-wide N sub-tiles of 64 keys);
+                                   // at the end W^V_dec,h
+constexpr int kTile = 32768;
+constexpr int kSub = 8192;         // [64 rows][64] sub-tile of a key / value tile
 constexpr int kBar = kVt + 65536;
 constexpr int kSmem = kBar + 1024 + 1024;
 
@@ -102,6 +108,11 @@ __device__ __forceinline__ void tie32(float (&v)[32]) {
                  "+r"(r[30]), "+r"(r[31])
                :
                : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait2(float (&a)[32], float (&b)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  tie32(a);
+  tie32(b);
 }
 __device__ __forceinline__ void tmem_ld_wait4(float (&a)[32], float (&b)[32], float (&c)[32], float (&d)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -174,11 +185,11 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
   uint64_t* setup_full = bars;         // q_h and W_dec,h landed
   uint64_t* qw_acc = setup_full + 1;   // q_h W_dec,h in TMEM
   uint64_t* qw_ready = qw_acc + 1;     // ... and in the A tile as bf16 (prep)
-  uint64_t* kfull = qw_ready + 1;      // key tile complete (producer tx + 128 prep arrivals)
-  uint64_t* vfull = kfull + 1;         // value tile complete
-  uint64_t* kfree = vfull + 1;         // S(j) done: the key tile may be refilled
-  uint64_t* vfree = kfree + 1;         // PV(j) done: the value tile may be refilled
-  uint64_t* s_full = vfree + 1;        // [2]
+  uint64_t* kfull = qw_ready + 1;      // [2] key tile complete (producer tx + 64 prep arrivals)
+  uint64_t* vfull = kfull + 2;         // [2] value tile complete
+  uint64_t* kfree = vfull + 2;         // [2] S(j) done: the key tile may be refilled
+  uint64_t* vfree = kfree + 2;         // [2] PV(j) done: the value tile may be refilled
+  uint64_t* s_full = vfree + 2;        // [2]
   uint64_t* p_full = s_full + 2;       // [2]
   uint64_t* pv_done = p_full + 2;
   uint64_t* acc_done = pv_done + 1;    // the last PV finished: O_c and cbar final
@@ -193,16 +204,18 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
   const int h = blockIdx.y;
   const int q0 = blockIdx.x * 128;
   const int C = a.H * 128;
-  const int NT = (int)((a.T + 127) / 128);
+  const int NT = (int)((a.T + kKeys - 1) / kKeys);
 
   if (threadIdx.x == 0) {
     mbar_init(setup_full, 1);
     mbar_init(qw_acc, 1);
     mbar_init(qw_ready, 128);
-    mbar_init(kfull, 129);
-    mbar_init(vfull, 129);
-    mbar_init(kfree, 1);
-    mbar_init(vfree, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kfull[i], kKeys + 1);
+      mbar_init(&vfull[i], kKeys + 1);
+      mbar_init(&kfree[i], 1);
+      mbar_init(&vfree[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
@@ -225,11 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  auto SC = [&](int b) { return tmem + 128 * b; };  // S / P slots; slot 0 holds q W_dec at the start
-  const uint32_t OC = tmem + 256;                   // [O_c | cbar], 256 columns
+  auto SC = [&](int b) { return tmem + 64 * b; };  // S / P slots, 64 columns each
+  const uint32_t OC = tmem + 128;                  // [O_c | cbar], 256 columns
+  const uint32_t QW = tmem + 384;                  // q W_dec (setup)
   uint8_t* At = smem + kA;
   uint8_t* Kt = smem + kKt;
   uint8_t* Vt = smem + kVt;
+  auto KT = [&](int b) { return Kt + b * kTile; };
+  auto VT = [&](int b) { return Vt + b * kTile; };
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -242,30 +258,31 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
       tma_load(At + 16384, &maps.q, h * 128 + 64, q0, setup_full, pol_stream);
       tma_load(Kt, &maps.deck, 0, h * 128, setup_full, pol_keep);  // [K = d][N = i], MN-major B
       tma_load(Kt + 16384, &maps.deck, 64, h * 128, setup_full, pol_keep);
-      int pk = 0, pv = 0;
-      int k_armed = -1, v_armed = -1;  // last tile whose loads were issued (drained after an abort)
+      int k_last = -1, v_last = -1;  // last tile loaded (the loads of it and of the tile before are drained after an abort)
       bool dv_armed = false;
       for (int j = 0; j < NT && ok; ++j) {
-        // coefficients of the key tile, once S(j-1) (or the q W_dec product) is done with the tile
+        const int b = j & 1;
+        // coefficients of the key tile, once S(j-2) is done with the buffer (tile 0: once the
+        // q W_dec product is done with W_dec,h, which it overlaps)
         if (j == 0) {
           if (!wait(qw_acc, 0, abort_flag, a.err, 0x2100u)) ok = false;
-        } else if (!wait(kfree, pk++ & 1, abort_flag, a.err, 0x2101u)) {
+        } else if (j >= 2 && !wait(&kfree[b], ((j - 2) >> 1) & 1, abort_flag, a.err, 0x2101u)) {
           ok = false;
         }
         if (!ok) break;
-        mbar_arrive_expect_tx(kfull, 32768u);
-        tma_load(Kt + 32768, &maps.ckh, 0, j * 128, kfull, pol_keep);
-        tma_load(Kt + 49152, &maps.ckh, 64, j * 128, kfull, pol_keep);
-        k_armed = j;
-        if (j >= 1 && !wait(vfree, pv++ & 1, abort_flag, a.err, 0x2102u)) ok = false;
+        mbar_arrive_expect_tx(&kfull[b], 16384u);
+        tma_load(KT(b) + 2 * kSub, &maps.ckh, 0, j * kKeys, &kfull[b], pol_keep);
+        tma_load(KT(b) + 3 * kSub, &maps.ckh, 64, j * kKeys, &kfull[b], pol_keep);
+        k_last = j;
+        if (j >= 2 && !wait(&vfree[b], ((j - 2) >> 1) & 1, abort_flag, a.err, 0x2102u)) ok = false;
         if (!ok) break;
-        mbar_arrive_expect_tx(vfull, 32768u);
-        tma_load(Vt + 32768, &maps.cvh, 0, j * 128, vfull, pol_keep);
-        tma_load(Vt + 49152, &maps.cvh, 64, j * 128, vfull, pol_keep);
-        v_armed = j;
+        mbar_arrive_expect_tx(&vfull[b], 16384u);
+        tma_load(VT(b) + 2 * kSub, &maps.cvh, 0, j * kKeys, &vfull[b], pol_keep);
+        tma_load(VT(b) + 3 * kSub, &maps.cvh, 64, j * kKeys, &vfull[b], pol_keep);
+        v_last = j;
       }
-      // W^V_dec,h for the final product, once the last PV is done with the value tile
-      if (ok && wait(vfree, pv++ & 1, abort_flag, a.err, 0x2103u)) {
+      // W^V_dec,h for the final product, once every MMA is done with the value tiles
+      if (ok && wait(acc_done, 0, abort_flag, a.err, 0x2103u)) {
         mbar_arrive_expect_tx(dv_full, 32768u);
         tma_load(Vt, &maps.decv, 0, h * 128, dv_full, pol_keep);  // [N = d][K = i], K-major B
         tma_load(Vt + 16384, &maps.decv, 64, h * 128, dv_full, pol_keep);
@@ -280,8 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
           }
         };
         drain(setup_full, 0);
-        if (k_armed >= 0) drain(kfull, k_armed & 1);
-        if (v_armed >= 0) drain(vfull, v_armed & 1);
+        for (int j = k_last - 1; j <= k_last; ++j)
+          if (j >= 0) drain(&kfull[j & 1], (j >> 1) & 1);
+        for (int j = v_last - 1; j <= v_last; ++j)
+          if (j >= 0) drain(&vfull[j & 1], (j >> 1) & 1);
         if (dv_armed) drain(dv_full, 0);
       }
     }
@@ -290,7 +309,6 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
     if (lane == 0) {
       const uint32_t id128 = idesc_bf16(128, 128);
       const uint64_t ad = desc_sw128(smem_u32(At));
-      const uint64_t kd = desc_sw128(smem_u32(Kt));
       // q W_dec,h: A = q_h (K = d), B = W_dec,h (MN-major)
       wait(setup_full, 0, abort_flag, a.err, 0x2200u);
       tc_fence_after();
@@ -300,39 +318,42 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
-          umma(SC(0), ad + off, bd + (uint64_t)k * (2048 >> 4), idm, k == 0 ? 0u : 1u);
+          umma(QW, ad + off, bd + (uint64_t)k * (2048 >> 4), idm, k == 0 ? 0u : 1u);
         }
         umma_commit(qw_acc);
       }
       wait(qw_ready, 0, abort_flag, a.err, 0x2201u);
       tc_fence_after();
+      const uint32_t id64 = idesc_bf16(128, kKeys);
+      const uint32_t idv = idesc_bf16_bmn(128, 256);
       for (int j = 0; j <= NT; ++j) {
         if (j < NT) {
           const int b = j & 1;
-          // S(j) = [q | q W_dec] [centres | coef]^T, K = 256
-          wait(kfull, j & 1, abort_flag, a.err, 0x2210u);
+          // S(j) = [q | q W_dec] [centres | coef]^T, K = 256, N = 64 keys
+          wait(&kfull[b], (j >> 1) & 1, abort_flag, a.err, 0x2210u + b);
           tc_fence_after();
+          const uint64_t kd = desc_sw128(smem_u32(KT(b)));
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
-            umma(SC(b), ad + off, kd + off, id128, k == 0 ? 0u : 1u);
+            const uint32_t aoff = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
+            const uint32_t boff = (k >> 2) * (kSub >> 4) + (k & 3) * 2;
+            umma(SC(b), ad + aoff, kd + boff, id64, k == 0 ? 0u : 1u);
           }
           umma_commit(&s_full[b]);
-          umma_commit(kfree);
+          umma_commit(&kfree[b]);
         }
         if (j >= 1) {
           const int t = j - 1, b = t & 1;
-          // [O_c | cbar] += P(t) [centres | coef], N = 256, P from TMEM
+          // [O_c | cbar] += P(t) [centres | coef], K = 64 keys, N = 256, P from TMEM
           wait(&p_full[b], (t >> 1) & 1, abort_flag, a.err, 0x2220u + b);
-          wait(vfull, t & 1, abort_flag, a.err, 0x2230u);
+          wait(&vfull[b], (t >> 1) & 1, abort_flag, a.err, 0x2230u + b);
           tc_fence_after();
-          const uint64_t vd = desc_mn_sw128(smem_u32(Vt), 16384);
-          const uint32_t idv = idesc_bf16_bmn(128, 256);
+          const uint64_t vd = desc_mn_sw128(smem_u32(VT(b)), kSub);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
+          for (int k = 0; k < kKeys / 16; ++k)
             umma_ts(OC, SC(b) + k * 8, vd + (uint64_t)k * (2048 >> 4), idv, (t == 0 && k == 0) ? 0u : 1u);
           umma_commit(pv_done);
-          umma_commit(vfree);
+          umma_commit(&vfree[b]);
         }
       }
       umma_commit(acc_done);
@@ -378,37 +399,45 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
       tc_fence_before();
       fence_async_smem();
     };
-    // the head's 128 channels of the centre of this row's key, fetched ahead of
-    // the wait for the tile, then stored into sub-tiles 0, 1 of it
-    auto fetch_rows = [&](const __nv_bfloat16* cent, const uint8_t* assign, int j, uint4 (&w)[16]) {
-      const int64_t t = (int64_t)j * 128 + row;
+    // The head's 128 channels (256 bytes) of the centre of each key: the warps
+    // of lane quarters 0, 1 gather the 64 rows of a key tile, those of quarters
+    // 2, 3 the rows of a value tile, 32 rows per warp.  A half warp reads one
+    // row (16 bytes a lane), two rows per instruction, so a load touches two
+    // rows' lines rather than 32.  Rows are fetched ahead of the wait for their
+    // buffer, then stored into sub-tiles 0, 1 of it.
+    const bool is_v = qd >= 2;
+    const int r0 = (qd & 1) * 32;  // this warp's first row of a tile
+    const int ch = lane & 15;      // 16-byte chunk of a row
+    const __nv_bfloat16* cent = is_v ? a.cent_v : a.cent_k;
+    const uint8_t* assign = is_v ? a.assign_v : a.assign_k;
+    uint64_t* tfull = is_v ? vfull : kfull;
+    uint64_t* tfree = is_v ? vfree : kfree;
+    auto fetch_row = [&](int j, uint4 (&w)[16]) {
+      const int64_t t = (int64_t)j * kKeys + r0 + lane;  // a lane holds the centre of one row
       int c = t < a.T ? (int)assign[t] : 0;
       c = c < a.n_c ? c : a.n_c - 1;
-      const uint4* src = reinterpret_cast<const uint4*>(cent + (int64_t)c * C + h * 128);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) w[i] = __ldg(src + i);
+      for (int i = 0; i < 16; ++i) {
+        const int cr = __shfl_sync(0xffffffffu, c, 2 * i + (lane >> 4));
+        w[i] = __ldg(reinterpret_cast<const uint4*>(cent + (int64_t)cr * C + h * 128) + ch);
+      }
     };
-    auto store_rows = [&](const uint4 (&w)[16], uint8_t* tile) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) *reinterpret_cast<uint4*>(tile + (i / 8) * 16384 + sw128_off(row, i % 8)) = w[i];
-      fence_async_smem();
-    };
-    uint4 wk[16], wv[16];
-    fetch_rows(a.cent_k, a.assign_k, 0, wk);
-    wait(qw_acc, 0, abort_flag, a.err, 0x2300u);
+    uint4 w[16];
+    fetch_row(0, w);
+    wait(qw_acc, 0, abort_flag, a.err, 0x2300u);  // also: W_dec,h in key buffer 0 is no longer read
     tc_fence_after();
-    to_bf16(SC(0), At + 32768);
+    to_bf16(QW, At + 32768);
     mbar_arrive(qw_ready);
-    int pk = 0, pv = 0;
     for (int j = 0; j < NT; ++j) {
-      if (j >= 1) wait(kfree, pk++ & 1, abort_flag, a.err, 0x2301u);
-      store_rows(wk, Kt);
-      mbar_arrive(kfull);
-      fetch_rows(a.cent_v, a.assign_v, j, wv);
-      if (j >= 1) wait(vfree, pv++ & 1, abort_flag, a.err, 0x2302u);
-      store_rows(wv, Vt);
-      mbar_arrive(vfull);
-      if (j + 1 < NT) fetch_rows(a.cent_k, a.assign_k, j + 1, wk);
+      const int b = j & 1;
+      if (j >= 2) wait(&tfree[b], ((j - 2) >> 1) & 1, abort_flag, a.err, 0x2301u + (is_v ? 2 : 0) + b);
+      uint8_t* tile = is_v ? VT(b) : KT(b);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        *reinterpret_cast<uint4*>(tile + (ch / 8) * kSub + sw128_off(r0 + 2 * i + (lane >> 4), ch % 8)) = w[i];
+      fence_async_smem();
+      mbar_arrive(&tfull[b]);
+      if (j + 1 < NT) fetch_row(j + 1, w);
     }
     // cbar (TMEM) -> bf16 A operand in the key-tile area, once every S and PV is done
     wait(acc_done, 0, abort_flag, a.err, 0x2303u);
@@ -427,24 +456,22 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
       const uint32_t sc = lane_addr + (SC(b) - tmem);
       wait(&s_full[b], (j >> 1) & 1, abort_flag, a.err, 0x2400u + b);
       tc_fence_after();
-      const int64_t kbase = (int64_t)j * 128;
-      const int nvalid = a.T - kbase < 128 ? (int)(a.T - kbase) : 128;
-      float sv[4][32];
+      const int64_t kbase = (int64_t)j * kKeys;
+      const int nvalid = a.T - kbase < kKeys ? (int)(a.T - kbase) : kKeys;
+      float sv[2][32];
       tmem_ld32_async(sc, sv[0]);
       tmem_ld32_async(sc + 32, sv[1]);
-      tmem_ld32_async(sc + 64, sv[2]);
-      tmem_ld32_async(sc + 96, sv[3]);
-      tmem_ld_wait4(sv[0], sv[1], sv[2], sv[3]);
-      if (nvalid < 128) {
+      tmem_ld_wait2(sv[0], sv[1]);
+      if (nvalid < kKeys) {
 #pragma unroll
-        for (int pc = 0; pc < 4; ++pc)
+        for (int pc = 0; pc < 2; ++pc)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (pc * 32 + i >= nvalid) sv[pc][i] = -INFINITY;
       }
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc)
+      for (int pc = 0; pc < 2; ++pc)
 #pragma unroll
         for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], sv[pc][i]);
       const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
@@ -458,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
       }
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
+      for (int pc = 0; pc < 2; ++pc) {
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -553,8 +580,8 @@ cudaError_t tc_mixed_attend(const kvc_layer_desc* d, const kvc_predictor* p, con
   tc::mixed::Maps m;
   memset(&m, 0, sizeof(m));
   bool ok = tc::map2d(&m.q, Q, (uint64_t)n_q, C, 128) && tc::map2d(&m.deck, p->k_dec, C, 128, 128) &&
-            tc::map2d(&m.decv, p->v_dec, C, 128, 128) && tc::map2d(&m.ckh, ckh, T, 128, 128) &&
-            tc::map2d(&m.cvh, cvh, T, 128, 128);
+            tc::map2d(&m.decv, p->v_dec, C, 128, 128) && tc::map2d(&m.ckh, ckh, T, 128, tc::mixed::kKeys) &&
+            tc::map2d(&m.cvh, cvh, T, 128, tc::mixed::kKeys);
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
