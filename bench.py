@@ -46,7 +46,7 @@ UNIT = "KV tokens/s"
 # profiles/ (codec_xlayer_wan_layer.md, attention_cluster_wan.md,
 # mixed_attention_cluster.md); set to None when a kernel changes after its capture.
 TRAFFIC = {"encode_xlayer": 674717696 + 202756608, "decode_xlayer": 437384192 + 152241920,
-           "attention_c2": 769948672 + 8668416, "attention_c4": 26633216 + 512}
+           "attention_c2": 769948672 + 8668416, "attention_c4": None}
 
 
 def peaks():
