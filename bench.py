@@ -44,9 +44,11 @@ UNIT = "KV tokens/s"
 
 # DRAM bytes (read + write) per launch, from the ncu captures summarised under
 # profiles/ (codec_xlayer_wan_layer.md, attention_cluster_wan.md,
-# mixed_attention_cluster.md); set to None when a kernel changes after its capture.
+# mixed_attention_cluster.md, temporal_codec_layer.md); set to None when a
+# kernel changes after its capture.
 TRAFFIC = {"encode_xlayer": 674717696 + 202756608, "decode_xlayer": 437384192 + 152241920,
-           "attention_c2": 769948672 + 8668416, "attention_c4": None}
+           "attention_c2": 769948672 + 8668416, "attention_c4": 26442240 + 768,
+           "temporal_encode": 1467036672 + 353639168}
 
 
 def peaks():
@@ -321,7 +323,7 @@ def row_temporal(dev, hbm, reps=3) -> dict:
         gbs = byts / (ms * 1e-3) / 1e9
         out[name] = {"ms": ms, "tokens_per_s": T / (ms * 1e-3),
                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                                  "traffic": None}}
+                                  "traffic": TRAFFIC["temporal_encode"] if name == "encode" else None}}
     out["workload"] = "temporal codec, one layer: 65536 tokens x 40 heads x 128, 1560-token frames, INT4 g64"
     return out
 
@@ -528,7 +530,8 @@ def main():
             rows["c4_cluster"] = row_cluster(dev, hbm, tf_burst)
         rows = rows or None
         if not args.no_cpu:
-            cpu = oracle_xlayer_rate(xb.wl, 192, L_RUN, 20.0)
+            # about 10 s of host work: 2048 of the tokens through every layer
+            cpu = oracle_xlayer_rate(xb.wl, 2048, L_RUN, 20.0)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
