@@ -182,33 +182,49 @@ cudaError_t codec_cluster(const kvc_layer_desc* d, const kvc_predictor* p, bool 
                           const kvc_codes* c, void* Kr, void* Vr, Carve& ws, cudaStream_t st) {
   const int C = d->n_heads * d->head_dim, m = p->code_dim, nc = p->n_clusters;
   cudaError_t e;
-  for (int which = 0; which < 2; ++which) {
-    const TS* cent = (const TS*)(which ? p->v_centroids : p->k_centroids);
-    const TS* encw = (const TS*)(which ? p->v_enc : p->k_enc);
-    const TS* dec = (const TS*)(which ? p->v_dec : p->k_dec);
-    float* cn = nullptr;
-    float* P = nullptr;
-    if (enc) {
-      cn = (float*)ws.take(nc * sizeof(float));
-      P = (float*)ws.take((size_t)nc * m * sizeof(float));
+  float* cns[2] = {nullptr, nullptr};
+  float* Ps[2] = {nullptr, nullptr};
+  if (enc)
+    for (int which = 0; which < 2; ++which) {
+      cns[which] = (float*)ws.take(nc * sizeof(float));
+      Ps[which] = (float*)ws.take((size_t)nc * m * sizeof(float));
     }
-    if constexpr (std::is_same<TS, __nv_bfloat16>::value && std::is_same<TP, __half>::value) {
-      if (tc_cluster_supported(d, p)) {
-        // the tensor-core encode forms P itself (the same accumulation as the tokens' coefficients)
-        ClusterPrepArgs<TS> pa{nc, C, m, cent, encw, cn, P};
-        if (enc && (e = launch_cluster_norms(pa, st)) != cudaSuccess) return e;
+  if constexpr (std::is_same<TS, __nv_bfloat16>::value && std::is_same<TP, __half>::value) {
+    if (tc_cluster_supported(d, p)) {
+      if (enc) {
+        // centre norms, then P = C E^T of both tensors on the tensor cores (the same
+        // accumulation as the tokens' coefficients) in one launch
+        for (int which = 0; which < 2; ++which) {
+          ClusterPrepArgs<TS> pa{nc, C, m, (const TS*)(which ? p->v_centroids : p->k_centroids),
+                                 (const TS*)(which ? p->v_enc : p->k_enc), cns[which], Ps[which]};
+          if ((e = launch_cluster_norms(pa, st)) != cudaSuccess) return e;
+        }
+        const float* const cnc[2] = {cns[0], cns[1]};
+        if ((e = tc_cluster_prepare(d, p, cnc, Ps, st)) != cudaSuccess) return e;
+      }
+      for (int which = 0; which < 2; ++which) {
+        const TS* cent = (const TS*)(which ? p->v_centroids : p->k_centroids);
+        const TS* encw = (const TS*)(which ? p->v_enc : p->k_enc);
+        const TS* dec = (const TS*)(which ? p->v_dec : p->k_dec);
         void* codes = which ? c->v_codes : c->k_codes;
         void* params = which ? c->v_params : c->k_params;
         void* assign = which ? c->v_assign : c->k_assign;
         void* rec = which ? Vr : Kr;
-        if (enc && (e = tc_cluster_encode(d, p, which ? V : K, cent, encw, cn, P, codes, params, assign, st)) !=
-                       cudaSuccess)
+        if (enc && (e = tc_cluster_encode(d, p, which ? V : K, cent, encw, cns[which], Ps[which], codes, params,
+                                          assign, st)) != cudaSuccess)
           return e;
         // the encode's reconstruction is the decode of what it wrote, so the two agree bit for bit
         if (rec && (e = tc_cluster_decode(d, p, codes, params, assign, cent, dec, rec, st)) != cudaSuccess) return e;
-        continue;
       }
+      return cudaSuccess;
     }
+  }
+  for (int which = 0; which < 2; ++which) {
+    const TS* cent = (const TS*)(which ? p->v_centroids : p->k_centroids);
+    const TS* encw = (const TS*)(which ? p->v_enc : p->k_enc);
+    const TS* dec = (const TS*)(which ? p->v_dec : p->k_dec);
+    float* cn = cns[which];
+    float* P = Ps[which];
     if (enc) {
       ClusterPrepArgs<TS> pa{nc, C, m, cent, encw, cn, P};
       if ((e = launch_cluster_prep(pa, st)) != cudaSuccess) return e;

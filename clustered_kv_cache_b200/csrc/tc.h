@@ -23,6 +23,10 @@ size_t tc_mixed_workspace(const kvc_layer_desc* d);
 cudaError_t tc_mixed_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
                             const kvc_codes* c, float scale, void* O, void* ws, size_t ws_bytes, cudaStream_t st);
 bool tc_cluster_supported(const kvc_layer_desc* d, const kvc_predictor* p);
+// P = C E^T of both tensors (K: [0], V: [1]) on the tensor cores, one launch;
+// the encode of either tensor reads its P
+cudaError_t tc_cluster_prepare(const kvc_layer_desc* d, const kvc_predictor* p, const float* const cnorm[2],
+                               float* const P[2], cudaStream_t st);
 cudaError_t tc_cluster_encode(const kvc_layer_desc* d, const kvc_predictor* p, const void* X, const void* cent,
                               const void* enc, const float* cnorm, float* P, void* codes, void* params,
                               void* assign, cudaStream_t st);

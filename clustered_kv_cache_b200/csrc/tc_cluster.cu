@@ -57,9 +57,14 @@ struct EncArgs {
 
 // PMODE: the rows are the centres themselves and the kernel writes Y = C E^T to
 // P (fp32), so that a token equal to its centre gets Y - P[a] = 0 exactly (the
-// same products summed in the same order).
+// same products summed in the same order).  blockIdx.y selects the tensor
+// (maps0 / a0 or maps1 / a1), so the short P passes of K and V share a launch.
 template <int BITS, int G, bool PMODE>
-__global__ void __launch_bounds__(kEncThreads, 1) enc_kernel(const __grid_constant__ EncMaps maps, const EncArgs a) {
+__global__ void __launch_bounds__(kEncThreads, 1)
+    enc_kernel(const __grid_constant__ EncMaps maps0, const EncArgs a0, const __grid_constant__ EncMaps maps1,
+               const EncArgs a1) {
+  const EncMaps& maps = blockIdx.y ? maps1 : maps0;
+  const EncArgs a = blockIdx.y ? a1 : a0;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kEncBar);
@@ -508,12 +513,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_kernel(const __grid_consta
   }
 }
 
+// one tensor (n = 1) or two of the same row count (n = 2: m1 / a1 as the second)
 template <int BITS, int G, bool PMODE = false>
-static cudaError_t launch_enc(const EncMaps& m, const EncArgs& a, cudaStream_t st) {
+static cudaError_t launch_enc(const EncMaps& m, const EncArgs& a, cudaStream_t st, int n = 1,
+                              const EncMaps* m1 = nullptr, const EncArgs* a1 = nullptr) {
   auto k = enc_kernel<BITS, G, PMODE>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmem);
   if (e != cudaSuccess) return e;
-  k<<<(unsigned)((a.T + 127) / 128), kEncThreads, kEncSmem, st>>>(m, a);
+  const dim3 grid((unsigned)((a.T + 127) / 128), (unsigned)n);
+  k<<<grid, kEncThreads, kEncSmem, st>>>(m, a, n == 2 ? *m1 : m, n == 2 ? *a1 : a);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -552,19 +560,31 @@ cudaError_t tc_cluster_encode(const kvc_layer_desc* d, const kvc_predictor* p, c
     return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
-  // P = C E^T by the same tensor-core accumulation as the tokens' X E^T
-  {
-    tc::cluster::EncMaps pm = m;
-    if (!tc::map2d(&pm.x, cent, (uint64_t)p->n_clusters, C, 128)) return cudaErrorInvalidValue;
-    tc::cluster::EncArgs pa{err, (int64_t)p->n_clusters, (int)C, p->n_clusters, cnorm, P, nullptr, nullptr, nullptr};
-    cudaError_t e = tc::cluster::launch_enc<4, 32, true>(pm, pa, st);
-    if (e != cudaSuccess) return e;
-  }
   tc::cluster::EncArgs a{err, (int64_t)T, (int)C, p->n_clusters, cnorm, P, (uint8_t*)codes, (__half2*)params,
                          (uint8_t*)assign};
   if (d->bits == 2)
     return d->group == 32 ? tc::cluster::launch_enc<2, 32>(m, a, st) : tc::cluster::launch_enc<2, 64>(m, a, st);
   return d->group == 32 ? tc::cluster::launch_enc<4, 32>(m, a, st) : tc::cluster::launch_enc<4, 64>(m, a, st);
+}
+
+cudaError_t tc_cluster_prepare(const kvc_layer_desc* d, const kvc_predictor* p, const float* const cnorm[2],
+                               float* const P[2], cudaStream_t st) {
+  const uint64_t C = (uint64_t)d->n_heads * d->head_dim;
+  const void* cent[2] = {p->k_centroids, p->v_centroids};
+  const void* enc[2] = {p->k_enc, p->v_enc};
+  unsigned* err = tc_error_word();
+  if (!err) return cudaErrorInvalidDevice;
+  tc::cluster::EncMaps m[2];
+  tc::cluster::EncArgs a[2];
+  for (int w = 0; w < 2; ++w) {
+    memset(&m[w], 0, sizeof(m[w]));
+    if (!(tc::map2d(&m[w].x, cent[w], (uint64_t)p->n_clusters, C, 128) &&
+          tc::map2d(&m[w].cent, cent[w], (uint64_t)p->n_clusters, C, 256) && tc::map2d(&m[w].enc, enc[w], 128, C, 128)))
+      return cudaErrorInvalidValue;
+    a[w] = tc::cluster::EncArgs{err, (int64_t)p->n_clusters, (int)C, p->n_clusters, cnorm[w], P[w],
+                                nullptr, nullptr, nullptr};
+  }
+  return tc::cluster::launch_enc<4, 32, true>(m[0], a[0], st, 2, &m[1], &a[1]);
 }
 
 cudaError_t tc_cluster_decode(const kvc_layer_desc* d, const kvc_predictor* p, const void* codes, const void* params,
