@@ -27,16 +27,17 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint3
 namespace temporal {
 
 constexpr int kThreads = 320;
-constexpr int kKb = 0;                   // K^ tiles [2] (frame f in buffer f & 1)
-constexpr int kVb = kKb + 2 * 32768;     // V^ tile
-constexpr int kAK = kVb + 32768;         // AK_h as 4 sub-tiles [128 out][64 in]
+constexpr int kAK = 0;                   // AK_h as 4 sub-tiles [128 out][64 in]
 constexpr int kAV = kAK + 65536;         // AV_h
-constexpr int kBar = kAV + 65536;
+constexpr int kX = kAV + 65536;          // three staged [128][128] bf16 tiles: x of K(f), V(f) in turn
+                                         // (encode); the supplied history at the start (continuation)
+constexpr int kBar = kX + 3 * 32768;
 constexpr int kSmem = kBar + 1024 + 1024;
 
 struct Maps {
   CUtensorMap ak, av;      // [H*128][256]
   CUtensorMap ksrc, vsrc;  // history: [2F][C], [F][C] (continuation only)
+  CUtensorMap xk, xv;      // clean K, V [T][C] (encode)
 };
 
 struct Args {
@@ -53,6 +54,16 @@ struct Args {
   __nv_bfloat16* vrec;  // optional
 };
 
+// 16 consecutive 32-bit TMEM columns of this thread's lane (no wait)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]), "r"(w[9]),
+      "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
+
 template <bool ENC, int G>
 __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_constant__ Maps maps, const Args a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -61,10 +72,13 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
   uint64_t* w_full = bars;           // maps (+ history) landed
   uint64_t* kacc_full = bars + 1;    // K prediction of a frame in TMEM
   uint64_t* vacc_full = bars + 2;    // V prediction of a frame in TMEM
-  uint64_t* kready = bars + 3;       // K^ of a frame in its tile (K epilogue, 128 arrivals)
-  uint64_t* vready = bars + 4;       // V^ of a frame in its tile (V epilogue)
+  uint64_t* kready = bars + 3;       // K^ of a frame in its TMEM slot (K epilogue, 128 arrivals)
+  uint64_t* vready = bars + 4;       // V^ of a frame in its TMEM slot (V epilogue)
   uint64_t* mma_done = bars + 5;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
+  uint64_t* h_ready = bars + 6;      // initial history in TMEM (both epilogue groups, 256 arrivals)
+  uint64_t* x_full = bars + 7;       // [3] staged tile landed
+  uint64_t* x_free = bars + 10;      // [3] staged tile read (128 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -75,8 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
   const int64_t F = a.F;
   const int nf = (int)((a.T + F - 1) / F);
   const bool cont = a.anchor_bits == 0;
-  auto Kb = [&](int f) { return smem + kKb + (f & 1) * 32768; };
-  uint8_t* Vb = smem + kVb;
+  auto xs = [&](int i) { return smem + kX + (i % 3) * 32768; };  // staged tile of ring item i
 
   if (threadIdx.x == 0) {
     mbar_init(w_full, 1);
@@ -85,58 +98,95 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
     mbar_init(kready, 128);
     mbar_init(vready, 128);
     mbar_init(mma_done, 1);
+    mbar_init(h_ready, 256);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&x_full[i], 1);
+      mbar_init(&x_free[i], 128);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
   }
-  // without a history the lag-2 input of frame 1 is zero: clear the tile of frame -1
-  if (!cont)
-    for (int e = threadIdx.x; e < 32768 / 16; e += kThreads) reinterpret_cast<uint4*>(Kb(1))[e] = make_uint4(0, 0, 0, 0);
-  fence_async_smem();
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // K accumulator cols [0,128), V accumulator [128,256)
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: K accumulator [0,128), V accumulator [128,256), then the
+  // reconstructed state as bf16 pairs (the A operands of the predictions): K^ of
+  // frame f in [256 + 64 (f & 1), +64), V^ of the previous frame in [384, 448)
+  const uint32_t KACC = tmem, VACC = tmem + 128;
+  auto KH = [&](int f) { return tmem + 256 + (uint32_t)(f & 1) * 64; };
+  const uint32_t VH = tmem + 384;
 
   if (warp == 0) {
     if (lane == 0) {
+      // ================================================================ TMA: maps, history, staged x
       const uint64_t pol = policy_evict_last();
+      const uint64_t pol_x = policy_evict_first();
       mbar_arrive_expect_tx(w_full, 131072u + (cont ? 98304u : 0u));
       for (int c = 0; c < 4; ++c) {
         tma_load(smem + kAK + c * 16384, &maps.ak, c * 64, h * 128, w_full, pol);
         tma_load(smem + kAV + c * 16384, &maps.av, c * 64, h * 128, w_full, pol);
       }
-      if (cont) {  // K^ of frames -1 (tile 1) and -2 (tile 0), V^ of frame -1
+      if (cont) {  // K^ of frames -1 (slot 0) and -2 (slot 1), V^ of frame -1 (slot 2)
         for (int c = 0; c < 2; ++c) {
-          tma_load(Kb(1) + c * 16384, &maps.ksrc, h * 128 + c * 64, (int)(F + s0), w_full, pol);
-          tma_load(Kb(0) + c * 16384, &maps.ksrc, h * 128 + c * 64, s0, w_full, pol);
-          tma_load(Vb + c * 16384, &maps.vsrc, h * 128 + c * 64, s0, w_full, pol);
+          tma_load(xs(0) + c * 16384, &maps.ksrc, h * 128 + c * 64, (int)(F + s0), w_full, pol_x);
+          tma_load(xs(1) + c * 16384, &maps.ksrc, h * 128 + c * 64, s0, w_full, pol_x);
+          tma_load(xs(2) + c * 16384, &maps.vsrc, h * 128 + c * 64, s0, w_full, pol_x);
+        }
+      }
+      if (ENC) {
+        // ring items: x of K(f) is item 2f, x of V(f) item 2f + 1, in slot item % 3
+        bool ok = !cont || wait(h_ready, 0, abort_flag, a.err, 0x2120u);  // the history left the slots
+        int last = -1;
+        for (int i = 0; i < 2 * nf && ok; ++i) {
+          const int use = i / 3;
+          if (use >= 1 && !wait(&x_free[i % 3], (use - 1) & 1, abort_flag, a.err, 0x2121u)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap* m = (i & 1) ? &maps.xv : &maps.xk;
+          const int row = (int)((i >> 1) * F + s0);
+          mbar_arrive_expect_tx(&x_full[i % 3], 32768u);
+          tma_load(xs(i), m, h * 128, row, &x_full[i % 3], pol_x);
+          tma_load(xs(i) + 16384, m, h * 128 + 64, row, &x_full[i % 3], pol_x);
+          last = i;
+        }
+        if (*abort_flag) {  // the loads this thread issued land before the CTA can leave
+          for (int i = last - 2; i <= last; ++i) {
+            if (i < 0) continue;
+            const long long w0 = clock64();
+            while (!mbar_test(&x_full[i % 3], (i / 3) & 1) && clock64() - w0 < kWaitBudget) {
+            }
+          }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      bool ok = wait(w_full, 0, abort_flag, a.err, 0x2100u);
+      // ================================================================ MMA
+      bool ok = wait(w_full, 0, abort_flag, a.err, 0x2100u) && wait(h_ready, 0, abort_flag, a.err, 0x2101u);
       tc_fence_after();
       const uint32_t id = idesc_bf16(128, 128);
-      // D = [A0 | A1] W^T over 256 inputs: W as 4 sub-tiles of 64 inputs
-      auto mma256 = [&](uint32_t d, const uint8_t* A0, const uint8_t* A1, const uint8_t* W) {
+      // D = [A0 | A1] W^T over 256 inputs, A0 / A1 in TMEM (64 columns of bf16 pairs
+      // each), W as 4 sub-tiles of 64 inputs
+      auto mma256 = [&](uint32_t d, uint32_t A0, uint32_t A1, const uint8_t* W) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const uint64_t ad = desc_sw128(smem_u32((c < 2 ? A0 : A1) + (c & 1) * 16384));
+          const uint32_t ab = (c < 2 ? A0 : A1) + (uint32_t)(c & 1) * 32;
           const uint64_t bd = desc_sw128(smem_u32(W + c * 16384));
 #pragma unroll
-          for (int k = 0; k < 4; ++k) umma(d, ad + 2 * k, bd + 2 * k, id, (c == 0 && k == 0) ? 0u : 1u);
+          for (int k = 0; k < 4; ++k) umma_ts_if(1u, d, ab + k * 8, bd + 2 * k, id, (c == 0 && k == 0) ? 0u : 1u);
         }
       };
       int kr = 0, vr = 0;  // completions of kready / vready seen
-      // frame f's K prediction: [K^_{f-1} | K^_{f-2}] AK^T; K^_{f-2} sits in the tile of frame f
+      // frame f's K prediction: [K^_{f-1} | K^_{f-2}] AK^T; K^_{f-2} sits in the slot of frame f
       auto issue_k = [&](int f) {
-        mma256(tmem, Kb(f - 1), Kb(f), smem + kAK);
+        mma256(KACC, KH(f - 1), KH(f), smem + kAK);
         umma_commit(kacc_full);
       };
       if (cont && ok) issue_k(0);
@@ -151,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
           if (f > 0 && !wait(vready, vr++ & 1, abort_flag, a.err, 0x2111u)) ok = false;
           tc_fence_after();
           if (ok) {
-            mma256(tmem + 128, Kb(f), Vb, smem + kAV);
+            mma256(VACC, KH(f), VH, smem + kAV);
             umma_commit(vacc_full);
           }
         }
@@ -167,12 +217,47 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const int64_t s = s0 + row;
-    const uint32_t acc_addr = tmem + ((uint32_t)(q * 32) << 16) + (isv ? 128 : 0);
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t acc_addr = lane_off + (isv ? VACC : KACC);
     uint64_t* acc_full = isv ? vacc_full : kacc_full;
     int acc_use = 0;
     const int64_t F0 = cont ? 0 : (F < a.T ? F : a.T);
     const int arb = 128 * a.anchor_bits / 8;
+    // row r of a staged [128][128] bf16 tile (two 128-byte-swizzled 64-column sub-tiles) as 64 words
+    auto read_row = [&](const uint8_t* tile, uint4 (&w)[16]) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) w[c] = *reinterpret_cast<const uint4*>(tile + (c / 8) * 16384 + sw128_off(row, c % 8));
+    };
+    auto row_to_tmem = [&](const uint4 (&w)[16], uint32_t col) {
+      const uint32_t* u = reinterpret_cast<const uint32_t*>(w);
+      uint32_t lo[32], hi[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) lo[i] = u[i], hi[i] = u[32 + i];
+      tmem_st32u(lane_off + col, lo);
+      tmem_st32u(lane_off + col + 32, hi);
+    };
+    // the state before frame 0: the supplied history, or (no history) a zero
+    // K^ of frame -1 as the lag-2 input of frame 1
     wait(w_full, 0, abort_flag, a.err, 0x2200u);
+    if (cont) {
+      uint4 w[16];
+      if (!isv) {
+        read_row(xs(0), w);
+        row_to_tmem(w, KH(-1) - tmem);
+        read_row(xs(1), w);
+        row_to_tmem(w, KH(-2) - tmem);
+      } else {
+        read_row(xs(2), w);
+        row_to_tmem(w, VH - tmem);
+      }
+    } else if (!isv) {
+      uint4 w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) w[i] = make_uint4(0, 0, 0, 0);
+      row_to_tmem(w, KH(-1) - tmem);
+    }
+    tc_fence_before();
+    mbar_arrive(h_ready);
     for (int f = 0; f < nf; ++f) {
       const int64_t n_f = (a.T - f * F) < F ? (a.T - f * F) : F;
       const bool valid = s < n_f;
@@ -189,11 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       uint4 xin[16];
       uint4 cin[4];
       __half2 pin[NG];
-      if (ENC) {
-        const __nv_bfloat16* X = (isv ? a.V : a.K) + t * C + h * 128;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          xin[i] = valid ? __ldcs(reinterpret_cast<const uint4*>(X) + i) : make_uint4(0, 0, 0, 0);
+      if (ENC) {  // x of this row from the staged tile, which is then released
+        const int i = 2 * f + (isv ? 1 : 0);
+        wait(&x_full[i % 3], (i / 3) & 1, abort_flag, a.err, 0x2220u + isv);
+        read_row(xs(i), xin);
+        mbar_arrive(&x_free[i % 3]);
       } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -208,7 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
         acc_use++;
         tc_fence_after();
       }
-      uint8_t* tile = isv ? Vb : Kb(f);
+      // the new state goes to the slot its own prediction was the last to read
+      const uint32_t state = lane_off + (isv ? VH : KH(f));
       uint32_t cw[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
       const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
       __nv_bfloat16* rec = isv ? a.vrec : a.krec;
@@ -259,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
           } else {
             tmem_ld32(acc_addr + e0, p);
           }
-          uint4 recw[4];
+          uint32_t recw[16];  // 32 reconstructed values as bf16 pairs
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             const int e = e0 + ch * 8;
@@ -277,17 +363,16 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
               else
                 dequant8<4>(cwin[e / 8], e, sf, zf, &p[ch * 8], r);
             }
-            uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(r[2 * i], r[2 * i + 1]);
-            recw[ch] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int i = 0; i < 4; ++i) recw[ch * 4 + i] = pack_bf16x2(r[2 * i], r[2 * i + 1]);
           }
-          // the tile of K^_f is being read by K(f)'s MMA (lag 2) until acc_full: safe now
+          // the slot was last read by this frame's prediction, which is complete (acc_full)
+          tmem_st16(state + e0 / 2, recw);
+          if (rec && valid) {
+            uint4* dst = reinterpret_cast<uint4*>(rec + t * C + h * 128 + e0);
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int e = e0 + ch * 8;
-            *reinterpret_cast<uint4*>(tile + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) = recw[ch];
-            if (rec && valid) reinterpret_cast<uint4*>(rec + t * C + h * 128 + e)[0] = recw[ch];
+            for (int ch = 0; ch < 4; ++ch)
+              dst[ch] = make_uint4(recw[4 * ch], recw[4 * ch + 1], recw[4 * ch + 2], recw[4 * ch + 3]);
           }
         }
       }
@@ -297,11 +382,9 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
         for (int i = 0; i < 4; ++i)
           if (i * 16 < row_bytes) dst[i] = make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]);
       }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      fence_async_smem();
       mbar_arrive(isv ? vready : kready);
-      // the V epilogue of frame f needs K^_f in the tile before the MMA of V(f) reads both;
-      // the MMA waits kready(f) and vready(f-1), so no extra ordering is needed here
     }
   }
 
@@ -309,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -345,6 +428,7 @@ cudaError_t tc_temporal_layer(const kvc_layer_desc* d, const kvc_predictor* p, b
   memset(&m, 0, sizeof(m));
   bool ok = tc::map2d(&m.ak, p->k_block, H * 128, 256, 128) && tc::map2d(&m.av, p->v_block, H * 128, 256, 128);
   if (ok && d->anchor_bits == 0) ok = tc::map2d(&m.ksrc, Ks, 2 * F, C, 128) && tc::map2d(&m.vsrc, Vs, F, C, 128);
+  if (ok && enc) ok = tc::map2d(&m.xk, K, (uint64_t)d->n_tokens, C, 128) && tc::map2d(&m.xv, V, (uint64_t)d->n_tokens, C, 128);
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
