@@ -817,6 +817,22 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint3
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [frames][rows][cols] view of a row-major [frames * rows][cols] tensor,
+// boxes of box_rows x 64 columns of one frame with the 128-byte swizzle: a box
+// that reaches past a frame's last row is clipped there.
+bool map3d_frames(CUtensorMap* m, const void* base, uint64_t frames, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, frames};
+  cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Streaming multiprocessors of the current device (0 on error).
 static int sm_count() {
   static int cached[64] = {};

@@ -23,6 +23,8 @@ namespace kvc {
 namespace tc {
 
 bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool map3d_frames(CUtensorMap* m, const void* base, uint64_t frames, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows);
 
 namespace temporal {
 
@@ -38,6 +40,9 @@ struct Maps {
   CUtensorMap ak, av;      // [H*128][256]
   CUtensorMap ksrc, vsrc;  // history: [2F][C], [F][C] (continuation only)
   CUtensorMap xk, xv;      // clean K, V [T][C] (encode)
+  // reconstructions written by decode: whole frames as [frames][F][C], the
+  // partial last frame as [rows][C]
+  CUtensorMap kr3, vr3, krt, vrt;
 };
 
 struct Args {
@@ -53,6 +58,13 @@ struct Args {
   __nv_bfloat16* krec;  // optional
   __nv_bfloat16* vrec;  // optional
 };
+
+__device__ __forceinline__ void tma_store3(const CUtensorMap* m, int x, int y, int z, const void* src) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
+               : "memory");
+}
 
 // 16 consecutive 32-bit TMEM columns of this thread's lane (no wait)
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
@@ -258,6 +270,20 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
     }
     tc_fence_before();
     mbar_arrive(h_ready);
+    // Decode writes the reconstruction through a staged tile (K: slot 0, V: slot
+    // 2, idle in decode once the history is in TMEM) and TMA stores of one frame's
+    // rows; encode (whose ring holds x) stores it row by row when asked for.
+    __nv_bfloat16* rec = isv ? a.vrec : a.krec;
+    const bool stage = !ENC && rec != nullptr;
+    uint8_t* stile = xs(isv ? 2 : 0);
+    const bool elected = warp == (isv ? 6 : 2) && lane == 0;
+    auto gsync = [&] {
+      if (isv)
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+      else
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+    };
+    const int64_t nff = a.T / F;  // whole frames
     for (int f = 0; f < nf; ++f) {
       const int64_t n_f = (a.T - f * F) < F ? (a.T - f * F) : F;
       const bool valid = s < n_f;
@@ -297,7 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       const uint32_t state = lane_off + (isv ? VH : KH(f));
       uint32_t cw[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
       const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
-      __nv_bfloat16* rec = isv ? a.vrec : a.krec;
+      if (stage) {  // the staged tile's previous store has read it
+        if (elected) bulk_wait_read0();
+        gsync();
+      }
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         float sf, zf;
@@ -368,7 +397,14 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
           }
           // the slot was last read by this frame's prediction, which is complete (acc_full)
           tmem_st16(state + e0 / 2, recw);
-          if (rec && valid) {
+          if (stage) {
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              const int e = e0 + ch * 8;
+              *reinterpret_cast<uint4*>(stile + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =
+                  make_uint4(recw[4 * ch], recw[4 * ch + 1], recw[4 * ch + 2], recw[4 * ch + 3]);
+            }
+          } else if (rec && valid) {
             uint4* dst = reinterpret_cast<uint4*>(rec + t * C + h * 128 + e0);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch)
@@ -385,7 +421,24 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       mbar_arrive(isv ? vready : kready);
+      if (stage) {  // rows past the frame's end are clipped by the maps
+        fence_async_smem();
+        gsync();
+        if (elected && s0 < n_f) {
+          if (f < nff) {
+            const CUtensorMap* m = isv ? &maps.vr3 : &maps.kr3;
+            tma_store3(m, h * 128, s0, f, stile);
+            tma_store3(m, h * 128 + 64, s0, f, stile + 16384);
+          } else {
+            const CUtensorMap* m = isv ? &maps.vrt : &maps.krt;
+            tma_store(m, h * 128, s0, stile);
+            tma_store(m, h * 128 + 64, s0, stile + 16384);
+          }
+          bulk_commit();
+        }
+      }
     }
+    if (elected) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -429,6 +482,15 @@ cudaError_t tc_temporal_layer(const kvc_layer_desc* d, const kvc_predictor* p, b
   bool ok = tc::map2d(&m.ak, p->k_block, H * 128, 256, 128) && tc::map2d(&m.av, p->v_block, H * 128, 256, 128);
   if (ok && d->anchor_bits == 0) ok = tc::map2d(&m.ksrc, Ks, 2 * F, C, 128) && tc::map2d(&m.vsrc, Vs, F, C, 128);
   if (ok && enc) ok = tc::map2d(&m.xk, K, (uint64_t)d->n_tokens, C, 128) && tc::map2d(&m.xv, V, (uint64_t)d->n_tokens, C, 128);
+  if (ok && !enc) {
+    const uint64_t T = (uint64_t)d->n_tokens, nff = T / F, tail = T - nff * F;
+    auto maps_for = [&](void* r, CUtensorMap* m3, CUtensorMap* mt) {
+      if (!r) return true;
+      return (nff == 0 || tc::map3d_frames(m3, r, nff, F, C, 128)) &&
+             (tail == 0 || tc::map2d(mt, static_cast<char*>(r) + nff * F * C * 2, tail, C, 128));
+    };
+    ok = maps_for(Kr, &m.kr3, &m.krt) && maps_for(Vr, &m.vr3, &m.vrt);
+  }
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
