@@ -48,7 +48,8 @@ UNIT = "KV tokens/s"
 # kernel changes after its capture.
 TRAFFIC = {"encode_xlayer": 674717696 + 202756608, "decode_xlayer": 437384192 + 152241920,
            "attention_c2": 769948672 + 8668416, "attention_c4": 26442240 + 768,
-           "temporal_encode": None}
+           "temporal_encode": 1425952000 + 356744960,
+           "temporal_decode": 574324480 + 1285428224}
 
 
 def peaks():
@@ -323,7 +324,7 @@ def row_temporal(dev, hbm, reps=3) -> dict:
         gbs = byts / (ms * 1e-3) / 1e9
         out[name] = {"ms": ms, "tokens_per_s": T / (ms * 1e-3),
                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                                  "traffic": TRAFFIC["temporal_encode"] if name == "encode" else None}}
+                                  "traffic": TRAFFIC["temporal_" + name]}}
     out["workload"] = "temporal codec, one layer: 65536 tokens x 40 heads x 128, 1560-token frames, INT4 g64"
     return out
 
