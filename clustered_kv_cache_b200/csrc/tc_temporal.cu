@@ -6,13 +6,16 @@
 //
 // One CTA per (128-position tile, head) walks every frame of the call in order.
 // The head's two 128x256 maps stay in shared memory; the reconstructed state
-// lives in three bf16 tiles (K of frames f and f-1, V of frame f-1) that serve
-// directly as MMA operands: each new reconstruction overwrites the tile that
-// its own prediction was the last to read.  Per frame the MMA of V(f) and of
-// K(f+1) are issued together once K^_f exists, and two epilogue groups
-// quantize V(f) and K(f+1) side by side.
+// (K of frames f and f-1, V of frame f-1) lives in tensor memory as bf16 pairs
+// and is the A operand of the prediction MMAs: each new reconstruction
+// overwrites the slot that its own prediction was the last to read.  Per frame
+// the MMA of V(f) and of K(f+1) are issued together once K^_f exists, and two
+// epilogue groups quantize V(f) and K(f+1) side by side.  A three-slot ring of
+// shared-memory tiles moved by TMA carries x to the encode epilogues about a
+// frame ahead, the reconstruction out of the decode epilogues, and the supplied
+// history of a continuation call into tensor memory.
 //
-// Warp roles: 0 TMA (maps, history), 1 MMA + TMEM, 2-5 K epilogue, 6-9 V epilogue.
+// Warp roles: 0 TMA (maps, history, x), 1 MMA + TMEM, 2-5 K epilogue, 6-9 V epilogue.
 #include <cuda.h>
 #include <string.h>
 
