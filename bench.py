@@ -47,7 +47,7 @@ UNIT = "KV tokens/s"
 # mixed_attention_cluster.md, temporal_codec_layer.md); set to None when a
 # kernel changes after its capture.
 TRAFFIC = {"encode_xlayer": 674717696 + 202756608, "decode_xlayer": 437384192 + 152241920,
-           "attention_c2": 769948672 + 8668416, "attention_c4": 26442240 + 768,
+           "attention_c2": 769948672 + 8668416, "attention_c4": None,
            "temporal_encode": 1425952000 + 356744960,
            "temporal_decode": 574324480 + 1285428224}
 

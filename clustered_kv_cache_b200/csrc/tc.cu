@@ -891,10 +891,10 @@ bool tc_codec_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
   return tc::encode_fn() != nullptr;
 }
 
-size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int64_t) {
+size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int64_t n_q) {
   if (op != KVC_OP_ATTEND) return 0;
   if (tc_attend_supported(d, p, 0)) return tc_attend_workspace(d, p);
-  if (tc_mixed_supported(d, p)) return tc_mixed_workspace(d);
+  if (tc_mixed_supported(d, p)) return tc_mixed_workspace(d, n_q);
   return 0;
 }
 

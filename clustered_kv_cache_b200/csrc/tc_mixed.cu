@@ -68,6 +68,12 @@ struct Args {
   const uint8_t* assign_k;  // [T]
   const uint8_t* assign_v;
   __nv_bfloat16* O;  // [n_q][H][128]
+  // key splits: with ks > 1 this launch's keys are one split of the history
+  // and the kernel writes its unnormalised output, running max and sum to
+  // opart [n_q][H][128] and ml [n_q][H][2] (this split's part of the workspace)
+  int ks;
+  float* opart;
+  float* ml;
 };
 
 __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
@@ -178,7 +184,12 @@ __global__ void coef_dequant_kernel(const uint8_t* codes, const __half2* params,
 
 // ---------------------------------------------------------------- the attention kernel
 
-__global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constant__ Maps maps, const Args a) {
+// blockIdx.z picks the key split (maps0 / a0 or maps1 / a1: the split's keys,
+// assignments and coefficients, offsets applied by the host)
+__global__ void __launch_bounds__(kThreads, 1)
+    mixed_kernel(const __grid_constant__ Maps maps0, const Args a0, const __grid_constant__ Maps maps1, const Args a1) {
+  const Maps& maps = blockIdx.z ? maps1 : maps0;
+  const Args a = blockIdx.z ? a1 : a0;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBar);
@@ -517,12 +528,21 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
     wait(o_done, 0, abort_flag, a.err, 0x2402u);
     tc_fence_after();
     const int64_t qrow = (int64_t)q0 + row;
+    // one split: O / l as bf16; several: this split's O (relative to 2^m_used)
+    // and (m_used, l), merged by the combine kernel
+    const bool part = a.ks > 1;
+    if (part && qrow < a.n_q) *reinterpret_cast<float2*>(a.ml + (qrow * a.H + h) * 2) = make_float2(m_used, l);
     const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
+#pragma unroll 1
     for (int pc = 0; pc < 4; ++pc) {
       float ov[32];
       tmem_ld32(lane_addr + (OC - tmem) + pc * 32, ov);
-      if (qrow < a.n_q) {
+      if (qrow >= a.n_q) continue;
+      if (part) {
+        float4* dst = reinterpret_cast<float4*>(a.opart + (qrow * a.H + h) * 128 + pc * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+      } else {
         uint4* dst = reinterpret_cast<uint4*>(a.O + (qrow * a.H + h) * 128 + pc * 32);
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -543,10 +563,49 @@ __global__ void __launch_bounds__(kThreads, 1) mixed_kernel(const __grid_constan
   }
 }
 
+// Merge of the key splits of every (query, head) row: with m the largest of the
+// splits' running maxima, O = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
+// One warp per row, four channels a lane.
+__global__ void combine_kernel(const float* opart, const float* ml, int ks, int64_t rows, __nv_bfloat16* O) {
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (r >= rows) return;
+  const int lane = threadIdx.x & 31;
+  float m = -INFINITY;
+  for (int s = 0; s < ks; ++s) m = fmaxf(m, ml[(s * rows + r) * 2]);
+  float l = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < ks; ++s) {
+    const float2 sl = *reinterpret_cast<const float2*>(ml + (s * rows + r) * 2);
+    const float w = sl.x == -INFINITY ? 0.f : exp2f(sl.x - m);
+    l += w * sl.y;
+    const float4 v = reinterpret_cast<const float4*>(opart + (s * rows + r) * 128)[lane];
+    o.x += w * v.x;
+    o.y += w * v.y;
+    o.z += w * v.z;
+    o.w += w * v.w;
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  reinterpret_cast<uint2*>(O + r * 128)[lane] = make_uint2(pack_bf16x2(o.x * inv, o.y * inv), pack_bf16x2(o.z * inv, o.w * inv));
+}
+
 }  // namespace mixed
 }  // namespace tc
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+namespace {
+constexpr int kMaxSplits = 2;
+size_t mixed_parts_bytes(const kvc_layer_desc* d, int64_t n_q) {
+  const size_t rows = (size_t)(n_q > 0 ? n_q : 0) * d->n_heads;
+  return align256(kMaxSplits * rows * 128 * sizeof(float)) + align256(kMaxSplits * rows * 2 * sizeof(float));
+}
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+}  // namespace
+
 
 bool tc_mixed_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
   if (p->kind != KVC_PRED_CLUSTER) return false;
@@ -558,12 +617,16 @@ bool tc_mixed_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
   return true;
 }
 
-size_t tc_mixed_workspace(const kvc_layer_desc* d) { return 2 * align256((size_t)d->n_tokens * 128 * 2); }
+// dequantized coefficients of K and V, then room for the key splits' partial results
+size_t tc_mixed_workspace(const kvc_layer_desc* d, int64_t n_q) {
+  return 2 * align256((size_t)d->n_tokens * 128 * 2) + mixed_parts_bytes(d, n_q);
+}
 
 cudaError_t tc_mixed_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
                             const kvc_codes* c, float scale, void* O, void* ws, size_t ws_bytes, cudaStream_t st) {
   const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128;
-  if (ws_bytes < tc_mixed_workspace(d)) return cudaErrorInvalidValue;
+  const size_t coef_bytes = 2 * align256((size_t)T * 128 * 2);
+  if (ws_bytes < coef_bytes) return cudaErrorInvalidValue;
   __nv_bfloat16* ckh = static_cast<__nv_bfloat16*>(ws);
   __nv_bfloat16* cvh = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + align256(T * 128 * 2));
   // dequantized coefficients of every token
@@ -585,15 +648,47 @@ cudaError_t tc_mixed_attend(const kvc_layer_desc* d, const kvc_predictor* p, con
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
-  tc::mixed::Args a{err, n_q, (int64_t)T, (int)H, p->n_clusters, scale * 1.4426950408889634f,
-                    (const __nv_bfloat16*)p->k_centroids, (const __nv_bfloat16*)p->v_centroids,
-                    (const uint8_t*)c->k_assign, (const uint8_t*)c->v_assign, (__nv_bfloat16*)O};
+  // Two key splits when they shorten the run: (query tile, head) CTAs in waves
+  // of one per SM, each split half as long; the splits' partials are merged after.
+  const int64_t tiles = (n_q + 127) / 128 * (int64_t)H;
+  const int64_t nkt = ((int64_t)T + tc::mixed::kKeys - 1) / tc::mixed::kKeys;
+  const int sms = device_sms();
+  int ks = 1;
+  if (sms > 0 && nkt >= 2 && ws_bytes >= coef_bytes + mixed_parts_bytes(d, n_q)) {
+    const int64_t w1 = (tiles + sms - 1) / sms, w2 = (2 * tiles + sms - 1) / sms;
+    if (w2 < 2 * w1) ks = 2;  // 2 splits of half the work: w2 / 2 < w1
+  }
+  float* opart = reinterpret_cast<float*>(static_cast<char*>(ws) + coef_bytes);
+  float* ml = reinterpret_cast<float*>(static_cast<char*>(ws) + coef_bytes +
+                                       align256(kMaxSplits * (size_t)n_q * H * 128 * sizeof(float)));
+  const int64_t rows = n_q * (int64_t)H;
+  tc::mixed::Args a0{err, n_q, (int64_t)T, (int)H, p->n_clusters, scale * 1.4426950408889634f,
+                     (const __nv_bfloat16*)p->k_centroids, (const __nv_bfloat16*)p->v_centroids,
+                     (const uint8_t*)c->k_assign, (const uint8_t*)c->v_assign, (__nv_bfloat16*)O, ks, opart, ml};
+  tc::mixed::Maps m1 = m;
+  tc::mixed::Args a1 = a0;
+  if (ks > 1) {  // split 0: the first ceil(tiles / 2) key tiles; split 1: the rest
+    const uint64_t T0 = (uint64_t)((nkt + 1) / 2) * tc::mixed::kKeys, T1 = T - T0;
+    a0.T = (int64_t)T0;
+    a1.T = (int64_t)T1;
+    a1.assign_k += T0;
+    a1.assign_v += T0;
+    a1.opart = opart + rows * 128;
+    a1.ml = ml + rows * 2;
+    if (!(tc::map2d(&m1.ckh, ckh + T0 * 128, T1, 128, tc::mixed::kKeys) &&
+          tc::map2d(&m1.cvh, cvh + T0 * 128, T1, 128, tc::mixed::kKeys)))
+      return cudaErrorInvalidValue;
+  }
   auto k = tc::mixed::mixed_kernel;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::mixed::kSmem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((n_q + 127) / 128), (unsigned)H);
-  k<<<grid, tc::mixed::kThreads, tc::mixed::kSmem, st>>>(m, a);
+  dim3 grid((unsigned)((n_q + 127) / 128), (unsigned)H, (unsigned)ks);
+  k<<<grid, tc::mixed::kThreads, tc::mixed::kSmem, st>>>(m, a0, m1, a1);
   count_launches(1);
+  if (ks > 1) {
+    tc::mixed::combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(opart, ml, ks, rows, (__nv_bfloat16*)O);
+    count_launches(1);
+  }
   return cudaGetLastError();
 }
 

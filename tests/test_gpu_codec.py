@@ -643,7 +643,10 @@ def test_tiny_fp32_attention():
         assert U.rel_l2(U.to64(Og), ref) <= U.ATT_TOL[f32]
 
 
-@pytest.mark.parametrize("n_q,T,H,n_c", [(100, 1000, 4, 32), (33, 300, 16, 256), (300, 2000 - 9, 16, 256)])
+# T = 60 is one key tile, so the kernel runs unsplit; the others run as two key
+# splits merged by the combine kernel
+@pytest.mark.parametrize("n_q,T,H,n_c", [(100, 1000, 4, 32), (33, 300, 16, 256), (300, 2000 - 9, 16, 256),
+                                         (70, 60, 4, 16)])
 def test_mixed_dimensional_attention(n_q, T, H, n_c):
     cw = synth.cluster_layer(seed=synth.SEED_BASE + 105, T=T, H=H, n_c=n_c, iters=3)
     D = 128
