@@ -258,6 +258,29 @@ def run_reference(args, rank: int):
 # ---------------------------------------------------------------- extra rows (N = 1)
 
 
+# ---------------------------------------------------------------- ranks (N > 1: weak scaling)
+
+
+def shard_seed(rank: int) -> int:
+    """Seed of a rank's own 32760-token shard (every rank codes different tokens)."""
+    return synth.SEED_BASE + 1 + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value: every multi-rank time is the max over ranks."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(ms_step: float, world: int, layers: int) -> float:
+    """Whole-job KV tokens/s: every rank's tokens, encoded and decoded through
+    every layer, over the slowest rank's step time."""
+    return 2 * T_TOK * layers * world / (ms_step * 1e-3)
+
+
 def synced_ok():
     """Waits for the device and fails on a kernel-reported error (an expired
     wait, a bad launch): a timing of such a run is no measurement."""
@@ -416,7 +439,7 @@ def main():
     build.build()
     hbm, tf_burst, tf_sust, peak_kind = peaks()
 
-    xb = XLayerBench(dev, synth.SEED_BASE + 1 + 1000 * rank, args.layers)
+    xb = XLayerBench(dev, shard_seed(rank), args.layers)
     L_RUN = args.layers
     torch.cuda.synchronize()
 
@@ -449,14 +472,9 @@ def main():
     launches = kvc.kvc_launch_counter() - launches0
     clk = clocks.stop()
     assert kvc.kvc_get_device_error() == 0
-    ms_total = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     ms_step = ms_total / args.steps
-    units_per_step = 2 * T_TOK * L_RUN * world
-    value = units_per_step / (ms_step * 1e-3)
+    value = job_value(ms_step, world, L_RUN)
 
     enc_ms = statistics.mean(x for k in range(args.steps) for x in time_events(ev_enc[k][1:]))
     dec_ms = statistics.mean(x for k in range(args.steps) for x in time_events(ev_dec[k][1:]))
@@ -504,12 +522,8 @@ def main():
             e2e_step()
         e.record()
         torch.cuda.synchronize()
-        ms_e2e = s.elapsed_time(e) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": units_per_step / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": bi,
+        ms_e2e = max_over_ranks(s.elapsed_time(e) / args.e2e_steps, world, dev)
+        e2e = {"value": job_value(ms_e2e, world, L_RUN), "unit": UNIT, "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": bo, "ms_per_step": ms_e2e}
         del hK, hV, hcodes
 
