@@ -436,7 +436,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     from clustered_kv_cache_b200 import build
 
-    build.build()
+    # one rank builds (if the in-tree library is stale); the others wait for it
+    if rank == 0:
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
     hbm, tf_burst, tf_sust, peak_kind = peaks()
 
     xb = XLayerBench(dev, shard_seed(rank), args.layers)
