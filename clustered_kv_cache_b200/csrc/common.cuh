@@ -184,5 +184,7 @@ struct RowCodec {
 
 // adds n to the process-wide launch counter (kvc_launch_counter)
 void count_launches(unsigned long long n);
+// Records the text of a failed CUDA call for kvc_last_cuda_error() and returns KVC_ERR_CUDA.
+kvc_status record_cuda_error(cudaError_t e);
 
 }  // namespace kvc

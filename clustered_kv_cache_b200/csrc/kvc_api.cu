@@ -15,16 +15,18 @@ using namespace kvc;
 namespace kvc {
 static std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned long long n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+static thread_local char g_last_cuda[256] = "";
+
+kvc_status record_cuda_error(cudaError_t e) {
+  snprintf(g_last_cuda, sizeof(g_last_cuda), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return KVC_ERR_CUDA;
+}
 }  // namespace kvc
 
 namespace {
 
-thread_local char g_last_cuda[256] = "";
-
-kvc_status cuda_fail(cudaError_t e) {
-  snprintf(g_last_cuda, sizeof(g_last_cuda), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
-  return KVC_ERR_CUDA;
-}
+kvc_status cuda_fail(cudaError_t e) { return record_cuda_error(e); }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

@@ -8,6 +8,8 @@
 // handed out by someone else, or a plugin host that forbids cudaMalloc on its
 // threads.  kvc_encode_layer_cluster_static keeps that scratch in a file-scope
 // __device__ array instead, so it allocates nothing.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -24,25 +26,59 @@ constexpr size_t kTableFloats = kMaxCentres + (size_t)kMaxCentres * kCodeDim;
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) float g_cluster_scratch[2 * kTableFloats];
 
+// Set-up, once per device: the device address of g_cluster_scratch, looked up
+// with that device current.  In host code the symbol's name is only a stand-in
+// for that address.  The address belongs to the device's current context, so
+// the cache also keeps that context's unique id and repeats the lookup when
+// the id changes (after cudaDeviceReset the next call sees a new context).
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-float* g_scratch_ptr[kMaxDevices] = {};
+struct ScratchSlot {
+  float* ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+ScratchSlot g_slot[kMaxDevices];
 
-// Device address of g_cluster_scratch on the current device; looked up once
-// per device (in host code the symbol is only a stand-in for that address).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if unknown).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 cudaError_t scratch_for_current_device(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long id = current_context_id();  // 0 before the runtime has made a context current
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  ScratchSlot& slot = g_slot[dev];
+  if (!slot.ptr || id == 0 || slot.ctx_id != id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_cluster_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = static_cast<float*>(p);
+    if ((e = cudaGetSymbolAddress(&p, g_cluster_scratch)) != cudaSuccess) return e;
+    slot.ptr = static_cast<float*>(p);
+    slot.ctx_id = current_context_id();  // the lookup made the device's primary context current
   }
-  *out = g_scratch_ptr[dev];
+  *out = slot.ptr;
   return cudaSuccess;
 }
 
@@ -78,7 +114,8 @@ extern "C" kvc_status kvc_encode_layer_cluster_static(const kvc_layer_desc* d, c
                                                       void* stream) {
   using namespace kvc;
   if (!d || !p || !c || p->kind != KVC_PRED_CLUSTER) return KVC_ERR_INVALID_ARGUMENT;
-  if (d->n_tokens < 0 || d->n_heads < 1 || (d->head_dim != 64 && d->head_dim != 128)) return KVC_ERR_INVALID_ARGUMENT;
+  if (d->n_tokens < 0 || d->n_heads < 1) return KVC_ERR_INVALID_ARGUMENT;
+  if (d->head_dim != 64 && d->head_dim != 128) return KVC_ERR_UNSUPPORTED;  // as kvc_encode_layer
   // the scratch array holds tables for at most 256 centres of 128 coefficients
   if (p->n_clusters < 1 || p->n_clusters > kMaxCentres || p->code_dim != kCodeDim) return KVC_ERR_UNSUPPORTED;
   if (d->dtype != KVC_F32 && d->dtype != KVC_BF16) return KVC_ERR_UNSUPPORTED;
@@ -95,9 +132,9 @@ extern "C" kvc_status kvc_encode_layer_cluster_static(const kvc_layer_desc* d, c
   }
   if ((K_rec && !aligned16(K_rec)) || (V_rec && !aligned16(V_rec))) return KVC_ERR_MISALIGNED;
   float* scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) return KVC_ERR_CUDA;
+  cudaError_t e = scratch_for_current_device(&scratch);
+  if (e != cudaSuccess) return record_cuda_error(e);
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e;
   if (d->dtype == KVC_F32) {
     e = d->param_dtype == KVC_F32 ? encode<float, float>(d, p, K, V, c, K_rec, V_rec, scratch, st)
                                   : encode<float, __half>(d, p, K, V, c, K_rec, V_rec, scratch, st);
@@ -105,5 +142,5 @@ extern "C" kvc_status kvc_encode_layer_cluster_static(const kvc_layer_desc* d, c
     e = d->param_dtype == KVC_F32 ? encode<__nv_bfloat16, float>(d, p, K, V, c, K_rec, V_rec, scratch, st)
                                   : encode<__nv_bfloat16, __half>(d, p, K, V, c, K_rec, V_rec, scratch, st);
   }
-  return e == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  return e == cudaSuccess ? KVC_OK : record_cuda_error(e);
 }

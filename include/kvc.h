@@ -233,9 +233,10 @@ KVC_API uint64_t kvc_launch_counter(void);
  *  at most 256 centres of 128 coefficients (about 264 KB, held by every GPU that
  *  loads the library until the process exits); larger n_clusters or another
  *  code_dim return KVC_ERR_UNSUPPORTED before anything runs.
- *  It calls no cudaMalloc / cudaFree.  The first call on a device looks up the
- *  array's device address (cudaGetSymbolAddress), so make that first call
- *  before any stream capture.  Every call writes the whole table before
+ *  It calls no cudaMalloc / cudaFree.  The first call on a device (and the
+ *  first after that device's context was replaced, e.g. by cudaDeviceReset)
+ *  looks up the array's device address (cudaGetSymbolAddress), so make that
+ *  first call before any stream capture.  Every call writes the whole table before
  *  reading it, so nothing carries over between calls, but all calls share the
  *  one array: calls that can overlap on the GPU (other streams, other threads)
  *  race and must be serialized by the caller. */

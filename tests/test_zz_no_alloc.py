@@ -32,6 +32,13 @@ def test_static_entry_rejects_more_centres_than_its_array_holds():
         pred = kvc.Predictor(kvc.PRED_CLUSTER, 0, n_c, m, *([0x1000] * 12))
         assert fn(ctypes.byref(desc), ctypes.byref(pred), ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1000),
                   ctypes.byref(c), None, None, None) == 2
+    # a head_dim the library does not implement: the same status as kvc_encode_layer
+    odd = kvc.make_desc(100, 2, 96, torch.bfloat16, 4, 32, torch.float16)
+    pred = kvc.Predictor(kvc.PRED_CLUSTER, 0, 16, 128, *([0x1000] * 12))
+    args = (ctypes.byref(odd), ctypes.byref(pred), ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1000), ctypes.byref(c))
+    assert fn(*args, None, None, None) == 2
+    assert L.kvc_encode_layer(args[0], args[1], args[2], args[3], None, None, args[4], None, None, None,
+                              ctypes.c_size_t(0), None) == 2
 
 
 @pytest.mark.gpu
