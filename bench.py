@@ -185,22 +185,26 @@ def time_events(pairs):
 # ---------------------------------------------------------------- oracle timing (CPU)
 
 
-def blas_threads() -> int:
+def cpu_model() -> str:
     try:
-        from threadpoolctl import threadpool_info
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return 1
 
+def oracle_xlayer_rate(wl, n_tok: int, layers: int, budget_s: float, threads: int = 1) -> dict:
+    """Times the plain fp64 C++ oracle's closed-loop encode + decode of `n_tok`
+    tokens through `layers` layers (tokens are independent, so this is an exact
+    sample of the workload).  threads = 1: the single-threaded oracle; more:
+    its thread driver over disjoint token runs.  Returns tokens/s (encoded +
+    decoded)."""
+    from oracle import kvc_oracle_c as O
 
-def oracle_xlayer_rate(wl, n_tok: int, layers: int, budget_s: float) -> dict:
-    """Times the fp64 oracle's closed-loop encode + decode of `n_tok` tokens
-    through `layers` layers (tokens are independent, so this is an exact sample
-    of the workload).  Returns tokens/s (encoded + decoded)."""
-    from oracle import kvc_oracle as O
-
+    O.build()
     idx = torch.linspace(0, wl.K[0].shape[0] - 1, n_tok).long()
     t64 = lambda t: t[idx.to(t.device)].detach().cpu().double().numpy()
     K = [t64(k) for k in wl.K[:layers]]
@@ -210,20 +214,38 @@ def oracle_xlayer_rate(wl, n_tok: int, layers: int, budget_s: float) -> dict:
     d = O.Desc(n_tok, H, D, "bf16", 2, 32, "f16")
     t0 = time.perf_counter()
     done = 0
-    ck, cv, Kh, Vh = O.encode_layer_none(d0, K[0], V[0])
-    Kd, Vd = O.decode_layer_none(d0, ck, cv)
+    ck, cv, Kh, Vh = O.encode_layer_none(d0, K[0], V[0], threads=threads)
+    Kd, Vd = O.decode_layer_none(d0, ck, cv, threads=threads)
     done += 2
     for l in range(1, layers):
-        ck, cv, Kh2, Vh2 = O.encode_layer_xlayer(d, W[l], K[l], V[l], Kh, Vh)
-        Kd, Vd = O.decode_layer_xlayer(d, W[l], ck, cv, Kd, Vd)
+        ck, cv, Kh2, Vh2 = O.encode_layer_xlayer(d, W[l], K[l], V[l], Kh, Vh, threads=threads)
+        Kd, Vd = O.decode_layer_xlayer(d, W[l], ck, cv, Kd, Vd, threads=threads)
         Kh, Vh = Kh2, Vh2
         done += 2
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": done * n_tok / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    return {"value": done * n_tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{n_tok} of {T_TOK} tokens (evenly spaced) through {done // 2} of {L_LAYERS} layers, "
-                      f"encode + decode, fp64 numpy; {dt:.1f} s"}
+                      f"encode + decode, plain fp64 C++ oracle on {threads} thread(s); {dt:.1f} s"}
+
+
+def cpu_baseline_line(wl, layers: int) -> dict:
+    """The oracle on one host core (the baseline) and, beside it, its thread
+    driver on every core of the box."""
+    one = oracle_xlayer_rate(wl, 256, layers, 12.0, threads=1)
+    n = O_threads()
+    box = oracle_xlayer_rate(wl, 256 * n, layers, 12.0, threads=n)
+    one["whole_box"] = {"value": box["value"], "unit": UNIT, "cores": n, "sample": box["sample"]}
+    one["cpu_model"] = cpu_model()
+    one["nproc"] = os.cpu_count()
+    return one
+
+
+def O_threads() -> int:
+    from oracle import kvc_oracle_c as O
+
+    return O.default_threads()
 
 
 def run_reference(args, rank: int):
@@ -233,12 +255,13 @@ def run_reference(args, rank: int):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     wl = synth.wan_xlayer(seed=synth.SEED_BASE + 1, device=dev, L=L_LAYERS, T=T_TOK if dev == "cuda" else 512,
                           H=H, D=D, rank=RANK)
+    n = O_threads()
     for _ in range(args.warmup):
-        oracle_xlayer_rate(wl, 64, 2, 5.0)
+        oracle_xlayer_rate(wl, 4 * n, 2, 5.0, threads=n)
     vals, secs = [], []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        r = oracle_xlayer_rate(wl, 256, L_LAYERS, 8.0)
+        r = oracle_xlayer_rate(wl, 16 * n, L_LAYERS, 8.0, threads=n)
         secs.append(time.perf_counter() - t0)
         vals.append(r["value"])
     value = statistics.median(vals)
@@ -250,7 +273,7 @@ def run_reference(args, rank: int):
                                    "anchor, rank 64; each step a bounded token sample", "global_batch": T_TOK,
                        "seq_len": T_TOK, "parallelism": "host cores"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
-                             "sample": r["sample"]},
+                             "sample": r["sample"], "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -551,8 +574,8 @@ def main():
             rows["c4_cluster"] = row_cluster(dev, hbm, tf_burst)
         rows = rows or None
         if not args.no_cpu:
-            # about 10 s of host work: 2048 of the tokens through every layer
-            cpu = oracle_xlayer_rate(xb.wl, 2048, L_RUN, 20.0)
+            # about 25 s of host work: the single-threaded oracle, then its thread driver
+            cpu = cpu_baseline_line(xb.wl, L_RUN)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -1,5 +1,8 @@
 """Parity of the CUDA codec (through the C ABI) with the fp64 oracle.
 
+The reference is the plain single-threaded C++ oracle (oracle/kvc_oracle.cpp,
+driven over disjoint tokens / heads / query rows by its thread driver); the
+numpy oracle is used only for the score margins of the clustered assignment.
 Each test feeds the GPU and the oracle the same seeded inputs; where a layer's
 prediction source is a reconstruction, both receive the oracle's (teacher
 forcing), so each call is checked on its own.  Tolerances: tests/kvc_testutil.
@@ -10,7 +13,8 @@ import pytest
 import torch
 
 from clustered_kv_cache_b200 import kvc, synth
-from oracle import kvc_oracle as O
+from oracle import kvc_oracle as ON
+from oracle import kvc_oracle_c as O
 
 import kvc_testutil as U
 
@@ -520,7 +524,7 @@ def test_cluster_codec_parity(T, H, n_c):
         oc, xh = O.encode_tensor_cluster(od, X64, c64, U.to64(enc), U.to64(dec))
         a_gpu = getattr(buf, which + "_assign")[:T].cpu().numpy().astype(np.int64)
         # the assignment is unique where the best and second-best scores are apart
-        sc = O.cluster_scores(X64.reshape(T, -1), c64)
+        sc = ON.cluster_scores(X64.reshape(T, -1), c64)
         srt = np.sort(sc, axis=1)
         margin = srt[:, 1] - srt[:, 0]
         clear = margin > 1e-4 * np.abs(srt[:, 0]) + 1e-3

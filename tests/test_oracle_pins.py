@@ -1,8 +1,11 @@
-"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+"""Pins of the fp64 oracles against what the pages and the mathematics fix.
 
-Each test checks the oracle against something other than itself: a library
+Each test checks an oracle against something other than itself: a library
 routine, a value printed on the pages (tests/golden), a hand-worked example, a
-closed form, an invariant, or brute force on tiny inputs.  None needs a GPU.
+closed form, an invariant, or brute force on tiny inputs.  Every test runs on
+both oracles: the plain single-threaded C++ one (oracle/kvc_oracle.cpp, the
+parity reference of the GPU tests) and the numpy one (oracle/kvc_oracle.py).
+None needs a GPU.
 """
 
 import json
@@ -12,10 +15,16 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import kvc_oracle as O
+from oracle import kvc_oracle as O_NUMPY
+from oracle import kvc_oracle_c as O_CPP
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 RNG = np.random.default_rng(20261202)
+
+
+@pytest.fixture(params=["cpp", "numpy"])
+def O(request):
+    return O_CPP if request.param == "cpp" else O_NUMPY
 
 
 def _golden(name):
@@ -26,7 +35,7 @@ def _golden(name):
 # ---------------------------------------------------------------- rounding
 
 
-def test_round_to_f16_f32_match_numpy_casts():
+def test_round_to_f16_f32_match_numpy_casts(O):
     x = RNG.standard_normal(200_000) * np.exp2(RNG.integers(-30, 20, 200_000))
     # exact ties of both formats
     ties = np.array([1 + 2.0**-11, 1 + 3 * 2.0**-11, 2049.0, 2051.0, 1 + 2.0**-24, 1 + 3 * 2.0**-24,
@@ -38,7 +47,7 @@ def test_round_to_f16_f32_match_numpy_casts():
     np.testing.assert_array_equal(O.round_to(x, "f32"), x.astype(np.float32).astype(np.float64))
 
 
-def test_round_to_bf16_matches_torch_on_float32_inputs():
+def test_round_to_bf16_matches_torch_on_float32_inputs(O):
     x32 = (RNG.standard_normal(200_000) * np.exp2(RNG.integers(-40, 40, 200_000))).astype(np.float32)
     ties = np.array([1 + 2.0**-8, 1 + 3 * 2.0**-8, 257.0, 259.0, -(1 + 2.0**-8)], np.float32)
     x32 = np.concatenate([x32, ties])
@@ -51,7 +60,7 @@ def test_round_to_bf16_matches_torch_on_float32_inputs():
 
 @pytest.mark.parametrize("bits,group,param", [(2, 32, "f16"), (4, 32, "f16"), (4, 64, "f16"),
                                               (4, 32, "f32"), (8, 16, "f16")])
-def test_quantizer_matches_brute_force_nearest_level(bits, group, param):
+def test_quantizer_matches_brute_force_nearest_level(O, bits, group, param):
     r = RNG.standard_normal((64, 4 * group)) * np.exp2(RNG.integers(-3, 4, (64, 1)))
     q, s, z = O.quantize_groups(r, bits, group, param)
     L = (1 << bits) - 1
@@ -72,7 +81,7 @@ def test_quantizer_matches_brute_force_nearest_level(bits, group, param):
     assert np.all(q <= L)
 
 
-def test_quantizer_degenerate_group_and_exact_grid():
+def test_quantizer_degenerate_group_and_exact_grid(O):
     r = np.full((3, 32), 0.3)
     q, s, z = O.quantize_groups(r, 2, 32, "f16")
     assert np.all(q == 0) and np.all(s == 0)
@@ -87,7 +96,7 @@ def test_quantizer_degenerate_group_and_exact_grid():
 # ---------------------------------------------------------------- packing
 
 
-def test_pack_hand_worked_examples():
+def test_pack_hand_worked_examples(O):
     for case in _golden("pack_worked_example.json")["cases"]:
         codes = np.array(case["codes"], np.uint8)
         got = O.pack_codes(codes, case["bits"])
@@ -96,7 +105,7 @@ def test_pack_hand_worked_examples():
 
 
 @pytest.mark.parametrize("bits", [2, 4, 8])
-def test_pack_matches_numpy_unpackbits(bits):
+def test_pack_matches_numpy_unpackbits(O, bits):
     codes = RNG.integers(0, 1 << bits, (17, 128)).astype(np.uint8)
     packed = O.pack_codes(codes, bits)
     assert packed.shape == (17, 128 * bits // 8)
@@ -108,18 +117,18 @@ def test_pack_matches_numpy_unpackbits(bits):
 # ---------------------------------------------------------------- storage accounting
 
 
-def test_group_quantizer_ratios_printed_on_pages():
+def test_group_quantizer_ratios_printed_on_pages(O):
     g = _golden("page_compression_ratios.json")
     for key in ("int2_group_quantizer", "int4_group_quantizer"):
         e = g[key]
-        ratio = 16.0 / O.bits_per_element(e["bits"], 32, "f16")
+        d = O.Desc(n_tokens=1000, n_heads=12, head_dim=128, bits=e["bits"], group=32)
+        elems = 2 * 1000 * 12 * 128
+        ratio = 16.0 * elems / (8 * O.codes_bytes(d))
         assert round(ratio, e["printed_decimals"]) == pytest.approx(e["ratio"]), key
-    d = O.Desc(n_tokens=1000, n_heads=12, head_dim=128, bits=2, group=32)
-    elems = 2 * 1000 * 12 * 128
-    assert O.codes_bytes(d) * 8 / elems == pytest.approx(O.bits_per_element(2, 32, "f16"))
+        assert ratio == pytest.approx(16.0 / O_NUMPY.bits_per_element(e["bits"], 32, "f16"))
 
 
-def test_tempokv_anchor_sweep_slope():
+def test_tempokv_anchor_sweep_slope(O):
     """One anchor latent frame among ~180 (717 video frames): each extra anchor
     bit costs 1/180 bit per element; the printed ratios give the same slope."""
     e = _golden("page_compression_ratios.json")["tempokv_anchor_sweep"]
@@ -151,7 +160,7 @@ def _dense_dplr(block, w, u, H, D, Din_head, Cin_order):
     return M
 
 
-def test_dplr_prediction_equals_dense_map():
+def test_dplr_prediction_equals_dense_map(O):
     H, D, r, T = 3, 8, 2, 11
     rng = np.random.default_rng(1)
     Ks, Vs = rng.standard_normal((T, H, D)), rng.standard_normal((T, H, D))
@@ -173,7 +182,7 @@ def test_dplr_prediction_equals_dense_map():
                                                                       lambda h, i: h * D + i), rtol=1e-12)
 
 
-def test_low_rank_latent_is_not_rounded():
+def test_low_rank_latent_is_not_rounded(O):
     """The latent passes to the second factor at full precision: with U = I
     the first r outputs of a zero-block map are x W^T exactly."""
     H, D, r, T = 2, 4, 3, 5
@@ -195,7 +204,7 @@ def _grid_values(rng, shape):
     return v
 
 
-def test_exact_predictor_gives_zero_residual():
+def test_exact_predictor_gives_zero_residual(O):
     H, D, r, T = 2, 64, 4, 40
     rng = np.random.default_rng(3)
     K0, V0 = _grid_values(rng, (T, H, D)), _grid_values(rng, (T, H, D))
@@ -225,7 +234,7 @@ def test_exact_predictor_gives_zero_residual():
     np.testing.assert_array_equal(V1h, V1)
 
 
-def _chain_workload(L=6, T=300, H=2, D=64, r=4, seed=5):
+def _chain_workload(O, L=6, T=300, H=2, D=64, r=4, seed=5):
     rng = np.random.default_rng(seed)
     C = H * D
     K = [rng.standard_normal((T, H, D))]
@@ -246,8 +255,8 @@ def _chain_workload(L=6, T=300, H=2, D=64, r=4, seed=5):
     return K, V, W
 
 
-def test_closed_loop_error_does_not_accumulate_and_decode_replays_encode():
-    K, V, W = _chain_workload()
+def test_closed_loop_error_does_not_accumulate_and_decode_replays_encode(O):
+    K, V, W = _chain_workload(O)
     T, H, D = K[0].shape
     d_anchor = O.Desc(T, H, D, bits=4, group=32)
     d = O.Desc(T, H, D, bits=2, group=32)
@@ -278,7 +287,7 @@ def test_closed_loop_error_does_not_accumulate_and_decode_replays_encode():
 # ---------------------------------------------------------------- temporal predictor
 
 
-def test_temporal_exact_predictor_and_ragged_frame():
+def test_temporal_exact_predictor_and_ragged_frame(O):
     H, D, F = 2, 64, 10
     T = 4 * F + 3  # ragged last frame
     rng = np.random.default_rng(7)
@@ -311,7 +320,56 @@ def test_temporal_exact_predictor_and_ragged_frame():
     np.testing.assert_array_equal(Vd, V)
 
 
-def test_temporal_continuation_equals_one_sequence():
+def test_temporal_lag_order_with_asymmetric_maps(O):
+    """The K map's first D inputs read frame f-1 and its last D read frame f-2
+    (reading R9).  Frames built exactly as K_f = K_{f-1} + 0.5 P K_{f-2} (P a
+    permutation) code to zero residuals; a coder with the two lags swapped
+    would predict 0.5 P K_{f-1} + K_{f-2} and leave non-zero residuals."""
+    H, D, F = 2, 64, 8
+    T = 3 * F + 3  # few enough frames for every value to stay exact in bf16
+    rng = np.random.default_rng(15)
+    ak = np.zeros((H, D, 2 * D))
+    av = np.zeros((H, D, 2 * D))
+    for h in range(H):
+        ak[h, :, :D] = np.eye(D)  # lag 1
+        ak[h, :, D:] = 0.5 * np.eye(D)[rng.permutation(D)]  # lag 2
+        av[h, :, :D] = np.eye(D)[rng.permutation(D)]
+        av[h, :, D:] = 0.5 * np.eye(D)
+    K = np.zeros((T, H, D))
+    V = np.zeros((T, H, D))
+    K[:F] = _grid_values(rng, (F, H, D))
+    V[:F] = _grid_values(rng, (F, H, D))
+    for f in range(1, 4):
+        a, b = f * F, min(T, (f + 1) * F)
+        n = b - a
+        k2 = K[a - 2 * F:a - 2 * F + n] if f >= 2 else np.zeros((n, H, D))
+        K[a:b] = K[a - F:a - F + n] + np.einsum("thi,hoi->tho", k2, ak[:, :, D:])
+        V[a:b] = np.einsum("thi,hoi->tho", K[a:b], av[:, :, :D]) + 0.5 * V[a - F:a - F + n]
+    assert np.array_equal(O_NUMPY.round_to(K, "bf16"), K) and np.array_equal(O_NUMPY.round_to(V, "bf16"), V)
+    d = O.Desc(T, H, D, bits=2, group=32, frame_tokens=F, anchor_bits=2)
+    ck, cv, Kh, Vh = O.encode_layer_temporal(d, dict(ak=ak, av=av), K, V)
+    np.testing.assert_array_equal(Kh, K)
+    np.testing.assert_array_equal(Vh, V)
+    assert np.all(ck.s[F:] == 0) and np.all(cv.s[F:] == 0)
+    swapped = np.concatenate([ak[:, :, D:], ak[:, :, :D]], axis=-1)
+    ck2, _, _, _ = O.encode_layer_temporal(d, dict(ak=swapped, av=av), K, V)
+    assert np.any(ck2.s[2 * F:] > 0)
+
+
+def test_cluster_storage_closed_form(O):
+    """Per token and tensor: code_dim b-bit codes, one (scale, zero) pair of
+    two fp16 values per group, and a one-byte centre index (256 centres fit in
+    8 bits); for the 128 INT4 g32 coefficients that is 64 + 16 + 1 = 81 bytes."""
+    for T, m, bits, group, param in ((32768, 128, 4, 32, "f16"), (1000, 128, 2, 32, "f16"),
+                                     (7, 64, 8, 16, "f32")):
+        d = O.Desc(T, 16, 128, bits=bits, group=group, param=param)
+        pair = 2 * (2 if param == "f16" else 4)
+        per_token = m * bits // 8 + (m // group) * pair + 1
+        assert O.codes_bytes(d, "cluster", m) == 2 * T * per_token
+    assert O.codes_bytes(O.Desc(1, 16, 128, bits=4, group=32), "cluster", 128) == 2 * 81
+
+
+def test_temporal_continuation_equals_one_sequence(O):
     """Coding frames [0, 3) and then [3, 5) from the reconstructed history
     (K of frames 1 and 2, V of frame 2) gives the codes of one 5-frame call."""
     H, D, F = 2, 64, 12
@@ -336,7 +394,7 @@ def test_temporal_continuation_equals_one_sequence():
     assert O.codes_bytes(d2, "temporal") == 2 * 2 * F * H * (D * 2 // 8 + 2 * 2 * 2)
 
 
-def test_temporal_frame_zero_is_plain_group_rtn_at_anchor_bits():
+def test_temporal_frame_zero_is_plain_group_rtn_at_anchor_bits(O):
     H, D, F, T = 2, 64, 8, 20
     rng = np.random.default_rng(8)
     K = O.round_to(rng.standard_normal((T, H, D)), "bf16")
@@ -356,7 +414,7 @@ def test_temporal_frame_zero_is_plain_group_rtn_at_anchor_bits():
 # ---------------------------------------------------------------- clustered predictor
 
 
-def test_cluster_assignment_is_nearest_centre_by_euclidean_distance():
+def test_cluster_assignment_is_nearest_centre_by_euclidean_distance(O):
     rng = np.random.default_rng(9)
     cent = rng.standard_normal((16, 64))
     X = cent[rng.integers(0, 16, 200)] + 0.3 * rng.standard_normal((200, 64))
@@ -368,7 +426,7 @@ def test_cluster_assignment_is_nearest_centre_by_euclidean_distance():
     assert O.cluster_assign(cent[:1], cent2)[0] == 0
 
 
-def test_cluster_codec_is_exact_when_residual_is_on_grid_in_decoder_span():
+def test_cluster_codec_is_exact_when_residual_is_on_grid_in_decoder_span(O):
     H, D, m, T, nc = 2, 32, 32, 24, 4
     C = H * D
     rng = np.random.default_rng(10)
@@ -390,7 +448,7 @@ def test_cluster_codec_is_exact_when_residual_is_on_grid_in_decoder_span():
 # ---------------------------------------------------------------- attention
 
 
-def test_attention_matches_torch_sdpa_in_float64():
+def test_attention_matches_torch_sdpa_in_float64(O):
     rng = np.random.default_rng(11)
     Q, K, V = rng.standard_normal((7, 3, 16)), rng.standard_normal((29, 3, 16)), rng.standard_normal((29, 3, 16))
     got = O.attention(Q, K, V, 0.37)
@@ -399,7 +457,7 @@ def test_attention_matches_torch_sdpa_in_float64():
     np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-13)
 
 
-def test_attention_special_cases():
+def test_attention_special_cases(O):
     rng = np.random.default_rng(12)
     Q = rng.standard_normal((4, 2, 8))
     K1 = np.repeat(rng.standard_normal((1, 2, 8)), 9, axis=0)
@@ -411,7 +469,7 @@ def test_attention_special_cases():
     np.testing.assert_allclose(O.attention(Q, K + shift, V, 0.5), O.attention(Q, K, V, 0.5), atol=1e-12)
 
 
-def test_mixed_attention_equals_attention_on_reconstructed_keys():
+def test_mixed_attention_equals_attention_on_reconstructed_keys(O):
     H, D, m, T, nc = 2, 32, 16, 50, 8
     C = H * D
     rng = np.random.default_rng(13)
