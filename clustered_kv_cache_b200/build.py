@@ -29,7 +29,8 @@ def _stale() -> bool:
         return True
     t = os.path.getmtime(LIB)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
-    deps.append(os.path.join(HERE, "..", "include", "kvc.h"))
+    inc = os.path.join(HERE, "..", "include")
+    deps.extend(os.path.join(inc, f) for f in os.listdir(inc))
     return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
 
 

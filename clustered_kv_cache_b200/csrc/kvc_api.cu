@@ -364,8 +364,8 @@ kvc_status kvc_decode_layer(const kvc_layer_desc* desc, const kvc_predictor* pre
 
 kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
                                  const kvc_codes* codes, const void* K_src, const void* V_src, const void* K_self,
-                                 const void* V_self, int64_t n_self, float scale, void* O, void* ws, size_t ws_bytes,
-                                 void* stream) {
+                                 const void* V_self, int64_t n_self, float scale, void* O, void* K_rec_opt,
+                                 void* V_rec_opt, void* ws, size_t ws_bytes, void* stream) {
   kvc_status s = check_desc(d, p);
   if (s != KVC_OK) return s;
   if (p->kind == KVC_PRED_TEMPORAL) return KVC_ERR_UNSUPPORTED;
@@ -376,7 +376,7 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
   if (n_self > 0 && (!K_self || !V_self)) return KVC_ERR_INVALID_ARGUMENT;
   if (p->kind == KVC_PRED_XLAYER_DPLR && (!K_src || !V_src)) return KVC_ERR_INVALID_ARGUMENT;
   if (d->n_tokens + n_self == 0 && n_q > 0) return KVC_ERR_INVALID_ARGUMENT;  // softmax over no keys
-  const void* ptrs[] = {Q, K_src, V_src, K_self, V_self, O, ws};
+  const void* ptrs[] = {Q, K_src, V_src, K_self, V_self, O, K_rec_opt, V_rec_opt, ws};
   for (const void* q : ptrs)
     if (q && !aligned16(q)) return KVC_ERR_MISALIGNED;
   if (!codes_aligned(p, codes)) return KVC_ERR_MISALIGNED;
@@ -385,8 +385,20 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
   if (n_q == 0) return KVC_OK;
   cudaStream_t st = (cudaStream_t)stream;
   if (tc_attend_supported(d, p, n_self)) {
-    cudaError_t e = tc_attend(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, ws, ws_bytes, st);
+    cudaError_t e = tc_attend(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, K_rec_opt,
+                              V_rec_opt, ws, ws_bytes, st);
     return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+  }
+  // the clustered history's reconstruction, when asked for, is its decode (the
+  // attention itself never rebuilds it)
+  if (p->kind == KVC_PRED_CLUSTER && (K_rec_opt || V_rec_opt) && d->n_tokens > 0) {
+    Carve none{nullptr, 0};
+    kvc_status s2 = dispatch(d, [&](auto* ts, auto* tp) -> cudaError_t {
+      using TS = std::remove_pointer_t<decltype(ts)>;
+      using TP = std::remove_pointer_t<decltype(tp)>;
+      return codec_cluster<TS, TP>(d, p, false, nullptr, nullptr, codes, K_rec_opt, V_rec_opt, none, st);
+    });
+    if (s2 != KVC_OK) return s2;
   }
   if (tc_mixed_supported(d, p)) {
     cudaError_t e = tc_mixed_attend(d, p, Q, n_q, codes, scale, O, ws, ws_bytes, st);
@@ -405,10 +417,13 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
                           (const Pair<TP>*)codes->v_params, (const uint8_t*)codes->v_assign, (TS*)O};
       return launch_mixed_attention(a, st);
     }
-    // decode the history into workspace, then attend over [history; self]
+    // decode the history (into the caller's outputs when given, else the
+    // workspace), then attend over [history; self]
     const size_t bytes = (size_t)d->n_tokens * H * D * sizeof(TS);
     TS* Kh = (TS*)cv.take(bytes);
     TS* Vh = (TS*)cv.take(bytes);
+    if (K_rec_opt) Kh = (TS*)K_rec_opt;
+    if (V_rec_opt) Vh = (TS*)V_rec_opt;
     cudaError_t e = codec_xlayer<TS, TP>(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh, cv, st);
     if (e != cudaSuccess) return e;
     AttnArgs<TS> a{n_q, d->n_tokens, n_self, H, scale, (const TS*)Q, Kh, Vh, (const TS*)K_self,

@@ -28,6 +28,9 @@
 #include <cuda.h>
 #include <string.h>
 
+#include <atomic>
+
+#include "../../include/kvc_testing.h"
 #include "tc.h"
 #include "tc_ptx.cuh"
 
@@ -56,6 +59,10 @@ cudaError_t tc_read_and_clear_error(unsigned int* value) {
 }
 
 namespace tc {
+
+// One-shot test hook of kvc_testing_inject_stall (read and cleared by the next
+// cross-layer codec launch).
+static std::atomic<int> g_inject_stall{0};
 
 constexpr int kThreads = 352;     // 11 warps: producer, MMA, two epilogue groups of 4, MMA sync
 constexpr int kSyncWarp = 10;
@@ -89,6 +96,9 @@ struct Args {
   int store_v;  // V^_l is written (always for decode)
   // latent mode: the layer's latents as bf16 hi / lo pairs, [T][r] each
   __nv_bfloat16 *zk_hi, *zk_lo, *zv_hi, *zv_lo;
+  // test hook (kvc_testing_inject_stall): 1 = CTA 0's producer leaves its first
+  // stage unarmed, so that the consumer's bounded wait runs out
+  int inject;
 };
 
 template <int RC>
@@ -191,11 +201,20 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       uint32_t issued_ph[S];  // ... in this phase of full[i]
       for (int i = 0; i < S; ++i) issued[i] = 0, issued_ph[i] = 0;
       bool ok = true;
+      bool stall = a.inject == 1 && blockIdx.x == 0;  // test hook: one stage is never armed
       auto load = [&](const CUtensorMap* ma, int ax, int ay, uint64_t pa, const CUtensorMap* mb, int bx, int by,
                       uint32_t bbytes) {
         if (!ok) return;
         if (!wait(&empty[s], ph ^ 1, abort_flag, a.err, 0x100u + s)) {
           ok = false;
+          return;
+        }
+        if (stall) {  // neither armed nor loaded: the MMA side's wait on full[s] runs out
+          stall = false;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1;
+          }
           return;
         }
         mbar_arrive_expect_tx(&full[s], (ma ? 16384u : 0u) + bbytes);
@@ -922,7 +941,7 @@ cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool
   if (!err) return cudaErrorInvalidDevice;
   tc::Args a{err, (int64_t)T, (int)H, d->bits, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
              (uint8_t*)c->k_codes, (__half2*)c->k_params, (uint8_t*)c->v_codes, (__half2*)c->v_params,
-             (enc && !Vr) ? 0 : 1, nullptr, nullptr, nullptr, nullptr};
+             (enc && !Vr) ? 0 : 1, nullptr, nullptr, nullptr, nullptr, tc::g_inject_stall.exchange(0)};
   const int rc = (int)(r / 64);
   return enc ? tc::dispatch<tc::kEncode>(d->group, rc, m, a, st) : tc::dispatch<tc::kDecode>(d->group, rc, m, a, st);
 }
@@ -947,9 +966,11 @@ cudaError_t latent_layer(const kvc_layer_desc* d, const kvc_predictor* p, const 
   if (!err) return cudaErrorInvalidDevice;
   Args a{err, (int64_t)T, (int)H, d->bits, nullptr, nullptr, (uint8_t*)c->k_codes, (__half2*)c->k_params,
          (uint8_t*)c->v_codes, (__half2*)c->v_params, 0, (__nv_bfloat16*)zk_hi, (__nv_bfloat16*)zk_lo,
-         (__nv_bfloat16*)zv_hi, (__nv_bfloat16*)zv_lo};
+         (__nv_bfloat16*)zv_hi, (__nv_bfloat16*)zv_lo, 0};
   return dispatch<kLatent>(d->group, (int)(r / 64), m, a, st);
 }
 }  // namespace tc
 
 }  // namespace kvc
+
+extern "C" void kvc_testing_inject_stall(int what) { kvc::tc::g_inject_stall.store(what == 1 ? 1 : 0); }

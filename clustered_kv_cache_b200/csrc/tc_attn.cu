@@ -15,6 +15,9 @@
 // work: each CTA decodes every CQ-th key tile and pushes it into the others'
 // shared memory, so a key tile is decoded once per cluster instead of once per
 // query tile.  S = Q K^T and O += P V^ run on tcgen05; P stays in tensor memory.
+// When the caller asks for the decoded history as well (K_rec_opt / V_rec_opt),
+// the first cluster of each head also stores every tile it decodes with TMA
+// stores of the same shared-memory tile it pushes to its peers.
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2-5 decode
 // epilogue (TMEM -> K^ / V^ tiles, pushed to the cluster), 6-9 softmax (S -> P,
@@ -60,6 +63,7 @@ struct Maps {
   CUtensorMap uk, uv;        // [C][r]
   CUtensorMap zkh, zkl, zvh, zvl;  // latents [T][r]
   CUtensorMap ck, cv, pk, pv;      // codes / params as bytes, for L2 prefetches
+  CUtensorMap kr, vr;              // optional decoded-history outputs [T][C]
 };
 
 struct Args {
@@ -72,6 +76,7 @@ struct Args {
   const uint8_t* vcodes;
   const __half2* vparams;
   __nv_bfloat16* O;  // [n_q][H][128]
+  int store_k, store_v;  // write the decoded history through maps.kr / maps.vr
 };
 
 // MN-major operand (N contiguous), 128-byte swizzle: sub-tiles of 64 N values
@@ -537,16 +542,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
       fence_async_smem();
       asm volatile("bar.sync 1, 128;" ::: "memory");
     };
+    // the first cluster of each head writes the decoded history when asked to
+    const bool first_cluster = blockIdx.x < (unsigned)CQ;
+    const bool st_k = first_cluster && a.store_k, st_v = first_cluster && a.store_v;
     // the tile is complete here: announce it to every peer, push it, and mark it locally
-    auto publish = [&](uint8_t* tile, uint64_t* bar) {
+    auto publish = [&](uint8_t* tile, uint64_t* bar, const CUtensorMap* out, int j) {
       if (!elected) return;
       // each peer armed its slot barrier for these bytes (see the MMA warp)
       for (int p = 1; p < CQ; ++p) {
         const uint32_t peer = (uint32_t)((rank + p) % CQ);
         push_to_peer(peer_addr(tile, peer), tile, 32768u, peer_addr(bar, peer));
       }
+      if (out) {  // rows past T are clipped by the map
+        tma_store(out, h * 128, j * 128, tile);
+        tma_store(out, h * 128 + 64, j * 128, tile + 16384);
+      }
       bulk_commit();
       mbar_arrive(bar);
+    };
+    // a slot that a TMA store still reads is not rewritten (the peers' pushes are
+    // known to be complete once the slot's free barrier has gathered them)
+    auto slot_stored = [&](bool stored) {
+      if (!stored) return;
+      if (elected) bulk_wait_read0();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
     };
     for (int j = rank; j < NH; j += CQ) {
       const int b = j & 1;
@@ -557,15 +576,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
       fetch(a.kcodes + rowi * RB, a.kparams + rowi * NG, valid, kin);
       wait(d_full, dfu++ & 1, abort_flag, a.err, 0x1400u);
       if (j >= 2) wait(kfree, kfu++ & 1, abort_flag, a.err, 0x1401u);
+      slot_stored(st_k && j >= 2);
       tc_fence_after();
       emit(kin, Kt(b));
-      publish(Kt(b), &kfull[b]);
+      publish(Kt(b), &kfull[b], st_k ? &maps.kr : nullptr, j);
       fetch(a.vcodes + rowi * RB, a.vparams + rowi * NG, valid, vin);
       wait(d_full, dfu++ & 1, abort_flag, a.err, 0x1402u);
       if (j >= 2) wait(vfree, vfu++ & 1, abort_flag, a.err, 0x1403u);
+      slot_stored(st_v && j >= 2);
       tc_fence_after();
       emit(vin, Vt(b));
-      publish(Vt(b), &vfull[b]);
+      publish(Vt(b), &vfull[b], st_v ? &maps.vr : nullptr, j);
     }
     if (elected) bulk_wait_all();
   } else if (has_q) {
@@ -734,7 +755,7 @@ size_t tc_attend_workspace(const kvc_layer_desc* d, const kvc_predictor* p) {
 
 cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q, const kvc_codes* c,
                       const void* Ks, const void* Vs, const void* K_self, const void* V_self, int64_t n_self,
-                      float scale, void* O, void* ws, size_t ws_bytes, cudaStream_t st) {
+                      float scale, void* O, void* K_rec, void* V_rec, void* ws, size_t ws_bytes, cudaStream_t st) {
   const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128, r = (uint64_t)p->rank;
   if (ws_bytes < tc_attend_workspace(d, p)) return cudaErrorInvalidValue;
   char* w = static_cast<char*>(ws);
@@ -765,12 +786,15 @@ cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const voi
          tc::map2d_bytes(&m.cv, c->v_codes, T, H * rb, (uint32_t)rb, 128) &&
          (d->group != 32 || (tc::map2d_bytes(&m.pk, c->k_params, T, H * 16, 16, 128) &&
                              tc::map2d_bytes(&m.pv, c->v_params, T, H * 16, 16, 128)));
+  const bool sk = K_rec && T > 0, sv = V_rec && T > 0;
+  if (ok && sk) ok = tc::map2d(&m.kr, K_rec, T, C, 128);
+  if (ok && sv) ok = tc::map2d(&m.vr, V_rec, T, C, 128);
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
   tc::attn::Args a{err, n_q, (int64_t)T, n_self, (int)H, d->bits, d->group, scale * 1.4426950408889634f,
                    (const uint8_t*)c->k_codes, (const __half2*)c->k_params, (const uint8_t*)c->v_codes,
-                   (const __half2*)c->v_params, (__nv_bfloat16*)O};
+                   (const __half2*)c->v_params, (__nv_bfloat16*)O, sk ? 1 : 0, sv ? 1 : 0};
   return tc::attn::dispatch(r == 0 ? 0 : r == 64 ? 1 : 2, d->group, d->bits, m, a, st);
 }
 

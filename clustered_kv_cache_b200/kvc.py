@@ -26,7 +26,7 @@ STATUS = {0: "KVC_OK", 1: "KVC_ERR_INVALID_ARGUMENT", 2: "KVC_ERR_UNSUPPORTED", 
 
 EXPORTED = ["kvc_codes_sizes", "kvc_codes_bytes", "kvc_workspace_bytes", "kvc_encode_layer", "kvc_decode_layer",
             "kvc_attend_compressed", "kvc_pack_codes", "kvc_unpack_codes", "kvc_get_device_error",
-            "kvc_status_string", "kvc_last_cuda_error", "kvc_launch_counter"]
+            "kvc_status_string", "kvc_last_cuda_error", "kvc_launch_counter", "kvc_testing_inject_stall"]
 
 
 class KvcError(RuntimeError):
@@ -79,7 +79,7 @@ def lib():
         "kvc_workspace_bytes": (SZ, [I, D, PR, I64]),
         "kvc_encode_layer": (I, [D, PR, V, V, V, V, CO, V, V, V, SZ, V]),
         "kvc_decode_layer": (I, [D, PR, CO, V, V, V, V, V, SZ, V]),
-        "kvc_attend_compressed": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, SZ, V]),
+        "kvc_attend_compressed": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, V, V, SZ, V]),
         "kvc_pack_codes": (I, [V, I64, I, V, V]),
         "kvc_unpack_codes": (I, [V, I64, I, V, V]),
         "kvc_get_device_error": (I, [V]),
@@ -210,14 +210,16 @@ def kvc_decode_layer(desc, pred, codes: CodeBuffers, K_src, V_src, K_rec, V_rec,
 
 
 def kvc_attend_compressed(desc, pred, Q, codes: CodeBuffers, K_src, V_src, K_self, V_self, scale: float, O,
-                          ws=None, stream=None):
+                          ws=None, stream=None, K_rec=None, V_rec=None):
+    """K_rec / V_rec: optional outputs of the decoded history (K_rec_opt / V_rec_opt)."""
     c = codes.struct()
     wp, wn = _ws(ws)
     n_q = 0 if Q is None else Q.shape[0]
     n_self = 0 if K_self is None else K_self.shape[0]
     _check(lib().kvc_attend_compressed(ctypes.byref(desc), ctypes.byref(pred), _ptr(Q), n_q, ctypes.byref(c),
                                        _ptr(K_src), _ptr(V_src), _ptr(K_self), _ptr(V_self), n_self,
-                                       ctypes.c_float(scale), _ptr(O), wp, wn, _stream(stream)),
+                                       ctypes.c_float(scale), _ptr(O), _ptr(K_rec), _ptr(V_rec), wp, wn,
+                                       _stream(stream)),
            "kvc_attend_compressed")
 
 
@@ -252,3 +254,13 @@ def kvc_encode_layer_cluster_static(desc, pred, K, V, codes: CodeBuffers, K_rec=
     c = codes.struct()
     _check(fn(ctypes.byref(desc), ctypes.byref(pred), _ptr(K), _ptr(V), ctypes.byref(c), _ptr(K_rec), _ptr(V_rec),
               _stream(stream)), "kvc_encode_layer_cluster_static")
+
+
+def kvc_testing_inject_stall(what: int = 1):
+    """Test hook (include/kvc_testing.h): the next tensor-core cross-layer codec
+    launch leaves one pipeline stage unarmed, so a bounded device wait runs out
+    and kvc_get_device_error() reports KVC_ERR_DEVICE_TIMEOUT."""
+    fn = lib().kvc_testing_inject_stall
+    fn.restype = None
+    fn.argtypes = [ctypes.c_int]
+    fn(int(what))

@@ -194,11 +194,18 @@ KVC_API kvc_status kvc_decode_layer(const kvc_layer_desc* desc, const kvc_predic
  * never written to device memory).  CLUSTER: scores and values are computed on
  * the stored coefficients, q.c_a + (W_dec^T q).coef, without rebuilding full
  * keys ("NanoKV ...", abstract: the Fast variant); n_self must be 0.
- * TEMPORAL: KVC_ERR_UNSUPPORTED.  O [n_q][H][D] is written. */
+ * TEMPORAL: KVC_ERR_UNSUPPORTED.  O [n_q][H][D] is written.
+ *  K_rec_opt, V_rec_opt: optional [T][H][D] outputs (NULL = not wanted) that
+ *    receive the decoded history, the same values kvc_decode_layer writes,
+ *    e.g. as the next layer's K_src / V_src.  For NONE / XLAYER on the
+ *    tensor-core path they are stored from the tiles the attention decodes
+ *    on chip anyway; CLUSTER runs its decode for them.  With n_q = 0 the call
+ *    does nothing at all (kvc_decode_layer decodes a history alone). */
 KVC_API kvc_status kvc_attend_compressed(const kvc_layer_desc* desc, const kvc_predictor* pred, const void* Q,
                                  int64_t n_q, const kvc_codes* codes, const void* K_src, const void* V_src,
                                  const void* K_self, const void* V_self, int64_t n_self, float scale,
-                                 void* O, void* ws, size_t ws_bytes, void* stream);
+                                 void* O, void* K_rec_opt, void* V_rec_opt, void* ws, size_t ws_bytes,
+                                 void* stream);
 
 /* Pack n codes (uint8, each < 2^bits) into n*bits/8 bytes, LSB first;
  * n*bits must be a multiple of 128 (whole 16-byte words). */

@@ -501,7 +501,7 @@ void kvo_cluster_decode(int64_t T, int C, int m, int group, int sfmt, const int6
 void kvo_attention(int64_t nq, int64_t nk, int H, int D, double scale, const double* Q, const double* K,
                    const double* V, double* O) {
   const int C = H * D;
-  std::vector<double> sc(nk > 0 ? nk : 1);
+  std::vector<double> sc(nk > 0 ? nk : 1), acc(D);
   for (int64_t i = 0; i < nq; ++i)
     for (int h = 0; h < H; ++h) {
       const double* q = Q + i * C + h * D;
@@ -517,12 +517,14 @@ void kvo_attention(int64_t nq, int64_t nk, int H, int D, double scale, const dou
         sc[t] = std::exp(sc[t] - m);
         l += sc[t];
       }
-      double* o = O + i * C + h * D;
-      for (int d = 0; d < D; ++d) {
-        double acc = 0.0;
-        for (int64_t t = 0; t < nk; ++t) acc += sc[t] * V[t * C + h * D + d];
-        o[d] = acc / l;
+      // o[d] = sum_t p_t v_t[d] in key order (keys outer, so V is read row by row)
+      for (int d = 0; d < D; ++d) acc[d] = 0.0;
+      for (int64_t t = 0; t < nk; ++t) {
+        const double* v = V + t * C + h * D;
+        for (int d = 0; d < D; ++d) acc[d] += sc[t] * v[d];
       }
+      double* o = O + i * C + h * D;
+      for (int d = 0; d < D; ++d) o[d] = acc[d] / l;
     }
 }
 
@@ -538,7 +540,7 @@ void kvo_mixed_attention(int64_t nq, int64_t T, int H, int D, int m, int nc, dou
                          const double* ck, const int64_t* ak, const double* cent_k, const double* dec_k,
                          const double* cv, const int64_t* av, const double* cent_v, const double* dec_v, double* O) {
   const int C = H * D;
-  std::vector<double> table(nc), qt(m), sc(T > 0 ? T : 1), mass(nc), cbar(m);
+  std::vector<double> table(nc), qt(m), sc(T > 0 ? T : 1), mass(nc), cbar(m), cacc(D);
   for (int64_t i = 0; i < nq; ++i)
     for (int h = 0; h < H; ++h) {
       const double* q = Q + i * C + h * D;
@@ -547,11 +549,10 @@ void kvo_mixed_attention(int64_t nq, int64_t T, int H, int D, int m, int nc, dou
         for (int d = 0; d < D; ++d) acc += q[d] * cent_k[(int64_t)j * C + h * D + d];
         table[j] = acc;
       }
-      for (int k = 0; k < m; ++k) {
-        double acc = 0.0;
-        for (int d = 0; d < D; ++d) acc += q[d] * dec_k[(int64_t)(h * D + d) * m + k];
-        qt[k] = acc;
-      }
+      // qt[k] = sum_d q[d] W_dec[h D + d][k] in channel order (channels outer)
+      for (int k = 0; k < m; ++k) qt[k] = 0.0;
+      for (int d = 0; d < D; ++d)
+        for (int k = 0; k < m; ++k) qt[k] += q[d] * dec_k[(int64_t)(h * D + d) * m + k];
       double mx = -INFINITY;
       for (int64_t t = 0; t < T; ++t) {
         double acc = 0.0;
@@ -571,13 +572,15 @@ void kvo_mixed_attention(int64_t nq, int64_t T, int H, int D, int m, int nc, dou
         mass[av[t]] += p;
         for (int k = 0; k < m; ++k) cbar[k] += p * cv[t * m + k];
       }
+      // sum_j m_j c^V_j[d] in centre order (centres outer), plus W^V_dec cbar
+      for (int d = 0; d < D; ++d) cacc[d] = 0.0;
+      for (int j = 0; j < nc; ++j)
+        for (int d = 0; d < D; ++d) cacc[d] += mass[j] * cent_v[(int64_t)j * C + h * D + d];
       double* o = O + i * C + h * D;
       for (int d = 0; d < D; ++d) {
-        double acc = 0.0;
-        for (int j = 0; j < nc; ++j) acc += mass[j] * cent_v[(int64_t)j * C + h * D + d];
         double acc2 = 0.0;
         for (int k = 0; k < m; ++k) acc2 += dec_v[(int64_t)(h * D + d) * m + k] * cbar[k];
-        o[d] = acc + acc2;
+        o[d] = cacc[d] + acc2;
       }
     }
 }

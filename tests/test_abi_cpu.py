@@ -1,5 +1,5 @@
 """Host-side checks of the C ABI: the library loads on a machine without a GPU,
-exports every entry point include/kvc.h declares, reports the closed-form
+exports every entry point include/*.h declares, reports the closed-form
 storage the oracle computes, and rejects bad arguments before any launch."""
 
 import ctypes
@@ -13,7 +13,8 @@ from clustered_kv_cache_b200 import build as kbuild
 from clustered_kv_cache_b200 import kvc
 from oracle import kvc_oracle as O
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "kvc.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+HEADERS = sorted(os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -23,9 +24,11 @@ def L():
 
 
 def test_exports_every_declared_entry_point(L):
-    with open(HEADER) as f:
-        declared = re.findall(r"KVC_API\s+[\w\s\*]+?\b(kvc_\w+)\s*\(", f.read())
-    assert len(declared) >= 11
+    declared = []
+    for h in HEADERS:
+        with open(h) as f:
+            declared += re.findall(r"KVC_API\s+[\w\s\*]+?\b(kvc_\w+)\s*\(", f.read())
+    assert len(declared) >= 13 and "kvc_testing_inject_stall" in declared
     assert sorted(declared) == sorted(set(declared))
     for name in declared:
         assert hasattr(L, name), name
@@ -82,12 +85,17 @@ def test_validation_errors_without_launch(L):
     # attention over a temporal history is not offered; clustered attention takes no self tokens
     tp = kvc.Predictor(kvc.PRED_TEMPORAL, 0, 0, 0, *([0x1000] * 12))
     st = L.kvc_attend_compressed(ctypes.byref(kvc.make_desc(100, 2, 128, frame_tokens=10)), ctypes.byref(tp), q, 4,
-                                 ctypes.byref(c), None, None, None, None, 0, 1.0, q, None, 0, None)
+                                 ctypes.byref(c), None, None, None, None, 0, 1.0, q, None, None, None, 0, None)
     assert st == 2
     cp = kvc.Predictor(kvc.PRED_CLUSTER, 0, 16, 128, *([0x1000] * 12))
     st = L.kvc_attend_compressed(ctypes.byref(good), ctypes.byref(cp), q, 4, ctypes.byref(c), None, None, q, q, 8,
-                                 1.0, q, None, 0, None)
+                                 1.0, q, None, None, None, 0, None)
     assert st == 2
+    # a misaligned optional history output is refused before anything runs
+    xp = kvc.Predictor(kvc.PRED_XLAYER_DPLR, 0, 0, 0, *([0x1000] * 12))
+    st = L.kvc_attend_compressed(ctypes.byref(good), ctypes.byref(xp), q, 4, ctypes.byref(c), q, q, None, None, 0,
+                                 1.0, q, ctypes.c_void_p(0x1008), None, None, 0, None)
+    assert st == 3
     assert L.kvc_pack_codes(q, 100, 2, q, None) == 1  # not whole 16-byte words
     assert L.kvc_pack_codes(q, 64, 3, q, None) == 2
 

@@ -430,35 +430,28 @@ def test_temporal_whole_chain_exact_predictor():
     np.testing.assert_array_equal(q.s, ck.s)
 
 
-def test_temporal_full_size_sampled_positions():
-    """One full layer of the large-backbone case (65536 tokens, 40 heads, 1560
-    tokens per frame, INT4 g64).  (a) The whole-layer call: the anchor frame at
-    sampled positions against the oracle; later frames follow their own closed
-    loop, so there the reconstruction error must match the oracle's in
-    distribution.  (b) A continued call of three frames from a supplied history,
-    against the oracle at sampled positions."""
+def _per_head(c: "O.Coded") -> "O.Coded":
+    """A coded [n, H, ...] tensor viewed as n*H single-head rows (each head's
+    temporal chain is independent of the others)."""
+    f = lambda a: a.reshape((a.shape[0] * a.shape[1], 1) + a.shape[2:])
+    return O.Coded(f(c.q), f(c.s), f(c.z))
+
+
+def test_temporal_continued_call_full_shape():
+    """A continued call of three 1560-token frames of the large-backbone case
+    (40 heads, INT4 g64) from a supplied history (the clean frames 18 and 19,
+    bf16 values shared by both sides), against the oracle at sampled
+    positions, frame by frame.  Each (position, head) chain whose earlier frames
+    differ anywhere is only checked for validity from there on.  (The
+    whole-layer call is checked in test_gpu_full_size.py.)"""
     tw = synth.temporal_layer(seed=synth.SEED_BASE + 3, device="cuda")
     T, H, D = tw.K.shape
     F = tw.frame_tokens
     hf = torch.float16
-    buf, Kr, Vr = _temporal_call(tw.ak, tw.av, tw.K, tw.V, F, 4, 64, hf, 4)
     n_last = T - (T // F) * F
     pos = np.sort(np.concatenate([np.arange(0, 4), np.arange(n_last - 2, n_last + 2), [F - 1],
                                   np.random.default_rng(5).choice(np.arange(n_last + 2, F - 1), 15, replace=False)]))
-    n_frames = (T + F - 1) // F
-    rows = np.array([f * F + s for f in range(n_frames) for s in pos if f * F + s < T])
-    sub = lambda t: U.to64(t[torch.from_numpy(rows).to(t.device)])
-    od = _odesc(len(rows), H, D, torch.bfloat16, 4, 64, hf, len(pos), 4)
     w64 = dict(ak=U.to64(tw.ak), av=U.to64(tw.av))
-    ck, cv, Kh, Vh = O.encode_layer_temporal(od, w64, sub(tw.K), sub(tw.V))
-    np0 = len(pos)
-    qk = U.codes_from_gpu(buf.k_codes[: F * H * D // 2], (F, H, D), 4)[pos]
-    U.assert_codes_close(qk, ck.q[:np0], "anchor K codes")
-    for x, rec, ref in ((tw.K, Kr, Kh), (tw.V, Vr, Vh)):
-        e_gpu = np.sqrt(np.mean((sub(rec) - sub(x)) ** 2))
-        e_ref = np.sqrt(np.mean((ref - sub(x)) ** 2))
-        assert abs(e_gpu / e_ref - 1) < 0.02, (e_gpu, e_ref)
-    # (b) frames 20..22 continued from the clean frames 18, 19 (bf16 values shared by both sides)
     f0, nf = 20, 3
     a, b = f0 * F, (f0 + nf) * F
     k_hist = tw.K[(f0 - 2) * F:f0 * F].reshape(2, F, H, D)
@@ -473,22 +466,21 @@ def test_temporal_full_size_sampled_positions():
     fk, fv, fKh, fVh = O.encode_layer_temporal(ofs, w64, sb(tw.K[a:b]), sb(tw.V[a:b]), kh64, vh64)
     fek, fev = U.exact_temporal(ofs, w64, fk, fv, fKh, fVh, kh64, vh64)
     erk, erv = U.err_temporal(ofs, w64, fKh, fVh, kh64, vh64)
-    # inside the call each frame is predicted from the call's own earlier frames: a
-    # position whose earlier frames differ anywhere is only checked for validity
     npos = len(pos)
-    diverged = np.zeros(npos, bool)
+    diverged = np.zeros(npos * H, bool)  # per (position, head)
     gq = {w: U.codes_from_gpu(getattr(fb, w + "_codes"), (nf * F, H, D), 4)[rows_b] for w in "kv"}
     gp = {w: U.params_from_gpu(getattr(fb, w + "_params"), (nf * F, H, D // 64), "f16") for w in "kv"}
+    flat = lambda x: x.reshape(x.shape[0] * x.shape[1], 1, x.shape[2])
     for f in range(nf):
         sl = slice(f * npos, (f + 1) * npos)
-        cut = lambda c: O.Coded(c.q[sl], c.s[sl], c.z[sl])
+        cut = lambda c: _per_head(O.Coded(c.q[sl], c.s[sl], c.z[sl]))
         kf = diverged.copy()
         for which, oc, rec, ref, ex, x, er in (("k", fk, fK, fKh, fek, tw.K[a:b], erk),
                                               ("v", fv, fV, fVh, fev, tw.V[a:b], erv)):
             s_, z_ = gp[which]
-            g = O.Coded(gq[which][sl], s_[rows_b][sl], z_[rows_b][sl])
-            kf = kf | _compare(g, cut(oc), sb(rec)[sl], ref[sl], ex[sl], sb(x)[sl], "bf16", 64,
-                               f"{which} continued frame {f}", "f16", er[sl], kf)
+            g = _per_head(O.Coded(gq[which][sl], s_[rows_b][sl], z_[rows_b][sl]))
+            kf = kf | _compare(g, cut(oc), flat(sb(rec)[sl]), flat(ref[sl]), flat(ex[sl]), flat(sb(x)[sl]), "bf16",
+                               64, f"{which} continued frame {f}", "f16", flat(er[sl]), kf)
         diverged |= kf
 
 
@@ -499,6 +491,42 @@ def _cluster_pred(cw: synth.ClusterWorkload, n_c):
     w = dict(k_centroids=cw.k_centroids.cuda(), k_enc=cw.k_enc.cuda(), k_dec=cw.k_dec.cuda(),
              v_centroids=cw.v_centroids.cuda(), v_enc=cw.v_enc.cuda(), v_dec=cw.v_dec.cuda())
     return kvc.make_predictor(kvc.PRED_CLUSTER, w, n_clusters=n_c, code_dim=cw.k_enc.shape[0])
+
+
+def _check_cluster(cw, buf, Kr, Vr, T, H, D, dtype, param, n_c):
+    """Assignments, coefficient codes, (scale, zero) pairs and reconstructions
+    of both tensors against the C++ oracle."""
+    od = _odesc(T, H, D, dtype, 4, 32, param)
+    p = U.np_param(param)
+    for which, X, cent, enc, dec, rec in (("k", cw.K, cw.k_centroids, cw.k_enc, cw.k_dec, Kr),
+                                          ("v", cw.V, cw.v_centroids, cw.v_enc, cw.v_dec, Vr)):
+        X64, c64 = U.to64(X), U.to64(cent)
+        oc, xh = O.encode_tensor_cluster(od, X64, c64, U.to64(enc), U.to64(dec))
+        a_gpu = getattr(buf, which + "_assign")[:T].cpu().numpy().astype(np.int64)
+        # the assignment is unique where the best and second-best scores are apart
+        sc = ON.cluster_scores(X64.reshape(T, -1), c64)
+        srt = np.sort(sc, axis=1)
+        margin = srt[:, 1] - srt[:, 0]
+        clear = margin > 1e-4 * np.abs(srt[:, 0]) + 1e-3
+        np.testing.assert_array_equal(a_gpu[clear], oc.assign[clear])
+        assert np.all(sc[np.arange(T), a_gpu] <= srt[:, 0] + 1e-4 * np.abs(srt[:, 0]) + 1e-3)
+        assert clear.mean() > 0.99
+        q = U.codes_from_gpu(getattr(buf, which + "_codes"), (T, 128), 4)
+        s, z = U.params_from_gpu(getattr(buf, which + "_params"), (T, 4), p)
+        U.assert_codes_close(q, oc.q, which + " coefficient codes")
+        ecoef = U.err_cluster(X64.reshape(T, -1), c64, oc.assign, U.to64(enc))
+        pdiff = U.assert_params_close(s[clear], z[clear], oc.s[clear], oc.z[clear], p, which + " params",
+                                      levels=15, err=ecoef[clear], group=32)
+        exact = (c64[oc.assign] + ON.dequantize_groups(oc.q, oc.s, oc.z, 32) @ U.to64(dec).T).reshape(T, H, D)
+        # a token whose centre, any code or any (scale, zero) differs has every channel moved
+        tok_flip = (q != oc.q).any(axis=1) | ~clear
+        tok_flip[np.flatnonzero(clear)[pdiff.any(axis=1)]] = True
+        flip = np.repeat(tok_flip, H * D).reshape(T, H, D)
+        coef_hat = ON.dequantize_groups(oc.q, oc.s, oc.z, 32)
+        erec = (128 * U.U32 * (np.abs(coef_hat) @ np.abs(U.to64(dec)).T) + U.U32 * np.abs(c64[oc.assign]))
+        if rec is not None:
+            U.assert_recon_close(U.to64(rec), xh, exact, X64, flip, od.state, which + " recon",
+                                 err=erec.reshape(T, H, D))
 
 
 @pytest.mark.parametrize("T,H,n_c", [(1000, 4, 32), (300, 16, 256), (2000 - 5, 16, 256)])
@@ -517,34 +545,42 @@ def test_cluster_codec_parity(T, H, n_c):
     kvc.kvc_decode_layer(desc, pred, buf, None, None, Kd, Vd, kvc.alloc_workspace(kvc.OP_DECODE, desc, pred))
     _sync_ok()
     assert torch.equal(Kd, Kr) and torch.equal(Vd, Vr)
-    od = _odesc(T, H, D, bf, 4, 32, hf)
-    for which, X, cent, enc, dec, rec in (("k", cw.K, cw.k_centroids, cw.k_enc, cw.k_dec, Kr),
-                                          ("v", cw.V, cw.v_centroids, cw.v_enc, cw.v_dec, Vr)):
-        X64, c64 = U.to64(X), U.to64(cent)
-        oc, xh = O.encode_tensor_cluster(od, X64, c64, U.to64(enc), U.to64(dec))
-        a_gpu = getattr(buf, which + "_assign")[:T].cpu().numpy().astype(np.int64)
-        # the assignment is unique where the best and second-best scores are apart
-        sc = ON.cluster_scores(X64.reshape(T, -1), c64)
-        srt = np.sort(sc, axis=1)
-        margin = srt[:, 1] - srt[:, 0]
-        clear = margin > 1e-4 * np.abs(srt[:, 0]) + 1e-3
-        np.testing.assert_array_equal(a_gpu[clear], oc.assign[clear])
-        assert np.all(sc[np.arange(T), a_gpu] <= srt[:, 0] + 1e-4 * np.abs(srt[:, 0]) + 1e-3)
-        assert clear.mean() > 0.99
-        q = U.codes_from_gpu(getattr(buf, which + "_codes"), (T, 128), 4)
-        s, z = U.params_from_gpu(getattr(buf, which + "_params"), (T, 4), "f16")
-        U.assert_codes_close(q, oc.q, which + " coefficient codes")
-        ecoef = U.err_cluster(X64.reshape(T, -1), c64, oc.assign, U.to64(enc))
-        pdiff = U.assert_params_close(s[clear], z[clear], oc.s[clear], oc.z[clear], "f16", which + " params",
-                                      levels=15, err=ecoef[clear], group=32)
-        exact = (c64[oc.assign] + O.dequantize_groups(oc.q, oc.s, oc.z, 32) @ U.to64(dec).T).reshape(T, H, D)
-        # a token whose centre, any code or any (scale, zero) differs has every channel moved
-        tok_flip = (q != oc.q).any(axis=1) | ~clear
-        tok_flip[np.flatnonzero(clear)[pdiff.any(axis=1)]] = True
-        flip = np.repeat(tok_flip, H * D).reshape(T, H, D)
-        coef_hat = O.dequantize_groups(oc.q, oc.s, oc.z, 32)
-        erec = (128 * U.U32 * (np.abs(coef_hat) @ np.abs(U.to64(dec)).T) + U.U32 * np.abs(c64[oc.assign]))
-        U.assert_recon_close(U.to64(rec), xh, exact, X64, flip, "bf16", which + " recon", err=erec.reshape(T, H, D))
+    _check_cluster(cw, buf, Kr, Vr, T, H, D, bf, hf, n_c)
+
+
+@pytest.mark.parametrize("dtype,T,H,n_c", [(torch.float32, 300, 2, 16), (torch.bfloat16, 257, 3, 40)])
+def test_cluster_codec_cuda_core_path(dtype, T, H, n_c):
+    """fp32 data, or a joint row of 384 channels (not a multiple of 256): the
+    CUDA-core kernels, against the oracle."""
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 109, T=T, H=H, n_c=n_c, iters=3, dtype=dtype)
+    D = 128
+    param = torch.float32 if dtype == torch.float32 else torch.float16
+    desc = _desc(T, H, D, dtype, 4, 32, param)
+    pred = _cluster_pred(cw, n_c)
+    buf = kvc.alloc_codes(desc, pred)
+    K, V = cw.K.cuda(), cw.V.cuda()
+    Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_encode_layer(desc, pred, K, V, None, None, buf, Kr, Vr, kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred))
+    Kd, Vd = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_decode_layer(desc, pred, buf, None, None, Kd, Vd, kvc.alloc_workspace(kvc.OP_DECODE, desc, pred))
+    _sync_ok()
+    assert torch.equal(Kd, Kr) and torch.equal(Vd, Vr)
+    _check_cluster(cw, buf, Kr, Vr, T, H, D, dtype, param, n_c)
+
+
+def test_cluster_static_entry_against_the_oracle():
+    """The clustered encode that allocates nothing, against the oracle."""
+    T, H, D, n_c = 700, 4, 128, 64
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 110, T=T, H=H, n_c=n_c, iters=3)
+    bf, hf = torch.bfloat16, torch.float16
+    desc = _desc(T, H, D, bf, 4, 32, hf)
+    pred = _cluster_pred(cw, n_c)
+    buf = kvc.alloc_codes(desc, pred)
+    K, V = cw.K.cuda(), cw.V.cuda()
+    Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_encode_layer_cluster_static(desc, pred, K, V, buf, Kr, Vr)
+    _sync_ok()
+    _check_cluster(cw, buf, Kr, Vr, T, H, D, bf, hf, n_c)
 
 
 # ---------------------------------------------------------------- attention
@@ -668,3 +704,66 @@ def test_mixed_dimensional_attention(n_q, T, H, n_c):
     ref = O.mixed_attention(U.to64(Q), ck, U.to64(cw.k_centroids), U.to64(cw.k_dec), cv, U.to64(cw.v_centroids),
                             U.to64(cw.v_dec), od, D ** -0.5)
     assert U.rel_l2(U.to64(Og), ref) <= U.ATT_TOL[torch.bfloat16]
+
+
+# ---------------------------------------------------------------- decoded history out of the attention
+
+
+def _history_outputs_case(desc, pred, buf, Q, Ks, Vs, Kself, Vself, scale, T, H, D, dtype):
+    """kvc_attend_compressed with K_rec_opt / V_rec_opt: the outputs equal
+    kvc_decode_layer's bit for bit, and O equals the call without them."""
+    n_q = Q.shape[0]
+    ws = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q)
+    O1 = torch.empty(n_q, H, D, dtype=dtype, device="cuda")
+    O2 = torch.empty_like(O1)
+    kvc.kvc_attend_compressed(desc, pred, Q, buf, Ks, Vs, Kself, Vself, scale, O1, ws)
+    Kh = torch.full((T, H, D), float("nan"), dtype=dtype, device="cuda")
+    Vh = torch.full_like(Kh, float("nan"))
+    kvc.kvc_attend_compressed(desc, pred, Q, buf, Ks, Vs, Kself, Vself, scale, O2, ws, K_rec=Kh, V_rec=Vh)
+    Kd, Vd = torch.empty_like(Kh), torch.empty_like(Vh)
+    kvc.kvc_decode_layer(desc, pred, buf, Ks, Vs, Kd, Vd, kvc.alloc_workspace(kvc.OP_DECODE, desc, pred))
+    _sync_ok()
+    assert torch.equal(Kh, Kd) and torch.equal(Vh, Vd), "decoded history differs from kvc_decode_layer"
+    assert torch.equal(O1, O2), "asking for the history changed the attention output"
+    # only one of the two
+    Kh1 = torch.full_like(Kh, float("nan"))
+    kvc.kvc_attend_compressed(desc, pred, Q, buf, Ks, Vs, Kself, Vself, scale, O2, ws, K_rec=Kh1)
+    _sync_ok()
+    assert torch.equal(Kh1, Kd)
+
+
+@pytest.mark.parametrize("n_q,n_self,T,rank", [(700, 130, 16 * 128 - 7, 64), (129, 0, 300, 0), (1100, 0, 9 * 128, 128)])
+def test_attention_history_outputs_cross_layer(n_q, n_self, T, rank):
+    """Tensor-core path: 700 queries are two clusters of query tiles per head;
+    the first cluster stores the tiles it decodes (ragged T clips the last)."""
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 107, L=2, T=T, rank=rank, calib_tokens=1024)
+    H, D = 12, 128
+    bf, hf = torch.bfloat16, torch.float16
+    desc = _desc(T, H, D, bf, 2, 32, hf)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=rank)
+    buf, _, _ = _xlayer_gpu(desc, pred, wl.K[1].cuda(), wl.V[1].cuda(), wl.K[0].cuda(), wl.V[0].cuda())
+    Q = synth.queries(31, n_q, H, D).cuda()
+    Ks = synth.queries(32, n_self, H, D).cuda() if n_self else None
+    Vs = synth.queries(33, n_self, H, D).cuda() if n_self else None
+    _history_outputs_case(desc, pred, buf, Q, wl.K[0].cuda(), wl.V[0].cuda(), Ks, Vs, D ** -0.5, T, H, D, bf)
+
+
+def test_attention_history_outputs_fp32_and_clustered():
+    """CUDA-core path (fp32 tiny layer) and the clustered history."""
+    wl = synth.tiny_xlayer()
+    T, H, D = wl.K[0].shape
+    f32 = torch.float32
+    desc = _desc(T, H, D, f32, 4, 32, f32)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=wl.rank)
+    buf, _, _ = _xlayer_gpu(desc, pred, wl.K[1].cuda(), wl.V[1].cuda(), wl.K[0].cuda(), wl.V[0].cuda())
+    Q = synth.queries(7, 64, H, D, dtype=f32).cuda()
+    _history_outputs_case(desc, pred, buf, Q, wl.K[0].cuda(), wl.V[0].cuda(), None, None, 0.125, T, H, D, f32)
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 108, T=500, H=16, n_c=64, iters=3)
+    bf, hf = torch.bfloat16, torch.float16
+    cdesc = _desc(500, 16, 128, bf, 4, 32, hf)
+    cpred = _cluster_pred(cw, 64)
+    cbuf = kvc.alloc_codes(cdesc, cpred)
+    kvc.kvc_encode_layer(cdesc, cpred, cw.K.cuda(), cw.V.cuda(), None, None, cbuf, None, None,
+                         kvc.alloc_workspace(kvc.OP_ENCODE, cdesc, cpred))
+    Qc = synth.queries(8, 90, 16, 128).cuda()
+    _history_outputs_case(cdesc, cpred, cbuf, Qc, None, None, None, None, 128 ** -0.5, 500, 16, 128, bf)

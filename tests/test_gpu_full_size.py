@@ -1,0 +1,211 @@
+"""Parity at the benchmark's own sizes and launch configurations.
+
+Each test runs the CUDA path on the full workload the benchmark times and
+checks it against the plain C++ oracle where the oracle can compute the
+result one unit at a time: sampled query rows of the attentions (rows are
+independent), sampled tokens of the clustered codec (tokens are independent
+given the centres), and sampled spatial positions of the temporal codec
+(positions are independent), frame by frame.  Tolerances: tests/kvc_testutil.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from clustered_kv_cache_b200 import kvc, synth
+from oracle import kvc_oracle as ON
+from oracle import kvc_oracle_c as O
+
+import kvc_testutil as U
+from test_gpu_codec import _cluster_pred, _compare, _desc, _oracle_codes_to_gpu, _temporal_call, _temporal_gpu_coded
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from clustered_kv_cache_b200 import build
+
+    build.build()
+    kvc.lib()
+
+
+def _rows(n, k, seed):
+    """k sorted sample rows of range(n), always including the first and last tiles' edges."""
+    rng = np.random.default_rng(seed)
+    edge = np.array([0, 1, 127, 128, n - 129, n - 128, n - 2, n - 1])
+    mid = rng.choice(np.arange(n), k - len(edge), replace=False)
+    return np.unique(np.concatenate([edge, mid]))
+
+
+def test_compressed_attention_at_the_benchmark_size():
+    """4680 queries (3 latent frames) over the 32760-token INT2 history of a
+    Wan-shaped layer (rank 64) plus the 4680 chunk tokens: 37 query tiles per
+    head, ten clusters of four per head, as the benchmark launches it.  The
+    history codes are the oracle's; 256 sampled query rows are compared."""
+    l = 15
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 1, device="cuda", L=16, rank=64, layers_needed=[l])
+    T, H, D = wl.K[l].shape
+    n_q = 3 * 1560
+    bf, hf = torch.bfloat16, torch.float16
+    od = O.Desc(T, H, D, "bf16", 2, 32, "f16")
+    w64 = {k: U.to64(v) for k, v in wl.weights[l].items()}
+    Ks, Vs = U.to64(wl.K[l - 1]), U.to64(wl.V[l - 1])  # shared layer-14 sources (teacher forcing)
+    ck, cv, Kh, Vh = O.encode_layer_xlayer(od, w64, U.to64(wl.K[l]), U.to64(wl.V[l]), Ks, Vs)
+    buf = _oracle_codes_to_gpu(ck, cv, 2, "f16")
+    Q = synth.queries(synth.SEED_BASE + 2, n_q, H, D, device="cuda")
+    Kself = synth.queries(synth.SEED_BASE + 12, n_q, H, D, device="cuda")
+    Vself = synth.queries(synth.SEED_BASE + 22, n_q, H, D, device="cuda")
+    desc = _desc(T, H, D, bf, 2, 32, hf)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl.weights[l], rank=64)
+    Og = torch.empty(n_q, H, D, dtype=bf, device="cuda")
+    ws = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q)
+    Kr = torch.empty(T, H, D, dtype=bf, device="cuda")
+    kvc.kvc_attend_compressed(desc, pred, Q, buf, wl.K[l - 1], wl.V[l - 1], Kself, Vself, D ** -0.5, Og, ws,
+                              K_rec=Kr)
+    torch.cuda.synchronize()
+    assert kvc.kvc_get_device_error() == 0
+    rows = _rows(n_q, 256, 41)
+    ref = O.attention(U.to64(Q)[rows], np.concatenate([Kh, U.to64(Kself)]), np.concatenate([Vh, U.to64(Vself)]),
+                      D ** -0.5)
+    err = U.rel_l2(U.to64(Og)[rows], ref)
+    U.OBSERVED.append({"check": "C2 attention, 256 sampled rows", "rel_l2": err})
+    assert err <= U.ATT_TOL[bf], err
+    # the decoded history the attention stored matches the oracle's reconstruction
+    rec = U.to64(Kr)
+    flip = np.abs(rec - Kh) > 1e-3 * (np.abs(U.to64(wl.K[l])) + 1.0)
+    assert flip.mean() < 1e-3, flip.mean()
+
+
+def test_clustered_codec_at_the_benchmark_size():
+    """32768 tokens x 16 heads x 128, 256 centres, INT4 g32 coefficients: the
+    whole-layer encode and decode against the oracle on 512 sampled tokens."""
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 4, device="cuda")
+    T, H, D = cw.K.shape
+    bf, hf = torch.bfloat16, torch.float16
+    desc = _desc(T, H, D, bf, 4, 32, hf)
+    pred = _cluster_pred(cw, 256)
+    buf = kvc.alloc_codes(desc, pred)
+    Kr, Vr = torch.empty_like(cw.K), torch.empty_like(cw.V)
+    kvc.kvc_encode_layer(desc, pred, cw.K, cw.V, None, None, buf, Kr, Vr, kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred))
+    Kd, Vd = torch.empty_like(Kr), torch.empty_like(Vr)
+    kvc.kvc_decode_layer(desc, pred, buf, None, None, Kd, Vd, kvc.alloc_workspace(kvc.OP_DECODE, desc, pred))
+    torch.cuda.synchronize()
+    assert kvc.kvc_get_device_error() == 0
+    assert torch.equal(Kd, Kr) and torch.equal(Vd, Vr)
+    rows = _rows(T, 512, 43)
+    ri = torch.from_numpy(rows).cuda()
+    od = O.Desc(len(rows), H, D, "bf16", 4, 32, "f16")
+    for which, X, cent, enc, dec, rec in (("k", cw.K, cw.k_centroids, cw.k_enc, cw.k_dec, Kr),
+                                          ("v", cw.V, cw.v_centroids, cw.v_enc, cw.v_dec, Vr)):
+        X64, c64 = U.to64(X[ri]), U.to64(cent)
+        oc, xh = O.encode_tensor_cluster(od, X64, c64, U.to64(enc), U.to64(dec))
+        n = len(rows)
+        a_gpu = getattr(buf, which + "_assign")[ri].cpu().numpy().astype(np.int64)
+        sc = ON.cluster_scores(X64.reshape(n, -1), c64)
+        srt = np.sort(sc, axis=1)
+        clear = (srt[:, 1] - srt[:, 0]) > 1e-4 * np.abs(srt[:, 0]) + 1e-3
+        np.testing.assert_array_equal(a_gpu[clear], oc.assign[clear])
+        q = U.codes_from_gpu(getattr(buf, which + "_codes"), (T, 128), 4)[rows]
+        s, z = U.params_from_gpu(getattr(buf, which + "_params"), (T, 4), "f16")
+        s, z = s[rows], z[rows]
+        U.assert_codes_close(q, oc.q, which + " coefficient codes (full layer, sampled tokens)")
+        ecoef = U.err_cluster(X64.reshape(n, -1), c64, oc.assign, U.to64(enc))
+        pdiff = U.assert_params_close(s[clear], z[clear], oc.s[clear], oc.z[clear], "f16", which + " params (full layer)",
+                                      levels=15, err=ecoef[clear], group=32)
+        exact = (c64[oc.assign] + ON.dequantize_groups(oc.q, oc.s, oc.z, 32) @ U.to64(dec).T).reshape(n, H, D)
+        tok_flip = (q != oc.q).any(axis=1) | ~clear
+        tok_flip[np.flatnonzero(clear)[pdiff.any(axis=1)]] = True
+        flip = np.repeat(tok_flip, H * D).reshape(n, H, D)
+        coef_hat = ON.dequantize_groups(oc.q, oc.s, oc.z, 32)
+        erec = 128 * U.U32 * (np.abs(coef_hat) @ np.abs(U.to64(dec)).T) + U.U32 * np.abs(c64[oc.assign])
+        U.assert_recon_close(U.to64(rec[ri]), xh, exact, X64, flip, "bf16", which + " recon (full layer)",
+                             err=erec.reshape(n, H, D))
+
+
+def test_mixed_attention_at_the_benchmark_size():
+    """1560 queries over the 32768-token clustered history (16 heads), with the
+    key splits the benchmark's launch uses; history codes from the oracle; 256
+    sampled query rows compared."""
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 4, device="cuda")
+    T, H, D = cw.K.shape
+    od = O.Desc(T, H, D, "bf16", 4, 32, "f16")
+    ck, _ = O.encode_tensor_cluster(od, U.to64(cw.K), U.to64(cw.k_centroids), U.to64(cw.k_enc), U.to64(cw.k_dec),
+                                    reconstruct=False)
+    cv, _ = O.encode_tensor_cluster(od, U.to64(cw.V), U.to64(cw.v_centroids), U.to64(cw.v_enc), U.to64(cw.v_dec),
+                                    reconstruct=False)
+    buf = _oracle_codes_to_gpu(ck, cv, 4, "f16", assign=True)
+    n_q = 1560
+    Q = synth.queries(synth.SEED_BASE + 5, n_q, H, D, device="cuda")
+    desc = _desc(T, H, D, torch.bfloat16, 4, 32, torch.float16)
+    pred = _cluster_pred(cw, 256)
+    Og = torch.empty(n_q, H, D, dtype=torch.bfloat16, device="cuda")
+    kvc.kvc_attend_compressed(desc, pred, Q, buf, None, None, None, None, D ** -0.5, Og,
+                              kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q))
+    torch.cuda.synchronize()
+    assert kvc.kvc_get_device_error() == 0
+    rows = _rows(n_q, 256, 47)
+    ref = O.mixed_attention(U.to64(Q)[rows], ck, U.to64(cw.k_centroids), U.to64(cw.k_dec), cv,
+                            U.to64(cw.v_centroids), U.to64(cw.v_dec), od, D ** -0.5)
+    err = U.rel_l2(U.to64(Og)[rows], ref)
+    U.OBSERVED.append({"check": "C4 mixed attention, 256 sampled rows", "rel_l2": err})
+    assert err <= U.ATT_TOL[torch.bfloat16], err
+
+
+def _per_head(c: "O.Coded") -> "O.Coded":
+    """A coded [n, H, ...] tensor viewed as n*H single-head rows."""
+    f = lambda a: a.reshape((a.shape[0] * a.shape[1], 1) + a.shape[2:])
+    return O.Coded(f(c.q), f(c.s), f(c.z))
+
+
+def test_temporal_whole_layer_element_by_element():
+    """The whole 65536-token, 40-head layer in one call (the benchmark's
+    launch), against the oracle's frame chain at sampled positions, frame by
+    frame and element by element.  Each (position, head) has its own chain; one
+    whose earlier frames differ anywhere (a flipped code, pair or
+    reconstruction) follows its own closed loop from there on and is only
+    checked for validity."""
+    tw = synth.temporal_layer(seed=synth.SEED_BASE + 3, device="cuda")
+    T, H, D = tw.K.shape
+    F = tw.frame_tokens
+    hf = torch.float16
+    buf, Kr, Vr = _temporal_call(tw.ak, tw.av, tw.K, tw.V, F, 4, 64, hf, 4)
+    n_last = T - (T // F) * F
+    pos = np.unique(np.concatenate([np.arange(0, 3), np.arange(n_last - 2, n_last + 2), [127, 128, F - 1],
+                                    np.random.default_rng(5).choice(np.arange(n_last + 2, F - 1), 14, replace=False)]))
+    n_frames = (T + F - 1) // F
+    rows = np.array([f * F + s for f in range(n_frames) for s in pos if f * F + s < T])
+    ri = torch.from_numpy(rows).cuda()
+    sub = lambda t: U.to64(t[ri])
+    od = O.Desc(len(rows), H, D, "bf16", 4, 64, "f16", len(pos), 4)
+    w64 = dict(ak=U.to64(tw.ak), av=U.to64(tw.av))
+    ck, cv, Kh, Vh = O.encode_layer_temporal(od, w64, sub(tw.K), sub(tw.V))
+    ek, ev = U.exact_temporal(od, w64, ck, cv, Kh, Vh)
+    erk, erv = U.err_temporal(od, w64, Kh, Vh)
+    gk = _temporal_gpu_coded(buf, T, H, D, F, 4, 4, 64, "f16", "k")
+    gv = _temporal_gpu_coded(buf, T, H, D, F, 4, 4, 64, "f16", "v")
+    gk, gv = O.Coded(gk.q[rows], gk.s[rows], gk.z[rows]), O.Coded(gv.q[rows], gv.s[rows], gv.z[rows])
+    recK, recV, xK, xV = sub(Kr), sub(Vr), sub(tw.K), sub(tw.V)
+    flat = lambda a: a.reshape(a.shape[0] * a.shape[1], 1, a.shape[2])
+    npos = len(pos)
+    diverged = np.zeros(npos * H, bool)  # per (position, head)
+    on_chain = 0
+    start = 0
+    for f in range(n_frames):
+        n = int(np.sum(f * F + pos < T))  # the partial last frame holds the first positions
+        sl = slice(start, start + n)
+        start += n
+        cut = lambda c: _per_head(O.Coded(c.q[sl], c.s[sl], c.z[sl]))
+        kf = diverged[:n * H].copy()
+        for which, gc, oc, rec, ref, ex, x, er in (("k", gk, ck, recK, Kh, ek, xK, erk),
+                                                   ("v", gv, cv, recV, Vh, ev, xV, erv)):
+            kf = kf | _compare(cut(gc), cut(oc), flat(rec[sl]), flat(ref[sl]), flat(ex[sl]), flat(x[sl]), "bf16",
+                               64, f"{which} frame {f} (whole-layer call)", "f16", flat(er[sl]), kf)
+        diverged[:n * H] |= kf
+        on_chain += int((~diverged[:n * H]).sum())
+    units = len(rows) * H
+    U.OBSERVED.append({"check": "C3 whole layer", "position_head_frames_on_chain": on_chain, "of": units})
+    # most (position, head) chains stay on the oracle's chain for most frames
+    assert on_chain >= 0.3 * units, (on_chain, units)

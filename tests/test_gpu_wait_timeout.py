@@ -1,0 +1,59 @@
+"""Failure detection without a GPU fault: a bounded device wait that runs out.
+
+The test hook kvc_testing_inject_stall makes the next cross-layer codec launch
+leave one TMA pipeline stage unarmed, so the MMA side's wait on it can never
+succeed.  The wait gives up after its bounded time (about two seconds), the
+kernel records KVC_ERR_DEVICE_TIMEOUT in the device error word, every role
+returns and the loads already issued are drained.  The host reads the status,
+and the context stays usable: the next launch codes the layer correctly.
+"""
+
+import time
+
+import pytest
+import torch
+
+from clustered_kv_cache_b200 import kvc, synth
+
+pytestmark = pytest.mark.gpu
+
+KVC_ERR_DEVICE_TIMEOUT = 6
+
+
+def test_bounded_wait_runs_out_and_reports_a_timeout():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from clustered_kv_cache_b200 import build
+
+    build.build()
+    T, H, D, r = 3 * 128 + 11, 12, 128, 64
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 111, L=2, T=T, rank=r, calib_tokens=1024)
+    bf, hf = torch.bfloat16, torch.float16
+    desc = kvc.make_desc(T, H, D, bf, 2, 32, hf)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=r)
+    K, V, Ks, Vs = (t.cuda() for t in (wl.K[1], wl.V[1], wl.K[0], wl.V[0]))
+    ws = kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred)
+
+    def encode():
+        buf = kvc.alloc_codes(desc, pred)
+        Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+        kvc.kvc_encode_layer(desc, pred, K, V, Ks, Vs, buf, Kr, Vr, ws)
+        return buf, Kr, Vr
+
+    # a clean launch first: the reference result, and no error pending
+    ref, Kr0, Vr0 = encode()
+    assert kvc.kvc_get_device_error() == 0
+    # the faulted launch: the launch itself succeeds, the bounded wait runs out on the device
+    kvc.kvc_testing_inject_stall(1)
+    t0 = time.perf_counter()
+    encode()
+    status = kvc.kvc_get_device_error()  # synchronizes the stream
+    elapsed = time.perf_counter() - t0
+    assert status == KVC_ERR_DEVICE_TIMEOUT, status
+    assert elapsed < 60.0, elapsed
+    # read-and-clear: nothing pending now, and the hook was one-shot
+    assert kvc.kvc_get_device_error() == 0
+    buf, Kr, Vr = encode()
+    assert kvc.kvc_get_device_error() == 0
+    assert torch.equal(Kr, Kr0) and torch.equal(Vr, Vr0)
+    assert torch.equal(buf.k_codes, ref.k_codes) and torch.equal(buf.v_codes, ref.v_codes)
