@@ -432,6 +432,32 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
   });
 }
 
+kvc_status kvc_attend_compressed_debiased(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q,
+                                          int64_t n_q, const kvc_codes* codes, const void* K_src, const void* V_src,
+                                          const void* K_self, const void* V_self, int64_t n_self, float scale,
+                                          void* O, void* K_rec_opt, void* V_rec_opt, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  kvc_status s = check_desc(d, p);
+  if (s != KVC_OK) return s;
+  // the corrected softmax is written for the tensor-core cross-layer attention
+  if (!tc_attend_supported(d, p, n_self) || d->n_tokens == 0) return KVC_ERR_UNSUPPORTED;
+  if ((s = check_weights(p)) != KVC_OK) return s;
+  if (n_q < 0 || n_self < 0) return KVC_ERR_INVALID_ARGUMENT;
+  if (!codes_ok(p, codes) || (n_q > 0 && (!Q || !O))) return KVC_ERR_INVALID_ARGUMENT;
+  if (n_self > 0 && (!K_self || !V_self)) return KVC_ERR_INVALID_ARGUMENT;
+  if (!K_src || !V_src) return KVC_ERR_INVALID_ARGUMENT;
+  const void* ptrs[] = {Q, K_src, V_src, K_self, V_self, O, K_rec_opt, V_rec_opt, ws};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return KVC_ERR_MISALIGNED;
+  if (!codes_aligned(p, codes)) return KVC_ERR_MISALIGNED;
+  const size_t need = kvc_workspace_bytes(KVC_OP_ATTEND, d, p, n_q);
+  if (ws_bytes < need || (need && !ws)) return KVC_ERR_WORKSPACE_TOO_SMALL;
+  if (n_q == 0) return KVC_OK;
+  cudaError_t e = tc_attend(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, K_rec_opt, V_rec_opt,
+                            ws, ws_bytes, (cudaStream_t)stream, true);
+  return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+}
+
 kvc_status kvc_pack_codes(const uint8_t* codes, int64_t n, int bits, void* packed, void* stream) {
   if (bits != 2 && bits != 4 && bits != 8) return KVC_ERR_UNSUPPORTED;
   if (n < 0 || (n * bits) % 128) return KVC_ERR_INVALID_ARGUMENT;

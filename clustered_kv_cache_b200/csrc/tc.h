@@ -18,7 +18,7 @@ size_t tc_attend_workspace(const kvc_layer_desc* d, const kvc_predictor* p);
 cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
                       const kvc_codes* c, const void* Ks, const void* Vs, const void* K_self, const void* V_self,
                       int64_t n_self, float scale, void* O, void* K_rec, void* V_rec, void* ws, size_t ws_bytes,
-                      cudaStream_t st);
+                      cudaStream_t st, bool jensen = false);
 bool tc_mixed_supported(const kvc_layer_desc* d, const kvc_predictor* p);
 size_t tc_mixed_workspace(const kvc_layer_desc* d, int64_t n_q);
 cudaError_t tc_mixed_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,

@@ -77,6 +77,7 @@ struct Args {
   const __half2* vparams;
   __nv_bfloat16* O;  // [n_q][H][128]
   int store_k, store_v;  // write the decoded history through maps.kr / maps.vr
+  float jensen_log2;     // JC: 0.5 scale^2 log2(e) / 12 (Jensen term per |q_g|^2 s_g^2, in log2 units)
 };
 
 // MN-major operand (N contiguous), 128-byte swizzle: sub-tiles of 64 N values
@@ -208,7 +209,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16
 // decoder announces the bytes on each peer's kfull / vfull and pushes the tile
 // with a bulk copy that completes there.
 
-template <int RC, int G, int BITS>
+template <int RC, int G, int BITS, bool JC>
 __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __grid_constant__ Maps maps, const Args a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -337,9 +338,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
           load(&maps.zkh, c * 64, t0, &maps.uk, c * 64, h * 128);
           load(&maps.zkl, c * 64, t0, &maps.uk, c * 64, h * 128);
         }
-        // V: [K^_{l,h} (resident) | V^_{l-1,h}] BV_h^T + [Z_V hi | lo] UV_h^T
-        for (int c = 0; c < 2; ++c) load(nullptr, 0, 0, &maps.bv, c * 64, h * 128);
+        // V: [K^_{l,h} (resident) | V^_{l-1,h}] BV_h^T + [Z_V hi | lo] UV_h^T, the V^_{l-1,h}
+        // half first as in the codec kernel, so that the sums round the same way
         for (int c = 0; c < 2; ++c) load(&maps.vs, h * 128 + c * 64, t0, &maps.bv, 128 + c * 64, h * 128);
+        for (int c = 0; c < 2; ++c) load(nullptr, 0, 0, &maps.bv, c * 64, h * 128);
         for (int c = 0; c < RC; ++c) {
           load(&maps.zvh, c * 64, t0, &maps.uv, c * 64, h * 128);
           load(&maps.zvl, c * 64, t0, &maps.uv, c * 64, h * 128);
@@ -411,8 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
         umma_commit(d_full);
       };
       auto dec_v = [&](int b) {
-        for (int c = 0; c < 2; ++c) chunk(DC, c == 0, Kt(b) + c * 16384);
-        for (int c = 0; c < 2 + 2 * RC; ++c) chunk(DC, false, nullptr);
+        for (int c = 0; c < 2; ++c) chunk(DC, c == 0, nullptr);  // V^_{l-1,h} half
+        for (int c = 0; c < 2; ++c) chunk(DC, false, Kt(b) + c * 16384);
+        for (int c = 0; c < 2 * RC; ++c) chunk(DC, false, nullptr);
         umma_commit(d_full);
       };
       // slot of tile t released (S(t) / PV(t) issued): to the decoder of tile t+2, or locally
@@ -596,13 +599,45 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
     const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16);
     const float c = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
+    // Jensen correction: |q_g|^2 of this thread's query row, from the Q tile
+    constexpr int NGQ = 128 / G;
+    float qn[JC ? NGQ : 1];
+    if (JC) {
+      wait(q_full, 0, abort_flag, a.err, 0x1504u);
+#pragma unroll
+      for (int g = 0; g < NGQ; ++g) qn[g] = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {  // 16-byte chunk k of the row: elements 8k .. 8k + 7
+        const uint4 u = *reinterpret_cast<const uint4*>(Qs + (k / 8) * 16384 + sw128_off(row, k % 8));
+        float x[8];
+        unpack_bf16x8(u, x, 0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qn[(8 * k) / G] = fmaf(x[i], x[i], qn[(8 * k) / G]);
+      }
+    }
     for (int j = 0; j < NT; ++j) {
       const int b = j & 1;
       const uint32_t sc = lane_addr + (SC(b) - tmem);
+      const bool hist = j < NH;
+      // JC: lane l holds the Jensen weights w_g = s_g^2 jensen_log2 of keys l, l + 32,
+      // l + 64, l + 96 of a history tile (loaded before the S wait hides their latency)
+      float w[JC ? 4 : 1][JC ? NGQ : 1];
+      if (JC && hist) {
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+          const int64_t t = (int64_t)j * 128 + pc * 32 + lane;
+          const __half2* pr = a.kparams + (t * a.H + h) * NGQ;
+#pragma unroll
+          for (int g = 0; g < NGQ; ++g) {
+            const float sg = t < a.T ? __low2float(pr[g]) : 0.f;
+            w[pc][g] = sg * sg * a.jensen_log2;
+          }
+        }
+      }
       wait(&s_full[b], (j >> 1) & 1, abort_flag, a.err, 0x1500u + b);
       tc_fence_after();
-      const int64_t kbase = j < NH ? (int64_t)j * 128 : (int64_t)(j - NH) * 128;
-      const int64_t klim = j < NH ? a.T : a.n_self;
+      const int64_t kbase = hist ? (int64_t)j * 128 : (int64_t)(j - NH) * 128;
+      const int64_t klim = hist ? a.T : a.n_self;
       const int nvalid = klim - kbase < 128 ? (int)(klim - kbase) : 128;
       // the whole S row in registers: four loads, one wait
       float sv[4][32];
@@ -611,6 +646,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
       tmem_ld32_async(sc + 64, sv[2]);
       tmem_ld32_async(sc + 96, sv[3]);
       tmem_ld_wait(sv[0], sv[1], sv[2], sv[3]);
+      if (JC) {
+        // scores in log2 units, history keys lowered by their Jensen term
+        // sum_g |q_g|^2 w_g (key pc * 32 + i's weights come from lane i)
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float corr = 0.f;
+            if (hist) {
+#pragma unroll
+              for (int g = 0; g < NGQ; ++g) corr = fmaf(qn[g], __shfl_sync(0xffffffffu, w[pc][g], i), corr);
+            }
+            sv[pc][i] = fmaf(sv[pc][i], c, -corr);
+          }
+      }
       if (nvalid < 128) {
 #pragma unroll
         for (int pc = 0; pc < 4; ++pc)
@@ -623,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
       for (int pc = 0; pc < 4; ++pc)
 #pragma unroll
         for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], sv[pc][i]);
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * (JC ? 1.f : c);
       // lazy rescale: only when the tile's max exceeds the one in use by 2^8
       const bool need = mt > m_used + 8.f;
       float alpha = 1.f;
@@ -639,8 +689,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(sv[pc][2 * i], c, -m_used));
-          const float p1 = ex2_approx(fmaf(sv[pc][2 * i + 1], c, -m_used));
+          const float p0 = ex2_approx(JC ? sv[pc][2 * i] - m_used : fmaf(sv[pc][2 * i], c, -m_used));
+          const float p1 = ex2_approx(JC ? sv[pc][2 * i + 1] - m_used : fmaf(sv[pc][2 * i + 1], c, -m_used));
           ls[i & 3] += p0 + p1;
           w[i] = pack_bf16x2(p0, p1);
         }
@@ -695,9 +745,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
   }
 }
 
-template <int RC, int G, int BITS>
+template <int RC, int G, int BITS, bool JC>
 static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
-  auto k = attend_cluster_kernel<RC, G, BITS>;
+  auto k = attend_cluster_kernel<RC, G, BITS, JC>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   const unsigned nqt = (unsigned)((a.n_q + 127) / 128);
@@ -719,15 +769,16 @@ static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int RC>
+template <int RC, bool JC>
 static cudaError_t dispatch_gb(int group, int bits, const Maps& m, const Args& a, cudaStream_t st) {
-  if (group == 32) return bits == 2 ? launch<RC, 32, 2>(m, a, st) : launch<RC, 32, 4>(m, a, st);
-  return bits == 2 ? launch<RC, 64, 2>(m, a, st) : launch<RC, 64, 4>(m, a, st);
+  if (group == 32) return bits == 2 ? launch<RC, 32, 2, JC>(m, a, st) : launch<RC, 32, 4, JC>(m, a, st);
+  return bits == 2 ? launch<RC, 64, 2, JC>(m, a, st) : launch<RC, 64, 4, JC>(m, a, st);
 }
+template <bool JC>
 static cudaError_t dispatch(int rc, int group, int bits, const Maps& m, const Args& a, cudaStream_t st) {
-  if (rc == 0) return dispatch_gb<0>(group, bits, m, a, st);
-  if (rc == 1) return dispatch_gb<1>(group, bits, m, a, st);
-  return dispatch_gb<2>(group, bits, m, a, st);
+  if (rc == 0) return dispatch_gb<0, JC>(group, bits, m, a, st);
+  if (rc == 1) return dispatch_gb<1, JC>(group, bits, m, a, st);
+  return dispatch_gb<2, JC>(group, bits, m, a, st);
 }
 
 }  // namespace attn
@@ -755,7 +806,8 @@ size_t tc_attend_workspace(const kvc_layer_desc* d, const kvc_predictor* p) {
 
 cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q, const kvc_codes* c,
                       const void* Ks, const void* Vs, const void* K_self, const void* V_self, int64_t n_self,
-                      float scale, void* O, void* K_rec, void* V_rec, void* ws, size_t ws_bytes, cudaStream_t st) {
+                      float scale, void* O, void* K_rec, void* V_rec, void* ws, size_t ws_bytes, cudaStream_t st,
+                      bool jensen) {
   const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128, r = (uint64_t)p->rank;
   if (ws_bytes < tc_attend_workspace(d, p)) return cudaErrorInvalidValue;
   char* w = static_cast<char*>(ws);
@@ -794,8 +846,11 @@ cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const voi
   if (!err) return cudaErrorInvalidDevice;
   tc::attn::Args a{err, n_q, (int64_t)T, n_self, (int)H, d->bits, d->group, scale * 1.4426950408889634f,
                    (const uint8_t*)c->k_codes, (const __half2*)c->k_params, (const uint8_t*)c->v_codes,
-                   (const __half2*)c->v_params, (__nv_bfloat16*)O, sk ? 1 : 0, sv ? 1 : 0};
-  return tc::attn::dispatch(r == 0 ? 0 : r == 64 ? 1 : 2, d->group, d->bits, m, a, st);
+                   (const __half2*)c->v_params, (__nv_bfloat16*)O, sk ? 1 : 0, sv ? 1 : 0,
+                   0.5f * scale * scale * 1.4426950408889634f / 12.f};
+  const int rc = r == 0 ? 0 : r == 64 ? 1 : 2;
+  return jensen ? tc::attn::dispatch<true>(rc, d->group, d->bits, m, a, st)
+                : tc::attn::dispatch<false>(rc, d->group, d->bits, m, a, st);
 }
 
 }  // namespace kvc

@@ -26,7 +26,8 @@ STATUS = {0: "KVC_OK", 1: "KVC_ERR_INVALID_ARGUMENT", 2: "KVC_ERR_UNSUPPORTED", 
 
 EXPORTED = ["kvc_codes_sizes", "kvc_codes_bytes", "kvc_workspace_bytes", "kvc_encode_layer", "kvc_decode_layer",
             "kvc_attend_compressed", "kvc_pack_codes", "kvc_unpack_codes", "kvc_get_device_error",
-            "kvc_status_string", "kvc_last_cuda_error", "kvc_launch_counter", "kvc_testing_inject_stall"]
+            "kvc_status_string", "kvc_last_cuda_error", "kvc_launch_counter", "kvc_testing_inject_stall",
+            "kvc_attend_compressed_debiased"]
 
 
 class KvcError(RuntimeError):
@@ -80,6 +81,7 @@ def lib():
         "kvc_encode_layer": (I, [D, PR, V, V, V, V, CO, V, V, V, SZ, V]),
         "kvc_decode_layer": (I, [D, PR, CO, V, V, V, V, V, SZ, V]),
         "kvc_attend_compressed": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, V, V, SZ, V]),
+        "kvc_attend_compressed_debiased": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, V, V, SZ, V]),
         "kvc_pack_codes": (I, [V, I64, I, V, V]),
         "kvc_unpack_codes": (I, [V, I64, I, V, V]),
         "kvc_get_device_error": (I, [V]),
@@ -221,6 +223,20 @@ def kvc_attend_compressed(desc, pred, Q, codes: CodeBuffers, K_src, V_src, K_sel
                                        ctypes.c_float(scale), _ptr(O), _ptr(K_rec), _ptr(V_rec), wp, wn,
                                        _stream(stream)),
            "kvc_attend_compressed")
+
+
+def kvc_attend_compressed_debiased(desc, pred, Q, codes: CodeBuffers, K_src, V_src, K_self, V_self, scale: float,
+                                   O, ws=None, stream=None, K_rec=None, V_rec=None):
+    """kvc_attend_compressed with the Jensen-bias correction of the history keys."""
+    c = codes.struct()
+    wp, wn = _ws(ws)
+    n_q = 0 if Q is None else Q.shape[0]
+    n_self = 0 if K_self is None else K_self.shape[0]
+    _check(lib().kvc_attend_compressed_debiased(ctypes.byref(desc), ctypes.byref(pred), _ptr(Q), n_q,
+                                                ctypes.byref(c), _ptr(K_src), _ptr(V_src), _ptr(K_self),
+                                                _ptr(V_self), n_self, ctypes.c_float(scale), _ptr(O), _ptr(K_rec),
+                                                _ptr(V_rec), wp, wn, _stream(stream)),
+           "kvc_attend_compressed_debiased")
 
 
 def kvc_pack_codes(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None):

@@ -207,6 +207,27 @@ KVC_API kvc_status kvc_attend_compressed(const kvc_layer_desc* desc, const kvc_p
                                  void* O, void* K_rec_opt, void* V_rec_opt, void* ws, size_t ws_bytes,
                                  void* stream);
 
+/* kvc_attend_compressed with the Jensen-bias correction of the quantized
+ * history (the abstract on the "Jensen bias" of INT2 key caches, among the
+ * related papers listed on the "CORAL-KV ..." page): quantization noise on a
+ * cached key inflates E[exp(score)], so history keys steal attention mass from
+ * the uncompressed chunk.  Each history key t's score (never a K_self key's) is
+ * lowered, for each query and head, by
+ *     0.5 * scale^2 * sum_g |q_g|^2 * s_{t,g}^2 / 12,
+ * g over the key row's quantization groups, q_g the query's channels of group
+ * g and s_{t,g} the stored residual scale: the second-order exponent of a
+ * uniform rounding error of step s, which the correction removes in
+ * expectation.  It reads only the stored scales (no extra memory).  Same
+ * arguments and outputs as kvc_attend_compressed; implemented for the
+ * tensor-core cross-layer path (KVC_PRED_XLAYER_DPLR, bf16, head_dim 128,
+ * fp16 params, T > 0); other layers return KVC_ERR_UNSUPPORTED. */
+KVC_API kvc_status kvc_attend_compressed_debiased(const kvc_layer_desc* desc, const kvc_predictor* pred,
+                                                  const void* Q, int64_t n_q, const kvc_codes* codes,
+                                                  const void* K_src, const void* V_src, const void* K_self,
+                                                  const void* V_self, int64_t n_self, float scale, void* O,
+                                                  void* K_rec_opt, void* V_rec_opt, void* ws, size_t ws_bytes,
+                                                  void* stream);
+
 /* Pack n codes (uint8, each < 2^bits) into n*bits/8 bytes, LSB first;
  * n*bits must be a multiple of 128 (whole 16-byte words). */
 KVC_API kvc_status kvc_pack_codes(const uint8_t* codes, int64_t n, int bits, void* packed, void* stream);

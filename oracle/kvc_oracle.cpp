@@ -498,9 +498,38 @@ void kvo_cluster_decode(int64_t T, int C, int m, int group, int sfmt, const int6
 // head, s_t = scale q.k_t, m = max_t s_t, p_t = exp(s_t - m),
 // o = sum_t p_t v_t / sum_t p_t.  Q [nq][H][D]; K, V [nk][H][D].
 
+// Jensen-bias correction (the abstract on the "Jensen bias" of INT2 key caches,
+// among the related papers listed on the CORAL-KV page): quantization noise e on a cached key raises
+// E[exp(scale q.(k + e))] above exp(scale q.k); to second order (the
+// log-moment of a uniform rounding error of step s is x^2 s^2 / 24 + O(x^4))
+// the excess is exp(0.5 scale^2 sum_g |q_g|^2 s_g^2 / 12), g over the key's
+// quantization groups.  Subtracting that exponent from the score of every
+// quantized key removes the bias in expectation; uncompressed keys are left
+// alone.  q: one head's query row (D values); sk: the key's group scales.
+static double jensen_term(const double* q, const double* sk, int D, int group, double scale) {
+  double acc = 0.0;
+  for (int g = 0; g < D / group; ++g) {
+    double qn = 0.0;
+    for (int i = 0; i < group; ++i) qn += q[g * group + i] * q[g * group + i];
+    acc += qn * sk[g] * sk[g] / 12.0;
+  }
+  return 0.5 * scale * scale * acc;
+}
+
+void kvo_attention_corrected(int64_t nq, int64_t nk, int H, int D, double scale, const double* Q, const double* K,
+                             const double* V, int64_t n_hist, const double* s_hist, int group, double* O);
+
 void kvo_attention(int64_t nq, int64_t nk, int H, int D, double scale, const double* Q, const double* K,
                    const double* V, double* O) {
-  const int C = H * D;
+  kvo_attention_corrected(nq, nk, H, D, scale, Q, K, V, 0, nullptr, 1, O);
+}
+
+// As kvo_attention; the first n_hist keys are quantized history whose group
+// scales s_hist [n_hist][H][D / group] give each one's Jensen correction
+// (s_hist NULL: no correction).
+void kvo_attention_corrected(int64_t nq, int64_t nk, int H, int D, double scale, const double* Q, const double* K,
+                             const double* V, int64_t n_hist, const double* s_hist, int group, double* O) {
+  const int C = H * D, ng = D / group;
   std::vector<double> sc(nk > 0 ? nk : 1), acc(D);
   for (int64_t i = 0; i < nq; ++i)
     for (int h = 0; h < H; ++h) {
@@ -510,6 +539,7 @@ void kvo_attention(int64_t nq, int64_t nk, int H, int D, double scale, const dou
         double dot = 0.0;
         for (int d = 0; d < D; ++d) dot += q[d] * K[t * C + h * D + d];
         sc[t] = dot * scale;
+        if (s_hist && t < n_hist) sc[t] -= jensen_term(q, s_hist + (t * H + h) * ng, D, group, scale);
         if (sc[t] > m) m = sc[t];
       }
       double l = 0.0;

@@ -474,6 +474,30 @@ def attention(Q, K, V, scale: float) -> np.ndarray:
     return O.transpose(1, 0, 2)
 
 
+def jensen_correction(Q, s_hist, group: int, scale: float) -> np.ndarray:
+    """Jensen-bias term of every (head, query, quantized key): [H, Nq, T].
+
+    (The abstract on the "Jensen bias" of INT2 key caches, among the related
+    papers listed on the CORAL-KV page.)  Uniform rounding noise of step s
+    on a key raises E[exp(scale q.k^)] by exp(0.5 scale^2 sum_g |q_g|^2 s_g^2/12)
+    to second order; this is that exponent."""
+    Nq, H, D = Q.shape
+    qn = (Q.reshape(Nq, H, D // group, group) ** 2).sum(-1)  # [Nq,H,NG]
+    var = np.asarray(s_hist, np.float64) ** 2 / 12.0  # [T,H,NG]
+    return 0.5 * scale * scale * np.einsum("qhg,thg->hqt", qn, var)
+
+
+def attention_corrected(Q, K, V, scale: float, n_hist: int, s_hist, group: int) -> np.ndarray:
+    """Naive attention whose first n_hist (quantized) keys have their scores
+    lowered by the Jensen-bias term; the remaining keys are uncompressed."""
+    S = np.matmul(Q.transpose(1, 0, 2), K.transpose(1, 2, 0)) * scale  # [H,Nq,Nk]
+    S[:, :, :n_hist] -= jensen_correction(Q, s_hist, group, scale)
+    m = S.max(axis=-1, keepdims=True)
+    p = np.exp(S - m)
+    O = np.matmul(p, V.transpose(1, 0, 2)) / p.sum(axis=-1, keepdims=True)
+    return O.transpose(1, 0, 2)
+
+
 def mixed_attention(Q, ck: Coded, cent_k, dec_k, cv: Coded, cent_v, dec_v,
                     desc: Desc, scale: float) -> np.ndarray:
     """Attention computed on the stored coefficients (reading R11).

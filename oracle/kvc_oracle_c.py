@@ -375,13 +375,35 @@ def attention(Q, K, V, scale: float, threads=None) -> np.ndarray:
     return O
 
 
+def attention_corrected(Q, K, V, scale: float, n_hist: int, s_hist, group: int, threads=None) -> np.ndarray:
+    """Softmax attention in which each of the first n_hist (quantized) keys'
+    scores is lowered by its Jensen-bias term 0.5 scale^2 sum_g |q_g|^2 s_g^2 / 12
+    (the abstract on the "Jensen bias" of INT2 key caches, CORAL-KV page);
+    s_hist [n_hist, H, D/group]."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    nq, H, D = Q.shape
+    nk = K.shape[0]
+    sh = _f64(s_hist)
+    O = np.empty((nq, H, D))
+
+    def run(a, b):
+        lib().kvo_attention_corrected(_i(b - a), _i(nk), H, D, ctypes.c_double(scale), _p(Q[a:b]), _p(K), _p(V),
+                                      _i(n_hist), _p(sh), group, _p(O[a:b]))
+
+    _drive(_runs(nq, threads), run)
+    return O
+
+
 def attend_compressed_xlayer(desc: Desc, w: dict, Q, ck: Coded, cv: Coded, K_src, V_src, K_self, V_self,
-                             scale: float, threads=None) -> np.ndarray:
+                             scale: float, threads=None, jensen: bool = False) -> np.ndarray:
     """Softmax attention of Q over [decoded history ; uncompressed chunk]."""
     K_hist, V_hist = decode_layer_xlayer(desc, w, ck, cv, K_src, V_src, threads)
+    T = K_hist.shape[0]
     if K_self is not None and len(K_self):
         K_hist = np.concatenate([K_hist, _f64(K_self)], axis=0)
         V_hist = np.concatenate([V_hist, _f64(V_self)], axis=0)
+    if jensen:
+        return attention_corrected(Q, K_hist, V_hist, scale, T, ck.s, desc.group, threads)
     return attention(Q, K_hist, V_hist, scale, threads)
 
 

@@ -93,7 +93,14 @@ def param_ulp(v, param: str) -> np.ndarray:
     return np.spacing(np.abs(v).astype(np.float16 if param == "f16" else np.float32)).astype(np.float64)
 
 
-PARAM_FLIP_BUDGET = 5e-2
+# fp16 (scale, zero) pairs that may differ from the oracle's, as a fraction of
+# the groups with identical inputs, plus three groups of slack for small
+# samples.  Observed on a B200 over every parity check: at most 0.6 % of the
+# groups in samples of 1000 or more (a residual moved by fp32 accumulation
+# error crosses an fp16 rounding boundary), 1 group of 70 at worst in the
+# small per-frame samples.
+PARAM_FLIP_RATE = 2e-2
+PARAM_FLIP_SLACK_GROUPS = 3
 
 
 U32 = 2.0 ** -23  # fp32 rounding unit, allowing for truncating accumulation
@@ -111,9 +118,9 @@ def assert_params_close(s_gpu, z_gpu, s_ref, z_ref, param: str, what="params", l
     per element, how far its prediction can be from the exact one (0 when
     there is no prediction).  Each stored value may then differ from the
     oracle's by that bound plus one rounding step of the parameter dtype, and
-    (fp16) at most 5 % of the groups may differ at all (a residual shift of
-    1e-5 crosses an fp16 rounding boundary of a value near 1 with probability
-    about 2e-5 / 2^-11 = 4 %).  `skip` marks groups whose inputs already
+    (fp16) at most PARAM_FLIP_RATE of the groups, plus PARAM_FLIP_SLACK_GROUPS
+    groups, may differ at all (a residual moved by the accumulation error
+    crosses an fp16 rounding boundary now and then).  `skip` marks groups whose inputs already
     differ (an earlier flipped code); they are not checked and do not count
     against the budget.  Returns the mask of groups whose pair differs."""
     ds = np.abs(s_gpu - s_ref)
@@ -129,10 +136,12 @@ def assert_params_close(s_gpu, z_gpu, s_ref, z_ref, param: str, what="params", l
     assert np.all((ds <= us * 1.0001) | ~ok), f"{what}: a scale is outside its bound (worst {np.max((ds / us)[ok]):.2f})"
     assert np.all((dz <= uz * 1.0001) | ~ok), f"{what}: a zero is outside its bound (worst {np.max((dz / uz)[ok]):.2f})"
     diff = (ds > 0) | (dz > 0)
-    rate = float(diff[ok].mean()) if ok.any() else 0.0  # among groups with the same inputs on both sides
-    OBSERVED.append({"check": what, "param_groups_differing": rate, "groups": int(ok.sum())})
+    n_ok = int(ok.sum())
+    rate = float(diff[ok].mean()) if n_ok else 0.0  # among groups with the same inputs on both sides
+    OBSERVED.append({"check": what, "param": param, "param_groups_differing": rate, "groups": n_ok})
     if param == "f16":
-        assert rate <= PARAM_FLIP_BUDGET, f"{what}: {rate:.2e} of the groups differ"
+        budget = PARAM_FLIP_RATE + PARAM_FLIP_SLACK_GROUPS / max(n_ok, 1)
+        assert rate <= budget, f"{what}: {rate:.2e} of the groups differ (budget {budget:.2e})"
         return diff
     return np.zeros(s_ref.shape, bool)
 

@@ -767,3 +767,40 @@ def test_attention_history_outputs_fp32_and_clustered():
                          kvc.alloc_workspace(kvc.OP_ENCODE, cdesc, cpred))
     Qc = synth.queries(8, 90, 16, 128).cuda()
     _history_outputs_case(cdesc, cpred, cbuf, Qc, None, None, None, None, 128 ** -0.5, 500, 16, 128, bf)
+
+
+# ---------------------------------------------------------------- Jensen-bias-corrected attention
+
+
+@pytest.mark.parametrize("n_q,n_self,T,rank,group", [(300, 130, 3 * 128 + 5, 64, 32), (700, 256, 16 * 128 - 7, 64, 32),
+                                                     (129, 64, 256, 0, 64)])
+def test_debiased_attention_cross_layer(n_q, n_self, T, rank, group):
+    """kvc_attend_compressed_debiased against the oracle's corrected softmax
+    (history codes by the oracle).  Queries are scaled so that the correction
+    moves the output well beyond the tolerance: the GPU result must be close to
+    the corrected reference and not to the plain one."""
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 112, L=2, T=T, rank=rank, calib_tokens=1024)
+    H, D = 12, 128
+    bf, hf = torch.bfloat16, torch.float16
+    od = _odesc(T, H, D, bf, 2, group, hf)
+    w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
+    Ks, Vs = U.to64(wl.K[0]), U.to64(wl.V[0])
+    ck, cv, _, _ = O.encode_layer_xlayer(od, w64, U.to64(wl.K[1]), U.to64(wl.V[1]), Ks, Vs)
+    buf = _oracle_codes_to_gpu(ck, cv, 2, "f16")
+    Q = (synth.queries(41, n_q, H, D).float() * 3).to(bf)
+    Kself, Vself = synth.queries(42, n_self, H, D), synth.queries(43, n_self, H, D)
+    desc = _desc(T, H, D, bf, 2, group, hf)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=rank)
+    Og = torch.empty(n_q, H, D, dtype=bf, device="cuda")
+    ws = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q)
+    kvc.kvc_attend_compressed_debiased(desc, pred, Q.cuda(), buf, wl.K[0].cuda(), wl.V[0].cuda(), Kself.cuda(),
+                                       Vself.cuda(), D ** -0.5, Og, ws)
+    _sync_ok()
+    args = (od, w64, U.to64(Q), ck, cv, Ks, Vs, U.to64(Kself), U.to64(Vself), D ** -0.5)
+    ref = O.attend_compressed_xlayer(*args, jensen=True)
+    plain = O.attend_compressed_xlayer(*args)
+    err = U.rel_l2(U.to64(Og), ref)
+    moved = U.rel_l2(plain, ref)
+    U.OBSERVED.append({"check": f"debiased attention T={T}", "rel_l2": err, "correction_moves": moved})
+    assert err <= U.ATT_TOL[bf], err
+    assert err < 0.25 * moved, (err, moved)

@@ -485,3 +485,60 @@ def test_mixed_attention_equals_attention_on_reconstructed_keys(O):
     Kx = O.decode_tensor_cluster(d, ck, cent_k, E, exact=True)
     Vx = O.decode_tensor_cluster(d, cv, cent_v, E, exact=True)
     np.testing.assert_allclose(fast, O.attention(Q, Kx, Vx, 0.25), rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------- Jensen-bias correction
+
+
+def test_jensen_correction_is_the_second_order_log_moment_of_rounding_noise(O):
+    """A key rounded with step s carries noise e ~ U(-s/2, s/2) per element, and
+    log E[exp(a e)] = log(sinh(a s / 2) / (a s / 2)) exactly; its second-order
+    term a^2 s^2 / 24 summed over the channels is the correction.  One quantized
+    history key and one chunk key with the same k: the ratio of their weights
+    is exp(-correction)."""
+    rng = np.random.default_rng(16)
+    D, group, scale = 64, 32, 0.3
+    q = rng.standard_normal((1, 1, D)) * np.exp2(rng.integers(-1, 2, (1, 1, D)))
+    k = rng.standard_normal((1, 1, D))
+    s = np.array([[[0.04, 0.11]]])  # unequal group scales: a swapped or shared group would show
+    K = np.concatenate([k, k])
+    V = np.zeros((2, 1, D))
+    V[0, 0, 0] = V[1, 0, 1] = 1.0
+    out = O.attention_corrected(q, K, V, scale, 1, s, group)
+    c = np.log(out[0, 0, 1] / out[0, 0, 0])
+    a = scale * q[0, 0]
+    x = a * np.repeat(s[0, 0], group) / 2
+    exact = np.sum(np.log(np.sinh(x) / x))
+    assert c > 0 and abs(c - exact) <= 1e-3 * exact, (c, exact)
+    # with no quantized keys, or lossless ones, it is plain attention
+    Q = rng.standard_normal((3, 2, D))
+    Kr, Vr = rng.standard_normal((9, 2, D)), rng.standard_normal((9, 2, D))
+    np.testing.assert_allclose(O.attention_corrected(Q, Kr, Vr, 0.4, 0, np.zeros((0, 2, 2)), group),
+                               O.attention(Q, Kr, Vr, 0.4), atol=1e-14)
+    np.testing.assert_allclose(O.attention_corrected(Q, Kr, Vr, 0.4, 9, np.zeros((9, 2, 2)), group),
+                               O.attention(Q, Kr, Vr, 0.4), atol=1e-14)
+
+
+def test_jensen_correction_removes_the_bias_in_expectation(O):
+    """Monte Carlo: keys k + e with e uniform of step s in each group; the mean
+    over noise draws of exp(score - correction) matches exp(score) of the
+    clean key, while the uncorrected mean is biased upward."""
+    rng = np.random.default_rng(17)
+    D, group, scale, n = 64, 32, 0.5, 200_000
+    q = rng.standard_normal(D)
+    k = rng.standard_normal(D)
+    s = np.array([0.3, 0.6])
+    e = (rng.random((n, D)) - 0.5) * np.repeat(s, group)
+    raw = scale * (k + e) @ q
+    # the oracle's correction for this query and key, read off a two-key attention
+    K = np.stack([k, k])[:, None, :]
+    V = np.zeros((2, 1, D))
+    V[0, 0, 0] = V[1, 0, 1] = 1.0
+    out = O.attention_corrected(q[None, None, :], K, V, scale, 1, s[None, None, :], group)
+    c = np.log(out[0, 0, 1] / out[0, 0, 0])
+    clean = np.exp(scale * k @ q)
+    biased = np.mean(np.exp(raw)) / clean - 1
+    fixed = np.mean(np.exp(raw - c)) / clean - 1
+    se = np.std(np.exp(raw)) / clean / np.sqrt(n)
+    assert biased > 10 * se
+    assert abs(fixed) < 4 * se + 0.02 * biased, (fixed, biased, se)
