@@ -42,12 +42,13 @@ METRIC = "KV tokens/s encoded+decoded (GB/s vs HBM peak); compressed-attn TFLOP/
 UNIT = "KV tokens/s"
 
 
-# DRAM bytes (read + write) per launch, from the ncu captures summarised under
+# DRAM bytes (read + write) per call, from the ncu captures summarised under
 # profiles/ (codec_xlayer_wan_layer.md, attention_cluster_wan.md,
-# mixed_attention_cluster.md, temporal_codec_layer.md); set to None when a
-# kernel changes after its capture.
-TRAFFIC = {"encode_xlayer": 674717696 + 202756608, "decode_xlayer": 437384192 + 152241920,
-           "attention_c2": 769948672 + 8668416, "attention_c4": None,
+# mixed_attention_cluster.md, cluster_codec_decode.md, temporal_codec_layer.md);
+# set to None when a kernel changes after its capture.
+TRAFFIC = {"encode_xlayer": 675341568 + 202485760, "decode_xlayer": 437443584 + 151249408,
+           "attention_c2": 745406720 + 7559680, "attention_c4": 26443520 + 146944,
+           "decode_c4": 4399616 + 80381696 + 4467712 + 80104704,
            "temporal_encode": 1425952000 + 356744960,
            "temporal_decode": 574324480 + 1285428224}
 
@@ -345,6 +346,73 @@ def row_attention(xb: XLayerBench, hbm, tf_burst, tf_sust, reps=3) -> dict:
                          "frac": tflops / tf_burst, "traffic": TRAFFIC["attention_c2"], "peak_kind": "burst bf16"}}
 
 
+def row_attention_debiased(xb: XLayerBench, hbm, tf_burst, reps=3) -> dict:
+    """The C2 attention with the Jensen-bias correction of the history keys
+    (kvc_attend_compressed_debiased), same inputs and FLOP count."""
+    dev = xb.wl.K[0].device
+    n_q = 3 * 1560
+    Q = synth.queries(synth.SEED_BASE + 2, n_q, H, D, device=dev)
+    Ks = synth.queries(synth.SEED_BASE + 12, n_q, H, D, device=dev)
+    Vs = synth.queries(synth.SEED_BASE + 22, n_q, H, D, device=dev)
+    O_ = torch.empty(n_q, H, D, dtype=torch.bfloat16, device=dev)
+    l = 15
+    ws = kvc.alloc_workspace(kvc.OP_ATTEND, xb.desc, xb.preds[l], n_q, device=dev)
+    Kh, Vh = xb.keep
+    call = lambda: kvc.kvc_attend_compressed_debiased(xb.desc, xb.preds[l], Q, xb.codes[l], Kh, Vh, Ks, Vs,
+                                                      D ** -0.5, O_, ws)
+    call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for s_, e_ in ev:
+        s_.record()
+        call()
+        e_.record()
+    synced_ok()
+    ms = statistics.median(time_events(ev))
+    total = 4 * n_q * (T_TOK + n_q) * H * D + XLayerBench.layer_flops()
+    tflops = total / (ms * 1e-3) / 1e12
+    return {"workload": "as c2_attention, with the Jensen-bias correction of the 32760 history keys",
+            "ms": ms, "value": tflops, "unit": "TFLOP/s (attention + one in-kernel decode of the history)",
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_burst, "unit": "TFLOP/s",
+                         "frac": tflops / tf_burst, "traffic": None, "peak_kind": "burst bf16"}}
+
+
+def row_eden2(dev, hbm, reps=3) -> dict:
+    """One predicted Wan-shaped layer (32760 tokens x 12 heads x 128, rank 64)
+    coded with the H64 / EDEN-2 residual codec: encode and decode."""
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 1, device=dev, L=2, T=T_TOK, H=H, D=D, rank=RANK,
+                          layers_needed=[1])
+    cb = synth.eden2_codebook().to(dev)
+    bf, hf = torch.bfloat16, torch.float16
+    desc = kvc.make_desc(T_TOK, H, D, bf, 2, 64, hf, residual_codec=kvc.RESIDUAL_H64_EDEN2)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl.weights[1], rank=RANK, residual_codebook=cb)
+    buf = kvc.alloc_codes(desc, pred, dev)
+    Kr, Vr = torch.empty_like(wl.K[1]), torch.empty_like(wl.V[1])
+    wse = kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred, device=dev)
+    wsd = kvc.alloc_workspace(kvc.OP_DECODE, desc, pred, device=dev)
+    enc = lambda: kvc.kvc_encode_layer(desc, pred, wl.K[1], wl.V[1], wl.K[0], wl.V[0], buf, Kr, Vr, wse)
+    dec = lambda: kvc.kvc_decode_layer(desc, pred, buf, wl.K[0], wl.V[0], Kr, Vr, wsd)
+    out = {"workload": "cross-layer layer, 32760 tokens x 12 heads x 128, rank 64, H64 / EDEN-2 residuals "
+                       "(4-bit index per pair, fp16 scale per 64 values)"}
+    C = H * D
+    w = sum(t.numel() * t.element_size() for t in wl.weights[1].values())
+    for name, fn, nio in (("encode", enc, 3), ("decode", dec, 2)):
+        fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for s_, e_ in ev:
+            s_.record()
+            fn()
+            e_.record()
+        synced_ok()
+        ms = statistics.median(time_events(ev))
+        byts = 2 * T_TOK * C * 2 * nio + kvc.kvc_codes_bytes(desc, pred) + w
+        gbs = byts / (ms * 1e-3) / 1e9
+        out[name] = {"ms": ms, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                            "frac": gbs / hbm, "traffic": None}}
+    return out
+
+
 def row_temporal(dev, hbm, reps=3) -> dict:
     tw = synth.temporal_layer(seed=synth.SEED_BASE + 3, device=dev)
     T, Hh, Dd = tw.K.shape
@@ -421,7 +489,7 @@ def row_cluster(dev, hbm, tf_burst, reps=3) -> dict:
             byts = 2 * T * C * 2 + kvc.kvc_codes_bytes(desc, pred)
             gbs = byts / (ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
-        roof["traffic"] = TRAFFIC["attention_c4"] if name == "attention" else None
+        roof["traffic"] = {"attention": TRAFFIC["attention_c4"], "decode": TRAFFIC["decode_c4"]}.get(name)
         out[name] = {"ms": ms, "roofline": roof}
     return out
 
@@ -436,7 +504,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the extra per-row measurements")
-    ap.add_argument("--rows", default="c2,c3,c4", help="which extra rows to measure (comma-separated)")
+    ap.add_argument("--rows", default="c2,c2j,c3,c4,eden2",
+                    help="which extra rows to measure (comma-separated)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--layers", type=int, default=L_LAYERS,
@@ -561,10 +630,13 @@ def main():
     if world == 1:
         want = set(args.rows.split(",")) if not args.no_rows else set()
         rows = {}
-        if "c2" in want and L_RUN > 15:
+        if ("c2" in want or "c2j" in want) and L_RUN > 15:
             xb.encode_chain(keep_layer=15)
             torch.cuda.synchronize()
-            rows["c2_attention"] = row_attention(xb, hbm, tf_burst, tf_sust)
+            if "c2" in want:
+                rows["c2_attention"] = row_attention(xb, hbm, tf_burst, tf_sust)
+            if "c2j" in want:
+                rows["c2_attention_debiased"] = row_attention_debiased(xb, hbm, tf_burst)
             xb.keep = None
             torch.cuda.empty_cache()
         if "c3" in want:
@@ -572,6 +644,9 @@ def main():
             torch.cuda.empty_cache()
         if "c4" in want:
             rows["c4_cluster"] = row_cluster(dev, hbm, tf_burst)
+            torch.cuda.empty_cache()
+        if "eden2" in want:
+            rows["c1_eden2_layer"] = row_eden2(dev, hbm)
         rows = rows or None
         if not args.no_cpu:
             # about 25 s of host work: the single-threaded oracle, then its thread driver

@@ -49,6 +49,14 @@ kvc_status check_desc(const kvc_layer_desc* d, const kvc_predictor* p) {
   if (d->dtype != KVC_F32 && d->dtype != KVC_BF16) return KVC_ERR_UNSUPPORTED;
   if (d->param_dtype != KVC_F32 && d->param_dtype != KVC_F16) return KVC_ERR_UNSUPPORTED;
   if (d->bits != 2 && d->bits != 4 && d->bits != 8) return KVC_ERR_UNSUPPORTED;
+  if (d->residual_codec == KVC_RESIDUAL_H64_EDEN2) {
+    // one scale per 64 transformed values, 4 bits per pair (the INT2 rate)
+    if (p->kind != KVC_PRED_NONE && p->kind != KVC_PRED_XLAYER_DPLR) return KVC_ERR_UNSUPPORTED;
+    if (d->bits != 2 || d->group != 64) return KVC_ERR_UNSUPPORTED;
+    if (p->kind == KVC_PRED_XLAYER_DPLR && (p->rank < 0 || p->rank > 128)) return KVC_ERR_UNSUPPORTED;
+    return KVC_OK;
+  }
+  if (d->residual_codec != KVC_RESIDUAL_RTN) return KVC_ERR_UNSUPPORTED;
   switch (p->kind) {
     case KVC_PRED_NONE:
     case KVC_PRED_XLAYER_DPLR:
@@ -78,6 +86,11 @@ Sizes sizes_of(const kvc_layer_desc* d, const kvc_predictor* p) {
   const size_t T = (size_t)d->n_tokens, H = d->n_heads, D = d->head_dim;
   const size_t pair = 2 * (size_t)param_size(d->param_dtype);
   Sizes s{0, 0, 0};
+  if (d->residual_codec == KVC_RESIDUAL_H64_EDEN2) {
+    s.codes = T * H * D / 4;  // a 4-bit index per pair
+    s.params = T * H * (D / 64) * (size_t)param_size(d->param_dtype);
+    return s;
+  }
   if (p->kind == KVC_PRED_CLUSTER) {
     const size_t m = p->code_dim;
     s.codes = T * m * d->bits / 8;
@@ -152,10 +165,11 @@ cudaError_t codec_xlayer(const kvc_layer_desc* d, const kvc_predictor* p, bool e
     LatentArgs<TS> la{T, C, r, (const TS*)Ks, nullptr, (const TS*)p->k_w, Zk};
     if ((e = launch_latent(la, st)) != cudaSuccess) return e;
   }
+  const float* cb = d->residual_codec == KVC_RESIDUAL_H64_EDEN2 ? (const float*)p->residual_codebook : nullptr;
   HeadsArgs<TS, TP> hk{T, H, d->bits, d->group, r,
                        pred ? (const TS*)Ks : nullptr, nullptr, pred ? (const TS*)p->k_block : nullptr,
                        Zk, (const TS*)p->k_u, (const TS*)K,
-                       (uint8_t*)c->k_codes, (Pair<TP>*)c->k_params, (TS*)Kr};
+                       (uint8_t*)c->k_codes, (Pair<TP>*)c->k_params, (TS*)Kr, cb};
   if ((e = launch_heads(hk, D, enc, st)) != cudaSuccess) return e;
   if (r) {
     LatentArgs<TS> la{T, C, r, (const TS*)Kr, (const TS*)Vs, (const TS*)p->v_w, Zv};
@@ -164,7 +178,7 @@ cudaError_t codec_xlayer(const kvc_layer_desc* d, const kvc_predictor* p, bool e
   HeadsArgs<TS, TP> hv{T, H, d->bits, d->group, r,
                        pred ? (const TS*)Kr : nullptr, pred ? (const TS*)Vs : nullptr,
                        pred ? (const TS*)p->v_block : nullptr, Zv, (const TS*)p->v_u, (const TS*)V,
-                       (uint8_t*)c->v_codes, (Pair<TP>*)c->v_params, (TS*)Vr};
+                       (uint8_t*)c->v_codes, (Pair<TP>*)c->v_params, (TS*)Vr, cb};
   return launch_heads(hv, D, enc, st);
 }
 
@@ -278,6 +292,12 @@ kvc_status check_weights(const kvc_predictor* p) {
   return KVC_OK;
 }
 
+kvc_status check_codebook(const kvc_layer_desc* d, const kvc_predictor* p) {
+  if (d->residual_codec != KVC_RESIDUAL_H64_EDEN2) return KVC_OK;
+  if (!p->residual_codebook) return KVC_ERR_INVALID_ARGUMENT;
+  return aligned16(p->residual_codebook) ? KVC_OK : KVC_ERR_MISALIGNED;
+}
+
 kvc_status codec_common(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
                         const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, void* ws,
                         size_t ws_bytes, void* stream) {
@@ -285,6 +305,7 @@ kvc_status codec_common(const kvc_layer_desc* d, const kvc_predictor* p, bool en
   if (s != KVC_OK) return s;
   if (d->n_tokens == 0) return KVC_OK;  // nothing to code
   if ((s = check_weights(p)) != KVC_OK) return s;
+  if ((s = check_codebook(d, p)) != KVC_OK) return s;
   if (!codes_ok(p, c)) return KVC_ERR_INVALID_ARGUMENT;
   if (enc && (!K || !V)) return KVC_ERR_INVALID_ARGUMENT;
   if (p->kind == KVC_PRED_TEMPORAL && d->anchor_bits == 0 && (!Ks || !Vs)) return KVC_ERR_INVALID_ARGUMENT;
@@ -345,6 +366,10 @@ size_t kvc_codes_bytes(const kvc_layer_desc* desc, const kvc_predictor* pred) {
 
 size_t kvc_workspace_bytes(int op, const kvc_layer_desc* desc, const kvc_predictor* pred, int64_t n_q) {
   if (check_desc(desc, pred) != KVC_OK) return 0;
+  if (op == KVC_OP_REFIT_K || op == KVC_OP_REFIT_V)
+    return pred->kind == KVC_PRED_XLAYER_DPLR
+               ? refit_workspace(desc->n_tokens, desc->n_heads, desc->head_dim, pred->rank, op == KVC_OP_REFIT_V)
+               : 0;
   size_t a = simt_workspace(op, desc, pred);
   size_t b = tc_workspace(op, desc, pred, n_q);
   return a > b ? a : b;
@@ -370,6 +395,7 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
   if (s != KVC_OK) return s;
   if (p->kind == KVC_PRED_TEMPORAL) return KVC_ERR_UNSUPPORTED;
   if ((s = check_weights(p)) != KVC_OK) return s;
+  if ((s = check_codebook(d, p)) != KVC_OK) return s;
   if (n_q < 0 || n_self < 0) return KVC_ERR_INVALID_ARGUMENT;
   if (p->kind == KVC_PRED_CLUSTER && n_self != 0) return KVC_ERR_UNSUPPORTED;
   if (!codes_ok(p, codes) || (n_q > 0 && (!Q || !O))) return KVC_ERR_INVALID_ARGUMENT;
@@ -455,6 +481,36 @@ kvc_status kvc_attend_compressed_debiased(const kvc_layer_desc* d, const kvc_pre
   if (n_q == 0) return KVC_OK;
   cudaError_t e = tc_attend(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, K_rec_opt, V_rec_opt,
                             ws, ws_bytes, (cudaStream_t)stream, true);
+  return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+}
+
+kvc_status kvc_refit_block_diag(const kvc_layer_desc* d, const kvc_predictor* p, int tensor, const void* X0,
+                                const void* X1, const void* Y, float ridge, void* block_out, void* ws,
+                                size_t ws_bytes, void* stream) {
+  kvc_status s = check_desc(d, p);
+  if (s != KVC_OK) return s;
+  if (p->kind != KVC_PRED_XLAYER_DPLR) return KVC_ERR_UNSUPPORTED;
+  if (tensor != 0 && tensor != 1) return KVC_ERR_INVALID_ARGUMENT;
+  if (d->n_tokens < 1 || !(ridge >= 0.f)) return KVC_ERR_INVALID_ARGUMENT;
+  if (!X0 || !Y || !block_out || (tensor == 1 && !X1)) return KVC_ERR_INVALID_ARGUMENT;
+  const void* w = tensor ? p->v_w : p->k_w;
+  const void* u = tensor ? p->v_u : p->k_u;
+  if (p->rank > 0 && (!w || !u)) return KVC_ERR_INVALID_ARGUMENT;
+  const void* ptrs[] = {X0, tensor ? X1 : nullptr, Y, block_out, ws, p->rank ? w : nullptr, p->rank ? u : nullptr};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return KVC_ERR_MISALIGNED;
+  const size_t need = kvc_workspace_bytes(tensor ? KVC_OP_REFIT_V : KVC_OP_REFIT_K, d, p, 0);
+  if (ws_bytes < need || !ws) return KVC_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = (cudaStream_t)stream;
+  const void* x1 = tensor ? X1 : nullptr;
+  cudaError_t e;
+  if (d->dtype == KVC_F32)
+    e = launch_refit<float>(d->n_tokens, d->n_heads, d->head_dim, p->rank, (const float*)X0, (const float*)x1,
+                            (const float*)Y, (const float*)w, (const float*)u, ridge, (float*)block_out, ws, st);
+  else
+    e = launch_refit<__nv_bfloat16>(d->n_tokens, d->n_heads, d->head_dim, p->rank, (const __nv_bfloat16*)X0,
+                                    (const __nv_bfloat16*)x1, (const __nv_bfloat16*)Y, (const __nv_bfloat16*)w,
+                                    (const __nv_bfloat16*)u, ridge, (__nv_bfloat16*)block_out, ws, st);
   return e == cudaSuccess ? KVC_OK : cuda_fail(e);
 }
 

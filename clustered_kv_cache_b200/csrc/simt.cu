@@ -85,6 +85,128 @@ __global__ void __launch_bounds__(kThreads) latent_kernel(LatentArgs<TS> a) {
   }
 }
 
+// ============================================================== H64 / EDEN-2 rows
+//
+// "CORAL-KV: Compact Cross-Layer Prediction and Residual Coding for
+// Autoregressive Video KV Caches", Fig. 5 (H_n on each non-overlapping group of
+// n residual channels; one shared scale per 64 values) and Fig. 9 (16 EDEN-2
+// points over pairs of H64-transformed residuals).  A row of D = 32 E values
+// is held by a warp, lane l holding elements [l E, (l + 1) E); a 64-channel
+// group spans 64 / E lanes.  The orthonormal Walsh-Hadamard transform
+// y_i = (1/8) sum_j (-1)^popcount(i & j) r_j runs as six butterfly stages, the
+// low log2(E) index bits inside a lane and the others across lanes by xor
+// shuffles.  Pairs (y_2p, y_2p+1) sit inside a lane.
+
+template <int E>
+__device__ __forceinline__ void walsh64(float (&v)[E]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int b = 1; b < E; b <<= 1)  // index bits inside the lane
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (!(e & b)) {
+        const float a = v[e], c = v[e + b];
+        v[e] = a + c;
+        v[e + b] = a - c;
+      }
+#pragma unroll
+  for (int o = 1; o < 64 / E; o <<= 1) {  // index bits across lanes
+    const bool upper = lane & o;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float w = __shfl_xor_sync(0xffffffffu, v[e], o);
+      v[e] = upper ? w - v[e] : v[e] + w;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] *= 0.125f;
+}
+
+// sum over the lanes of this lane's 64-channel group
+template <int E>
+__device__ __forceinline__ float group_sum64(float x) {
+#pragma unroll
+  for (int o = 1; o < 64 / E; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Encodes the residual r of this lane's elements; writes the pair indices and
+// the group scale, returns the decoded residual in rh.  cb: 16 points in
+// shared memory.
+template <int E, typename TP>
+__device__ __forceinline__ void eden2_encode(const float (&r)[E], const float* cb, uint8_t* row_codes,
+                                             TP* row_scales, float (&rh)[E]) {
+  static_assert(E % 2 == 0, "pairs inside a lane");
+  const int lane = threadIdx.x & 31;
+  float y[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) y[e] = r[e];
+  walsh64<E>(y);
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) ss = fmaf(y[e], y[e], ss);
+  const float sumsq = group_sum64<E>(ss);
+  int k[E / 2];
+  float dot = 0.f;
+  const float inv_sigma = sumsq > 0.f ? 1.f / sqrtf(sumsq * (1.f / 64.f)) : 0.f;
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) {
+    const float u0 = y[2 * i] * inv_sigma, u1 = y[2 * i + 1] * inv_sigma;
+    int best = 0;
+    float bd = INFINITY;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float d0 = u0 - cb[2 * j], d1 = u1 - cb[2 * j + 1];
+      const float d = fmaf(d0, d0, d1 * d1);
+      if (d < bd) {  // strict: ties keep the lowest index
+        bd = d;
+        best = j;
+      }
+    }
+    k[i] = sumsq > 0.f ? best : 0;
+    dot = fmaf(y[2 * i], cb[2 * k[i]], fmaf(y[2 * i + 1], cb[2 * k[i] + 1], dot));
+  }
+  dot = group_sum64<E>(dot);
+  const TP S = from_f<TP>(sumsq > 0.f && dot > 0.f ? sumsq / dot : 0.f);
+  const float sf = to_f(S);
+  if ((lane % (64 / E)) == 0) row_scales[lane / (64 / E)] = S;
+  // indices: pair p of the row at bits [4p, 4p + 4); this lane holds pairs lane E/2 + i
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) w |= (uint32_t)k[i] << (4 * i);
+  if (E >= 4) {
+    if (E == 4) row_codes[lane] = (uint8_t)w;
+    else *reinterpret_cast<uint16_t*>(row_codes + lane * (E / 4)) = (uint16_t)w;
+  } else {  // one pair per lane: two lanes per byte
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, w, 1);
+    if (!(lane & 1)) row_codes[lane / 2] = (uint8_t)(w | (hi << 4));
+  }
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) {
+    rh[2 * i] = sf * cb[2 * k[i]];
+    rh[2 * i + 1] = sf * cb[2 * k[i] + 1];
+  }
+  walsh64<E>(rh);
+}
+
+template <int E, typename TP>
+__device__ __forceinline__ void eden2_decode(const uint8_t* row_codes, const TP* row_scales, const float* cb,
+                                             float (&rh)[E]) {
+  const int lane = threadIdx.x & 31;
+  uint32_t w;
+  if (E == 4) w = row_codes[lane];
+  else if (E > 4) w = *reinterpret_cast<const uint16_t*>(row_codes + lane * (E / 4));
+  else w = (uint32_t)row_codes[lane / 2] >> ((lane & 1) * 4);
+  const float sf = to_f(row_scales[lane / (64 / E)]);
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) {
+    const int k = (w >> (4 * i)) & 15;
+    rh[2 * i] = sf * cb[2 * k];
+    rh[2 * i + 1] = sf * cb[2 * k + 1];
+  }
+  walsh64<E>(rh);
+}
+
 // ============================================================== per-head codec rows
 
 template <typename TS, typename TP, int D, bool ENC>
@@ -123,6 +245,8 @@ __global__ void __launch_bounds__(kThreads) heads_kernel(HeadsArgs<TS, TP> a) {
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < NJ; ++j) sP[(ty * 4 + i) * D + tx + 32 * j] = acc[i][j];
+  __shared__ float sCb[32];  // the H64 / EDEN-2 points
+  if (a.codebook && threadIdx.x < 32) sCb[threadIdx.x] = a.codebook[threadIdx.x];
   __syncthreads();
   RowCodec<E> rc{a.bits, a.group};
   const int row_bytes = D * a.bits / 8;
@@ -134,6 +258,27 @@ __global__ void __launch_bounds__(kThreads) heads_kernel(HeadsArgs<TS, TP> a) {
     float p[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) p[e] = sP[i * D + lane * E + e];
+    if (a.codebook) {  // H64 / EDEN-2 residuals: D/4 code bytes and D/64 scales per row
+      uint8_t* rcodes = a.codes + row * (D / 4);
+      TP* rsc = reinterpret_cast<TP*>(a.params) + row * (D / 64);
+      float rh[E];
+      if (ENC) {
+        float x[E], r[E];
+        load_vec<TS, E>(a.x + row * D + lane * E, x);
+#pragma unroll
+        for (int e = 0; e < E; ++e) r[e] = x[e] - p[e];
+        eden2_encode<E, TP>(r, sCb, rcodes, rsc, rh);
+      } else {
+        eden2_decode<E, TP>(rcodes, rsc, sCb, rh);
+      }
+      if (a.rec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = p[e] + rh[e];
+        store_vec<TS, E>(a.rec + row * D + lane * E, o);
+      }
+      continue;
+    }
     int q[E];
     float s, z;
     uint8_t* rcodes = a.codes + row * row_bytes;

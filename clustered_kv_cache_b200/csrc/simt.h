@@ -28,8 +28,9 @@ struct HeadsArgs {
   const TS* U;      // [C][r]
   const TS* x;      // clean rows (encode)
   uint8_t* codes;   // [T][H][D*bits/8]
-  Pair<TP>* params; // [T][H][D/group]
+  Pair<TP>* params; // [T][H][D/group] (H64 / EDEN-2: [T][H][D/64] scales of type TP)
   TS* rec;          // [T][H][D] or NULL
+  const float* codebook;  // H64 / EDEN-2 points [16][2], or NULL for the scalar quantizer
 };
 
 template <typename TS, typename TP>
@@ -123,6 +124,11 @@ template <typename TS>
 cudaError_t launch_attention(const AttnArgs<TS>& a, int D, cudaStream_t st);
 template <typename TS, typename TP>
 cudaError_t launch_mixed_attention(const MixedArgs<TS, TP>& a, cudaStream_t st);
+// video-adapted refit of the per-head blocks (refit.cu); X1 == NULL: the K block
+size_t refit_workspace(int64_t T, int H, int D, int r, bool v);
+template <typename TS>
+cudaError_t launch_refit(int64_t T, int H, int D, int r, const TS* X0, const TS* X1, const TS* Y, const TS* W,
+                         const TS* U, float ridge, TS* block, void* ws, cudaStream_t st);
 cudaError_t launch_pack(const uint8_t* codes, int64_t n, int bits, void* packed, cudaStream_t st);
 cudaError_t launch_unpack(const void* packed, int64_t n, int bits, uint8_t* codes, cudaStream_t st);
 

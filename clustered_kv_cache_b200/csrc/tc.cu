@@ -901,7 +901,7 @@ static cudaError_t dispatch(int group, int rc, const Maps& m, const Args& a, cud
 }  // namespace tc
 
 bool tc_codec_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
-  if (p->kind != KVC_PRED_XLAYER_DPLR) return false;
+  if (p->kind != KVC_PRED_XLAYER_DPLR || d->residual_codec != KVC_RESIDUAL_RTN) return false;
   if (d->dtype != KVC_BF16 || d->head_dim != 128 || d->param_dtype != KVC_F16) return false;
   if (d->bits != 2 && d->bits != 4) return false;
   if (d->group != 32 && d->group != 64) return false;

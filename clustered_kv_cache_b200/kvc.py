@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libkvc.so")
 
 KVC_F32, KVC_BF16, KVC_F16 = 0, 1, 2
 PRED_NONE, PRED_XLAYER_DPLR, PRED_TEMPORAL, PRED_CLUSTER = 0, 1, 2, 3
-OP_ENCODE, OP_DECODE, OP_ATTEND = 0, 1, 2
+OP_ENCODE, OP_DECODE, OP_ATTEND, OP_REFIT_K, OP_REFIT_V = 0, 1, 2, 3, 4
 
 STATUS = {0: "KVC_OK", 1: "KVC_ERR_INVALID_ARGUMENT", 2: "KVC_ERR_UNSUPPORTED", 3: "KVC_ERR_MISALIGNED",
           4: "KVC_ERR_WORKSPACE_TOO_SMALL", 5: "KVC_ERR_CUDA", 6: "KVC_ERR_DEVICE_TIMEOUT"}
@@ -27,7 +27,7 @@ STATUS = {0: "KVC_OK", 1: "KVC_ERR_INVALID_ARGUMENT", 2: "KVC_ERR_UNSUPPORTED", 
 EXPORTED = ["kvc_codes_sizes", "kvc_codes_bytes", "kvc_workspace_bytes", "kvc_encode_layer", "kvc_decode_layer",
             "kvc_attend_compressed", "kvc_pack_codes", "kvc_unpack_codes", "kvc_get_device_error",
             "kvc_status_string", "kvc_last_cuda_error", "kvc_launch_counter", "kvc_testing_inject_stall",
-            "kvc_attend_compressed_debiased"]
+            "kvc_attend_compressed_debiased", "kvc_refit_block_diag"]
 
 
 class KvcError(RuntimeError):
@@ -39,14 +39,15 @@ class KvcError(RuntimeError):
 class LayerDesc(ctypes.Structure):
     _fields_ = [("n_tokens", ctypes.c_int64), ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("bits", ctypes.c_int32), ("group", ctypes.c_int32),
-                ("param_dtype", ctypes.c_int32), ("frame_tokens", ctypes.c_int32), ("anchor_bits", ctypes.c_int32)]
+                ("param_dtype", ctypes.c_int32), ("frame_tokens", ctypes.c_int32), ("anchor_bits", ctypes.c_int32),
+                ("residual_codec", ctypes.c_int32)]
 
 
 class Predictor(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("rank", ctypes.c_int32), ("n_clusters", ctypes.c_int32),
                 ("code_dim", ctypes.c_int32)] + [(n, ctypes.c_void_p) for n in (
                     "k_block", "k_w", "k_u", "v_block", "v_w", "v_u", "k_centroids", "k_enc", "k_dec",
-                    "v_centroids", "v_enc", "v_dec")]
+                    "v_centroids", "v_enc", "v_dec", "residual_codebook")]
 
 
 class Codes(ctypes.Structure):
@@ -82,6 +83,7 @@ def lib():
         "kvc_decode_layer": (I, [D, PR, CO, V, V, V, V, V, SZ, V]),
         "kvc_attend_compressed": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, V, V, SZ, V]),
         "kvc_attend_compressed_debiased": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, V, V, SZ, V]),
+        "kvc_refit_block_diag": (I, [D, PR, ctypes.c_int, V, V, V, F, V, V, SZ, V]),
         "kvc_pack_codes": (I, [V, I64, I, V, V]),
         "kvc_unpack_codes": (I, [V, I64, I, V, V]),
         "kvc_get_device_error": (I, [V]),
@@ -126,16 +128,24 @@ def _check(status: int, where: str):
         raise KvcError(status, where, detail)
 
 
+RESIDUAL_RTN, RESIDUAL_H64_EDEN2 = 0, 1
+
+
 def make_desc(n_tokens: int, n_heads: int, head_dim: int, dtype=torch.bfloat16, bits: int = 2, group: int = 32,
-              param_dtype=torch.float16, frame_tokens: int = 0, anchor_bits: int = 4) -> LayerDesc:
+              param_dtype=torch.float16, frame_tokens: int = 0, anchor_bits: int = 4,
+              residual_codec: int = RESIDUAL_RTN) -> LayerDesc:
     return LayerDesc(n_tokens, n_heads, head_dim, _DT[dtype], bits, group, _DT[param_dtype], frame_tokens,
-                     anchor_bits)
+                     anchor_bits, residual_codec)
 
 
 def make_predictor(kind: int, weights: dict | None = None, rank: int = 0, n_clusters: int = 0,
-                   code_dim: int = 0) -> Predictor:
+                   code_dim: int = 0, residual_codebook: torch.Tensor | None = None) -> Predictor:
+    """residual_codebook: the 16 H64 / EDEN-2 points, fp32 [16, 2] on the device."""
     p = Predictor(kind, rank, n_clusters, code_dim)
-    for k, v in (weights or {}).items():
+    weights = dict(weights or {})
+    if residual_codebook is not None:
+        weights["residual_codebook"] = residual_codebook
+    for k, v in weights.items():
         if v is not None:
             setattr(p, k, _ptr(v))
     p._keep = weights  # keep the tensors alive with the struct
@@ -237,6 +247,14 @@ def kvc_attend_compressed_debiased(desc, pred, Q, codes: CodeBuffers, K_src, V_s
                                                 _ptr(V_self), n_self, ctypes.c_float(scale), _ptr(O), _ptr(K_rec),
                                                 _ptr(V_rec), wp, wn, _stream(stream)),
            "kvc_attend_compressed_debiased")
+
+
+def kvc_refit_block_diag(desc, pred, tensor: int, X0, X1, Y, ridge: float, block_out, ws=None, stream=None):
+    """Video-adapted refit of the per-head blocks (tensor 0: K, 1: V)."""
+    wp, wn = _ws(ws)
+    _check(lib().kvc_refit_block_diag(ctypes.byref(desc), ctypes.byref(pred), int(tensor), _ptr(X0), _ptr(X1),
+                                      _ptr(Y), ctypes.c_float(ridge), _ptr(block_out), wp, wn, _stream(stream)),
+           "kvc_refit_block_diag")
 
 
 def kvc_pack_codes(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None):

@@ -20,6 +20,7 @@ seed; the same seed on the same device type gives the same tensors.
 
 from __future__ import annotations
 
+import functools
 import math
 from dataclasses import dataclass, field
 
@@ -371,3 +372,50 @@ def cluster_layer(seed: int = SEED_BASE + 4, device="cpu", T: int = 32768, H: in
         out[name + "_enc"] = E.T.to(dtype).contiguous()
     return ClusterWorkload(out["k"], out["v"], out["k_cent"], out["v_cent"], out["k_enc"], out["k_dec"],
                            out["v_enc"], out["v_dec"])
+
+
+# ---------------------------------------------------------------------------
+# EDEN-2 codebook (input of the H64 / EDEN-2 residual codec)
+# ---------------------------------------------------------------------------
+
+
+@functools.lru_cache(maxsize=4)
+def _eden2_codebook_cached(n_points: int, iters: int, grid: int, span: float) -> torch.Tensor:
+    return _eden2_lloyd(n_points, iters, grid, span)
+
+
+def eden2_codebook(n_points: int = 16, iters: int = 300, grid: int = 801, span: float = 6.0) -> torch.Tensor:
+    """The 16 two-dimensional reconstruction points of the EDEN-2 residual
+    quantizer ("CORAL-KV ...", Fig. 9(a) pictures them over H64-transformed
+    residual pairs but prints no values): the Lloyd-Max quantizer of the
+    standard two-dimensional Gaussian (an orthonormal Hadamard transform makes
+    the normalised residual pairs close to that), computed here offline by
+    Lloyd iterations over a deterministic quadrature grid, starting from a
+    centre point, a ring of 5 and a ring of 10.  Returns fp32 [16, 2], sorted
+    by radius then angle.  Not a codec step: both the GPU path and the oracle
+    receive these values as an input."""
+    return _eden2_codebook_cached(n_points, iters, grid, span).clone()
+
+
+def _eden2_lloyd(n_points: int, iters: int, grid: int, span: float) -> torch.Tensor:
+    assert n_points == 16
+    ax = torch.linspace(-span, span, grid, dtype=torch.float64)
+    X, Y = torch.meshgrid(ax, ax, indexing="ij")
+    P = torch.stack([X.reshape(-1), Y.reshape(-1)], 1)
+    w = torch.exp(-0.5 * (P * P).sum(1))
+    w = w / w.sum()
+    ang5 = torch.arange(5, dtype=torch.float64) * (2 * math.pi / 5)
+    ang10 = torch.arange(10, dtype=torch.float64) * (2 * math.pi / 10) + math.pi / 10
+    C = torch.cat([torch.zeros(1, 2, dtype=torch.float64),
+                   torch.stack([ang5.cos(), ang5.sin()], 1) * 1.0,
+                   torch.stack([ang10.cos(), ang10.sin()], 1) * 2.2])
+    for _ in range(iters):
+        d = torch.cdist(P, C)
+        lab = d.argmin(1)
+        mass = torch.zeros(16, dtype=torch.float64).index_add_(0, lab, w)
+        sums = torch.zeros(16, 2, dtype=torch.float64).index_add_(0, lab, P * w[:, None])
+        C = sums / mass[:, None]
+    r = C.norm(dim=1)
+    a = torch.atan2(C[:, 1], C[:, 0])
+    order = sorted(range(16), key=lambda i: (round(float(r[i]), 6), float(a[i])))
+    return C[order].float().contiguous()

@@ -70,6 +70,12 @@ typedef enum {
 
 typedef enum { KVC_F32 = 0, KVC_BF16 = 1, KVC_F16 = 2 } kvc_dtype;
 
+/* Residual codecs (kvc_layer_desc.residual_codec). */
+typedef enum {
+  KVC_RESIDUAL_RTN = 0,       /* scalar asymmetric group quantizer (the default) */
+  KVC_RESIDUAL_H64_EDEN2 = 1  /* H64 Hadamard transform + EDEN-2 pair quantizer */
+} kvc_residual_codec;
+
 typedef enum {
   KVC_PRED_NONE = 0,
   KVC_PRED_XLAYER_DPLR = 1,
@@ -87,7 +93,17 @@ typedef enum {
  *  frame_tokens: tokens per frame (temporal only; token t = f*frame_tokens+s).
  *  anchor_bits: temporal only: bits of frame 0, coded with prediction 0
  *         (2, 4 or 8); or 0 when the call continues a sequence, whose
- *         reconstructed history then arrives in K_src / V_src. */
+ *         reconstructed history then arrives in K_src / V_src.
+ *  residual_codec: KVC_RESIDUAL_RTN, or KVC_RESIDUAL_H64_EDEN2 ("CORAL-KV ...",
+ *         Fig. 5, Fig. 9, Table 9): each group of 64 residual channels is
+ *         multiplied by the orthonormal Sylvester Walsh-Hadamard matrix
+ *         H64 / 8; its 32 pairs (y_2p, y_2p+1), normalised by
+ *         sigma = sqrt(mean y^2), take the 4-bit index of the nearest of 16
+ *         points (pred->residual_codebook; ties to the lowest index); one
+ *         scale per group, S = |y|^2 / <y, c> (EDEN's unbiased scale, 0 when
+ *         y = 0 or <y, c> <= 0), is stored in param_dtype; decoding applies
+ *         H64 / 8 to S c.  Requires bits = 2 (4 bits per pair), group = 64 and
+ *         KVC_PRED_NONE or KVC_PRED_XLAYER_DPLR; runs on the CUDA cores. */
 typedef struct {
   int64_t n_tokens;
   int32_t n_heads;
@@ -98,6 +114,7 @@ typedef struct {
   int32_t param_dtype;
   int32_t frame_tokens;
   int32_t anchor_bits;
+  int32_t residual_codec;
 } kvc_layer_desc;
 
 /* Predictor weights (device pointers, dtype of the layer, read only).
@@ -108,7 +125,9 @@ typedef struct {
  *  TEMPORAL:    k_block [H][D][2D] over [K_{f-1},h | K_{f-2},h],
  *               v_block [H][D][2D] over [K_f,h | V_{f-1},h].
  *  CLUSTER:     k_centroids [n_clusters][C], k_enc [code_dim][C],
- *               k_dec [C][code_dim], and the same for v; n_clusters <= 256. */
+ *               k_dec [C][code_dim], and the same for v; n_clusters <= 256.
+ *  residual_codebook: with KVC_RESIDUAL_H64_EDEN2, the 16 two-dimensional
+ *               points as fp32 [16][2] (device memory); else ignored. */
 typedef struct {
   int32_t kind;
   int32_t rank;
@@ -118,6 +137,7 @@ typedef struct {
   const void *v_block, *v_w, *v_u;
   const void *k_centroids, *k_enc, *k_dec;
   const void *v_centroids, *v_enc, *v_dec;
+  const void* residual_codebook;
 } kvc_predictor;
 
 /* Compressed storage of one layer (device pointers, caller-owned).
@@ -129,6 +149,9 @@ typedef struct {
  *    frames at bits.
  *  CLUSTER: k_codes [T][code_dim*bits/8], k_params [T][code_dim/group][2],
  *    k_assign [T] uint8 centre index.
+ *  H64 / EDEN-2 residuals: k_codes [T][H][D/4] bytes, pair p's index at bits
+ *    [4p, 4p+4) of the row, least significant first; k_params [T][H][D/64]
+ *    scales in param_dtype (one value per group, no zero-point).
  *  The v_* members hold V the same way.  Sizes: kvc_codes_sizes(). */
 typedef struct {
   void *k_codes, *k_params, *v_codes, *v_params;
@@ -154,7 +177,7 @@ KVC_API kvc_status kvc_codes_sizes(const kvc_layer_desc* desc, const kvc_predict
 KVC_API size_t kvc_codes_bytes(const kvc_layer_desc* desc, const kvc_predictor* pred);
 
 /* Operation codes of kvc_workspace_bytes. */
-enum { KVC_OP_ENCODE = 0, KVC_OP_DECODE = 1, KVC_OP_ATTEND = 2 };
+enum { KVC_OP_ENCODE = 0, KVC_OP_DECODE = 1, KVC_OP_ATTEND = 2, KVC_OP_REFIT_K = 3, KVC_OP_REFIT_V = 4 };
 
 /* Device workspace (bytes) that `op` needs for this layer; n_q = number of
  * query rows (attend only).  The caller passes a buffer of at least this size
@@ -227,6 +250,26 @@ KVC_API kvc_status kvc_attend_compressed_debiased(const kvc_layer_desc* desc, co
                                                   const void* V_self, int64_t n_self, float scale, void* O,
                                                   void* K_rec_opt, void* V_rec_opt, void* ws, size_t ws_bytes,
                                                   void* stream);
+
+/* Video-adapted block-DPLR refit ("CORAL-KV ...", Fig. 4: the low-rank
+ * factors stay fixed and the per-head block-diagonal terms are refitted for
+ * each filled cache block): for each head h,
+ *     block_h^T = (X_h^T X_h + ridge I)^{-1} X_h^T (Y_h - LR_h)
+ * over the desc->n_tokens tokens of the block, LR the fixed low-rank term
+ * (X_flat W^T) U^T of pred (rank may be 0).
+ *  tensor 0 (K): X0 = K^_{l-1} [T][H][D] (X1 ignored), Y = K_l, W/U = k_w/k_u;
+ *                block_out [H][D][D] (a k_block).
+ *  tensor 1 (V): X0 = K^_l, X1 = V^_{l-1} [T][H][D], Y = V_l, W/U = v_w/v_u;
+ *                block_out [H][D][2D] (a v_block).
+ * Since V's input is the reconstructed K of the same layer, a video-adapted
+ * layer refits K, encodes (for K^_l), refits V, and encodes again.  Computed in
+ * fp32 on the CUDA cores (Gram matrices, then a Cholesky solve per head) and
+ * written in the layer dtype; ridge >= 0 must make X_h^T X_h + ridge I
+ * positive definite.  KVC_PRED_XLAYER_DPLR only; ws of
+ * kvc_workspace_bytes(KVC_OP_REFIT_K / KVC_OP_REFIT_V, ...). */
+KVC_API kvc_status kvc_refit_block_diag(const kvc_layer_desc* desc, const kvc_predictor* pred, int tensor,
+                                        const void* X0, const void* X1, const void* Y, float ridge, void* block_out,
+                                        void* ws, size_t ws_bytes, void* stream);
 
 /* Pack n codes (uint8, each < 2^bits) into n*bits/8 bytes, LSB first;
  * n*bits must be a multiple of 128 (whole 16-byte words). */

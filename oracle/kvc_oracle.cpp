@@ -54,6 +54,9 @@
 //  R11 mixed-dimensional attention: V is clustered and coded like K; the
 //     output is sum_j m_j c^V_j + W^V_dec sum_t p_t coef^V_t, m_j the softmax
 //     mass of the tokens assigned to centre j.
+//  E1-E6 the H64 / EDEN-2 residual codec ("CORAL-KV ...", Fig. 5, Fig. 9,
+//     Table 9): see eden2_code_group below.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -141,6 +144,126 @@ void decode_row(const uint8_t* q, const double* s, const double* z, const double
                 double* xhat) {
   for (int i = 0; i < n; ++i) xhat[i] = round_to(pred[i] + dequant(q[i], s[i / group], z[i / group]), sfmt);
 }
+
+// ---------------------------------------------------------------- H64 / EDEN-2 residual codec
+// ["CORAL-KV ...", Fig. 5 (H_n transforms each non-overlapping group of n
+// residual channels; one shared scale per 64 values), Fig. 9 (16 EDEN-2
+// reconstruction points over pairs of H64-transformed residuals), Table 9 (the
+// H64 / EDEN-2 residual codec beside scalar INT2).]  Readings:
+//  E1 a group is 64 consecutive residual channels of a (token, head) row; it
+//     is transformed by the orthonormal Sylvester Walsh-Hadamard matrix,
+//     y_i = (1/8) sum_j (-1)^popcount(i & j) r_j.
+//  E2 the 32 pairs of a group are (y_2p, y_2p+1).
+//  E3 the 16 two-dimensional points are an input (the pages picture but do not
+//     print them).
+//  E4 the pairs are normalised by sigma = sqrt(mean_i y_i^2) and each takes the
+//     index of its nearest point (ties to the lowest index); the one stored
+//     scale is EDEN's unbiased one, S = |y|^2 / <y, c>, rounded to the
+//     parameter format (S = 0 when y = 0 or <y, c> <= 0).
+//  E5 index of pair p at bits [4p, 4p + 4) of the row, least significant first
+//     (4 bits per pair: the 2 bits per value of INT2).
+//  E6 the decoded residual is the inverse transform of S c (the transform is
+//     its own inverse), and x^ = round_state(pred + r^).
+
+inline double walsh(int i, int j) { return (__builtin_popcount((unsigned)(i & j)) & 1) ? -1.0 : 1.0; }
+
+// The transform of E1 (and its inverse, the same map).
+void hadamard64(const double* in, double* out) {
+  for (int i = 0; i < 64; ++i) {
+    double acc = 0.0;
+    for (int j = 0; j < 64; ++j) acc += walsh(i, j) * in[j];
+    out[i] = acc / 8.0;
+  }
+}
+
+// One group of 64 residuals r -> 32 indices, the stored scale, and the decoded
+// residual rh (E1-E6).  cb: 16 points [16][2].
+void eden2_code_group(const double* r, int pfmt, const double* cb, uint8_t* idx, double* S, double* rh) {
+  double y[64], yh[64];
+  hadamard64(r, y);
+  double sumsq = 0.0;
+  for (int i = 0; i < 64; ++i) sumsq += y[i] * y[i];
+  double dot = 0.0;
+  if (sumsq > 0.0) {
+    const double sigma = std::sqrt(sumsq / 64.0);
+    for (int p = 0; p < 32; ++p) {
+      const double u0 = y[2 * p] / sigma, u1 = y[2 * p + 1] / sigma;
+      int best = 0;
+      double bd = 0.0;
+      for (int k = 0; k < 16; ++k) {
+        const double d0 = u0 - cb[2 * k], d1 = u1 - cb[2 * k + 1];
+        const double d = d0 * d0 + d1 * d1;
+        if (k == 0 || d < bd) {
+          best = k;
+          bd = d;
+        }
+      }
+      idx[p] = (uint8_t)best;
+      dot += y[2 * p] * cb[2 * best] + y[2 * p + 1] * cb[2 * best + 1];
+    }
+  } else {
+    for (int p = 0; p < 32; ++p) idx[p] = 0;
+  }
+  *S = (sumsq > 0.0 && dot > 0.0) ? round_to(sumsq / dot, pfmt) : 0.0;
+  for (int p = 0; p < 32; ++p) {
+    yh[2 * p] = *S * cb[2 * idx[p]];
+    yh[2 * p + 1] = *S * cb[2 * idx[p] + 1];
+  }
+  hadamard64(yh, rh);
+}
+
+void eden2_decode_group(const uint8_t* idx, double S, const double* cb, double* rh) {
+  double yh[64];
+  for (int p = 0; p < 32; ++p) {
+    yh[2 * p] = S * cb[2 * idx[p]];
+    yh[2 * p + 1] = S * cb[2 * idx[p] + 1];
+  }
+  hadamard64(yh, rh);
+}
+
+// A row of n values coded against its prediction with H64 / EDEN-2: q receives
+// n / 2 pair indices, s the n / 64 scales (z is unused and set to 0).
+void eden2_code_row(const double* x, const double* pred, int n, int pfmt, int sfmt, const double* cb, uint8_t* q,
+                    double* s, double* z, double* xhat) {
+  double r[64], rh[64];
+  for (int g = 0; g < n / 64; ++g) {
+    for (int i = 0; i < 64; ++i) r[i] = x[g * 64 + i] - pred[g * 64 + i];
+    eden2_code_group(r, pfmt, cb, q + g * 32, s + g, rh);
+    z[g] = 0.0;
+    for (int i = 0; i < 64; ++i) xhat[g * 64 + i] = round_to(pred[g * 64 + i] + rh[i], sfmt);
+  }
+}
+
+void eden2_decode_row(const uint8_t* q, const double* s, const double* pred, int n, int sfmt, const double* cb,
+                      double* xhat) {
+  double rh[64];
+  for (int g = 0; g < n / 64; ++g) {
+    eden2_decode_group(q + g * 32, s[g], cb, rh);
+    for (int i = 0; i < 64; ++i) xhat[g * 64 + i] = round_to(pred[g * 64 + i] + rh[i], sfmt);
+  }
+}
+
+// The residual codec of a layer: cb == NULL is the scalar group quantizer
+// (R1-R4), otherwise H64 / EDEN-2 with codebook cb.  Codes are per element
+// (scalar) or per pair (EDEN-2): `qn` entries per row of n values.
+struct RowCoder {
+  int bits, group, pfmt, sfmt;
+  const double* cb;
+  int qn(int n) const { return cb ? n / 2 : n; }
+  int sn(int n) const { return cb ? n / 64 : n / group; }
+  void code(const double* x, const double* pred, int n, uint8_t* q, double* s, double* z, double* xhat) const {
+    if (cb)
+      eden2_code_row(x, pred, n, pfmt, sfmt, cb, q, s, z, xhat);
+    else
+      code_row(x, pred, n, bits, group, pfmt, sfmt, q, s, z, xhat);
+  }
+  void decode(const uint8_t* q, const double* s, const double* z, const double* pred, int n, double* xhat) const {
+    if (cb)
+      eden2_decode_row(q, s, pred, n, sfmt, cb, xhat);
+    else
+      decode_row(q, s, z, pred, n, group, sfmt, xhat);
+  }
+};
 
 // ---------------------------------------------------------------- cross-layer block-DPLR prediction
 // [CORAL abstract, Fig. 3]
@@ -301,28 +424,31 @@ void kvo_predict_xlayer_v(int64_t T, int H, int D, int r, const double* Kh, cons
 }
 
 // ---------------------------------------------------------------- one layer, null predictor (anchor)
-// [CORAL Fig. 8; TEMPO appendix Table 7]: every row coded against 0.
+// [CORAL Fig. 8; TEMPO appendix Table 7]: every row coded against 0.  cb:
+// NULL for the scalar group quantizer, else the 16 EDEN-2 points ([16][2]);
+// q then holds D / 2 pair indices per row and s D / 64 scales.
 
 void kvo_encode_none(int64_t T, int H, int D, int bits, int group, int pfmt, int sfmt, const double* X, uint8_t* q,
-                     double* s, double* z, double* xhat) {
-  const int ng = D / group;
+                     double* s, double* z, double* xhat, const double* cb) {
+  const RowCoder rc{bits, group, pfmt, sfmt, cb};
+  const int qn = rc.qn(D), sn = rc.sn(D);
   std::vector<double> zero(D, 0.0);
   for (int64_t t = 0; t < T; ++t)
     for (int h = 0; h < H; ++h) {
       const int64_t row = t * H + h;
-      code_row(X + row * D, zero.data(), D, bits, group, pfmt, sfmt, q + row * D, s + row * ng, z + row * ng,
-               xhat + row * D);
+      rc.code(X + row * D, zero.data(), D, q + row * qn, s + row * sn, z + row * sn, xhat + row * D);
     }
 }
 
 void kvo_decode_none(int64_t T, int H, int D, int group, int sfmt, const uint8_t* q, const double* s, const double* z,
-                     double* xhat) {
-  const int ng = D / group;
+                     double* xhat, const double* cb) {
+  const RowCoder rc{0, group, 0, sfmt, cb};
+  const int qn = rc.qn(D), sn = rc.sn(D);
   std::vector<double> zero(D, 0.0);
   for (int64_t t = 0; t < T; ++t)
     for (int h = 0; h < H; ++h) {
       const int64_t row = t * H + h;
-      decode_row(q + row * D, s + row * ng, z + row * ng, zero.data(), D, group, sfmt, xhat + row * D);
+      rc.decode(q + row * qn, s + row * sn, z + row * sn, zero.data(), D, xhat + row * D);
     }
 }
 
@@ -331,27 +457,28 @@ void kvo_decode_none(int64_t T, int H, int D, int group, int sfmt, const uint8_t
 // then V, whose prediction reads the reconstructed K_l.  Tokens do not
 // interact.  K, V, Ks, Vs, kh, vh: [T][H][D]; bk [H][D][D], wk [r][C],
 // uk [C][r], bv [H][D][2D], wv [r][2C], uv [C][r].  `pk`, `pv` (optional,
-// may be NULL) receive the predictions.
+// may be NULL) receive the predictions.  cb as for kvo_encode_none.
 
 void kvo_encode_xlayer(int64_t T, int H, int D, int r, int bits, int group, int pfmt, int sfmt, const double* K,
                        const double* V, const double* Ks, const double* Vs, const double* bk, const double* wk,
                        const double* uk, const double* bv, const double* wv, const double* uv, uint8_t* qk, double* sk,
                        double* zk, uint8_t* qv, double* sv, double* zv, double* kh, double* vh, double* pk,
-                       double* pv) {
-  const int C = H * D, ng = D / group;
+                       double* pv, const double* cb) {
+  const RowCoder rc{bits, group, pfmt, sfmt, cb};
+  const int C = H * D, qn = rc.qn(D), sn = rc.sn(D);
   std::vector<double> pred(C);
   for (int64_t t = 0; t < T; ++t) {
-    const int64_t o = t * C, og = t * H * ng;
+    const int64_t o = t * C, oq = t * H * qn, og = t * H * sn;
     predict_k_token(H, D, r, Ks + o, bk, wk, uk, pred.data());
     if (pk) std::memcpy(pk + o, pred.data(), sizeof(double) * C);
     for (int h = 0; h < H; ++h)
-      code_row(K + o + h * D, pred.data() + h * D, D, bits, group, pfmt, sfmt, qk + o + h * D, sk + og + h * ng,
-               zk + og + h * ng, kh + o + h * D);
+      rc.code(K + o + h * D, pred.data() + h * D, D, qk + oq + h * qn, sk + og + h * sn, zk + og + h * sn,
+              kh + o + h * D);
     predict_v_token(H, D, r, kh + o, Vs + o, bv, wv, uv, pred.data());
     if (pv) std::memcpy(pv + o, pred.data(), sizeof(double) * C);
     for (int h = 0; h < H; ++h)
-      code_row(V + o + h * D, pred.data() + h * D, D, bits, group, pfmt, sfmt, qv + o + h * D, sv + og + h * ng,
-               zv + og + h * ng, vh + o + h * D);
+      rc.code(V + o + h * D, pred.data() + h * D, D, qv + oq + h * qn, sv + og + h * sn, zv + og + h * sn,
+              vh + o + h * D);
   }
 }
 
@@ -359,20 +486,24 @@ void kvo_encode_xlayer(int64_t T, int H, int D, int r, int bits, int group, int 
 void kvo_decode_xlayer(int64_t T, int H, int D, int r, int group, int sfmt, const uint8_t* qk, const double* sk,
                        const double* zk, const uint8_t* qv, const double* sv, const double* zv, const double* Ks,
                        const double* Vs, const double* bk, const double* wk, const double* uk, const double* bv,
-                       const double* wv, const double* uv, double* kh, double* vh) {
-  const int C = H * D, ng = D / group;
+                       const double* wv, const double* uv, double* kh, double* vh, const double* cb) {
+  const RowCoder rc{0, group, 0, sfmt, cb};
+  const int C = H * D, qn = rc.qn(D), sn = rc.sn(D);
   std::vector<double> pred(C);
   for (int64_t t = 0; t < T; ++t) {
-    const int64_t o = t * C, og = t * H * ng;
+    const int64_t o = t * C, oq = t * H * qn, og = t * H * sn;
     predict_k_token(H, D, r, Ks + o, bk, wk, uk, pred.data());
     for (int h = 0; h < H; ++h)
-      decode_row(qk + o + h * D, sk + og + h * ng, zk + og + h * ng, pred.data() + h * D, D, group, sfmt,
-                 kh + o + h * D);
+      rc.decode(qk + oq + h * qn, sk + og + h * sn, zk + og + h * sn, pred.data() + h * D, D, kh + o + h * D);
     predict_v_token(H, D, r, kh + o, Vs + o, bv, wv, uv, pred.data());
     for (int h = 0; h < H; ++h)
-      decode_row(qv + o + h * D, sv + og + h * ng, zv + og + h * ng, pred.data() + h * D, D, group, sfmt,
-                 vh + o + h * D);
+      rc.decode(qv + oq + h * qn, sv + og + h * sn, zv + og + h * sn, pred.data() + h * D, D, vh + o + h * D);
   }
+}
+
+// The H64 / EDEN-2 transform of E1 on rows of 64 values (exported for the pins).
+void kvo_hadamard64(const double* in, int64_t rows, double* out) {
+  for (int64_t t = 0; t < rows; ++t) hadamard64(in + t * 64, out + t * 64);
 }
 
 // ---------------------------------------------------------------- one temporal layer
@@ -615,6 +746,81 @@ void kvo_mixed_attention(int64_t nq, int64_t T, int H, int D, int m, int nc, dou
     }
 }
 
+// ---------------------------------------------------------------- video-adapted block-DPLR refit
+// ["CORAL-KV ...", Fig. 4: the video-adapted block-DPLR keeps its low-rank
+// factors fixed and refits the block-diagonal terms for each filled cache
+// block.]  Reading V1: the refit is a ridge least-squares fit of each head's
+// block on the block's tokens, against the target left after the fixed
+// low-rank term:
+//   B_h^T = (X_h^T X_h + ridge I)^{-1} X_h^T (Y_h - LR_h),
+// X_h the head's predictor input (K: K^_{l-1,h}; V: [K^_{l,h} | V^_{l-1,h}]),
+// Y_h the clean values, LR = (X_flat W^T) U^T the fixed low-rank prediction.
+// Solved by a Cholesky factorisation G = L L^T and two triangular solves.
+// X0, X1 [T][H][D] (X1 NULL for K); Y [T][H][D]; w [r][Cin], u [C][r];
+// block [H][D][din] with din = D (K) or 2 D (V).
+void kvo_refit_block_diag(int64_t T, int H, int D, int r, const double* X0, const double* X1, const double* Y,
+                          const double* w, const double* u, double ridge, double* block) {
+  const int C = H * D, din = X1 ? 2 * D : D, cin = X1 ? 2 * C : C;
+  // the fixed low-rank prediction of every token, all heads
+  std::vector<double> lat(r > 0 ? r : 1), lr((size_t)T * C, 0.0);
+  for (int64_t t = 0; t < T; ++t) {
+    for (int j = 0; j < r; ++j) {
+      double acc = 0.0;
+      for (int c = 0; c < C; ++c) acc += X0[t * C + c] * w[(int64_t)j * cin + c];
+      if (X1)
+        for (int c = 0; c < C; ++c) acc += X1[t * C + c] * w[(int64_t)j * cin + C + c];
+      lat[j] = acc;
+    }
+    for (int o = 0; o < C; ++o) {
+      double acc = 0.0;
+      for (int j = 0; j < r; ++j) acc += lat[j] * u[(int64_t)o * r + j];
+      lr[t * C + o] = acc;
+    }
+  }
+  std::vector<double> G((size_t)din * din), Rhs((size_t)din * D), x(din), L((size_t)din * din);
+  for (int h = 0; h < H; ++h) {
+    std::fill(G.begin(), G.end(), 0.0);
+    std::fill(Rhs.begin(), Rhs.end(), 0.0);
+    for (int64_t t = 0; t < T; ++t) {
+      for (int i = 0; i < D; ++i) x[i] = X0[t * C + h * D + i];
+      if (X1)
+        for (int i = 0; i < D; ++i) x[D + i] = X1[t * C + h * D + i];
+      for (int i = 0; i < din; ++i) {
+        for (int j = 0; j < din; ++j) G[(size_t)i * din + j] += x[i] * x[j];
+        for (int o = 0; o < D; ++o) Rhs[(size_t)i * D + o] += x[i] * (Y[t * C + h * D + o] - lr[t * C + h * D + o]);
+      }
+    }
+    for (int i = 0; i < din; ++i) G[(size_t)i * din + i] += ridge;
+    // Cholesky: G = L L^T (lower triangular L)
+    for (int j = 0; j < din; ++j) {
+      double d = G[(size_t)j * din + j];
+      for (int k = 0; k < j; ++k) d -= L[(size_t)j * din + k] * L[(size_t)j * din + k];
+      const double ljj = std::sqrt(d);
+      L[(size_t)j * din + j] = ljj;
+      for (int i = j + 1; i < din; ++i) {
+        double v = G[(size_t)i * din + j];
+        for (int k = 0; k < j; ++k) v -= L[(size_t)i * din + k] * L[(size_t)j * din + k];
+        L[(size_t)i * din + j] = v / ljj;
+      }
+    }
+    // for each output channel o: L z = rhs_o, then L^T b = z; block[h][o][i] = b_i
+    std::vector<double> z(din), b(din);
+    for (int o = 0; o < D; ++o) {
+      for (int i = 0; i < din; ++i) {
+        double v = Rhs[(size_t)i * D + o];
+        for (int k = 0; k < i; ++k) v -= L[(size_t)i * din + k] * z[k];
+        z[i] = v / L[(size_t)i * din + i];
+      }
+      for (int i = din - 1; i >= 0; --i) {
+        double v = z[i];
+        for (int k = i + 1; k < din; ++k) v -= L[(size_t)k * din + i] * b[k];
+        b[i] = v / L[(size_t)i * din + i];
+      }
+      for (int i = 0; i < din; ++i) block[((int64_t)h * D + o) * din + i] = b[i];
+    }
+  }
+}
+
 // ---------------------------------------------------------------- storage accounting
 // [TEMPO Tables 1-3 (5.33x), Table 8 (3.20x), appendix Table 7]: bytes of
 // codes + (scale, zero) pairs (+ one-byte centre indices) of one layer's K and
@@ -623,6 +829,8 @@ void kvo_mixed_attention(int64_t nq, int64_t T, int H, int D, int m, int nc, dou
 int64_t kvo_codes_bytes(int kind, int64_t T, int H, int D, int bits, int group, int param_bytes, int F,
                         int anchor_bits, int m) {
   const int64_t pair = 2 * (int64_t)param_bytes;
+  // H64 / EDEN-2 (kind 3): a 4-bit index per pair of values and one scale per 64 values
+  if (kind == 3) return 2 * T * H * ((int64_t)(D / 2) * 4 / 8 + (D / 64) * (int64_t)param_bytes);
   if (kind == 2) return 2 * T * ((int64_t)m * bits / 8 + (m / group) * pair + 1);
   const int64_t row_params = (D / group) * pair;
   if (kind == 1) {

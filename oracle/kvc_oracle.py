@@ -111,6 +111,7 @@ class Desc:
     param: str = "f16"  # dtype of the stored (scale, zero) pair ("f16" | "f32")
     frame_tokens: int = 0  # temporal codec only
     anchor_bits: int = 4  # temporal codec: bits of frame 0
+    codec: str = "rtn"  # residual codec: "rtn" (scalar group quantizer) | "eden2" (H64 / EDEN-2)
 
     @property
     def channels(self) -> int:
@@ -206,6 +207,8 @@ def codes_bytes(desc: Desc, kind: str = "none", code_dim: int = 0) -> int:
     """
     T, H, D = desc.n_tokens, desc.n_heads, desc.head_dim
     pb = 2 * _PARAM_BYTES[desc.param]
+    if desc.codec == "eden2":  # a 4-bit index per pair of values, one scale per 64 values
+        return 2 * T * H * ((D // 2) * 4 // 8 + (D // 64) * _PARAM_BYTES[desc.param])
     if kind == "cluster":
         per_tok = code_dim * desc.bits // 8 + (code_dim // desc.group) * pb + 1
         return 2 * T * per_tok
@@ -221,20 +224,78 @@ def codes_bytes(desc: Desc, kind: str = "none", code_dim: int = 0) -> int:
 
 
 # --------------------------------------------------------------------------
+# H64 / EDEN-2 residual codec [CORAL Fig. 5, Fig. 9, Table 9]
+# --------------------------------------------------------------------------
+#
+# E1 groups of 64 consecutive residual channels are transformed by the
+#    orthonormal Sylvester Walsh-Hadamard matrix H64 / 8;
+# E2 the 32 pairs of a group are (y_2p, y_2p+1);
+# E3 the 16 two-dimensional points are an input (pictured, not printed);
+# E4 pairs normalised by sigma = sqrt(mean y^2) take the nearest point's index
+#    (ties to the lowest); the stored scale is EDEN's S = |y|^2 / <y, c>,
+#    rounded to the parameter dtype (0 when y = 0 or <y, c> <= 0);
+# E5 pair p's 4-bit index at bits [4p, 4p+4) of the row;
+# E6 the decoded residual is H64 / 8 applied to S c.
+
+
+def hadamard_matrix(n: int = 64) -> np.ndarray:
+    """Sylvester's construction H_2n = [[H, H], [H, -H]] from H_1 = [1]."""
+    Hm = np.ones((1, 1))
+    while Hm.shape[0] < n:
+        Hm = np.block([[Hm, Hm], [Hm, -Hm]])
+    return Hm
+
+
+def eden2_code(r, param: str, codebook):
+    """r [..., 64] -> (indices [..., 32], scale [...], decoded residual [..., 64])."""
+    Hn = hadamard_matrix(64) / 8.0
+    cb = np.asarray(codebook, np.float64).reshape(16, 2)
+    y = np.asarray(r, np.float64) @ Hn.T
+    sumsq = (y * y).sum(-1)
+    pairs = y.reshape(y.shape[:-1] + (32, 2))
+    sigma = np.sqrt(sumsq / 64.0)
+    u = pairs / np.where(sigma > 0, sigma, 1.0)[..., None, None]
+    d = ((u[..., :, None, :] - cb) ** 2).sum(-1)  # [..., 32, 16]
+    idx = np.where((sumsq > 0)[..., None], d.argmin(-1), 0)
+    dot = (pairs * cb[idx]).sum((-1, -2))
+    S = np.where((sumsq > 0) & (dot > 0), round_to(sumsq / np.where(dot > 0, dot, 1.0), param), 0.0)
+    return idx.astype(np.uint8), S, eden2_decode(idx, S, cb)
+
+
+def eden2_decode(idx, S, codebook) -> np.ndarray:
+    Hn = hadamard_matrix(64) / 8.0
+    cb = np.asarray(codebook, np.float64).reshape(16, 2)
+    yh = np.asarray(S, np.float64)[..., None, None] * cb[np.asarray(idx, np.int64)]
+    return yh.reshape(yh.shape[:-2] + (64,)) @ Hn.T
+
+
+# --------------------------------------------------------------------------
 # One coded tensor: residual -> codes -> reconstruction (closed loop)
 # --------------------------------------------------------------------------
 
 
-def code_residual(x, pred, bits: int, group: int, param: str, state: str):
+def code_residual(x, pred, bits: int, group: int, param: str, state: str, codec: str = "rtn", codebook=None):
     """r = x - pred is quantized; the reconstruction pred + deq(r) is rounded to
-    the state dtype (readings R1-R5).  Returns (q, s, z, x_hat)."""
+    the state dtype (readings R1-R5).  Returns (q, s, z, x_hat); with the
+    H64 / EDEN-2 codec q holds pair indices and s the per-64 scales."""
     r = np.asarray(x, dtype=np.float64) - pred
+    if codec == "eden2":
+        n = r.shape[-1]
+        rg = r.reshape(r.shape[:-1] + (n // 64, 64))
+        idx, S, rh = eden2_code(rg, param, codebook)
+        q = idx.reshape(r.shape[:-1] + (n // 2,))
+        return q, S, np.zeros_like(S), round_to(pred + rh.reshape(r.shape), state)
     q, s, z = quantize_groups(r, bits, group, param)
     x_hat = round_to(pred + dequantize_groups(q, s, z, group), state)
     return q, s, z, x_hat
 
 
-def decode_residual(q, s, z, pred, group: int, state: str) -> np.ndarray:
+def decode_residual(q, s, z, pred, group: int, state: str, codec: str = "rtn", codebook=None) -> np.ndarray:
+    if codec == "eden2":
+        q = np.asarray(q)
+        idx = q.reshape(q.shape[:-1] + (q.shape[-1] // 32, 32))
+        rh = eden2_decode(idx, s, codebook)
+        return round_to(pred + rh.reshape(np.shape(pred)), state)
     return round_to(pred + dequantize_groups(q, s, z, group), state)
 
 
@@ -287,25 +348,26 @@ class Coded:
     assign: np.ndarray | None = None  # clustered codec: centre index per token
 
 
-def encode_layer_none(desc: Desc, K, V):
+def encode_layer_none(desc: Desc, K, V, codebook=None):
     """Anchor / RTN: the null predictor, every row coded directly
     [CORAL Fig. 8 INT4 anchor]."""
-    zero = np.zeros(K.shape)
+    zero = np.zeros(np.shape(K))
     out = []
     for x in (K, V):
-        q, s, z, xh = code_residual(x, zero, desc.bits, desc.group, desc.param, desc.state)
+        q, s, z, xh = code_residual(x, zero, desc.bits, desc.group, desc.param, desc.state, desc.codec, codebook)
         out.append((Coded(q, s, z), xh))
     return out[0][0], out[1][0], out[0][1], out[1][1]
 
 
-def decode_layer_none(desc: Desc, ck: Coded, cv: Coded):
-    zero = np.zeros(ck.q.shape)
-    K = decode_residual(ck.q, ck.s, ck.z, zero, desc.group, desc.state)
-    V = decode_residual(cv.q, cv.s, cv.z, zero, desc.group, desc.state)
+def decode_layer_none(desc: Desc, ck: Coded, cv: Coded, codebook=None):
+    T, H = ck.q.shape[:2]
+    zero = np.zeros((T, H, desc.head_dim))
+    K = decode_residual(ck.q, ck.s, ck.z, zero, desc.group, desc.state, desc.codec, codebook)
+    V = decode_residual(cv.q, cv.s, cv.z, zero, desc.group, desc.state, desc.codec, codebook)
     return K, V
 
 
-def encode_layer_xlayer(desc: Desc, w: dict, K, V, K_src, V_src):
+def encode_layer_xlayer(desc: Desc, w: dict, K, V, K_src, V_src, codebook=None):
     """One Coral layer l>0: K first (its prediction needs only layer l-1), then V,
     whose prediction needs the reconstructed K^_l [CORAL Fig. 3].
 
@@ -313,18 +375,18 @@ def encode_layer_xlayer(desc: Desc, w: dict, K, V, K_src, V_src):
     Returns (coded K, coded V, K^_l, V^_l).
     """
     pk = xlayer_predict_k(K_src, w["k_block"], w["k_w"], w["k_u"])
-    qk, sk, zk, K_hat = code_residual(K, pk, desc.bits, desc.group, desc.param, desc.state)
+    qk, sk, zk, K_hat = code_residual(K, pk, desc.bits, desc.group, desc.param, desc.state, desc.codec, codebook)
     pv = xlayer_predict_v(K_hat, V_src, w["v_block"], w["v_w"], w["v_u"])
-    qv, sv, zv, V_hat = code_residual(V, pv, desc.bits, desc.group, desc.param, desc.state)
+    qv, sv, zv, V_hat = code_residual(V, pv, desc.bits, desc.group, desc.param, desc.state, desc.codec, codebook)
     return Coded(qk, sk, zk), Coded(qv, sv, zv), K_hat, V_hat
 
 
-def decode_layer_xlayer(desc: Desc, w: dict, ck: Coded, cv: Coded, K_src, V_src):
+def decode_layer_xlayer(desc: Desc, w: dict, ck: Coded, cv: Coded, K_src, V_src, codebook=None):
     """Replays the encoder's prediction chain from the codes."""
     pk = xlayer_predict_k(K_src, w["k_block"], w["k_w"], w["k_u"])
-    K_hat = decode_residual(ck.q, ck.s, ck.z, pk, desc.group, desc.state)
+    K_hat = decode_residual(ck.q, ck.s, ck.z, pk, desc.group, desc.state, desc.codec, codebook)
     pv = xlayer_predict_v(K_hat, V_src, w["v_block"], w["v_w"], w["v_u"])
-    V_hat = decode_residual(cv.q, cv.s, cv.z, pv, desc.group, desc.state)
+    V_hat = decode_residual(cv.q, cv.s, cv.z, pv, desc.group, desc.state, desc.codec, codebook)
     return K_hat, V_hat
 
 
@@ -543,6 +605,31 @@ def attend_compressed_xlayer(desc: Desc, w: dict, Q, ck: Coded, cv: Coded, K_src
     else:
         K_all, V_all = K_hist, V_hist
     return attention(Q, K_all, V_all, scale)
+
+
+# --------------------------------------------------------------------------
+# Video-adapted block-DPLR refit [CORAL Fig. 4]
+# --------------------------------------------------------------------------
+
+
+def refit_block_diag(X0, X1, Y, w_lr, u_lr, ridge: float) -> np.ndarray:
+    """Each head's block refitted on a filled cache block with the low-rank
+    factors fixed (reading V1): B_h^T = (X_h^T X_h + ridge I)^-1 X_h^T (Y_h - LR_h)
+    with X_h = X0_h (K) or [X0_h | X1_h] (V) and LR the fixed low-rank term."""
+    X0 = np.asarray(X0, np.float64)
+    T, H, D = X0.shape
+    flat = X0.reshape(T, H * D) if X1 is None else np.concatenate(
+        [X0.reshape(T, H * D), np.asarray(X1, np.float64).reshape(T, H * D)], axis=1)
+    lr = _lowrank(flat, None if w_lr is None else np.asarray(w_lr, np.float64),
+                  None if u_lr is None else np.asarray(u_lr, np.float64), T, H, D)
+    R = np.asarray(Y, np.float64) - lr
+    Xh = X0 if X1 is None else np.concatenate([X0, np.asarray(X1, np.float64)], axis=-1)  # [T,H,din]
+    din = Xh.shape[-1]
+    out = np.empty((H, D, din))
+    for h in range(H):
+        G = Xh[:, h, :].T @ Xh[:, h, :] + ridge * np.eye(din)
+        out[h] = np.linalg.solve(G, Xh[:, h, :].T @ R[:, h, :]).T
+    return out
 
 
 def rel_l2(a, b) -> float:

@@ -157,6 +157,8 @@ def unpack_codes(packed, bits: int, n: int) -> np.ndarray:
 
 def codes_bytes(desc: Desc, kind: str = "none", code_dim: int = 0) -> int:
     k = {"none": 0, "xlayer": 0, "temporal": 1, "cluster": 2}[kind]
+    if getattr(desc, "codec", "rtn") == "eden2":
+        k = 3
     return int(lib().kvo_codes_bytes(k, _i(desc.n_tokens), desc.n_heads, desc.head_dim, desc.bits, desc.group,
                                      _PARAM_BYTES[desc.param], desc.frame_tokens, desc.anchor_bits, code_dim))
 
@@ -164,37 +166,61 @@ def codes_bytes(desc: Desc, kind: str = "none", code_dim: int = 0) -> int:
 # ---------------------------------------------------------------- layers
 
 
-def _empty_coded(T, H, D, group):
+def _empty_coded(T, H, D, group, eden=False):
+    """Codes of a [T, H, D] tensor: per element (scalar quantizer) or per pair
+    (H64 / EDEN-2: D / 2 indices, D / 64 scales, zeros unused)."""
+    if eden:
+        return (np.empty((T, H, D // 2), np.uint8), np.empty((T, H, D // 64)), np.zeros((T, H, D // 64)))
     return (np.empty((T, H, D), np.uint8), np.empty((T, H, D // group)), np.empty((T, H, D // group)))
 
 
-def encode_layer_none(desc: Desc, K, V, threads=None):
+def _cb(desc: Desc, codebook):
+    """The EDEN-2 points as a contiguous float64 [16, 2] array (None: scalar codec)."""
+    if getattr(desc, "codec", "rtn") != "eden2":
+        return None
+    assert codebook is not None, "the H64 / EDEN-2 codec needs its 16 points"
+    cb = _f64(codebook).reshape(16, 2)
+    return cb
+
+
+def encode_layer_none(desc: Desc, K, V, threads=None, codebook=None):
     """Anchor: both tensors coded against prediction 0 [CORAL Fig. 8]."""
+    cb = _cb(desc, codebook)
     out = []
     for X in (K, V):
         X = _f64(X)
         T, H, D = X.shape
-        q, s, z = _empty_coded(T, H, D, desc.group)
+        q, s, z = _empty_coded(T, H, D, desc.group, cb is not None)
         xh = np.empty_like(X)
 
         def run(a, b):
             lib().kvo_encode_none(_i(b - a), H, D, desc.bits, desc.group, _FMT[desc.param], _FMT[desc.state],
-                                  _p(X[a:b]), _p(q[a:b]), _p(s[a:b]), _p(z[a:b]), _p(xh[a:b]))
+                                  _p(X[a:b]), _p(q[a:b]), _p(s[a:b]), _p(z[a:b]), _p(xh[a:b]), _p(cb))
 
         _drive(_runs(T, threads, 64), run)
         out.append((Coded(q, s, z), xh))
     return out[0][0], out[1][0], out[0][1], out[1][1]
 
 
-def decode_layer_none(desc: Desc, ck: Coded, cv: Coded, threads=None):
+def decode_layer_none(desc: Desc, ck: Coded, cv: Coded, threads=None, codebook=None):
+    cb = _cb(desc, codebook)
     res = []
     for c in (ck, cv):
         q, s, z = np.ascontiguousarray(c.q), _f64(c.s), _f64(c.z)
-        T, H, D = q.shape
+        T, H = q.shape[:2]
+        D = desc.head_dim
         xh = np.empty((T, H, D))
-        lib().kvo_decode_none(_i(T), H, D, desc.group, _FMT[desc.state], _p(q), _p(s), _p(z), _p(xh))
+        lib().kvo_decode_none(_i(T), H, D, desc.group, _FMT[desc.state], _p(q), _p(s), _p(z), _p(xh), _p(cb))
         res.append(xh)
     return res[0], res[1]
+
+
+def hadamard64(x) -> np.ndarray:
+    """The orthonormal Sylvester Walsh-Hadamard transform of rows of 64 values."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    lib().kvo_hadamard64(_p(x), _i(x.size // 64), _p(out))
+    return out
 
 
 def _xw(w: dict):
@@ -225,14 +251,16 @@ def xlayer_predict_v(K_rec, V_src, v_block, v_w, v_u) -> np.ndarray:
     return out
 
 
-def encode_layer_xlayer(desc: Desc, w: dict, K, V, K_src, V_src, threads=None, with_pred: bool = False):
+def encode_layer_xlayer(desc: Desc, w: dict, K, V, K_src, V_src, threads=None, with_pred: bool = False,
+                        codebook=None):
     """One Coral layer l > 0 [CORAL Fig. 3]; returns (coded K, coded V, K^_l,
     V^_l) and, with `with_pred`, the two predictions as well."""
     K, V, Ks, Vs = _f64(K), _f64(V), _f64(K_src), _f64(V_src)
     T, H, D = K.shape
+    cb = _cb(desc, codebook)
     r, bk, wk, uk, bv, wv, uv = _xw(w)
-    qk, sk, zk = _empty_coded(T, H, D, desc.group)
-    qv, sv, zv = _empty_coded(T, H, D, desc.group)
+    qk, sk, zk = _empty_coded(T, H, D, desc.group, cb is not None)
+    qv, sv, zv = _empty_coded(T, H, D, desc.group, cb is not None)
     kh, vh = np.empty_like(K), np.empty_like(V)
     pk = np.empty_like(K) if with_pred else None
     pv = np.empty_like(V) if with_pred else None
@@ -242,16 +270,17 @@ def encode_layer_xlayer(desc: Desc, w: dict, K, V, K_src, V_src, threads=None, w
                                 _p(K[a:b]), _p(V[a:b]), _p(Ks[a:b]), _p(Vs[a:b]), _p(bk), _p(wk), _p(uk), _p(bv),
                                 _p(wv), _p(uv), _p(qk[a:b]), _p(sk[a:b]), _p(zk[a:b]), _p(qv[a:b]), _p(sv[a:b]),
                                 _p(zv[a:b]), _p(kh[a:b]), _p(vh[a:b]), _p(pk[a:b]) if with_pred else None,
-                                _p(pv[a:b]) if with_pred else None)
+                                _p(pv[a:b]) if with_pred else None, _p(cb))
 
     _drive(_runs(T, threads, 16), run)
     out = (Coded(qk, sk, zk), Coded(qv, sv, zv), kh, vh)
     return out + (pk, pv) if with_pred else out
 
 
-def decode_layer_xlayer(desc: Desc, w: dict, ck: Coded, cv: Coded, K_src, V_src, threads=None):
+def decode_layer_xlayer(desc: Desc, w: dict, ck: Coded, cv: Coded, K_src, V_src, threads=None, codebook=None):
     Ks, Vs = _f64(K_src), _f64(V_src)
     T, H, D = Ks.shape
+    cb = _cb(desc, codebook)
     r, bk, wk, uk, bv, wv, uv = _xw(w)
     qk, sk, zk = np.ascontiguousarray(ck.q), _f64(ck.s), _f64(ck.z)
     qv, sv, zv = np.ascontiguousarray(cv.q), _f64(cv.s), _f64(cv.z)
@@ -260,7 +289,7 @@ def decode_layer_xlayer(desc: Desc, w: dict, ck: Coded, cv: Coded, K_src, V_src,
     def run(a, b):
         lib().kvo_decode_xlayer(_i(b - a), H, D, r, desc.group, _FMT[desc.state], _p(qk[a:b]), _p(sk[a:b]),
                                 _p(zk[a:b]), _p(qv[a:b]), _p(sv[a:b]), _p(zv[a:b]), _p(Ks[a:b]), _p(Vs[a:b]), _p(bk),
-                                _p(wk), _p(uk), _p(bv), _p(wv), _p(uv), _p(kh[a:b]), _p(vh[a:b]))
+                                _p(wk), _p(uk), _p(bv), _p(wv), _p(uv), _p(kh[a:b]), _p(vh[a:b]), _p(cb))
 
     _drive(_runs(T, threads, 16), run)
     return kh, vh
@@ -395,9 +424,9 @@ def attention_corrected(Q, K, V, scale: float, n_hist: int, s_hist, group: int, 
 
 
 def attend_compressed_xlayer(desc: Desc, w: dict, Q, ck: Coded, cv: Coded, K_src, V_src, K_self, V_self,
-                             scale: float, threads=None, jensen: bool = False) -> np.ndarray:
+                             scale: float, threads=None, jensen: bool = False, codebook=None) -> np.ndarray:
     """Softmax attention of Q over [decoded history ; uncompressed chunk]."""
-    K_hist, V_hist = decode_layer_xlayer(desc, w, ck, cv, K_src, V_src, threads)
+    K_hist, V_hist = decode_layer_xlayer(desc, w, ck, cv, K_src, V_src, threads, codebook)
     T = K_hist.shape[0]
     if K_self is not None and len(K_self):
         K_hist = np.concatenate([K_hist, _f64(K_self)], axis=0)
@@ -427,3 +456,22 @@ def mixed_attention(Q, ck: Coded, cent_k, dec_k, cv: Coded, cent_v, dec_v, desc:
 
     _drive(_runs(nq, threads), run)
     return O
+
+
+# ---------------------------------------------------------------- video-adapted refit
+
+
+def refit_block_diag(X0, X1, Y, w_lr, u_lr, ridge: float) -> np.ndarray:
+    """Ridge least-squares refit of every head's block-diagonal map with the
+    low-rank factors fixed ("CORAL-KV ...", Fig. 4, video-adapted block-DPLR):
+    returns block [H, D, din] (din = D for K, 2 D for V with X1 given)."""
+    X0, Y = _f64(X0), _f64(Y)
+    T, H, D = X0.shape
+    X1 = None if X1 is None else _f64(X1)
+    r = int(np.shape(w_lr)[0]) if w_lr is not None else 0
+    din = 2 * D if X1 is not None else D
+    w = _f64(w_lr) if r else np.zeros(1)
+    u = _f64(u_lr) if r else np.zeros(1)
+    out = np.empty((H, D, din))
+    lib().kvo_refit_block_diag(_i(T), H, D, r, _p(X0), _p(X1), _p(Y), _p(w), _p(u), ctypes.c_double(ridge), _p(out))
+    return out

@@ -804,3 +804,141 @@ def test_debiased_attention_cross_layer(n_q, n_self, T, rank, group):
     U.OBSERVED.append({"check": f"debiased attention T={T}", "rel_l2": err, "correction_moves": moved})
     assert err <= U.ATT_TOL[bf], err
     assert err < 0.25 * moved, (err, moved)
+
+
+# ---------------------------------------------------------------- H64 / EDEN-2 residual codec
+
+
+def _eden_from_gpu(codes, params, T, H, D, param):
+    """Pair indices [T, H, D/2] and scales [T, H, D/64] from the GPU buffers."""
+    raw = codes[: T * H * D // 4].cpu().numpy().reshape(T, H, D // 4)
+    idx = np.stack([raw & 15, raw >> 4], axis=-1).reshape(T, H, D // 2)
+    n = T * H * (D // 64)
+    dt = torch.float16 if param == "f16" else torch.float32
+    s = params[: n * (2 if param == "f16" else 4)].view(dt).reshape(T, H, D // 64).cpu().double().numpy()
+    return idx, s
+
+
+def _check_eden(idx_g, s_g, rec_g, oc, rec_ref, pred_ref, x, cb, state, param, what, skip=None, perr=0.0):
+    """Indices, scales and reconstructions of one tensor coded with H64 /
+    EDEN-2.  A group whose index or scale differs (a near tie of the nearest
+    point, or an fp16 rounding boundary) must reconstruct its own codes; the
+    fraction of such groups is bounded like the scalar codec's parameters.
+    Returns the per-token mask of tokens that differ anywhere."""
+    from scipy.linalg import hadamard
+
+    T, H, D = x.shape
+    keep = np.ones(T, bool) if skip is None else ~skip
+    U.assert_codes_close(idx_g[keep], oc.q[keep], what + " pair indices")
+    gi = (idx_g != oc.q).reshape(T, H, D // 64, 32).any(-1)
+    # fp16 scales either agree or sit on two sides of a rounding boundary; fp32
+    # scales of the same indices differ only in their last bits (fp32 sums)
+    gs = s_g != oc.s if param == "f16" else np.abs(s_g - oc.s) > 1e-5 * np.abs(oc.s)
+    gdiff = (gi | gs) & keep[:, None, None]
+    n_ok = int(keep.sum()) * H * (D // 64)
+    rate = gdiff.sum() / max(n_ok, 1)
+    U.OBSERVED.append({"check": what + " groups differing", "param": param, "param_groups_differing": float(rate),
+                       "groups": n_ok})
+    assert rate <= U.PARAM_FLIP_RATE + U.PARAM_FLIP_SLACK_GROUPS / max(n_ok, 1), (what, rate)
+    # scales of agreeing groups: one rounding step of the parameter format plus the fp32 error
+    same = ~gi & keep[:, None, None]
+    ulp = U.param_ulp(oc.s, param)
+    assert np.all(np.abs(s_g - oc.s)[same] <= 1.0001 * (ulp[same] + 1e-4 * np.abs(oc.s[same]))), what + " scales"
+    # every group reconstructs its own codes around the oracle's prediction
+    Hs = hadamard(64).astype(np.float64) / 8.0
+    yh = s_g[..., None, None] * cb[idx_g.reshape(T, H, D // 64, 32)]
+    own = pred_ref + (yh.reshape(T, H, D // 64, 64) @ Hs.T).reshape(T, H, D)
+    tol = 1e-3 * (np.abs(x) + 1.0)
+    # the GPU's fp32 prediction (perr) and its two fp32 transforms (six butterfly stages each)
+    err = perr + 8 * U.U32 * (np.abs(own) + np.abs(pred_ref)) + 64 * U.U32 * np.abs(s_g).max()
+    ulp_s = np.abs(O.round_to(own, state) - own) + np.spacing(np.abs(own).astype(np.float32))
+    live = keep[:, None, None]
+    bad = live & (np.abs(rec_g - own) > tol + err + ulp_s)
+    assert not np.any(bad), f"{what}: {int(bad.sum())} values do not reconstruct their own codes"
+    flip = np.repeat(gdiff, 64, axis=-1)
+    U.assert_recon_close(np.where(live, rec_g, rec_ref), rec_ref, own, x, flip | ~live, state, what + " recon")
+    return (gdiff.reshape(T, -1).any(1)) | (rec_g != rec_ref).reshape(T, -1).any(1)
+
+
+@pytest.mark.parametrize("dtype,T,H,D,rank", [(torch.bfloat16, 3 * 128 + 41, 12, 128, 64),
+                                              (torch.bfloat16, 97, 3, 64, 0), (torch.float32, 130, 2, 128, 8)])
+def test_eden2_codec_parity(dtype, T, H, D, rank):
+    """An anchor layer and a predicted cross-layer layer with the H64 / EDEN-2
+    residual codec, against the oracle (teacher-forced layer-0 sources)."""
+    cbt = synth.eden2_codebook()
+    cb = cbt.double().numpy()
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 113, L=2, T=T, H=H, D=D, rank=rank, calib_tokens=512, dtype=dtype)
+    param_t = torch.float16 if dtype == torch.bfloat16 else torch.float32
+    p = U.np_param(param_t)
+    state = U.np_state(dtype)
+    desc = kvc.make_desc(T, H, D, dtype, 2, 64, param_t, residual_codec=kvc.RESIDUAL_H64_EDEN2)
+    od = O.Desc(T, H, D, state, 2, 64, p, codec="eden2")
+    # anchor
+    p0 = kvc.make_predictor(kvc.PRED_NONE, residual_codebook=cbt.cuda())
+    buf0 = kvc.alloc_codes(desc, p0)
+    K0, V0 = wl.K[0].cuda(), wl.V[0].cuda()
+    K0r, V0r = torch.empty_like(K0), torch.empty_like(V0)
+    kvc.kvc_encode_layer(desc, p0, K0, V0, None, None, buf0, K0r, V0r)
+    K0d, V0d = torch.empty_like(K0), torch.empty_like(V0)
+    kvc.kvc_decode_layer(desc, p0, buf0, None, None, K0d, V0d)
+    _sync_ok()
+    assert torch.equal(K0d, K0r) and torch.equal(V0d, V0r)
+    ck0, cv0, K0h, V0h = O.encode_layer_none(od, U.to64(wl.K[0]), U.to64(wl.V[0]), codebook=cb)
+    zero = np.zeros((T, H, D))
+    for which, oc, rec, ref, x in (("k", ck0, K0r, K0h, wl.K[0]), ("v", cv0, V0r, V0h, wl.V[0])):
+        idx, s = _eden_from_gpu(getattr(buf0, which + "_codes"), getattr(buf0, which + "_params"), T, H, D, p)
+        _check_eden(idx, s, U.to64(rec), oc, ref, zero, U.to64(x), cb, state, p, f"anchor {which}")
+    # a predicted layer from the clean layer-0 values (shared by both sides)
+    w = {k: v.cuda() for k, v in wl.weights[1].items()}
+    p1 = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, w, rank=rank, residual_codebook=cbt.cuda())
+    buf, Kr, Vr = _xlayer_gpu(desc, p1, wl.K[1].cuda(), wl.V[1].cuda(), K0, V0)
+    w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
+    Ks, Vs = U.to64(wl.K[0]), U.to64(wl.V[0])
+    ck, cv, Kh, Vh, pk, pv = O.encode_layer_xlayer(od, w64, U.to64(wl.K[1]), U.to64(wl.V[1]), Ks, Vs, codebook=cb,
+                                                   with_pred=True)
+    errk, errv = U.err_xlayer(od, w64, Ks, Vs, Kh)
+    idx, s = _eden_from_gpu(buf.k_codes, buf.k_params, T, H, D, p)
+    kflip = _check_eden(idx, s, U.to64(Kr), ck, Kh, pk, U.to64(wl.K[1]), cb, state, p, "layer 1 K", perr=errk)
+    idx, s = _eden_from_gpu(buf.v_codes, buf.v_params, T, H, D, p)
+    _check_eden(idx, s, U.to64(Vr), cv, Vh, pv, U.to64(wl.V[1]), cb, state, p, "layer 1 V", skip=kflip, perr=errv)
+
+
+# ---------------------------------------------------------------- video-adapted refit
+
+
+@pytest.mark.parametrize("dtype,T,H,D,rank", [(torch.bfloat16, 1560, 12, 128, 64), (torch.float32, 300, 2, 64, 8),
+                                              (torch.bfloat16, 701, 4, 128, 0)])
+def test_refit_block_diag(dtype, T, H, D, rank):
+    """kvc_refit_block_diag (K and V blocks) against the oracle's ridge
+    least-squares fit, and the refitted block predicts the block's own tokens
+    at least as well as the offline one."""
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 114, L=2, T=T, H=H, D=D, rank=rank, calib_tokens=512, dtype=dtype)
+    w = {k: v.cuda() for k, v in wl.weights[1].items()}
+    param = torch.float16 if dtype == torch.bfloat16 else torch.float32
+    desc = _desc(T, H, D, dtype, 2, 32, param)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, w, rank=rank)
+    ridge = 1e-2 * T
+    w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
+    state = U.np_state(dtype)
+    for tensor, X0, X1, Y, wk, uk, off in ((0, wl.K[0], None, wl.K[1], "k_w", "k_u", "k_block"),
+                                           (1, wl.K[1], wl.V[0], wl.V[1], "v_w", "v_u", "v_block")):
+        din = D if tensor == 0 else 2 * D
+        out = torch.full((H, D, din), float("nan"), dtype=dtype, device="cuda")
+        ws = kvc.alloc_workspace(kvc.OP_REFIT_V if tensor else kvc.OP_REFIT_K, desc, pred)
+        kvc.kvc_refit_block_diag(desc, pred, tensor, X0.cuda(), None if X1 is None else X1.cuda(), Y.cuda(), ridge,
+                                 out, ws)
+        _sync_ok()
+        ref = O.refit_block_diag(U.to64(X0), None if X1 is None else U.to64(X1), U.to64(Y),
+                                 w64[wk] if rank else None, w64[uk] if rank else None, ridge)
+        got = U.to64(out)
+        rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        U.OBSERVED.append({"check": f"refit tensor {tensor} T={T}", "rel_fro": float(rel)})
+        # fp32 Gram sums and Cholesky against fp64, then one rounding to the layer dtype
+        assert rel <= 2e-3 if state == "bf16" else rel <= 1e-4, rel
+        assert np.all(np.abs(got - ref) <= 1e-3 * np.abs(ref).max() + np.abs(O.round_to(ref, state) - ref) * 2.01)
+        # the refitted block fits the block's own tokens better than the offline one
+        Xh = U.to64(X0) if X1 is None else np.concatenate([U.to64(X0), U.to64(X1)], -1)
+        flat = Xh.reshape(T, H, 2, D).transpose(0, 2, 1, 3).reshape(T, -1) if X1 is not None else Xh.reshape(T, -1)
+        lr = ((flat @ w64[wk].T) @ w64[uk].T).reshape(T, H, D) if rank else 0.0
+        res = lambda B: np.linalg.norm(U.to64(Y) - lr - np.einsum("thi,hoi->tho", Xh, B))
+        assert res(got) <= res(w64[off]) * 1.0001

@@ -156,3 +156,29 @@ def test_thread_count_does_not_change_results():
             _same_coded(x, y, "threads")
     Q = RNG.standard_normal((17, 2, 64))
     np.testing.assert_array_equal(C.attention(Q, K, V, 0.1, threads=1), C.attention(Q, K, V, 0.1, threads=6))
+
+
+def test_eden2_codec_layers():
+    """The H64 / EDEN-2 codec through an anchor layer and a cross-layer layer."""
+    from clustered_kv_cache_b200 import synth
+
+    cb = synth.eden2_codebook().double().numpy()
+    w, K, V, Ks, Vs = _xlayer_inputs(90, 3, 128, 16, "bf16", 77)
+    d = N.Desc(90, 3, 128, "bf16", 2, 64, "f16", codec="eden2")
+    a = N.encode_layer_none(d, K, V, codebook=cb)
+    b = C.encode_layer_none(d, K, V, threads=2, codebook=cb)
+    for i in range(2):
+        _same_coded(a[i], b[i], "anchor eden2")
+        np.testing.assert_array_equal(a[2 + i], b[2 + i])
+    a = N.encode_layer_xlayer(d, w, K, V, Ks, Vs, codebook=cb)
+    b = C.encode_layer_xlayer(d, w, K, V, Ks, Vs, threads=3, codebook=cb)
+    _same_coded(a[0], b[0], "K")
+    _same_coded(a[1], b[1], "V")
+    np.testing.assert_array_equal(a[2], b[2])
+    np.testing.assert_array_equal(a[3], b[3])
+    kd, vd = C.decode_layer_xlayer(d, w, b[0], b[1], Ks, Vs, codebook=cb)
+    np.testing.assert_array_equal(kd, b[2])
+    np.testing.assert_array_equal(vd, b[3])
+    nk, nv = N.decode_layer_xlayer(d, w, b[0], b[1], Ks, Vs, codebook=cb)
+    np.testing.assert_array_equal(nk, kd)
+    assert C.codes_bytes(d) == N.codes_bytes(d)

@@ -542,3 +542,126 @@ def test_jensen_correction_removes_the_bias_in_expectation(O):
     se = np.std(np.exp(raw)) / clean / np.sqrt(n)
     assert biased > 10 * se
     assert abs(fixed) < 4 * se + 0.02 * biased, (fixed, biased, se)
+
+
+# ---------------------------------------------------------------- H64 / EDEN-2 residual codec
+
+
+def _cb():
+    from clustered_kv_cache_b200 import synth
+
+    return synth.eden2_codebook().double().numpy()
+
+
+def test_h64_is_the_orthonormal_sylvester_hadamard_transform(O):
+    """The transform matches scipy's Hadamard matrix (Sylvester order) / 8,
+    and applying it twice gives the identity."""
+    from scipy.linalg import hadamard
+
+    rng = np.random.default_rng(18)
+    x = rng.standard_normal((5, 64))
+    Hs = hadamard(64).astype(np.float64) / 8.0
+    y = O.hadamard64(x) if O is O_CPP else x @ (O.hadamard_matrix(64) / 8.0).T
+    np.testing.assert_allclose(y, x @ Hs.T, rtol=1e-13, atol=1e-13)
+    back = O.hadamard64(y) if O is O_CPP else y @ (O.hadamard_matrix(64) / 8.0).T
+    np.testing.assert_allclose(back, x, rtol=1e-13, atol=1e-13)
+
+
+def _eden_rows(O, x, cb, param="f16", state="f64"):
+    """One tensor [T, 1, D] coded by the anchor path with the EDEN-2 codec."""
+    T, D = x.shape
+    d = O.Desc(T, 1, D, state, 2, 64, param, codec="eden2")
+    c, _, xh, _ = O.encode_layer_none(d, x[:, None, :], x[:, None, :], codebook=cb)
+    return c, xh[:, 0, :]
+
+
+def test_eden2_is_lossless_on_scaled_codebook_points(O):
+    """Residuals whose transform is exactly S times codebook points (a 4 x 4
+    grid codebook, dyadic S) come back exactly: indices, scale (EDEN's
+    |y|^2 / <y, c> = S) and values."""
+    g1 = np.array([-1.5, -0.5, 0.5, 1.5])
+    cb = np.array([[a, b] for a in g1 for b in g1])
+    rng = np.random.default_rng(19)
+    k = rng.integers(0, 16, (6, 64))  # 32 pairs per group, 2 groups per row
+    S = np.array([0.5, 0.25, 2.0, 1.0, 0.125, 4.0])
+    y = S[:, None, None] * cb[k]  # [6, 64, 2] = 6 rows x 128 values
+    y = y.reshape(6, 2, 64)
+    x = (y @ (np.asarray(__import__("scipy.linalg", fromlist=["hadamard"]).hadamard(64), float).T / 8.0)).reshape(6, 128)
+    c, xh = _eden_rows(O, x, cb)
+    np.testing.assert_array_equal(c.q.reshape(6, 64), k)
+    np.testing.assert_array_equal(c.s.reshape(6, 2), np.repeat(S[:, None], 2, 1))
+    np.testing.assert_allclose(xh, x, rtol=0, atol=1e-14)
+
+
+def test_eden2_indices_are_the_nearest_points_and_the_scale_is_unbiased(O):
+    """Brute force over the 16 points on the sigma-normalised pairs, the scale
+    satisfies <S c, y> = |y|^2 up to its fp16 rounding, a zero residual codes
+    to zeros, and the bits per value are those of INT2."""
+    cb = _cb()
+    rng = np.random.default_rng(20)
+    x = rng.standard_normal((40, 128)) * np.exp2(rng.integers(-3, 3, (40, 1)))
+    x[3] = 0.0
+    c, xh = _eden_rows(O, x, cb)
+    from scipy.linalg import hadamard
+
+    Hs = hadamard(64).astype(float) / 8.0
+    y = x.reshape(40, 2, 64) @ Hs.T
+    sig = np.sqrt((y * y).mean(-1))
+    u = (y / np.where(sig > 0, sig, 1)[..., None]).reshape(40, 2, 32, 2)
+    d = ((u[..., None, :] - cb) ** 2).sum(-1)
+    best = d.argmin(-1)
+    srt = np.sort(d, -1)
+    tie = (srt[..., 1] - srt[..., 0]) < 1e-12
+    q = c.q.reshape(40, 2, 32)
+    assert np.all((q == best) | tie)
+    assert np.all(q[3] == 0) and np.all(c.s.reshape(40, 2)[3] == 0) and np.all(xh[3] == 0)
+    yh = c.s.reshape(40, 2)[..., None, None] * cb[q]
+    lhs = (yh * y.reshape(40, 2, 32, 2)).sum((-1, -2))
+    rhs = (y * y).sum(-1)
+    live = rhs > 0
+    np.testing.assert_allclose(lhs[live], rhs[live], rtol=2.0 ** -10)
+    dd = O.Desc(1000, 12, 128, "bf16", 2, 64, "f16", codec="eden2")
+    assert O.codes_bytes(dd) * 8 / (2 * 1000 * 12 * 128) == pytest.approx(2 + 16 / 64)
+
+
+def test_eden2_beats_scalar_int2_on_gaussian_residuals(O):
+    """The point of the transform and the 2-D points: on Gaussian residuals the
+    H64 / EDEN-2 codec (2.25 bits per value) has lower error than scalar INT2
+    with fp16 (scale, zero) per 64 values (2.5 bits per value)."""
+    cb = _cb()
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((200, 128))
+    _, xe = _eden_rows(O, x, cb)
+    d = O.Desc(200, 1, 128, "f64", 2, 64, "f16")
+    _, _, xs, _ = O.encode_layer_none(d, x[:, None, :], x[:, None, :])
+    assert np.mean((xe - x) ** 2) < 0.8 * np.mean((xs[:, 0] - x) ** 2)
+
+
+# ---------------------------------------------------------------- video-adapted refit
+
+
+def test_refit_recovers_an_exact_block_and_satisfies_the_normal_equations(O):
+    """Targets made exactly by a block-DPLR map: with a vanishing ridge the
+    refit returns that map's blocks; with a ridge the result satisfies the
+    normal equations X^T (Y - LR - X B^T) = ridge B^T; rank 0 without a ridge
+    is plain per-head least squares (numpy lstsq)."""
+    rng = np.random.default_rng(22)
+    T, H, D, r = 300, 2, 16, 3
+    X0, X1 = rng.standard_normal((T, H, D)), rng.standard_normal((T, H, D))
+    Bv = rng.standard_normal((H, D, 2 * D)) * 0.3
+    w, u = rng.standard_normal((r, 2 * H * D)) * 0.1, rng.standard_normal((H * D, r))
+    flat = np.concatenate([X0.reshape(T, -1), X1.reshape(T, -1)], 1)
+    lr = ((flat @ w.T) @ u.T).reshape(T, H, D)
+    Xh = np.concatenate([X0, X1], -1)
+    Y = np.einsum("thi,hoi->tho", Xh, Bv) + lr
+    np.testing.assert_allclose(O.refit_block_diag(X0, X1, Y, w, u, 1e-12), Bv, atol=1e-9)
+    Yn = Y + 0.5 * rng.standard_normal(Y.shape)
+    ridge = 7.0
+    B = O.refit_block_diag(X0, X1, Yn, w, u, ridge)
+    for h in range(H):
+        res = Yn[:, h] - lr[:, h] - Xh[:, h] @ B[h].T
+        np.testing.assert_allclose(Xh[:, h].T @ res, ridge * B[h].T, atol=1e-9)
+    B0 = O.refit_block_diag(X0, None, Yn, None, None, 0.0)
+    for h in range(H):
+        ref = np.linalg.lstsq(X0[:, h], Yn[:, h], rcond=None)[0].T
+        np.testing.assert_allclose(B0[h], ref, atol=1e-10)
