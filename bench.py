@@ -602,14 +602,17 @@ def main():
         bi = sum(t.numel() * t.element_size() for t in hK + hV)
         bo = sum(t.numel() * t.element_size() for c in hcodes for t in c)
 
+        stream = torch.cuda.current_stream()
+
         def e2e_step():
+            # every byte moves through the library's C ABI: host inputs in, codes out
             for l in range(L_RUN):
-                xb.wl.K[l].copy_(hK[l], non_blocking=True)
-                xb.wl.V[l].copy_(hV[l], non_blocking=True)
+                kvc.kvc_copy_to_device(xb.wl.K[l], hK[l], stream)
+                kvc.kvc_copy_to_device(xb.wl.V[l], hV[l], stream)
             xb.step()
             for c, hc in zip(xb.codes, hcodes):
                 for src, dst in zip((c.k_codes, c.k_params, c.v_codes, c.v_params), hc):
-                    dst.copy_(src, non_blocking=True)
+                    kvc.kvc_copy_to_host(dst, src, stream)
 
         e2e_step()
         torch.cuda.synchronize()

@@ -532,6 +532,20 @@ kvc_status kvc_unpack_codes(const void* packed, int64_t n, int bits, uint8_t* co
   return e == cudaSuccess ? KVC_OK : cuda_fail(e);
 }
 
+kvc_status kvc_copy_to_device(void* dst, const void* src, size_t bytes, void* stream) {
+  if (bytes == 0) return KVC_OK;
+  if (!dst || !src) return KVC_ERR_INVALID_ARGUMENT;
+  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, (cudaStream_t)stream);
+  return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+}
+
+kvc_status kvc_copy_to_host(void* dst, const void* src, size_t bytes, void* stream) {
+  if (bytes == 0) return KVC_OK;
+  if (!dst || !src) return KVC_ERR_INVALID_ARGUMENT;
+  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+}
+
 kvc_status kvc_get_device_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e);

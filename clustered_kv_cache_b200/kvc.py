@@ -27,7 +27,7 @@ STATUS = {0: "KVC_OK", 1: "KVC_ERR_INVALID_ARGUMENT", 2: "KVC_ERR_UNSUPPORTED", 
 EXPORTED = ["kvc_codes_sizes", "kvc_codes_bytes", "kvc_workspace_bytes", "kvc_encode_layer", "kvc_decode_layer",
             "kvc_attend_compressed", "kvc_pack_codes", "kvc_unpack_codes", "kvc_get_device_error",
             "kvc_status_string", "kvc_last_cuda_error", "kvc_launch_counter", "kvc_testing_inject_stall",
-            "kvc_attend_compressed_debiased", "kvc_refit_block_diag"]
+            "kvc_attend_compressed_debiased", "kvc_refit_block_diag", "kvc_copy_to_device", "kvc_copy_to_host"]
 
 
 class KvcError(RuntimeError):
@@ -84,6 +84,8 @@ def lib():
         "kvc_attend_compressed": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, V, V, SZ, V]),
         "kvc_attend_compressed_debiased": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, V, V, SZ, V]),
         "kvc_refit_block_diag": (I, [D, PR, ctypes.c_int, V, V, V, F, V, V, SZ, V]),
+        "kvc_copy_to_device": (I, [V, V, SZ, V]),
+        "kvc_copy_to_host": (I, [V, V, SZ, V]),
         "kvc_pack_codes": (I, [V, I64, I, V, V]),
         "kvc_unpack_codes": (I, [V, I64, I, V, V]),
         "kvc_get_device_error": (I, [V]),
@@ -255,6 +257,22 @@ def kvc_refit_block_diag(desc, pred, tensor: int, X0, X1, Y, ridge: float, block
     _check(lib().kvc_refit_block_diag(ctypes.byref(desc), ctypes.byref(pred), int(tensor), _ptr(X0), _ptr(X1),
                                       _ptr(Y), ctypes.c_float(ridge), _ptr(block_out), wp, wn, _stream(stream)),
            "kvc_refit_block_diag")
+
+
+def kvc_copy_to_device(dst: torch.Tensor, src: torch.Tensor, stream=None):
+    """Copies a host tensor (pinned for asynchrony) into a device tensor of the same size."""
+    n = src.numel() * src.element_size()
+    assert dst.numel() * dst.element_size() >= n
+    _check(lib().kvc_copy_to_device(_ptr(dst), ctypes.c_void_p(src.data_ptr()), n, _stream(stream)),
+           "kvc_copy_to_device")
+
+
+def kvc_copy_to_host(dst: torch.Tensor, src: torch.Tensor, stream=None):
+    """Copies a device tensor into a host tensor (pinned for asynchrony) of the same size."""
+    n = src.numel() * src.element_size()
+    assert dst.numel() * dst.element_size() >= n
+    _check(lib().kvc_copy_to_host(ctypes.c_void_p(dst.data_ptr()), _ptr(src), n, _stream(stream)),
+           "kvc_copy_to_host")
 
 
 def kvc_pack_codes(codes: torch.Tensor, bits: int, packed: torch.Tensor, stream=None):

@@ -278,6 +278,13 @@ KVC_API kvc_status kvc_pack_codes(const uint8_t* codes, int64_t n, int bits, voi
 /* Inverse of kvc_pack_codes. */
 KVC_API kvc_status kvc_unpack_codes(const void* packed, int64_t n, int bits, uint8_t* codes, void* stream);
 
+/* Host <-> device copies for callers that keep the cache's inputs and codes in
+ * host memory: one stream-ordered cudaMemcpyAsync of `bytes` bytes (pinned
+ * host memory makes it asynchronous).  dst / src: device and host pointers as
+ * the names say; KVC_ERR_INVALID_ARGUMENT for NULL pointers with bytes > 0. */
+KVC_API kvc_status kvc_copy_to_device(void* dst_device, const void* src_host, size_t bytes, void* stream);
+KVC_API kvc_status kvc_copy_to_host(void* dst_host, const void* src_device, size_t bytes, void* stream);
+
 /* Synchronizes `stream`, returns the first device-side error recorded since
  * the last call (KVC_OK if none) and clears it. */
 KVC_API kvc_status kvc_get_device_error(void* stream);
