@@ -45,6 +45,7 @@ bool row_layout_ok(int n, int group) {
 kvc_status check_desc(const kvc_layer_desc* d, const kvc_predictor* p) {
   if (!d || !p) return KVC_ERR_INVALID_ARGUMENT;
   if (d->n_tokens < 0 || d->n_heads < 1) return KVC_ERR_INVALID_ARGUMENT;
+  if (d->q_heads < 0 || (d->q_heads > 0 && d->q_heads % d->n_heads)) return KVC_ERR_INVALID_ARGUMENT;
   if (d->head_dim != 64 && d->head_dim != 128) return KVC_ERR_UNSUPPORTED;
   if (d->dtype != KVC_F32 && d->dtype != KVC_BF16) return KVC_ERR_UNSUPPORTED;
   if (d->param_dtype != KVC_F32 && d->param_dtype != KVC_F16) return KVC_ERR_UNSUPPORTED;
@@ -398,6 +399,7 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
   if ((s = check_codebook(d, p)) != KVC_OK) return s;
   if (n_q < 0 || n_self < 0) return KVC_ERR_INVALID_ARGUMENT;
   if (p->kind == KVC_PRED_CLUSTER && n_self != 0) return KVC_ERR_UNSUPPORTED;
+  if (p->kind == KVC_PRED_CLUSTER && d->q_heads > 0 && d->q_heads != d->n_heads) return KVC_ERR_UNSUPPORTED;
   if (!codes_ok(p, codes) || (n_q > 0 && (!Q || !O))) return KVC_ERR_INVALID_ARGUMENT;
   if (n_self > 0 && (!K_self || !V_self)) return KVC_ERR_INVALID_ARGUMENT;
   if (p->kind == KVC_PRED_XLAYER_DPLR && (!K_src || !V_src)) return KVC_ERR_INVALID_ARGUMENT;
@@ -452,8 +454,8 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
     if (V_rec_opt) Vh = (TS*)V_rec_opt;
     cudaError_t e = codec_xlayer<TS, TP>(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh, cv, st);
     if (e != cudaSuccess) return e;
-    AttnArgs<TS> a{n_q, d->n_tokens, n_self, H, scale, (const TS*)Q, Kh, Vh, (const TS*)K_self,
-                   (const TS*)V_self, (TS*)O};
+    AttnArgs<TS> a{n_q, d->n_tokens, n_self, H, d->q_heads > 0 ? d->q_heads : H, scale, (const TS*)Q, Kh, Vh,
+                   (const TS*)K_self, (const TS*)V_self, (TS*)O};
     return launch_attention(a, D, st);
   });
 }

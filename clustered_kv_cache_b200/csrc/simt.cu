@@ -605,14 +605,15 @@ __global__ void __launch_bounds__(kThreads) attention_kernel(AttnArgs<TS> a) {
   float* sS = sV + 32 * D;          // [32][33]
   constexpr int DJ = D / 8;
   const int64_t q0 = (int64_t)blockIdx.x * 32;
-  const int h = blockIdx.y;
+  const int hq = blockIdx.y;        // query head
+  const int h = hq / (a.Hq / a.H);  // its KV head (grouped-query attention when Hq > H)
   const int H = a.H;
   const int tid = threadIdx.x;
   const int qr = tid >> 3, sub = tid & 7;
   for (int e = tid; e < 32 * D; e += kThreads) {
     const int r = e / D, d = e % D;
     const int64_t q = q0 + r;
-    sQ[e] = q < a.n_q ? to_f(a.Q[(q * H + h) * D + d]) : 0.f;
+    sQ[e] = q < a.n_q ? to_f(a.Q[(q * a.Hq + hq) * D + d]) : 0.f;
   }
   float o[DJ];
 #pragma unroll
@@ -673,7 +674,7 @@ __global__ void __launch_bounds__(kThreads) attention_kernel(AttnArgs<TS> a) {
   if (q < a.n_q) {
     const float inv = 1.f / lrow;
 #pragma unroll
-    for (int j = 0; j < DJ; ++j) a.O[(q * H + h) * D + sub + 8 * j] = from_f<TS>(o[j] * inv);
+    for (int j = 0; j < DJ; ++j) a.O[(q * a.Hq + hq) * D + sub + 8 * j] = from_f<TS>(o[j] * inv);
   }
 }
 
@@ -952,7 +953,7 @@ cudaError_t launch_cluster(const ClusterArgs<TS, TP>& a, bool encode, cudaStream
 template <typename TS>
 cudaError_t launch_attention(const AttnArgs<TS>& a, int D, cudaStream_t st) {
   if (a.n_q == 0) return cudaSuccess;
-  dim3 grid(div_up(a.n_q, 32), a.H);
+  dim3 grid(div_up(a.n_q, 32), a.Hq);
   const size_t smem = (32 * D + 32 * (D + 1) + 32 * D + 32 * 33) * sizeof(float);
   cudaError_t e;
   if (D == 128) {

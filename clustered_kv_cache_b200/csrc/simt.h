@@ -80,6 +80,7 @@ template <typename TS>
 struct AttnArgs {
   int64_t n_q, n_hist, n_self;
   int H;
+  int Hq;  // query heads, a multiple of H (Q and O are [n_q][Hq][D])
   float scale;
   const TS* Q;
   const TS* Kh;

@@ -70,6 +70,7 @@ struct Args {
   unsigned* err;
   int64_t n_q, T, n_self;
   int H, bits, group;
+  int Hq;  // query heads (a multiple of H); query head h reads KV head h / (Hq / H)
   float scale_log2;  // softmax scale * log2(e)
   const uint8_t* kcodes;
   const __half2* kparams;
@@ -233,7 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
+  const int hq = blockIdx.y;           // query head
+  const int h = hq / (a.Hq / a.H);     // its KV head (grouped-query attention when Hq > H)
   const int q0 = blockIdx.x * 128;
   const bool has_q = q0 < a.n_q;  // the last cluster of a head may hold CTAs past the queries
   const int rank = (int)cluster_rank();
@@ -319,8 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
       };
       if (has_q) {
         mbar_arrive_expect_tx(q_full, 32768u);
-        tma_load(Qs, &maps.q, h * 128, q0, q_full, pol_stream);
-        tma_load(Qs + 16384, &maps.q, h * 128 + 64, q0, q_full, pol_stream);
+        tma_load(Qs, &maps.q, hq * 128, q0, q_full, pol_stream);
+        tma_load(Qs + 16384, &maps.q, hq * 128 + 64, q0, q_full, pol_stream);
       }
       // decode operands of this CTA's history tiles, in the order the MMA warp takes them
       for (int j = rank; j < NH && ok; j += CQ) {
@@ -545,8 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
       fence_async_smem();
       asm volatile("bar.sync 1, 128;" ::: "memory");
     };
-    // the first cluster of each head writes the decoded history when asked to
-    const bool first_cluster = blockIdx.x < (unsigned)CQ;
+    // the first cluster of the first query head of each KV head writes the
+    // decoded history when asked to
+    const bool first_cluster = blockIdx.x < (unsigned)CQ && hq % (a.Hq / a.H) == 0;
     const bool st_k = first_cluster && a.store_k, st_v = first_cluster && a.store_v;
     // the tile is complete here: announce it to every peer, push it, and mark it locally
     auto publish = [&](uint8_t* tile, uint64_t* bar, const CUtensorMap* out, int j) {
@@ -723,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_cluster_kernel(const __gri
       float ov[32];
       tmem_ld32(lane_addr + (OC - tmem) + pc * 32, ov);
       if (qrow < a.n_q) {
-        uint4* dst = reinterpret_cast<uint4*>(a.O + (qrow * a.H + h) * 128 + pc * 32);
+        uint4* dst = reinterpret_cast<uint4*>(a.O + (qrow * a.Hq + hq) * 128 + pc * 32);
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t w[4];
@@ -753,7 +756,7 @@ static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
   const unsigned nqt = (unsigned)((a.n_q + 127) / 128);
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((nqt + CQ - 1) / CQ * CQ, (unsigned)a.H);
+  cfg.gridDim = dim3((nqt + CQ - 1) / CQ * CQ, (unsigned)a.Hq);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = st;
@@ -822,8 +825,9 @@ cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const voi
   }
   tc::attn::Maps m;
   memset(&m, 0, sizeof(m));
+  const uint64_t Hq = d->q_heads > 0 ? (uint64_t)d->q_heads : H;
   const uint64_t Th = T > 0 ? T : 1;  // maps need a non-empty extent; no history tile is read when T = 0
-  bool ok = tc::map2d(&m.q, Q, (uint64_t)n_q, C, 128) && tc::map2d(&m.ks, T ? Ks : Q, Th, C, 128) &&
+  bool ok = tc::map2d(&m.q, Q, (uint64_t)n_q, Hq * 128, 128) && tc::map2d(&m.ks, T ? Ks : Q, Th, C, 128) &&
             tc::map2d(&m.vs, T ? Vs : Q, Th, C, 128) && tc::map2d(&m.bk, p->k_block, H * 128, 128, 128) &&
             tc::map2d(&m.bv, p->v_block, H * 128, 256, 128);
   if (ok && n_self > 0)
@@ -844,7 +848,7 @@ cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const voi
   if (!ok) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
-  tc::attn::Args a{err, n_q, (int64_t)T, n_self, (int)H, d->bits, d->group, scale * 1.4426950408889634f,
+  tc::attn::Args a{err, n_q, (int64_t)T, n_self, (int)H, d->bits, d->group, (int)Hq, scale * 1.4426950408889634f,
                    (const uint8_t*)c->k_codes, (const __half2*)c->k_params, (const uint8_t*)c->v_codes,
                    (const __half2*)c->v_params, (__nv_bfloat16*)O, sk ? 1 : 0, sv ? 1 : 0,
                    0.5f * scale * scale * 1.4426950408889634f / 12.f};

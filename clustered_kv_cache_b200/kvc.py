@@ -40,7 +40,7 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [("n_tokens", ctypes.c_int64), ("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("bits", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("param_dtype", ctypes.c_int32), ("frame_tokens", ctypes.c_int32), ("anchor_bits", ctypes.c_int32),
-                ("residual_codec", ctypes.c_int32)]
+                ("residual_codec", ctypes.c_int32), ("q_heads", ctypes.c_int32)]
 
 
 class Predictor(ctypes.Structure):
@@ -135,9 +135,9 @@ RESIDUAL_RTN, RESIDUAL_H64_EDEN2 = 0, 1
 
 def make_desc(n_tokens: int, n_heads: int, head_dim: int, dtype=torch.bfloat16, bits: int = 2, group: int = 32,
               param_dtype=torch.float16, frame_tokens: int = 0, anchor_bits: int = 4,
-              residual_codec: int = RESIDUAL_RTN) -> LayerDesc:
+              residual_codec: int = RESIDUAL_RTN, q_heads: int = 0) -> LayerDesc:
     return LayerDesc(n_tokens, n_heads, head_dim, _DT[dtype], bits, group, _DT[param_dtype], frame_tokens,
-                     anchor_bits, residual_codec)
+                     anchor_bits, residual_codec, q_heads)
 
 
 def make_predictor(kind: int, weights: dict | None = None, rank: int = 0, n_clusters: int = 0,

@@ -103,7 +103,13 @@ typedef enum {
  *         scale per group, S = |y|^2 / <y, c> (EDEN's unbiased scale, 0 when
  *         y = 0 or <y, c> <= 0), is stored in param_dtype; decoding applies
  *         H64 / 8 to S c.  Requires bits = 2 (4 bits per pair), group = 64 and
- *         KVC_PRED_NONE or KVC_PRED_XLAYER_DPLR; runs on the CUDA cores. */
+ *         KVC_PRED_NONE or KVC_PRED_XLAYER_DPLR; runs on the CUDA cores.
+ *  q_heads: attention only: query heads, 0 (= n_heads) or a multiple of
+ *         n_heads (grouped-query attention, as in MAGI-1's native GQA,
+ *         "CORAL-KV ...", Table 3): query head j attends over the history of
+ *         KV head j / (q_heads / n_heads); Q and O are then [n_q][q_heads][D]
+ *         while the history, K_self and V_self keep n_heads.  Not for
+ *         KVC_PRED_CLUSTER (KVC_ERR_UNSUPPORTED). */
 typedef struct {
   int64_t n_tokens;
   int32_t n_heads;
@@ -115,6 +121,7 @@ typedef struct {
   int32_t frame_tokens;
   int32_t anchor_bits;
   int32_t residual_codec;
+  int32_t q_heads;
 } kvc_layer_desc;
 
 /* Predictor weights (device pointers, dtype of the layer, read only).
@@ -209,7 +216,7 @@ KVC_API kvc_status kvc_decode_layer(const kvc_layer_desc* desc, const kvc_predic
                             const void* K_src, const void* V_src, void* K_rec, void* V_rec, void* ws,
                             size_t ws_bytes, void* stream);
 
-/* Softmax attention of Q [n_q][H][D] over this layer's compressed history,
+/* Softmax attention of Q [n_q][H][D] (H = desc->q_heads when set) over this layer's compressed history,
  * followed by n_self uncompressed tokens K_self / V_self [n_self][H][D]
  * (non-causal; n_self may be 0 and the pointers NULL):
  *   O = softmax(scale * Q [K_hist; K_self]^T) [V_hist; V_self].

@@ -647,24 +647,29 @@ static double jensen_term(const double* q, const double* sk, int D, int group, d
   return 0.5 * scale * scale * acc;
 }
 
-void kvo_attention_corrected(int64_t nq, int64_t nk, int H, int D, double scale, const double* Q, const double* K,
-                             const double* V, int64_t n_hist, const double* s_hist, int group, double* O);
+void kvo_attention_corrected(int64_t nq, int64_t nk, int Hq, int H, int D, double scale, const double* Q,
+                             const double* K, const double* V, int64_t n_hist, const double* s_hist, int group,
+                             double* O);
 
 void kvo_attention(int64_t nq, int64_t nk, int H, int D, double scale, const double* Q, const double* K,
                    const double* V, double* O) {
-  kvo_attention_corrected(nq, nk, H, D, scale, Q, K, V, 0, nullptr, 1, O);
+  kvo_attention_corrected(nq, nk, H, H, D, scale, Q, K, V, 0, nullptr, 1, O);
 }
 
-// As kvo_attention; the first n_hist keys are quantized history whose group
-// scales s_hist [n_hist][H][D / group] give each one's Jensen correction
-// (s_hist NULL: no correction).
-void kvo_attention_corrected(int64_t nq, int64_t nk, int H, int D, double scale, const double* Q, const double* K,
-                             const double* V, int64_t n_hist, const double* s_hist, int group, double* O) {
-  const int C = H * D, ng = D / group;
+// As kvo_attention, with Hq query heads over H key / value heads (Hq a multiple
+// of H: query head hq reads head hq / (Hq / H), grouped-query attention); the
+// first n_hist keys are quantized history whose group scales
+// s_hist [n_hist][H][D / group] give each one's Jensen correction (s_hist
+// NULL: no correction).  Q, O [nq][Hq][D]; K, V [nk][H][D].
+void kvo_attention_corrected(int64_t nq, int64_t nk, int Hq, int H, int D, double scale, const double* Q,
+                             const double* K, const double* V, int64_t n_hist, const double* s_hist, int group,
+                             double* O) {
+  const int C = H * D, Cq = Hq * D, ng = D / group, g = Hq / H;
   std::vector<double> sc(nk > 0 ? nk : 1), acc(D);
   for (int64_t i = 0; i < nq; ++i)
-    for (int h = 0; h < H; ++h) {
-      const double* q = Q + i * C + h * D;
+    for (int hq = 0; hq < Hq; ++hq) {
+      const int h = hq / g;
+      const double* q = Q + i * Cq + hq * D;
       double m = -INFINITY;
       for (int64_t t = 0; t < nk; ++t) {
         double dot = 0.0;
@@ -684,7 +689,7 @@ void kvo_attention_corrected(int64_t nq, int64_t nk, int H, int D, double scale,
         const double* v = V + t * C + h * D;
         for (int d = 0; d < D; ++d) acc[d] += sc[t] * v[d];
       }
-      double* o = O + i * C + h * D;
+      double* o = O + i * Cq + hq * D;
       for (int d = 0; d < D; ++d) o[d] = acc[d] / l;
     }
 }

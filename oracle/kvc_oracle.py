@@ -523,12 +523,20 @@ def decode_tensor_cluster(desc: Desc, c: Coded, centroids, dec, exact: bool = Fa
 # --------------------------------------------------------------------------
 
 
+def _gqa(Q, X):
+    """Key / value heads repeated for the query heads that read them."""
+    g = Q.shape[1] // X.shape[1]
+    return X if g == 1 else np.repeat(np.asarray(X), g, axis=1)
+
+
 def attention(Q, K, V, scale: float) -> np.ndarray:
     """Naive two-pass softmax attention, fp64.
 
-    Q [Nq,H,D], K [Nk,H,D], V [Nk,H,D] -> O [Nq,H,D];
-    m = max_k s, p = exp(s - m), o = sum p v / sum p.
+    Q [Nq,Hq,D], K [Nk,H,D], V [Nk,H,D] -> O [Nq,Hq,D];
+    m = max_k s, p = exp(s - m), o = sum p v / sum p.  Hq a multiple of H:
+    query head j reads head j // (Hq // H) (grouped-query attention).
     """
+    K, V = _gqa(Q, K), _gqa(Q, V)
     S = np.matmul(Q.transpose(1, 0, 2), K.transpose(1, 2, 0)) * scale  # [H,Nq,Nk]
     m = S.max(axis=-1, keepdims=True)
     p = np.exp(S - m)
@@ -552,6 +560,7 @@ def jensen_correction(Q, s_hist, group: int, scale: float) -> np.ndarray:
 def attention_corrected(Q, K, V, scale: float, n_hist: int, s_hist, group: int) -> np.ndarray:
     """Naive attention whose first n_hist (quantized) keys have their scores
     lowered by the Jensen-bias term; the remaining keys are uncompressed."""
+    K, V, s_hist = _gqa(Q, K), _gqa(Q, V), _gqa(Q, s_hist)
     S = np.matmul(Q.transpose(1, 0, 2), K.transpose(1, 2, 0)) * scale  # [H,Nq,Nk]
     S[:, :, :n_hist] -= jensen_correction(Q, s_hist, group, scale)
     m = S.max(axis=-1, keepdims=True)

@@ -391,14 +391,16 @@ def decode_tensor_cluster(desc: Desc, c: Coded, centroids, dec, exact: bool = Fa
 
 
 def attention(Q, K, V, scale: float, threads=None) -> np.ndarray:
-    """Naive two-pass softmax attention; query rows split over threads."""
+    """Naive two-pass softmax attention; query rows split over threads.  Q may
+    have a multiple of K's heads (grouped-query attention)."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
-    nq, H, D = Q.shape
-    nk = K.shape[0]
-    O = np.empty((nq, H, D))
+    nq, Hq, D = Q.shape
+    nk, H = K.shape[:2]
+    O = np.empty((nq, Hq, D))
 
     def run(a, b):
-        lib().kvo_attention(_i(b - a), _i(nk), H, D, ctypes.c_double(scale), _p(Q[a:b]), _p(K), _p(V), _p(O[a:b]))
+        lib().kvo_attention_corrected(_i(b - a), _i(nk), Hq, H, D, ctypes.c_double(scale), _p(Q[a:b]), _p(K), _p(V),
+                                      _i(0), None, 1, _p(O[a:b]))
 
     _drive(_runs(nq, threads), run)
     return O
@@ -410,13 +412,13 @@ def attention_corrected(Q, K, V, scale: float, n_hist: int, s_hist, group: int, 
     (the abstract on the "Jensen bias" of INT2 key caches, CORAL-KV page);
     s_hist [n_hist, H, D/group]."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
-    nq, H, D = Q.shape
-    nk = K.shape[0]
+    nq, Hq, D = Q.shape
+    nk, H = K.shape[:2]
     sh = _f64(s_hist)
-    O = np.empty((nq, H, D))
+    O = np.empty((nq, Hq, D))
 
     def run(a, b):
-        lib().kvo_attention_corrected(_i(b - a), _i(nk), H, D, ctypes.c_double(scale), _p(Q[a:b]), _p(K), _p(V),
+        lib().kvo_attention_corrected(_i(b - a), _i(nk), Hq, H, D, ctypes.c_double(scale), _p(Q[a:b]), _p(K), _p(V),
                                       _i(n_hist), _p(sh), group, _p(O[a:b]))
 
     _drive(_runs(nq, threads), run)

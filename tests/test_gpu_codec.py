@@ -942,3 +942,59 @@ def test_refit_block_diag(dtype, T, H, D, rank):
         lr = ((flat @ w64[wk].T) @ w64[uk].T).reshape(T, H, D) if rank else 0.0
         res = lambda B: np.linalg.norm(U.to64(Y) - lr - np.einsum("thi,hoi->tho", Xh, B))
         assert res(got) <= res(w64[off]) * 1.0001
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+
+@pytest.mark.parametrize("n_q,n_self,T,H,group_q,jensen", [(300, 130, 3 * 128 + 5, 4, 2, False),
+                                                           (129, 0, 256, 2, 4, False), (200, 64, 300, 4, 3, True)])
+def test_grouped_query_attention_cross_layer(n_q, n_self, T, H, group_q, jensen):
+    """q_heads = group_q x n_heads on the tensor-core path: query head j reads
+    KV head j // group_q; history codes by the oracle."""
+    D = 128
+    Hq = H * group_q
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 115, L=2, T=T, H=H, rank=16, calib_tokens=512)
+    bf, hf = torch.bfloat16, torch.float16
+    od = _odesc(T, H, D, bf, 2, 32, hf)
+    w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
+    Ks, Vs = U.to64(wl.K[0]), U.to64(wl.V[0])
+    ck, cv, _, _ = O.encode_layer_xlayer(od, w64, U.to64(wl.K[1]), U.to64(wl.V[1]), Ks, Vs)
+    buf = _oracle_codes_to_gpu(ck, cv, 2, "f16")
+    Q = synth.queries(51, n_q, Hq, D)
+    Kself, Vself = synth.queries(52, n_self, H, D), synth.queries(53, n_self, H, D)
+    desc = kvc.make_desc(T, H, D, bf, 2, 32, hf, q_heads=Hq)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=16)
+    Og = torch.empty(n_q, Hq, D, dtype=bf, device="cuda")
+    ws = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q)
+    fn = kvc.kvc_attend_compressed_debiased if jensen else kvc.kvc_attend_compressed
+    fn(desc, pred, Q.cuda(), buf, wl.K[0].cuda(), wl.V[0].cuda(), Kself.cuda() if n_self else None,
+       Vself.cuda() if n_self else None, D ** -0.5, Og, ws)
+    _sync_ok()
+    ref = O.attend_compressed_xlayer(od, w64, U.to64(Q), ck, cv, Ks, Vs, U.to64(Kself) if n_self else None,
+                                     U.to64(Vself) if n_self else None, D ** -0.5, jensen=jensen)
+    err = U.rel_l2(U.to64(Og), ref)
+    U.OBSERVED.append({"check": f"GQA attention Hq={Hq} H={H}", "rel_l2": err})
+    assert err <= U.ATT_TOL[bf], err
+
+
+def test_grouped_query_attention_cuda_core_path():
+    """The fp32 tiny history (CUDA-core attention) with 4 query heads per KV head."""
+    wl = synth.tiny_xlayer()
+    T, H, D = wl.K[0].shape
+    f32 = torch.float32
+    od = _odesc(T, H, D, f32, 4, 32, f32)
+    ck0, cv0, K0h, V0h = O.encode_layer_none(od, U.to64(wl.K[0]), U.to64(wl.V[0]))
+    w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
+    ck1, cv1, _, _ = O.encode_layer_xlayer(od, w64, U.to64(wl.K[1]), U.to64(wl.V[1]), K0h, V0h)
+    Q = synth.queries(9, 40, 4 * H, D, dtype=f32)
+    desc = kvc.make_desc(T, H, D, f32, 4, 32, f32, q_heads=4 * H)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=wl.rank)
+    buf = _oracle_codes_to_gpu(ck1, cv1, 4, "f32")
+    Og = torch.empty(40, 4 * H, D, device="cuda")
+    kvc.kvc_attend_compressed(desc, pred, Q.cuda(), buf, torch.from_numpy(K0h).float().cuda(),
+                              torch.from_numpy(V0h).float().cuda(), None, None, 0.125, Og,
+                              kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, 40))
+    _sync_ok()
+    ref = O.attend_compressed_xlayer(od, w64, U.to64(Q), ck1, cv1, K0h, V0h, None, None, 0.125)
+    assert U.rel_l2(U.to64(Og), ref) <= U.ATT_TOL[f32]

@@ -665,3 +665,15 @@ def test_refit_recovers_an_exact_block_and_satisfies_the_normal_equations(O):
     for h in range(H):
         ref = np.linalg.lstsq(X0[:, h], Yn[:, h], rcond=None)[0].T
         np.testing.assert_allclose(B0[h], ref, atol=1e-10)
+
+
+def test_grouped_query_attention_matches_torch_sdpa(O):
+    """Query head j reads KV head j // (Hq / H): torch's SDPA with enable_gqa
+    (fp64) gives the same outputs."""
+    rng = np.random.default_rng(23)
+    Q = rng.standard_normal((9, 6, 16))
+    K, V = rng.standard_normal((31, 2, 16)), rng.standard_normal((31, 2, 16))
+    got = O.attention(Q, K, V, 0.3)
+    t = lambda x: torch.from_numpy(x).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(Q), t(K), t(V), scale=0.3, enable_gqa=True)
+    np.testing.assert_allclose(got, ref[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-13)
