@@ -861,10 +861,15 @@ def _check_eden(idx_g, s_g, rec_g, oc, rec_ref, pred_ref, x, cb, state, param, w
 
 
 @pytest.mark.parametrize("dtype,T,H,D,rank", [(torch.bfloat16, 3 * 128 + 41, 12, 128, 64),
+                                              (torch.bfloat16, 2 * 128 + 7, 4, 128, 0),
+                                              (torch.bfloat16, 300, 2, 128, 128),
                                               (torch.bfloat16, 97, 3, 64, 0), (torch.float32, 130, 2, 128, 8)])
 def test_eden2_codec_parity(dtype, T, H, D, rank):
     """An anchor layer and a predicted cross-layer layer with the H64 / EDEN-2
-    residual codec, against the oracle (teacher-forced layer-0 sources)."""
+    residual codec, against the oracle (teacher-forced layer-0 sources).  bf16
+    with head_dim 128 and rank 0 / 64 / 128 runs the tensor-core codec (the
+    epilogue transforms and codes each 64-value group in one thread); the other
+    shapes run the CUDA-core kernels."""
     cbt = synth.eden2_codebook()
     cb = cbt.double().numpy()
     wl = synth.wan_xlayer(seed=synth.SEED_BASE + 113, L=2, T=T, H=H, D=D, rank=rank, calib_tokens=512, dtype=dtype)
@@ -954,7 +959,7 @@ def test_grouped_query_attention_cross_layer(n_q, n_self, T, H, group_q, jensen)
     KV head j // group_q; history codes by the oracle."""
     D = 128
     Hq = H * group_q
-    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 115, L=2, T=T, H=H, rank=16, calib_tokens=512)
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 115, L=2, T=T, H=H, rank=64, calib_tokens=512)
     bf, hf = torch.bfloat16, torch.float16
     od = _odesc(T, H, D, bf, 2, 32, hf)
     w64 = {k: U.to64(v) for k, v in wl.weights[1].items()}
@@ -964,7 +969,7 @@ def test_grouped_query_attention_cross_layer(n_q, n_self, T, H, group_q, jensen)
     Q = synth.queries(51, n_q, Hq, D)
     Kself, Vself = synth.queries(52, n_self, H, D), synth.queries(53, n_self, H, D)
     desc = kvc.make_desc(T, H, D, bf, 2, 32, hf, q_heads=Hq)
-    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=16)
+    pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=64)
     Og = torch.empty(n_q, Hq, D, dtype=bf, device="cuda")
     ws = kvc.alloc_workspace(kvc.OP_ATTEND, desc, pred, n_q)
     fn = kvc.kvc_attend_compressed_debiased if jensen else kvc.kvc_attend_compressed
