@@ -344,6 +344,38 @@ kvc_status codec_common(const kvc_layer_desc* d, const kvc_predictor* p, bool en
   });
 }
 
+// Attention over a predicted (or anchor) history: the history is decoded once
+// (into the caller's outputs when given, else the workspace), then attended
+// with the chunk's own keys; jensen: the debiased scores (tensor cores only).
+kvc_status attend_decoded(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
+                          const kvc_codes* codes, const void* K_src, const void* V_src, const void* K_self,
+                          const void* V_self, int64_t n_self, float scale, void* O, void* K_rec_opt, void* V_rec_opt,
+                          void* ws, size_t ws_bytes, cudaStream_t st, bool jensen) {
+  Carve cv{(char*)ws, ws_bytes};
+  return dispatch(d, [&](auto* ts, auto* tp) -> cudaError_t {
+    using TS = std::remove_pointer_t<decltype(ts)>;
+    using TP = std::remove_pointer_t<decltype(tp)>;
+    const int H = d->n_heads, D = d->head_dim;
+    const size_t bytes = (size_t)d->n_tokens * H * D * sizeof(TS);
+    TS* Kh = (TS*)cv.take(bytes);
+    TS* Vh = (TS*)cv.take(bytes);
+    if (K_rec_opt) Kh = (TS*)K_rec_opt;
+    if (V_rec_opt) Vh = (TS*)V_rec_opt;
+    if (d->n_tokens > 0) {
+      cudaError_t e = tc_codec_supported(d, p)
+                          ? tc_codec_layer(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh, nullptr, 0, st)
+                          : codec_xlayer<TS, TP>(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh, cv, st);
+      if (e != cudaSuccess) return e;
+    }
+    if (tc_flash_supported(d))
+      return tc_flash(d, Q, n_q, Kh, Vh, K_self, V_self, n_self, scale, O, jensen ? codes->k_params : nullptr, st);
+    if (jensen) return cudaErrorNotSupported;
+    AttnArgs<TS> a{n_q, d->n_tokens, n_self, H, d->q_heads > 0 ? d->q_heads : H, scale, (const TS*)Q, Kh, Vh,
+                   (const TS*)K_self, (const TS*)V_self, (TS*)O};
+    return launch_attention(a, D, st);
+  });
+}
+
 }  // namespace
 
 extern "C" {
@@ -412,11 +444,6 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
   if (ws_bytes < need || (need && !ws)) return KVC_ERR_WORKSPACE_TOO_SMALL;
   if (n_q == 0) return KVC_OK;
   cudaStream_t st = (cudaStream_t)stream;
-  if (tc_attend_supported(d, p, n_self)) {
-    cudaError_t e = tc_attend(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, K_rec_opt,
-                              V_rec_opt, ws, ws_bytes, st);
-    return e == cudaSuccess ? KVC_OK : cuda_fail(e);
-  }
   // the clustered history's reconstruction, when asked for, is its decode (the
   // attention itself never rebuilds it)
   if (p->kind == KVC_PRED_CLUSTER && (K_rec_opt || V_rec_opt) && d->n_tokens > 0) {
@@ -432,32 +459,21 @@ kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p
     cudaError_t e = tc_mixed_attend(d, p, Q, n_q, codes, scale, O, ws, ws_bytes, st);
     return e == cudaSuccess ? KVC_OK : cuda_fail(e);
   }
-  Carve cv{(char*)ws, ws_bytes};
-  return dispatch(d, [&](auto* ts, auto* tp) -> cudaError_t {
-    using TS = std::remove_pointer_t<decltype(ts)>;
-    using TP = std::remove_pointer_t<decltype(tp)>;
-    const int H = d->n_heads, D = d->head_dim;
-    if (p->kind == KVC_PRED_CLUSTER) {
+  if (p->kind == KVC_PRED_CLUSTER) {
+    return dispatch(d, [&](auto* ts, auto* tp) -> cudaError_t {
+      using TS = std::remove_pointer_t<decltype(ts)>;
+      using TP = std::remove_pointer_t<decltype(tp)>;
+      const int H = d->n_heads, D = d->head_dim;
       MixedArgs<TS, TP> a{n_q, d->n_tokens, H, D, H * D, p->n_clusters, d->bits, d->group, scale,
                           (const TS*)Q, (const TS*)p->k_centroids, (const TS*)p->k_dec, (const TS*)p->v_centroids,
                           (const TS*)p->v_dec, (const uint8_t*)codes->k_codes, (const Pair<TP>*)codes->k_params,
                           (const uint8_t*)codes->k_assign, (const uint8_t*)codes->v_codes,
                           (const Pair<TP>*)codes->v_params, (const uint8_t*)codes->v_assign, (TS*)O};
       return launch_mixed_attention(a, st);
-    }
-    // decode the history (into the caller's outputs when given, else the
-    // workspace), then attend over [history; self]
-    const size_t bytes = (size_t)d->n_tokens * H * D * sizeof(TS);
-    TS* Kh = (TS*)cv.take(bytes);
-    TS* Vh = (TS*)cv.take(bytes);
-    if (K_rec_opt) Kh = (TS*)K_rec_opt;
-    if (V_rec_opt) Vh = (TS*)V_rec_opt;
-    cudaError_t e = codec_xlayer<TS, TP>(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh, cv, st);
-    if (e != cudaSuccess) return e;
-    AttnArgs<TS> a{n_q, d->n_tokens, n_self, H, d->q_heads > 0 ? d->q_heads : H, scale, (const TS*)Q, Kh, Vh,
-                   (const TS*)K_self, (const TS*)V_self, (TS*)O};
-    return launch_attention(a, D, st);
-  });
+    });
+  }
+  return attend_decoded(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, K_rec_opt, V_rec_opt,
+                        ws, ws_bytes, st, false);
 }
 
 kvc_status kvc_attend_compressed_debiased(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q,
@@ -467,8 +483,9 @@ kvc_status kvc_attend_compressed_debiased(const kvc_layer_desc* d, const kvc_pre
                                           void* stream) {
   kvc_status s = check_desc(d, p);
   if (s != KVC_OK) return s;
-  // the corrected softmax is written for the tensor-core cross-layer attention
-  if (!tc_attend_supported(d, p, n_self) || d->n_tokens == 0) return KVC_ERR_UNSUPPORTED;
+  // the corrected softmax is written for the tensor-core attention over an
+  // INT-coded cross-layer history
+  if (!tc_flash_debiased_supported(d, p) || d->n_tokens == 0) return KVC_ERR_UNSUPPORTED;
   if ((s = check_weights(p)) != KVC_OK) return s;
   if (n_q < 0 || n_self < 0) return KVC_ERR_INVALID_ARGUMENT;
   if (!codes_ok(p, codes) || (n_q > 0 && (!Q || !O))) return KVC_ERR_INVALID_ARGUMENT;
@@ -481,9 +498,8 @@ kvc_status kvc_attend_compressed_debiased(const kvc_layer_desc* d, const kvc_pre
   const size_t need = kvc_workspace_bytes(KVC_OP_ATTEND, d, p, n_q);
   if (ws_bytes < need || (need && !ws)) return KVC_ERR_WORKSPACE_TOO_SMALL;
   if (n_q == 0) return KVC_OK;
-  cudaError_t e = tc_attend(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, K_rec_opt, V_rec_opt,
-                            ws, ws_bytes, (cudaStream_t)stream, true);
-  return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+  return attend_decoded(d, p, Q, n_q, codes, K_src, V_src, K_self, V_self, n_self, scale, O, K_rec_opt, V_rec_opt,
+                        ws, ws_bytes, (cudaStream_t)stream, true);
 }
 
 kvc_status kvc_refit_block_diag(const kvc_layer_desc* d, const kvc_predictor* p, int tensor, const void* X0,

@@ -13,12 +13,13 @@ cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool
 bool tc_temporal_supported(const kvc_layer_desc* d, const kvc_predictor* p);
 cudaError_t tc_temporal_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
                               const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, cudaStream_t st);
-bool tc_attend_supported(const kvc_layer_desc* d, const kvc_predictor* p, int64_t n_self);
-size_t tc_attend_workspace(const kvc_layer_desc* d, const kvc_predictor* p);
-cudaError_t tc_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,
-                      const kvc_codes* c, const void* Ks, const void* Vs, const void* K_self, const void* V_self,
-                      int64_t n_self, float scale, void* O, void* K_rec, void* V_rec, void* ws, size_t ws_bytes,
-                      cudaStream_t st, bool jensen = false);
+// flash attention over a decoded bf16 history [T][H][128] and the chunk's own
+// keys; k_params non-null: the debiased variant (the history's K scale pairs)
+bool tc_flash_supported(const kvc_layer_desc* d);
+bool tc_flash_debiased_supported(const kvc_layer_desc* d, const kvc_predictor* p);
+cudaError_t tc_flash(const kvc_layer_desc* d, const void* Q, int64_t n_q, const void* Kh, const void* Vh,
+                     const void* K_self, const void* V_self, int64_t n_self, float scale, void* O,
+                     const void* k_params, cudaStream_t st);
 bool tc_mixed_supported(const kvc_layer_desc* d, const kvc_predictor* p);
 size_t tc_mixed_workspace(const kvc_layer_desc* d, int64_t n_q);
 cudaError_t tc_mixed_attend(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,

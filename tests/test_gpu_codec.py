@@ -856,7 +856,9 @@ def _check_eden(idx_g, s_g, rec_g, oc, rec_ref, pred_ref, x, cb, state, param, w
     bad = live & (np.abs(rec_g - own) > tol + err + ulp_s)
     assert not np.any(bad), f"{what}: {int(bad.sum())} values do not reconstruct their own codes"
     flip = np.repeat(gdiff, 64, axis=-1)
-    U.assert_recon_close(np.where(live, rec_g, rec_ref), rec_ref, own, x, flip | ~live, state, what + " recon")
+    # a rounding tie of the state dtype is judged with the same GPU error bound
+    U.assert_recon_close(np.where(live, rec_g, rec_ref), rec_ref, own, x, flip | ~live, state, what + " recon",
+                         err=err)
     return (gdiff.reshape(T, -1).any(1)) | (rec_g != rec_ref).reshape(T, -1).any(1)
 
 
