@@ -132,20 +132,31 @@ class XLayerBench:
         mk = lambda: torch.empty(T_TOK, H, D, dtype=bf, device=device)
         self.er = [(mk(), mk()), (mk(), mk())]  # encode-chain reconstructions (ping-pong)
         self.dr = [(mk(), mk()), (mk(), mk())]  # decode-chain reconstructions
-        self.keep = None  # (K^_14, V^_14) for the attention row
+        self.keep = None  # (K^_{l-1}, V^_{l-1}) for the attention row over layer l
+        self.attn_layer = min(15, layers - 1)  # layer 15 of 30 (a smaller run: its last layer)
 
-    def encode_chain(self, ev=None, keep_layer=None):
+    def encode_chain(self, ev=None, keep_layer=None, before=None, after=None):
+        """before(l) / after(l): hooks around the encode of layer l (the end-to-end
+        step orders its copies against them)."""
         K, V = self.wl.K, self.wl.V
         Kr, Vr = self.er[0]
+        if before:
+            before(0)
         kvc.kvc_encode_layer(self.desc0, self.pred0, K[0], V[0], None, None, self.codes[0], Kr, Vr)
+        if after:
+            after(0)
         for l in range(1, self.L):
             Ks, Vs = self.er[(l - 1) % 2]
             Kr, Vr = self.er[l % 2]
+            if before:
+                before(l)
             if ev is not None:
                 ev[l][0].record()
             kvc.kvc_encode_layer(self.desc, self.preds[l], K[l], V[l], Ks, Vs, self.codes[l], Kr, Vr, self.ws_enc)
             if ev is not None:
                 ev[l][1].record()
+            if after:
+                after(l)
             if keep_layer is not None and l == keep_layer - 1:
                 self.keep = (Kr.clone(), Vr.clone())
 
@@ -325,7 +336,7 @@ def row_attention(xb: XLayerBench, hbm, tf_burst, tf_sust, reps=3) -> dict:
     Ks = synth.queries(synth.SEED_BASE + 12, n_q, H, D, device=dev)
     Vs = synth.queries(synth.SEED_BASE + 22, n_q, H, D, device=dev)
     O_ = torch.empty(n_q, H, D, dtype=torch.bfloat16, device=dev)
-    l = 15
+    l = xb.attn_layer
     ws = kvc.alloc_workspace(kvc.OP_ATTEND, xb.desc, xb.preds[l], n_q, device=dev)
     Kh, Vh = xb.keep
     call = lambda: kvc.kvc_attend_compressed(xb.desc, xb.preds[l], Q, xb.codes[l], Kh, Vh, Ks, Vs, D ** -0.5,
@@ -373,7 +384,7 @@ def row_attention_debiased(xb: XLayerBench, hbm, tf_burst, reps=3) -> dict:
     Ks = synth.queries(synth.SEED_BASE + 12, n_q, H, D, device=dev)
     Vs = synth.queries(synth.SEED_BASE + 22, n_q, H, D, device=dev)
     O_ = torch.empty(n_q, H, D, dtype=torch.bfloat16, device=dev)
-    l = 15
+    l = xb.attn_layer
     ws = kvc.alloc_workspace(kvc.OP_ATTEND, xb.desc, xb.preds[l], n_q, device=dev)
     Kh, Vh = xb.keep
     call = lambda: kvc.kvc_attend_compressed_debiased(xb.desc, xb.preds[l], Q, xb.codes[l], Kh, Vh, Ks, Vs,
@@ -620,23 +631,44 @@ def main():
         bi = sum(t.numel() * t.element_size() for t in hK + hV)
         bo = sum(t.numel() * t.element_size() for c in hcodes for t in c)
 
-        stream = torch.cuda.current_stream()
+        comp = torch.cuda.current_stream()
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(L_RUN)]    # layer l's inputs on the device
+        ev_enc = [torch.cuda.Event() for _ in range(L_RUN)]   # layer l encoded (its inputs read, codes written)
+        ev_out = [torch.cuda.Event() for _ in range(L_RUN)]   # layer l's codes on the host
 
         def e2e_step():
-            # every byte moves through the library's C ABI: host inputs in, codes out
+            # every byte moves through the library's C ABI: host inputs in, codes out.
+            # Three streams, ordered per layer by events: the inputs of layer l+1
+            # are copied in while layer l is encoded, and the codes of layer l are
+            # copied out while the next layers run (copies in and out use the two
+            # directions of the link at once).
             for l in range(L_RUN):
-                kvc.kvc_copy_to_device(xb.wl.K[l], hK[l], stream)
-                kvc.kvc_copy_to_device(xb.wl.V[l], hV[l], stream)
-            xb.step()
-            for c, hc in zip(xb.codes, hcodes):
+                h2d.wait_event(ev_enc[l])  # the previous step's encode of layer l has read its inputs
+                kvc.kvc_copy_to_device(xb.wl.K[l], hK[l], h2d)
+                kvc.kvc_copy_to_device(xb.wl.V[l], hV[l], h2d)
+                ev_in[l].record(h2d)
+
+            def before(l):
+                comp.wait_event(ev_in[l])
+                comp.wait_event(ev_out[l])  # the previous step's codes of layer l are out
+
+            xb.encode_chain(before=before, after=lambda l: ev_enc[l].record(comp))
+            for l, (c, hc) in enumerate(zip(xb.codes, hcodes)):
+                d2h.wait_event(ev_enc[l])
                 for src, dst in zip((c.k_codes, c.k_params, c.v_codes, c.v_params), hc):
-                    kvc.kvc_copy_to_host(dst, src, stream)
+                    kvc.kvc_copy_to_host(dst, src, d2h)
+                ev_out[l].record(d2h)
+            xb.decode_chain()
+            comp.wait_stream(h2d)
+            comp.wait_stream(d2h)
 
         e2e_step()
         torch.cuda.synchronize()
         barrier()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
+        h2d.wait_stream(comp)  # the timed copies start after the start event
         for _ in range(args.e2e_steps):
             e2e_step()
         e.record()
@@ -651,8 +683,8 @@ def main():
     if world == 1:
         want = set(args.rows.split(",")) if not args.no_rows else set()
         rows = {}
-        if ("c2" in want or "c2j" in want) and L_RUN > 15:
-            xb.encode_chain(keep_layer=15)
+        if ("c2" in want or "c2j" in want) and L_RUN >= 2:
+            xb.encode_chain(keep_layer=xb.attn_layer)
             torch.cuda.synchronize()
             if "c2" in want:
                 rows["c2_attention"] = row_attention(xb, hbm, tf_burst, tf_sust)

@@ -915,9 +915,14 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       if (elected) {
         if (PAIR) mbar_arrive_remote(lead_bar(&acc_empty[b]));
         if ((!is_v || a.store_v) && t0 < a.T) {  // (a pair's odd CTA may be past the last token)
-          const CUtensorMap* m = is_v ? &maps.vo : &maps.ko;
-          tma_store(m, h * 128, t0, recon(b));
-          tma_store(m, h * 128 + 64, t0, recon(b) + 16384);
+          if (is_v) {
+            tma_store(&maps.vo, h * 128, t0, recon(b));
+            tma_store(&maps.vo, h * 128 + 64, t0, recon(b) + 16384);
+          } else {  // K^_l is read back by this tile's V heads: kept in L2 until then
+            const uint64_t keep = policy_evict_last();
+            tma_store_hint(&maps.ko, h * 128, t0, recon(b), keep);
+            tma_store_hint(&maps.ko, h * 128 + 64, t0, recon(b) + 16384, keep);
+          }
         }
         bulk_commit();
         if (!is_v && RC) {

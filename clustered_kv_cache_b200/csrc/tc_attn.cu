@@ -137,6 +137,21 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x on the FMA pipe, for the share of the softmax weights that would
+// otherwise queue on the (16 per cycle per SM) exponential unit: x = n + f with
+// n = rint(x) (the 1.5 * 2^23 addition leaves n in the low mantissa bits) and
+// f in [-0.5, 0.5]; 2^f by a cubic fitted here to the relative error of 2^f on
+// that interval (Lawson-weighted least squares on Chebyshev nodes, max relative
+// error 7.5e-5, below the 2^-9 of the bf16 the weights are rounded to); 2^n
+// added to the exponent field.  x is clamped at -126 (weights below 2^-126 are
+// kept at about 2^-126: nothing at that scale survives the fp32 sums).
+__device__ __forceinline__ float ex2_cubic(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -169,7 +184,8 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
   uint64_t* x_full = kv_empty + S;   // [S] JC: the stage's Jensen B operand written
   uint64_t* q_full = x_full + S;
   uint64_t* qx_full = q_full + 1;    // JC: the Jensen A operand written
-  uint64_t* s_full = qx_full + 1;    // [2]
+  uint64_t* q_tmem = qx_full + 1;    // Q copied into tensor memory (the softmax warps)
+  uint64_t* s_full = q_tmem + 1;     // [2]
   uint64_t* p_full = s_full + 2;     // [2]
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_done = pv_done + 1;
@@ -194,6 +210,7 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
     }
     mbar_init(q_full, 1);
     mbar_init(qx_full, 1);
+    mbar_init(q_tmem, 128);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
@@ -213,6 +230,9 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t OC = tmem + 256;
+  // Q as bf16 pairs: the A operand of S = Q K^T comes from tensor memory, so the
+  // S MMAs read only K from shared memory
+  const uint32_t QC = tmem + 384;
   auto SC = [&](int b) { return tmem + 128 * b; };
   uint8_t* Qs = smem + L::kQ;
   auto Kt = [&](int s) { return smem + L::kK + s * 32768; };
@@ -272,8 +292,7 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
     if (lane == 0) {
       const uint32_t id128 = idesc_bf16(128, 128);
       const uint32_t idv = idesc_bf16_bmn(128, 128);
-      const uint64_t qd = desc_sw128(smem_u32(Qs));
-      bool ok = wait(q_full, 0, abort_flag, a.err, 0x1310u);
+      bool ok = wait(q_tmem, 0, abort_flag, a.err, 0x1310u);
       if (JC && ok) ok = wait(qx_full, 0, abort_flag, a.err, 0x1311u);
       for (int j = 0; j <= NT && ok; ++j) {
         if (j < NT) {
@@ -287,7 +306,7 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
-            umma(SC(b), qd + off, kd + off, id128, k == 0 ? 0u : 1u);
+            umma_ts(SC(b), QC + k * 8, kd + off, id128, k == 0 ? 0u : 1u);
           }
           if (JC && j < NH)  // the Jensen term of the history keys: one K = 16 step
             umma(SC(b), desc_sw128(smem_u32(Qx)), desc_sw128(smem_u32(Kx(s))), id128, 1u);
@@ -320,6 +339,25 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(qd * 32) << 16);
     const float c = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
+    // this thread's Q row, from the 128-byte-swizzled tile, into tensor memory
+    wait(q_full, 0, abort_flag, a.err, 0x1505u);
+    {
+      uint32_t qw[64];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {  // 16-byte chunk k of the row: elements 8k .. 8k + 7
+        const uint4 u = *reinterpret_cast<const uint4*>(Qs + (k / 8) * 16384 + sw128_off(row, k % 8));
+        qw[4 * k] = u.x;
+        qw[4 * k + 1] = u.y;
+        qw[4 * k + 2] = u.z;
+        qw[4 * k + 3] = u.w;
+      }
+      uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&qw[0]);
+      uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&qw[32]);
+      tmem_st32u(lane_addr + (QC - tmem), lo);
+      tmem_st32u(lane_addr + (QC - tmem) + 32, hi);
+    }
+    tc_fence_before();
+    mbar_arrive(q_tmem);
     for (int j = 0; j < NT; ++j) {
       const int b = j & 1;
       const uint32_t sc = lane_addr + (SC(b) - tmem);
@@ -364,8 +402,12 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(sv[pc][2 * i], c, -m_used));
-          const float p1 = ex2_approx(fmaf(sv[pc][2 * i + 1], c, -m_used));
+          // a quarter of the weights on the FMA pipe balances its issue slots
+          // against the exponential unit's throughput
+          const float x0 = fmaf(sv[pc][2 * i], c, -m_used), x1 = fmaf(sv[pc][2 * i + 1], c, -m_used);
+          const bool fma_pipe = (i & 3) == 3;
+          const float p0 = fma_pipe ? ex2_cubic(x0) : ex2_approx(x0);
+          const float p1 = fma_pipe ? ex2_cubic(x1) : ex2_approx(x1);
           ls[i & 3] += p0 + p1;
           w[i] = pack_bf16x2(p0, p1);
         }

@@ -104,6 +104,13 @@ __device__ __forceinline__ void tma_store(const CUtensorMap* m, int x, int y, co
                "r"(x), "r"(y), "r"(smem_u32(src))
                : "memory");
 }
+// the same with an L2 eviction policy for the written lines
+__device__ __forceinline__ void tma_store_hint(const CUtensorMap* m, int x, int y, const void* src, uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(smem_u32(src)), "l"(policy)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }

@@ -15,7 +15,11 @@
 // frame ahead, the reconstruction out of the decode epilogues, and the supplied
 // history of a continuation call into tensor memory.
 //
-// Warp roles: 0 TMA (maps, history, x), 1 MMA + TMEM, 2-5 K epilogue, 6-9 V epilogue.
+// Warp roles: 0 TMA (maps, history, x), 1 MMA + TMEM, 2-9 K epilogue, 10-17 V
+// epilogue.  An epilogue group is eight warps: two per TMEM lane quarter, one
+// for each 64-column half of the row, so that the per-frame chain (prediction
+// MMA, then the epilogue that writes the state the next MMA reads) runs each
+// row's quantization on two warps.
 #include <cuda.h>
 #include <string.h>
 
@@ -31,7 +35,8 @@ bool map3d_frames(CUtensorMap* m, const void* base, uint64_t frames, uint64_t ro
 
 namespace temporal {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
+constexpr int kGroup = 256;  // threads of an epilogue group
 constexpr int kAK = 0;                   // AK_h as 4 sub-tiles [128 out][64 in]
 constexpr int kAV = kAK + 65536;         // AV_h
 constexpr int kX = kAV + 65536;          // three staged [128][128] bf16 tiles: x of K(f), V(f) in turn
@@ -79,6 +84,26 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16
       : "memory");
 }
 
+// 16 consecutive fp32 TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 8 consecutive 32-bit TMEM columns of this thread's lane (no wait)
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&w)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 template <bool ENC, int G>
 __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_constant__ Maps maps, const Args a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -87,13 +112,18 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
   uint64_t* w_full = bars;           // maps (+ history) landed
   uint64_t* kacc_full = bars + 1;    // K prediction of a frame in TMEM
   uint64_t* vacc_full = bars + 2;    // V prediction of a frame in TMEM
-  uint64_t* kready = bars + 3;       // K^ of a frame in its TMEM slot (K epilogue, 128 arrivals)
+  uint64_t* kready = bars + 3;       // K^ of a frame in its TMEM slot (K epilogue, 256 arrivals)
   uint64_t* vready = bars + 4;       // V^ of a frame in its TMEM slot (V epilogue)
   uint64_t* mma_done = bars + 5;
-  uint64_t* h_ready = bars + 6;      // initial history in TMEM (both epilogue groups, 256 arrivals)
-  uint64_t* x_full = bars + 7;       // [3] staged tile landed
-  uint64_t* x_free = bars + 10;      // [3] staged tile read (128 arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* h_ready = bars + 6;      // initial history in TMEM (both epilogue groups, 512 arrivals)
+  // Ring item i (x of K(f) for i = 2f, of V(f) for i = 2f + 1) lands in slot
+  // i % 3 and completes on x_full[slot][i & 1]: the slots alternate between K
+  // and V items, and a barrier that only one group waits on shows that group
+  // each of its phases in order (a parity wait cannot tell a phase from the one
+  // two later).  The j-th item of a group in a slot is item i with j = i / 6.
+  uint64_t* x_full = bars + 7;       // [3][2] staged tile landed, per slot and group
+  uint64_t* x_free = bars + 13;      // [3] staged tile read (256 arrivals; only the producer waits)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -110,13 +140,14 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
     mbar_init(w_full, 1);
     mbar_init(kacc_full, 1);
     mbar_init(vacc_full, 1);
-    mbar_init(kready, 128);
-    mbar_init(vready, 128);
+    mbar_init(kready, kGroup);
+    mbar_init(vready, kGroup);
     mbar_init(mma_done, 1);
-    mbar_init(h_ready, 256);
+    mbar_init(h_ready, 2 * kGroup);
     for (int i = 0; i < 3; ++i) {
-      mbar_init(&x_full[i], 1);
-      mbar_init(&x_free[i], 128);
+      mbar_init(&x_full[2 * i], 1);
+      mbar_init(&x_full[2 * i + 1], 1);
+      mbar_init(&x_free[i], kGroup);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -166,16 +197,17 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
           }
           const CUtensorMap* m = (i & 1) ? &maps.xv : &maps.xk;
           const int row = (int)((i >> 1) * F + s0);
-          mbar_arrive_expect_tx(&x_full[i % 3], 32768u);
-          tma_load(xs(i), m, h * 128, row, &x_full[i % 3], pol_x);
-          tma_load(xs(i) + 16384, m, h * 128 + 64, row, &x_full[i % 3], pol_x);
+          uint64_t* xf = &x_full[2 * (i % 3) + (i & 1)];
+          mbar_arrive_expect_tx(xf, 32768u);
+          tma_load(xs(i), m, h * 128, row, xf, pol_x);
+          tma_load(xs(i) + 16384, m, h * 128 + 64, row, xf, pol_x);
           last = i;
         }
         if (*abort_flag) {  // the loads this thread issued land before the CTA can leave
           for (int i = last - 2; i <= last; ++i) {
             if (i < 0) continue;
             const long long w0 = clock64();
-            while (!mbar_test(&x_full[i % 3], (i / 3) & 1) && clock64() - w0 < kWaitBudget) {
+            while (!mbar_test(&x_full[2 * (i % 3) + (i & 1)], (i / 6) & 1) && clock64() - w0 < kWaitBudget) {
             }
           }
         }
@@ -227,9 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       }
     }
   } else {
-    // ================================================================ epilogues: warps 2-5 K, 6-9 V
-    const bool isv = warp >= 6;
-    const int q = warp & 3;
+    // ================================================================ epilogues: warps 2-9 K, 10-17 V
+    const bool isv = warp >= 10;
+    const int q = warp & 3;                  // TMEM lane quarter
+    const int hc = ((warp - 2) >> 2) & 1;    // 64-column half of the row
     const int row = q * 32 + lane;
     const int64_t s = s0 + row;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
@@ -238,38 +271,38 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
     int acc_use = 0;
     const int64_t F0 = cont ? 0 : (F < a.T ? F : a.T);
     const int arb = 128 * a.anchor_bits / 8;
-    // row r of a staged [128][128] bf16 tile (two 128-byte-swizzled 64-column sub-tiles) as 64 words
-    auto read_row = [&](const uint8_t* tile, uint4 (&w)[16]) {
+    // this thread's half of row r of a staged [128][128] bf16 tile (two
+    // 128-byte-swizzled 64-column sub-tiles: the half is sub-tile hc) as 32 words
+    auto read_half = [&](const uint8_t* tile, uint4 (&w)[8]) {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) w[c] = *reinterpret_cast<const uint4*>(tile + (c / 8) * 16384 + sw128_off(row, c % 8));
+      for (int c = 0; c < 8; ++c) w[c] = *reinterpret_cast<const uint4*>(tile + hc * 16384 + sw128_off(row, c));
     };
-    auto row_to_tmem = [&](const uint4 (&w)[16], uint32_t col) {
+    auto half_to_tmem = [&](const uint4 (&w)[8], uint32_t col) {
       const uint32_t* u = reinterpret_cast<const uint32_t*>(w);
-      uint32_t lo[32], hi[32];
+      uint32_t v[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) lo[i] = u[i], hi[i] = u[32 + i];
-      tmem_st32u(lane_off + col, lo);
-      tmem_st32u(lane_off + col + 32, hi);
+      for (int i = 0; i < 32; ++i) v[i] = u[i];
+      tmem_st32u(lane_off + col + hc * 32, v);
     };
     // the state before frame 0: the supplied history, or (no history) a zero
     // K^ of frame -1 as the lag-2 input of frame 1
     wait(w_full, 0, abort_flag, a.err, 0x2200u);
     if (cont) {
-      uint4 w[16];
+      uint4 w[8];
       if (!isv) {
-        read_row(xs(0), w);
-        row_to_tmem(w, KH(-1) - tmem);
-        read_row(xs(1), w);
-        row_to_tmem(w, KH(-2) - tmem);
+        read_half(xs(0), w);
+        half_to_tmem(w, KH(-1) - tmem);
+        read_half(xs(1), w);
+        half_to_tmem(w, KH(-2) - tmem);
       } else {
-        read_row(xs(2), w);
-        row_to_tmem(w, VH - tmem);
+        read_half(xs(2), w);
+        half_to_tmem(w, VH - tmem);
       }
     } else if (!isv) {
-      uint4 w[16];
+      uint4 w[8];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) w[i] = make_uint4(0, 0, 0, 0);
-      row_to_tmem(w, KH(-1) - tmem);
+      for (int i = 0; i < 8; ++i) w[i] = make_uint4(0, 0, 0, 0);
+      half_to_tmem(w, KH(-1) - tmem);
     }
     tc_fence_before();
     mbar_arrive(h_ready);
@@ -279,14 +312,16 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
     __nv_bfloat16* rec = isv ? a.vrec : a.krec;
     const bool stage = !ENC && rec != nullptr;
     uint8_t* stile = xs(isv ? 2 : 0);
-    const bool elected = warp == (isv ? 6 : 2) && lane == 0;
+    const bool elected = warp == (isv ? 10 : 2) && lane == 0;
     auto gsync = [&] {
       if (isv)
-        asm volatile("bar.sync 2, 128;" ::: "memory");
+        asm volatile("bar.sync 2, 256;" ::: "memory");
       else
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
     };
     const int64_t nff = a.T / F;  // whole frames
+    constexpr int NG = 128 / G, NP = G / 32;
+    constexpr int NGH = NG / 2;  // groups of the half row
     for (int f = 0; f < nf; ++f) {
       const int64_t n_f = (a.T - f * F) < F ? (a.T - f * F) : F;
       const bool valid = s < n_f;
@@ -296,25 +331,25 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       const int64_t t = f * F + s;
       const int64_t rowi = t * H + h;
       const int row_bytes = 128 * bits / 8;
+      const int half_bytes = row_bytes / 2;
       const int64_t cofs = rowi < F0 * H ? rowi * arb : F0 * H * arb + (rowi - F0 * H) * row_bytes;
-      uint8_t* codes = (isv ? a.vcodes : a.kcodes) + cofs;
-      __half2* params = (isv ? a.vparams : a.kparams) + rowi * (128 / G);
-      constexpr int NG = 128 / G, NP = G / 32;
-      uint4 xin[16];
-      uint4 cin[4];
-      __half2 pin[NG];
-      if (ENC) {  // x of this row from the staged tile, which is then released
+      uint8_t* codes = (isv ? a.vcodes : a.kcodes) + cofs + hc * half_bytes;
+      __half2* params = (isv ? a.vparams : a.kparams) + rowi * NG + hc * NGH;
+      uint4 xin[8];
+      uint4 cin[2];
+      __half2 pin[NGH];
+      if (ENC) {  // x of this half row from the staged tile, which is then released
         const int i = 2 * f + (isv ? 1 : 0);
-        wait(&x_full[i % 3], (i / 3) & 1, abort_flag, a.err, 0x2220u + isv);
-        read_row(xs(i), xin);
+        wait(&x_full[2 * (i % 3) + (i & 1)], (i / 6) & 1, abort_flag, a.err, 0x2220u + isv);
+        read_half(xs(i), xin);
         mbar_arrive(&x_free[i % 3]);
       } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          cin[i] = (valid && i * 16 < row_bytes) ? __ldcs(reinterpret_cast<const uint4*>(codes) + i)
-                                                 : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 2; ++i)
+          cin[i] = (valid && i * 16 < half_bytes) ? __ldcs(reinterpret_cast<const uint4*>(codes) + i)
+                                                  : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int g = 0; g < NG; ++g) pin[g] = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
+        for (int g = 0; g < NGH; ++g) pin[g] = valid ? params[g] : __floats2half2_rn(0.f, 0.f);
       }
       // V(f) reads K^_f: the V epilogue of frame f starts after the K epilogue of f
       if (!anchor) {
@@ -324,30 +359,31 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       }
       // the new state goes to the slot its own prediction was the last to read
       const uint32_t state = lane_off + (isv ? VH : KH(f));
-      uint32_t cw[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
+      uint32_t cw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       const uint32_t* cwin = reinterpret_cast<const uint32_t*>(cin);
       if (stage) {  // the staged tile's previous store has read it
         if (elected) bulk_wait_read0();
         gsync();
       }
 #pragma unroll
-      for (int g = 0; g < NG; ++g) {
+      for (int gh = 0; gh < NGH; ++gh) {
+        const int g = hc * NGH + gh;  // group of the row
         float sf, zf;
         if (ENC) {
           float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-          for (int pc = 0; pc < NP; ++pc) {
-            float p[32];
+          for (int pc = 0; pc < 2 * NP; ++pc) {  // 16 columns at a time (the register budget)
+            float p[16];
             if (anchor) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) p[i] = 0.f;
+              for (int i = 0; i < 16; ++i) p[i] = 0.f;
             } else {
-              tmem_ld32(acc_addr + g * G + pc * 32, p);
+              tmem_ld16(acc_addr + g * G + pc * 16, p);
             }
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
               float x[8];
-              unpack_bf16x8(xin[(g * G + pc * 32) / 8 + ch], x, 0);
+              unpack_bf16x8(xin[(gh * G + pc * 16) / 8 + ch], x, 0);
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const float r = x[i] - p[ch * 8 + i];
@@ -360,27 +396,28 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
           const __half zh = __float2half_rn(mn);
           sf = __half2float(sh);
           zf = __half2float(zh);
-          if (valid) params[g] = __halves2half2(sh, zh);
+          if (valid) params[gh] = __halves2half2(sh, zh);
         } else {
-          const float2 fz = __half22float2(pin[g]);
+          const float2 fz = __half22float2(pin[gh]);
           sf = fz.x;
           zf = fz.y;
         }
         const float inv = sf > 0.f ? 1.f / sf : 0.f;
 #pragma unroll
-        for (int pc = 0; pc < NP; ++pc) {
-          const int e0 = g * G + pc * 32;
-          float p[32];
+        for (int pc = 0; pc < 2 * NP; ++pc) {
+          const int e0 = g * G + pc * 16;   // element of the row
+          const int h0 = gh * G + pc * 16;  // element of the half row
+          float p[16];
           if (anchor) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) p[i] = 0.f;
+            for (int i = 0; i < 16; ++i) p[i] = 0.f;
           } else {
-            tmem_ld32(acc_addr + e0, p);
+            tmem_ld16(acc_addr + e0, p);
           }
-          uint32_t recw[16];  // 32 reconstructed values as bf16 pairs
+          uint32_t recw[8];  // 16 reconstructed values as bf16 pairs
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int e = e0 + ch * 8;
+          for (int ch = 0; ch < 2; ++ch) {
+            const int e = h0 + ch * 8;
             float r[8];  // reconstruction
             if (ENC) {
               float x[8];
@@ -399,10 +436,10 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
             for (int i = 0; i < 4; ++i) recw[ch * 4 + i] = pack_bf16x2(r[2 * i], r[2 * i + 1]);
           }
           // the slot was last read by this frame's prediction, which is complete (acc_full)
-          tmem_st16(state + e0 / 2, recw);
+          tmem_st8(state + e0 / 2, recw);
           if (stage) {
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
               const int e = e0 + ch * 8;
               *reinterpret_cast<uint4*>(stile + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =
                   make_uint4(recw[4 * ch], recw[4 * ch + 1], recw[4 * ch + 2], recw[4 * ch + 3]);
@@ -410,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
           } else if (rec && valid) {
             uint4* dst = reinterpret_cast<uint4*>(rec + t * C + h * 128 + e0);
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch)
+            for (int ch = 0; ch < 2; ++ch)
               dst[ch] = make_uint4(recw[4 * ch], recw[4 * ch + 1], recw[4 * ch + 2], recw[4 * ch + 3]);
           }
         }
@@ -418,8 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       if (ENC && valid) {
         uint4* dst = reinterpret_cast<uint4*>(codes);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (i * 16 < row_bytes) dst[i] = make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]);
+        for (int i = 0; i < 2; ++i)
+          if (i * 16 < half_bytes) dst[i] = make_uint4(cw[4 * i], cw[4 * i + 1], cw[4 * i + 2], cw[4 * i + 3]);
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();

@@ -20,7 +20,10 @@ pytestmark = pytest.mark.gpu
 KVC_ERR_DEVICE_TIMEOUT = 6
 
 
-def test_bounded_wait_runs_out_and_reports_a_timeout():
+@pytest.mark.parametrize("op", ["encode", "decode"])
+def test_bounded_wait_runs_out_and_reports_a_timeout(op):
+    """Encode runs single CTAs, decode CTA pairs (whose loads complete on the
+    pair leader's barriers): both give up, report and leave the context usable."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from clustered_kv_cache_b200 import build
@@ -33,27 +36,33 @@ def test_bounded_wait_runs_out_and_reports_a_timeout():
     pred = kvc.make_predictor(kvc.PRED_XLAYER_DPLR, {k: v.cuda() for k, v in wl.weights[1].items()}, rank=r)
     K, V, Ks, Vs = (t.cuda() for t in (wl.K[1], wl.V[1], wl.K[0], wl.V[0]))
     ws = kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred)
-
-    def encode():
-        buf = kvc.alloc_codes(desc, pred)
-        Kr, Vr = torch.empty_like(K), torch.empty_like(V)
-        kvc.kvc_encode_layer(desc, pred, K, V, Ks, Vs, buf, Kr, Vr, ws)
-        return buf, Kr, Vr
-
+    ref = kvc.alloc_codes(desc, pred)
+    Kr0, Vr0 = torch.empty_like(K), torch.empty_like(V)
     # a clean launch first: the reference result, and no error pending
-    ref, Kr0, Vr0 = encode()
+    kvc.kvc_encode_layer(desc, pred, K, V, Ks, Vs, ref, Kr0, Vr0, ws)
     assert kvc.kvc_get_device_error() == 0
+
+    def run():
+        if op == "encode":
+            buf = kvc.alloc_codes(desc, pred)
+            Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+            kvc.kvc_encode_layer(desc, pred, K, V, Ks, Vs, buf, Kr, Vr, ws)
+            return buf, Kr, Vr
+        Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+        kvc.kvc_decode_layer(desc, pred, ref, Ks, Vs, Kr, Vr, kvc.alloc_workspace(kvc.OP_DECODE, desc, pred))
+        return ref, Kr, Vr
+
     # the faulted launch: the launch itself succeeds, the bounded wait runs out on the device
     kvc.kvc_testing_inject_stall(1)
     t0 = time.perf_counter()
-    encode()
+    run()
     status = kvc.kvc_get_device_error()  # synchronizes the stream
     elapsed = time.perf_counter() - t0
     assert status == KVC_ERR_DEVICE_TIMEOUT, status
     assert elapsed < 60.0, elapsed
     # read-and-clear: nothing pending now, and the hook was one-shot
     assert kvc.kvc_get_device_error() == 0
-    buf, Kr, Vr = encode()
+    buf, Kr, Vr = run()
     assert kvc.kvc_get_device_error() == 0
     assert torch.equal(Kr, Kr0) and torch.equal(Vr, Vr0)
     assert torch.equal(buf.k_codes, ref.k_codes) and torch.equal(buf.v_codes, ref.v_codes)
