@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       half_to_tmem(w, KH(-1) - tmem);
     }
     tc_fence_before();
+    fence_async_smem();  // (continuation) the history slots are read; TMA loads x into them next
     mbar_arrive(h_ready);
     // Decode writes the reconstruction through a staged tile (K: slot 0, V: slot
     // 2, idle in decode once the history is in TMEM) and TMA stores of one frame's
@@ -342,6 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
         const int i = 2 * f + (isv ? 1 : 0);
         wait(&x_full[2 * (i % 3) + (i & 1)], (i / 6) & 1, abort_flag, a.err, 0x2220u + isv);
         read_half(xs(i), xin);
+        // the next TMA load into this slot is an async-proxy write: order this
+        // thread's generic reads of the slot before it
+        fence_async_smem();
         mbar_arrive(&x_free[i % 3]);
       } else {
 #pragma unroll
