@@ -46,11 +46,12 @@ UNIT = "KV tokens/s"
 # profiles/ (codec_xlayer_wan_layer.md, attention_cluster_wan.md,
 # mixed_attention_cluster.md, cluster_codec_decode.md, temporal_codec_layer.md);
 # set to None when a kernel changes after its capture.
-TRAFFIC = {"encode_xlayer": None, "decode_xlayer": None,
-           "attention_c2": None, "attention_c4": 26443520 + 146944,
+TRAFFIC = {"encode_xlayer": 676536064 + 187995648, "decode_xlayer": 431820800 + 138174976,
+           "attention_c2": 244925696 + 13229312, "attention_c4": 26443520 + 146944,
            "decode_c4": 4399616 + 80381696 + 4467712 + 80104704,
-           "temporal_encode": None,
-           "temporal_decode": 574324480 + 1285428224}
+           "temporal_encode": 1434010000 + 372614912,
+           "temporal_decode": 574324480 + 1285428224,
+           "eden2_encode": 664999168 + 177946880}
 
 
 def peaks():
@@ -370,9 +371,11 @@ def row_attention(xb: XLayerBench, hbm, tf_burst, tf_sust, reps=3) -> dict:
     return {"workload": "4680 queries x (32760 compressed + 4680 chunk) keys, 12 heads x 128, layer 15",
             "ms": ms, "value": tflops, "unit": "TFLOP/s (attention + one decode of the history)",
             "decode_ms": ms_dec, "attention_kernel_ms": ms_attn,
-            "attention_kernel": {"achieved": tf_attn, "unit": "TFLOP/s", "frac": tf_attn / tf_burst},
+            "attention_kernel": {"achieved": tf_attn, "unit": "TFLOP/s", "frac": tf_attn / tf_burst,
+                                 "traffic": TRAFFIC["attention_c2"]},
             "roofline": {"bound": "tensor", "achieved": tflops, "peak": tf_burst, "unit": "TFLOP/s",
-                         "frac": tflops / tf_burst, "traffic": TRAFFIC["attention_c2"], "peak_kind": "burst bf16"}}
+                         "frac": tflops / tf_burst, "traffic": TRAFFIC["attention_c2"] + TRAFFIC["decode_xlayer"],
+                         "peak_kind": "burst bf16"}}
 
 
 def row_attention_debiased(xb: XLayerBench, hbm, tf_burst, reps=3) -> dict:
@@ -438,7 +441,7 @@ def row_eden2(dev, hbm, reps=3) -> dict:
         byts = 2 * T_TOK * C * 2 * nio + kvc.kvc_codes_bytes(desc, pred) + w
         gbs = byts / (ms * 1e-3) / 1e9
         out[name] = {"ms": ms, "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                                            "frac": gbs / hbm, "traffic": None}}
+                                            "frac": gbs / hbm, "traffic": TRAFFIC.get("eden2_" + name)}}
     return out
 
 

@@ -220,17 +220,18 @@ KVC_API kvc_status kvc_decode_layer(const kvc_layer_desc* desc, const kvc_predic
  * followed by n_self uncompressed tokens K_self / V_self [n_self][H][D]
  * (non-causal; n_self may be 0 and the pointers NULL):
  *   O = softmax(scale * Q [K_hist; K_self]^T) [V_hist; V_self].
- * NONE / XLAYER: the history is decoded tile by tile on chip (bf16, D = 128:
- * never written to device memory).  CLUSTER: scores and values are computed on
- * the stored coefficients, q.c_a + (W_dec^T q).coef, without rebuilding full
- * keys ("NanoKV ...", abstract: the Fast variant); n_self must be 0.
- * TEMPORAL: KVC_ERR_UNSUPPORTED.  O [n_q][H][D] is written.
+ * NONE / XLAYER: the history is decoded once (the codec's decode, into
+ * K_rec_opt / V_rec_opt when given, else into the workspace) and attended with
+ * the chunk's own keys (bf16, D = 128: a tensor-core flash attention).  CLUSTER:
+ * scores and values are computed on the stored coefficients, q.c_a +
+ * (W_dec^T q).coef, without rebuilding full keys ("NanoKV ...", abstract: the
+ * Fast variant); n_self must be 0.  TEMPORAL: KVC_ERR_UNSUPPORTED.
+ * O [n_q][H][D] is written.
  *  K_rec_opt, V_rec_opt: optional [T][H][D] outputs (NULL = not wanted) that
  *    receive the decoded history, the same values kvc_decode_layer writes,
- *    e.g. as the next layer's K_src / V_src.  For NONE / XLAYER on the
- *    tensor-core path they are stored from the tiles the attention decodes
- *    on chip anyway; CLUSTER runs its decode for them.  With n_q = 0 the call
- *    does nothing at all (kvc_decode_layer decodes a history alone). */
+ *    e.g. as the next layer's K_src / V_src; CLUSTER runs its decode for them.
+ *    With n_q = 0 the call does nothing at all (kvc_decode_layer decodes a
+ *    history alone). */
 KVC_API kvc_status kvc_attend_compressed(const kvc_layer_desc* desc, const kvc_predictor* pred, const void* Q,
                                  int64_t n_q, const kvc_codes* codes, const void* K_src, const void* V_src,
                                  const void* K_self, const void* V_self, int64_t n_self, float scale,
@@ -249,8 +250,9 @@ KVC_API kvc_status kvc_attend_compressed(const kvc_layer_desc* desc, const kvc_p
  * uniform rounding error of step s, which the correction removes in
  * expectation.  It reads only the stored scales (no extra memory).  Same
  * arguments and outputs as kvc_attend_compressed; implemented for the
- * tensor-core cross-layer path (KVC_PRED_XLAYER_DPLR, bf16, head_dim 128,
- * fp16 params, T > 0); other layers return KVC_ERR_UNSUPPORTED. */
+ * tensor-core attention over a cross-layer history with scalar residual codes
+ * (KVC_PRED_XLAYER_DPLR, KVC_RESIDUAL_RTN, bf16, head_dim 128, fp16 params,
+ * group 32 or 64, T > 0); other layers return KVC_ERR_UNSUPPORTED. */
 KVC_API kvc_status kvc_attend_compressed_debiased(const kvc_layer_desc* desc, const kvc_predictor* pred,
                                                   const void* Q, int64_t n_q, const kvc_codes* codes,
                                                   const void* K_src, const void* V_src, const void* K_self,
