@@ -376,6 +376,50 @@ kvc_status attend_decoded(const kvc_layer_desc* d, const kvc_predictor* p, const
   });
 }
 
+// A chain of predicted layers: layer i of the call predicts from layer i-1's
+// reconstruction (K_src / V_src for i = 0).  One persistent launch on the
+// tensor cores where every layer is supported there, else the layers in turn.
+kvc_status layers_common(const kvc_layer_desc* d, const kvc_predictor* preds, int n, bool enc,
+                         const void* const* K, const void* const* V, const void* K_src, const void* V_src,
+                         const kvc_codes* c, void* const* K_rec, void* const* V_rec, void* ws, size_t ws_bytes,
+                         void* stream) {
+  if (!d || !preds || n < 1 || !c || !K_rec || !V_rec || !K_src || !V_src) return KVC_ERR_INVALID_ARGUMENT;
+  if (enc && (!K || !V)) return KVC_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < n; ++i) {
+    kvc_status s = check_desc(d, &preds[i]);
+    if (s != KVC_OK) return s;
+    if (preds[i].kind != KVC_PRED_XLAYER_DPLR) return KVC_ERR_UNSUPPORTED;
+    if ((s = check_weights(&preds[i])) != KVC_OK) return s;
+    if ((s = check_codebook(d, &preds[i])) != KVC_OK) return s;
+    if (!codes_ok(&preds[i], &c[i])) return KVC_ERR_INVALID_ARGUMENT;
+    if (!codes_aligned(&preds[i], &c[i])) return KVC_ERR_MISALIGNED;
+    if (!K_rec[i] || !V_rec[i] || (enc && (!K[i] || !V[i]))) return KVC_ERR_INVALID_ARGUMENT;
+    const void* ptrs[] = {K_rec[i], V_rec[i], enc ? K[i] : nullptr, enc ? V[i] : nullptr};
+    for (const void* q : ptrs)
+      if (q && !aligned16(q)) return KVC_ERR_MISALIGNED;
+    // a layer's reconstruction is the next layer's source: it may not overwrite its own source
+    const void* ks = i ? K_rec[i - 1] : K_src;
+    const void* vs = i ? V_rec[i - 1] : V_src;
+    if (K_rec[i] == ks || V_rec[i] == vs || K_rec[i] == V_rec[i]) return KVC_ERR_INVALID_ARGUMENT;
+  }
+  if (!aligned16(K_src) || !aligned16(V_src) || (ws && !aligned16(ws))) return KVC_ERR_MISALIGNED;
+  const size_t need = kvc_layers_workspace_bytes(enc ? KVC_OP_ENCODE : KVC_OP_DECODE, d, preds, n);
+  if (ws_bytes < need || (need && !ws)) return KVC_ERR_WORKSPACE_TOO_SMALL;
+  if (d->n_tokens == 0) return KVC_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (tc_codec_layers_supported(d, preds, n)) {
+    cudaError_t e = tc_codec_layers(d, preds, n, enc, K, V, K_src, V_src, c, K_rec, V_rec, ws, ws_bytes, st);
+    return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+  }
+  for (int i = 0; i < n; ++i) {
+    const void* ks = i ? K_rec[i - 1] : K_src;
+    const void* vs = i ? V_rec[i - 1] : V_src;
+    kvc_status s = codec_common(d, &preds[i], enc, enc ? K[i] : nullptr, enc ? V[i] : nullptr, ks, vs, &c[i],
+                                K_rec[i], V_rec[i], ws, ws_bytes, stream);
+    if (s != KVC_OK) return s;
+  }
+  return KVC_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -418,6 +462,33 @@ kvc_status kvc_decode_layer(const kvc_layer_desc* desc, const kvc_predictor* pre
                             const void* K_src, const void* V_src, void* K_rec, void* V_rec, void* ws, size_t ws_bytes,
                             void* stream) {
   return codec_common(desc, pred, false, nullptr, nullptr, K_src, V_src, codes, K_rec, V_rec, ws, ws_bytes, stream);
+}
+
+size_t kvc_layers_workspace_bytes(int op, const kvc_layer_desc* desc, const kvc_predictor* preds, int n_layers) {
+  if (!desc || !preds || n_layers < 1 || (op != KVC_OP_ENCODE && op != KVC_OP_DECODE)) return 0;
+  size_t per = 0;
+  for (int i = 0; i < n_layers; ++i) {
+    if (check_desc(desc, &preds[i]) != KVC_OK) return 0;
+    const size_t w = kvc_workspace_bytes(op, desc, &preds[i], 0);
+    per = w > per ? w : per;
+  }
+  const size_t fused = tc_codec_layers_supported(desc, preds, n_layers) ? tc_codec_layers_workspace(desc, n_layers) : 0;
+  return fused > per ? fused : per;
+}
+
+
+kvc_status kvc_encode_layers(const kvc_layer_desc* desc, const kvc_predictor* preds, int n_layers,
+                             const void* const* K, const void* const* V, const void* K_src, const void* V_src,
+                             const kvc_codes* out, void* const* K_rec, void* const* V_rec, void* ws,
+                             size_t ws_bytes, void* stream) {
+  return layers_common(desc, preds, n_layers, true, K, V, K_src, V_src, out, K_rec, V_rec, ws, ws_bytes, stream);
+}
+
+kvc_status kvc_decode_layers(const kvc_layer_desc* desc, const kvc_predictor* preds, int n_layers,
+                             const kvc_codes* codes, const void* K_src, const void* V_src, void* const* K_rec,
+                             void* const* V_rec, void* ws, size_t ws_bytes, void* stream) {
+  return layers_common(desc, preds, n_layers, false, nullptr, nullptr, K_src, V_src, codes, K_rec, V_rec, ws,
+                       ws_bytes, stream);
 }
 
 kvc_status kvc_attend_compressed(const kvc_layer_desc* d, const kvc_predictor* p, const void* Q, int64_t n_q,

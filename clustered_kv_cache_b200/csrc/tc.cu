@@ -30,6 +30,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <vector>
 
 #include "../../include/kvc_testing.h"
 #include "tc.h"
@@ -84,17 +85,34 @@ struct Maps {
   CUtensorMap xk, xv, ck, cv, pk, pv;
 };
 
-struct Args {
-  unsigned* err;  // device error word
-  int64_t T;
-  int H, bits;
+// the per-layer buffers of a call
+struct Ptrs {
   const __nv_bfloat16* xk;  // clean K (encode)
   const __nv_bfloat16* xv;  // clean V (encode)
   uint8_t* kcodes;
   __half2* kparams;
   uint8_t* vcodes;
   __half2* vparams;
+};
+
+// one layer of a multi-layer call, in device memory (tensor maps 64-byte aligned)
+struct alignas(64) LayerDev {
+  Maps maps;
+  Ptrs p;
+};
+
+struct Args {
+  unsigned* err;  // device error word
+  int64_t T;
+  int H, bits;
+  Ptrs p;
   int store_v;  // V^_l is written (always for decode)
+  // multi-layer calls: the layers' maps and buffers, and one counter per
+  // (layer, tile) that the tile's epilogue groups raise once its reconstruction
+  // is stored (the next layer's tile waits for it)
+  const LayerDev* layers;
+  int n_layers;
+  unsigned* flags;
   // test hook (kvc_testing_inject_stall): 1 = CTA 0's producer leaves its first
   // stage unarmed, so that the consumer's bounded wait runs out
   int inject;
@@ -135,7 +153,7 @@ __device__ __forceinline__ void walsh64_thread(float (&v)[64]) {
 
 // ---------------------------------------------------------------- the kernel
 
-template <int MODE, int G, int RC, int BITS, bool PAIR, bool EDEN>
+template <int MODE, int G, int RC, int BITS, bool PAIR, bool EDEN, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_constant__ Maps maps, const Args a) {
   constexpr bool ENC = MODE == kEncode;
   static_assert(!EDEN || (G == 64 && BITS == 2), "EDEN-2 codes 64-value groups at 4 bits a pair");
@@ -159,12 +177,22 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_cb = reinterpret_cast<float*>(smem + L::kBarOff + 512);  // EDEN-2 codebook
+  // item hand-off ring of a dynamically scheduled call: slot k & 3 holds the k-th
+  // item of this CTA (-1: none) and whether its K latent was loaded ahead
+  uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff + 256);  // [4]
+  volatile int* s_item = reinterpret_cast<volatile int*>(smem + L::kBarOff + 288);  // [4]
+  volatile int* s_pf = s_item + 4;                                                 // [4]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H;
   const int C = H * 128;
   const int NCH = C / 64;
-  // persistent CTAs: this CTA codes tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+  // persistent CTAs: this CTA codes items blockIdx.x, blockIdx.x + gridDim.x, ...
+  // An item is a tile of one layer; a multi-layer call orders them layer by
+  // layer, and the tile of layer l waits for the same tile of layer l-1.  A
+  // multi-layer call of single CTAs (DYN) instead takes its items in that order
+  // from a global ticket counter as it goes, so that a CTA slowed by a wait
+  // codes fewer items rather than holding up a fixed share.
   // A pair (cluster of two) codes 256-token tiles: the even CTA (the leader,
   // which issues the MMAs) its first 128 tokens, the odd one the rest.
   const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
@@ -173,13 +201,38 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   const int nunits = (int)(PAIR ? gridDim.x >> 1 : gridDim.x);
   const int span = PAIR ? 256 : 128;
   const int ntiles = (int)((a.T + span - 1) / span);
-  const int my_tiles = unit < ntiles ? (ntiles - 1 - unit) / nunits + 1 : 0;
-  auto tile_t0 = [&](int it) { return (unit + it * nunits) * span + (int)crank * 128; };
+  const int nitems = (MULTI ? a.n_layers : 1) * ntiles;
+  const int my_tiles = unit < nitems ? (nitems - 1 - unit) / nunits + 1 : 0;  // items of this CTA
+  constexpr bool DYN = MULTI && !PAIR;
+  auto item_of = [&](int it) { return unit + it * nunits; };  // the static order
+  auto tile_t0 = [&](int i) { return (i % ntiles) * span + (int)crank * 128; };
+  auto layer_of = [&](int i) { return MULTI ? i / ntiles : 0; };
+  // the maps and buffers of a layer (a single-layer launch has them as arguments)
+  auto LM = [&](int l) -> const Maps* {
+    if constexpr (MULTI) return &a.layers[l].maps;
+    else return &maps;
+  };
+  auto LP = [&](int l) -> const Ptrs& {
+    if constexpr (MULTI) return a.layers[l].p;
+    else return a.p;
+  };
+  // a tile's counter reaches flag_full once every epilogue group coding it has
+  // stored its reconstruction
+  constexpr unsigned flag_full = PAIR ? 4u : 2u;
+  auto flag_of = [&](int l, int i) { return a.flags + (size_t)l * ntiles + i % ntiles; };
+  unsigned* ticket = a.flags + (size_t)(MULTI ? a.n_layers : 0) * ntiles;  // DYN: next item to take
   // the leader's barriers, as shared::cluster addresses (a pair's arrivals and TMA bytes land there)
   auto lead_bar = [&](uint64_t* b) { return PAIR ? mapa_rank(b, crank & ~1u) : smem_u32(b); };
   // With rank 64 the TMEM has room for two latent slots, so the next tile's K
   // latent streams in during this tile's V heads.
   constexpr bool OVL = RC == 1;
+  // The next item's K latent is loaded during this item's V heads.  In a
+  // multi-layer call that needs the next item's own dependency first.  With the
+  // static order it is an earlier item (no cycle of waits) only while the grid
+  // has fewer units than a layer has tiles, so with more the overlap is off; with
+  // DYN the dependency is only tested, and an item whose dependency is not yet
+  // stored loads its latent when it starts.
+  const bool ovl = OVL && (DYN || !MULTI || nunits < ntiles);
   const int HH = 2 * H;  // heads per tile (K then V)
 
   if (threadIdx.x == 0) {
@@ -199,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     mbar_init(z_ready, PAIR ? 2 : kGroupThreads);
     mbar_init(khat_stored, 2);
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&item_bar[i], 1);
     *abort_flag = 0;
     if (EDEN)
       for (int i = 0; i < 32; ++i) s_cb[i] = a.codebook[i];
@@ -227,6 +281,21 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   auto stageB = [&](int s) { return smem + L::kStageOff + s * L::kStage + 16384; };
   auto recon = [&](int b) { return smem + L::kReconOff + b * L::kRecon; };
   const uint32_t in_base = smem_u32(smem + L::kInOff);
+  // DYN: wait until the producer has published this CTA's k-th item.  The wait
+  // does not end on an abort (the producer publishes a closing -1 on every path,
+  // and all threads of a group must walk the same items); it has a bound of its
+  // own, four times the producer's, which is longer than any producer wait.
+  auto item_wait = [&](int k) -> bool {
+    const long long w0 = clock64();
+    while (!mbar_test(&item_bar[k & 3], (k >> 2) & 1)) {
+      if (clock64() - w0 > 4 * kWaitBudget) {
+        *abort_flag = 1;
+        atomicCAS(a.err, 0u, 0xB10u);
+        return false;
+      }
+    }
+    return true;
+  };
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -301,52 +370,125 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       };
       const uint32_t wbytes = R * 128;
       constexpr int rbytes = 128 * BITS / 8;
-      for (int it = 0; it < my_tiles && ok; ++it) {
-        const int t0 = tile_t0(it);
-        const int nt0 = it + 1 < my_tiles ? tile_t0(it + 1) : -1;
+      // Multi-layer calls: before the first load of an item that reads layer
+      // l-1's reconstruction, the same tile of layer l-1 must be stored (bounded
+      // wait on its counter, then a proxy fence for the TMA loads that follow)
+      auto dep_wait = [&](int i) {
+        if constexpr (MULTI) {
+          const int l = layer_of(i);
+          if (l == 0 || !ok) return;
+          const unsigned* f = flag_of(l - 1, i);
+          const long long w0 = clock64();
+          unsigned v;
+          while (true) {
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+            if (v >= flag_full) break;
+            if (*abort_flag) {
+              ok = false;
+              return;
+            }
+            if (clock64() - w0 > kWaitBudget) {
+              *abort_flag = 1;
+              atomicCAS(a.err, 0u, 0xB00u);
+              ok = false;
+              return;
+            }
+          }
+          fence_async_global();
+        }
+      };
+      // DYN: one test of an item's dependency (no wait)
+      auto dep_ready = [&](int i) -> bool {
+        const int l = layer_of(i);
+        if (l == 0) return true;
+        unsigned v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag_of(l - 1, i)) : "memory");
+        if (v < flag_full) return false;
+        fence_async_global();
+        return true;
+      };
+      auto take = [&]() -> int {
+        if (!ok) return -1;
+        const int i = (int)atomicAdd(ticket, 1u);
+        return i < nitems ? i : -1;
+      };
+      int npub = 0;           // DYN: items published (the last may be the closing -1)
+      bool pub_open = false;  // the last one published is an item, not -1
+      auto publish = [&](int i, bool pf) {
+        s_item[npub & 3] = i;
+        s_pf[npub & 3] = pf ? 1 : 0;
+        mbar_arrive(&item_bar[npub & 3]);  // release: the slot is written before the phase completes
+        ++npub;
+        pub_open = i >= 0;
+      };
+      int cur = DYN ? take() : (my_tiles > 0 ? item_of(0) : -1);
+      bool cur_pf = false;  // the current item's K latent was loaded during the previous item
+      if (DYN) publish(cur, false);
+      for (int it = 0; cur >= 0 && ok; ++it) {
+        const int t0 = tile_t0(cur);
+        int nxt = DYN ? -1 : (it + 1 < my_tiles ? item_of(it + 1) : -1);
+        bool nxt_pf = false;
+        const Maps& mp = *LM(layer_of(cur));
         // the epilogue of head h reads its clean inputs (encode) or codes (decode)
         // from global memory: bring them into L2 as the head's operands stream in
         auto prefetch_head = [&](bool is_v, int h) {
           if (t0 >= a.T) return;  // a pair's odd CTA past the last token
           if (ENC) {
-            const CUtensorMap* m = is_v ? &maps.xv : &maps.xk;
+            const CUtensorMap* m = is_v ? &mp.xv : &mp.xk;
             tma_prefetch(m, h * 128, t0);
             tma_prefetch(m, h * 128 + 64, t0);
           } else {
-            tma_prefetch(is_v ? &maps.cv : &maps.ck, h * rbytes, t0);
-            if (G == 32) tma_prefetch(is_v ? &maps.pv : &maps.pk, h * 16, t0);
+            tma_prefetch(is_v ? &mp.cv : &mp.ck, h * rbytes, t0);
+            if (G == 32) tma_prefetch(is_v ? &mp.pv : &mp.pk, h * 16, t0);
           }
         };
-        if (RC && (!OVL || it == 0))
-          for (int c = 0; c < NCH; ++c) load(&maps.ks, c * 64, t0, pol_keep, &maps.wk, c * 64, 0, wbytes);
+        if (!cur_pf) dep_wait(cur);  // (else the previous item checked it)
+        if (RC && !cur_pf)
+          for (int c = 0; c < NCH; ++c) load(&mp.ks, c * 64, t0, pol_keep, &mp.wk, c * 64, 0, wbytes);
         for (int h = 0; h < H && ok; ++h) {
           prefetch_head(false, h);
           for (int j = 0; j < 2; ++j)
-            load(&maps.ks, h * 128 + j * 64, t0, pol_stream, &maps.bk, j * 64, h * 128, 16384);
-          for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, 0, &maps.uk, j * 64, h * 128, 16384);
-          if (RC && h >= 2) load2(&maps.wv, (h - 2) * 128, (h - 2) * 128 + 64, 0, wbytes);
+            load(&mp.ks, h * 128 + j * 64, t0, pol_stream, &mp.bk, j * 64, h * 128, 16384);
+          for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, 0, &mp.uk, j * 64, h * 128, 16384);
+          if (RC && h >= 2) load2(&mp.wv, (h - 2) * 128, (h - 2) * 128 + 64, 0, wbytes);
           if (RC)  // the V latent's V^_{l-1} half, interleaved with the K heads
             for (int c = 2 * h; c < 2 * h + 2; ++c)
-              load(&maps.vs, c * 64, t0, pol_keep, &maps.wv, C + c * 64, 0, wbytes);
+              load(&mp.vs, c * 64, t0, pol_keep, &mp.wv, C + c * 64, 0, wbytes);
         }
         if (RC)
-          for (int g = H >= 2 ? H - 2 : 0; g < H; ++g) load2(&maps.wv, g * 128, g * 128 + 64, 0, wbytes);
+          for (int g = H >= 2 ? H - 2 : 0; g < H; ++g) load2(&mp.wv, g * 128, g * 128 + 64, 0, wbytes);
         for (int h = 0; h < H && ok; ++h) {
           prefetch_head(true, h);
           for (int j = 0; j < 2; ++j)
-            load(&maps.vs, h * 128 + j * 64, t0, pol_stream, &maps.bv, 128 + j * 64, h * 128, 16384);
+            load(&mp.vs, h * 128 + j * 64, t0, pol_stream, &mp.bv, 128 + j * 64, h * 128, 16384);
           if (h == 0) {  // K^_l is read back once both epilogue groups have stored it
             if (ok && !wait(khat_stored, it & 1, abort_flag, a.err, 0x200u)) ok = false;
             if (ok) fence_async_global();
           }
           for (int j = 0; j < 2; ++j)
-            load(&maps.ko, h * 128 + j * 64, t0, pol_stream, &maps.bv, j * 64, h * 128, 16384);
-          for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, 0, &maps.uv, j * 64, h * 128, 16384);
-          if (OVL && nt0 >= 0)  // the next tile's K latent, interleaved with the V heads
+            load(&mp.ko, h * 128 + j * 64, t0, pol_stream, &mp.bv, j * 64, h * 128, 16384);
+          for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, 0, &mp.uv, j * 64, h * 128, 16384);
+          if (h == 0) {  // the next item, and whether its K latent streams in now
+            if (DYN) {
+              nxt = take();
+              nxt_pf = ovl && nxt >= 0 && ok && dep_ready(nxt);
+              publish(nxt, nxt_pf);
+            } else {
+              nxt_pf = ovl && nxt >= 0;
+              if (nxt_pf) dep_wait(nxt);
+            }
+          }
+          if (nxt_pf) {  // the next item's K latent, interleaved with the V heads
+            const Maps& nm = *LM(layer_of(nxt));
+            const int nt0 = tile_t0(nxt);
             for (int c = 2 * h; c < 2 * h + 2; ++c)
-              load(&maps.ks, c * 64, nt0, pol_keep, &maps.wk, c * 64, 0, wbytes);
+              load(&nm.ks, c * 64, nt0, pol_keep, &nm.wk, c * 64, 0, wbytes);
+          }
         }
+        cur = nxt;
+        cur_pf = nxt_pf;
       }
+      if (DYN && pub_open) publish(-1, false);  // an abort left the walk early: close it
       if (!ok && (!PAIR || leader)) {
         // drain: the loads already issued must land before the CTA exits
         for (int i = 0; i < S; ++i) {
@@ -461,10 +603,36 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       auto acq = [&](int b) {
         if (use[b] >= 1) wt(&acc_empty[b], (use[b] - 1) & 1, 0x400u + b);
       };
-      for (int it = 0; it < my_tiles; ++it) {
+      // the k-th item's state: 0 none, 1 an item, 2 an item whose K latent is
+      // loaded during item k-1.  DYN: the sync warp reads the hand-off slot and
+      // passes the state to the issuing warp through one barrier reduction (the
+      // issuing warp reads no shared memory).
+      auto item_state = [&](int k) -> int {
+        if constexpr (DYN) {
+          bool has = false, pf = false;
+          if (!ISSUE) {
+            if (lane == 0) item_wait(k);
+            __syncwarp();
+            has = s_item[k & 3] >= 0;
+            pf = has && s_pf[k & 3] != 0;
+          }
+          const uint32_t pred = (!ISSUE && ((lane == 0 && has) || (lane == 1 && pf))) ? 1u : 0u;
+          uint32_t n;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.popc.u32 %0, 3, 64, p;\n\t}"
+              : "=r"(n)
+              : "r"(pred)
+              : "memory");
+          return (int)n;
+        } else {
+          return k < my_tiles ? (ovl && k > 0 ? 2 : 1) : 0;
+        }
+      };
+      int st_cur = item_state(0);
+      for (int it = 0; st_cur; ++it) {
         const uint32_t zk = zk_col(it), zv = zv_col(it);
-        const bool has_next = it + 1 < my_tiles;
-        if (RC && (!OVL || it == 0)) {
+        int st_next = 0;
+        if (RC && st_cur != 2) {
           for (int c = 0; c < NCH; c += 2)
             group(2, nop, [&](int i, int st) { issue(st, zk, R, c + i == 0, nullptr, nullptr); });
           commit(zk_full);
@@ -530,10 +698,12 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           if (RC) lowrank(b, zv, h == 0, 0x601u);
           commit(&acc_full[b]);
           use[b]++;
-          if (OVL && has_next)
+          if (h == 0) st_next = item_state(it + 1);
+          if (st_next == 2)
             group(2, nop, [&](int i, int st) { issue(st, zk_col(it + 1), R, 2 * h + i == 0, nullptr, nullptr); });
         }
-        if (OVL && has_next) commit(zk_full);
+        if (st_next == 2) commit(zk_full);
+        st_cur = st_next;
       }
       if (ISSUE) {
         // every issued MMA completes before TMEM is released
@@ -631,14 +801,15 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     // one head of this group: h its index, is_v K or V, t0 the tile.  The
     // groups of the row are processed by a rolled loop (the kernel's code must
     // stay small enough for the instruction caches).
-    auto head = [&](int h, bool is_v, int t0) {
+    auto head = [&](int h, bool is_v, int t0, int l) {
       const int b = grp;
       const int64_t t = (int64_t)t0 + row;
       const bool valid = t < a.T;
       const int64_t rowi = t * H + h;
-      uint32_t* codes = reinterpret_cast<uint32_t*>((is_v ? a.vcodes : a.kcodes) + rowi * RB);
-      __half2* params = (is_v ? a.vparams : a.kparams) + rowi * NG;
-      const uint4* X = reinterpret_cast<const uint4*>((is_v ? a.xv : a.xk) + t * C + h * 128);
+      const Ptrs& pp = LP(l);
+      uint32_t* codes = reinterpret_cast<uint32_t*>((is_v ? pp.vcodes : pp.kcodes) + rowi * RB);
+      __half2* params = (is_v ? pp.vparams : pp.kparams) + rowi * NG;
+      const uint4* X = reinterpret_cast<const uint4*>((is_v ? pp.xv : pp.xk) + t * C + h * 128);
       // inputs of the current group: x (encode) or code words and (scale, zero)
       uint4 xc[ENC ? XQ : 1];
       uint32_t cc[ENC ? 1 : GW];
@@ -646,14 +817,14 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       auto stage_x = [&](int g) {
 #pragma unroll
         for (int i = 0; i < XQ; ++i)
-          cp_async16(chunk((g & 1) * XQ + i), valid ? (const void*)(X + g * XQ + i) : (const void*)a.xk,
+          cp_async16(chunk((g & 1) * XQ + i), valid ? (const void*)(X + g * XQ + i) : (const void*)pp.xk,
                      valid ? 16u : 0u);
         cp_async_commit();
       };
       auto stage_xe = [&](int g) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          cp_async16(chunk(i), valid ? (const void*)(X + g * 8 + i) : (const void*)a.xk, valid ? 16u : 0u);
+          cp_async16(chunk(i), valid ? (const void*)(X + g * 8 + i) : (const void*)pp.xk, valid ? 16u : 0u);
         cp_async_commit();
       };
       if (STX) {
@@ -663,12 +834,12 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       if (STE) stage_xe(0);
       if (!ENC) {  // rows past T copy nothing and read zeros (source: the buffers' first bytes)
         const uint8_t* src = reinterpret_cast<const uint8_t*>(codes);
-        const void* c0 = is_v ? a.vcodes : a.kcodes;
-        const __half2* p0 = is_v ? a.vparams : a.kparams;
+        const void* c0 = is_v ? pp.vcodes : pp.kcodes;
+        const __half2* p0 = is_v ? pp.vparams : pp.kparams;
 #pragma unroll
         for (int i = 0; i < RB / 16; ++i) cp_async16(chunk(i), valid ? (const void*)(src + 16 * i) : c0, valid ? 16u : 0u);
         if (EDEN) {  // the row's two fp16 scales
-          const __half* es = reinterpret_cast<const __half*>(is_v ? a.vparams : a.kparams) + rowi * 2;
+          const __half* es = reinterpret_cast<const __half*>(is_v ? pp.vparams : pp.kparams) + rowi * 2;
           cp_async4(chunk(4), valid ? (const void*)es : (const void*)p0, valid ? 4u : 0u);
         } else if (G == 32) {
           cp_async16(chunk(4), valid ? params : p0, valid ? 16u : 0u);
@@ -782,7 +953,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
             const __half sh = __float2half_rn(ss > 0.f && yc > 0.f ? ss / yc : 0.f);
             sf = __half2float(sh);
             if (valid) {
-              reinterpret_cast<__half*>(is_v ? a.vparams : a.kparams)[rowi * 2 + g] = sh;
+              reinterpret_cast<__half*>(is_v ? pp.vparams : pp.kparams)[rowi * 2 + g] = sh;
               *reinterpret_cast<uint4*>(codes + g * 4) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
             }
           } else {
@@ -916,12 +1087,12 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         if (PAIR) mbar_arrive_remote(lead_bar(&acc_empty[b]));
         if ((!is_v || a.store_v) && t0 < a.T) {  // (a pair's odd CTA may be past the last token)
           if (is_v) {
-            tma_store(&maps.vo, h * 128, t0, recon(b));
-            tma_store(&maps.vo, h * 128 + 64, t0, recon(b) + 16384);
+            tma_store(&LM(l)->vo, h * 128, t0, recon(b));
+            tma_store(&LM(l)->vo, h * 128 + 64, t0, recon(b) + 16384);
           } else {  // K^_l is read back by this tile's V heads: kept in L2 until then
             const uint64_t keep = policy_evict_last();
-            tma_store_hint(&maps.ko, h * 128, t0, recon(b), keep);
-            tma_store_hint(&maps.ko, h * 128 + 64, t0, recon(b) + 16384, keep);
+            tma_store_hint(&LM(l)->ko, h * 128, t0, recon(b), keep);
+            tma_store_hint(&LM(l)->ko, h * 128 + 64, t0, recon(b) + 16384, keep);
           }
         }
         bulk_commit();
@@ -936,9 +1107,17 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
 
     // After an abort every wait returns at once; the loops still run to the end
     // so that all threads of a group meet at every named barrier.
-    for (int it = 0; it < my_tiles; ++it) {
-      const int t0 = tile_t0(it);
-      if (RC && grp == 0 && (!OVL || it == 0)) {
+    for (int it = 0;; ++it) {
+      int cur;
+      if constexpr (DYN) {
+        cur = item_wait(it) ? s_item[it & 3] : -1;
+      } else {
+        cur = it < my_tiles ? item_of(it) : -1;
+      }
+      if (cur < 0) break;
+      const int t0 = tile_t0(cur), l = layer_of(cur);
+      // the item's K latent (loaded at its start, or during the previous item's V heads)
+      if (RC && grp == 0) {
         wait(zk_full, zk_use++ & 1, abort_flag, a.err, 0x900u);
         tc_fence_after();
         convert_latent(zk_col(it));
@@ -959,14 +1138,17 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
             convert_latent(zv_col(it));
           }
         }
-        if (((it * HH + u) & 1) == grp) head(u < H ? u : u - H, u >= H, t0);
+        if (((it * HH + u) & 1) == grp) head(u < H ? u : u - H, u >= H, t0, l);
       }
-      if (OVL && RC && grp == 0 && it + 1 < my_tiles) {
-        // the next tile's K latent: its last chunk follows this tile's last V MMA,
-        // so the latent tile in shared memory is free
-        wait(zk_full, zk_use++ & 1, abort_flag, a.err, 0x902u);
-        tc_fence_after();
-        convert_latent(zk_col(it + 1));
+      if constexpr (MULTI) {
+        // this group's reconstruction of the item is in memory: release it to the
+        // next layer's tile (the async-proxy stores complete, then a proxy fence
+        // before the generic release)
+        if (elected) {
+          bulk_wait_all();
+          fence_async_global();
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(flag_of(l, cur)) : "memory");
+        }
       }
     }
     if (elected) bulk_wait_all();
@@ -1069,33 +1251,36 @@ static int sm_count() {
 template <int MODE>
 constexpr bool kPaired = MODE == kDecode;
 
-template <int MODE, int G, int RC, int BITS, bool EDEN = false>
+// Multi-layer launches wait across CTAs (a tile of layer l on the same tile of
+// layer l-1), so their grid is at most what is resident at once.
+template <int MODE, int G, int RC, int BITS, bool EDEN = false, bool MULTI = false>
 static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
+  const int64_t nl = MULTI ? a.n_layers : 1;
   if constexpr (!kPaired<MODE>) {
-    auto k = xlayer_tc_kernel<MODE, G, RC, BITS, false, EDEN>;
+    auto k = xlayer_tc_kernel<MODE, G, RC, BITS, false, EDEN, MULTI>;
     const int smem = Layout<RC, false>::kBytes + 1024;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    // persistent: at most one CTA per SM, each looping over token tiles
-    const int64_t ntiles = (a.T + 127) / 128;
-    const int grid = (int)(ntiles < sms ? ntiles : sms);
+    int per_sm = 1;
+    if (MULTI && ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, smem)) != cudaSuccess))
+      return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    // persistent: at most one CTA per SM, each looping over token tiles (of each layer)
+    const int64_t nitems = (a.T + 127) / 128 * nl;
+    const int grid = (int)(nitems < sms ? nitems : sms);
     k<<<grid, kThreads, smem, st>>>(m, a);
     count_launches(1);
     return cudaGetLastError();
   } else {
-    // pairs: clusters of two CTAs, each pair looping over 256-token tiles
-    auto k = xlayer_tc_kernel<MODE, G, RC, BITS, true, EDEN>;
+    // pairs: clusters of two CTAs, each pair looping over 256-token tiles (of each layer)
+    auto k = xlayer_tc_kernel<MODE, G, RC, BITS, true, EDEN, MULTI>;
     const int smem = Layout<RC, true>::kBytes + 1024;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int64_t npairs = (a.T + 255) / 256;
-    const int max_pairs = sms / 2;
-    const int grid = 2 * (int)(npairs < max_pairs ? npairs : max_pairs);
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -1106,22 +1291,33 @@ static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    int max_pairs = sms / 2;
+    if (MULTI) {
+      cfg.gridDim = dim3((unsigned)(2 * max_pairs));
+      int active = 0;
+      if ((e = cudaOccupancyMaxActiveClusters(&active, k, &cfg)) != cudaSuccess) return e;
+      if (active < 1) return cudaErrorInvalidConfiguration;
+      max_pairs = active < max_pairs ? active : max_pairs;
+    }
+    const int64_t npairs = (a.T + 255) / 256 * nl;
+    const int grid = 2 * (int)(npairs < max_pairs ? npairs : max_pairs);
+    cfg.gridDim = dim3((unsigned)grid);
     e = cudaLaunchKernelEx(&cfg, k, m, a);
     count_launches(1);
     return e != cudaSuccess ? e : cudaGetLastError();
   }
 }
 
-template <int MODE, int BITS>
+template <int MODE, int BITS, bool MULTI = false>
 static cudaError_t dispatch_bits(int group, int rc, const Maps& m, const Args& a, cudaStream_t st) {
   if (group == 32) {
-    if (rc == 0) return launch<MODE, 32, 0, BITS>(m, a, st);
-    if (rc == 1) return launch<MODE, 32, 1, BITS>(m, a, st);
-    return launch<MODE, 32, 2, BITS>(m, a, st);
+    if (rc == 0) return launch<MODE, 32, 0, BITS, false, MULTI>(m, a, st);
+    if (rc == 1) return launch<MODE, 32, 1, BITS, false, MULTI>(m, a, st);
+    return launch<MODE, 32, 2, BITS, false, MULTI>(m, a, st);
   }
-  if (rc == 0) return launch<MODE, 64, 0, BITS>(m, a, st);
-  if (rc == 1) return launch<MODE, 64, 1, BITS>(m, a, st);
-  return launch<MODE, 64, 2, BITS>(m, a, st);
+  if (rc == 0) return launch<MODE, 64, 0, BITS, false, MULTI>(m, a, st);
+  if (rc == 1) return launch<MODE, 64, 1, BITS, false, MULTI>(m, a, st);
+  return launch<MODE, 64, 2, BITS, false, MULTI>(m, a, st);
 }
 
 // H64 / EDEN-2 residuals: 64-value groups, 4 bits a pair
@@ -1132,10 +1328,10 @@ static cudaError_t dispatch_eden(int rc, const Maps& m, const Args& a, cudaStrea
   return launch<MODE, 64, 2, 2, true>(m, a, st);
 }
 
-template <int MODE>
+template <int MODE, bool MULTI = false>
 static cudaError_t dispatch(int group, int rc, const Maps& m, const Args& a, cudaStream_t st) {
-  return a.bits == 2 ? dispatch_bits<MODE, 2>(group, rc, m, a, st)
-                     : dispatch_bits<MODE, 4>(group, rc, m, a, st);
+  return a.bits == 2 ? dispatch_bits<MODE, 2, MULTI>(group, rc, m, a, st)
+                     : dispatch_bits<MODE, 4, MULTI>(group, rc, m, a, st);
 }
 
 // The weight maps: a pair's CTA loads half of each box's rows.
@@ -1170,30 +1366,40 @@ size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int
   return 0;
 }
 
+namespace tc {
+// the tensor maps of one layer's call
+static bool layer_maps(Maps& m, const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K,
+                       const void* V, const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr) {
+  const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128;
+  const bool pair = !enc;  // decode runs as CTA pairs
+  memset(&m, 0, sizeof(m));
+  bool ok = map2d(&m.ks, Ks, T, C, 128) && map2d(&m.vs, Vs, T, C, 128) && map2d(&m.ko, Kr, T, C, 128) &&
+            map2d(&m.vo, Vr ? Vr : Kr, T, C, 128) && weight_maps(m, d, p, pair);
+  const uint64_t rb = 128 * (uint64_t)d->bits / 8;
+  if (ok && enc) ok = map2d(&m.xk, K, T, C, 128) && map2d(&m.xv, V, T, C, 128);
+  if (ok && !enc)
+    ok = map2d_bytes(&m.ck, c->k_codes, T, H * rb, (uint32_t)rb, 128) &&
+         map2d_bytes(&m.cv, c->v_codes, T, H * rb, (uint32_t)rb, 128) &&
+         (d->group != 32 || (map2d_bytes(&m.pk, c->k_params, T, H * 16, 16, 128) &&
+                             map2d_bytes(&m.pv, c->v_params, T, H * 16, 16, 128)));
+  return ok;
+}
+static Ptrs layer_ptrs(const void* K, const void* V, const kvc_codes* c) {
+  return Ptrs{(const __nv_bfloat16*)K, (const __nv_bfloat16*)V, (uint8_t*)c->k_codes, (__half2*)c->k_params,
+              (uint8_t*)c->v_codes, (__half2*)c->v_params};
+}
+}  // namespace tc
+
 cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
                            const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, void*, size_t,
                            cudaStream_t st) {
-  const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128, r = p->rank;
-  const bool pair = !enc;  // decode runs as CTA pairs
+  const uint64_t H = d->n_heads, r = p->rank;
   tc::Maps m;
-  memset(&m, 0, sizeof(m));
-  bool ok = tc::map2d(&m.ks, Ks, T, C, 128) && tc::map2d(&m.vs, Vs, T, C, 128) &&
-            tc::map2d(&m.ko, Kr, T, C, 128) && tc::map2d(&m.vo, Vr ? Vr : Kr, T, C, 128) &&
-            tc::weight_maps(m, d, p, pair);
-  const uint64_t rb = 128 * (uint64_t)d->bits / 8;
-  if (ok && enc) ok = tc::map2d(&m.xk, K, T, C, 128) && tc::map2d(&m.xv, V, T, C, 128);
-  if (ok && !enc)
-    ok = tc::map2d_bytes(&m.ck, c->k_codes, T, H * rb, (uint32_t)rb, 128) &&
-         tc::map2d_bytes(&m.cv, c->v_codes, T, H * rb, (uint32_t)rb, 128) &&
-         (d->group != 32 || (tc::map2d_bytes(&m.pk, c->k_params, T, H * 16, 16, 128) &&
-                             tc::map2d_bytes(&m.pv, c->v_params, T, H * 16, 16, 128)));
-  if (!ok) return cudaErrorInvalidValue;
+  if (!tc::layer_maps(m, d, p, enc, K, V, Ks, Vs, c, Kr, Vr)) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
-  tc::Args a{err, (int64_t)T, (int)H, d->bits, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
-             (uint8_t*)c->k_codes, (__half2*)c->k_params, (uint8_t*)c->v_codes, (__half2*)c->v_params,
-             (enc && !Vr) ? 0 : 1, tc::g_inject_stall.exchange(0),
-             (const float*)p->residual_codebook};
+  tc::Args a{err, (int64_t)d->n_tokens, (int)H, d->bits, tc::layer_ptrs(K, V, c), (enc && !Vr) ? 0 : 1,
+             nullptr, 0, nullptr, tc::g_inject_stall.exchange(0), (const float*)p->residual_codebook};
   const int rc = (int)(r / 64);
   if (d->residual_codec == KVC_RESIDUAL_H64_EDEN2)
     return enc ? tc::dispatch_eden<tc::kEncode>(rc, m, a, st) : tc::dispatch_eden<tc::kDecode>(rc, m, a, st);
@@ -1201,6 +1407,58 @@ cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool
              : tc::dispatch<tc::kDecode>(d->group, rc, m, a, st);
 }
 
+
+
+// ---------------------------------------------------------------- multi-layer calls
+
+static size_t align256u(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool tc_codec_layers_supported(const kvc_layer_desc* d, const kvc_predictor* preds, int n) {
+  if (n < 1 || d->residual_codec != KVC_RESIDUAL_RTN) return false;
+  for (int i = 0; i < n; ++i)
+    if (!tc_codec_supported(d, &preds[i]) || preds[i].rank != preds[0].rank) return false;
+  return true;
+}
+
+size_t tc_codec_layers_workspace(const kvc_layer_desc* d, int n) {
+  const size_t ntiles = ((size_t)d->n_tokens + 127) / 128;
+  // the layer table, then a counter per (layer, 128-token tile) and the item ticket
+  return align256u((size_t)n * sizeof(tc::LayerDev)) + align256u(((size_t)n * ntiles + 1) * sizeof(unsigned));
+}
+
+cudaError_t tc_codec_layers(const kvc_layer_desc* d, const kvc_predictor* preds, int n, bool enc,
+                            const void* const* K, const void* const* V, const void* Ks0, const void* Vs0,
+                            const kvc_codes* c, void* const* Kr, void* const* Vr, void* ws, size_t ws_bytes,
+                            cudaStream_t st) {
+  if (ws_bytes < tc_codec_layers_workspace(d, n) || !ws) return cudaErrorInvalidValue;
+  // layer i of the call reads the reconstruction of layer i-1 (Ks0 / Vs0 for i = 0)
+  std::vector<tc::LayerDev> host((size_t)n);
+  for (int i = 0; i < n; ++i) {
+    const void* ks = i ? Kr[i - 1] : Ks0;
+    const void* vs = i ? Vr[i - 1] : Vs0;
+    const void* k = enc ? K[i] : nullptr;
+    const void* v = enc ? V[i] : nullptr;
+    if (!tc::layer_maps(host[i].maps, d, &preds[i], enc, k, v, ks, vs, &c[i], Kr[i], Vr[i]))
+      return cudaErrorInvalidValue;
+    host[i].p = tc::layer_ptrs(k, v, &c[i]);
+  }
+  char* w = static_cast<char*>(ws);
+  tc::LayerDev* dev = reinterpret_cast<tc::LayerDev*>(w);
+  unsigned* flags = reinterpret_cast<unsigned*>(w + align256u((size_t)n * sizeof(tc::LayerDev)));
+  const size_t ntiles = ((size_t)d->n_tokens + 127) / 128;
+  cudaError_t e = cudaMemcpyAsync(dev, host.data(), (size_t)n * sizeof(tc::LayerDev), cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(flags, 0, ((size_t)n * ntiles + 1) * sizeof(unsigned), st)) != cudaSuccess) return e;
+  unsigned* err = tc_error_word();
+  if (!err) return cudaErrorInvalidDevice;
+  tc::Maps none;
+  memset(&none, 0, sizeof(none));
+  tc::Args a{err, (int64_t)d->n_tokens, (int)d->n_heads, d->bits, tc::Ptrs{}, 1, dev, n, flags,
+             tc::g_inject_stall.exchange(0), nullptr};
+  const int rc = (int)(preds[0].rank / 64);
+  return enc ? tc::dispatch<tc::kEncode, true>(d->group, rc, none, a, st)
+             : tc::dispatch<tc::kDecode, true>(d->group, rc, none, a, st);
+}
 
 }  // namespace kvc
 

@@ -10,6 +10,14 @@ size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int
 cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
                            const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, void* ws,
                            size_t ws_bytes, cudaStream_t st);
+// a chain of n predicted layers in one persistent launch (layer i reads layer
+// i-1's reconstruction; Ks0 / Vs0 for i = 0); Kr / Vr of every layer required
+bool tc_codec_layers_supported(const kvc_layer_desc* d, const kvc_predictor* preds, int n);
+size_t tc_codec_layers_workspace(const kvc_layer_desc* d, int n);
+cudaError_t tc_codec_layers(const kvc_layer_desc* d, const kvc_predictor* preds, int n, bool enc,
+                            const void* const* K, const void* const* V, const void* Ks0, const void* Vs0,
+                            const kvc_codes* c, void* const* Kr, void* const* Vr, void* ws, size_t ws_bytes,
+                            cudaStream_t st);
 bool tc_temporal_supported(const kvc_layer_desc* d, const kvc_predictor* p);
 cudaError_t tc_temporal_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K, const void* V,
                               const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr, cudaStream_t st);

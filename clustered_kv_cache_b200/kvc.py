@@ -27,7 +27,8 @@ STATUS = {0: "KVC_OK", 1: "KVC_ERR_INVALID_ARGUMENT", 2: "KVC_ERR_UNSUPPORTED", 
 EXPORTED = ["kvc_codes_sizes", "kvc_codes_bytes", "kvc_workspace_bytes", "kvc_encode_layer", "kvc_decode_layer",
             "kvc_attend_compressed", "kvc_pack_codes", "kvc_unpack_codes", "kvc_get_device_error",
             "kvc_status_string", "kvc_last_cuda_error", "kvc_launch_counter", "kvc_testing_inject_stall",
-            "kvc_attend_compressed_debiased", "kvc_refit_block_diag", "kvc_copy_to_device", "kvc_copy_to_host"]
+            "kvc_attend_compressed_debiased", "kvc_refit_block_diag", "kvc_copy_to_device", "kvc_copy_to_host",
+            "kvc_encode_layers", "kvc_decode_layers", "kvc_layers_workspace_bytes"]
 
 
 class KvcError(RuntimeError):
@@ -85,6 +86,9 @@ def lib():
         "kvc_attend_compressed_debiased": (I, [D, PR, V, I64, CO, V, V, V, V, I64, F, V, V, V, V, SZ, V]),
         "kvc_refit_block_diag": (I, [D, PR, ctypes.c_int, V, V, V, F, V, V, SZ, V]),
         "kvc_copy_to_device": (I, [V, V, SZ, V]),
+        "kvc_encode_layers": (I, [D, PR, I, P(V), P(V), V, V, CO, P(V), P(V), V, SZ, V]),
+        "kvc_decode_layers": (I, [D, PR, I, CO, V, V, P(V), P(V), V, SZ, V]),
+        "kvc_layers_workspace_bytes": (SZ, [I, D, PR, I]),
         "kvc_copy_to_host": (I, [V, V, SZ, V]),
         "kvc_pack_codes": (I, [V, I64, I, V, V]),
         "kvc_unpack_codes": (I, [V, I64, I, V, V]),
@@ -214,6 +218,47 @@ def kvc_encode_layer(desc, pred, K, V, K_src, V_src, codes: CodeBuffers, K_rec=N
     _check(lib().kvc_encode_layer(ctypes.byref(desc), ctypes.byref(pred), _ptr(K), _ptr(V), _ptr(K_src),
                                   _ptr(V_src), ctypes.byref(c), _ptr(K_rec), _ptr(V_rec), wp, wn, _stream(stream)),
            "kvc_encode_layer")
+
+
+def _preds(preds) -> ctypes.Array:
+    return (Predictor * len(preds))(*preds)  # the structs' copies; the tensors stay with `preds`
+
+
+def _codes(codes) -> ctypes.Array:
+    return (Codes * len(codes))(*[c.struct() for c in codes])
+
+
+def _ptrs(ts) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ts))(*[_ptr(t) for t in ts])
+
+
+def kvc_layers_workspace_bytes(op: int, desc: LayerDesc, preds) -> int:
+    return lib().kvc_layers_workspace_bytes(op, ctypes.byref(desc), _preds(preds), len(preds))
+
+
+def alloc_layers_workspace(op: int, desc: LayerDesc, preds, device="cuda") -> torch.Tensor | None:
+    n = kvc_layers_workspace_bytes(op, desc, preds)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def kvc_encode_layers(desc, preds, K, V, K_src, V_src, codes, K_rec, V_rec, ws=None, stream=None):
+    """Layers i = 0 .. len(preds)-1 of a cross-layer chain in one call; layer i
+    predicts from K_rec[i-1] / V_rec[i-1] (K_src / V_src for i = 0).  K, V, codes,
+    K_rec, V_rec: lists of one entry per layer."""
+    n = len(preds)
+    assert len(K) == len(V) == len(codes) == len(K_rec) == len(V_rec) == n
+    wp, wn = _ws(ws)
+    _check(lib().kvc_encode_layers(ctypes.byref(desc), _preds(preds), n, _ptrs(K), _ptrs(V), _ptr(K_src),
+                                   _ptr(V_src), _codes(codes), _ptrs(K_rec), _ptrs(V_rec), wp, wn, _stream(stream)),
+           "kvc_encode_layers")
+
+
+def kvc_decode_layers(desc, preds, codes, K_src, V_src, K_rec, V_rec, ws=None, stream=None):
+    n = len(preds)
+    assert len(codes) == len(K_rec) == len(V_rec) == n
+    wp, wn = _ws(ws)
+    _check(lib().kvc_decode_layers(ctypes.byref(desc), _preds(preds), n, _codes(codes), _ptr(K_src), _ptr(V_src),
+                                   _ptrs(K_rec), _ptrs(V_rec), wp, wn, _stream(stream)), "kvc_decode_layers")
 
 
 def kvc_decode_layer(desc, pred, codes: CodeBuffers, K_src, V_src, K_rec, V_rec, ws=None, stream=None):

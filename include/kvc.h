@@ -216,6 +216,38 @@ KVC_API kvc_status kvc_decode_layer(const kvc_layer_desc* desc, const kvc_predic
                             const void* K_src, const void* V_src, void* K_rec, void* V_rec, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* A chain of n_layers predicted (KVC_PRED_XLAYER_DPLR) layers in one call
+ * ("CORAL-KV ...", Fig. 3: layer l predicts from the reconstruction of layer
+ * l-1).  Layer i of the call (0-based) predicts from the reconstruction of layer
+ * i-1, or from K_src / V_src [T][H][D] for i = 0, and writes its own to
+ * K_rec[i] / V_rec[i] [T][H][D] (all required).  Results are identical, byte for
+ * byte, to n_layers kvc_encode_layer / kvc_decode_layer calls in order.
+ *  desc:          shared by every layer; preds[i], out[i] / codes[i] (arrays of
+ *                 n_layers) are layer i's predictor and codes; K[i], V[i] its
+ *                 clean values (encode).
+ *  K_rec, V_rec:  arrays of n_layers device pointers.  K_rec[i] may be the
+ *                 buffer of layer i-2 (two buffers in turn suffice) but not of
+ *                 layer i-1 (its source); KVC_ERR_INVALID_ARGUMENT otherwise.
+ *  ws, ws_bytes:  kvc_layers_workspace_bytes(KVC_OP_ENCODE or KVC_OP_DECODE,
+ *                 desc, preds, n_layers).
+ * With bf16, head_dim 128, scalar residual codes and equal ranks in {0, 64,
+ * 128} the call is one persistent tensor-core launch that walks (layer, token
+ * tile) items in layer order; the tile of layer i waits (bounded) for the same
+ * tile of layer i-1, so the layers' wave tails overlap.  Other shapes run the
+ * layers in turn.  The INT4 anchor layer is a separate kvc_encode_layer. */
+KVC_API kvc_status kvc_encode_layers(const kvc_layer_desc* desc, const kvc_predictor* preds, int n_layers,
+                                     const void* const* K, const void* const* V, const void* K_src,
+                                     const void* V_src, const kvc_codes* out, void* const* K_rec,
+                                     void* const* V_rec, void* ws, size_t ws_bytes, void* stream);
+KVC_API kvc_status kvc_decode_layers(const kvc_layer_desc* desc, const kvc_predictor* preds, int n_layers,
+                                     const kvc_codes* codes, const void* K_src, const void* V_src,
+                                     void* const* K_rec, void* const* V_rec, void* ws, size_t ws_bytes,
+                                     void* stream);
+/* Workspace bytes of kvc_encode_layers (op KVC_OP_ENCODE) or kvc_decode_layers
+ * (KVC_OP_DECODE); 0 for an invalid description. */
+KVC_API size_t kvc_layers_workspace_bytes(int op, const kvc_layer_desc* desc, const kvc_predictor* preds,
+                                          int n_layers);
+
 /* Softmax attention of Q [n_q][H][D] (H = desc->q_heads when set) over this layer's compressed history,
  * followed by n_self uncompressed tokens K_self / V_self [n_self][H][D]
  * (non-causal; n_self may be 0 and the pointers NULL):

@@ -104,3 +104,34 @@ def test_status_strings(L):
     for s in range(7):
         assert kvc.kvc_status_string(s)
     assert kvc.kvc_status_string(99) == "unknown status"
+
+
+def test_multi_layer_validation_without_launch(L):
+    """kvc_encode_layers / kvc_decode_layers refuse bad chains before anything runs."""
+    d = kvc.make_desc(100, 2, 128, torch.bfloat16, 2, 32)
+    xp = kvc.Predictor(kvc.PRED_XLAYER_DPLR, 0, 0, 0, *([0x1000] * 12))
+    preds = (kvc.Predictor * 2)(xp, xp)
+    c = kvc.Codes(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    codes = (kvc.Codes * 2)(c, c)
+    P = lambda *a: (ctypes.c_void_p * len(a))(*a)
+    x = P(0x1000, 0x2000)
+    need = L.kvc_layers_workspace_bytes(kvc.OP_ENCODE, ctypes.byref(d), preds, 2)
+    assert L.kvc_layers_workspace_bytes(kvc.OP_ATTEND, ctypes.byref(d), preds, 2) == 0
+    assert L.kvc_layers_workspace_bytes(kvc.OP_ENCODE, ctypes.byref(d), preds, 0) == 0
+
+    def enc(n=2, Kr=None, Vr=None, Ks=0x1000, ws=0x100000, wsn=None):
+        Kr = Kr or P(0x3000, 0x5000)
+        Vr = Vr or P(0x4000, 0x6000)
+        return L.kvc_encode_layers(ctypes.byref(d), preds, n, x, x, Ks, 0x1000, codes, Kr, Vr, ws,
+                                   need if wsn is None else wsn, None)
+
+    assert enc(n=0) == 1
+    assert enc(Ks=None) == 1                                   # layer 0's sources
+    assert enc(Kr=P(0x3000, 0x3000)) == 1                      # layer 1 would overwrite its own source
+    assert enc(Kr=P(0x1000, 0x5000)) == 1                      # layer 0 would overwrite the chain's source
+    assert enc(Kr=P(0x3000, 0x5008)) == 3                      # misaligned
+    if need:
+        assert enc(wsn=need - 1) == 4
+    tp = kvc.Predictor(kvc.PRED_TEMPORAL, 0, 0, 0, *([0x1000] * 12))
+    assert L.kvc_decode_layers(ctypes.byref(kvc.make_desc(100, 2, 128, frame_tokens=10)), (kvc.Predictor * 1)(tp),
+                               1, (kvc.Codes * 1)(c), 0x1000, 0x1000, P(0x3000), P(0x4000), None, 0, None) == 2

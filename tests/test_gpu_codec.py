@@ -1005,3 +1005,70 @@ def test_grouped_query_attention_cuda_core_path():
     _sync_ok()
     ref = O.attend_compressed_xlayer(od, w64, U.to64(Q), ck1, cv1, K0h, V0h, None, None, 0.125)
     assert U.rel_l2(U.to64(Og), ref) <= U.ATT_TOL[f32]
+
+
+# ---------------------------------------------------------------- the chain of layers in one call
+
+
+@pytest.mark.parametrize("L,T,H,rank,bits,group,pingpong", [(5, 3 * 128 + 41, 4, 64, 2, 32, False),
+                                                            (5, 2 * 256 + 7, 3, 128, 4, 64, True),
+                                                            (5, 300, 2, 0, 2, 64, True), (5, 128, 2, 64, 2, 32, False),
+                                                            (61, 300, 2, 64, 2, 32, True),
+                                                            (3, 40 * 128 + 3, 2, 64, 2, 32, True)])
+def test_layer_chain_in_one_call_matches_layer_calls(L, T, H, rank, bits, group, pingpong):
+    """kvc_encode_layers / kvc_decode_layers (one persistent launch walking
+    (layer, tile) items, each tile waiting on the same tile of the layer before)
+    against kvc_encode_layer / kvc_decode_layer called layer by layer: the same
+    arithmetic, so every code, parameter and reconstruction is identical.  With
+    `pingpong` the chain reuses two reconstruction buffers in turn.  60 layers of
+    3 tiles give more items than SMs with fewer tiles than CTAs (the latent
+    overlap across items is off there); 40 tiles give CTAs several items each."""
+    D = 128
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 121, device="cuda", L=L, T=T, H=H, rank=rank, calib_tokens=512)
+    bf, hf = torch.bfloat16, torch.float16
+    desc = _desc(T, H, D, bf, bits, group, hf)
+    preds = [kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl.weights[l], rank=rank) for l in range(1, L)]
+    n = L - 1
+    # the reference: layer calls in turn from layer 0's clean values
+    ws = kvc.alloc_workspace(kvc.OP_ENCODE, desc, preds[0])
+    wsd = kvc.alloc_workspace(kvc.OP_DECODE, desc, preds[0])
+    ref_codes, ref_K, ref_V, ref_Kd, ref_Vd = [], [], [], [], []
+    Ks, Vs = wl.K[0], wl.V[0]
+    for i in range(n):
+        buf = kvc.alloc_codes(desc, preds[i])
+        Kr, Vr = torch.empty_like(Ks), torch.empty_like(Vs)
+        kvc.kvc_encode_layer(desc, preds[i], wl.K[i + 1], wl.V[i + 1], Ks, Vs, buf, Kr, Vr, ws)
+        ref_codes.append(buf), ref_K.append(Kr), ref_V.append(Vr)
+        Ks, Vs = Kr, Vr
+    Ks, Vs = wl.K[0], wl.V[0]
+    for i in range(n):
+        Kd, Vd = torch.empty_like(Ks), torch.empty_like(Vs)
+        kvc.kvc_decode_layer(desc, preds[i], ref_codes[i], Ks, Vs, Kd, Vd, wsd)
+        ref_Kd.append(Kd), ref_Vd.append(Vd)
+        Ks, Vs = Kd, Vd
+    # the chain in one call
+    codes = [kvc.alloc_codes(desc, p) for p in preds]
+    mk = lambda: torch.zeros_like(wl.K[0])
+    if pingpong:
+        bufs = [(mk(), mk()), (mk(), mk())]
+        Kr = [bufs[i % 2][0] for i in range(n)]
+        Vr = [bufs[i % 2][1] for i in range(n)]
+    else:
+        Kr = [mk() for _ in range(n)]
+        Vr = [mk() for _ in range(n)]
+    wse = kvc.alloc_layers_workspace(kvc.OP_ENCODE, desc, preds)
+    kvc.kvc_encode_layers(desc, preds, wl.K[1:], wl.V[1:], wl.K[0], wl.V[0], codes, Kr, Vr, wse)
+    _sync_ok()
+    for i in range(n):
+        for name in ("k_codes", "k_params", "v_codes", "v_params"):
+            assert torch.equal(getattr(codes[i], name), getattr(ref_codes[i], name)), (i, name)
+    for i in range(n - 2 if pingpong else 0, n):  # (the ping-pong buffers hold the last two layers)
+        assert torch.equal(Kr[i], ref_K[i]) and torch.equal(Vr[i], ref_V[i]), i
+    Kd = [mk() for _ in range(n)]
+    Vd = [mk() for _ in range(n)]
+    wsdl = kvc.alloc_layers_workspace(kvc.OP_DECODE, desc, preds)
+    kvc.kvc_decode_layers(desc, preds, codes, wl.K[0], wl.V[0], Kd, Vd, wsdl)
+    _sync_ok()
+    for i in range(n):
+        assert torch.equal(Kd[i], ref_Kd[i]) and torch.equal(Vd[i], ref_Vd[i]), i
+        assert torch.equal(Kd[i], ref_K[i]) and torch.equal(Vd[i], ref_V[i]), i  # decode replays encode
