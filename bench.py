@@ -43,10 +43,12 @@ UNIT = "KV tokens/s"
 
 
 # DRAM bytes (read + write) per call, from the ncu captures summarised under
-# profiles/ (codec_xlayer_wan_layer.md, attention_cluster_wan.md,
-# mixed_attention_cluster.md, cluster_codec_decode.md, temporal_codec_layer.md);
+# profiles/ (codec_xlayer_wan_layer.md, codec_xlayer_fused_wan.md, attention_flash_wan.md,
+# mixed_attention_cluster.md, cluster_codec_decode.md, temporal_codec_layer.md, codec_xlayer_eden2.md);
 # set to None when a kernel changes after its capture.
-TRAFFIC = {"encode_xlayer": 676536064 + 187995648, "decode_xlayer": 431820800 + 138174976,
+TRAFFIC = {"encode_xlayer": 678559232 + 188143104, "decode_xlayer": 428340480 + 137626112,
+           # per layer of the fused walk (a 4-layer launch's DRAM bytes / 4; scaled by the layer count)
+           "encode_xlayer_fused": (2837343488 + 916343040) // 4, "decode_xlayer_fused": (2087463168 + 744328704) // 4,
            "attention_c2": 244925696 + 13229312, "attention_c4": 26443520 + 146944,
            "decode_c4": 4399616 + 80381696 + 4467712 + 80104704,
            "temporal_encode": 1434010000 + 372614912,
@@ -130,6 +132,9 @@ class XLayerBench:
                      [kvc.alloc_codes(self.desc, self.preds[l], device) for l in range(1, layers)]
         self.ws_enc = kvc.alloc_workspace(kvc.OP_ENCODE, self.desc, self.preds[1], device=device)
         self.ws_dec = kvc.alloc_workspace(kvc.OP_DECODE, self.desc, self.preds[1], device=device)
+        if layers >= 2:  # the fused calls over layers 1 .. L-1 (one launch each way)
+            self.ws_enc_all = kvc.alloc_layers_workspace(kvc.OP_ENCODE, self.desc, self.preds[1:], device=device)
+            self.ws_dec_all = kvc.alloc_layers_workspace(kvc.OP_DECODE, self.desc, self.preds[1:], device=device)
         mk = lambda: torch.empty(T_TOK, H, D, dtype=bf, device=device)
         self.er = [(mk(), mk()), (mk(), mk())]  # encode-chain reconstructions (ping-pong)
         self.dr = [(mk(), mk()), (mk(), mk())]  # decode-chain reconstructions
@@ -173,9 +178,38 @@ class XLayerBench:
             if ev is not None:
                 ev[l][1].record()
 
+    def encode_fused(self, ev=None):
+        """The anchor layer, then layers 1 .. L-1 in one kvc_encode_layers launch
+        (the same ping-pong reconstruction buffers as the per-layer chain)."""
+        K, V = self.wl.K, self.wl.V
+        Kr0, Vr0 = self.er[0]
+        kvc.kvc_encode_layer(self.desc0, self.pred0, K[0], V[0], None, None, self.codes[0], Kr0, Vr0)
+        if self.L < 2:
+            return
+        if ev is not None:
+            ev[0].record()
+        kvc.kvc_encode_layers(self.desc, self.preds[1:], K[1:], V[1:], Kr0, Vr0, self.codes[1:],
+                              [self.er[l % 2][0] for l in range(1, self.L)],
+                              [self.er[l % 2][1] for l in range(1, self.L)], self.ws_enc_all)
+        if ev is not None:
+            ev[1].record()
+
+    def decode_fused(self, ev=None):
+        Kr0, Vr0 = self.dr[0]
+        kvc.kvc_decode_layer(self.desc0, self.pred0, self.codes[0], None, None, Kr0, Vr0)
+        if self.L < 2:
+            return
+        if ev is not None:
+            ev[0].record()
+        kvc.kvc_decode_layers(self.desc, self.preds[1:], self.codes[1:], Kr0, Vr0,
+                              [self.dr[l % 2][0] for l in range(1, self.L)],
+                              [self.dr[l % 2][1] for l in range(1, self.L)], self.ws_dec_all)
+        if ev is not None:
+            ev[1].record()
+
     def step(self, ev_enc=None, ev_dec=None):
-        self.encode_chain(ev_enc)
-        self.decode_chain(ev_dec)
+        self.encode_fused(ev_enc)
+        self.decode_fused(ev_dec)
 
     # algorithmic traffic / work of one predicted layer
     def layer_bytes(self, encode: bool) -> int:
@@ -582,9 +616,8 @@ def main():
     torch.cuda.synchronize()
     assert kvc.kvc_get_device_error() == 0
 
-    mk = lambda: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(L_RUN)]
-    ev_enc = [mk() for _ in range(args.steps)]
+    mk = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    ev_enc = [mk() for _ in range(args.steps)]  # around the fused call of layers 1 .. L-1
     ev_dec = [mk() for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
@@ -606,23 +639,28 @@ def main():
     ms_step = ms_total / args.steps
     value = job_value(ms_step, world, L_RUN)
 
-    enc_ms = statistics.mean(x for k in range(args.steps) for x in time_events(ev_enc[k][1:]))
-    dec_ms = statistics.mean(x for k in range(args.steps) for x in time_events(ev_dec[k][1:]))
-    enc_b, dec_b = xb.layer_bytes(True), xb.layer_bytes(False)
+    # the dominant launch: the fused call over the n_pred = L-1 predicted layers
+    n_pred = max(L_RUN - 1, 1)
+    enc_ms = statistics.mean(time_events(ev_enc)) if L_RUN >= 2 else float("nan")
+    dec_ms = statistics.mean(time_events(ev_dec)) if L_RUN >= 2 else float("nan")
+    enc_b, dec_b = n_pred * xb.layer_bytes(True), n_pred * xb.layer_bytes(False)
     enc_gbs, dec_gbs = enc_b / (enc_ms * 1e-3) / 1e9, dec_b / (dec_ms * 1e-3) / 1e9
     dom_enc = enc_ms >= dec_ms
+    tkey = "encode_xlayer_fused" if dom_enc else "decode_xlayer_fused"
     roof = {"bound": "hbm", "achieved": enc_gbs if dom_enc else dec_gbs, "peak": hbm, "unit": "GB/s",
             "frac": (enc_gbs if dom_enc else dec_gbs) / hbm,
-            "traffic": TRAFFIC["encode_xlayer"] if dom_enc else TRAFFIC["decode_xlayer"],
-            "kernel": "kvc_encode_layer (cross-layer, one layer)" if dom_enc else
-                      "kvc_decode_layer (cross-layer, one layer)",
+            "traffic": TRAFFIC[tkey] * n_pred if tkey in TRAFFIC else None,
+            "kernel": f"kvc_encode_layers (cross-layer, {n_pred} layers in one launch)" if dom_enc else
+                      f"kvc_decode_layers (cross-layer, {n_pred} layers in one launch)",
             "bytes_per_launch": enc_b if dom_enc else dec_b, "ms_per_launch": enc_ms if dom_enc else dec_ms,
             "peak_kind": peak_kind}
     flops = XLayerBench.layer_flops()
-    detail = {"encode_layer": {"ms": enc_ms, "GB/s": enc_gbs, "frac_hbm": enc_gbs / hbm, "bytes": enc_b,
-                               "TFLOP/s": flops / (enc_ms * 1e-3) / 1e12},
-              "decode_layer": {"ms": dec_ms, "GB/s": dec_gbs, "frac_hbm": dec_gbs / hbm, "bytes": dec_b,
-                               "TFLOP/s": flops / (dec_ms * 1e-3) / 1e12}}
+    detail = {"encode_layers": {"ms": enc_ms, "ms_per_layer": enc_ms / n_pred, "GB/s": enc_gbs,
+                                "frac_hbm": enc_gbs / hbm, "bytes": enc_b,
+                                "TFLOP/s": n_pred * flops / (enc_ms * 1e-3) / 1e12},
+              "decode_layers": {"ms": dec_ms, "ms_per_layer": dec_ms / n_pred, "GB/s": dec_gbs,
+                                "frac_hbm": dec_gbs / hbm, "bytes": dec_b,
+                                "TFLOP/s": n_pred * flops / (dec_ms * 1e-3) / 1e12}}
 
     # end to end: inputs from pinned host memory, codes back to the host
     e2e = None

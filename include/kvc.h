@@ -229,7 +229,11 @@ KVC_API kvc_status kvc_decode_layer(const kvc_layer_desc* desc, const kvc_predic
  *                 buffer of layer i-2 (two buffers in turn suffice) but not of
  *                 layer i-1 (its source); KVC_ERR_INVALID_ARGUMENT otherwise.
  *  ws, ws_bytes:  kvc_layers_workspace_bytes(KVC_OP_ENCODE or KVC_OP_DECODE,
- *                 desc, preds, n_layers).
+ *                 desc, preds, n_layers).  It holds the call's layer table and
+ *                 its per-tile counters, so calls in flight at the same time
+ *                 need workspaces of their own.
+ * A device wait that runs out (bounded, about two seconds) ends the launch and
+ * is reported by kvc_get_device_error as KVC_ERR_DEVICE_TIMEOUT.
  * With bf16, head_dim 128, scalar residual codes and equal ranks in {0, 64,
  * 128} the call is one persistent tensor-core launch that walks (layer, token
  * tile) items in layer order; the tile of layer i waits (bounded) for the same

@@ -17,7 +17,8 @@ from oracle import kvc_oracle as ON
 from oracle import kvc_oracle_c as O
 
 import kvc_testutil as U
-from test_gpu_codec import _cluster_pred, _compare, _desc, _oracle_codes_to_gpu, _temporal_call, _temporal_gpu_coded
+from test_gpu_codec import (_cluster_pred, _compare, _desc, _odesc, _oracle_codes_to_gpu, _temporal_call,
+                            _temporal_gpu_coded)
 
 pytestmark = pytest.mark.gpu
 
@@ -261,3 +262,63 @@ def test_repeated_calls_are_bit_identical():
             ref = cur
         else:
             assert all(torch.equal(a, b) for a, b in zip(ref, cur)), "cross-layer codec or attention differs"
+
+
+def test_fused_layer_walk_at_the_benchmark_size():
+    """The benchmark's cross-layer step as it launches it: the 29 predicted
+    layers of a 30-layer, 32760-token, 12-head, rank-64 INT2 workload in one
+    kvc_encode_layers launch and one kvc_decode_layers launch (items of every
+    layer in flight at once, each waiting on its tile of the layer below).  It
+    must give the bytes of the 29 one-layer calls, its decode must replay its
+    encode, and sampled tokens of three layers (first, middle, last) must match
+    the oracle coding that layer from the walk's own reconstruction of the
+    layer below."""
+    L, T, H, D, R = 30, 32760, 12, 128, 64
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 1, device="cuda", L=L, T=T, H=H, D=D, rank=R)
+    bf, hf = torch.bfloat16, torch.float16
+    desc = _desc(T, H, D, bf, 2, 32, hf)
+    preds = [kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl.weights[l], rank=R) for l in range(1, L)]
+    n = L - 1
+    mk = lambda: [torch.empty_like(wl.K[0]) for _ in range(n)]
+    codes, Kr, Vr = [kvc.alloc_codes(desc, p) for p in preds], mk(), mk()
+    kvc.kvc_encode_layers(desc, preds, wl.K[1:], wl.V[1:], wl.K[0], wl.V[0], codes, Kr, Vr,
+                          kvc.alloc_layers_workspace(kvc.OP_ENCODE, desc, preds))
+    assert kvc.kvc_get_device_error() == 0
+    Kd, Vd = mk(), mk()
+    kvc.kvc_decode_layers(desc, preds, codes, wl.K[0], wl.V[0], Kd, Vd,
+                          kvc.alloc_layers_workspace(kvc.OP_DECODE, desc, preds))
+    assert kvc.kvc_get_device_error() == 0
+    for i in range(n):
+        assert torch.equal(Kd[i], Kr[i]) and torch.equal(Vd[i], Vr[i]), f"layer {i + 1}: decode != encode"
+    del Kd, Vd
+    # the one-layer calls, layer by layer from the same sources
+    ws = kvc.alloc_workspace(kvc.OP_ENCODE, desc, preds[0])
+    Ks, Vs = wl.K[0], wl.V[0]
+    k1, v1 = torch.empty_like(wl.K[0]), torch.empty_like(wl.V[0])
+    for i in range(n):
+        c1 = kvc.alloc_codes(desc, preds[i])
+        kvc.kvc_encode_layer(desc, preds[i], wl.K[i + 1], wl.V[i + 1], Ks, Vs, c1, k1, v1, ws)
+        assert kvc.kvc_get_device_error() == 0
+        for name in ("k_codes", "k_params", "v_codes", "v_params"):
+            assert torch.equal(getattr(c1, name), getattr(codes[i], name)), f"layer {i + 1} {name}"
+        assert torch.equal(k1, Kr[i]) and torch.equal(v1, Vr[i]), f"layer {i + 1} reconstruction"
+        Ks, Vs = Kr[i], Vr[i]
+    del k1, v1
+    # the oracle on sampled tokens, from the walk's own reconstruction of the layer below
+    idx = _rows(T, 192, 29)
+    sub = lambda t: U.to64(t[torch.from_numpy(idx).to(t.device)])
+    od = _odesc(len(idx), H, D, bf, 2, 32, hf)
+    for l in (1, 15, 29):
+        Ks, Vs = (wl.K[0], wl.V[0]) if l == 1 else (Kr[l - 2], Vr[l - 2])
+        w64 = {k: U.to64(v) for k, v in wl.weights[l].items()}
+        ck, cv, Kh, Vh = O.encode_layer_xlayer(od, w64, sub(wl.K[l]), sub(wl.V[l]), sub(Ks), sub(Vs))
+        ek, ev = U.exact_xlayer(od, w64, ck, cv, sub(Ks), sub(Vs), Kh)
+        errk, errv = U.err_xlayer(od, w64, sub(Ks), sub(Vs), Kh)
+        kflip = None
+        for which, oc, rec, ref, ex, x, er in (("k", ck, Kr[l - 1], Kh, ek, wl.K[l], errk),
+                                               ("v", cv, Vr[l - 1], Vh, ev, wl.V[l], errv)):
+            q = U.codes_from_gpu(getattr(codes[l - 1], which + "_codes"), (T, H, D), 2)[idx]
+            s_, z_ = U.params_from_gpu(getattr(codes[l - 1], which + "_params"), (T, H, D // 32), "f16")
+            gc = O.Coded(q, s_[idx], z_[idx])
+            kflip = _compare(gc, oc, sub(rec), ref, ex, sub(x), "bf16", 32, f"layer {l} {which} (sampled tokens)",
+                             "f16", er, kflip)
