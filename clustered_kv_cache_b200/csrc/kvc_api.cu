@@ -219,21 +219,21 @@ cudaError_t codec_cluster(const kvc_layer_desc* d, const kvc_predictor* p, bool 
         const float* const cnc[2] = {cns[0], cns[1]};
         if ((e = tc_cluster_prepare(d, p, cnc, Ps, st)) != cudaSuccess) return e;
       }
-      for (int which = 0; which < 2; ++which) {
-        const TS* cent = (const TS*)(which ? p->v_centroids : p->k_centroids);
-        const TS* encw = (const TS*)(which ? p->v_enc : p->k_enc);
-        const TS* dec = (const TS*)(which ? p->v_dec : p->k_dec);
-        void* codes = which ? c->v_codes : c->k_codes;
-        void* params = which ? c->v_params : c->k_params;
-        void* assign = which ? c->v_assign : c->k_assign;
-        void* rec = which ? Vr : Kr;
-        if (enc && (e = tc_cluster_encode(d, p, which ? V : K, cent, encw, cns[which], Ps[which], codes, params,
-                                          assign, st)) != cudaSuccess)
-          return e;
-        // the encode's reconstruction is the decode of what it wrote, so the two agree bit for bit
-        if (rec && (e = tc_cluster_decode(d, p, codes, params, assign, cent, dec, rec, st)) != cudaSuccess) return e;
+      // K and V share each launch: the token pass of both, then the decode of both
+      void* const codes[2] = {c->k_codes, c->v_codes};
+      void* const params[2] = {c->k_params, c->v_params};
+      void* const assign[2] = {c->k_assign, c->v_assign};
+      if (enc) {
+        const void* const X[2] = {K, V};
+        const float* const cnc[2] = {cns[0], cns[1]};
+        if ((e = tc_cluster_encode(d, p, X, cnc, Ps, codes, params, assign, st)) != cudaSuccess) return e;
       }
-      return cudaSuccess;
+      // the encode's reconstruction is the decode of what it wrote, so the two agree bit for bit
+      const void* const ccodes[2] = {codes[0], codes[1]};
+      const void* const cparams[2] = {params[0], params[1]};
+      const void* const cassign[2] = {assign[0], assign[1]};
+      void* const rec[2] = {Kr, Vr};
+      return tc_cluster_decode(d, p, ccodes, cparams, cassign, rec, st);
     }
   }
   for (int which = 0; which < 2; ++which) {

@@ -37,11 +37,14 @@ bool tc_cluster_supported(const kvc_layer_desc* d, const kvc_predictor* p);
 // the encode of either tensor reads its P
 cudaError_t tc_cluster_prepare(const kvc_layer_desc* d, const kvc_predictor* p, const float* const cnorm[2],
                                float* const P[2], cudaStream_t st);
-cudaError_t tc_cluster_encode(const kvc_layer_desc* d, const kvc_predictor* p, const void* X, const void* cent,
-                              const void* enc, const float* cnorm, float* P, void* codes, void* params,
-                              void* assign, cudaStream_t st);
-cudaError_t tc_cluster_decode(const kvc_layer_desc* d, const kvc_predictor* p, const void* codes, const void* params,
-                              const void* assign, const void* cent, const void* dec, void* out, cudaStream_t st);
+// The token pass of both tensors (K: [0], V: [1]) in one launch
+cudaError_t tc_cluster_encode(const kvc_layer_desc* d, const kvc_predictor* p, const void* const X[2],
+                              const float* const cnorm[2], float* const P[2], void* const codes[2],
+                              void* const params[2], void* const assign[2], cudaStream_t st);
+// x^ = c_a + coef^ W_dec^T for each tensor whose out[w] is given, in one launch
+cudaError_t tc_cluster_decode(const kvc_layer_desc* d, const kvc_predictor* p, const void* const codes[2],
+                              const void* const params[2], const void* const assign[2], void* const out[2],
+                              cudaStream_t st);
 // reads the device error word of the current device and resets it to 0
 cudaError_t tc_read_and_clear_error(unsigned int* value);
 // device address of the error word on the current device (nullptr on failure)

@@ -29,6 +29,7 @@ namespace tc {
 bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 bool map2d_bytes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                  uint32_t box_rows);
+bool map2d_bytes_sw64(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 namespace cluster {
 
@@ -280,7 +281,7 @@ constexpr int kDecSmem = kDecBar + 1024 + 1024;
 
 struct DecMaps {
   CUtensorMap dec;  // [C][128], box 256 rows
-  CUtensorMap out;  // x^ [T][C] as bytes, box 32 rows x 64 bytes
+  CUtensorMap out;  // x^ [T][C] as bytes, box 32 rows x 64 bytes, 64-byte swizzle
 };
 struct DecArgs {
   unsigned* err;
@@ -293,8 +294,15 @@ struct DecArgs {
   __nv_bfloat16* out;         // [T][C]
 };
 
+// blockIdx.y selects the tensor (maps0 / a0 or maps1 / a1): the K and V decodes
+// of a layer share one launch, so that their 2 x 256 tiles fill the SMs' waves
+// together.
 template <int BITS, int G>
-__global__ void __launch_bounds__(kDecThreads, 1) dec_kernel(const __grid_constant__ DecMaps maps, const DecArgs a) {
+__global__ void __launch_bounds__(kDecThreads, 1)
+    dec_kernel(const __grid_constant__ DecMaps maps0, const DecArgs a0, const __grid_constant__ DecMaps maps1,
+               const DecArgs a1) {
+  const DecMaps& maps = blockIdx.y ? maps1 : maps0;
+  const DecArgs a = blockIdx.y ? a1 : a0;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecBar);
@@ -446,25 +454,38 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_kernel(const __grid_consta
       fence_async_smem();
       mbar_arrive(a_ready);
     }
+    // The centre rows are gathered coalesced: lane l fetches the 16-byte piece
+    // l & 3 of the 64 bytes a box holds for rows (l >> 2) + 8 j, j = 0..3, of
+    // this warp's 32 tokens (a load instruction covers 8 rows x 64 contiguous
+    // bytes; a row per lane would touch 32 lines per instruction).
     int c = t < a.T ? (int)a.assign[t] : 0;
     c = c < a.n_c ? c : a.n_c - 1;
-    const __nv_bfloat16* crow = a.cent + (int64_t)c * a.C;
+    const __nv_bfloat16* cbase[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int cj = __shfl_sync(0xffffffffu, c, (lane >> 2) + 8 * j);
+      cbase[j] = a.cent + (int64_t)cj * a.C + (lane & 3) * 8;
+    }
     // x^ leaves through shared memory and TMA stores (row-per-thread global
     // stores cost a request per 16 bytes): per 32 columns the warp fills one of
-    // its two [32 rows][64 bytes] boxes, a lane writing its row's 16-byte pieces
-    // in an order rotated by lane / 2 so that a store instruction touches eight
-    // different bank groups
+    // its two [32 rows][64 bytes] boxes, laid out with the 64-byte swizzle (the
+    // store's tensor map undoes it): piece q of row r at chunk q ^ ((r >> 1) & 3).
+    // The gathered centre pieces are first written to the box (8 whole rows per
+    // instruction); each lane then reads its own row's four pieces, adds the
+    // product and writes the result in place.  The swizzle spreads a row-per-lane
+    // access of one piece over eight bank groups.
+    auto sw = [](int r, int q) { return r * 64 + ((q ^ ((r >> 1) & 3)) << 4); };
     uint8_t* obox = smem + kDecOut + (warp - 2) * 4096;
     int ob = 0;
     for (int n = 0; n < NN; ++n) {
       const int b = n & 1;
-      // this half chunk's centre values, fetched while the MMAs run
+      // this half chunk's centre pieces, fetched while the MMAs run
       uint4 cv[16];
-      {
-        const uint4* cr = reinterpret_cast<const uint4*>(crow + n * 256 + grp * 128);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) cv[i] = __ldg(cr + i);
-      }
+      for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          cv[cb * 4 + j] = __ldg(reinterpret_cast<const uint4*>(cbase[j] + n * 256 + grp * 128 + cb * 32));
       wait(&acc_full[b], (n >> 1) & 1, abort_flag, a.err, 0x3600u + b);
       tc_fence_after();
 #pragma unroll
@@ -472,24 +493,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) dec_kernel(const __grid_consta
         const int col = n * 256 + grp * 128 + cb * 32;  // output channel
         float v[32];
         tmem_ld32(lane_addr + b * 256 + grp * 128 + cb * 32, v);
-        uint4 w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float cc[8];
-          unpack_bf16x8(cv[cb * 4 + i], cc, 0);
-          w[i] = make_uint4(pack_bf16x2(cc[0] + v[8 * i], cc[1] + v[8 * i + 1]),
-                            pack_bf16x2(cc[2] + v[8 * i + 2], cc[3] + v[8 * i + 3]),
-                            pack_bf16x2(cc[4] + v[8 * i + 4], cc[5] + v[8 * i + 5]),
-                            pack_bf16x2(cc[6] + v[8 * i + 6], cc[7] + v[8 * i + 7]));
-        }
         uint8_t* box = obox + ob * 2048;
         if (lane == 0) bulk_wait_read1();  // the store that last read this box is done with it
         __syncwarp();
 #pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(box + sw((lane >> 2) + 8 * j, lane & 3)) = cv[cb * 4 + j];
+        __syncwarp();
+#pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int j = (i + (lane >> 1)) & 3;
-          const uint4 val = j == 0 ? w[0] : (j == 1 ? w[1] : (j == 2 ? w[2] : w[3]));
-          *reinterpret_cast<uint4*>(box + lane * 64 + j * 16) = val;
+          uint4* piece = reinterpret_cast<uint4*>(box + sw(lane, i));
+          float cc[8];
+          unpack_bf16x8(*piece, cc, 0);
+          const float* vi = v + 8 * i;
+          *piece = make_uint4(pack_bf16x2(cc[0] + vi[0], cc[1] + vi[1]), pack_bf16x2(cc[2] + vi[2], cc[3] + vi[3]),
+                              pack_bf16x2(cc[4] + vi[4], cc[5] + vi[5]), pack_bf16x2(cc[6] + vi[6], cc[7] + vi[7]));
         }
         fence_async_smem();
         __syncwarp();
@@ -525,12 +543,14 @@ static cudaError_t launch_enc(const EncMaps& m, const EncArgs& a, cudaStream_t s
   count_launches(1);
   return cudaGetLastError();
 }
+// one tensor (n = 1) or two of the same row count (n = 2: m[1] / a[1] as the second)
 template <int BITS, int G>
-static cudaError_t launch_dec(const DecMaps& m, const DecArgs& a, cudaStream_t st) {
+static cudaError_t launch_dec(const DecMaps* m, const DecArgs* a, int n, cudaStream_t st) {
   auto k = dec_kernel<BITS, G>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
   if (e != cudaSuccess) return e;
-  k<<<(unsigned)((a.T + 127) / 128), kDecThreads, kDecSmem, st>>>(m, a);
+  const dim3 grid((unsigned)((a[0].T + 127) / 128), (unsigned)n);
+  k<<<grid, kDecThreads, kDecSmem, st>>>(m[0], a[0], m[n - 1], a[n - 1]);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -549,22 +569,30 @@ bool tc_cluster_supported(const kvc_layer_desc* d, const kvc_predictor* p) {
   return true;
 }
 
-cudaError_t tc_cluster_encode(const kvc_layer_desc* d, const kvc_predictor* p, const void* X, const void* cent,
-                              const void* enc, const float* cnorm, float* P, void* codes, void* params,
-                              void* assign, cudaStream_t st) {
+cudaError_t tc_cluster_encode(const kvc_layer_desc* d, const kvc_predictor* p, const void* const X[2],
+                              const float* const cnorm[2], float* const P[2], void* const codes[2],
+                              void* const params[2], void* const assign[2], cudaStream_t st) {
   const uint64_t T = (uint64_t)d->n_tokens, C = (uint64_t)d->n_heads * d->head_dim;
-  tc::cluster::EncMaps m;
-  memset(&m, 0, sizeof(m));
-  if (!(tc::map2d(&m.x, X, T, C, 128) && tc::map2d(&m.cent, cent, (uint64_t)p->n_clusters, C, 256) &&
-        tc::map2d(&m.enc, enc, 128, C, 128)))
-    return cudaErrorInvalidValue;
+  const void* cent[2] = {p->k_centroids, p->v_centroids};
+  const void* enc[2] = {p->k_enc, p->v_enc};
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
-  tc::cluster::EncArgs a{err, (int64_t)T, (int)C, p->n_clusters, cnorm, P, (uint8_t*)codes, (__half2*)params,
-                         (uint8_t*)assign};
+  tc::cluster::EncMaps m[2];
+  tc::cluster::EncArgs a[2];
+  for (int w = 0; w < 2; ++w) {
+    memset(&m[w], 0, sizeof(m[w]));
+    if (!(tc::map2d(&m[w].x, X[w], T, C, 128) && tc::map2d(&m[w].cent, cent[w], (uint64_t)p->n_clusters, C, 256) &&
+          tc::map2d(&m[w].enc, enc[w], 128, C, 128)))
+      return cudaErrorInvalidValue;
+    a[w] = tc::cluster::EncArgs{err, (int64_t)T, (int)C, p->n_clusters, cnorm[w], P[w], (uint8_t*)codes[w],
+                                (__half2*)params[w], (uint8_t*)assign[w]};
+  }
+  using namespace tc::cluster;
   if (d->bits == 2)
-    return d->group == 32 ? tc::cluster::launch_enc<2, 32>(m, a, st) : tc::cluster::launch_enc<2, 64>(m, a, st);
-  return d->group == 32 ? tc::cluster::launch_enc<4, 32>(m, a, st) : tc::cluster::launch_enc<4, 64>(m, a, st);
+    return d->group == 32 ? launch_enc<2, 32>(m[0], a[0], st, 2, &m[1], &a[1])
+                          : launch_enc<2, 64>(m[0], a[0], st, 2, &m[1], &a[1]);
+  return d->group == 32 ? launch_enc<4, 32>(m[0], a[0], st, 2, &m[1], &a[1])
+                        : launch_enc<4, 64>(m[0], a[0], st, 2, &m[1], &a[1]);
 }
 
 cudaError_t tc_cluster_prepare(const kvc_layer_desc* d, const kvc_predictor* p, const float* const cnorm[2],
@@ -587,20 +615,32 @@ cudaError_t tc_cluster_prepare(const kvc_layer_desc* d, const kvc_predictor* p, 
   return tc::cluster::launch_enc<4, 32, true>(m[0], a[0], st, 2, &m[1], &a[1]);
 }
 
-cudaError_t tc_cluster_decode(const kvc_layer_desc* d, const kvc_predictor* p, const void* codes, const void* params,
-                              const void* assign, const void* cent, const void* dec, void* out, cudaStream_t st) {
+cudaError_t tc_cluster_decode(const kvc_layer_desc* d, const kvc_predictor* p, const void* const codes[2],
+                              const void* const params[2], const void* const assign[2], void* const out[2],
+                              cudaStream_t st) {
   const uint64_t T = (uint64_t)d->n_tokens, C = (uint64_t)d->n_heads * d->head_dim;
-  tc::cluster::DecMaps m;
-  memset(&m, 0, sizeof(m));
-  if (!tc::map2d(&m.dec, dec, C, 128, 256) || !tc::map2d_bytes(&m.out, out, T, C * 2, 64, 32))
-    return cudaErrorInvalidValue;
+  const void* cent[2] = {p->k_centroids, p->v_centroids};
+  const void* dec[2] = {p->k_dec, p->v_dec};
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
-  tc::cluster::DecArgs a{err, (int64_t)T, (int)C, p->n_clusters, (const uint8_t*)codes, (const __half2*)params,
-                         (const uint8_t*)assign, (const __nv_bfloat16*)cent, (__nv_bfloat16*)out};
+  tc::cluster::DecMaps m[2];
+  tc::cluster::DecArgs a[2];
+  int n = 0;
+  for (int w = 0; w < 2; ++w) {
+    if (!out[w]) continue;
+    memset(&m[n], 0, sizeof(m[n]));
+    if (!tc::map2d(&m[n].dec, dec[w], C, 128, 256) || !tc::map2d_bytes_sw64(&m[n].out, out[w], T, C * 2, 32))
+      return cudaErrorInvalidValue;
+    a[n] = tc::cluster::DecArgs{err, (int64_t)T, (int)C, p->n_clusters, (const uint8_t*)codes[w],
+                                (const __half2*)params[w], (const uint8_t*)assign[w], (const __nv_bfloat16*)cent[w],
+                                (__nv_bfloat16*)out[w]};
+    ++n;
+  }
+  if (n == 0) return cudaSuccess;
+  using namespace tc::cluster;
   if (d->bits == 2)
-    return d->group == 32 ? tc::cluster::launch_dec<2, 32>(m, a, st) : tc::cluster::launch_dec<2, 64>(m, a, st);
-  return d->group == 32 ? tc::cluster::launch_dec<4, 32>(m, a, st) : tc::cluster::launch_dec<4, 64>(m, a, st);
+    return d->group == 32 ? launch_dec<2, 32>(m, a, n, st) : launch_dec<2, 64>(m, a, n, st);
+  return d->group == 32 ? launch_dec<4, 32>(m, a, n, st) : launch_dec<4, 64>(m, a, n, st);
 }
 
 }  // namespace kvc
