@@ -41,14 +41,16 @@ template <bool JC>
 struct Cfg {
   static constexpr int kWarps = JC ? 7 : 6;
   static constexpr int kThreads = kWarps * 32;
-  static constexpr int S = JC ? 2 : 3;  // K / V tile pairs in flight
+  static constexpr int S = 3;  // K / V tile pairs in flight
   // shared memory (offsets from a 1024-aligned base)
-  static constexpr int kQ = 0;                    // Q tile, two [128][64] sub-tiles
+  // Q tile, two [128][64] sub-tiles.  Once Q is in tensor memory, JC keeps the
+  // Jensen operands in its first sub-tile, four K = 16 slices of 16 columns:
+  // slice 0 the A operand, slice 1 + s the B operand of stage s.
+  static constexpr int kQ = 0;
   static constexpr int kK = kQ + 32768;           // K tiles [S]
   static constexpr int kV = kK + S * 32768;       // V tiles [S]
-  static constexpr int kQx = kV + S * 32768;      // JC: A of the Jensen MMA, [128][64] (16 columns used)
-  static constexpr int kKx = kQx + (JC ? 16384 : 0);  // JC: B of the Jensen MMA [S]
-  static constexpr int kBar = kKx + (JC ? S * 16384 : 0);
+  static constexpr int kBar = kV + S * 32768;
+  static_assert(!JC || S <= 3, "the Jensen tile holds the A slice and one B slice per stage");
   static constexpr int kSmem = kBar + 1024 + 1024;  // + barriers + alignment slack
 };
 
@@ -237,8 +239,7 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
   uint8_t* Qs = smem + L::kQ;
   auto Kt = [&](int s) { return smem + L::kK + s * 32768; };
   auto Vt = [&](int s) { return smem + L::kV + s * 32768; };
-  uint8_t* Qx = smem + L::kQx;
-  auto Kx = [&](int s) { return smem + L::kKx + s * 16384; };
+  uint8_t* X = smem + L::kQ;  // JC: the Jensen operands, after Q has moved to tensor memory
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -308,8 +309,10 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
             const uint32_t off = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
             umma_ts(SC(b), QC + k * 8, kd + off, id128, k == 0 ? 0u : 1u);
           }
-          if (JC && j < NH)  // the Jensen term of the history keys: one K = 16 step
-            umma(SC(b), desc_sw128(smem_u32(Qx)), desc_sw128(smem_u32(Kx(s))), id128, 1u);
+          if (JC && j < NH) {  // the Jensen term of the history keys: one K = 16 step (slices 0 and 1 + s)
+            const uint64_t xd = desc_sw128(smem_u32(X));
+            umma(SC(b), xd, xd + 2 * (s + 1), id128, 1u);
+          }
           umma_commit(&s_full[b]);
         }
         if (j >= 1) {
@@ -452,31 +455,41 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
     }
   } else if (JC) {
     // ================================================================ Jensen operands (warp 6)
-    // A (once): row r, logical column g < NG holds -|q_g|^2 * 0.5 scale / 12;
-    // B (per history tile): key row k, column g holds s_g^2.  Logical columns
-    // NG .. 15 are zero; the MMA reads columns 0 .. 15 of the 128-byte-swizzled rows.
+    // A (once, slice 0): row r, logical column g < NG holds -|q_g|^2 * 0.5 scale / 12;
+    // B (per history tile, slice 1 + stage): key row k, column g holds s_g^2.
+    // Logical columns NG .. 15 of a slice are zero; the MMA reads the slice's
+    // 16 columns of the 128-byte-swizzled rows.  The tile lies over Q's first
+    // sub-tile, so it is written once the softmax warps have moved Q to tensor
+    // memory (and this warp has read the rows it needs).
     constexpr int GQ = 128 / NG;  // channels per group
     if (!wait(q_full, 0, abort_flag, a.err, 0x1600u)) {
       // the MMA warp gives up as well
     } else {
-      for (int r = lane; r < 128; r += 32) {
-        float qn[NG];
+      float qn[4][NG];  // rows lane + 32 i
 #pragma unroll
-        for (int g = 0; g < NG; ++g) qn[g] = 0.f;
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane + 32 * i;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) qn[i][g] = 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {  // 16-byte chunk k of the row: elements 8k .. 8k + 7
           const uint4 u = *reinterpret_cast<const uint4*>(Qs + (k / 8) * 16384 + sw128_off(r, k % 8));
           float x[8];
           unpack_bf16x8(u, x, 0);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) qn[(8 * k) / GQ] = fmaf(x[i], x[i], qn[(8 * k) / GQ]);
+          for (int e = 0; e < 8; ++e) qn[i][(8 * k) / GQ] = fmaf(x[e], x[e], qn[i][(8 * k) / GQ]);
         }
+      }
+      wait(q_tmem, 0, abort_flag, a.err, 0x1601u);  // after an abort the MMA warp issues nothing
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane + 32 * i;
         float v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = i < NG ? qn[i] * a.jensen_a : 0.f;
+        for (int g = 0; g < 16; ++g) v[g] = g < NG ? qn[i][g] * a.jensen_a : 0.f;
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch)
-          *reinterpret_cast<uint4*>(Qx + sw128_off(r, ch)) =
+          *reinterpret_cast<uint4*>(X + sw128_off(r, ch)) =
               make_uint4(pack_bf16x2(v[8 * ch], v[8 * ch + 1]), pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
                          pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]), pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
       }
@@ -518,7 +531,7 @@ __global__ void __launch_bounds__(Cfg<JC>::kThreads, 1)
           }
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch)
-            *reinterpret_cast<uint4*>(Kx(s) + sw128_off(r, ch)) =
+            *reinterpret_cast<uint4*>(X + sw128_off(r, 2 * (s + 1) + ch)) =
                 make_uint4(pack_bf16x2(v[8 * ch], v[8 * ch + 1]), pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
                            pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]), pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
         }
