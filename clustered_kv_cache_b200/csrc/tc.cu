@@ -176,7 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   uint64_t* mma_done = khat_stored + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* s_cb = reinterpret_cast<float*>(smem + L::kBarOff + 512);  // EDEN-2 codebook
+  float* s_cb = reinterpret_cast<float*>(smem + L::kBarOff + 512);  // EDEN-2 codebook [16][2]
+  // the search's form of point j: (-2 c_j0, -2 c_j1, |c_j|^2, 0)
+  float4* s_cq = reinterpret_cast<float4*>(smem + L::kBarOff + 640);  // [16]
   // item hand-off ring of a dynamically scheduled call: slot k & 3 holds the k-th
   // item of this CTA (-1: none) and whether its K latent was loaded ahead
   uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff + 256);  // [4]
@@ -254,8 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     mbar_init(mma_done, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&item_bar[i], 1);
     *abort_flag = 0;
-    if (EDEN)
+    if (EDEN) {
       for (int i = 0; i < 32; ++i) s_cb[i] = a.codebook[i];
+      for (int j = 0; j < 16; ++j) {
+        const float c0 = a.codebook[2 * j], c1 = a.codebook[2 * j + 1];
+        s_cq[j] = make_float4(-2.f * c0, -2.f * c1, fmaf(c0, c0, c1 * c1), 0.f);
+      }
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_async_smem();
   }
@@ -927,19 +934,23 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
             const float inv_sigma = ss > 0.f ? 1.f / sigma : 0.f;
 #pragma unroll
             for (int e = 0; e < 64; ++e) y[e] *= inv_sigma;
+            // |u - c|^2 = |u|^2 + |c|^2 - 2 <u, c>: per pair the point with the least
+            // |c|^2 - 2 <u, c> (two FMAs); the index goes into the pair's nibble of
+            // gw with one three-input logic op (j replicated over all nibbles)
             float bd[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) bd[i] = INFINITY;
 #pragma unroll 1
             for (int j = 0; j < 16; ++j) {  // points in index order: a strict < keeps the lowest
-              const float c0 = s_cb[2 * j], c1 = s_cb[2 * j + 1];
+              const float4 cq = s_cq[j];
+              const uint32_t jr = (uint32_t)j * 0x11111111u;
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
-                const float d0 = y[2 * i] - c0, d1 = y[2 * i + 1] - c1;
-                const float d = fmaf(d0, d0, d1 * d1);
+                const float d = fmaf(y[2 * i], cq.x, fmaf(y[2 * i + 1], cq.y, cq.z));
                 if (d < bd[i]) {
                   bd[i] = d;
-                  gw[i / 8] = (gw[i / 8] & ~(15u << (4 * (i % 8)))) | ((uint32_t)j << (4 * (i % 8)));
+                  const uint32_t m = 15u << (4 * (i % 8));
+                  gw[i / 8] = (gw[i / 8] & ~m) | (jr & m);
                 }
               }
             }
