@@ -97,6 +97,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 16 or 32 consecutive fp32 TMEM columns of this thread's lane
+template <int W>
+__device__ __forceinline__ void tmem_ldw(uint32_t taddr, float (&v)[W]) {
+  static_assert(W == 16 || W == 32, "16 or 32 columns");
+  if constexpr (W == 16)
+    tmem_ld16(taddr, v);
+  else
+    tmem_ld32(taddr, v);
+}
 // 8 consecutive 32-bit TMEM columns of this thread's lane (no wait)
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&w)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(w[0]),
@@ -321,8 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
         asm volatile("bar.sync 1, 256;" ::: "memory");
     };
     const int64_t nff = a.T / F;  // whole frames
-    constexpr int NG = 128 / G, NP = G / 32;
+    constexpr int NG = 128 / G;
     constexpr int NGH = NG / 2;  // groups of the half row
+    // accumulator columns per TMEM round trip: encode (x not in registers) 32,
+    // decode 16 (the register budget of 576 threads is 96 a thread)
+    constexpr int PW = ENC ? 32 : 16;
+    constexpr int NPW = G / PW;
     for (int f = 0; f < nf; ++f) {
       const int64_t n_f = (a.T - f * F) < F ? (a.T - f * F) : F;
       const bool valid = s < n_f;
@@ -336,17 +349,16 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
       const int64_t cofs = rowi < F0 * H ? rowi * arb : F0 * H * arb + (rowi - F0 * H) * row_bytes;
       uint8_t* codes = (isv ? a.vcodes : a.kcodes) + cofs + hc * half_bytes;
       __half2* params = (isv ? a.vparams : a.kparams) + rowi * NG + hc * NGH;
-      uint4 xin[8];
       uint4 cin[2];
       __half2 pin[NGH];
-      if (ENC) {  // x of this half row from the staged tile, which is then released
-        const int i = 2 * f + (isv ? 1 : 0);
-        wait(&x_full[2 * (i % 3) + (i & 1)], (i / 6) & 1, abort_flag, a.err, 0x2220u + isv);
-        read_half(xs(i), xin);
-        // the next TMA load into this slot is an async-proxy write: order this
-        // thread's generic reads of the slot before it
-        fence_async_smem();
-        mbar_arrive(&x_free[i % 3]);
+      // encode: x of this half row is read from its staged tile in both passes
+      // (x in registers would cost 32 of the 96; the tile is released at the end)
+      const int xi = 2 * f + (isv ? 1 : 0);  // ring item of x
+      auto xq = [&](int c8) {  // 16-byte chunk c8 (elements 8 c8 .. 8 c8 + 7) of the half row
+        return *reinterpret_cast<const uint4*>(xs(xi) + hc * 16384 + sw128_off(row, c8));
+      };
+      if (ENC) {
+        wait(&x_full[2 * (xi % 3) + (xi & 1)], (xi / 6) & 1, abort_flag, a.err, 0x2220u + isv);
       } else {
 #pragma unroll
         for (int i = 0; i < 2; ++i)
@@ -376,18 +388,18 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
         if (ENC) {
           float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-          for (int pc = 0; pc < 2 * NP; ++pc) {  // 16 columns at a time (the register budget)
-            float p[16];
+          for (int pc = 0; pc < NPW; ++pc) {
+            float p[PW];
             if (anchor) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) p[i] = 0.f;
+              for (int i = 0; i < PW; ++i) p[i] = 0.f;
             } else {
-              tmem_ld16(acc_addr + g * G + pc * 16, p);
+              tmem_ldw(acc_addr + g * G + pc * PW, p);
             }
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int ch = 0; ch < PW / 8; ++ch) {
               float x[8];
-              unpack_bf16x8(xin[(gh * G + pc * 16) / 8 + ch], x, 0);
+              unpack_bf16x8(xq((gh * G + pc * PW) / 8 + ch), x, 0);
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const float r = x[i] - p[ch * 8 + i];
@@ -408,24 +420,24 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
         }
         const float inv = sf > 0.f ? 1.f / sf : 0.f;
 #pragma unroll
-        for (int pc = 0; pc < 2 * NP; ++pc) {
-          const int e0 = g * G + pc * 16;   // element of the row
-          const int h0 = gh * G + pc * 16;  // element of the half row
-          float p[16];
+        for (int pc = 0; pc < NPW; ++pc) {
+          const int e0 = g * G + pc * PW;   // element of the row
+          const int h0 = gh * G + pc * PW;  // element of the half row
+          float p[PW];
           if (anchor) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) p[i] = 0.f;
+            for (int i = 0; i < PW; ++i) p[i] = 0.f;
           } else {
-            tmem_ld16(acc_addr + e0, p);
+            tmem_ldw(acc_addr + e0, p);
           }
-          uint32_t recw[8];  // 16 reconstructed values as bf16 pairs
+          uint32_t recw[PW / 2];  // PW reconstructed values as bf16 pairs
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
+          for (int ch = 0; ch < PW / 8; ++ch) {
             const int e = h0 + ch * 8;
             float r[8];  // reconstruction
             if (ENC) {
               float x[8];
-              unpack_bf16x8(xin[e / 8], x, 0);
+              unpack_bf16x8(xq(e / 8), x, 0);
               if (bits == 2)
                 cw[e / 16] |= quant8<2>(x, &p[ch * 8], sf, zf, inv, r) << ((e % 16) * 2);
               else
@@ -440,10 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
             for (int i = 0; i < 4; ++i) recw[ch * 4 + i] = pack_bf16x2(r[2 * i], r[2 * i + 1]);
           }
           // the slot was last read by this frame's prediction, which is complete (acc_full)
-          tmem_st8(state + e0 / 2, recw);
+#pragma unroll
+          for (int k = 0; k < PW / 16; ++k)
+            tmem_st8(state + e0 / 2 + 8 * k, *reinterpret_cast<const uint32_t(*)[8]>(&recw[8 * k]));
           if (stage) {
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int ch = 0; ch < PW / 8; ++ch) {
               const int e = e0 + ch * 8;
               *reinterpret_cast<uint4*>(stile + (e / 64) * 16384 + sw128_off(row, (e % 64) / 8)) =
                   make_uint4(recw[4 * ch], recw[4 * ch + 1], recw[4 * ch + 2], recw[4 * ch + 3]);
@@ -451,10 +465,16 @@ __global__ void __launch_bounds__(kThreads, 1) temporal_kernel(const __grid_cons
           } else if (rec && valid) {
             uint4* dst = reinterpret_cast<uint4*>(rec + t * C + h * 128 + e0);
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
+            for (int ch = 0; ch < PW / 8; ++ch)
               dst[ch] = make_uint4(recw[4 * ch], recw[4 * ch + 1], recw[4 * ch + 2], recw[4 * ch + 3]);
           }
         }
+      }
+      if (ENC) {
+        // x is read: the next TMA load into this slot is an async-proxy write, so
+        // this thread's generic reads of the slot are ordered before it
+        fence_async_smem();
+        mbar_arrive(&x_free[xi % 3]);
       }
       if (ENC && valid) {
         uint4* dst = reinterpret_cast<uint4*>(codes);
