@@ -51,9 +51,9 @@ TRAFFIC = {"encode_xlayer": 678559232 + 188143104, "decode_xlayer": 428340480 + 
            "encode_xlayer_fused": (2837343488 + 916343040) // 4, "decode_xlayer_fused": (2087463168 + 744328704) // 4,
            "attention_c2": 244925696 + 13229312, "attention_c4": 26443520 + 146944,
            "decode_c4": 9409024 + 214975232,
-           "temporal_encode": 1434010000 + 372614912,
-           "temporal_decode": 574324480 + 1285428224,
-           "eden2_encode": 664999168 + 177946880}
+           "temporal_encode": 1424011008 + 351590400,
+           "temporal_decode": 659118080 + 1286398464,
+           "eden2_encode": 664736000 + 177576448}
 
 
 def peaks():
