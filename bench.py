@@ -48,7 +48,7 @@ UNIT = "KV tokens/s"
 # set to None when a kernel changes after its capture.
 TRAFFIC = {"encode_xlayer": 678559232 + 188143104, "decode_xlayer": 428340480 + 137626112,
            # per layer of the fused walk (a 4-layer launch's DRAM bytes / 4; scaled by the layer count)
-           "encode_xlayer_fused": (2837343488 + 916343040) // 4, "decode_xlayer_fused": (2087463168 + 744328704) // 4,
+           "encode_xlayer_fused": (2882488064 + 912262656) // 4, "decode_xlayer_fused": (2091626496 + 743751424) // 4,
            "attention_c2": 244925696 + 13229312, "attention_c4": 26443520 + 146944,
            "decode_c4": 9409024 + 214975232,
            "temporal_encode": 1424011008 + 351590400,

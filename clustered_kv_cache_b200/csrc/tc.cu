@@ -179,11 +179,6 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   float* s_cb = reinterpret_cast<float*>(smem + L::kBarOff + 512);  // EDEN-2 codebook [16][2]
   // the search's form of point j: (-2 c_j0, -2 c_j1, |c_j|^2, 0)
   float4* s_cq = reinterpret_cast<float4*>(smem + L::kBarOff + 640);  // [16]
-  // item hand-off ring of a dynamically scheduled call: slot k & 3 holds the k-th
-  // item of this CTA (-1: none) and whether its K latent was loaded ahead
-  uint64_t* item_bar = reinterpret_cast<uint64_t*>(smem + L::kBarOff + 256);  // [4]
-  volatile int* s_item = reinterpret_cast<volatile int*>(smem + L::kBarOff + 288);  // [4]
-  volatile int* s_pf = s_item + 4;                                                 // [4]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H;
@@ -191,10 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   const int NCH = C / 64;
   // persistent CTAs: this CTA codes items blockIdx.x, blockIdx.x + gridDim.x, ...
   // An item is a tile of one layer; a multi-layer call orders them layer by
-  // layer, and the tile of layer l waits for the same tile of layer l-1.  A
-  // multi-layer call of single CTAs (DYN) instead takes its items in that order
-  // from a global ticket counter as it goes, so that a CTA slowed by a wait
-  // codes fewer items rather than holding up a fixed share.
+  // layer, and the tile of layer l waits for the same tile of layer l-1.
   // A pair (cluster of two) codes 256-token tiles: the even CTA (the leader,
   // which issues the MMAs) its first 128 tokens, the odd one the rest.
   const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
@@ -205,7 +197,6 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   const int ntiles = (int)((a.T + span - 1) / span);
   const int nitems = (MULTI ? a.n_layers : 1) * ntiles;
   const int my_tiles = unit < nitems ? (nitems - 1 - unit) / nunits + 1 : 0;  // items of this CTA
-  constexpr bool DYN = MULTI && !PAIR;
   auto item_of = [&](int it) { return unit + it * nunits; };  // the static order
   auto tile_t0 = [&](int i) { return (i % ntiles) * span + (int)crank * 128; };
   auto layer_of = [&](int i) { return MULTI ? i / ntiles : 0; };
@@ -222,19 +213,16 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   // stored its reconstruction
   constexpr unsigned flag_full = PAIR ? 4u : 2u;
   auto flag_of = [&](int l, int i) { return a.flags + (size_t)l * ntiles + i % ntiles; };
-  unsigned* ticket = a.flags + (size_t)(MULTI ? a.n_layers : 0) * ntiles;  // DYN: next item to take
   // the leader's barriers, as shared::cluster addresses (a pair's arrivals and TMA bytes land there)
   auto lead_bar = [&](uint64_t* b) { return PAIR ? mapa_rank(b, crank & ~1u) : smem_u32(b); };
   // With rank 64 the TMEM has room for two latent slots, so the next tile's K
   // latent streams in during this tile's V heads.
   constexpr bool OVL = RC == 1;
   // The next item's K latent is loaded during this item's V heads.  In a
-  // multi-layer call that needs the next item's own dependency first.  With the
-  // static order it is an earlier item (no cycle of waits) only while the grid
-  // has fewer units than a layer has tiles, so with more the overlap is off; with
-  // DYN the dependency is only tested, and an item whose dependency is not yet
-  // stored loads its latent when it starts.
-  const bool ovl = OVL && (DYN || !MULTI || nunits < ntiles);
+  // multi-layer call that needs the next item's own dependency first; it is an
+  // earlier item (no cycle of waits) only while the grid has fewer units than a
+  // layer has tiles, so with more the overlap is off (each item loads its latent).
+  const bool ovl = OVL && (!MULTI || nunits < ntiles);
   const int HH = 2 * H;  // heads per tile (K then V)
 
   if (threadIdx.x == 0) {
@@ -254,7 +242,6 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     mbar_init(z_ready, PAIR ? 2 : kGroupThreads);
     mbar_init(khat_stored, 2);
     mbar_init(mma_done, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(&item_bar[i], 1);
     *abort_flag = 0;
     if (EDEN) {
       for (int i = 0; i < 32; ++i) s_cb[i] = a.codebook[i];
@@ -288,21 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   auto stageB = [&](int s) { return smem + L::kStageOff + s * L::kStage + 16384; };
   auto recon = [&](int b) { return smem + L::kReconOff + b * L::kRecon; };
   const uint32_t in_base = smem_u32(smem + L::kInOff);
-  // DYN: wait until the producer has published this CTA's k-th item.  The wait
-  // does not end on an abort (the producer publishes a closing -1 on every path,
-  // and all threads of a group must walk the same items); it has a bound of its
-  // own, four times the producer's, which is longer than any producer wait.
-  auto item_wait = [&](int k) -> bool {
-    const long long w0 = clock64();
-    while (!mbar_test(&item_bar[k & 3], (k >> 2) & 1)) {
-      if (clock64() - w0 > 4 * kWaitBudget) {
-        *abort_flag = 1;
-        atomicCAS(a.err, 0u, 0xB10u);
-        return false;
-      }
-    }
-    return true;
-  };
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -404,36 +376,11 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           fence_async_global();
         }
       };
-      // DYN: one test of an item's dependency (no wait)
-      auto dep_ready = [&](int i) -> bool {
-        const int l = layer_of(i);
-        if (l == 0) return true;
-        unsigned v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag_of(l - 1, i)) : "memory");
-        if (v < flag_full) return false;
-        fence_async_global();
-        return true;
-      };
-      auto take = [&]() -> int {
-        if (!ok) return -1;
-        const int i = (int)atomicAdd(ticket, 1u);
-        return i < nitems ? i : -1;
-      };
-      int npub = 0;           // DYN: items published (the last may be the closing -1)
-      bool pub_open = false;  // the last one published is an item, not -1
-      auto publish = [&](int i, bool pf) {
-        s_item[npub & 3] = i;
-        s_pf[npub & 3] = pf ? 1 : 0;
-        mbar_arrive(&item_bar[npub & 3]);  // release: the slot is written before the phase completes
-        ++npub;
-        pub_open = i >= 0;
-      };
-      int cur = DYN ? take() : (my_tiles > 0 ? item_of(0) : -1);
+      int cur = my_tiles > 0 ? item_of(0) : -1;
       bool cur_pf = false;  // the current item's K latent was loaded during the previous item
-      if (DYN) publish(cur, false);
       for (int it = 0; cur >= 0 && ok; ++it) {
         const int t0 = tile_t0(cur);
-        int nxt = DYN ? -1 : (it + 1 < my_tiles ? item_of(it + 1) : -1);
+        const int nxt = it + 1 < my_tiles ? item_of(it + 1) : -1;
         bool nxt_pf = false;
         const Maps& mp = *LM(layer_of(cur));
         // the epilogue of head h reads its clean inputs (encode) or codes (decode)
@@ -475,15 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           for (int j = 0; j < 2; ++j)
             load(&mp.ko, h * 128 + j * 64, t0, pol_stream, &mp.bv, j * 64, h * 128, 16384);
           for (int j = 0; j < RC; ++j) load(nullptr, 0, 0, 0, &mp.uv, j * 64, h * 128, 16384);
-          if (h == 0) {  // the next item, and whether its K latent streams in now
-            if (DYN) {
-              nxt = take();
-              nxt_pf = ovl && nxt >= 0 && ok && dep_ready(nxt);
-              publish(nxt, nxt_pf);
-            } else {
-              nxt_pf = ovl && nxt >= 0;
-              if (nxt_pf) dep_wait(nxt);
-            }
+          if (h == 0) {  // whether the next item's K latent streams in now
+            nxt_pf = ovl && nxt >= 0;
+            if (nxt_pf) dep_wait(nxt);
           }
           if (nxt_pf) {  // the next item's K latent, interleaved with the V heads
             const Maps& nm = *LM(layer_of(nxt));
@@ -495,7 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         cur = nxt;
         cur_pf = nxt_pf;
       }
-      if (DYN && pub_open) publish(-1, false);  // an abort left the walk early: close it
       if (!ok && (!PAIR || leader)) {
         // drain: the loads already issued must land before the CTA exits
         for (int i = 0; i < S; ++i) {
@@ -610,31 +550,9 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       auto acq = [&](int b) {
         if (use[b] >= 1) wt(&acc_empty[b], (use[b] - 1) & 1, 0x400u + b);
       };
-      // the k-th item's state: 0 none, 1 an item, 2 an item whose K latent is
-      // loaded during item k-1.  DYN: the sync warp reads the hand-off slot and
-      // passes the state to the issuing warp through one barrier reduction (the
-      // issuing warp reads no shared memory).
-      auto item_state = [&](int k) -> int {
-        if constexpr (DYN) {
-          bool has = false, pf = false;
-          if (!ISSUE) {
-            if (lane == 0) item_wait(k);
-            __syncwarp();
-            has = s_item[k & 3] >= 0;
-            pf = has && s_pf[k & 3] != 0;
-          }
-          const uint32_t pred = (!ISSUE && ((lane == 0 && has) || (lane == 1 && pf))) ? 1u : 0u;
-          uint32_t n;
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.popc.u32 %0, 3, 64, p;\n\t}"
-              : "=r"(n)
-              : "r"(pred)
-              : "memory");
-          return (int)n;
-        } else {
-          return k < my_tiles ? (ovl && k > 0 ? 2 : 1) : 0;
-        }
-      };
+      // the k-th item's state: 0 none, 1 an item, 2 an item whose K latent was
+      // loaded during item k-1
+      auto item_state = [&](int k) -> int { return k < my_tiles ? (ovl && k > 0 ? 2 : 1) : 0; };
       int st_cur = item_state(0);
       for (int it = 0; st_cur; ++it) {
         const uint32_t zk = zk_col(it), zv = zv_col(it);
@@ -1119,12 +1037,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     // After an abort every wait returns at once; the loops still run to the end
     // so that all threads of a group meet at every named barrier.
     for (int it = 0;; ++it) {
-      int cur;
-      if constexpr (DYN) {
-        cur = item_wait(it) ? s_item[it & 3] : -1;
-      } else {
-        cur = it < my_tiles ? item_of(it) : -1;
-      }
+      const int cur = it < my_tiles ? item_of(it) : -1;
       if (cur < 0) break;
       const int t0 = tile_t0(cur), l = layer_of(cur);
       // the item's K latent (loaded at its start, or during the previous item's V heads)
@@ -1272,10 +1185,11 @@ static int sm_count() {
 }
 
 // Decode runs as CTA pairs (each SM streams half of every weight box; measured
-// 7% faster); encode as single CTAs, whose heavier epilogue gains nothing from
-// the pair's lock step.
-template <int MODE>
-constexpr bool kPaired = MODE == kDecode;
+// 7% faster).  A one-layer encode runs as single CTAs, whose heavier epilogue
+// gains nothing from the pair's lock step; a multi-layer encode, whose items
+// fill each other's wave tails, runs as pairs (29 layers: 6.1 -> 5.8 ms).
+template <int MODE, bool MULTI>
+constexpr bool kPaired = MODE == kDecode || MULTI;
 
 // Multi-layer launches wait across CTAs (a tile of layer l on the same tile of
 // layer l-1), so their grid is at most what is resident at once.
@@ -1284,7 +1198,7 @@ static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
   const int64_t nl = MULTI ? a.n_layers : 1;
-  if constexpr (!kPaired<MODE>) {
+  if constexpr (!kPaired<MODE, MULTI>) {
     auto k = xlayer_tc_kernel<MODE, G, RC, BITS, false, EDEN, MULTI>;
     const int smem = Layout<RC, false>::kBytes + 1024;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1394,10 +1308,12 @@ size_t tc_workspace(int op, const kvc_layer_desc* d, const kvc_predictor* p, int
 
 namespace tc {
 // the tensor maps of one layer's call
-static bool layer_maps(Maps& m, const kvc_layer_desc* d, const kvc_predictor* p, bool enc, const void* K,
-                       const void* V, const void* Ks, const void* Vs, const kvc_codes* c, void* Kr, void* Vr) {
+// pair: the maps of a CTA-pair launch (half weight boxes), which decode and
+// multi-layer calls use
+static bool layer_maps(Maps& m, const kvc_layer_desc* d, const kvc_predictor* p, bool pair, bool enc,
+                       const void* K, const void* V, const void* Ks, const void* Vs, const kvc_codes* c, void* Kr,
+                       void* Vr) {
   const uint64_t T = (uint64_t)d->n_tokens, H = d->n_heads, C = H * 128;
-  const bool pair = !enc;  // decode runs as CTA pairs
   memset(&m, 0, sizeof(m));
   bool ok = map2d(&m.ks, Ks, T, C, 128) && map2d(&m.vs, Vs, T, C, 128) && map2d(&m.ko, Kr, T, C, 128) &&
             map2d(&m.vo, Vr ? Vr : Kr, T, C, 128) && weight_maps(m, d, p, pair);
@@ -1421,7 +1337,7 @@ cudaError_t tc_codec_layer(const kvc_layer_desc* d, const kvc_predictor* p, bool
                            cudaStream_t st) {
   const uint64_t H = d->n_heads, r = p->rank;
   tc::Maps m;
-  if (!tc::layer_maps(m, d, p, enc, K, V, Ks, Vs, c, Kr, Vr)) return cudaErrorInvalidValue;
+  if (!tc::layer_maps(m, d, p, !enc, enc, K, V, Ks, Vs, c, Kr, Vr)) return cudaErrorInvalidValue;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
   tc::Args a{err, (int64_t)d->n_tokens, (int)H, d->bits, tc::layer_ptrs(K, V, c), (enc && !Vr) ? 0 : 1,
@@ -1448,8 +1364,8 @@ bool tc_codec_layers_supported(const kvc_layer_desc* d, const kvc_predictor* pre
 
 size_t tc_codec_layers_workspace(const kvc_layer_desc* d, int n) {
   const size_t ntiles = ((size_t)d->n_tokens + 127) / 128;
-  // the layer table, then a counter per (layer, 128-token tile) and the item ticket
-  return align256u((size_t)n * sizeof(tc::LayerDev)) + align256u(((size_t)n * ntiles + 1) * sizeof(unsigned));
+  // the layer table, then a counter per (layer, 128-token tile)
+  return align256u((size_t)n * sizeof(tc::LayerDev)) + align256u((size_t)n * ntiles * sizeof(unsigned));
 }
 
 cudaError_t tc_codec_layers(const kvc_layer_desc* d, const kvc_predictor* preds, int n, bool enc,
@@ -1464,7 +1380,7 @@ cudaError_t tc_codec_layers(const kvc_layer_desc* d, const kvc_predictor* preds,
     const void* vs = i ? Vr[i - 1] : Vs0;
     const void* k = enc ? K[i] : nullptr;
     const void* v = enc ? V[i] : nullptr;
-    if (!tc::layer_maps(host[i].maps, d, &preds[i], enc, k, v, ks, vs, &c[i], Kr[i], Vr[i]))
+    if (!tc::layer_maps(host[i].maps, d, &preds[i], true, enc, k, v, ks, vs, &c[i], Kr[i], Vr[i]))
       return cudaErrorInvalidValue;
     host[i].p = tc::layer_ptrs(k, v, &c[i]);
   }
@@ -1474,7 +1390,7 @@ cudaError_t tc_codec_layers(const kvc_layer_desc* d, const kvc_predictor* preds,
   const size_t ntiles = ((size_t)d->n_tokens + 127) / 128;
   cudaError_t e = cudaMemcpyAsync(dev, host.data(), (size_t)n * sizeof(tc::LayerDev), cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(flags, 0, ((size_t)n * ntiles + 1) * sizeof(unsigned), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(flags, 0, (size_t)n * ntiles * sizeof(unsigned), st)) != cudaSuccess) return e;
   unsigned* err = tc_error_word();
   if (!err) return cudaErrorInvalidDevice;
   tc::Maps none;

@@ -1010,6 +1010,63 @@ def test_grouped_query_attention_cuda_core_path():
 # ---------------------------------------------------------------- the chain of layers in one call
 
 
+@pytest.mark.parametrize("case", ["fp32", "rank16", "mixed_ranks", "eden2"])
+def test_layer_chain_other_shapes_match_layer_calls(case):
+    """Shapes the fused walk does not take (fp32 values, a rank off the
+    tensor-core list, layers of different ranks, H64 / EDEN-2 residuals) run the
+    layers in turn inside kvc_encode_layers / kvc_decode_layers: every code,
+    parameter and reconstruction must equal the one-layer calls'."""
+    L, T, H, D = 4, 2 * 128 + 19, 3, 128
+    dtype = torch.float32 if case == "fp32" else torch.bfloat16
+    r0 = 16 if case in ("fp32", "rank16") else 64
+    wl = synth.wan_xlayer(seed=synth.SEED_BASE + 122, device="cuda", L=L, T=T, H=H, rank=r0, calib_tokens=512,
+                          dtype=dtype)
+    if case == "mixed_ranks":
+        wl128 = synth.wan_xlayer(seed=synth.SEED_BASE + 122, device="cuda", L=L, T=T, H=H, rank=128,
+                                 calib_tokens=512, layers_needed=[2])
+        preds = [kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl.weights[1], rank=64),
+                 kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl128.weights[2], rank=128),
+                 kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl.weights[3], rank=64)]
+    elif case == "eden2":
+        cb = synth.eden2_codebook().cuda()
+        preds = [kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl.weights[l], rank=r0, residual_codebook=cb)
+                 for l in range(1, L)]
+    else:
+        preds = [kvc.make_predictor(kvc.PRED_XLAYER_DPLR, wl.weights[l], rank=r0) for l in range(1, L)]
+    if case == "eden2":
+        desc = kvc.make_desc(T, H, D, dtype, 2, 64, torch.float16, residual_codec=kvc.RESIDUAL_H64_EDEN2)
+    else:
+        desc = _desc(T, H, D, dtype, 2, 32, torch.float32 if case == "fp32" else torch.float16)
+    n = L - 1
+    ref_codes, ref_K, ref_V = [], [], []
+    Ks, Vs = wl.K[0], wl.V[0]
+    for i in range(n):
+        buf = kvc.alloc_codes(desc, preds[i])
+        Kr, Vr = torch.empty_like(Ks), torch.empty_like(Vs)
+        kvc.kvc_encode_layer(desc, preds[i], wl.K[i + 1], wl.V[i + 1], Ks, Vs, buf, Kr, Vr,
+                             kvc.alloc_workspace(kvc.OP_ENCODE, desc, preds[i]))
+        ref_codes.append(buf), ref_K.append(Kr), ref_V.append(Vr)
+        Ks, Vs = Kr, Vr
+    _sync_ok()
+    codes = [kvc.alloc_codes(desc, p) for p in preds]
+    Kr = [torch.zeros_like(wl.K[0]) for _ in range(n)]
+    Vr = [torch.zeros_like(wl.V[0]) for _ in range(n)]
+    kvc.kvc_encode_layers(desc, preds, wl.K[1:], wl.V[1:], wl.K[0], wl.V[0], codes, Kr, Vr,
+                          kvc.alloc_layers_workspace(kvc.OP_ENCODE, desc, preds))
+    _sync_ok()
+    for i in range(n):
+        for name in ("k_codes", "k_params", "v_codes", "v_params"):
+            assert torch.equal(getattr(codes[i], name), getattr(ref_codes[i], name)), (case, i, name)
+        assert torch.equal(Kr[i], ref_K[i]) and torch.equal(Vr[i], ref_V[i]), (case, i)
+    Kd = [torch.zeros_like(wl.K[0]) for _ in range(n)]
+    Vd = [torch.zeros_like(wl.V[0]) for _ in range(n)]
+    kvc.kvc_decode_layers(desc, preds, codes, wl.K[0], wl.V[0], Kd, Vd,
+                          kvc.alloc_layers_workspace(kvc.OP_DECODE, desc, preds))
+    _sync_ok()
+    for i in range(n):
+        assert torch.equal(Kd[i], ref_K[i]) and torch.equal(Vd[i], ref_V[i]), (case, i)  # decode replays encode
+
+
 @pytest.mark.parametrize("L,T,H,rank,bits,group,pingpong", [(5, 3 * 128 + 41, 4, 64, 2, 32, False),
                                                             (5, 2 * 256 + 7, 3, 128, 4, 64, True),
                                                             (5, 300, 2, 0, 2, 64, True), (5, 128, 2, 64, 2, 32, False),
