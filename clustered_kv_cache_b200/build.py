@@ -12,7 +12,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libkvc.so")
-SOURCES = ["kvc_api.cu", "simt.cu", "tc.cu", "tc_attn.cu", "tc_temporal.cu", "tc_mixed.cu", "tc_cluster.cu", "noalloc.cu", "refit.cu"]
+SOURCES = ["kvc_api.cu", "simt.cu", "tc.cu", "tc_attn.cu", "tc_temporal.cu", "tc_mixed.cu", "tc_cluster.cu", "noalloc.cu",
+           "refit.cu", "anchor.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC,-fvisibility=hidden", "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills"]
 

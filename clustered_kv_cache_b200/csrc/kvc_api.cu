@@ -329,6 +329,10 @@ kvc_status codec_common(const kvc_layer_desc* d, const kvc_predictor* p, bool en
     cudaError_t e = tc_temporal_layer(d, p, enc, K, V, Ks, Vs, c, Kr, Vr, st);
     return e == cudaSuccess ? KVC_OK : cuda_fail(e);
   }
+  if (anchor_supported(d, p)) {
+    cudaError_t e = anchor_layer(d, enc, K, V, c, Kr, Vr, st);
+    return e == cudaSuccess ? KVC_OK : cuda_fail(e);
+  }
   Carve cv{(char*)ws, ws_bytes};
   return dispatch(d, [&](auto* ts, auto* tp) -> cudaError_t {
     using TS = std::remove_pointer_t<decltype(ts)>;
@@ -362,9 +366,12 @@ kvc_status attend_decoded(const kvc_layer_desc* d, const kvc_predictor* p, const
     if (K_rec_opt) Kh = (TS*)K_rec_opt;
     if (V_rec_opt) Vh = (TS*)V_rec_opt;
     if (d->n_tokens > 0) {
-      cudaError_t e = tc_codec_supported(d, p)
-                          ? tc_codec_layer(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh, nullptr, 0, st)
-                          : codec_xlayer<TS, TP>(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh, cv, st);
+      cudaError_t e =
+          tc_codec_supported(d, p)  ? tc_codec_layer(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh,
+                                                     nullptr, 0, st)
+          : anchor_supported(d, p) ? anchor_layer(d, false, nullptr, nullptr, codes, Kh, Vh, st)
+                                   : codec_xlayer<TS, TP>(d, p, false, nullptr, nullptr, K_src, V_src, codes, Kh, Vh,
+                                                          cv, st);
       if (e != cudaSuccess) return e;
     }
     if (tc_flash_supported(d))

@@ -45,6 +45,12 @@ cudaError_t tc_cluster_encode(const kvc_layer_desc* d, const kvc_predictor* p, c
 cudaError_t tc_cluster_decode(const kvc_layer_desc* d, const kvc_predictor* p, const void* const codes[2],
                               const void* const params[2], const void* const assign[2], void* const out[2],
                               cudaStream_t st);
+// The anchor layer (no predictor; bf16 values, fp16 (scale, zero), 2 or 4 bits,
+// groups of 32 or 64): a streaming kernel over both tensors, sharing the
+// quantizer arithmetic of the tensor-core epilogues (anchor.cu)
+bool anchor_supported(const kvc_layer_desc* d, const kvc_predictor* p);
+cudaError_t anchor_layer(const kvc_layer_desc* d, bool enc, const void* K, const void* V, const kvc_codes* c,
+                         void* Kr, void* Vr, cudaStream_t st);
 // reads the device error word of the current device and resets it to 0
 cudaError_t tc_read_and_clear_error(unsigned int* value);
 // device address of the error word on the current device (nullptr on failure)

@@ -108,6 +108,7 @@ def test_pack_unpack_bit_exact(bits):
     (torch.bfloat16, torch.float16, 4, 32, 300, 12, 128),
     (torch.bfloat16, torch.float16, 2, 32, 97, 3, 128),
     (torch.bfloat16, torch.float16, 2, 64, 65, 2, 64),
+    (torch.bfloat16, torch.float16, 4, 64, 33, 5, 128),
     (torch.float32, torch.float32, 4, 32, 130, 2, 64),
     (torch.bfloat16, torch.float16, 8, 16, 40, 2, 128),
 ])

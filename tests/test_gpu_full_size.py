@@ -322,3 +322,32 @@ def test_fused_layer_walk_at_the_benchmark_size():
             gc = O.Coded(q, s_[idx], z_[idx])
             kflip = _compare(gc, oc, sub(rec), ref, ex, sub(x), "bf16", 32, f"layer {l} {which} (sampled tokens)",
                              "f16", er, kflip)
+
+
+def test_anchor_layer_at_the_benchmark_size():
+    """The benchmark's INT4 g32 anchor layer (32760 tokens x 12 heads x 128, no
+    predictor) in the streaming launch it times: sampled tokens against the
+    oracle (tokens are independent), and the decode replays the encode."""
+    T, H, D = 32760, 12, 128
+    g = torch.Generator(device="cuda").manual_seed(2024)
+    K = (torch.randn(T, H, D, generator=g, device="cuda") * 1.5).to(torch.bfloat16)
+    V = torch.randn(T, H, D, generator=g, device="cuda").to(torch.bfloat16)
+    desc = _desc(T, H, D, torch.bfloat16, 4, 32, torch.float16)
+    pred = kvc.make_predictor(kvc.PRED_NONE)
+    buf = kvc.alloc_codes(desc, pred)
+    Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_encode_layer(desc, pred, K, V, None, None, buf, Kr, Vr)
+    Kd, Vd = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_decode_layer(desc, pred, buf, None, None, Kd, Vd)
+    assert kvc.kvc_get_device_error() == 0
+    assert torch.equal(Kd, Kr) and torch.equal(Vd, Vr)
+    idx = _rows(T, 256, 31)
+    ti = torch.from_numpy(idx).cuda()
+    od = _odesc(len(idx), H, D, torch.bfloat16, 4, 32, torch.float16)
+    ck, cv, Kh, Vh = O.encode_layer_none(od, U.to64(K[ti]), U.to64(V[ti]))
+    for which, oc, rec, ref, x in (("k", ck, Kr, Kh, K), ("v", cv, Vr, Vh, V)):
+        q = U.codes_from_gpu(getattr(buf, which + "_codes"), (T, H, D), 4)[idx]
+        s_, z_ = U.params_from_gpu(getattr(buf, which + "_params"), (T, H, D // 32), "f16")
+        gc = O.Coded(q, s_[idx], z_[idx])
+        _compare(gc, oc, U.to64(rec[ti]), ref, U.exact_none(oc, 32), U.to64(x[ti]), od.state, 32,
+                 which + " (sampled tokens)", "f16")
