@@ -58,7 +58,8 @@ struct EncArgs {
 
 // PMODE: the rows are the centres themselves and the kernel writes Y = C E^T to
 // P (fp32), so that a token equal to its centre gets Y - P[a] = 0 exactly (the
-// same products summed in the same order).  blockIdx.y selects the tensor
+// same products summed in the same order); it loads no centre box and issues
+// no S products, which P does not need.  blockIdx.y selects the tensor
 // (maps0 / a0 or maps1 / a1), so the short P passes of K and V share a launch.
 template <int BITS, int G, bool PMODE>
 __global__ void __launch_bounds__(kEncThreads, 1)
@@ -117,9 +118,10 @@ __global__ void __launch_bounds__(kEncThreads, 1)
       uint32_t issued_ph[kEncStages] = {};
       for (int c = 0; c < NCH; ++c) {
         if (!wait(&empty[s], ph ^ 1, abort_flag, a.err, 0x3100u + s)) break;
-        mbar_arrive_expect_tx(&full[s], (uint32_t)kEncStage);
+        // the P pass needs Y only: no centre box, and no S products below
+        mbar_arrive_expect_tx(&full[s], PMODE ? 32768u : (uint32_t)kEncStage);
         tma_load(stX(s), &maps.x, c * 64, t0, &full[s], pol_stream);
-        tma_load(stC(s), &maps.cent, c * 64, 0, &full[s], pol_keep);
+        if (!PMODE) tma_load(stC(s), &maps.cent, c * 64, 0, &full[s], pol_keep);
         tma_load(stE(s), &maps.enc, c * 64, 0, &full[s], pol_keep);
         issued[s] = 1;
         issued_ph[s] = ph;
@@ -149,8 +151,10 @@ __global__ void __launch_bounds__(kEncThreads, 1)
         const uint64_t ad = desc_sw128(smem_u32(stX(s)));
         const uint64_t cd = desc_sw128(smem_u32(stC(s)));
         const uint64_t ed = desc_sw128(smem_u32(stE(s)));
+        if (!PMODE) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma(SC, ad + 2 * k, cd + 2 * k, id256, (c == 0 && k == 0) ? 0u : 1u);
+          for (int k = 0; k < 4; ++k) umma(SC, ad + 2 * k, cd + 2 * k, id256, (c == 0 && k == 0) ? 0u : 1u);
+        }
 #pragma unroll
         for (int k = 0; k < 4; ++k) umma(YC, ad + 2 * k, ed + 2 * k, id128, (c == 0 && k == 0) ? 0u : 1u);
         umma_commit(&empty[s]);

@@ -549,6 +549,35 @@ def test_cluster_codec_parity(T, H, n_c):
     _check_cluster(cw, buf, Kr, Vr, T, H, D, bf, hf, n_c)
 
 
+def test_cluster_token_equal_to_its_centre_codes_zero():
+    """A token equal to a centre has the coefficients Y - P[a] = 0 exactly: P = C E^T
+    comes from the token pass's own products in the same order (the P pass over the
+    centre table).  Such tokens take that centre, and every (scale, zero) pair of
+    theirs is exactly 0, so their reconstruction is the centre itself."""
+    T, H, n_c = 333, 16, 256
+    cw = synth.cluster_layer(seed=synth.SEED_BASE + 105, T=T, H=H, n_c=n_c, iters=5)
+    D = 128
+    bf, hf = torch.bfloat16, torch.float16
+    rows = torch.arange(0, T, 7)
+    js = (rows * 37) % n_c
+    K, V = cw.K.clone(), cw.V.clone()
+    K.view(T, H * D)[rows] = cw.k_centroids[js].to(bf)
+    V.view(T, H * D)[rows] = cw.v_centroids[js].to(bf)
+    desc = _desc(T, H, D, bf, 4, 32, hf)
+    pred = _cluster_pred(cw, n_c)
+    buf = kvc.alloc_codes(desc, pred)
+    K, V = K.cuda(), V.cuda()
+    Kr, Vr = torch.empty_like(K), torch.empty_like(V)
+    kvc.kvc_encode_layer(desc, pred, K, V, None, None, buf, Kr, Vr, kvc.alloc_workspace(kvc.OP_ENCODE, desc, pred))
+    _sync_ok()
+    for which, X, rec in (("k", K, Kr), ("v", V, Vr)):
+        a = getattr(buf, which + "_assign").cpu().long()
+        assert torch.equal(a[rows], js), which
+        params = getattr(buf, which + "_params").view(torch.uint8).view(torch.float16).view(T, -1).cpu().float()
+        assert float(params[rows].abs().sum()) == 0.0, which
+        assert torch.equal(rec.view(T, -1)[rows.cuda()], X.view(T, -1)[rows.cuda()]), which
+
+
 @pytest.mark.parametrize("dtype,T,H,n_c", [(torch.float32, 300, 2, 16), (torch.bfloat16, 257, 3, 40)])
 def test_cluster_codec_cuda_core_path(dtype, T, H, n_c):
     """fp32 data, or a joint row of 384 channels (not a multiple of 256): the
