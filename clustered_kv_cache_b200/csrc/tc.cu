@@ -120,14 +120,20 @@ struct Args {
   const float* codebook;
 };
 
-template <int RC, bool PAIR>
+// SLIM: a paired decode of 2-bit codes in 32-value groups stages only 48 bytes a
+// thread (two chunks of code words, one of (scale, zero) pairs), so its input
+// slots are 64 bytes and the 16 KB this frees hold a sixth pipeline stage
+template <int MODE, int G, int BITS, bool PAIR, bool EDEN>
+constexpr bool kSlim = PAIR && MODE == 1 && !EDEN && BITS == 2 && G == 32;
+
+template <int RC, bool PAIR, bool SLIM = false>
 struct Layout {
   // pipeline stages (the latent lives in TMEM, not here); a CTA of a pair holds
   // half of every B operand, so its stages are smaller and there are more of them
-  static constexpr int S = PAIR ? 5 : 4;
+  static constexpr int S = PAIR ? (SLIM ? 6 : 5) : 4;
   static constexpr int kStage = PAIR ? 24576 : 32768;  // A 16 KB + B 16 KB (pair: B 8 KB)
   static constexpr int kRecon = 32768;  // [128][128] bf16 as two 64-column sub-tiles
-  static constexpr int kIn = 128;       // staged epilogue inputs: bytes per epilogue thread
+  static constexpr int kIn = SLIM ? 64 : 128;  // staged epilogue inputs: bytes per epilogue thread
   static constexpr int kStageOff = 0;
   static constexpr int kReconOff = S * kStage;
   static constexpr int kInOff = kReconOff + 2 * kRecon;
@@ -157,7 +163,8 @@ template <int MODE, int G, int RC, int BITS, bool PAIR, bool EDEN, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_constant__ Maps maps, const Args a) {
   constexpr bool ENC = MODE == kEncode;
   static_assert(!EDEN || (G == 64 && BITS == 2), "EDEN-2 codes 64-value groups at 4 bits a pair");
-  using L = Layout<RC, PAIR>;
+  constexpr bool SLIM = kSlim<MODE, G, BITS, PAIR, EDEN>;
+  using L = Layout<RC, PAIR, SLIM>;
   constexpr int S = L::S;
   constexpr int R = RC * 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -721,7 +728,8 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
     constexpr bool STX = ENC && G == 32;
     constexpr bool STE = ENC && EDEN;  // EDEN-2 encode: x of the next 64-value group in the slot
     const uint32_t slot = in_base + (uint32_t)(grp * 128 + row) * L::kIn;
-    auto chunk = [&](int c) { return slot + (((uint32_t)c ^ (uint32_t)(row & 7)) << 4); };
+    auto chunk = [&](int c) { return slot + (((uint32_t)c ^ (uint32_t)(row & (L::kIn / 16 - 1))) << 4); };
+    constexpr int PCH = SLIM ? 2 : 4;  // the chunk of the (scale, zero) pairs (decode)
 
     // one head of this group: h its index, is_v K or V, t0 the tile.  The
     // groups of the row are processed by a rolled loop (the kernel's code must
@@ -765,12 +773,12 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
         for (int i = 0; i < RB / 16; ++i) cp_async16(chunk(i), valid ? (const void*)(src + 16 * i) : c0, valid ? 16u : 0u);
         if (EDEN) {  // the row's two fp16 scales
           const __half* es = reinterpret_cast<const __half*>(is_v ? pp.vparams : pp.kparams) + rowi * 2;
-          cp_async4(chunk(4), valid ? (const void*)es : (const void*)p0, valid ? 4u : 0u);
+          cp_async4(chunk(PCH), valid ? (const void*)es : (const void*)p0, valid ? 4u : 0u);
         } else if (G == 32) {
-          cp_async16(chunk(4), valid ? params : p0, valid ? 16u : 0u);
+          cp_async16(chunk(PCH), valid ? params : p0, valid ? 16u : 0u);
         } else {
 #pragma unroll
-          for (int i = 0; i < NG; ++i) cp_async4(chunk(4) + 4 * i, valid ? params + i : p0, valid ? 4u : 0u);
+          for (int i = 0; i < NG; ++i) cp_async4(chunk(PCH) + 4 * i, valid ? params + i : p0, valid ? 4u : 0u);
         }
         cp_async_commit();
       }
@@ -790,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
             co[i] = w.x;
             co[i + 1] = w.y;
           }
-          const uint32_t pw = lds32(chunk(4) + 4 * g);
+          const uint32_t pw = lds32(chunk(PCH) + 4 * g);
           po = *reinterpret_cast<const __half2*>(&pw);
         }
       };
@@ -886,7 +894,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
               *reinterpret_cast<uint4*>(codes + g * 4) = make_uint4(gw[0], gw[1], gw[2], gw[3]);
             }
           } else {
-            const uint32_t sw = lds32(chunk(4));
+            const uint32_t sw = lds32(chunk(PCH));
             sf = __half2float(__ushort_as_half((unsigned short)(g ? sw >> 16 : sw & 0xffffu)));
 #pragma unroll
             for (int i = 0; i < 4; ++i) gw[i] = cc[i];
@@ -1216,7 +1224,7 @@ static cudaError_t launch(const Maps& m, const Args& a, cudaStream_t st) {
   } else {
     // pairs: clusters of two CTAs, each pair looping over 256-token tiles (of each layer)
     auto k = xlayer_tc_kernel<MODE, G, RC, BITS, true, EDEN, MULTI>;
-    const int smem = Layout<RC, true>::kBytes + 1024;
+    const int smem = Layout<RC, true, kSlim<MODE, G, BITS, true, EDEN>>::kBytes + 1024;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
