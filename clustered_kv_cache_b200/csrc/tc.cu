@@ -527,24 +527,17 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
           for (int k = 0; k < 4; ++k) mma_ss(lead, d, ad2 + 2 * k, bd + 2 * k, idesc, 1u);
         }
       };
-      // n chunks from the next n stages, after the waits in pre(): one hand-off
+      // n chunks from the next n stages, after the waits in pre(): one hand-off a
+      // stage, so that a stage's MMAs are issued as soon as it has landed
       auto group = [&](int n, auto&& pre, auto&& body) {
-        if (!ISSUE) {
-          pre();
-          int ss = s;
-          uint32_t pp = ph;
-          for (int i = 0; i < n; ++i) {
-            wt(&full[ss], pp, 0x300u + ss);
-            if (++ss == S) {
-              ss = 0;
-              pp ^= 1;
-            }
-          }
-          __syncwarp();
-        }
-        asm volatile("bar.sync 3, 64;" ::: "memory");
-        if (ISSUE) tc_fence_after();
         for (int i = 0; i < n; ++i) {
+          if (!ISSUE) {
+            if (i == 0) pre();
+            wt(&full[s], ph, 0x300u + s);
+            __syncwarp();
+          }
+          asm volatile("bar.sync 3, 64;" ::: "memory");
+          if (ISSUE) tc_fence_after();
           body(i, s);
           commit(&empty[s]);
           if (++s == S) {
