@@ -46,9 +46,9 @@ UNIT = "KV tokens/s"
 # profiles/ (codec_xlayer_wan_layer.md, codec_xlayer_fused_wan.md, attention_flash_wan.md,
 # mixed_attention_cluster.md, cluster_codec_decode.md, temporal_codec_layer.md, codec_xlayer_eden2.md);
 # set to None when a kernel changes after its capture.
-TRAFFIC = {"encode_xlayer": 678559232 + 188143104, "decode_xlayer": 428340480 + 137626112,
+TRAFFIC = {"encode_xlayer": 679453184 + 187834368, "decode_xlayer": 430907648 + 137585920,
            # per layer of the fused walk (a 4-layer launch's DRAM bytes / 4; scaled by the layer count)
-           "encode_xlayer_fused": (2882488064 + 912262656) // 4, "decode_xlayer_fused": (2091626496 + 743751424) // 4,
+           "encode_xlayer_fused": (2892781056 + 912364800) // 4, "decode_xlayer_fused": (2074051072 + 744571648) // 4,
            "attention_c2": 244925696 + 13229312, "attention_c4": 26443520 + 146944,
            "decode_c4": 9409024 + 214975232,
            "temporal_encode": 1424011008 + 351590400,
