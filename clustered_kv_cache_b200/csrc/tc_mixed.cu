@@ -12,7 +12,8 @@
 //
 // so per (128-query tile, head) the kernel is a flash attention with 256-wide
 // rows on both sides: A = [q_h | q_h W_dec,h] (its second half computed on the
-// tensor cores at the start), 64-key tiles [centre rows | coefficients] for the
+// tensor cores at the start; the score MMAs read A from tensor memory, so only
+// the key tile comes from shared memory), 64-key tiles [centre rows | coefficients] for the
 // keys and for the values, double-buffered so that a tile's gather and load
 // overlap the MMAs of the one before; the value product accumulates
 // [O_c | cbar] (256 TMEM columns) and the end adds cbar W^V_dec,h^T.  The sum
@@ -38,6 +39,16 @@ namespace tc {
 bool map2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 namespace mixed {
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane (no wait)
+__device__ __forceinline__ void tmem_st16w(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]), "r"(w[9]),
+      "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
+}
 
 constexpr int kThreads = 320;
 constexpr int kKeys = 64;  // keys per tile
@@ -195,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBar);
   uint64_t* setup_full = bars;         // q_h and W_dec,h landed
   uint64_t* qw_acc = setup_full + 1;   // q_h W_dec,h in TMEM
-  uint64_t* qw_ready = qw_acc + 1;     // ... and in the A tile as bf16 (prep)
+  uint64_t* qw_ready = qw_acc + 1;     // ... and [q | q W_dec] as bf16 pairs in TMEM (prep)
   uint64_t* kfull = qw_ready + 1;      // [2] key tile complete (producer tx + 64 prep arrivals)
   uint64_t* vfull = kfull + 2;         // [2] value tile complete
   uint64_t* kfree = vfull + 2;         // [2] S(j) done: the key tile may be refilled
@@ -340,15 +351,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j <= NT; ++j) {
         if (j < NT) {
           const int b = j & 1;
-          // S(j) = [q | q W_dec] [centres | coef]^T, K = 256, N = 64 keys
+          // S(j) = [q | q W_dec] [centres | coef]^T, K = 256, N = 64 keys; A from
+          // tensor memory (bf16 pairs, 8 columns a K step), so the MMAs read only
+          // the key tile from shared memory
           wait(&kfull[b], (j >> 1) & 1, abort_flag, a.err, 0x2210u + b);
           tc_fence_after();
           const uint64_t kd = desc_sw128(smem_u32(KT(b)));
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const uint32_t aoff = (k >> 2) * (16384 >> 4) + (k & 3) * 2;
             const uint32_t boff = (k >> 2) * (kSub >> 4) + (k & 3) * 2;
-            umma(SC(b), ad + aoff, kd + boff, id64, k == 0 ? 0u : 1u);
+            umma_ts(SC(b), QW + k * 8, kd + boff, id64, k == 0 ? 0u : 1u);
           }
           umma_commit(&s_full[b]);
           umma_commit(&kfree[b]);
@@ -433,12 +445,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         w[i] = __ldg(reinterpret_cast<const uint4*>(cent + (int64_t)cr * C + h * 128) + ch);
       }
     };
+    wait(setup_full, 0, abort_flag, a.err, 0x2305u);  // q in At (read below through the generic proxy)
+    wait(qw_acc, 0, abort_flag, a.err, 0x2300u);      // also: W_dec,h in key buffer 0 is no longer read
+    tc_fence_after();
+    // A of the score MMAs into tensor memory, over the q W_dec accumulator (this
+    // thread's lane): columns [0, 64) q and [64, 128) q W_dec as bf16 pairs.  Block
+    // k of 32 fp32 columns of q W_dec becomes 16 columns of pairs at 64 + 16 k,
+    // highest block first, so that no block is overwritten before it is read.
+    {
+#pragma unroll 1
+      for (int k = 3; k >= 0; --k) {
+        float v[32];
+        tmem_ld32(lane_addr + (QW - tmem) + 32 * k, v);
+        uint32_t p16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p16[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        tmem_st16w(lane_addr + (QW - tmem) + 64 + 16 * k, p16);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      }
+#pragma unroll 1
+      for (int k = 0; k < 4; ++k) {  // q elements 32 k .. 32 k + 31: chunks 4 k .. 4 k + 3 of the row
+        uint32_t p16[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int cc = 4 * k + c;  // 16-byte chunk of the 256-byte row (sub-tile cc / 8)
+          const uint4 u = *reinterpret_cast<const uint4*>(At + (cc >> 3) * 16384 + sw128_off(row, cc & 7));
+          p16[4 * c] = u.x;
+          p16[4 * c + 1] = u.y;
+          p16[4 * c + 2] = u.z;
+          p16[4 * c + 3] = u.w;
+        }
+        tmem_st16w(lane_addr + (QW - tmem) + 16 * k, p16);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+    }
+    mbar_arrive(qw_ready);
     uint4 w[16];
     fetch_row(0, w);
-    wait(qw_acc, 0, abort_flag, a.err, 0x2300u);  // also: W_dec,h in key buffer 0 is no longer read
-    tc_fence_after();
-    to_bf16(QW, At + 32768);
-    mbar_arrive(qw_ready);
     for (int j = 0; j < NT; ++j) {
       const int b = j & 1;
       if (j >= 2) wait(&tfree[b], ((j - 2) >> 1) & 1, abort_flag, a.err, 0x2301u + (is_v ? 2 : 0) + b);
