@@ -49,7 +49,7 @@ UNIT = "KV tokens/s"
 TRAFFIC = {"encode_xlayer": 679453184 + 187834368, "decode_xlayer": 430907648 + 137585920,
            # per layer of the fused walk (a 4-layer launch's DRAM bytes / 4; scaled by the layer count)
            "encode_xlayer_fused": (2892781056 + 912364800) // 4, "decode_xlayer_fused": (2074051072 + 744571648) // 4,
-           "attention_c2": 244925696 + 13229312, "attention_c4": None,
+           "attention_c2": 244925696 + 13229312, "attention_c4": 26439936 + 141056,
            "decode_c4": 9409024 + 214975232,
            "temporal_encode": 1424011008 + 351590400,
            "temporal_decode": 659118080 + 1286398464,
