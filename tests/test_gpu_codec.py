@@ -1101,7 +1101,10 @@ def test_layer_chain_other_shapes_match_layer_calls(case):
                                                             (5, 2 * 256 + 7, 3, 128, 4, 64, True),
                                                             (5, 300, 2, 0, 2, 64, True), (5, 128, 2, 64, 2, 32, False),
                                                             (61, 300, 2, 64, 2, 32, True),
-                                                            (3, 40 * 128 + 3, 2, 64, 2, 32, True)])
+                                                            (3, 40 * 128 + 3, 2, 64, 2, 32, True),
+                                                            (2, 1, 2, 64, 2, 32, False),
+                                                            (3, 129, 3, 64, 4, 64, True),
+                                                            (3, 256, 2, 128, 2, 32, False)])
 def test_layer_chain_in_one_call_matches_layer_calls(L, T, H, rank, bits, group, pingpong):
     """kvc_encode_layers / kvc_decode_layers (one persistent launch walking
     (layer, tile) items, each tile waiting on the same tile of the layer before)
@@ -1109,7 +1112,9 @@ def test_layer_chain_in_one_call_matches_layer_calls(L, T, H, rank, bits, group,
     arithmetic, so every code, parameter and reconstruction is identical.  With
     `pingpong` the chain reuses two reconstruction buffers in turn.  60 layers of
     3 tiles give more items than SMs with fewer tiles than CTAs (the latent
-    overlap across items is off there); 40 tiles give CTAs several items each."""
+    overlap across items is off there); 40 tiles give CTAs several items each.
+    Edges: one layer of one token (the second CTA of the pair has no rows), 129
+    tokens (it has one), and exactly one 256-token pair tile."""
     D = 128
     wl = synth.wan_xlayer(seed=synth.SEED_BASE + 121, device="cuda", L=L, T=T, H=H, rank=rank, calib_tokens=512)
     bf, hf = torch.bfloat16, torch.float16
