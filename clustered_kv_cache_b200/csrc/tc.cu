@@ -124,7 +124,7 @@ struct Args {
 // thread (two chunks of code words, one of (scale, zero) pairs), so its input
 // slots are 64 bytes and the 16 KB this frees hold a sixth pipeline stage
 template <int MODE, int G, int BITS, bool PAIR, bool EDEN>
-constexpr bool kSlim = PAIR && MODE == 1 && !EDEN && BITS == 2 && G == 32;
+constexpr bool kSlim = PAIR && MODE == kDecode && !EDEN && BITS == 2 && G == 32;
 
 template <int RC, bool PAIR, bool SLIM = false>
 struct Layout {
