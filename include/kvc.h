@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
   KVC_OK = 0,
   KVC_ERR_INVALID_ARGUMENT = 1, /* NULL where a buffer is required, bad sizes */
-  KVC_ERR_UNSUPPORTED = 2,      /* a combination this build does not implement */
+  KVC_ERR_UNSUPPORTED = 2,      /* a combination the library does not implement */
   KVC_ERR_MISALIGNED = 3,       /* a device pointer not 16-byte aligned */
   KVC_ERR_WORKSPACE_TOO_SMALL = 4,
   KVC_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed */
