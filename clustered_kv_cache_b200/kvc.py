@@ -241,12 +241,18 @@ def alloc_layers_workspace(op: int, desc: LayerDesc, preds, device="cuda") -> to
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
+def _same_length(n: int, **lists) -> None:
+    for name, seq in lists.items():
+        if len(seq) != n:
+            raise ValueError(f"{name} has {len(seq)} entries for {n} layers")
+
+
 def kvc_encode_layers(desc, preds, K, V, K_src, V_src, codes, K_rec, V_rec, ws=None, stream=None):
     """Layers i = 0 .. len(preds)-1 of a cross-layer chain in one call; layer i
     predicts from K_rec[i-1] / V_rec[i-1] (K_src / V_src for i = 0).  K, V, codes,
-    K_rec, V_rec: lists of one entry per layer."""
+    K_rec, V_rec: lists of one entry per layer; ws from alloc_layers_workspace."""
     n = len(preds)
-    assert len(K) == len(V) == len(codes) == len(K_rec) == len(V_rec) == n
+    _same_length(n, K=K, V=V, codes=codes, K_rec=K_rec, V_rec=V_rec)
     wp, wn = _ws(ws)
     _check(lib().kvc_encode_layers(ctypes.byref(desc), _preds(preds), n, _ptrs(K), _ptrs(V), _ptr(K_src),
                                    _ptr(V_src), _codes(codes), _ptrs(K_rec), _ptrs(V_rec), wp, wn, _stream(stream)),
@@ -254,8 +260,11 @@ def kvc_encode_layers(desc, preds, K, V, K_src, V_src, codes, K_rec, V_rec, ws=N
 
 
 def kvc_decode_layers(desc, preds, codes, K_src, V_src, K_rec, V_rec, ws=None, stream=None):
+    """The decode of kvc_encode_layers: layer i replays its prediction from
+    K_rec[i-1] / V_rec[i-1] (K_src / V_src for i = 0) and adds its decoded
+    residual; the reconstructions equal the encode's byte for byte."""
     n = len(preds)
-    assert len(codes) == len(K_rec) == len(V_rec) == n
+    _same_length(n, codes=codes, K_rec=K_rec, V_rec=V_rec)
     wp, wn = _ws(ws)
     _check(lib().kvc_decode_layers(ctypes.byref(desc), _preds(preds), n, _codes(codes), _ptr(K_src), _ptr(V_src),
                                    _ptrs(K_rec), _ptrs(V_rec), wp, wn, _stream(stream)), "kvc_decode_layers")

@@ -135,3 +135,13 @@ def test_multi_layer_validation_without_launch(L):
     tp = kvc.Predictor(kvc.PRED_TEMPORAL, 0, 0, 0, *([0x1000] * 12))
     assert L.kvc_decode_layers(ctypes.byref(kvc.make_desc(100, 2, 128, frame_tokens=10)), (kvc.Predictor * 1)(tp),
                                1, (kvc.Codes * 1)(c), 0x1000, 0x1000, P(0x3000), P(0x4000), None, 0, None) == 2
+
+
+def test_multi_layer_binding_rejects_mismatched_lists():
+    """The binding checks the per-layer lists before any call reaches the library."""
+    d = kvc.make_desc(100, 2, 128, torch.bfloat16, 2, 32)
+    p = kvc.Predictor(kvc.PRED_XLAYER_DPLR, 0, 0, 0)
+    with pytest.raises(ValueError, match="K_rec has 1 entries for 2 layers"):
+        kvc.kvc_encode_layers(d, [p, p], [None, None], [None, None], None, None, [None, None], [None], [None, None])
+    with pytest.raises(ValueError, match="codes has 3 entries for 2 layers"):
+        kvc.kvc_decode_layers(d, [p, p], [None, None, None], None, None, [None, None], [None, None])
