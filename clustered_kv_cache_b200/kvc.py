@@ -316,7 +316,8 @@ def kvc_refit_block_diag(desc, pred, tensor: int, X0, X1, Y, ridge: float, block
 def kvc_copy_to_device(dst: torch.Tensor, src: torch.Tensor, stream=None):
     """Copies a host tensor (pinned for asynchrony) into a device tensor of the same size."""
     n = src.numel() * src.element_size()
-    assert dst.numel() * dst.element_size() >= n
+    if dst.numel() * dst.element_size() < n:
+        raise ValueError(f"destination holds {dst.numel() * dst.element_size()} bytes, the copy {n}")
     _check(lib().kvc_copy_to_device(_ptr(dst), ctypes.c_void_p(src.data_ptr()), n, _stream(stream)),
            "kvc_copy_to_device")
 
@@ -324,7 +325,8 @@ def kvc_copy_to_device(dst: torch.Tensor, src: torch.Tensor, stream=None):
 def kvc_copy_to_host(dst: torch.Tensor, src: torch.Tensor, stream=None):
     """Copies a device tensor into a host tensor (pinned for asynchrony) of the same size."""
     n = src.numel() * src.element_size()
-    assert dst.numel() * dst.element_size() >= n
+    if dst.numel() * dst.element_size() < n:
+        raise ValueError(f"destination holds {dst.numel() * dst.element_size()} bytes, the copy {n}")
     _check(lib().kvc_copy_to_host(ctypes.c_void_p(dst.data_ptr()), _ptr(src), n, _stream(stream)),
            "kvc_copy_to_host")
 

@@ -398,7 +398,8 @@ def eden2_codebook(n_points: int = 16, iters: int = 300, grid: int = 801, span: 
 
 
 def _eden2_lloyd(n_points: int, iters: int, grid: int, span: float) -> torch.Tensor:
-    assert n_points == 16
+    if n_points != 16:
+        raise ValueError("the EDEN-2 codebook has 16 points (4-bit indices)")
     ax = torch.linspace(-span, span, grid, dtype=torch.float64)
     X, Y = torch.meshgrid(ax, ax, indexing="ij")
     P = torch.stack([X.reshape(-1), Y.reshape(-1)], 1)

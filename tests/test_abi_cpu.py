@@ -145,3 +145,12 @@ def test_multi_layer_binding_rejects_mismatched_lists():
         kvc.kvc_encode_layers(d, [p, p], [None, None], [None, None], None, None, [None, None], [None], [None, None])
     with pytest.raises(ValueError, match="codes has 3 entries for 2 layers"):
         kvc.kvc_decode_layers(d, [p, p], [None, None, None], None, None, [None, None], [None, None])
+
+
+def test_copy_helpers_reject_short_destinations():
+    """A destination smaller than the copy is refused before any library call."""
+    small, big = torch.empty(4, dtype=torch.uint8), torch.empty(8, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="destination holds 4 bytes, the copy 8"):
+        kvc.kvc_copy_to_device(small, big)
+    with pytest.raises(ValueError, match="destination holds 4 bytes, the copy 8"):
+        kvc.kvc_copy_to_host(small, big)
