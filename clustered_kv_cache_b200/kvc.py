@@ -4,6 +4,18 @@ Argument marshalling only: every function here turns torch tensors into device
 pointers and forwards to the C entry point of the same name; all computation
 happens in the library's CUDA kernels.  The library is loaded on first use and
 a missing or unloadable library raises ``KvcError`` (there is no fallback).
+
+A cross-layer chain, the anchor layer first and then layers 1 .. L-1 in one
+launch each way::
+
+    desc0 = make_desc(T, H, D, torch.bfloat16, 4, 32)          # INT4 anchor
+    desc = make_desc(T, H, D, torch.bfloat16, 2, 32)           # INT2 residuals
+    preds = [make_predictor(PRED_XLAYER_DPLR, w, rank=64) for w in weights]
+    kvc_encode_layer(desc0, make_predictor(PRED_NONE), K[0], V[0], None, None, codes0, K0r, V0r)
+    ws = alloc_layers_workspace(OP_ENCODE, desc, preds)
+    kvc_encode_layers(desc, preds, K[1:], V[1:], K0r, V0r, codes, K_rec, V_rec, ws)
+    kvc_decode_layers(desc, preds, codes, K0r, V0r, K_dec, V_dec,
+                      alloc_layers_workspace(OP_DECODE, desc, preds))
 """
 
 from __future__ import annotations
