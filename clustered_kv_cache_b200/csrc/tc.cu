@@ -143,18 +143,38 @@ struct Layout {
 
 // Orthonormal Walsh-Hadamard transform of one thread's 64 values (Sylvester
 // order: entry (i, j) = (-1)^popcount(i & j) / 8), six butterfly stages in registers.
+// Entries e and e + 2 (bit 1 of e clear) travel as one packed pair, so every
+// stage but the one over bit 1 does two butterflies an instruction; each entry
+// still takes one rounded addition a stage, in the same order.  The pairing
+// also puts the first coordinates of the point pairs 2m and 2m + 1 side by side
+// (entries 4m and 4m + 2), as the EDEN-2 search wants them.
 __device__ __forceinline__ void walsh64_thread(float (&v)[64]) {
 #pragma unroll
-  for (int b = 1; b < 64; b <<= 1)
+  for (int b = 1; b < 64; b <<= 1) {
 #pragma unroll
-    for (int e = 0; e < 64; ++e)
-      if (!(e & b)) {
-        const float x = v[e], y = v[e + b];
+    for (int e = 0; e < 64; ++e) {
+      if ((e & b) || (e & 2)) continue;
+      if (b == 2) {
+        const float x = v[e], y = v[e + 2];
         v[e] = x + y;
-        v[e + b] = x - y;
+        v[e + 2] = x - y;
+      } else {
+        const float2 x = make_float2(v[e], v[e + 2]), y = make_float2(v[e + b], v[e + b + 2]);
+        const float2 s = add2(x, y), d = sub2(x, y);
+        v[e] = s.x;
+        v[e + 2] = s.y;
+        v[e + b] = d.x;
+        v[e + b + 2] = d.y;
       }
+    }
+  }
 #pragma unroll
-  for (int e = 0; e < 64; ++e) v[e] *= 0.125f;
+  for (int e = 0; e < 64; ++e) {
+    if (e & 2) continue;
+    const float2 s = mul2(make_float2(v[e], v[e + 2]), make_float2(0.125f, 0.125f));
+    v[e] = s.x;
+    v[e + 2] = s.y;
+  }
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -184,8 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_cb = reinterpret_cast<float*>(smem + L::kBarOff + 512);  // EDEN-2 codebook [16][2]
-  // the search's form of point j: (-2 c_j0, -2 c_j1, |c_j|^2, 0)
-  float4* s_cq = reinterpret_cast<float4*>(smem + L::kBarOff + 640);  // [16]
+  // the search's form of point j, each term twice (one per lane of a packed
+  // pair): (-2 c_j0, -2 c_j0, -2 c_j1, -2 c_j1) and (|c_j|^2, |c_j|^2)
+  float4* s_cxy = reinterpret_cast<float4*>(smem + L::kBarOff + 640);  // [16]
+  float2* s_cz = reinterpret_cast<float2*>(smem + L::kBarOff + 896);   // [16]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H;
@@ -254,7 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
       for (int i = 0; i < 32; ++i) s_cb[i] = a.codebook[i];
       for (int j = 0; j < 16; ++j) {
         const float c0 = a.codebook[2 * j], c1 = a.codebook[2 * j + 1];
-        s_cq[j] = make_float4(-2.f * c0, -2.f * c1, fmaf(c0, c0, c1 * c1), 0.f);
+        s_cxy[j] = make_float4(-2.f * c0, -2.f * c0, -2.f * c1, -2.f * c1);
+        const float cc = fmaf(c0, c0, c1 * c1);
+        s_cz[j] = make_float2(cc, cc);
       }
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -852,24 +876,38 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
             const float sigma = sqrtf(ss * (1.f / 64.f));
             const float inv_sigma = ss > 0.f ? 1.f / sigma : 0.f;
 #pragma unroll
-            for (int e = 0; e < 64; ++e) y[e] *= inv_sigma;
+            for (int e = 0; e < 64; ++e) {
+              if (e & 2) continue;
+              const float2 u = mul2(make_float2(y[e], y[e + 2]), make_float2(inv_sigma, inv_sigma));
+              y[e] = u.x;
+              y[e + 2] = u.y;
+            }
             // |u - c|^2 = |u|^2 + |c|^2 - 2 <u, c>: per pair the point with the least
-            // |c|^2 - 2 <u, c> (two FMAs); the index goes into the pair's nibble of
-            // gw with one three-input logic op (j replicated over all nibbles)
+            // |c|^2 - 2 <u, c> (two FMAs, here packed over pairs 2m and 2m + 1:
+            // entries (4m, 4m + 2) and (4m + 1, 4m + 3)); the index goes into the
+            // pair's nibble of gw with one three-input logic op (j replicated over
+            // all nibbles)
             float bd[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) bd[i] = INFINITY;
 #pragma unroll 1
             for (int j = 0; j < 16; ++j) {  // points in index order: a strict < keeps the lowest
-              const float4 cq = s_cq[j];
+              const float4 cxy = s_cxy[j];
+              const float2 cz = s_cz[j];
               const uint32_t jr = (uint32_t)j * 0x11111111u;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float d = fmaf(y[2 * i], cq.x, fmaf(y[2 * i + 1], cq.y, cq.z));
-                if (d < bd[i]) {
-                  bd[i] = d;
-                  const uint32_t m = 15u << (4 * (i % 8));
-                  gw[i / 8] = (gw[i / 8] & ~m) | (jr & m);
+              for (int m = 0; m < 16; ++m) {
+                const float2 d2 = fma2(make_float2(y[4 * m], y[4 * m + 2]), make_float2(cxy.x, cxy.y),
+                                       fma2(make_float2(y[4 * m + 1], y[4 * m + 3]), make_float2(cxy.z, cxy.w), cz));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int i = 2 * m + h;
+                  const float d = h ? d2.y : d2.x;
+                  if (d < bd[i]) {
+                    bd[i] = d;
+                    const uint32_t msk = 15u << (4 * (i % 8));
+                    gw[i / 8] = (gw[i / 8] & ~msk) | (jr & msk);
+                  }
                 }
               }
             }
@@ -877,7 +915,8 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int k = (int)((gw[i / 8] >> (4 * (i % 8))) & 15u);
-              dot = fmaf(y[2 * i], s_cb[2 * k], fmaf(y[2 * i + 1], s_cb[2 * k + 1], dot));
+              const float2 c = reinterpret_cast<const float2*>(s_cb)[k];
+              dot = fmaf(y[2 * i], c.x, fmaf(y[2 * i + 1], c.y, dot));
             }
             const float yc = dot * sigma;  // <y, c>
             const __half sh = __float2half_rn(ss > 0.f && yc > 0.f ? ss / yc : 0.f);
@@ -895,8 +934,9 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int k = (int)((gw[i / 8] >> (4 * (i % 8))) & 15u);
-            y[2 * i] = sf * s_cb[2 * k];
-            y[2 * i + 1] = sf * s_cb[2 * k + 1];
+            const float2 c = reinterpret_cast<const float2*>(s_cb)[k];
+            y[2 * i] = sf * c.x;
+            y[2 * i + 1] = sf * c.y;
           }
           walsh64_thread(y);
 #pragma unroll
