@@ -53,7 +53,7 @@ TRAFFIC = {"encode_xlayer": 679453184 + 187834368, "decode_xlayer": 430907648 + 
            "decode_c4": 9409024 + 214975232,
            "temporal_encode": 1424011008 + 351590400,
            "temporal_decode": 659118080 + 1286398464,
-           "eden2_encode": 665347840 + 179403008, "eden2_decode": 414407936 + 136523520}
+           "eden2_encode": None, "eden2_decode": 414407936 + 136523520}
 
 
 def peaks():

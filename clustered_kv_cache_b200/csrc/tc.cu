@@ -890,7 +890,7 @@ __global__ void __launch_bounds__(kThreads, 1) xlayer_tc_kernel(const __grid_con
             float bd[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) bd[i] = INFINITY;
-#pragma unroll 1
+#pragma unroll 2  // two points in flight (one measured 1.5% slower, four 6%)
             for (int j = 0; j < 16; ++j) {  // points in index order: a strict < keeps the lowest
               const float4 cxy = s_cxy[j];
               const float2 cz = s_cz[j];
